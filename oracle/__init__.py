@@ -1,0 +1,198 @@
+"""Plain fp64 CPU oracle for the SparDA hot path -- TEST INFRASTRUCTURE.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never does, and
+this package imports nothing from it: the two share no code.
+
+The arithmetic lives in ``sparda_oracle.c`` (plain C, double precision, loops
+written straight from the definitions); this module only compiles it with gcc
+and marshals numpy arrays.  bf16 tensors are passed as ``uint16`` arrays of
+their raw bits and decoded exactly inside the C code.
+
+Sources: "SparDA: a fourth projection that lets sparse attention prefetch its
+own KV cache" (ai.thesatyajit.com/articles/sparda) -- section "The problem
+InfLLM-V2 leaves on the table" (eq. B_l(i)), section "The fourth projection"
+(Eq. 3-5, Algorithms 1 and 2), section "One Forecast head per GQA group"
+(Forecast indexer versus the multi-head baseline selector); and
+deepresearch2agi.pages.dev/sparda_sparse_decoupled_attention, section
+"架构细节" (mean-compressed keys).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sparda_oracle.c")
+_LIB = os.path.join(_HERE, "libsparda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libsparda_oracle.so`` (gcc, -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-D_DEFAULT_SOURCE", "-fPIC", "-shared",
+             "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        LL = ctypes.c_longlong
+        D = ctypes.c_double
+        lib.oracle_double_to_bf16.argtypes = [D]
+        lib.oracle_double_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_double.restype = D
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = I
+        lib.oracle_compress_keys.argtypes = [I, I, I, I, I, P, LL, LL, P, P]
+        lib.oracle_compress_keys.restype = None
+        lib.oracle_select.argtypes = [I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P]
+        lib.oracle_select.restype = None
+        lib.oracle_gather_blocks.argtypes = [I, I, I, I, I, I, I, I, I, I, P, P, P]
+        lib.oracle_gather_blocks.restype = None
+        lib.oracle_sparse_attention.argtypes = [I, I, I, I, I, I, I, I, D, P, P, P, LL, LL, P, I, P]
+        lib.oracle_sparse_attention.restype = None
+        lib.oracle_dense_causal_attention.argtypes = [I, I, I, I, I, I, I, D, P, P, P, P]
+        lib.oracle_dense_causal_attention.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 inputs are passed as uint16 arrays of raw bits, got %s" % a.dtype)
+    return a
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def double_to_bf16(x: float) -> int:
+    """Round one double to bf16 bits, to nearest, ties to even (one rounding)."""
+    return int(_load().oracle_double_to_bf16(float(x)))
+
+
+def bf16_to_double(bits: int) -> float:
+    return float(_load().oracle_bf16_to_double(int(bits)))
+
+
+def compress_keys(K: np.ndarray, blk: int = 64):
+    """Mean-pooled compressed keys.
+
+    K: uint16 [B][G][T][d].  Returns (kc_f64 [B][G][NB][d], kc_bf16 [B][G][NB][d]).
+    """
+    K = _u16(K)
+    B, G, T, d = K.shape
+    NB = (T + blk - 1) // blk
+    kc = np.empty((B, G, NB, d), np.float64)
+    kcb = np.empty((B, G, NB, d), np.uint16)
+    _load().oracle_compress_keys(B, G, T, d, blk, _ptr(K), T * d, d, _ptr(kc), _ptr(kcb))
+    return kc, kcb
+
+
+def select(F: np.ndarray, kc: np.ndarray, k: int, n_init: int, n_local: int, q_start: int,
+           blk: int = 64):
+    """Block sets init U local U top-k(F . Kc^T).
+
+    F:  uint16 [B][nq][G][nf][d] (nf = 1 for the Forecast indexer, nf = query heads
+        per group for the baseline multi-head selector, whose scores are summed).
+    kc: uint16 [B][G][NB][d].
+    Query token i sits at position q_start + i.
+    Returns (idx int32 [B][nq][G][S], kth [B][nq][G], kth1 [B][nq][G]).
+    """
+    F = _u16(F)
+    kc = _u16(kc)
+    B, nq, G, nf, d = F.shape
+    NB = kc.shape[2]
+    assert kc.shape == (B, G, NB, d)
+    last = q_start + nq - 1
+    if last // blk >= NB:
+        raise ValueError("query position %d needs block %d but Kc has %d blocks" % (last, last // blk, NB))
+    S = k + n_init + n_local
+    idx = np.empty((B, nq, G, S), np.int32)
+    kth = np.empty((B, nq, G), np.float64)
+    kth1 = np.empty((B, nq, G), np.float64)
+    _load().oracle_select(B, nq, G, nf, d, blk, NB, k, n_init, n_local, q_start,
+                          _ptr(F), _ptr(kc), _ptr(idx), _ptr(kth), _ptr(kth1))
+    return idx, kth, kth1
+
+
+def gather_blocks(host_kv: np.ndarray, idx: np.ndarray, pos: int, n_init: int, n_local: int,
+                  skip_resident: bool, slots: np.ndarray | None = None) -> np.ndarray:
+    """Byte copy of the selected blocks into slots.
+
+    host_kv: uint16 [B][G][NB][2][blk][d]; idx int32 [B][G][S].
+    Returns slots uint16 [B][G][S][2][blk][d] (entries not copied keep the
+    contents of ``slots`` if given, else zero).
+    """
+    host_kv = _u16(host_kv)
+    B, G, NB, two, blk, d = host_kv.shape
+    idx = np.ascontiguousarray(idx, np.int32)
+    S = idx.shape[-1]
+    if slots is None:
+        slots = np.zeros((B, G, S, 2, blk, d), np.uint16)
+    else:
+        slots = np.ascontiguousarray(slots.copy())
+    _load().oracle_gather_blocks(B, G, NB, S, blk, d, pos, n_init, n_local, int(skip_resident),
+                                 _ptr(host_kv), _ptr(idx), _ptr(slots))
+    return slots
+
+
+def sparse_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, q_start: int,
+                     T: int, blk: int = 64, scale: float = 0.0, bg_stride: int | None = None,
+                     blk_stride: int | None = None, G: int | None = None) -> np.ndarray:
+    """Attention over the keys of each query's block set (fp64 result).
+
+    Q: uint16 [B][nq][Hq][d]; idx int32 [B][nq][G][S].
+    K/V: uint16, either [B][G][T][d] (strides derived) or any buffer with the
+    row of token t of (b,g) at (b*G+g)*bg_stride + (t//blk)*blk_stride + (t%blk)*d.
+    """
+    Q = _u16(Q)
+    K = _u16(K)
+    V = _u16(V)
+    B, nq, Hq, d = Q.shape
+    idx = np.ascontiguousarray(idx, np.int32)
+    if G is None:
+        G = idx.shape[2]
+    S = idx.shape[3]
+    if bg_stride is None:
+        assert K.ndim == 4 and K.shape[0] == B and K.shape[1] == G and K.shape[3] == d
+        bg_stride = K.shape[2] * d
+        blk_stride = blk * d
+    O = np.empty((B, nq, Hq, d), np.float64)
+    _load().oracle_sparse_attention(B, nq, Hq, G, d, blk, T, q_start, float(scale), _ptr(Q),
+                                    _ptr(K), _ptr(V), int(bg_stride), int(blk_stride), _ptr(idx),
+                                    S, _ptr(O))
+    return O
+
+
+def dense_causal_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, q_start: int,
+                           scale: float = 0.0) -> np.ndarray:
+    """Textbook causal softmax attention.  Q [B][nq][Hq][d]; K/V [B][G][T][d]."""
+    Q = _u16(Q)
+    K = _u16(K)
+    V = _u16(V)
+    B, nq, Hq, d = Q.shape
+    G, T = K.shape[1], K.shape[2]
+    O = np.empty((B, nq, Hq, d), np.float64)
+    _load().oracle_dense_causal_attention(B, nq, Hq, G, d, T, q_start, float(scale), _ptr(Q),
+                                          _ptr(K), _ptr(V), _ptr(O))
+    return O
