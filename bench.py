@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the SparDA decode hot path on B200.
+
+Workload (one "step"): one decode token for B = 16 sequences at T = 131072
+through a 4-layer loop, 32 query heads in 8 GQA groups, head_dim 128, blocks
+of 64 tokens, top-k = 64 plus 1 initial and 2 local blocks.  Per layer l:
+  select  -- the layer's Forecast vectors F_l score layer l+1's compressed
+             keys (the last layer's select the next token's layer 0) and
+             keep init U top-k U local;
+  attend  -- the layer's queries attend over its selected 67 blocks.
+
+value  : decode tokens/s with every input resident in HBM (K/V of all four
+         layers, 34 GB, addressed by block id), timed with CUDA events.
+e2e    : the same loop through the C ABI with the K/V cache in pinned host
+         memory: per step Q and F are copied host->device, each layer's
+         selected blocks are gathered over the host link into device slots
+         on a side stream while the previous layer attends, and the output
+         is copied device->host.  Cold sets: every step refetches.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_sparda_b200 import workloads as W  # noqa: E402
+
+WORKLOAD = W.WORKLOADS["decode_loop_b16_t128k"]
+METRIC = "decode tokens/s at B=16,T=128K (sparse attn+select, % HBM roofline); select us/layer"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sparda", choices=["sparda", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-offload e2e leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="bound on the oracle's CPU-baseline sample")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# process plumbing
+# --------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, local):
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.path = tempfile.mktemp(prefix="sparda_clocks_", suffix=".csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), "--query-gpu=" + q, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    smax = float(c[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# the decode loop on one GPU
+# --------------------------------------------------------------------------
+
+class DecodeLoop:
+    def __init__(self, w: W.Workload, with_host: bool, seed_offset: int = 0):
+        import torch
+        from block_sparse_long_sparda_b200 import abi
+        self.torch, self.abi, self.w = torch, abi, w
+        dev = torch.device("cuda")
+        B, G, Hq, d, L, NB, S = w.B, w.G, w.Hq, w.d, w.layers, w.NB, w.S
+        self.p = abi.make_params(B, Hq, G, w.T, w.k, w.n_init, w.n_local)
+        seed = w.seed + 1000 * seed_offset
+        self.blk_elems = 2 * w.blk * d                      # one K|V block pair
+        # K/V cache of every layer, host layout [L][B][G][NB][2][64][128]
+        self.kv = torch.empty(L, B, G, NB, 2, w.blk, d, dtype=torch.bfloat16, device=dev)
+        for l in range(L):
+            W.torch_normal_bf16_(self.kv[l], seed * 16 + l)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed * 16 + 15)
+        self.Q = torch.randn(L, B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+        self.F = torch.randn(L, B, G, d, generator=gen, device=dev).to(torch.bfloat16)
+        # compressed keys of every layer (each block pooled as its own 64-token run)
+        self.kc = torch.empty(L, B, G, NB, d, dtype=torch.bfloat16, device=dev)
+        pc = abi.make_params(1, B * G * NB, B * G * NB, w.blk, 1)
+        for l in range(L):
+            abi.sparda_compress_keys(pc, self.kv[l], self.blk_elems, d, None, self.kc[l])
+        self.idx = torch.empty(L, B, G, S, dtype=torch.int32, device=dev)
+        self.O = torch.empty(L, B, Hq, d, dtype=torch.bfloat16, device=dev)
+        self.ws_sel = [abi.workspace(abi.SPARDA_OP_SELECT, self.p, 1, 1) for _ in range(L)]
+        self.ws_att = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, self.p)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        # layer 0's set comes from the previous token's last layer
+        abi.sparda_forecast_select(self.p, self.F[L - 1], 1, 1, w.T - 1, self.kc[0], self.idx[0],
+                                   self.ws_sel[0])
+        self.compute = torch.cuda.current_stream()
+        self.host_kv = None
+        if with_host:
+            self._setup_host()
+        torch.cuda.synchronize()
+
+    # ---- resident: all K/V in HBM, addressed by block id ----
+    def step_resident(self, ev=None):
+        abi, w = self.abi, self.w
+        L = w.layers
+        bg = w.NB * self.blk_elems
+        for l in range(L):
+            nxt = (l + 1) % L
+            if ev is not None:
+                ev[l][0].record()
+            abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
+                                       self.idx[nxt], self.ws_sel[l])
+            if ev is not None:
+                ev[l][1].record()
+            kv = self.kv[l]
+            abi.sparda_sparse_attn_decode(self.p, self.Q[l], kv, kv.view(-1)[w.blk * w.d:], bg,
+                                          self.blk_elems, self.idx[l], abi.SPARDA_ADDR_LOGICAL,
+                                          self.O[l], self.ws_att, self.status)
+            if ev is not None:
+                ev[l][2].record()
+
+    # ---- host offload: K/V in pinned host memory, gathered into slots ----
+    def _setup_host(self):
+        torch, w = self.torch, self.w
+        L = w.layers
+        nbytes = self.kv.numel() * 2
+        self.host_kv = torch.empty(self.kv.shape, dtype=torch.bfloat16)
+        rc = torch.cuda.cudart().cudaHostRegister(self.host_kv.data_ptr(), nbytes, 0)
+        if int(rc) != 0:
+            raise RuntimeError("cudaHostRegister of %.1f GB failed (%s)" % (nbytes / 1e9, rc))
+        self.host_kv.copy_(self.kv)
+        dev = torch.device("cuda")
+        self.slots = torch.empty(L, w.B, w.G, w.S, 2, w.blk, w.d, dtype=torch.bfloat16, device=dev)
+        # initial and local blocks stay resident in their slots (the same every step
+        # at a fixed decode position); top-k slots are refetched every step
+        c = (w.T - 1) // w.blk
+        for l in range(L):
+            self.slots[l, :, :, 0] = self.kv[l, :, :, 0]
+            for s in range(w.n_local):
+                self.slots[l, :, :, w.S - w.n_local + s] = self.kv[l, :, :, c - w.n_local + 1 + s]
+        self.side = torch.cuda.Stream()
+        self.sel_ev = [torch.cuda.Event() for _ in range(L)]
+        self.fetch_ev = [torch.cuda.Event() for _ in range(L)]
+        self.h_Q = self.Q.cpu().pin_memory()
+        self.h_F = self.F.cpu().pin_memory()
+        self.h_O = torch.empty(self.O.shape, dtype=torch.bfloat16).pin_memory()
+        # prime: layer 0's blocks for the first step
+        self.abi.sparda_prefetch_blocks(self.p, self.host_kv[0], self.idx[0], self.slots[0], True, 0,
+                                        self.status)
+        for l in range(L):
+            self.fetch_ev[l].record()
+
+    def unregister(self):
+        if self.host_kv is not None:
+            self.torch.cuda.cudart().cudaHostUnregister(self.host_kv.data_ptr())
+            self.host_kv = None
+
+    def step_e2e(self):
+        torch, abi, w = self.torch, self.abi, self.w
+        L = w.layers
+        self.Q.copy_(self.h_Q, non_blocking=True)
+        self.F.copy_(self.h_F, non_blocking=True)
+        bg = w.S * self.blk_elems
+        for l in range(L):
+            nxt = (l + 1) % L
+            abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
+                                       self.idx[nxt], self.ws_sel[l])
+            self.sel_ev[l].record(self.compute)
+            self.side.wait_event(self.sel_ev[l])
+            abi.sparda_prefetch_blocks(self.p, self.host_kv[nxt], self.idx[nxt], self.slots[nxt],
+                                       True, 0, self.status, stream=self.side)
+            self.fetch_ev[nxt].record(self.side)
+            self.compute.wait_event(self.fetch_ev[l])
+            sl = self.slots[l]
+            abi.sparda_sparse_attn_decode(self.p, self.Q[l], sl, sl.view(-1)[w.blk * w.d:], bg,
+                                          self.blk_elems, self.idx[l], abi.SPARDA_ADDR_SLOT,
+                                          self.O[l], self.ws_att, self.status)
+        self.h_O.copy_(self.O, non_blocking=True)
+
+    # algorithmic bytes per launch
+    def bytes_select(self):
+        w = self.w
+        ncand = (w.T - 1) // w.blk - w.n_local + 1 - w.n_init
+        return w.B * w.G * (ncand * w.d * 2 + w.d * 2 + w.S * 4)
+
+    def bytes_attn(self):
+        w = self.w
+        return w.B * w.G * w.S * self.blk_elems * 2 + 2 * w.B * w.Hq * w.d * 2 + w.B * w.G * w.S * 4
+
+
+def time_steps(fn, steps, world):
+    import torch
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    end.record()
+    end.synchronize()
+    ms = start.elapsed_time(end)
+    barrier(world)
+    return max_over_ranks(ms, world)
+
+
+# --------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample
+# --------------------------------------------------------------------------
+
+def oracle_baseline(loop: DecodeLoop, seconds: float):
+    """Time the fp64 oracle's select + attention for the same 4-layer loop on a
+    sample of the sequences (the compressed keys it scores are pooled by the
+    oracle itself from the same K/V bytes, outside the timed region)."""
+    import oracle
+    w = loop.w
+    import torch
+    nb = 1                                                   # sequences in the sample
+    L, G, NB, d, blk = w.layers, w.G, w.NB, w.d, w.blk
+
+    def bits(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    kv = [bits(loop.kv[l, :nb]) for l in range(L)]
+    Q = bits(loop.Q[:, :nb])
+    F = bits(loop.F[:, :nb])
+    kc = []
+    for l in range(L):
+        _, kcb = oracle.compress_keys(kv[l], blk, shape=(1, nb * G * NB, blk, d),
+                                      strides=(2 * blk * d, d))
+        kc.append(kcb.reshape(nb, G, NB, d))
+    idx0, _, _ = oracle.select(F[L - 1].reshape(nb, 1, G, 1, d), kc[0], w.k, w.n_init, w.n_local, w.T - 1)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        idx = idx0
+        for l in range(L):
+            nxt = (l + 1) % L
+            nidx, _, _ = oracle.select(F[l].reshape(nb, 1, G, 1, d), kc[nxt], w.k, w.n_init,
+                                       w.n_local, w.T - 1)
+            oracle.sparse_attention(Q[l].reshape(nb, 1, w.Hq, d), kv[l].reshape(-1),
+                                    kv[l].reshape(-1)[blk * d:], idx, w.T - 1, w.T, blk,
+                                    bg_stride=NB * 2 * blk * d, blk_stride=2 * blk * d, G=G)
+            idx = nidx
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 1000:
+            break
+    return {"value": nb * reps / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "%d of %d sequences x %d layers (select + sparse attention), %d reps, %.1f s"
+                      % (nb, w.B, L, reps, el)}
+
+
+# --------------------------------------------------------------------------
+# arms
+# --------------------------------------------------------------------------
+
+def run_sparda(args):
+    import torch
+    rank, world, local = dist_env()
+    init_dist(world, local)
+    from block_sparse_long_sparda_b200 import build
+    build.build()
+    w = WORKLOAD
+    want_e2e = not args.no_e2e
+    loop = DecodeLoop(w, with_host=want_e2e, seed_offset=rank)
+    L = w.layers
+
+    for _ in range(max(args.warmup, 3)):
+        loop.step_resident()
+    clocks = ClockSampler(local)
+    ms = time_steps(loop.step_resident, args.steps, world)
+    clk = clocks.stop()
+    # per-kernel durations inside a second timed pass on the same stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]
+    sel_ms, att_ms = [], []
+    for _ in range(args.steps):
+        loop.step_resident(evs)
+        torch.cuda.synchronize()
+        for l in range(L):
+            sel_ms.append(evs[l][0].elapsed_time(evs[l][1]))
+            att_ms.append(evs[l][1].elapsed_time(evs[l][2]))
+    st = int(loop.status.item())
+
+    ms_step = ms / args.steps
+    tokens = w.B * world
+    value = tokens / (ms_step / 1e3)
+    peak, peak_kind = measured_peaks()
+    att_us = statistics.mean(att_ms) * 1e3
+    sel_us = statistics.mean(sel_ms) * 1e3
+    att_gbs = loop.bytes_attn() / (att_us * 1e-6) / 1e9
+    sel_gbs = loop.bytes_select() / (sel_us * 1e-6) / 1e9
+    layer_bytes = loop.bytes_attn() + loop.bytes_select()
+    step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
+
+    e2e = None
+    if want_e2e:
+        for _ in range(max(args.warmup, 3)):
+            loop.step_e2e()
+        e_steps = max(3, min(args.steps, 10))
+        e_ms = time_steps(loop.step_e2e, e_steps, world) / e_steps
+        fetched = w.B * w.G * w.k * loop.blk_elems * 2 * L
+        e2e = {"value": w.B * world / (e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(loop.Q.numel() * 2 + loop.F.numel() * 2),
+               "d2h_bytes_per_step": int(loop.O.numel() * 2),
+               "ms_per_step": e_ms,
+               "host_link_bytes_per_step": fetched,
+               "host_link_GBps": fetched / (e_ms * 1e-3) / 1e9,
+               "note": "K/V in pinned host memory; every layer's top-k blocks gathered over the "
+                       "host link on a side stream (cold sets, no reuse across steps)"}
+        loop.unregister()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(loop, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "layers": L, "Hq": w.Hq,
+                       "G": w.G, "d": w.d, "block": w.blk, "k": w.k, "n_init": w.n_init,
+                       "n_local": w.n_local, "parallelism": "replicas" if world > 1 else "single",
+                       "kv": "all layers resident in HBM (34.4 GB), read by block id",
+                       "l2": "inputs larger than L2: 281 MB of selected K/V per layer, 4 layers"},
+            "select_us_per_layer": sel_us,
+            "attn_us_per_layer": att_us,
+            "select_GBps": sel_gbs,
+            "step_GBps": step_gbs,
+            "step_hbm_frac": step_gbs / peak,
+            "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel", "achieved": att_gbs,
+                         "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
+                         "traffic": None, "peak_kind": peak_kind,
+                         "bytes_per_launch": loop.bytes_attn()},
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "gpu_launches": args.steps * L * 3,
+            "device_status": st,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle (plain fp64 CPU code) on the host cores, same metric."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    import oracle
+    w = WORKLOAD
+    L, G, NB, d, blk = w.layers, w.G, w.NB, w.d, w.blk
+    nb = 1
+    rng = W.rng_for(w.seed, 99)
+    kv = [W.normal_bf16(rng, (nb, G, NB, 2, blk, d)) for _ in range(L)]
+    Q = W.normal_bf16(rng, (L, nb, w.Hq, d))
+    F = W.normal_bf16(rng, (L, nb, G, d))
+    kc = [oracle.compress_keys(kv[l], blk, shape=(1, nb * G * NB, blk, d), strides=(2 * blk * d, d))[1]
+          .reshape(nb, G, NB, d) for l in range(L)]
+    idx, _, _ = oracle.select(F[L - 1].reshape(nb, 1, G, 1, d), kc[0], w.k, w.n_init, w.n_local, w.T - 1)
+
+    def step():
+        nonlocal idx
+        for l in range(L):
+            nxt = (l + 1) % L
+            nidx, _, _ = oracle.select(F[l].reshape(nb, 1, G, 1, d), kc[nxt], w.k, w.n_init, w.n_local, w.T - 1)
+            oracle.sparse_attention(Q[l].reshape(nb, 1, w.Hq, d), kv[l].reshape(-1), kv[l].reshape(-1)[blk * d:],
+                                    idx, w.T - 1, w.T, blk, bg_stride=NB * 2 * blk * d,
+                                    blk_stride=2 * blk * d, G=G)
+            idx = nidx
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    v = nb * args.steps / el
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "layers": L, "Hq": w.Hq, "G": G,
+                   "d": d, "block": blk, "k": w.k},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "%d of %d sequences per step x %d layers (select + sparse "
+                                   "attention)" % (nb, w.B, L)},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_sparda(args)
+
+
+if __name__ == "__main__":
+    main()

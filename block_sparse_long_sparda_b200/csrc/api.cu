@@ -1,0 +1,176 @@
+// api.cu -- the extern "C" entry points of libsparda: argument validation on
+// the host, workspace sizing, and dispatch to the kernels.  Nothing here
+// synchronizes the device; every launch is checked with cudaGetLastError.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/sparda.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace sparda;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// shapes every entry point shares; returns a status
+int check_params(const sparda_params *p) {
+  if (!p) return SPARDA_EINVAL;
+  if (p->B < 0 || p->Hq <= 0 || p->G <= 0 || p->T < 1 || p->k < 0 || p->n_init < 0 ||
+      p->n_local < 0)
+    return SPARDA_EINVAL;
+  if (p->Hq % p->G != 0) return SPARDA_EINVAL;
+  if (p->d != kD || p->blk != kBlk) return SPARDA_EUNSUPPORTED;
+  const int r = p->Hq / p->G;
+  if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16) return SPARDA_EUNSUPPORTED;
+  if (p->k > 1024 || p->n_init > 64 || p->n_local > 64) return SPARDA_EUNSUPPORTED;
+  if (p->k + p->n_init + p->n_local < 1) return SPARDA_EINVAL;
+  return SPARDA_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARDA_OK : SPARDA_ECUDA; }
+
+bool stride_ok(long long s) { return s > 0 && (s % 8) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int sparda_version(void) { return 100; }
+
+const char *sparda_status_string(int status) {
+  switch (status) {
+    case SPARDA_OK: return "SPARDA_OK";
+    case SPARDA_EINVAL: return "SPARDA_EINVAL: invalid argument (null/misaligned pointer or bad shape)";
+    case SPARDA_EUNSUPPORTED: return "SPARDA_EUNSUPPORTED: shape outside this version (d=128, blk=64, Hq/G in {1,2,4,8,16})";
+    case SPARDA_ECUDA: return "SPARDA_ECUDA: a CUDA call or kernel launch failed";
+    case SPARDA_ERANGE: return "SPARDA_ERANGE: a block id outside the sequence was skipped on the device";
+    case SPARDA_ETIMEOUT: return "SPARDA_ETIMEOUT: a bounded device-side wait gave up";
+    case SPARDA_EWORKSPACE: return "SPARDA_EWORKSPACE: workspace missing or too small";
+    default: return "SPARDA: unknown status";
+  }
+}
+
+int sparda_status_from_device(int32_t word) {
+  if (word & SPARDA_DEV_TIMEOUT) return SPARDA_ETIMEOUT;
+  if (word & SPARDA_DEV_RANGE) return SPARDA_ERANGE;
+  return SPARDA_OK;
+}
+
+size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf) {
+  if (check_params(p) != SPARDA_OK) return 0;
+  switch (op) {
+    case SPARDA_OP_SELECT:
+      return nq < 1 ? 0 : plan_select(*p, nq, nf < 1 ? 1 : nf).ws_bytes;
+    case SPARDA_OP_ATTN_DECODE:
+      return plan_decode(*p).ws_bytes;
+    case SPARDA_OP_ATTN_PREFILL:
+      return nq < 1 ? 0 : prefill_ws_bytes(*p, nq);
+    default:
+      return 0;
+  }
+}
+
+int sparda_compress_keys(const sparda_params *p, const void *K, long long bg_stride,
+                         long long tok_stride, float *kc_f32, void *kc_bf16,
+                         sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (p->B == 0) return SPARDA_OK;
+  if (!K || (!kc_f32 && !kc_bf16)) return SPARDA_EINVAL;
+  if (!aligned16(K) || (kc_f32 && !aligned16(kc_f32)) || (kc_bf16 && !aligned16(kc_bf16)))
+    return SPARDA_EINVAL;
+  if (!stride_ok(tok_stride) || !stride_ok(bg_stride) || tok_stride < kD) return SPARDA_EINVAL;
+  if (p->G > 1 && bg_stride < (long long)p->T * tok_stride) return SPARDA_EINVAL;
+  return from_cuda(launch_compress(*p, static_cast<const uint16_t *>(K), bg_stride, tok_stride,
+                                   kc_f32, static_cast<uint16_t *>(kc_bf16),
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
+                           const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
+                           sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
+  if (nf > 16) return SPARDA_EUNSUPPORTED;
+  if (p->B == 0) return SPARDA_OK;
+  if (!F || !kc || !idx) return SPARDA_EINVAL;
+  if (!aligned16(F) || !aligned16(kc) || !aligned16(idx)) return SPARDA_EINVAL;
+  const SelectPlan pl = plan_select(*p, nq, nf);
+  if (!select_supported(pl)) return SPARDA_EUNSUPPORTED;
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), nq, nf, q_start,
+                                 static_cast<const uint16_t *>(kc), idx, ws,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_prefetch_blocks(const sparda_params *p, const void *host_kv, const int32_t *idx,
+                           void *slots, int skip_resident, int n_ctas, int32_t *dev_status,
+                           sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (n_ctas < 0) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!host_kv || !idx || !slots) return SPARDA_EINVAL;
+  if (!aligned16(host_kv) || !aligned16(idx) || !aligned16(slots)) return SPARDA_EINVAL;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, host_kv) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SPARDA_EINVAL;
+  }
+  if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr) return SPARDA_EINVAL;
+  const uint16_t *dev_view = static_cast<const uint16_t *>(attr.devicePointer);
+  if (!aligned16(dev_view)) return SPARDA_EINVAL;
+  return from_cuda(launch_prefetch(*p, dev_view, idx, static_cast<uint16_t *>(slots),
+                                   skip_resident, n_ctas, dev_status,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void *K,
+                              const void *V, long long bg_stride, long long blk_stride,
+                              const int32_t *idx, int addr_mode, void *O, void *ws,
+                              size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (addr_mode != SPARDA_ADDR_LOGICAL && addr_mode != SPARDA_ADDR_SLOT) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!Q || !K || !V || !idx || !O) return SPARDA_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O))
+    return SPARDA_EINVAL;
+  if (!stride_ok(bg_stride) || !stride_ok(blk_stride) || blk_stride < (long long)kBlk * kD)
+    return SPARDA_EINVAL;
+  const DecodePlan pl = plan_decode(*p);
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  return from_cuda(launch_attn_decode(*p, pl, static_cast<const uint16_t *>(Q),
+                                      static_cast<const uint16_t *>(K),
+                                      static_cast<const uint16_t *>(V), bg_stride, blk_stride,
+                                      idx, addr_mode, static_cast<uint16_t *>(O), ws, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, int q_start,
+                               const void *K, const void *V, long long bg_stride,
+                               long long tok_stride, const int32_t *idx, void *O, void *ws,
+                               size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (nq < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!Q || !K || !V || !idx || !O) return SPARDA_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O))
+    return SPARDA_EINVAL;
+  if (!stride_ok(bg_stride) || !stride_ok(tok_stride) || tok_stride < kD) return SPARDA_EINVAL;
+  if (tok_stride != kD) return SPARDA_EUNSUPPORTED;  // rows of a block must be contiguous
+  const size_t need = prefill_ws_bytes(*p, nq);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  return from_cuda(launch_attn_prefill(*p, static_cast<const uint16_t *>(Q), nq, q_start,
+                                       static_cast<const uint16_t *>(K),
+                                       static_cast<const uint16_t *>(V), bg_stride, tok_stride,
+                                       idx, static_cast<uint16_t *>(O), ws, ws_bytes, dev_status,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// compress.cu -- mean-pooled compressed keys (one per block of 64 tokens).
+//
+// [p1 "架构细节"]: the top-k part of a layer's block set is scored against the
+// block-mean of that layer's keys; [p4 "The problem InfLLM-V2 leaves on the
+// table"]: keys are mean-pooled into one compressed key per block.
+//
+// Design (B200): pure HBM streaming, 1/64 of the bytes written back.  One warp
+// owns one (b, g, block): lanes 0-15 cover one 256-byte key row with 16-byte
+// non-allocating loads, lanes 16-31 the next row, so every load instruction of
+// the warp reads two whole rows (512 contiguous bytes when rows are packed).
+// Eight rows per lane are in flight before any arithmetic.  fp32 accumulation,
+// one shuffle to join the two half-warps, IEEE division by the row count.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sparda {
+
+namespace {
+
+__device__ __forceinline__ void acc8(float (&a)[8], uint4 v) {
+  a[0] += bf16_lo(v.x);
+  a[1] += bf16_hi(v.x);
+  a[2] += bf16_lo(v.y);
+  a[3] += bf16_hi(v.y);
+  a[4] += bf16_lo(v.z);
+  a[5] += bf16_hi(v.z);
+  a[6] += bf16_lo(v.w);
+  a[7] += bf16_hi(v.w);
+}
+
+template <bool kContig>
+__global__ void __launch_bounds__(256, 3) compress_kernel(const uint16_t *__restrict__ K,
+                                                       long long bg_stride, long long tok_stride,
+                                                       int T, int NB, long long n_items,
+                                                       float *__restrict__ kc32,
+                                                       uint16_t *__restrict__ kc16) {
+  const int lane = threadIdx.x & 31;
+  const long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (item >= n_items) return;
+  const long long bg = item / NB;
+  const int j = (int)(item - bg * NB);
+  const int t0 = j * kBlk;
+  const int n = min(kBlk, T - t0);
+  const int half = lane >> 4;
+  const int c8 = lane & 15;
+  if (kContig) tok_stride = kD;  // rows packed: constant offsets, fewer live registers
+  const uint16_t *base = K + bg * bg_stride + (long long)t0 * tok_stride + c8 * 8;
+
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (n == kBlk) {
+#pragma unroll
+    for (int r0 = 0; r0 < kBlk / 2; r0 += 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = ldg_stream(base + (long long)(2 * (r0 + u) + half) * tok_stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc8(a, v[u]);
+    }
+  } else {
+    for (int t = half; t < n; t += 2) acc8(a, ldg_stream(base + (long long)t * tok_stride));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+  if (half) return;
+
+  const float fn = (float)n;
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = a[e] / fn;
+  if (kc32) {
+    float4 *o = reinterpret_cast<float4 *>(kc32 + item * kD + c8 * 8);
+    o[0] = make_float4(m[0], m[1], m[2], m[3]);
+    o[1] = make_float4(m[4], m[5], m[6], m[7]);
+  }
+  if (kc16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e]));
+      uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e + 1]));
+      w[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(kc16 + item * kD + c8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
+                            long long tok_stride, float *kc32, uint16_t *kc16,
+                            cudaStream_t stream) {
+  const int NB = (p.T + kBlk - 1) / kBlk;
+  const long long items = (long long)p.B * p.G * NB;
+  if (items == 0) return cudaSuccess;
+  const int warps = 8;
+  const long long grid = ceil_div_ll(items, warps);
+  if (tok_stride == kD)
+    compress_kernel<true><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride, p.T,
+                                                                   NB, items, kc32, kc16);
+  else
+    compress_kernel<false><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride,
+                                                                    p.T, NB, items, kc32, kc16);
+  return cudaGetLastError();
+}
+
+}  // namespace sparda

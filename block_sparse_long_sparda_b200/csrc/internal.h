@@ -1,0 +1,85 @@
+// internal.h -- launchers shared between the kernels and the C-ABI layer.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sparda.h"
+
+namespace sparda {
+
+// The three parts of a query's block set (eq. B_l(i) of the pages):
+// initial [0, init_hi), candidates [cand_lo, cand_hi), local [local_lo, c].
+struct BlockParts {
+  int c, init_hi, cand_lo, cand_hi, local_lo;
+};
+
+__host__ __device__ inline BlockParts block_parts(int pos, int blk, int n_init, int n_local) {
+  BlockParts r;
+  r.c = pos / blk;
+  r.local_lo = r.c - n_local + 1;
+  if (r.local_lo < 0) r.local_lo = 0;
+  r.init_hi = n_init < r.local_lo ? n_init : r.local_lo;
+  r.cand_lo = n_init;
+  r.cand_hi = r.local_lo > r.cand_lo ? r.local_lo : r.cand_lo;
+  return r;
+}
+
+// ---- compress -------------------------------------------------------------
+cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
+                            long long tok_stride, float *kc32, uint16_t *kc16,
+                            cudaStream_t stream);
+
+// ---- select ---------------------------------------------------------------
+struct SelectPlan {
+  long long n_problems;  // B * nq * G
+  int ncand_max;         // candidates of a query at the end of the sequence
+  int CH;                // candidate blocks scored per thread block
+  int n_chunks;          // thread blocks per problem
+  int kc;                // candidates kept per chunk: min(k, CH)
+  size_t ws_bytes;
+};
+SelectPlan plan_select(const sparda_params &p, int nq, int nf);
+int select_supported(const SelectPlan &plan);
+cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const uint16_t *F,
+                          int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,
+                          void *ws, cudaStream_t stream);
+
+// ---- prefetch -------------------------------------------------------------
+cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
+                            const int32_t *idx, uint16_t *slots, int skip_resident, int n_ctas,
+                            int32_t *dev_status, cudaStream_t stream);
+
+// ---- decode attention -----------------------------------------------------
+struct DecodePlan {
+  int S;            // list entries per (b, g)
+  int bps;          // list entries per split
+  int n_split;      // splits per (b, g)
+  size_t ws_bytes;  // partial results
+};
+DecodePlan plan_decode(const sparda_params &p);
+DecodePlan plan_gather(const sparda_params &p, long long pairs);
+// one query per (sequence, token, group) "pair", each with its own block list
+cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int nq, int q_start,
+                               const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                               long long bg_stride, long long blk_stride, const int32_t *idx,
+                               int addr_mode, uint16_t *O, void *ws, int32_t *dev_status,
+                               cudaStream_t stream);
+cudaError_t launch_attn_decode(const sparda_params &p, const DecodePlan &plan,
+                               const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                               long long bg_stride, long long blk_stride, const int32_t *idx,
+                               int addr_mode, uint16_t *O, void *ws, int32_t *dev_status,
+                               cudaStream_t stream);
+
+// ---- prefill attention ----------------------------------------------------
+size_t prefill_ws_bytes(const sparda_params &p, int nq);
+cudaError_t launch_attn_prefill(const sparda_params &p, const uint16_t *Q, int nq, int q_start,
+                                const uint16_t *K, const uint16_t *V, long long bg_stride,
+                                long long tok_stride, const int32_t *idx, uint16_t *O, void *ws,
+                                size_t ws_bytes, int32_t *dev_status, cudaStream_t stream);
+
+// environment overrides used for tuning sweeps (0 when unset)
+int env_int(const char *name);
+
+}  // namespace sparda

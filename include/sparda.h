@@ -1,0 +1,220 @@
+/*
+ * sparda.h -- C ABI of libsparda, the B200 (sm_100a) hot path of SparDA
+ * (Sparse Decoupled Attention): Forecast-driven lookahead block selection
+ * plus GQA block-sparse attention.
+ *
+ * Sources: "SparDA: a fourth projection that lets sparse attention prefetch
+ * its own KV cache" (ai.thesatyajit.com/articles/sparda) -- cited below as
+ * [p4 <section>] -- and deepresearch2agi.pages.dev/sparda_sparse_decoupled_attention
+ * -- cited as [p1 <section>].
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Return value: SPARDA_OK (0) or a negative status below.  Arguments are
+ *    validated on the host before anything is enqueued; a call that returns
+ *    an error has enqueued nothing, except SPARDA_ECUDA, which reports a
+ *    launch failure (cudaGetLastError after the launch; the call never
+ *    synchronizes).
+ *  - Calls are asynchronous on the given stream (a cudaStream_t; NULL means
+ *    the legacy default stream).  The library keeps no global state; calls
+ *    on different streams with disjoint buffers may run concurrently.
+ *  - All buffers are owned by the caller.  Device buffers are plain device
+ *    pointers; every pointer must be 16-byte aligned and every row stride a
+ *    multiple of 8 elements (16 bytes).
+ *  - bf16 tensors are passed as `const void *` to raw IEEE bfloat16 storage.
+ *  - Layouts are row-major, innermost index last.  Query head h belongs to
+ *    KV group (GQA group) h / (Hq / G).
+ *  - Supported shapes in this version: d = 128, blk = 64, Hq / G in
+ *    {1, 2, 4, 8, 16}; other values return SPARDA_EUNSUPPORTED.
+ *  - Block j of a sequence holds token positions [j*blk, (j+1)*blk).
+ *    NB = ceil(T / blk).  For a query at position pos, c = pos / blk is its
+ *    own block; its set is B = init U local U topk [p4 "The problem
+ *    InfLLM-V2 leaves on the table", eq. B_l(i)] with
+ *      local = [max(0, c - n_local + 1), c],
+ *      init  = [0, n_init) minus the local blocks,
+ *      topk  = the k best-scoring candidate blocks [n_init, c - n_local + 1),
+ *    stored as S = k + n_init + n_local int32 block ids in ascending order,
+ *    padded with -1 at the end when fewer blocks exist.
+ *  - dev_status (optional, device int32): kernels OR device-side findings
+ *    into it (SPARDA_DEV_RANGE: a block id outside [0, NB) or after the
+ *    query's own block was skipped; SPARDA_DEV_TIMEOUT: a bounded wait gave
+ *    up).  The caller zeroes it, reads it after synchronizing, and may turn
+ *    it into a status with sparda_status_from_device().
+ */
+#ifndef SPARDA_H_
+#define SPARDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *sparda_stream_t; /* == cudaStream_t */
+
+enum sparda_status {
+  SPARDA_OK = 0,
+  SPARDA_EINVAL = -1,       /* null / misaligned pointer, bad shape or size          */
+  SPARDA_EUNSUPPORTED = -2, /* valid but outside this version's shapes (d, blk, r)   */
+  SPARDA_ECUDA = -3,        /* a CUDA call or kernel launch failed                   */
+  SPARDA_ERANGE = -4,       /* device-side bounds finding (from the status word)     */
+  SPARDA_ETIMEOUT = -5,     /* a bounded device-side wait gave up                    */
+  SPARDA_EWORKSPACE = -6    /* workspace missing or smaller than sparda_workspace_size */
+};
+
+enum sparda_device_status_bits {
+  SPARDA_DEV_RANGE = 1,
+  SPARDA_DEV_TIMEOUT = 2
+};
+
+/* Shapes shared by every call.  T is the number of tokens present in the
+ * sequence (the context length); the decode query sits at position T - 1. */
+typedef struct sparda_params {
+  int B;        /* batch (sequences); B = 0 is a valid empty call              */
+  int Hq;       /* query heads                                                 */
+  int G;        /* GQA groups = KV heads; Hq % G == 0                          */
+  int d;        /* head dimension (128)                                        */
+  int blk;      /* tokens per block (64)                                       */
+  int T;        /* tokens present, >= 1                                        */
+  int k;        /* top-k budget (>= 0, <= 1024)                                */
+  int n_init;   /* initial blocks (>= 0, <= 64)                                */
+  int n_local;  /* local-window blocks (>= 0, <= 64)                           */
+  float scale;  /* attention logit scale; <= 0 means 1/sqrt(d)                 */
+} sparda_params;
+
+/* ops for sparda_workspace_size */
+enum sparda_op {
+  SPARDA_OP_COMPRESS = 0,
+  SPARDA_OP_SELECT = 1,
+  SPARDA_OP_PREFETCH = 2,
+  SPARDA_OP_ATTN_DECODE = 3,
+  SPARDA_OP_ATTN_PREFILL = 4
+};
+
+/* how sparda_sparse_attn_decode finds the storage of list entry s */
+enum sparda_addr_mode {
+  SPARDA_ADDR_LOGICAL = 0, /* block id idx[s] indexes the K/V buffer (KV resident)   */
+  SPARDA_ADDR_SLOT = 1     /* list position s indexes it (prefetched device slots)  */
+};
+
+/*
+ * sparda_compress_keys -- mean-pooled compressed keys.
+ *   [p1 "架构细节"]: top-k blocks are scored against the block-mean of the
+ *   layer's keys; [p4 "The problem InfLLM-V2 leaves on the table"]: keys are
+ *   mean-pooled into one compressed key per block.
+ *   Kc[b,g,j,:] = (1/n_j) sum_{t in block j, t < T} K[b,g,t,:]
+ * K        bf16, row (b,g,t) at K + (b*G+g)*bg_stride + t*tok_stride (elements)
+ * kc_f32   float [B][G][NB][d] or NULL
+ * kc_bf16  bf16  [B][G][NB][d] or NULL (round-to-nearest-even of the fp32 mean)
+ * At least one output must be non-NULL.  Accumulation is fp32.
+ */
+int sparda_compress_keys(const sparda_params *p, const void *K, long long bg_stride,
+                         long long tok_stride, float *kc_f32, void *kc_bf16,
+                         sparda_stream_t stream);
+
+/*
+ * sparda_forecast_select -- block sets from Forecast scores.
+ *   [p4 "The fourth projection", Eq. 4]:
+ *     B_{l+1} = B_init U B_local U f_top(F_l Kc_{l+1}^T, k)
+ *   [p4 "One Forecast head per GQA group"]: one Forecast vector per GQA group,
+ *   raw dot-product scores, top-k with no softmax.  With nf > 1 the nf
+ *   vectors of a group are the group's query heads and their scores are
+ *   summed: the multi-head baseline selector of the same section (whose
+ *   softmax after the sum cannot change the ranking and is not applied).
+ * F     bf16 [B][nq][G][nf][d]   (nf = 1: Forecast; nf = Hq/G: baseline)
+ * kc    bf16 [B][G][NB][d]       compressed keys of the layer being selected
+ * idx   int32 [B][nq][G][S]      output, ascending block ids, -1 padded
+ * Query token i sits at position q_start + i; 0 <= q_start, q_start + nq <= T.
+ * nq = 1 is the decode path; nq > 1 scores every query token (prefill).
+ * Ranking: higher fp32 score first, equal scores -> lower block index.
+ * ws    device workspace of sparda_workspace_size(SPARDA_OP_SELECT, p, nq, nf)
+ *       bytes; it must be zero-filled before its first use, and each call
+ *       leaves it zero-filled again.  Calls sharing one workspace must not
+ *       overlap on the device.
+ */
+int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
+                           const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
+                           sparda_stream_t stream);
+
+/*
+ * sparda_prefetch_blocks -- gather the selected K/V blocks of one layer from
+ * page-locked host memory into device slots, read by the GPU over the
+ * host link (zero-copy), so the block ids never travel back to the host.
+ *   [p4 "The fourth projection", Algorithm 2]: fetch(B_next, src = CPU
+ *   pinned, dst = GPU) launched on a dedicated prefetch stream; [p1
+ *   "UVA异步预取管线"]: the number of thread blocks adapts to the batch.
+ * host_kv  bf16 [B][G][NB][2][blk][d] (K block then V block), page-locked
+ *          and mapped (cudaHostAlloc(..., cudaHostAllocMapped) or
+ *          cudaHostRegister(..., cudaHostRegisterMapped)); the host pointer
+ *          is translated with cudaPointerGetAttributes.  Not pinned/mapped
+ *          -> SPARDA_EINVAL.
+ * idx      int32 [B][G][S] device, the layer's block sets (decode position T-1)
+ * slots    bf16 [B][G][S][2][blk][d] device; slot s receives block idx[s]
+ * skip_resident  nonzero: initial and local entries are not copied (the
+ *          caller keeps them resident in their slots); -1 entries never are.
+ * n_ctas   thread blocks to use, 0 = chosen from B
+ * A block id outside [0, NB) is skipped and flagged SPARDA_DEV_RANGE.
+ */
+int sparda_prefetch_blocks(const sparda_params *p, const void *host_kv, const int32_t *idx,
+                           void *slots, int skip_resident, int n_ctas, int32_t *dev_status,
+                           sparda_stream_t stream);
+
+/*
+ * sparda_sparse_attn_decode -- one decode query per sequence attends over
+ * the keys of its group's block set only, fp32 softmax and accumulation.
+ *   [p4 "The fourth projection", Eq. 5 / Algorithm 2]:
+ *     O_l = attention(Q_l, K_l[B_l], V_l[B_l])
+ * Q     bf16 [B][Hq][d], query at position T-1
+ * K, V  bf16; the block stored for list entry s of (b,g) starts at
+ *         base + (b*G+g)*bg_stride + m*blk_stride   (elements)
+ *       with m = idx[b,g,s] (SPARDA_ADDR_LOGICAL) or m = s (SPARDA_ADDR_SLOT);
+ *       its blk rows are contiguous (row stride d).  Separate [B][G][T][d]
+ *       tensors: bg_stride = T*d, blk_stride = blk*d.  Interleaved
+ *       [..][2][blk][d] storage: V = K + blk*d, blk_stride = 2*blk*d.
+ * idx   int32 [B][G][S]; keys after position T-1 are masked; -1 skipped.
+ *       A list must not repeat a block.
+ * O     bf16 [B][Hq][d]
+ * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_DECODE, ...)
+ */
+int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void *K,
+                              const void *V, long long bg_stride, long long blk_stride,
+                              const int32_t *idx, int addr_mode, void *O, void *ws,
+                              size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream);
+
+/*
+ * sparda_sparse_attn_prefill -- every token of a query chunk attends over the
+ * keys of its own block set (per token and group), causal, fp32 softmax.
+ *   [p4 "The fourth projection", Algorithm 1 / Eq. 5]:
+ *     O_l = attention(Q_l, K_l[B_l], V_l[B_l])   with all keys on the GPU
+ * Q     bf16 [B][nq][Hq][d]; token i at position q_start + i <= T - 1
+ * K, V  bf16, row (b,g,t) at base + (b*G+g)*bg_stride + t*tok_stride; this
+ *       version needs tok_stride == d (else SPARDA_EUNSUPPORTED)
+ * idx   int32 [B][nq][G][S] (as produced by sparda_forecast_select)
+ * O     bf16 [B][nq][Hq][d]
+ * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_PREFILL, p, nq, 0)
+ */
+int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, int q_start,
+                               const void *K, const void *V, long long bg_stride,
+                               long long tok_stride, const int32_t *idx, void *O, void *ws,
+                               size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream);
+
+/* Bytes of device workspace an op needs for these shapes (0: none). nf is
+ * the number of scoring vectors per group (select only). */
+size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf);
+
+/* Human-readable name of a status code (static string). */
+const char *sparda_status_string(int status);
+
+/* Map a device status word to SPARDA_OK / SPARDA_ERANGE / SPARDA_ETIMEOUT. */
+int sparda_status_from_device(int32_t word);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sparda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARDA_H_ */

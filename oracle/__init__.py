@@ -94,17 +94,26 @@ def bf16_to_double(bits: int) -> float:
     return float(_load().oracle_bf16_to_double(int(bits)))
 
 
-def compress_keys(K: np.ndarray, blk: int = 64):
+def compress_keys(K: np.ndarray, blk: int = 64, shape=None, strides=None):
     """Mean-pooled compressed keys.
 
     K: uint16 [B][G][T][d].  Returns (kc_f64 [B][G][NB][d], kc_bf16 [B][G][NB][d]).
+    With ``shape=(B, G, T, d)`` and ``strides=(bg_stride, tok_stride)`` (elements)
+    K may be any buffer holding row (b,g,t) at (b*G+g)*bg_stride + t*tok_stride.
     """
     K = _u16(K)
-    B, G, T, d = K.shape
+    if shape is None:
+        B, G, T, d = K.shape
+        bg_stride, tok_stride = T * d, d
+    else:
+        B, G, T, d = shape
+        bg_stride, tok_stride = strides
+        assert (B * G - 1) * bg_stride + (T - 1) * tok_stride + d <= K.size
     NB = (T + blk - 1) // blk
     kc = np.empty((B, G, NB, d), np.float64)
     kcb = np.empty((B, G, NB, d), np.uint16)
-    _load().oracle_compress_keys(B, G, T, d, blk, _ptr(K), T * d, d, _ptr(kc), _ptr(kcb))
+    _load().oracle_compress_keys(B, G, T, d, blk, _ptr(K), bg_stride, tok_stride, _ptr(kc),
+                                 _ptr(kcb))
     return kc, kcb
 
 

@@ -1,0 +1,98 @@
+"""Helpers shared by the GPU parity tests: host<->device marshalling of bf16
+bit arrays and the comparison rules (spec tolerances).
+
+Comparison rules
+- compressed keys: fp32 output within 1e-3 max abs of the fp64 oracle; the
+  bf16 output equals the oracle's one-step rounding except for rare double
+  rounding (>= 99.99% identical, never more than one unit in the last place);
+- block sets: bit-exact wherever the oracle's k-th and (k+1)-th scores differ
+  by more than 1e-3 relative; inside that band any set that keeps every block
+  scoring clearly above the band and adds only blocks inside it is valid;
+- attention outputs: max abs error <= 1e-2 and relative L2 error <= 5e-3.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from block_sparse_long_sparda_b200 import workloads as W
+
+ATTN_MAX_ABS = 1e-2
+ATTN_REL_L2 = 5e-3
+KC_MAX_ABS = 1e-3
+TIE_REL = 1e-3
+
+
+def dev_bf16(a: np.ndarray, device="cuda") -> torch.Tensor:
+    """uint16 bf16 bits (numpy) -> torch.bfloat16 on the device."""
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    """torch.bfloat16 (any device) -> uint16 numpy bits."""
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_f64(bits: np.ndarray) -> np.ndarray:
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def check_attention(gpu_bits: np.ndarray, oracle_f64: np.ndarray, what: str = ""):
+    g = bf16_f64(gpu_bits)
+    o = np.asarray(oracle_f64, np.float64)
+    assert g.shape == o.shape, (g.shape, o.shape)
+    assert np.all(np.isfinite(g)), what + ": non-finite output"
+    err = np.abs(g - o)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel = float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30))
+    assert max_abs <= ATTN_MAX_ABS, "%s: max abs %.3e" % (what, max_abs)
+    assert rel <= ATTN_REL_L2, "%s: rel L2 %.3e" % (what, rel)
+    return max_abs, rel
+
+
+def check_compressed(kc32: np.ndarray, kc16: np.ndarray, ora64: np.ndarray, ora16: np.ndarray):
+    err = float(np.abs(kc32.astype(np.float64) - ora64).max())
+    assert err <= KC_MAX_ABS, "fp32 Kc max abs %.3e" % err
+    same = np.mean(kc16 == ora16)
+    assert same >= 0.9999, "bf16 Kc identical fraction %.6f" % same
+    diff = np.abs(kc16.astype(np.int32) - ora16.astype(np.int32))
+    assert diff.max() <= 1, "bf16 Kc differs by more than one ulp"
+    return err, same
+
+
+def scores_f64(F_bits: np.ndarray, kc_bits: np.ndarray) -> np.ndarray:
+    """Summed dot products in fp64 for the band rule.
+    F [B][nq][G][nf][d], kc [B][G][NB][d] -> [B][nq][G][NB]."""
+    F = bf16_f64(F_bits).sum(axis=3)                      # sum over the nf vectors
+    kc = bf16_f64(kc_bits)
+    return np.einsum("bqgd,bgnd->bqgn", F, kc)
+
+
+def check_sets(gpu_idx: np.ndarray, ora_idx: np.ndarray, kth: np.ndarray, kth1: np.ndarray,
+               scores: np.ndarray | None, what: str = ""):
+    """gpu_idx/ora_idx [B][nq][G][S]; kth/kth1 [B][nq][G]; scores [B][nq][G][NB]."""
+    assert gpu_idx.shape == ora_idx.shape, (gpu_idx.shape, ora_idx.shape)
+    exact = bitexact = 0
+    for pos in np.ndindex(*gpu_idx.shape[:3]):
+        g, o = gpu_idx[pos], ora_idx[pos]
+        a, b = kth[pos], kth1[pos]
+        clear = not np.isfinite(b) or not np.isfinite(a) or abs(a - b) > TIE_REL * abs(a)
+        if np.array_equal(g, o):
+            bitexact += 1
+            exact += clear
+            continue
+        assert not clear, "%s %s: sets differ with a clear k-th gap\n gpu %s\n ora %s" % (what, pos, g, o)
+        assert scores is not None, "%s %s: near tie but no scores to check the band" % (what, pos)
+        valid = g[g >= 0]
+        assert len(set(valid.tolist())) == len(valid), "duplicate ids"
+        hi = a + TIE_REL * abs(a)
+        lo = a - TIE_REL * abs(a)
+        sc = scores[pos]
+        gs, os_ = set(g.tolist()) - {-1}, set(o.tolist()) - {-1}
+        for j in os_ - gs:
+            assert sc[j] <= hi, "%s %s: dropped block %d scoring above the band" % (what, pos, j)
+        for j in gs - os_:
+            assert sc[j] >= lo, "%s %s: added block %d scoring below the band" % (what, pos, j)
+        assert np.all(np.diff(g[g >= 0]) > 0), "not ascending"
+    return bitexact

@@ -1,0 +1,97 @@
+"""The C-ABI library: it loads without a GPU, exports every entry point the
+header declares, and its host-side validation rejects bad arguments before
+anything reaches the device.  No compute calls here."""
+import ctypes
+
+import pytest
+
+from block_sparse_long_sparda_b200 import abi, build
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return abi.lib()
+
+
+def test_every_declared_entry_point_is_exported(L):
+    names = abi.header_functions()
+    expected = {"sparda_compress_keys", "sparda_forecast_select", "sparda_prefetch_blocks",
+                "sparda_sparse_attn_decode", "sparda_sparse_attn_prefill",
+                "sparda_workspace_size", "sparda_status_string", "sparda_status_from_device",
+                "sparda_version"}
+    assert expected <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in abi._SIGS, "binding lacks " + n
+
+
+def test_status_strings_and_device_word(L):
+    for st in range(0, -7, -1):
+        assert abi.sparda_status_string(st).startswith("SPARDA")
+    assert abi.sparda_status_from_device(0) == abi.SPARDA_OK
+    assert abi.sparda_status_from_device(abi.SPARDA_DEV_RANGE) == abi.SPARDA_ERANGE
+    assert abi.sparda_status_from_device(abi.SPARDA_DEV_TIMEOUT | abi.SPARDA_DEV_RANGE) == abi.SPARDA_ETIMEOUT
+    assert abi.sparda_version() >= 100
+
+
+def _status(fn, *args):
+    return getattr(abi.lib(), fn)(*args)
+
+
+NULL = None
+
+
+def test_validation_rejects_before_launch(L):
+    p = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8)
+    byref = ctypes.byref
+    fake = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10008)           # 8-byte aligned only
+    # unsupported head dim / block size / group ratio
+    for bad in (abi.make_params(2, 32, 8, 4096, 8, d=64), abi.make_params(2, 32, 8, 4096, 8, blk=32),
+                abi.make_params(2, 24, 8, 4096, 8)):
+        st = _status("sparda_compress_keys", byref(bad), fake, 4096 * 128, 128, fake, NULL, NULL)
+        assert st in (abi.SPARDA_EUNSUPPORTED,), st
+    # Hq not a multiple of G
+    st = _status("sparda_compress_keys", byref(abi.make_params(2, 30, 8, 4096, 8)), fake, 1, 128, fake, NULL, NULL)
+    assert st == abi.SPARDA_EINVAL
+    # null inputs, no outputs, misaligned pointer, bad stride
+    assert _status("sparda_compress_keys", byref(p), NULL, 4096 * 128, 128, fake, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_compress_keys", byref(p), fake, 4096 * 128, 128, NULL, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_compress_keys", byref(p), odd, 4096 * 128, 128, fake, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_compress_keys", byref(p), fake, 4096 * 128, 100, fake, NULL, NULL) == abi.SPARDA_EINVAL
+    # select: query positions outside the sequence, too many scoring vectors
+    assert _status("sparda_forecast_select", byref(p), fake, 1, 1, 4096, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_forecast_select", byref(p), fake, 0, 1, 0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_forecast_select", byref(p), fake, 1, 17, 4095, fake, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    # a multi-chunk select without its workspace
+    big = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, big, 1, 1) > 0
+    assert _status("sparda_forecast_select", byref(big), fake, 1, 1, 131071, fake, fake, NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
+    # decode attention: bad address mode, bad block stride
+    assert _status("sparda_sparse_attn_decode", byref(p), fake, fake, fake, 4096 * 128, 64 * 128, fake, 7,
+                   fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_sparse_attn_decode", byref(p), fake, fake, fake, 4096 * 128, 63 * 128, fake, 0,
+                   fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
+    # prefill: rows of a block must be contiguous in this version
+    assert _status("sparda_sparse_attn_prefill", byref(p), fake, 16, 4000, fake, fake, 4096 * 256, 256, fake,
+                   fake, NULL, 0, NULL, NULL) == abi.SPARDA_EUNSUPPORTED
+    # prefetch: negative CTA count
+    assert _status("sparda_prefetch_blocks", byref(p), fake, fake, fake, 1, -1, NULL, NULL) == abi.SPARDA_EINVAL
+    # empty batch is a valid no-op
+    empty = abi.make_params(B=0, Hq=32, G=8, T=4096, k=8)
+    assert _status("sparda_compress_keys", byref(empty), NULL, 0, 128, NULL, NULL, NULL) == abi.SPARDA_OK
+    # an empty block set is not a valid request
+    none = abi.make_params(B=1, Hq=8, G=2, T=4096, k=0, n_init=0, n_local=0)
+    assert _status("sparda_compress_keys", byref(none), fake, 4096 * 128, 128, fake, NULL, NULL) == abi.SPARDA_EINVAL
+
+
+def test_workspace_sizes_scale_with_shapes(L):
+    small = abi.make_params(B=1, Hq=16, G=2, T=4096, k=4)
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, small, 1, 1) >= 0
+    cfg3 = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
+    dec = abi.sparda_workspace_size(abi.SPARDA_OP_ATTN_DECODE, cfg3)
+    assert dec > 0 and dec < 64 << 20
+    # the workspace of an op with no scratch is zero
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_COMPRESS, cfg3) == 0
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_PREFETCH, cfg3) == 0

@@ -1,0 +1,360 @@
+"""GPU parity: every entry point of libsparda, called through the C ABI, against
+the fp64 CPU oracle on the same seeded inputs, at sizes the oracle finishes in
+seconds that still span several thread blocks and a ragged tail, plus the
+degenerate cases of the method."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_sparda_b200 import abi, build
+from block_sparse_long_sparda_b200 import workloads as W
+from tests.parity import (bf16_f64, check_attention, check_compressed, check_sets, dev_bf16,
+                          host_bits, scores_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    abi.lib()
+    torch.cuda.init()
+
+
+def gpu_compress(K_bits, blk=64):
+    B, G, T, d = K_bits.shape
+    p = abi.make_params(B, G, G, T, 1)
+    K = dev_bf16(K_bits)
+    NB = (T + blk - 1) // blk
+    kc32 = torch.empty(B, G, NB, d, dtype=torch.float32, device="cuda")
+    kc16 = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_keys(p, K, T * d, d, kc32, kc16)
+    torch.cuda.synchronize()
+    return kc32.cpu().numpy(), host_bits(kc16)
+
+
+def gpu_select(F_bits, kc_bits, k, n_init, n_local, q_start, T, Hq=None):
+    """F [B][nq][G][nf][d] bits, kc [B][G][NB][d] bits -> idx [B][nq][G][S]."""
+    B, nq, G, nf, d = F_bits.shape
+    p = abi.make_params(B, Hq or G * max(nf, 1), G, T, k, n_init, n_local)
+    S = k + n_init + n_local
+    idx = torch.full((B, nq, G, S), -7, dtype=torch.int32, device="cuda")
+    ws = abi.workspace(abi.SPARDA_OP_SELECT, p, nq, nf)
+    abi.sparda_forecast_select(p, dev_bf16(F_bits), nq, nf, q_start, dev_bf16(kc_bits), idx, ws)
+    torch.cuda.synchronize()
+    out = idx.cpu().numpy()
+    assert not (out == -7).any(), "entries left unwritten"
+    return out
+
+
+def gpu_decode(Q_bits, K_bits, V_bits, idx, T, k, n_init=1, n_local=2, addr_mode=0,
+               bg_stride=None, blk_stride=None, status=None):
+    B, Hq, d = Q_bits.shape
+    G = idx.shape[1]
+    p = abi.make_params(B, Hq, G, T, k, n_init, n_local)
+    K = dev_bf16(K_bits)
+    V = dev_bf16(V_bits) if V_bits is not None else None
+    if bg_stride is None:
+        bg_stride, blk_stride = K_bits.shape[2] * d, 64 * d
+    O = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    ws = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p)
+    didx = torch.from_numpy(np.ascontiguousarray(idx, np.int32)).cuda()
+    if V is None:  # interleaved storage: V rows follow the K rows of each block
+        V = K.view(-1)[64 * d:]
+    abi.sparda_sparse_attn_decode(p, dev_bf16(Q_bits), K, V, bg_stride, blk_stride, didx,
+                                  addr_mode, O, ws, status)
+    torch.cuda.synchronize()
+    return host_bits(O)
+
+
+# --------------------------------------------------------------------------
+# compressed keys
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [4096, 4096 + 37, 64, 1])
+def test_compress_parity(T):
+    rng = W.rng_for(7, T)
+    K = W.normal_bf16(rng, (2, 3, T, 128))
+    kc32, kc16 = gpu_compress(K)
+    ora, orab = oracle.compress_keys(K)
+    check_compressed(kc32, kc16, ora, orab)
+
+
+def test_compress_decode_b4_t32k_planted():
+    w = W.WORKLOADS["decode_b4_t32k_planted"]
+    x = W.decode_inputs(w)
+    kc32, kc16 = gpu_compress(x["K"])
+    ora, orab = oracle.compress_keys(x["K"])
+    check_compressed(kc32, kc16, ora, orab)
+
+
+def test_compress_strided_rows():
+    rng = W.rng_for(8)
+    B, G, T, d = 1, 2, 300, 128
+    big = W.normal_bf16(rng, (B, G, T, 2 * d))          # each token row padded to 2d
+    p = abi.make_params(B, G, G, T, 1)
+    kc32 = torch.empty(B, G, 5, d, dtype=torch.float32, device="cuda")
+    abi.sparda_compress_keys(p, dev_bf16(big), T * 2 * d, 2 * d, kc32, None)
+    torch.cuda.synchronize()
+    ora, _ = oracle.compress_keys(np.ascontiguousarray(big[..., :d]))
+    assert np.abs(kc32.cpu().numpy() - ora).max() <= 1e-3
+
+
+# --------------------------------------------------------------------------
+# selection
+# --------------------------------------------------------------------------
+
+def _select_case(F, kc, k, n_init, n_local, q_start, T, what):
+    ora, kth, kth1 = oracle.select(F, kc, k, n_init, n_local, q_start)
+    got = gpu_select(F, kc, k, n_init, n_local, q_start, T)
+    return check_sets(got, ora, kth, kth1, scores_f64(F, kc), what)
+
+
+@pytest.mark.parametrize("name", ["decode_b1_t4k", "decode_b4_t32k_planted"])
+def test_select_decode_configs(name):
+    w = W.WORKLOADS[name]
+    x = W.decode_inputs(w)
+    _, kcb = oracle.compress_keys(x["K"])
+    F = x["F"].reshape(w.B, 1, w.G, 1, w.d)
+    _select_case(F, kcb, w.k, w.n_init, w.n_local, w.T - 1, w.T, name)
+
+
+@pytest.mark.parametrize("NB,B", [(128, 1), (2048, 16), (16384, 1), (16384, 4), (1000, 3)])
+def test_select_sweep_points(NB, B):
+    x = W.sweep_inputs(NB, B)
+    F = x["F"].reshape(B, 1, 8, 1, 128)
+    _select_case(F, x["kc"], 64, 1, 2, NB * 64 - 1, NB * 64, "sweep NB=%d B=%d" % (NB, B))
+
+
+@pytest.mark.parametrize("chunk", ["256", "512", "8192"])
+def test_select_forced_chunking(chunk, monkeypatch):
+    monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    x = W.sweep_inputs(3000, 2)
+    F = x["F"].reshape(2, 1, 8, 1, 128)
+    _select_case(F, x["kc"], 64, 1, 2, 3000 * 64 - 1, 3000 * 64, "chunk " + chunk)
+
+
+def test_select_baseline_multihead():
+    x = W.sweep_inputs(2048, 2)
+    Qg = x["Q"].reshape(2, 1, 8, 4, 128)                 # 4 query heads per group, summed
+    _select_case(Qg, x["kc"], 64, 1, 2, 2048 * 64 - 1, 2048 * 64, "baseline")
+
+
+@pytest.mark.parametrize("chunk", ["0", "256"])
+def test_select_exact_ties_lower_index_wins(chunk, monkeypatch):
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    rng = np.random.default_rng(3)
+    NB, B, G, d = 1500, 2, 4, 128
+    kc = np.zeros((B, G, NB, d), np.float32)
+    kc[..., 0] = rng.integers(-3, 4, size=(B, G, NB))     # many exact ties
+    F = np.zeros((B, 1, G, 1, d), np.float32)
+    F[..., 0] = 1.0
+    Fb, kcb = W.f32_to_bf16_bits(F), W.f32_to_bf16_bits(kc)
+    ora, _, _ = oracle.select(Fb, kcb, 100, 1, 2, NB * 64 - 1)
+    got = gpu_select(Fb, kcb, 100, 1, 2, NB * 64 - 1, NB * 64)
+    assert np.array_equal(got, ora)
+
+
+@pytest.mark.parametrize("k,n_init,n_local", [(0, 1, 2), (61, 1, 2), (70, 1, 2), (5, 0, 0),
+                                              (5, 3, 7), (1, 0, 1)])
+def test_select_degenerate_budgets(k, n_init, n_local):
+    rng = W.rng_for(11, k * 100 + n_init * 10 + n_local)
+    NB, B, G = 64, 2, 2
+    kc = W.normal_bf16(rng, (B, G, NB, 128))
+    F = W.normal_bf16(rng, (B, 1, G, 1, 128))
+    _select_case(F, kc, k, n_init, n_local, NB * 64 - 1, NB * 64, "budget")
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130, 4096 + 17])
+def test_select_short_and_ragged_sequences(T):
+    rng = W.rng_for(12, T)
+    NB = (T + 63) // 64
+    kc = W.normal_bf16(rng, (1, 2, NB, 128))
+    F = W.normal_bf16(rng, (1, 1, 2, 1, 128))
+    _select_case(F, kc, 4, 1, 2, T - 1, T, "T=%d" % T)
+
+
+def test_select_prefill_chunk():
+    rng = W.rng_for(13)
+    B, G, T, nq = 2, 4, 8192, 96
+    NB = T // 64
+    kc = W.normal_bf16(rng, (B, G, NB, 128))
+    F = W.normal_bf16(rng, (B, nq, G, 1, 128))
+    _select_case(F, kc, 16, 1, 2, T - nq, T, "prefill")
+    # a chunk that starts inside the first blocks (short candidate lists)
+    _select_case(F, kc, 16, 1, 2, 0, T, "prefill from 0")
+
+
+# --------------------------------------------------------------------------
+# decode attention
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["decode_b1_t4k", "decode_b4_t32k_planted"])
+def test_decode_attention_configs(name):
+    w = W.WORKLOADS[name]
+    x = W.decode_inputs(w)
+    _, kcb = oracle.compress_keys(x["K"])
+    idx, _, _ = oracle.select(x["F"].reshape(w.B, 1, w.G, 1, w.d), kcb, w.k, w.n_init, w.n_local, w.T - 1)
+    Q = x["Q"]
+    ora = oracle.sparse_attention(Q.reshape(w.B, 1, w.Hq, w.d), x["K"], x["V"], idx, w.T - 1, w.T)
+    got = gpu_decode(Q, x["K"], x["V"], idx[:, 0], w.T, w.k, w.n_init, w.n_local)
+    check_attention(got, ora[:, 0], name)
+
+
+def test_decode_every_block_is_dense_causal():
+    w = W.WORKLOADS["decode_b1_t4k"]
+    x = W.decode_inputs(w)
+    NB = w.NB
+    idx = np.broadcast_to(np.arange(NB, dtype=np.int32), (w.B, w.G, NB)).copy()
+    got = gpu_decode(x["Q"], x["K"], x["V"], idx, w.T, NB - 3)
+    dense = oracle.dense_causal_attention(x["Q"].reshape(w.B, 1, w.Hq, w.d), x["K"], x["V"], w.T - 1)
+    check_attention(got, dense[:, 0], "dense")
+
+
+@pytest.mark.parametrize("R,G", [(1, 4), (2, 4), (4, 2), (8, 2), (16, 1)])
+@pytest.mark.parametrize("T", [2048, 2048 + 17])
+def test_decode_group_ratios_and_ragged_tail(R, G, T):
+    rng = W.rng_for(20, R * 1000 + T)
+    B, d, k = 3, 128, 12
+    Hq = R * G
+    Q = W.normal_bf16(rng, (B, Hq, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, 1, 2, T - 1)
+    ora = oracle.sparse_attention(Q.reshape(B, 1, Hq, d), K, V, idx, T - 1, T)
+    got = gpu_decode(Q, K, V, idx[:, 0], T, k)
+    check_attention(got, ora[:, 0], "R=%d T=%d" % (R, T))
+
+
+def test_decode_padding_entries_are_skipped():
+    rng = W.rng_for(21)
+    B, G, R, T, d = 2, 2, 4, 640, 128                     # 10 blocks, 7 candidates < k
+    k = 12
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, 1, 2, T - 1)
+    assert (idx == -1).any()
+    ora = oracle.sparse_attention(Q.reshape(B, 1, G * R, d), K, V, idx, T - 1, T)
+    got = gpu_decode(Q, K, V, idx[:, 0], T, k)
+    check_attention(got, ora[:, 0], "padding")
+
+
+def test_decode_slot_mode_on_interleaved_slots():
+    rng = W.rng_for(22)
+    B, G, R, NB, d, k = 2, 4, 4, 40, 128, 8
+    T = NB * 64
+    S = k + 3
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    KV = W.normal_bf16(rng, (B, G, NB, 2, 64, d))         # host layout
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    K = np.ascontiguousarray(KV[:, :, :, 0].reshape(B, G, T, d))
+    V = np.ascontiguousarray(KV[:, :, :, 1].reshape(B, G, T, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, 1, 2, T - 1)
+    ora = oracle.sparse_attention(Q.reshape(B, 1, G * R, d), K, V, idx, T - 1, T)
+    slots = np.ascontiguousarray(KV[np.arange(B)[:, None, None], np.arange(G)[None, :, None], idx[:, 0]])
+    got = gpu_decode(Q, slots, None, idx[:, 0], T, k, addr_mode=abi.SPARDA_ADDR_SLOT,
+                     bg_stride=S * 2 * 64 * d, blk_stride=2 * 64 * d)
+    check_attention(got, ora[:, 0], "slots")
+    # the same blocks addressed by id in the full interleaved host layout
+    got2 = gpu_decode(Q, KV, None, idx[:, 0], T, k, addr_mode=abi.SPARDA_ADDR_LOGICAL,
+                      bg_stride=NB * 2 * 64 * d, blk_stride=2 * 64 * d)
+    check_attention(got2, ora[:, 0], "interleaved")
+
+
+def test_decode_out_of_range_ids_are_flagged_and_skipped():
+    rng = W.rng_for(23)
+    B, G, R, T, d = 1, 2, 4, 1024, 128
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    idx = np.array([[[0, 3, 99, 14, 15], [0, 5, 16, 14, 15]]], np.int32)   # 99 and 16 >= NB
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = gpu_decode(Q, K, V, idx, T, 2, status=status)
+    assert abi.sparda_status_from_device(int(status.item())) == abi.SPARDA_ERANGE
+    clean = np.where(idx >= 16, -1, idx)
+    ora = oracle.sparse_attention(Q.reshape(B, 1, G * R, d), K, V, clean[:, None], T - 1, T)
+    check_attention(got, ora[:, 0], "range")
+
+
+# --------------------------------------------------------------------------
+# prefetch
+# --------------------------------------------------------------------------
+
+def _pinned_bf16(bits: np.ndarray) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.pin_memory()
+
+
+@pytest.mark.parametrize("skip_resident", [False, True])
+def test_prefetch_parity(skip_resident):
+    rng = W.rng_for(30)
+    B, G, NB, d, k = 3, 4, 50, 128, 9
+    T = NB * 64
+    S = k + 3
+    host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    idx, _, _ = oracle.select(F, kc, k, 1, 2, T - 1)
+    idx = idx[:, 0]
+    p = abi.make_params(B, G * 4, G, T, k)
+    hkv = _pinned_bf16(host)
+    slots = torch.zeros(B, G, S, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_prefetch_blocks(p, hkv, torch.from_numpy(idx).cuda(), slots, skip_resident)
+    torch.cuda.synchronize()
+    ora = oracle.gather_blocks(host, idx, T - 1, 1, 2, skip_resident)
+    assert np.array_equal(host_bits(slots), ora)
+
+
+def test_prefetch_flags_out_of_range_and_rejects_pageable_memory():
+    B, G, NB, d = 1, 2, 8, 128
+    host = np.zeros((B, G, NB, 2, 64, d), np.uint16)
+    host[0, 1, 3] = 7
+    p = abi.make_params(B, 8, G, NB * 64, 2)
+    idx = torch.tensor([[[0, 3, 6, 7, 0], [0, 3, 50, 6, 7]]], dtype=torch.int32, device="cuda")[:, :, :5]
+    p = abi.make_params(B, 8, G, NB * 64, 2)
+    slots = torch.zeros(B, G, 5, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_prefetch_blocks(p, _pinned_bf16(host), idx, slots, False, 0, status)
+    torch.cuda.synchronize()
+    assert abi.sparda_status_from_device(int(status.item())) == abi.SPARDA_ERANGE
+    assert np.array_equal(host_bits(slots)[0, 1, 1], host[0, 1, 3])
+    pageable = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16)
+    with pytest.raises(abi.SpardaError) as e:
+        abi.sparda_prefetch_blocks(p, pageable, idx, slots, False)
+    assert e.value.status == abi.SPARDA_EINVAL
+
+
+# --------------------------------------------------------------------------
+# prefill attention
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,nq,R", [(8192, 160, 4), (4096 + 29, 77, 8), (700, 700, 2)])
+def test_prefill_attention_parity(T, nq, R):
+    rng = W.rng_for(40, T + nq)
+    B, G, d, k = 2, 2, 128, 8
+    Hq = G * R
+    q_start = T - nq
+    Q = W.normal_bf16(rng, (B, nq, Hq, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, 1, 2, q_start)
+    ora = oracle.sparse_attention(Q, K, V, idx, q_start, T)
+    p = abi.make_params(B, Hq, G, T, k)
+    O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device="cuda")
+    ws = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
+    abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, q_start, dev_bf16(K), dev_bf16(V), T * d, d,
+                                   torch.from_numpy(idx).cuda(), O, ws)
+    torch.cuda.synchronize()
+    check_attention(host_bits(O), ora, "prefill T=%d nq=%d" % (T, nq))
