@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import shutil
 import statistics
 import subprocess
 import sys
@@ -102,9 +103,11 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(index), "--query-gpu=" + q, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            cmd = ["nvidia-smi", "-i", str(index), "--query-gpu=" + q,
+                   "--format=csv,noheader,nounits", "-lms", "50"]
+            if shutil.which("stdbuf"):
+                cmd = ["stdbuf", "-oL"] + cmd        # line-buffered, so nothing is lost at stop
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -355,8 +358,17 @@ def run_sparda(args):
 
     for _ in range(max(args.warmup, 3)):
         loop.step_resident()
+    # clocks are sampled over a ~1 s busy window that contains the timed steps
+    # (untimed padding before and after keeps the GPU in the same state)
+    est = time_steps(loop.step_resident, 5, world) / 5
+    pad = max(1, int(400.0 / max(est, 1e-3)))
     clocks = ClockSampler(local)
+    for _ in range(pad):
+        loop.step_resident()
     ms = time_steps(loop.step_resident, args.steps, world)
+    for _ in range(pad):
+        loop.step_resident()
+    torch.cuda.synchronize()
     clk = clocks.stop()
     # per-kernel durations inside a second timed pass on the same stream
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]

@@ -53,10 +53,10 @@ cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
 
 // ---- decode attention -----------------------------------------------------
 struct DecodePlan {
-  int S;            // list entries per (b, g)
-  int bps;          // list entries per split
-  int n_split;      // splits per (b, g)
-  size_t ws_bytes;  // partial results
+  int S;            // list entries per (query, group) pair
+  long long n_cta;  // thread blocks (stream-K ranges of the flattened entries)
+  int max_cover;    // most thread blocks any pair's entries can span
+  size_t ws_bytes;  // segment partials + tickets
 };
 DecodePlan plan_decode(const sparda_params &p);
 DecodePlan plan_gather(const sparda_params &p, long long pairs);

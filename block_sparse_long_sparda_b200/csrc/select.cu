@@ -15,13 +15,15 @@
 // once.  Inside a CTA each half-warp scores 8 blocks per step: lane l loads
 // dims [8l, 8l+8) of the 8 rows (8 x 16-byte loads in flight), multiplies by
 // the Forecast slice, and a butterfly transpose-reduce (8 shuffles for 8
-// rows) leaves the full score of each row in a pair of lanes.  Scores become orderable
-// uint32 keys; a 4-pass 8-bit radix select finds the k-th key, and a block
-// scan in block order keeps everything above it plus the lowest-index ties,
-// so results come out already sorted by block id and ties go to the lower
-// id.  The chunks of a problem meet through an atomic ticket: the last CTA to
-// finish (no waiting) merges the chunks' survivors with the same select and
-// writes init U top-k U local.  No CTA ever waits for another.
+// rows) leaves the full score of each row in a pair of lanes.  Scores become
+// orderable uint32 keys.  A chunk CTA only streams and scores, writing its
+// keys to the workspace, so CTAs are short and many are in flight.  The
+// chunks of a problem meet through an atomic ticket: the last CTA to finish
+// (no waiting) loads every key of the problem from L2, a 4-pass 8-bit radix
+// select finds the k-th key, and a block scan in block order keeps
+// everything above it plus the lowest-index ties -- results come out sorted
+// by block id and ties go to the lower id -- and writes init U top-k U local.
+// No CTA ever waits for another.
 #include <algorithm>
 #include <cstdlib>
 
@@ -33,19 +35,17 @@ namespace sparda {
 namespace {
 
 constexpr int kSelThreads = 256;
-constexpr int kMergeCap = 8192;   // survivors one merge can hold
+constexpr int kMaxCand = 32768;   // candidates one problem may have (keys fit in shared memory)
 constexpr int kMaxNf = 16;
 
 struct SelArgs {
   const uint16_t *F;
   const uint16_t *kc;
   int32_t *idx;
-  uint32_t *counters;
-  uint32_t *cand_key;
-  int32_t *cand_idx;
-  int32_t *cand_cnt;
+  uint32_t *counters;   // one ticket per problem (multi-chunk only)
+  uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
   int nq, G, nf, NB, k, n_init, n_local, q_start, S;
-  int CH, n_chunks, kc_keep, cap;
+  int CH, n_chunks, cap;
 };
 
 // ---------------------------------------------------------------------------
@@ -260,8 +260,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __shared__ uint32_t scan_tmp[33];
   __shared__ int s_last;
 
-  const long long prob = blockIdx.x;
-  const int chunk = blockIdx.y;
+  // problems are laid out chunk-fastest so a problem's chunks run together
+  // and its merge overlaps the streaming of later problems
+  const long long prob = blockIdx.x / a.n_chunks;
+  const int chunk = (int)(blockIdx.x - prob * a.n_chunks);
   const int g = (int)(prob % a.G);
   const long long bi = prob / a.G;
   const int i = (int)(bi % a.nq);
@@ -270,8 +272,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   const int ncand = bp.cand_hi - bp.cand_lo;
   int32_t *out = a.idx + prob * a.S;
 
-  if (ncand <= a.k) {  // every candidate is kept: nothing to score
-    if (chunk == 0) write_set(out, bp, ncand, a.S, true);
+  if (ncand <= a.k || a.k == 0) {  // nothing to rank: every candidate, or none, is kept
+    if (chunk == 0) write_set(out, bp, min(ncand, a.k), a.S, true);
     return;
   }
 
@@ -288,32 +290,22 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   score_rows(kc_bg, fs, a.nf, lo, n, keys);
   __syncthreads();
 
-  const int E = a.CH / kSelThreads;
   uint32_t tau = 0;
   int need = 0;
+  int32_t *top = out + bp.init_hi;
 
-  if (a.n_chunks == 1) {  // n == ncand > k
+  if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
     radix_threshold(keys, n, a.k, hist, bc, tau, need);
-    int32_t *top = out + bp.init_hi;
     const int ntop = compact_kept(
-        keys, n, E, tau, need, scan_tmp, [&](int e) { return lo + e; },
+        keys, n, a.CH / kSelThreads, tau, need, scan_tmp, [&](int e) { return bp.cand_lo + e; },
         [&](int pos, uint32_t, int id) { top[pos] = id; });
     write_set(out, bp, ntop, a.S, false);
     return;
   }
 
-  // ---- chunk survivors -> workspace ----
-  const long long slot = prob * a.n_chunks + chunk;
-  uint32_t *ck = a.cand_key + slot * a.kc_keep;
-  int32_t *ci = a.cand_idx + slot * a.kc_keep;
-  if (n > a.k) radix_threshold(keys, n, a.k, hist, bc, tau, need);
-  const int cnt = compact_kept(
-      keys, n, E, tau, need, scan_tmp, [&](int e) { return lo + e; },
-      [&](int pos, uint32_t key, int id) {
-        ck[pos] = key;
-        ci[pos] = id;
-      });
-  if (threadIdx.x == 0) a.cand_cnt[slot] = cnt;
+  // ---- chunk scores -> workspace; the last chunk to finish ranks them all ----
+  uint32_t *pkeys = a.cand_key + prob * (long long)a.cap;
+  for (int e = threadIdx.x; e < n; e += kSelThreads) pkeys[chunk * a.CH + e] = keys[e];
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -323,28 +315,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-
-  // ---- last CTA of the problem: merge the chunks in block order ----
-  uint32_t *mkeys = dyn;
-  int32_t *mids = reinterpret_cast<int32_t *>(dyn + a.cap);
-  int M = 0;
-  for (int c = 0; c < a.n_chunks; ++c) {
-    const long long sl = prob * a.n_chunks + c;
-    const int cc = __ldcg(a.cand_cnt + sl);
-    for (int t = threadIdx.x; t < cc; t += kSelThreads) {
-      mkeys[M + t] = __ldcg(a.cand_key + sl * a.kc_keep + t);
-      mids[M + t] = __ldcg(a.cand_idx + sl * a.kc_keep + t);
-    }
-    M += cc;
-  }
+  for (int e = threadIdx.x; e < ncand; e += kSelThreads) keys[e] = __ldcg(pkeys + e);
   __syncthreads();
-  tau = 0;
-  need = 0;
-  if (M > a.k) radix_threshold(mkeys, M, a.k, hist, bc, tau, need);
-  int32_t *top = out + bp.init_hi;
-  const int EM = (a.cap + kSelThreads - 1) / kSelThreads;
+  radix_threshold(keys, ncand, a.k, hist, bc, tau, need);
+  const int E = (ncand + kSelThreads - 1) / kSelThreads;
   const int ntop = compact_kept(
-      mkeys, M, EM, tau, need, scan_tmp, [&](int e) { return mids[e]; },
+      keys, ncand, E, tau, need, scan_tmp, [&](int e) { return bp.cand_lo + e; },
       [&](int pos, uint32_t, int id) { top[pos] = id; });
   write_set(out, bp, ntop, a.S, false);
   if (threadIdx.x == 0) a.counters[prob] = 0u;
@@ -370,43 +346,33 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
   pl.n_chunks = 1;
   pl.kc = 0;
   pl.ws_bytes = 0;
-  if (pl.ncand_max <= p.k || pl.n_problems == 0) return pl;
+  if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
 
   const int forced = env_int("SPARDA_SELECT_CHUNK");
   int CH;
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
   } else {
-    // as large as possible while keeping >= 4 CTAs per SM in flight
-    CH = kSelThreads;
-    while (CH < 8192) {
-      const long long ctas = pl.n_problems * ceil_div_ll(pl.ncand_max, 2LL * CH);
-      if (ctas < 4LL * 148) break;
-      CH *= 2;
-    }
+    // short-lived streaming CTAs: about 512 blocks (128 KB of Kc) each, but
+    // one chunk per problem once there are plenty of problems (prefill)
+    CH = 512;
+    if (pl.n_problems >= 8LL * 148) CH = kMaxCand;
   }
-  // the merge must hold every chunk's survivors
-  while (CH < 8192 &&
-         ceil_div_ll(pl.ncand_max, CH) * (long long)std::min(p.k, CH) > kMergeCap)
-    CH *= 2;
+  if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
   pl.CH = CH;
   pl.n_chunks = (int)ceil_div_ll(pl.ncand_max, CH);
   if (pl.n_chunks > 1) {
-    pl.kc = std::min(p.k, CH);
-    const size_t slots = (size_t)pl.n_problems * pl.n_chunks;
+    pl.kc = pl.ncand_max;  // every candidate's key is kept for the final rank
     size_t off = ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;      // counters
-    off += ((slots * pl.kc * 4) + 255) & ~(size_t)255;                  // keys
-    off += ((slots * pl.kc * 4) + 255) & ~(size_t)255;                  // ids
-    off += ((slots * 4) + 255) & ~(size_t)255;                          // counts
+    off += (((size_t)pl.n_problems * pl.n_chunks * CH * 4) + 255) & ~(size_t)255;  // keys
     pl.ws_bytes = off;
   }
   return pl;
 }
 
 int select_supported(const SelectPlan &pl) {
-  if (pl.CH > 8192) return 0;
-  if (pl.n_chunks > 1 && (long long)pl.n_chunks * pl.kc > kMergeCap) return 0;
-  if (pl.n_chunks > 65535) return 0;
+  if (pl.CH > kMaxCand) return 0;
+  if (pl.ncand_max > kMaxCand) return 0;
   return 1;
 }
 
@@ -429,32 +395,24 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.S = p.k + p.n_init + p.n_local;
   a.CH = pl.CH;
   a.n_chunks = pl.n_chunks;
-  a.kc_keep = pl.kc;
-  a.cap = std::max(pl.CH, pl.n_chunks * pl.kc);
+  a.cap = pl.n_chunks * pl.CH;  // key slots per problem in the workspace
   a.counters = nullptr;
   a.cand_key = nullptr;
-  a.cand_idx = nullptr;
-  a.cand_cnt = nullptr;
   size_t smem = (size_t)pl.CH * 4;
   if (pl.n_chunks > 1) {
     char *w = static_cast<char *>(ws);
-    const size_t slots = (size_t)pl.n_problems * pl.n_chunks;
     a.counters = reinterpret_cast<uint32_t *>(w);
     w += ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
     a.cand_key = reinterpret_cast<uint32_t *>(w);
-    w += ((slots * pl.kc * 4) + 255) & ~(size_t)255;
-    a.cand_idx = reinterpret_cast<int32_t *>(w);
-    w += ((slots * pl.kc * 4) + 255) & ~(size_t)255;
-    a.cand_cnt = reinterpret_cast<int32_t *>(w);
-    smem = (size_t)a.cap * 8;
+    smem = (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid((unsigned)pl.n_problems, (unsigned)pl.n_chunks);
-  select_kernel<<<grid, kSelThreads, smem, stream>>>(a);
+  const long long grid = pl.n_problems * pl.n_chunks;
+  select_kernel<<<(unsigned)grid, kSelThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -177,6 +177,8 @@ int sparda_prefetch_blocks(const sparda_params *p, const void *host_kv, const in
  *       A list must not repeat a block.
  * O     bf16 [B][Hq][d]
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_DECODE, ...)
+ *       bytes, zero-filled before its first use (each call leaves its ticket
+ *       words zero again); calls sharing one workspace must not overlap.
  */
 int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void *K,
                               const void *V, long long bg_stride, long long blk_stride,
@@ -194,6 +196,8 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
  * idx   int32 [B][nq][G][S] (as produced by sparda_forecast_select)
  * O     bf16 [B][nq][Hq][d]
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_PREFILL, p, nq, 0)
+ *       bytes, zero-filled before its first use; calls sharing one workspace
+ *       must not overlap.
  */
 int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, int q_start,
                                const void *K, const void *V, long long bg_stride,
