@@ -3,76 +3,50 @@
 //
 // [p4 "The fourth projection", Eq. 5 / Algorithm 2]: O_l = attention(Q_l,
 // K_l[B_l], V_l[B_l]): each query head attends over the keys of its GQA
-// group's selected blocks only; fp32 softmax and accumulation.
+// group's selected blocks only; fp32 softmax, fp32 accumulation.
 //
-// Design (B200).  Decode attention reads 32 KB of K+V per selected block and
-// does 2*R*128 fp32 FMA per key (the R query heads of a group share every
-// key): about 4 FLOP/byte for R = 4, firmly HBM bound.  CUDA cores do the
-// math; the work is organised to keep HBM busy from the first to the last
-// microsecond:
+// Design (B200).  A selected block is 32 KB of K+V; the R query heads of a
+// group share it, so each block is a pair of tiny dense contractions:
+// S^T[64 keys x R] = K[64x128] Q^T and O^T[128 dims x R] += V^T P^T.  They run
+// on the 5th-generation tensor cores (tcgen05, bf16 operands in shared
+// memory, fp32 accumulators in TMEM), which leaves the CUDA cores only the
+// softmax -- a few dozen instructions per thread per block -- so the kernel
+// streams K/V at HBM speed instead of being bound by instruction issue:
 //  - stream-K: the (query, group) "pairs" and their list entries are
 //    flattened and cut into equal contiguous ranges, one per CTA, with a grid
-//    of exactly two resident CTAs per SM -- one wave, no tail.  A range may
-//    start or end inside a pair; each piece of a pair is a "segment";
-//  - the entry list of the range is read by all threads at once and compacted
+//    of two resident CTAs per SM -- one wave, no tail.  A range may start or
+//    end inside a pair; each piece of a pair is a "segment";
+//  - the entry list of a range is read by all threads at once and compacted
 //    with a block scan (one global-load latency per CTA);
-//  - every selected block (its K and V halves, plus the pair's query at the
-//    first block of a segment) is staged by the bulk-copy engine
-//    (cp.async.bulk, completion on an mbarrier) into an NSTAGE-deep ring that
-//    runs across segment boundaries;
-//  - the 64 keys of a staged block are split over the warps; within a warp,
-//    QK^T keeps each lane's slice of the R query vectors in registers, every
-//    lane converts only its own K elements, and a butterfly transpose-reduce
-//    turns per-lane partials into whole dot products with one shuffle per
-//    (key, head) pair; online softmax in the exp2 domain; P goes through a
-//    small shared tile; PV with each lane owning 4 output dims of all R heads;
-//  - at the end of a segment the warps merge in shared memory; a pair that a
-//    single CTA covers is normalised and written at once, otherwise the
-//    segment's (max, sum, unnormalised output) goes to the workspace and the
-//    last CTA to finish the pair (atomic ticket, no waiting) combines them.
-// Waits on the mbarriers are bounded: a timeout sets SPARDA_DEV_TIMEOUT, the
-// CTA drains its copies (bounded) and leaves.
+//  - TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) stages each
+//    block as [K lo-dims | V lo-dims | K hi-dims | V hi-dims] (8 KB each) in
+//    an NSTAGE ring, with the pair's query rows at the first block of a
+//    segment.  The M = 128 MMA for S^T reads rows 0-63 = the block's keys;
+//    its rows 64-127 alias the finite V tiles and are masked;
+//  - one thread issues the MMAs (N = 16: the group's heads, zero padded);
+//    softmax per head in the exp2 domain over the thread-per-key rows of
+//    S^T; P^T goes to shared memory as a bf16 K-major operand (the sum of
+//    probabilities uses the same rounded values); O^T is read back with one
+//    thread per output dim and rescaled in registers;
+//  - at the end of a segment a pair that a single CTA covers is normalised
+//    and written at once, otherwise the segment's (max, sum, unnormalised
+//    output) goes to the workspace and the last CTA to finish the pair
+//    (atomic ticket, no waiting) combines them.
+// Every wait (TMA, MMA completion) is bounded: a timeout sets
+// SPARDA_DEV_TIMEOUT, the CTA drains what it issued (bounded), frees its
+// TMEM and leaves.
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace sparda {
 
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kStageBytes = 2 * kBlk * kD * 2;  // K + V of one block = 32 KB
-constexpr int kGridTarget = 2 * 148;            // two resident CTAs per B200 SM
-
-struct DecArgs {
-  const uint16_t *Q, *K, *V;
-  long long bg_stride, blk_stride;
-  const int32_t *idx;
-  uint16_t *O;
-  float *ws_o;          // [pairs][max_cover][R][128] unnormalised segment outputs
-  float2 *ws_ml;        // [pairs][max_cover][R] (max, sum) in the exp2 domain
-  uint32_t *counters;   // [pairs] tickets, zero between calls
-  int32_t *status;
-  long long n_entries;  // pairs * S
-  int G, S, NB, addr_mode, nq, q_start, max_cover;
-  float scale_log2;
-};
-
-template <int N>
-__device__ __forceinline__ float transpose_reduce(float (&v)[N], int li) {
-#pragma unroll
-  for (int half = N / 2; half >= 1; half >>= 1) {
-    const bool up = (li & half) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = up ? v[i] : v[i + half];
-      const float keep = up ? v[i + half] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-    }
-  }
-  return v[0];
-}
+constexpr int kGridMax = 3 * 148;               // most CTAs a B200 keeps resident
 
 // the CTA whose range holds entry e (ranges: [c*E/C, (c+1)*E/C))
 __device__ __forceinline__ long long cta_of(long long e, long long E, long long C) {
@@ -108,48 +82,117 @@ __device__ int block_excl_scan(int v, int *tmp, int &total) {
   return r;
 }
 
-template <int R, int NWARP>
-struct Cfg {
-  static constexpr int NT = NWARP * 32;
-  static constexpr int DS = 64 / R;          // q dims per lane in QK
-  static constexpr int LPK = 2 * R;          // lanes per key in QK
-  static constexpr int KG = 32 / LPK;        // key groups per warp
-  static constexpr int KW = kBlk / NWARP;    // keys per warp per block
-  static constexpr int KPR = 2 * KG;         // keys per warp per QK round
-  static constexpr int ROUNDS = KW / KPR;
-  static constexpr int QBYTES = R * kD * 2;
-  static constexpr int STAGE = kStageBytes + ((QBYTES + 127) / 128) * 128;
-  static constexpr int MAX_ENT = 2 * NT;     // list entries one CTA may own
-  // per-warp P tiles, rounded to 128 B so the warp-merge area after them
-  // keeps the 16-byte alignment its vector stores need
-  static constexpr int PBUF = (NWARP * (KW * R + R) + 31) / 32 * 32;
-  static_assert(PBUF % 4 == 0, "merge area must stay 16-byte aligned");
+
+constexpr int kNQ = 16;                 // MMA N: the heads of a group, zero padded
+constexpr int kTile = 8192;             // 64 rows x 64 bf16, one swizzled tile
+constexpr int kUnitBytes = 4 * kTile;   // K lo | V lo | K hi | V hi
+constexpr int kMaxEnt = 128;            // list entries one CTA may own (one per thread)
+constexpr int kThreads = 128;
+
+struct TcArgs {
+  const uint16_t *Q;
+  uint16_t *O;
+  const int32_t *idx;
+  float *ws_o;          // [pairs][max_cover][R][128] unnormalised segment outputs
+  float2 *ws_ml;        // [pairs][max_cover][R] (max, sum) in the exp2 domain
+  uint32_t *counters;   // [pairs] tickets, zero between calls
+  int32_t *status;
+  long long n_entries;  // pairs * S
+  long long bg_rows, blk_rows;  // strides in 128-element rows
+  int G, S, NB, addr_mode, nq, q_start, max_cover;
+  float scale_log2;
+};
+
+template <int R>
+struct TcCfg {
+  static constexpr int QB = R * kD * 2;  // raw query rows of one pair
+  static constexpr int QB_AL = (QB + 127) / 128 * 128;
+  // stages (1024-aligned) | raw query ring | Q^T operand | P^T operand | slack
   static size_t smem(int nstage) {
-    return (size_t)nstage * STAGE + (size_t)PBUF * 4 + (size_t)NWARP * R * kD * 4 +
-           (size_t)2 * NWARP * R * 4;
+    return (size_t)nstage * kUnitBytes + (size_t)nstage * QB_AL + 4096 + 2048 + 1024;
   }
 };
 
-template <int R, int NWARP, int NSTAGE>
-__global__ void __launch_bounds__(NWARP * 32) attn_streamk_kernel(DecArgs a) {
-  using C = Cfg<R, NWARP>;
-  constexpr int NT = C::NT, DS = C::DS, LPK = C::LPK, KG = C::KG, KW = C::KW, KPR = C::KPR;
-  constexpr int ROUNDS = C::ROUNDS;
-  static_assert(ROUNDS >= 1 && KW % KPR == 0, "bad warp split");
-  static_assert(DS >= 4, "R too large");
+// End of a segment: normalise and write the pair's output if this CTA covers
+// the whole pair, else store the segment's (max, sum, unnormalised output) and
+// let the last CTA to finish the pair combine all of them.  Block-wide.
+template <int R>
+__device__ __forceinline__ void segment_flush(const TcArgs &a, long long pair, bool live,
+                                              long long E, long long NC, const float (&acc)[R],
+                                              const float (&m_run)[R], const float (&l_w)[R],
+                                              float (*red)[kNQ], int *s_last) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (lane == 0)
+#pragma unroll
+    for (int h = 0; h < R; ++h) red[warp][h] = live ? l_w[h] : 0.f;
+  __syncthreads();
+  const long long c_first = cta_of(pair * a.S, E, NC);
+  const long long c_last = cta_of(pair * a.S + a.S - 1, E, NC);
+  const int n_cover = (int)(c_last - c_first + 1);
+  const long long slot = pair * a.max_cover + (blockIdx.x - c_first);
+  const int dim = tid;
+#pragma unroll
+  for (int h = 0; h < R; ++h) {
+    const float L = red[0][h] + red[1][h] + red[2][h] + red[3][h];
+    const float o = live ? acc[h] : 0.f;
+    const float M = live ? m_run[h] : -INFINITY;
+    if (n_cover == 1) {
+      const float r = L > 0.f ? o / L : 0.f;
+      a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+    } else {
+      a.ws_o[(slot * R + h) * kD + dim] = o;
+      if (dim == 0) a.ws_ml[slot * R + h] = make_float2(M, L);
+    }
+  }
+  if (n_cover > 1) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) *s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
+    __syncthreads();
+    if (*s_last) {
+      __threadfence();
+      const long long base = pair * a.max_cover;
+#pragma unroll 1
+      for (int h = 0; h < R; ++h) {
+        float M = -INFINITY;
+        for (int c = 0; c < n_cover; ++c) M = fmaxf(M, __ldcg(&a.ws_ml[(base + c) * R + h].x));
+        float L = 0.f, o = 0.f;
+        for (int c = 0; c < n_cover; ++c) {
+          const float2 ml = __ldcg(&a.ws_ml[(base + c) * R + h]);
+          const float fw = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+          L += fw * ml.y;
+          o += fw * __ldcg(&a.ws_o[((base + c) * R + h) * kD + dim]);
+        }
+        const float r = L > 0.f ? o / L : 0.f;
+        a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+      }
+      if (tid == 0) a.counters[pair] = 0u;
+    }
+  }
+  __syncthreads();
+}
 
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t *stages = smem;
-  float *pbuf = reinterpret_cast<float *>(smem + NSTAGE * C::STAGE);
-  float *red_o = pbuf + C::PBUF;                 // [NWARP][R][128]
-  float *red_m = red_o + NWARP * R * kD;         // [NWARP][R]
-  float *red_l = red_m + NWARP * R;              // [NWARP][R]
+template <int R, int NSTAGE>
+__global__ void __launch_bounds__(kThreads) attn_tc_kernel(const __grid_constant__ CUtensorMap mapK,
+                                                           const __grid_constant__ CUtensorMap mapV,
+                                                           TcArgs a) {
+  using C = TcCfg<R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint8_t *stages = sm;                              // NSTAGE x 32 KB
+  uint8_t *qop = sm + NSTAGE * kUnitBytes;           // Q^T operand: 16 rows x 128 dims
+  uint8_t *pop = qop + 4096;                         // P^T operand: 16 rows x 64 keys
+  uint8_t *qraw = pop + 2048;                        // NSTAGE raw query slots
   __shared__ __align__(8) uint64_t full_bar[NSTAGE];
-  __shared__ int s_m[C::MAX_ENT];
-  __shared__ int s_rows[C::MAX_ENT];
-  __shared__ int s_seg[C::MAX_ENT];
+  __shared__ __align__(8) uint64_t mma1_bar, mma2_bar;
+  __shared__ uint32_t tmem_base;
+  __shared__ int s_row[kMaxEnt];   // TMA row coordinate of the block
+  __shared__ int s_rows[kMaxEnt];  // keys of the block at or before the query
+  __shared__ int s_seg[kMaxEnt];   // segment (pair - pair0)
   __shared__ int s_tmp[33];
   __shared__ int s_last;
+  __shared__ float red[4][kNQ];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long E = a.n_entries, NC = gridDim.x;
@@ -159,289 +202,267 @@ __global__ void __launch_bounds__(NWARP * 32) attn_streamk_kernel(DecArgs a) {
   const long long pair0 = e0 / a.S;
   const int n_seg = (int)((e1 - 1) / a.S - pair0 + 1);
 
-  // ---- the range's valid entries, in order ----
-  int m_[2], rows_[2], seg_[2], cnt = 0;
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const long long e = e0 + 2 * tid + u;
-    if (e >= e1) continue;
-    const long long pair = e / a.S;
-    const int s = (int)(e - pair * a.S);
-    const int j = a.idx[e];
-    if (j < 0) continue;
-    const int pos = a.q_start + (int)((pair / a.G) % a.nq);
-    if (j >= a.NB || j > pos / kBlk) {
-      flag_status(a.status, SPARDA_DEV_RANGE);
-      continue;
+  // ---- the range's valid entries, in order (at most kMaxEnt) ----
+  int row_ = 0, rows_ = 0, seg_ = 0, cnt = 0;
+  {
+    const long long e = e0 + tid;
+    if (tid < kMaxEnt && e < e1) {
+      const long long pair = e / a.S;
+      const int s = (int)(e - pair * a.S);
+      const int j = a.idx[e];
+      if (j >= 0) {
+        const int pos = a.q_start + (int)((pair / a.G) % a.nq);
+        if (j >= a.NB || j > pos / kBlk) {
+          flag_status(a.status, SPARDA_DEV_RANGE);
+        } else {
+          const long long kvpair = (pair / a.G) / a.nq * a.G + pair % a.G;
+          const int m = a.addr_mode == SPARDA_ADDR_SLOT ? s : j;
+          row_ = (int)(kvpair * a.bg_rows + (long long)m * a.blk_rows);
+          rows_ = min(kBlk, pos + 1 - j * kBlk);
+          seg_ = (int)(pair - pair0);
+          cnt = 1;
+        }
+      }
     }
-    m_[cnt] = a.addr_mode == SPARDA_ADDR_SLOT ? s : j;
-    rows_[cnt] = min(kBlk, pos + 1 - j * kBlk);
-    seg_[cnt] = (int)(pair - pair0);
-    ++cnt;
   }
   int nb;
-  const int off = block_excl_scan<NT>(cnt, s_tmp, nb);
-  for (int u = 0; u < cnt; ++u) {
-    s_m[off + u] = m_[u];
-    s_rows[off + u] = rows_[u];
-    s_seg[off + u] = seg_[u];
+  const int off = block_excl_scan<kThreads>(cnt, s_tmp, nb);
+  if (cnt) {
+    s_row[off] = row_;
+    s_rows[off] = rows_;
+    s_seg[off] = seg_;
   }
   if (tid == 0) {
     for (int st = 0; st < NSTAGE; ++st) mbar_init(&full_bar[st], 1);
+    mbar_init(&mma1_bar, 1);
+    mbar_init(&mma2_bar, 1);
     fence_mbar_init();
+    tc::prefetch_map(&mapK);
+    tc::prefetch_map(&mapV);
   }
+  if (warp == 0) tc::tmem_alloc(&tmem_base, 32);
+  // operand tiles start zeroed: rows >= R of Q^T and P^T stay zero
+  for (int i = tid; i < (4096 + 2048) / 16; i += kThreads)
+    reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  tc::fence_before_sync();
   __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base;
+  const uint32_t tS = tmem, tO = tmem + kNQ;
+  const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
+  constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
+  constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
+  // operand descriptors: fixed bases, advanced in 16-byte units
+  const uint64_t dK = tc::sdesc(stages, 16, 1024);          // S^T A operand (K tiles)
+  const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);  // O^T A operand (V^T)
+  const uint64_t dQ = tc::sdesc(qop, 16, 1024);
+  const uint64_t dP = tc::sdesc(pop, 16, 1024);
 
+  // thread 0 only: TMA for block bi into its stage (+ the pair's query rows
+  // at the first block of a segment)
   auto issue = [&](int bi) {
     const int st = bi % NSTAGE;
     const int seg = s_seg[bi];
-    const long long pair = pair0 + seg;
-    const long long kvpair = (pair / a.G) / a.nq * a.G + pair % a.G;
-    const uint32_t bytes = (uint32_t)s_rows[bi] * kD * 2;
     const bool first = bi == 0 || s_seg[bi - 1] != seg;
-    uint8_t *dst = stages + st * C::STAGE;
-    const long long off_kv = kvpair * a.bg_stride + (long long)s_m[bi] * a.blk_stride;
-    mbar_arrive_expect_tx(&full_bar[st], 2 * bytes + (first ? C::QBYTES : 0));
-    bulk_g2s(dst, a.K + off_kv, bytes, &full_bar[st]);
-    bulk_g2s(dst + kStageBytes / 2, a.V + off_kv, bytes, &full_bar[st]);
-    if (first) bulk_g2s(dst + kStageBytes, a.Q + pair * R * kD, C::QBYTES, &full_bar[st]);
+    uint8_t *dst = stages + st * kUnitBytes;
+    const int row = s_row[bi];
+    mbar_arrive_expect_tx(&full_bar[st], kUnitBytes + (first ? C::QB : 0));
+    tc::tma_load_2d(dst, &mapK, 0, row, &full_bar[st]);
+    tc::tma_load_2d(dst + kTile, &mapV, 0, row, &full_bar[st]);
+    tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
+    tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &full_bar[st]);
+    if (first) bulk_g2s(qraw + st * C::QB_AL, a.Q + (pair0 + seg) * R * kD, C::QB, &full_bar[st]);
+  };
+  // thread 0 only: S^T = K Q^T for block bi (rows 0-63 are its keys)
+  auto mma1 = [&](int bi) {
+    const uint64_t base = dK + (uint64_t)((bi % NSTAGE) * (kUnitBytes >> 4));
+    tc::fence_after_sync();
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      tc::mma_bf16(tS, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
+                   dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
+    tc::mma_commit(&mma1_bar);
   };
   if (tid == 0)
     for (int bi = 0; bi < min(nb, NSTAGE); ++bi) issue(bi);
 
-  const int kg = lane / LPK, li = lane % LPK;
-  const int my_head = li % R, my_kappa = li / R;
-  float qv[R][DS];
-  float m_run = -INFINITY, l_run = 0.f;  // for head my_head
-  float acc[R][4];
+  // per thread: acc = one output dim (tid) of every head; m_run uniform;
+  // l_w = this warp's share of the probability sums
+  float acc[R], m_run[R], l_w[R];
 #pragma unroll
-  for (int h = 0; h < R; ++h)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
-  float *pw = pbuf + warp * (KW * R + R);
-  float *alpha = pw + KW * R;
-
-  // ---- end of a segment: merge the warps, write or hand over ----
-  auto flush = [&](int f, bool live) {
-    const long long pair = pair0 + f;
-#pragma unroll
-    for (int h = 0; h < R; ++h)
-      *reinterpret_cast<float4 *>(red_o + (warp * R + h) * kD + lane * 4) =
-          live ? make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3])
-               : make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane < R) {
-      red_m[warp * R + lane] = live ? m_run : -INFINITY;
-      red_l[warp * R + lane] = live ? l_run : 0.f;
-    }
-    __syncthreads();
-    const long long c_first = cta_of(pair * a.S, E, NC);
-    const long long c_last = cta_of(pair * a.S + a.S - 1, E, NC);
-    const int n_cover = (int)(c_last - c_first + 1);
-    const long long slot = pair * a.max_cover + (blockIdx.x - c_first);
-    for (int t = tid; t < R * kD; t += NT) {
-      const int h = t / kD, dim = t % kD;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NWARP; ++w) M = fmaxf(M, red_m[w * R + h]);
-      float L = 0.f, o = 0.f;
-#pragma unroll
-      for (int w = 0; w < NWARP; ++w) {
-        const float mw = red_m[w * R + h];
-        const float fw = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-        L += fw * red_l[w * R + h];
-        o += fw * red_o[(w * R + h) * kD + dim];
-      }
-      if (n_cover == 1) {
-        const float r = L > 0.f ? o / L : 0.f;
-        a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-      } else {
-        a.ws_o[(slot * R + h) * kD + dim] = o;
-        if (dim == 0) a.ws_ml[slot * R + h] = make_float2(M, L);
-      }
-    }
-    if (n_cover > 1) {
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        const long long base = pair * a.max_cover;
-        for (int t = tid; t < R * kD; t += NT) {
-          const int h = t / kD, dim = t % kD;
-          float M = -INFINITY;
-          for (int c = 0; c < n_cover; ++c) M = fmaxf(M, __ldcg(&a.ws_ml[(base + c) * R + h].x));
-          float L = 0.f, o = 0.f;
-          for (int c = 0; c < n_cover; ++c) {
-            const float2 ml = __ldcg(&a.ws_ml[(base + c) * R + h]);
-            const float fw = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-            L += fw * ml.y;
-            o += fw * __ldcg(&a.ws_o[((base + c) * R + h) * kD + dim]);
-          }
-          const float r = L > 0.f ? o / L : 0.f;
-          a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
-        }
-        if (tid == 0) a.counters[pair] = 0u;
-      }
-    }
-    __syncthreads();
-  };
-
+  for (int h = 0; h < R; ++h) {
+    acc[h] = 0.f;
+    m_run[h] = -INFINITY;
+    l_w[h] = 0.f;
+  }
+  uint32_t ph1 = 0, ph2 = 0;
+  int early = -1;        // thread 0: block whose MMA1 is already in flight
+  bool bad = false;      // this thread saw a wait give up
   int cur = -1, next_flush = 0, abort_at = -1;
+  int issued_to = min(nb, NSTAGE);  // thread 0: blocks [0, issued_to) have TMA issued
+
 #pragma unroll 1
   for (int bi = 0; bi < nb; ++bi) {
     const int st = bi % NSTAGE;
-    const bool ok = mbar_wait_bounded(&full_bar[st], (uint32_t)((bi / NSTAGE) & 1));
-    if (!ok) flag_status(a.status, SPARDA_DEV_TIMEOUT);
-    if (__syncthreads_or(!ok)) {
+    const uint32_t tph = (uint32_t)((bi / NSTAGE) & 1);
+    const int seg = s_seg[bi];
+    if (seg != cur) {  // a new segment: its query arrived with this block
+      for (int f = next_flush; f < seg; ++f)
+        segment_flush<R>(a, pair0 + f, f == cur, E, NC, acc, m_run, l_w, red, &s_last);
+      next_flush = seg;
+      cur = seg;
+#pragma unroll
+      for (int h = 0; h < R; ++h) {
+        acc[h] = 0.f;
+        m_run[h] = -INFINITY;
+        l_w[h] = 0.f;
+      }
+      if (!mbar_wait_bounded(&full_bar[st], tph)) bad = true;
+      if (__syncthreads_or(bad)) {
+        abort_at = bi;
+        break;
+      }
+      const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
+      for (int i = tid; i < R * 16; i += kThreads) {
+        const int h = i >> 4, c8 = i & 15;
+        *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
+    if (tid == 0 && early != bi) {
+      if (mbar_wait_bounded(&full_bar[st], tph)) mma1(bi);
+      else bad = true;
+    }
+    if (!mbar_wait_bounded(&mma1_bar, ph1)) bad = true;
+    ph1 ^= 1;
+    tc::fence_after_sync();
+
+    // ---- softmax over this block's keys (thread = key, in warps 0 and 1) ----
+    const int rows = s_rows[bi];
+    float x[R];
+    if (warp < 2) {
+      float sv[16];
+      tc::tmem_ld16(tS + lane_sel, sv);
+      const bool valid = tid < rows;
+#pragma unroll
+      for (int h = 0; h < R; ++h) x[h] = valid ? sv[h] * a.scale_log2 : -INFINITY;
+#pragma unroll
+      for (int h = 0; h < R; ++h) {
+        const float mx = warp_max_xor(x[h], 1, 32);
+        if (lane == 0) red[warp][h] = mx;
+      }
+    }
+    tc::fence_before_sync();
+    if (__syncthreads_or(bad)) {
       abort_at = bi;
       break;
     }
-    const uint8_t *stage = stages + st * C::STAGE;
-    const int seg = s_seg[bi];
-    if (seg != cur) {
-      for (int f = next_flush; f < seg; ++f) flush(f, f == cur);
-      next_flush = seg;
-      cur = seg;
-      m_run = -INFINITY;
-      l_run = 0.f;
+    float corr[R];
 #pragma unroll
-      for (int h = 0; h < R; ++h)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
-      const uint16_t *qs = reinterpret_cast<const uint16_t *>(stage + kStageBytes);
+    for (int h = 0; h < R; ++h) {
+      const float mn = fmaxf(m_run[h], fmaxf(red[0][h], red[1][h]));
+      corr[h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[h] - mn);
+      m_run[h] = mn;
+      l_w[h] *= corr[h];
+    }
+    float pr[R];
+    if (warp < 2) {
 #pragma unroll
       for (int h = 0; h < R; ++h) {
-        if constexpr (DS >= 8) {
-#pragma unroll
-          for (int q8 = 0; q8 < DS / 8; ++q8) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(qs + h * kD + (q8 * LPK + li) * 8);
-            qv[h][q8 * 8 + 0] = bf16_lo(w.x); qv[h][q8 * 8 + 1] = bf16_hi(w.x);
-            qv[h][q8 * 8 + 2] = bf16_lo(w.y); qv[h][q8 * 8 + 3] = bf16_hi(w.y);
-            qv[h][q8 * 8 + 4] = bf16_lo(w.z); qv[h][q8 * 8 + 5] = bf16_hi(w.z);
-            qv[h][q8 * 8 + 6] = bf16_lo(w.w); qv[h][q8 * 8 + 7] = bf16_hi(w.w);
-          }
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2 *>(qs + h * kD + li * 4);
-          qv[h][0] = bf16_lo(w.x); qv[h][1] = bf16_hi(w.x);
-          qv[h][2] = bf16_lo(w.y); qv[h][3] = bf16_hi(w.y);
-        }
+        const float p = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - m_run[h]);
+        const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+        *reinterpret_cast<__nv_bfloat16 *>(pop + tc::sw128_offset(h, tid)) = pb;
+        pr[h] = __bfloat162float(pb);
       }
     }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
 
-    const uint16_t *Ks = reinterpret_cast<const uint16_t *>(stage);
-    const uint16_t *Vs = Ks + kBlk * kD;
-    const int rows = s_rows[bi];
-    const int kw0 = warp * KW;
-    const int wvalid = min(KW, rows - kw0);
-
-    if (wvalid > 0) {
-      // ---- S = q . k for this warp's keys ----
-      float sv[ROUNDS];
+    // ---- O^T(block) = V^T P^T; the next block's S^T right behind it ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+      const uint64_t base = dV + (uint64_t)(st * (kUnitBytes >> 4));
 #pragma unroll
-      for (int rd = 0; rd < ROUNDS; ++rd) {
-        float part[2 * R];
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint16_t *krow = Ks + (kw0 + rd * KPR + kk * KG + kg) * kD;
-          float kf[DS];
-          if constexpr (DS >= 8) {
-#pragma unroll
-            for (int q8 = 0; q8 < DS / 8; ++q8) {
-              const uint4 w = *reinterpret_cast<const uint4 *>(krow + (q8 * LPK + li) * 8);
-              kf[q8 * 8 + 0] = bf16_lo(w.x); kf[q8 * 8 + 1] = bf16_hi(w.x);
-              kf[q8 * 8 + 2] = bf16_lo(w.y); kf[q8 * 8 + 3] = bf16_hi(w.y);
-              kf[q8 * 8 + 4] = bf16_lo(w.z); kf[q8 * 8 + 5] = bf16_hi(w.z);
-              kf[q8 * 8 + 6] = bf16_lo(w.w); kf[q8 * 8 + 7] = bf16_hi(w.w);
-            }
-          } else {
-            const uint2 w = *reinterpret_cast<const uint2 *>(krow + li * 4);
-            kf[0] = bf16_lo(w.x); kf[1] = bf16_hi(w.x);
-            kf[2] = bf16_lo(w.y); kf[3] = bf16_hi(w.y);
-          }
-#pragma unroll
-          for (int h = 0; h < R; ++h) {
-            float s = 0.f;
-#pragma unroll
-            for (int e = 0; e < DS; ++e) s = fmaf(qv[h][e], kf[e], s);
-            part[kk * R + h] = s;
-          }
-        }
-        const float s = transpose_reduce<2 * R>(part, li);
-        const int key = kw0 + rd * KPR + my_kappa * KG + kg;
-        sv[rd] = key < rows ? s * a.scale_log2 : -INFINITY;
+      for (int k = 0; k < 4; ++k)
+        tc::mma_bf16(tO, base + (uint64_t)(k * 128), dP + (uint64_t)(k * 2), id2, k > 0);
+      tc::mma_commit(&mma2_bar);
+      const int nx = bi + 1;
+      if (nx < nb && s_seg[nx] == seg &&
+          mbar_test_wait(&full_bar[nx % NSTAGE], (uint32_t)((nx / NSTAGE) & 1))) {
+        mma1(nx);
+        early = nx;
       }
-
-      // ---- online softmax for head my_head over this warp's keys ----
-      float mb = sv[0];
-#pragma unroll
-      for (int rd = 1; rd < ROUNDS; ++rd) mb = fmaxf(mb, sv[rd]);
-      mb = warp_max_xor(mb, R, 32);  // lanes sharing a head differ in bits >= log2(R)
-      const float m_new = fmaxf(m_run, mb);
-      const float corr = (m_new == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-      float ps = 0.f;
-#pragma unroll
-      for (int rd = 0; rd < ROUNDS; ++rd) {
-        const float pv = (sv[rd] == -INFINITY) ? 0.f : exp2f(sv[rd] - m_new);
-        ps += pv;
-        pw[(rd * KPR + my_kappa * KG + kg) * R + my_head] = pv;
-      }
-      ps = warp_sum_xor(ps, R, 32);
-      l_run = l_run * corr + ps;
-      m_run = m_new;
-      if (lane < R) alpha[lane] = corr;  // lanes 0..R-1 hold heads 0..R-1
-      __syncwarp();
-
-      // ---- O = corr * O + P V ----
-#pragma unroll
-      for (int h = 0; h < R; ++h) {
-        const float al = alpha[h];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[h][e] *= al;
-      }
-#pragma unroll 4
-      for (int kk = 0; kk < wvalid; ++kk) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(Vs + (kw0 + kk) * kD + lane * 4);
-        const float v0 = bf16_lo(w.x), v1 = bf16_hi(w.x), v2 = bf16_lo(w.y), v3 = bf16_hi(w.y);
-        const float *prow = pw + kk * R;
-#pragma unroll
-        for (int h = 0; h < R; ++h) {
-          const float p = prow[h];
-          acc[h][0] = fmaf(p, v0, acc[h][0]);
-          acc[h][1] = fmaf(p, v1, acc[h][1]);
-          acc[h][2] = fmaf(p, v2, acc[h][2]);
-          acc[h][3] = fmaf(p, v3, acc[h][3]);
-        }
-      }
-      __syncwarp();
     }
-    __syncthreads();  // stage st fully consumed
-    if (tid == 0 && bi + NSTAGE < nb) issue(bi + NSTAGE);
+    if (warp < 2) {  // probability sums, while the tensor core works
+#pragma unroll
+      for (int h = 0; h < R; ++h) l_w[h] += warp_sum_xor(pr[h], 1, 32);
+    }
+    if (!mbar_wait_bounded(&mma2_bar, ph2)) bad = true;
+    ph2 ^= 1;
+    tc::fence_after_sync();
+    // both MMAs of block bi are done: its stage can be refilled
+    if (tid == 0 && bi + NSTAGE < nb && !bad) {
+      issue(bi + NSTAGE);
+      issued_to = bi + NSTAGE + 1;
+    }
+    {
+      float ov[16];
+      tc::tmem_ld16(tO + lane_sel, ov);
+#pragma unroll
+      for (int h = 0; h < R; ++h) acc[h] = acc[h] * corr[h] + ov[h];
+    }
+    tc::fence_before_sync();
   }
+  if (abort_at < 0 && __syncthreads_or(bad)) abort_at = nb;
 
   if (abort_at >= 0) {
-    // a copy never completed: give the ones still in flight a bounded chance
-    // to land before the CTA's shared memory is released, then leave
-    if (tid == 0)
-      for (int bj = abort_at; bj < min(nb, abort_at + NSTAGE); ++bj)
+    // something never completed: let what was issued land (bounded), then
+    // free TMEM and leave; the status word says why
+    flag_status(a.status, SPARDA_DEV_TIMEOUT);
+    if (tid == 0) {
+      for (int bj = max(0, abort_at); bj < issued_to; ++bj)
         (void)mbar_wait_bounded(&full_bar[bj % NSTAGE], (uint32_t)((bj / NSTAGE) & 1));
+      (void)mbar_wait_bounded(&mma1_bar, ph1);
+      (void)mbar_wait_bounded(&mma2_bar, ph2);
+    }
+    tc::fence_before_sync();
     __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 32);
     return;
   }
-  for (int f = next_flush; f < n_seg; ++f) flush(f, f == cur);
+  for (int f = next_flush; f < n_seg; ++f)
+    segment_flush<R>(a, pair0 + f, f == cur, E, NC, acc, m_run, l_w, red, &s_last);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 32);
 }
 
-template <int R, int NWARP, int NSTAGE>
-cudaError_t launch_r(const DecArgs &a, long long grid, cudaStream_t stream) {
-  const size_t smem = Cfg<R, NWARP>::smem(NSTAGE);
-  auto kern = attn_streamk_kernel<R, NWARP, NSTAGE>;
+template <int R, int NSTAGE>
+cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs &a,
+                      long long grid_max, long long grid_min, cudaStream_t stream) {
+  const size_t smem = TcCfg<R>::smem(NSTAGE);
+  auto kern = attn_tc_kernel<R, NSTAGE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)grid, NWARP * 32, smem, stream>>>(a);
+  // one wave: as many CTAs as the device keeps resident (never more than
+  // the plan sized the workspace for, never fewer than the lists need)
+  int dev = 0, n_sm = 148, occ = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem) != cudaSuccess || occ < 1)
+    occ = 1;
+  (void)cudaGetLastError();
+  long long grid = (long long)occ * n_sm;
+  const int forced = env_int("SPARDA_DECODE_CTAS");
+  if (forced > 0) grid = forced;
+  grid = std::max(grid, grid_min);
+  grid = std::min(grid, grid_max);
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(mk, mv, a);
   return cudaGetLastError();
 }
-
-int max_entries_per_cta(int R) { return R == 1 ? 2 * 64 : 2 * 128; }
 
 }  // namespace
 
@@ -450,13 +471,14 @@ DecodePlan plan_gather(const sparda_params &p, long long pairs) {
   pl.S = p.k + p.n_init + p.n_local;
   const int R = p.G > 0 ? p.Hq / p.G : 1;
   const long long E = pairs * pl.S;
-  long long C = kGridTarget;
+  // the workspace is sized for the largest grid a launch may use
+  long long C = std::max<long long>(kGridMax, ceil_div_ll(E, kMaxEnt));
   const int forced = env_int("SPARDA_DECODE_CTAS");
-  if (forced > 0) C = forced;
-  C = std::max<long long>(C, ceil_div_ll(E, max_entries_per_cta(R)));
+  if (forced > 0) C = std::max<long long>(C, forced);
   if (C > E) C = E;
   if (C < 1) C = 1;
   pl.n_cta = C;
+  pl.n_cta_min = std::min<long long>(C, ceil_div_ll(E, kMaxEnt));
   const long long w_min = std::max<long long>(E / C, 1);
   pl.max_cover = (int)(ceil_div_ll(pl.S, w_min) + 1);
   const size_t parts = (size_t)pairs * pl.max_cover * R;
@@ -477,19 +499,30 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   const long long pairs = (long long)p.B * nq * p.G;
   if (pairs == 0) return cudaSuccess;
   const int R = p.Hq / p.G;
-  DecArgs a;
+  const long long kv_pairs = (long long)p.B * p.G;
+  const int NB = (p.T + kBlk - 1) / kBlk;
+  const long long bg_rows = bg_stride / kD, blk_rows = blk_stride / kD;
+  // rows each tensor map may touch: up to the last row of the last block the
+  // strides can address, but never past the packed end of the buffer
+  const long long m_max = addr_mode == SPARDA_ADDR_SLOT ? pl.S - 1 : NB - 1;
+  long long extent = (kv_pairs - 1) * bg_rows + m_max * blk_rows + kBlk;
+  extent = std::min(extent, kv_pairs * bg_rows);
+  if (extent >= (1LL << 31)) return cudaErrorInvalidValue;
+  CUtensorMap mk, mv;
+  if (!tc::make_map_2d(&mk, K, kD, (uint64_t)extent, kD, 64, 64) ||
+      !tc::make_map_2d(&mv, V, kD, (uint64_t)extent, kD, 64, 64))
+    return cudaErrorNotSupported;
+  TcArgs a;
   a.Q = Q;
-  a.K = K;
-  a.V = V;
-  a.bg_stride = bg_stride;
-  a.blk_stride = blk_stride;
-  a.idx = idx;
   a.O = O;
+  a.idx = idx;
   a.status = dev_status;
   a.n_entries = pairs * pl.S;
+  a.bg_rows = bg_rows;
+  a.blk_rows = blk_rows;
   a.G = p.G;
   a.S = pl.S;
-  a.NB = (p.T + kBlk - 1) / kBlk;
+  a.NB = NB;
   a.addr_mode = addr_mode;
   a.nq = nq;
   a.q_start = q_start;
@@ -504,11 +537,11 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   w += ((parts * 8) + 255) & ~(size_t)255;
   a.counters = reinterpret_cast<uint32_t *>(w);
   switch (R) {
-    case 1: return launch_r<1, 2, 4>(a, pl.n_cta, stream);
-    case 2: return launch_r<2, 4, 3>(a, pl.n_cta, stream);
-    case 4: return launch_r<4, 4, 3>(a, pl.n_cta, stream);
-    case 8: return launch_r<8, 4, 2>(a, pl.n_cta, stream);
-    case 16: return launch_r<16, 4, 2>(a, pl.n_cta, stream);
+    case 1: return launch_tc<1, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+    case 2: return launch_tc<2, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+    case 4: return launch_tc<4, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+    case 8: return launch_tc<8, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+    case 16: return launch_tc<16, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -93,15 +93,28 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait suspends the thread in hardware until the phase completes or a
+// system-dependent time limit passes, so completion is seen at once
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; gives up after
 // kWaitCycles and returns false (the caller flags SPARDA_DEV_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-  if (mbar_test_wait(bar, parity)) return true;
-  long long t0 = clock64();
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
   for (;;) {
-    if (mbar_test_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > kWaitCycles) return false;
-    __nanosleep(20);
   }
 }
 

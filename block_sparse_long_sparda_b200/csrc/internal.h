@@ -54,7 +54,8 @@ cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
 // ---- decode attention -----------------------------------------------------
 struct DecodePlan {
   int S;            // list entries per (query, group) pair
-  long long n_cta;  // thread blocks (stream-K ranges of the flattened entries)
+  long long n_cta;      // most thread blocks a launch may use (sizes the workspace)
+  long long n_cta_min;  // fewest thread blocks the per-CTA list capacity allows
   int max_cover;    // most thread blocks any pair's entries can span
   size_t ws_bytes;  // segment partials + tickets
 };
