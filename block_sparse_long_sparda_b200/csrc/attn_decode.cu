@@ -107,35 +107,67 @@ template <int R>
 struct TcCfg {
   static constexpr int QB = R * kD * 2;  // raw query rows of one pair
   static constexpr int QB_AL = (QB + 127) / 128 * 128;
-  // stages (1024-aligned) | raw query ring | Q^T operand | P^T operand | slack
+  // stages (1024-aligned) | Q^T operand | two P^T operands | raw query ring | slack
   static size_t smem(int nstage) {
-    return (size_t)nstage * kUnitBytes + (size_t)nstage * QB_AL + 4096 + 2048 + 1024;
+    return (size_t)nstage * kUnitBytes + 4096 + 2 * 2048 + (size_t)nstage * QB_AL + 1024;
   }
 };
 
-// End of a segment: normalise and write the pair's output if this CTA covers
-// the whole pair, else store the segment's (max, sum, unnormalised output) and
-// let the last CTA to finish the pair combine all of them.  Block-wide.
+constexpr int kWarps = 8;               // 4 correction, producer, MMA, 2 softmax warps
+constexpr int kWsThreads = kWarps * 32;
+constexpr int kBarSoftmax = 1;          // named barrier: the two softmax warps
+constexpr int kBarCorr = 2;             // named barrier: the four correction warps
+constexpr int kWarpProducer = 2, kWarpMma = 3;  // softmax: warps 4, 5; correction: 0, 1, 6, 7
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// barrier among n threads that also ORs a flag over them
+__device__ __forceinline__ bool named_sync_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// bounded wait that also gives up when another role has given up
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// End of a segment, run by the 128 correction threads (thread = output
+// dim): normalise and write the pair's output if this CTA covers the whole
+// pair, else store the segment's (max, sum, unnormalised output) and let the
+// last CTA to finish the pair combine them.
 template <int R>
-__device__ __forceinline__ void segment_flush(const TcArgs &a, long long pair, bool live,
-                                              long long E, long long NC, const float (&acc)[R],
-                                              const float (&m_run)[R], const float (&l_w)[R],
-                                              float (*red)[kNQ], int *s_last) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (lane == 0)
-#pragma unroll
-    for (int h = 0; h < R; ++h) red[warp][h] = live ? l_w[h] : 0.f;
-  __syncthreads();
+__device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool live, long long E,
+                                          long long NC, const float (&acc)[R], const float *st_m,
+                                          const float *st_l, int *s_last, int dim) {
   const long long c_first = cta_of(pair * a.S, E, NC);
   const long long c_last = cta_of(pair * a.S + a.S - 1, E, NC);
   const int n_cover = (int)(c_last - c_first + 1);
   const long long slot = pair * a.max_cover + (blockIdx.x - c_first);
-  const int dim = tid;
 #pragma unroll
   for (int h = 0; h < R; ++h) {
-    const float L = red[0][h] + red[1][h] + red[2][h] + red[3][h];
+    const float L = live ? st_l[h] + st_l[kNQ + h] : 0.f;
+    const float M = live ? st_m[h] : -INFINITY;
     const float o = live ? acc[h] : 0.f;
-    const float M = live ? m_run[h] : -INFINITY;
     if (n_cover == 1) {
       const float r = L > 0.f ? o / L : 0.f;
       a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
@@ -146,9 +178,9 @@ __device__ __forceinline__ void segment_flush(const TcArgs &a, long long pair, b
   }
   if (n_cover > 1) {
     __threadfence();
-    __syncthreads();
-    if (tid == 0) *s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
-    __syncthreads();
+    named_sync(kBarCorr, 128);
+    if (dim == 0) *s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
+    named_sync(kBarCorr, 128);
     if (*s_last) {
       __threadfence();
       const long long base = pair * a.max_cover;
@@ -166,33 +198,37 @@ __device__ __forceinline__ void segment_flush(const TcArgs &a, long long pair, b
         const float r = L > 0.f ? o / L : 0.f;
         a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
       }
-      if (tid == 0) a.counters[pair] = 0u;
+      if (dim == 0) a.counters[pair] = 0u;
     }
   }
-  __syncthreads();
+  named_sync(kBarCorr, 128);
 }
 
 template <int R, int NSTAGE>
-__global__ void __launch_bounds__(kThreads) attn_tc_kernel(const __grid_constant__ CUtensorMap mapK,
-                                                           const __grid_constant__ CUtensorMap mapV,
-                                                           TcArgs a) {
+__global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_constant__ CUtensorMap mapK,
+                                                             const __grid_constant__ CUtensorMap mapV,
+                                                             TcArgs a) {
   using C = TcCfg<R>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
-  uint8_t *stages = sm;                              // NSTAGE x 32 KB
-  uint8_t *qop = sm + NSTAGE * kUnitBytes;           // Q^T operand: 16 rows x 128 dims
-  uint8_t *pop = qop + 4096;                         // P^T operand: 16 rows x 64 keys
-  uint8_t *qraw = pop + 2048;                        // NSTAGE raw query slots
-  __shared__ __align__(8) uint64_t full_bar[NSTAGE];
-  __shared__ __align__(8) uint64_t mma1_bar, mma2_bar;
+  uint8_t *stages = sm;                          // NSTAGE x 32 KB
+  uint8_t *qop = sm + NSTAGE * kUnitBytes;       // Q^T operand: 16 rows x 128 dims
+  uint8_t *pop = qop + 4096;                     // two P^T operands: 16 rows x 64 keys
+  uint8_t *qraw = pop + 2 * 2048;                // NSTAGE raw query slots
+  __shared__ __align__(8) uint64_t full_bar[NSTAGE], empty_bar[NSTAGE];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
   __shared__ uint32_t tmem_base;
   __shared__ int s_row[kMaxEnt];   // TMA row coordinate of the block
   __shared__ int s_rows[kMaxEnt];  // keys of the block at or before the query
   __shared__ int s_seg[kMaxEnt];   // segment (pair - pair0)
   __shared__ int s_tmp[33];
   __shared__ int s_last;
-  __shared__ float red[4][kNQ];
+  __shared__ volatile int s_abort;
+  __shared__ float red[2][kNQ];            // per-warp block maxima (softmax warps)
+  __shared__ float corr_s[2][kNQ];         // rescale factor of a block (double buffer)
+  __shared__ float seg_m[4][kNQ];          // running max at a segment's end (ring of 4)
+  __shared__ float seg_l[4][2][kNQ];       // per-warp sums at a segment's end
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long E = a.n_entries, NC = gridDim.x;
@@ -226,218 +262,282 @@ __global__ void __launch_bounds__(kThreads) attn_tc_kernel(const __grid_constant
     }
   }
   int nb;
-  const int off = block_excl_scan<kThreads>(cnt, s_tmp, nb);
+  const int off = block_excl_scan<kWsThreads>(cnt, s_tmp, nb);
   if (cnt) {
     s_row[off] = row_;
     s_rows[off] = rows_;
     s_seg[off] = seg_;
   }
   if (tid == 0) {
-    for (int st = 0; st < NSTAGE; ++st) mbar_init(&full_bar[st], 1);
-    mbar_init(&mma1_bar, 1);
-    mbar_init(&mma2_bar, 1);
+    for (int st = 0; st < NSTAGE; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 64);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], 128);
+    }
+    s_abort = 0;
     fence_mbar_init();
     tc::prefetch_map(&mapK);
     tc::prefetch_map(&mapV);
   }
-  if (warp == 0) tc::tmem_alloc(&tmem_base, 32);
-  // operand tiles start zeroed: rows >= R of Q^T and P^T stay zero
-  for (int i = tid; i < (4096 + 2048) / 16; i += kThreads)
+  if (warp == 0) tc::tmem_alloc(&tmem_base, 64);
+  for (int i = tid; i < (4096 + 4096) / 16; i += kWsThreads)  // Q^T, P^T rows >= R stay zero
     reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = tmem_base;
-  const uint32_t tS = tmem, tO = tmem + kNQ;
-  const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
-  constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
-  constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
-  // operand descriptors: fixed bases, advanced in 16-byte units
-  const uint64_t dK = tc::sdesc(stages, 16, 1024);          // S^T A operand (K tiles)
-  const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);  // O^T A operand (V^T)
-  const uint64_t dQ = tc::sdesc(qop, 16, 1024);
-  const uint64_t dP = tc::sdesc(pop, 16, 1024);
+  const uint32_t tmem = tmem_base;  // S0 | S1 | O0 | O1, 16 columns each
+  auto first_of = [&](int u) { return u == 0 || s_seg[u - 1] != s_seg[u]; };
+  auto last_of = [&](int u) { return u == nb - 1 || s_seg[u + 1] != s_seg[u]; };
 
-  // thread 0 only: TMA for block bi into its stage (+ the pair's query rows
-  // at the first block of a segment)
-  auto issue = [&](int bi) {
-    const int st = bi % NSTAGE;
-    const int seg = s_seg[bi];
-    const bool first = bi == 0 || s_seg[bi - 1] != seg;
-    uint8_t *dst = stages + st * kUnitBytes;
-    const int row = s_row[bi];
-    mbar_arrive_expect_tx(&full_bar[st], kUnitBytes + (first ? C::QB : 0));
-    tc::tma_load_2d(dst, &mapK, 0, row, &full_bar[st]);
-    tc::tma_load_2d(dst + kTile, &mapV, 0, row, &full_bar[st]);
-    tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
-    tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &full_bar[st]);
-    if (first) bulk_g2s(qraw + st * C::QB_AL, a.Q + (pair0 + seg) * R * kD, C::QB, &full_bar[st]);
-  };
-  // thread 0 only: S^T = K Q^T for block bi (rows 0-63 are its keys)
-  auto mma1 = [&](int bi) {
-    const uint64_t base = dK + (uint64_t)((bi % NSTAGE) * (kUnitBytes >> 4));
-    tc::fence_after_sync();
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      tc::mma_bf16(tS, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
-                   dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
-    tc::mma_commit(&mma1_bar);
-  };
-  if (tid == 0)
-    for (int bi = 0; bi < min(nb, NSTAGE); ++bi) issue(bi);
+  int produced = 0;  // producer: blocks whose TMA was issued
 
-  // per thread: acc = one output dim (tid) of every head; m_run uniform;
-  // l_w = this warp's share of the probability sums
-  float acc[R], m_run[R], l_w[R];
-#pragma unroll
-  for (int h = 0; h < R; ++h) {
-    acc[h] = 0.f;
-    m_run[h] = -INFINITY;
-    l_w[h] = 0.f;
-  }
-  uint32_t ph1 = 0, ph2 = 0;
-  int early = -1;        // thread 0: block whose MMA1 is already in flight
-  bool bad = false;      // this thread saw a wait give up
-  int cur = -1, next_flush = 0, abort_at = -1;
-  int issued_to = min(nb, NSTAGE);  // thread 0: blocks [0, issued_to) have TMA issued
-
+  if (warp == kWarpProducer) {
+    // ================= producer =================
+    if (lane == 0) {
 #pragma unroll 1
-  for (int bi = 0; bi < nb; ++bi) {
-    const int st = bi % NSTAGE;
-    const uint32_t tph = (uint32_t)((bi / NSTAGE) & 1);
-    const int seg = s_seg[bi];
-    if (seg != cur) {  // a new segment: its query arrived with this block
-      for (int f = next_flush; f < seg; ++f)
-        segment_flush<R>(a, pair0 + f, f == cur, E, NC, acc, m_run, l_w, red, &s_last);
-      next_flush = seg;
-      cur = seg;
-#pragma unroll
-      for (int h = 0; h < R; ++h) {
-        acc[h] = 0.f;
-        m_run[h] = -INFINITY;
-        l_w[h] = 0.f;
+      for (int u = 0; u < nb; ++u) {
+        const int st = u % NSTAGE;
+        if (u >= NSTAGE &&
+            !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), &s_abort))
+          break;
+        const bool first = first_of(u);
+        uint8_t *dst = stages + st * kUnitBytes;
+        const int row = s_row[u];
+        mbar_arrive_expect_tx(&full_bar[st], kUnitBytes + (first ? C::QB : 0));
+        tc::tma_load_2d(dst, &mapK, 0, row, &full_bar[st]);
+        tc::tma_load_2d(dst + kTile, &mapV, 0, row, &full_bar[st]);
+        tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
+        tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &full_bar[st]);
+        if (first)
+          bulk_g2s(qraw + st * C::QB_AL, a.Q + (pair0 + s_seg[u]) * R * kD, C::QB, &full_bar[st]);
+        produced = u + 1;
       }
-      if (!mbar_wait_bounded(&full_bar[st], tph)) bad = true;
-      if (__syncthreads_or(bad)) {
-        abort_at = bi;
+    }
+  } else if (warp == kWarpMma) {
+    // ================= MMA issuer =================
+    // O^T(v) is issued as soon as the softmax of v is done and O[v & 1] is
+    // free (it gates the correction and so the next softmax); S^T(u) as soon
+    // as its block has landed and S[u & 1] is free.
+    constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
+    constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
+    const uint64_t dK = tc::sdesc(stages, 16, 1024);
+    const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);
+    const uint64_t dQ = tc::sdesc(qop, 16, 1024);
+    const uint64_t dP = tc::sdesc(pop, 16, 1024);
+    int n1 = 0, n2 = 0;  // next S^T and next O^T to issue
+    long long t_idle = 0;
+    bool ok = true;
+#pragma unroll 1
+    while (n2 < nb) {
+      bool did = false;
+      if (n2 < n1) {
+        const int v = n2, st = v % NSTAGE;
+        bool ready = mbar_test_wait(&p_full[v & 1], (uint32_t)((v >> 1) & 1));
+        if (ready && v >= 2) ready = mbar_test_wait(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1));
+        if (__all_sync(0xffffffffu, ready)) {
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint64_t base = dV + (uint64_t)(st * (kUnitBytes >> 4));
+            const uint64_t bp = dP + (uint64_t)((v & 1) * (2048 >> 4));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc::mma_bf16(tmem + 2 * kNQ + (v & 1) * kNQ, base + (uint64_t)(k * 128),
+                           bp + (uint64_t)(k * 2), id2, k > 0);
+            tc::mma_commit(&o_full[v & 1]);
+            tc::mma_commit(&empty_bar[st]);
+          }
+          __syncwarp();
+          ++n2;
+          did = true;
+        }
+      }
+      if (n1 < nb) {
+        const int u = n1, st = u % NSTAGE;
+        bool ready = mbar_test_wait(&full_bar[st], (uint32_t)((u / NSTAGE) & 1));
+        if (ready && u >= 2) ready = mbar_test_wait(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1));
+        const bool first = first_of(u);
+        if (ready && first && u >= 1)  // the previous S^T must be done with the old query
+          ready = mbar_test_wait(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1));
+        if (__all_sync(0xffffffffu, ready)) {
+          if (first) {
+            const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
+            for (int i = lane; i < R * 16; i += 32) {
+              const int h = i >> 4, c8 = i & 15;
+              *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint64_t base = dK + (uint64_t)(st * (kUnitBytes >> 4));
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              tc::mma_bf16(tmem + (u & 1) * kNQ, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
+                           dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
+            tc::mma_commit(&s_full[u & 1]);
+          }
+          __syncwarp();
+          ++n1;
+          did = true;
+        }
+      }
+      if (did) {
+        t_idle = 0;
+      } else {
+        const long long now = clock64();
+        if (t_idle == 0) t_idle = now;
+        if (__any_sync(0xffffffffu, s_abort != 0 || now - t_idle > kWaitCycles)) {
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (!ok) s_abort = 1;
+  } else if (warp == 4 || warp == 5) {
+    // ================= softmax (thread = key of the block) =================
+    const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
+    const int key = tid - 128;
+    float m_run[R], l_t[R];
+    int smx_k = -1;  // count of segments with blocks, for the statistics ring
+    bool ok = true;
+#pragma unroll 1
+    for (int u = 0; u < nb; ++u) {
+      const int b = u & 1;
+      if (first_of(u)) {
+        ++smx_k;
+#pragma unroll
+        for (int h = 0; h < R; ++h) {
+          m_run[h] = -INFINITY;
+          l_t[h] = 0.f;
+        }
+      }
+      if (ok) ok = wait_or_abort(&s_full[b], (uint32_t)((u >> 1) & 1), &s_abort);
+      // block u-2 is fully corrected: its P^T and corr slots are free
+      if (ok && u >= 2) ok = wait_or_abort(&o_free[b], (uint32_t)(((u - 2) >> 1) & 1), &s_abort);
+      tc::fence_after_sync();
+      float x[R];
+      {
+        float sv[16];
+        tc::tmem_ld16(tmem + b * kNQ + lane_sel, sv);
+        const bool valid = key < s_rows[u];
+#pragma unroll
+        for (int h = 0; h < R; ++h) x[h] = valid ? sv[h] * a.scale_log2 : -INFINITY;
+#pragma unroll
+        for (int h = 0; h < R; ++h) {
+          const float mx = warp_max_xor(x[h], 1, 32);
+          if (lane == 0) red[warp - 4][h] = mx;
+        }
+      }
+      if (named_sync_or(kBarSoftmax, 64, !ok)) {
+        ok = false;
         break;
       }
-      const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
-      for (int i = tid; i < R * 16; i += kThreads) {
-        const int h = i >> 4, c8 = i & 15;
-        *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-    }
-    if (tid == 0 && early != bi) {
-      if (mbar_wait_bounded(&full_bar[st], tph)) mma1(bi);
-      else bad = true;
-    }
-    if (!mbar_wait_bounded(&mma1_bar, ph1)) bad = true;
-    ph1 ^= 1;
-    tc::fence_after_sync();
-
-    // ---- softmax over this block's keys (thread = key, in warps 0 and 1) ----
-    const int rows = s_rows[bi];
-    float x[R];
-    if (warp < 2) {
-      float sv[16];
-      tc::tmem_ld16(tS + lane_sel, sv);
-      const bool valid = tid < rows;
-#pragma unroll
-      for (int h = 0; h < R; ++h) x[h] = valid ? sv[h] * a.scale_log2 : -INFINITY;
+      float cr[R];
 #pragma unroll
       for (int h = 0; h < R; ++h) {
-        const float mx = warp_max_xor(x[h], 1, 32);
-        if (lane == 0) red[warp][h] = mx;
+        const float mn = fmaxf(m_run[h], fmaxf(red[0][h], red[1][h]));
+        cr[h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[h] - mn);
+        m_run[h] = mn;
       }
-    }
-    tc::fence_before_sync();
-    if (__syncthreads_or(bad)) {
-      abort_at = bi;
-      break;
-    }
-    float corr[R];
-#pragma unroll
-    for (int h = 0; h < R; ++h) {
-      const float mn = fmaxf(m_run[h], fmaxf(red[0][h], red[1][h]));
-      corr[h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[h] - mn);
-      m_run[h] = mn;
-      l_w[h] *= corr[h];
-    }
-    float pr[R];
-    if (warp < 2) {
+      uint8_t *pb = pop + b * 2048;
 #pragma unroll
       for (int h = 0; h < R; ++h) {
         const float p = (x[h] == -INFINITY) ? 0.f : exp2f(x[h] - m_run[h]);
-        const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-        *reinterpret_cast<__nv_bfloat16 *>(pop + tc::sw128_offset(h, tid)) = pb;
-        pr[h] = __bfloat162float(pb);
+        const __nv_bfloat16 pv = __float2bfloat16_rn(p);
+        *reinterpret_cast<__nv_bfloat16 *>(pb + tc::sw128_offset(h, key)) = pv;
+        l_t[h] = l_t[h] * cr[h] + __bfloat162float(pv);
       }
+      if (key < R) corr_s[b][key] = cr[key];
+      if (last_of(u)) {  // publish the segment's statistics
+#pragma unroll
+        for (int h = 0; h < R; ++h) {
+          const float ls = warp_sum_xor(l_t[h], 1, 32);
+          if (lane == 0) seg_l[smx_k & 3][warp - 4][h] = ls;
+        }
+        if (key < R) seg_m[smx_k & 3][key] = m_run[key];
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(&p_full[b]);
+      // both softmax warps finish the block before either reuses red[]
+      named_sync(kBarSoftmax, 64);
     }
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-
-    // ---- O^T(block) = V^T P^T; the next block's S^T right behind it ----
-    if (tid == 0) {
+    if (!ok) s_abort = 1;
+  } else {
+    // ============ correction (warps 0, 1, 6, 7; thread = output dim) ============
+    const int q = warp & 3;  // TMEM lane quadrant
+    const uint32_t lane_sel = (uint32_t)(q * 32) << 16;
+    const int dim = q * 32 + lane;
+    float acc[R];
+#pragma unroll
+    for (int h = 0; h < R; ++h) acc[h] = 0.f;
+    int cur = -1, next_flush = 0;
+    int live_k = -1;  // count of segments with blocks seen so far
+    bool ok = true;
+    // The statistics of a segment ending at block v-1 were published before
+    // p_full(v-1), which correction(v-1) already waited for.
+#pragma unroll 1
+    for (int v = 0; v < nb; ++v) {
+      const int seg = s_seg[v];
+      if (seg != cur) {
+        if (named_sync_or(kBarCorr, 128, !ok)) {
+          ok = false;
+          break;
+        }
+        for (int f = next_flush; f < seg; ++f)
+          seg_flush<R>(a, pair0 + f, f == cur, E, NC, acc, seg_m[live_k & 3],
+                       &seg_l[live_k & 3][0][0], &s_last, dim);
+        next_flush = seg;
+        cur = seg;
+        ++live_k;
+#pragma unroll
+        for (int h = 0; h < R; ++h) acc[h] = 0.f;
+      }
+      if (ok) ok = wait_or_abort(&o_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
+      if (ok) ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
+      // one vote for all four warps, so they always leave at the same barrier
+      if (named_sync_or(kBarCorr, 128, !ok)) {
+        ok = false;
+        break;
+      }
       tc::fence_after_sync();
-      const uint64_t base = dV + (uint64_t)(st * (kUnitBytes >> 4));
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        tc::mma_bf16(tO, base + (uint64_t)(k * 128), dP + (uint64_t)(k * 2), id2, k > 0);
-      tc::mma_commit(&mma2_bar);
-      const int nx = bi + 1;
-      if (nx < nb && s_seg[nx] == seg &&
-          mbar_test_wait(&full_bar[nx % NSTAGE], (uint32_t)((nx / NSTAGE) & 1))) {
-        mma1(nx);
-        early = nx;
-      }
-    }
-    if (warp < 2) {  // probability sums, while the tensor core works
-#pragma unroll
-      for (int h = 0; h < R; ++h) l_w[h] += warp_sum_xor(pr[h], 1, 32);
-    }
-    if (!mbar_wait_bounded(&mma2_bar, ph2)) bad = true;
-    ph2 ^= 1;
-    tc::fence_after_sync();
-    // both MMAs of block bi are done: its stage can be refilled
-    if (tid == 0 && bi + NSTAGE < nb && !bad) {
-      issue(bi + NSTAGE);
-      issued_to = bi + NSTAGE + 1;
-    }
-    {
       float ov[16];
-      tc::tmem_ld16(tO + lane_sel, ov);
+      tc::tmem_ld16(tmem + 2 * kNQ + (v & 1) * kNQ + lane_sel, ov);
 #pragma unroll
-      for (int h = 0; h < R; ++h) acc[h] = acc[h] * corr[h] + ov[h];
+      for (int h = 0; h < R; ++h) acc[h] = acc[h] * corr_s[v & 1][h] + ov[h];
+      tc::fence_before_sync();
+      mbar_arrive(&o_free[v & 1]);
     }
-    tc::fence_before_sync();
+    // all four warps agree before the last flushes (which use the barrier)
+    if (named_sync_or(kBarCorr, 128, !ok)) ok = false;
+    if (ok)
+      for (int f = next_flush; f < n_seg; ++f)
+        seg_flush<R>(a, pair0 + f, f == cur, E, NC, acc, seg_m[live_k & 3], &seg_l[live_k & 3][0][0],
+                     &s_last, dim);
+    if (!ok) s_abort = 1;
   }
-  if (abort_at < 0 && __syncthreads_or(bad)) abort_at = nb;
 
-  if (abort_at >= 0) {
-    // something never completed: let what was issued land (bounded), then
-    // free TMEM and leave; the status word says why
+  __syncthreads();
+  if (s_abort) {
+    // something never completed: give what was issued a bounded chance to
+    // land before the CTA's memory is released; the status word says why
     flag_status(a.status, SPARDA_DEV_TIMEOUT);
-    if (tid == 0) {
-      for (int bj = max(0, abort_at); bj < issued_to; ++bj)
-        (void)mbar_wait_bounded(&full_bar[bj % NSTAGE], (uint32_t)((bj / NSTAGE) & 1));
-      (void)mbar_wait_bounded(&mma1_bar, ph1);
-      (void)mbar_wait_bounded(&mma2_bar, ph2);
+    if (warp == kWarpProducer && lane == 0) {
+      for (int u = max(0, produced - NSTAGE); u < produced; ++u)
+        (void)mbar_wait_bounded(&full_bar[u % NSTAGE], (uint32_t)((u / NSTAGE) & 1));
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 32);
-    return;
   }
-  for (int f = next_flush; f < n_seg; ++f)
-    segment_flush<R>(a, pair0 + f, f == cur, E, NC, acc, m_run, l_w, red, &s_last);
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 32);
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, 64);
 }
 
 template <int R, int NSTAGE>
@@ -447,12 +547,14 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
   auto kern = attn_tc_kernel<R, NSTAGE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
   // one wave: as many CTAs as the device keeps resident (never more than
   // the plan sized the workspace for, never fewer than the lists need)
   int dev = 0, n_sm = 148, occ = 1;
   if (cudaGetDevice(&dev) == cudaSuccess)
     (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem) != cudaSuccess || occ < 1)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWsThreads, smem) != cudaSuccess || occ < 1)
     occ = 1;
   (void)cudaGetLastError();
   long long grid = (long long)occ * n_sm;
@@ -460,7 +562,7 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
   if (forced > 0) grid = forced;
   grid = std::max(grid, grid_min);
   grid = std::min(grid, grid_max);
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(mk, mv, a);
+  kern<<<(unsigned)grid, kWsThreads, smem, stream>>>(mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -536,14 +638,25 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.ws_ml = reinterpret_cast<float2 *>(w);
   w += ((parts * 8) + 255) & ~(size_t)255;
   a.counters = reinterpret_cast<uint32_t *>(w);
+  // ring depth: 3 x 32 KB with two resident CTAs per SM measured best; 4 and
+  // 6 (one CTA per SM, 5 when 16 heads share a group) stay selectable
+  // through SPARDA_DECODE_STAGES for sweeps
+  int stages = env_int("SPARDA_DECODE_STAGES");
+  if (stages == 0) stages = 3;
+#define SPARDA_LAUNCH_R(RR)                                                             \
+  if (stages <= 3) return launch_tc<RR, 3>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages == 4) return launch_tc<RR, 4>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (RR >= 16) return launch_tc<RR, 5>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  return launch_tc<RR, 6>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
   switch (R) {
-    case 1: return launch_tc<1, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
-    case 2: return launch_tc<2, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
-    case 4: return launch_tc<4, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
-    case 8: return launch_tc<8, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
-    case 16: return launch_tc<16, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+    case 1: SPARDA_LAUNCH_R(1)
+    case 2: SPARDA_LAUNCH_R(2)
+    case 4: SPARDA_LAUNCH_R(4)
+    case 8: SPARDA_LAUNCH_R(8)
+    case 16: SPARDA_LAUNCH_R(16)
     default: return cudaErrorInvalidValue;
   }
+#undef SPARDA_LAUNCH_R
 }
 
 cudaError_t launch_attn_decode(const sparda_params &p, const DecodePlan &pl, const uint16_t *Q,
