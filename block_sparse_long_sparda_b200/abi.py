@@ -69,6 +69,7 @@ _SIGS = {
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
+    "sparda_sparse_attn_decode_noalloc": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _P]),
     "sparda_workspace_size": (_SZ, [_I, _PP, _I, _I]),
     "sparda_status_string": (ctypes.c_char_p, [_I]),
     "sparda_status_from_device": (_I, [ctypes.c_int32]),
@@ -162,6 +163,21 @@ def sparda_sparse_attn_prefill(p, Q, nq, q_start, K, V, bg_stride, tok_stride, i
                                             _ptr(K), _ptr(V), int(bg_stride), int(tok_stride),
                                             _ptr(idx), _ptr(O), _ptr(ws), _nbytes(ws),
                                             _ptr(dev_status), _stream(stream)))
+
+
+def sparda_sparse_attn_decode_noalloc(p, Q, K, V, bg_stride, blk_stride, idx, addr_mode, O,
+                                      dev_status=None, stream=None):
+    """Decode attention for callers that cannot allocate device memory: the
+    scratch is a fixed device array inside the library (see include/sparda.h
+    for its size and the rule that calls must not overlap on the device)."""
+    _check("sparda_sparse_attn_decode_noalloc",
+           lib().sparda_sparse_attn_decode_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V),
+                                                   int(bg_stride), int(blk_stride), _ptr(idx),
+                                                   int(addr_mode), _ptr(O), _ptr(dev_status),
+                                                   _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def sparda_workspace_size(op, p, nq=1, nf=1) -> int:

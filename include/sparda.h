@@ -204,6 +204,29 @@ int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, in
                                long long tok_stride, const int32_t *idx, void *O, void *ws,
                                size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream);
 
+/*
+ * sparda_sparse_attn_decode_noalloc -- sparda_sparse_attn_decode for callers
+ * that cannot allocate device memory (code running under stream capture,
+ * runtimes that own all device memory and hand kernels fixed buffers).  The
+ * pages have no counterpart: this is a property of the library, not of the
+ * method.  Arguments and results are those of sparda_sparse_attn_decode
+ * without the workspace; the scratch lives in a fixed device array of
+ * SPARDA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.
+ *  - shapes needing more scratch than that return SPARDA_EWORKSPACE;
+ *  - every call shares the array, and each call clears the part that must
+ *    start at zero: calls that may overlap on the device race and must not
+ *    be issued;
+ *  - the first call on a device looks up the array's device address with
+ *    that device current; make it before any stream capture.
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+#define SPARDA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int sparda_sparse_attn_decode_noalloc(const sparda_params *p, const void *Q, const void *K,
+                                      const void *V, long long bg_stride, long long blk_stride,
+                                      const int32_t *idx, int addr_mode, void *O,
+                                      int32_t *dev_status, sparda_stream_t stream);
+
 /* Bytes of device workspace an op needs for these shapes (0: none). nf is
  * the number of scoring vectors per group (select only). */
 size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf);
