@@ -47,6 +47,7 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kGridMax = 3 * 148;               // most CTAs a B200 keeps resident
+constexpr int kMaxDevices = 64;
 
 // the CTA whose range holds entry e (ranges: [c*E/C, (c+1)*E/C))
 __device__ __forceinline__ long long cta_of(long long e, long long E, long long C) {
@@ -113,11 +114,11 @@ struct TcCfg {
   }
 };
 
-constexpr int kWarps = 8;               // 4 correction, producer, MMA, 2 softmax warps
+constexpr int kWarps = 9;               // 4 correction, producer, 2 MMA issuers, 2 softmax warps
 constexpr int kWsThreads = kWarps * 32;
 constexpr int kBarSoftmax = 1;          // named barrier: the two softmax warps
 constexpr int kBarCorr = 2;             // named barrier: the four correction warps
-constexpr int kWarpProducer = 2, kWarpMma = 3;  // softmax: warps 4, 5; correction: 0, 1, 6, 7
+constexpr int kWarpProducer = 2, kWarpMma = 3, kWarpMma2 = 8;  // softmax: 4, 5; correction: 0, 1, 6, 7
 
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -320,84 +321,72 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
       }
     }
   } else if (warp == kWarpMma) {
-    // ================= MMA issuer =================
-    // O^T(v) is issued as soon as the softmax of v is done and O[v & 1] is
-    // free (it gates the correction and so the next softmax); S^T(u) as soon
-    // as its block has landed and S[u & 1] is free.
+    // ================= S^T issuer =================
+    // S^T(u) as soon as its block has landed and the softmax of u-2 is done
+    // with S[u & 1].
     constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
-    constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
     const uint64_t dK = tc::sdesc(stages, 16, 1024);
-    const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);
     const uint64_t dQ = tc::sdesc(qop, 16, 1024);
-    const uint64_t dP = tc::sdesc(pop, 16, 1024);
-    int n1 = 0, n2 = 0;  // next S^T and next O^T to issue
-    long long t_idle = 0;
     bool ok = true;
 #pragma unroll 1
-    while (n2 < nb) {
-      bool did = false;
-      if (n2 < n1) {
-        const int v = n2, st = v % NSTAGE;
-        bool ready = mbar_test_wait(&p_full[v & 1], (uint32_t)((v >> 1) & 1));
-        if (ready && v >= 2) ready = mbar_test_wait(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1));
-        if (__all_sync(0xffffffffu, ready)) {
-          if (lane == 0) {
-            tc::fence_after_sync();
-            const uint64_t base = dV + (uint64_t)(st * (kUnitBytes >> 4));
-            const uint64_t bp = dP + (uint64_t)((v & 1) * (2048 >> 4));
+    for (int u = 0; u < nb && ok; ++u) {
+      const int st = u % NSTAGE;
+      ok = wait_or_abort(&full_bar[st], (uint32_t)((u / NSTAGE) & 1), &s_abort);
+      if (ok && u >= 2) ok = wait_or_abort(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1), &s_abort);
+      const bool first = first_of(u);
+      if (ok && first && u >= 1)  // the previous S^T must be done with the old query
+        ok = wait_or_abort(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1), &s_abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (first) {
+        const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
+        for (int i = lane; i < R * 16; i += 32) {
+          const int h = i >> 4, c8 = i & 15;
+          *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint64_t base = dK + (uint64_t)(st * (kUnitBytes >> 4));
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              tc::mma_bf16(tmem + 2 * kNQ + (v & 1) * kNQ, base + (uint64_t)(k * 128),
-                           bp + (uint64_t)(k * 2), id2, k > 0);
-            tc::mma_commit(&o_full[v & 1]);
-            tc::mma_commit(&empty_bar[st]);
-          }
-          __syncwarp();
-          ++n2;
-          did = true;
-        }
+        for (int k = 0; k < 8; ++k)
+          tc::mma_bf16(tmem + (u & 1) * kNQ, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
+                       dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
+        tc::mma_commit(&s_full[u & 1]);
       }
-      if (n1 < nb) {
-        const int u = n1, st = u % NSTAGE;
-        bool ready = mbar_test_wait(&full_bar[st], (uint32_t)((u / NSTAGE) & 1));
-        if (ready && u >= 2) ready = mbar_test_wait(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1));
-        const bool first = first_of(u);
-        if (ready && first && u >= 1)  // the previous S^T must be done with the old query
-          ready = mbar_test_wait(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1));
-        if (__all_sync(0xffffffffu, ready)) {
-          if (first) {
-            const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
-            for (int i = lane; i < R * 16; i += 32) {
-              const int h = i >> 4, c8 = i & 15;
-              *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-          }
-          if (lane == 0) {
-            tc::fence_after_sync();
-            const uint64_t base = dK + (uint64_t)(st * (kUnitBytes >> 4));
+      __syncwarp();
+    }
+    if (!ok) s_abort = 1;
+  } else if (warp == kWarpMma2) {
+    // ================= O^T issuer =================
+    // O^T(v) as soon as the softmax of v is done and the correction of v-2 has
+    // read O[v & 1]; its completion also frees the block's stage (the block's
+    // S^T finished before its softmax began).
+    constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
+    const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);
+    const uint64_t dP = tc::sdesc(pop, 16, 1024);
+    bool ok = true;
+#pragma unroll 1
+    for (int v = 0; v < nb && ok; ++v) {
+      const int st = v % NSTAGE;
+      ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
+      if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), &s_abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint64_t base = dV + (uint64_t)(st * (kUnitBytes >> 4));
+        const uint64_t bp = dP + (uint64_t)((v & 1) * (2048 >> 4));
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              tc::mma_bf16(tmem + (u & 1) * kNQ, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
-                           dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
-            tc::mma_commit(&s_full[u & 1]);
-          }
-          __syncwarp();
-          ++n1;
-          did = true;
-        }
+        for (int k = 0; k < 4; ++k)
+          tc::mma_bf16(tmem + 2 * kNQ + (v & 1) * kNQ, base + (uint64_t)(k * 128), bp + (uint64_t)(k * 2),
+                       id2, k > 0);
+        tc::mma_commit(&o_full[v & 1]);
+        tc::mma_commit(&empty_bar[st]);
       }
-      if (did) {
-        t_idle = 0;
-      } else {
-        const long long now = clock64();
-        if (t_idle == 0) t_idle = now;
-        if (__any_sync(0xffffffffu, s_abort != 0 || now - t_idle > kWaitCycles)) {
-          ok = false;
-          break;
-        }
-      }
+      __syncwarp();
     }
     if (!ok) s_abort = 1;
   } else if (warp == 4 || warp == 5) {
@@ -545,19 +534,33 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
                       long long grid_max, long long grid_min, cudaStream_t stream) {
   const size_t smem = TcCfg<R>::smem(NSTAGE);
   auto kern = attn_tc_kernel<R, NSTAGE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e != cudaSuccess) return e;
-  // one wave: as many CTAs as the device keeps resident (never more than
-  // the plan sized the workspace for, never fewer than the lists need)
-  int dev = 0, n_sm = 148, occ = 1;
-  if (cudaGetDevice(&dev) == cudaSuccess)
+  // per device, once: shared-memory attributes and how many CTAs stay
+  // resident (one wave: as many CTAs as the device keeps resident, never
+  // more than the plan sized the workspace for, never fewer than the lists
+  // need)
+  static int resident[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (resident[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    // resident CTAs per SM from the shared-memory budget (each CTA also
+    // holds its static shared memory and the per-block reservation)
+    int n_sm = 148, per_sm = 0, reserved = 0;
     (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kWsThreads, smem) != cudaSuccess || occ < 1)
-    occ = 1;
-  (void)cudaGetLastError();
-  long long grid = (long long)occ * n_sm;
+    (void)cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    (void)cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaFuncAttributes fa;
+    size_t stat = 4096;
+    if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess) stat = fa.sharedSizeBytes;
+    (void)cudaGetLastError();
+    int occ = per_sm > 0 ? (int)((size_t)per_sm / (smem + stat + (size_t)reserved)) : 1;
+    occ = std::max(1, std::min(occ, 3));
+    resident[dev] = occ * n_sm;
+  }
+  long long grid = resident[dev];
   const int forced = env_int("SPARDA_DECODE_CTAS");
   if (forced > 0) grid = forced;
   grid = std::max(grid, grid_min);

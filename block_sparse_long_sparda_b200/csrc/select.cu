@@ -94,10 +94,15 @@ __device__ void radix_threshold(const uint32_t *keys, int n, int k, uint32_t *hi
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kSelThreads) {
-      const uint32_t u = keys[i];
-      const bool match = pass == 0 ? true : (((u ^ prefix) >> (shift + 8)) == 0u);
-      if (match) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    // warp-aggregated: lanes holding the same digit add once (scores cluster
+    // in a few top-level bins, where plain atomics would serialise)
+    for (int base = warp * 32; base < n; base += kSelThreads) {
+      const int i = base + lane;
+      const uint32_t u = i < n ? keys[i] : 0u;
+      const bool match = i < n && (pass == 0 || ((u ^ prefix) >> (shift + 8)) == 0u);
+      const uint32_t bin = match ? ((u >> shift) & 255u) : 256u;
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -406,10 +411,16 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     a.cand_key = reinterpret_cast<uint32_t *>(w);
     smem = (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
+  if (smem > 48 * 1024) {  // raised once per device to the largest size used
+    static size_t raised[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (raised[dev] < smem) {
+      cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+      if (e != cudaSuccess) return e;
+      raised[dev] = smem;
+    }
   }
   const long long grid = pl.n_problems * pl.n_chunks;
   select_kernel<<<(unsigned)grid, kSelThreads, smem, stream>>>(a);
