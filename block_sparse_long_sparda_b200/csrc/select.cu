@@ -19,8 +19,8 @@
 // orderable uint32 keys.  A chunk CTA only streams and scores, writing its
 // keys to the workspace, so CTAs are short and many are in flight.  The
 // chunks of a problem meet through an atomic ticket: the last CTA to finish
-// (no waiting) loads every key of the problem from L2, a 4-pass 8-bit radix
-// select finds the k-th key, and a block scan in block order keeps
+// (no waiting) loads every key of the problem from L2, a binned search finds
+// the k-th key exactly, and a ballot-and-scan pass in block order keeps
 // everything above it plus the lowest-index ties -- results come out sorted
 // by block id and ties go to the lower id -- and writes init U top-k U local.
 // No CTA ever waits for another.
@@ -35,7 +35,7 @@ namespace sparda {
 namespace {
 
 constexpr int kSelThreads = 256;
-constexpr int kMaxCand = 32768;   // candidates one problem may have (keys fit in shared memory)
+constexpr int kMaxCand = 24576;   // candidates one problem may have (keys fit in shared memory)
 constexpr int kMaxNf = 16;
 
 struct SelArgs {
@@ -52,122 +52,221 @@ struct SelArgs {
 // block-wide helpers (blockDim.x == kSelThreads)
 // ---------------------------------------------------------------------------
 
-// Exclusive prefix sum over threads in thread order; `tmp` holds 33 words.
-__device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *tmp, uint32_t &total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int nw = kSelThreads / 32;
-  uint32_t x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += t;
-  }
-  if (lane == 31) tmp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = lane < nw ? tmp[lane] : 0u;
-    uint32_t incl = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane < nw) tmp[lane] = incl - w;
-    if (lane == nw - 1) tmp[32] = incl;
-  }
-  __syncthreads();
-  uint32_t r = tmp[warp] + x - v;
-  total = tmp[32];
-  __syncthreads();  // tmp may be reused by the next call
-  return r;
+// ---------------------------------------------------------------------------
+// exact k-th largest key
+// ---------------------------------------------------------------------------
+// Every pass below splits the current members -- the keys inside one
+// contiguous key interval, all keys at first -- into 256 bins by a bin
+// function that is monotone in the key, so the keys of one bin again form an
+// interval and equal keys share a bin.  The bin that holds the wanted rank
+// becomes the next members.  The first pass bins linearly in score value
+// (for the usual bell-shaped scores the wanted bin then holds a handful of
+// keys); later passes bin linearly in key space, which cuts the key range
+// about 256-fold per pass, so at most six more passes reach a single key.
+// Once 32 or fewer members remain, one warp ranks them exactly.  A pass costs
+// four block barriers and a fixed number of conflict-free shared-memory
+// reads per thread; no step depends on another thread's atomic result.
+struct RankSmem {
+  uint32_t hist[256];
+  uint32_t wmin[kSelThreads / 32], wmax[kSelThreads / 32], wsum[kSelThreads / 32];
+  uint32_t list[32];
+  uint32_t units[64];      // packed per-(round row, warp) counts in compaction
+  uint32_t bstar, rem, cnt, n_list, tau, need, carry;
+};
+
+__device__ __forceinline__ float key_to_score(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// The k-th largest key among keys[0, n) and how many keys equal to it are
-// kept.  Precondition: more than k of the keys are non-zero (valid), k >= 1.
-__device__ void radix_threshold(const uint32_t *keys, int n, int k, uint32_t *hist,
-                                uint32_t *bc, uint32_t &tau, int &need) {
+// the member set after a pass: keys in [lo, hi] whose bin is `b`
+struct Members {
+  bool all;          // no pass yet: every key
+  uint32_t lo, hi;
+  bool by_score;     // bins linear in score (else linear in key)
+  float base, inv;
+  uint32_t b;
+  __device__ __forceinline__ uint32_t bin(uint32_t u) const {
+    const float x = by_score ? (key_to_score(u) - base) * inv : (float)(u - lo) * inv;
+    return min(255u, __float2uint_rz(x));
+  }
+  __device__ __forceinline__ bool has(uint32_t u) const {
+    return all || (u >= lo && u <= hi && bin(u) == b);
+  }
+};
+
+// The k-th largest of keys[0, n) (tau) and how many keys equal to it are
+// kept (need); 1 <= k < n.
+__device__ void find_threshold(const uint32_t *keys, int n, int k, RankSmem &sm, uint32_t &tau,
+                               int &need) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0;
-  int rem = k;
+  constexpr int nw = kSelThreads / 32;
+  Members mem{};
+  mem.all = true;
+  uint32_t rem = (uint32_t)k, m = (uint32_t)n;
 #pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    // warp-aggregated: lanes holding the same digit add once (scores cluster
-    // in a few top-level bins, where plain atomics would serialise)
-    for (int base = warp * 32; base < n; base += kSelThreads) {
-      const int i = base + lane;
-      const uint32_t u = i < n ? keys[i] : 0u;
-      const bool match = i < n && (pass == 0 || ((u ^ prefix) >> (shift + 8)) == 0u);
-      const uint32_t bin = match ? ((u >> shift) & 255u) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-    }
-    __syncthreads();
-    if (warp == 0) {
-      uint32_t h[8], local = 0;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        h[b] = hist[lane * 8 + b];
-        local += h[b];
-      }
-      uint32_t suf = local;  // inclusive suffix sum over lanes
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += t;
-      }
-      uint32_t suf_next = __shfl_down_sync(0xffffffffu, suf, 1);
-      if (lane == 31) suf_next = 0;
-      if (suf >= (uint32_t)rem && suf_next < (uint32_t)rem) {
-        uint32_t above = suf_next;
-#pragma unroll
-        for (int b = 7; b >= 0; --b) {
-          if (above + h[b] >= (uint32_t)rem) {
-            bc[0] = (uint32_t)(lane * 8 + b);
-            bc[1] = (uint32_t)rem - above;
-            break;
-          }
-          above += h[b];
+  for (int pass = 0; pass < 12; ++pass) {
+    if (m <= 32u) {
+      // ---- exact rank of the last few members by one warp ----
+      if (tid == 0) sm.n_list = 0;
+      __syncthreads();
+      for (int e = tid; e < n; e += kSelThreads) {
+        const uint32_t u = keys[e];
+        if (mem.has(u)) {
+          const uint32_t slot = atomicAdd(&sm.n_list, 1u);
+          if (slot < 32u) sm.list[slot] = u;
         }
       }
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t cnt = min(sm.n_list, 32u);
+        const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
+        uint32_t gt = 0, ge = 0;
+        for (uint32_t j = 0; j < cnt; ++j) {
+          const uint32_t y = sm.list[j];
+          gt += y > x;
+          ge += y >= x;
+        }
+        if ((uint32_t)lane < cnt && gt < rem && ge >= rem) {
+          sm.tau = x;  // every lane holding this key writes the same values
+          sm.need = rem - gt;
+        }
+      }
+      __syncthreads();
+      tau = sm.tau;
+      need = (int)sm.need;
+      return;
+    }
+    // ---- key range of the members ----
+    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
+    for (int e = tid; e < n; e += kSelThreads) {
+      const uint32_t u = keys[e];
+      if (mem.has(u)) {
+        umin = min(umin, u);
+        umax = max(umax, u);
+      }
+    }
+    umin = __reduce_min_sync(0xffffffffu, umin);
+    umax = __reduce_max_sync(0xffffffffu, umax);
+    if (lane == 0) {
+      sm.wmin[warp] = umin;
+      sm.wmax[warp] = umax;
+    }
+    sm.hist[tid] = 0u;  // kSelThreads == 256 bins
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < nw; ++w) {
+      umin = min(umin, sm.wmin[w]);
+      umax = max(umax, sm.wmax[w]);
+    }
+    if (umin == umax) {  // the members are all one key
+      tau = umin;
+      need = (int)rem;
+      __syncthreads();  // wmin / wmax are rewritten by nobody after this
+      return;
+    }
+    // ---- bins over the members ----
+    Members nx{};
+    nx.all = false;
+    nx.lo = umin;
+    nx.hi = umax;
+    nx.by_score = false;
+    if (pass == 0) {
+      const float smin = key_to_score(umin), smax = key_to_score(umax);
+      const float inv = 256.0f / (smax - smin);
+      if (inv > 0.0f && inv < __int_as_float(0x7f800000)) {
+        nx.by_score = true;
+        nx.base = smin;
+        nx.inv = inv;
+      }
+    }
+    if (!nx.by_score) nx.inv = 256.0f / ((float)(umax - umin) + 1.0f);
+    for (int e = tid; e < n; e += kSelThreads) {
+      const uint32_t u = keys[e];
+      if (mem.has(u)) atomicAdd(&sm.hist[nx.bin(u)], 1u);
     }
     __syncthreads();
-    prefix |= bc[0] << shift;
-    rem = (int)bc[1];
+    // ---- the bin holding rank `rem` from the top: suffix sums over bins ----
+    const uint32_t h = sm.hist[tid];
+    uint32_t suf = h;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += t;
+    }
+    if (lane == 0) sm.wsum[warp] = suf;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < nw; ++w)
+      if (w > warp) suf += sm.wsum[w];
+    if (suf >= rem && suf - h < rem) {
+      sm.bstar = (uint32_t)tid;
+      sm.rem = rem - (suf - h);
+      sm.cnt = h;
+    }
+    __syncthreads();
+    nx.b = sm.bstar;
+    rem = sm.rem;
+    m = sm.cnt;
+    mem = nx;
   }
-  tau = prefix;
-  need = rem;
+  // not reached: the key range is a single key after at most seven passes
+  tau = 0xFFFFFFFFu;
+  need = 0;
 }
 
-// Keep keys > tau plus the first `need` keys == tau (in entry order), writing
-// them in entry order.  Each thread owns E consecutive entries.  Returns the
-// number kept (same value in every thread).
-template <class IdOf, class Out>
-__device__ int compact_kept(const uint32_t *keys, int n, int E, uint32_t tau, int need,
-                            uint32_t *scan_tmp, IdOf id_of, Out out) {
-  const int e0 = threadIdx.x * E;
-  const int e1 = min(n, e0 + E);
-  uint32_t packed = 0;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t u = keys[e];
-    packed += (u > tau ? 0x10000u : 0u) + (u == tau ? 1u : 0u);
-  }
-  uint32_t total;
-  const uint32_t before = block_exclusive_scan(packed, scan_tmp, total);
-  uint32_t gt_b = before >> 16, eq_b = before & 0xFFFFu;
-  for (int e = e0; e < e1; ++e) {
-    const uint32_t u = keys[e];
-    const bool gt = u > tau, eq = u == tau;
-    if (gt || (eq && (int)eq_b < need)) {
-      const uint32_t pos = gt_b + min(eq_b, (uint32_t)need);
-      out((int)pos, u, id_of(e));
+// Keep keys > tau plus the first `need` keys == tau (in entry order), in
+// entry order: out(pos, e) for each kept entry e, pos < limit.  Entries are
+// visited 32 consecutive ones per warp step; the position of each kept entry
+// comes from ballots inside the warp plus one block scan of per-warp counts
+// per round of 8 x 256 entries.  Returns the number kept.
+template <class Out>
+__device__ int compact_kept(const uint32_t *keys, int n, uint32_t tau, int need, int limit,
+                            RankSmem &sm, Out out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t carry = 0;  // packed (gt << 16 | eq) counts of earlier rounds
+#pragma unroll 1
+  for (int base = 0; base < n; base += 8 * kSelThreads) {
+    uint32_t bgt[8], beq[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = base + i * kSelThreads + tid;
+      const uint32_t u = e < n ? keys[e] : 0u;
+      bgt[i] = __ballot_sync(0xffffffffu, e < n && u > tau);
+      beq[i] = __ballot_sync(0xffffffffu, e < n && u == tau);
+      if (lane == 0) sm.units[i * 8 + warp] = ((uint32_t)__popc(bgt[i]) << 16) | (uint32_t)__popc(beq[i]);
     }
-    gt_b += gt;
-    eq_b += eq;
+    __syncthreads();
+    if (warp == 0) {  // exclusive scan of the 64 unit counts, two per lane
+      const uint32_t a0 = sm.units[2 * lane], a1 = sm.units[2 * lane + 1];
+      const uint32_t s = a0 + a1;
+      uint32_t x = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += t;
+      }
+      const uint32_t ex = carry + x - s;
+      sm.units[2 * lane] = ex;
+      sm.units[2 * lane + 1] = ex + a0;
+      if (lane == 31) sm.carry = carry + x;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t pre = sm.units[i * 8 + warp];
+      const uint32_t gt_b = (pre >> 16) + (uint32_t)__popc(bgt[i] & lt);
+      const uint32_t eq_b = (pre & 0xFFFFu) + (uint32_t)__popc(beq[i] & lt);
+      const bool gt = (bgt[i] >> lane) & 1u, eq = (beq[i] >> lane) & 1u;
+      if (gt || (eq && eq_b < (uint32_t)need)) {
+        const uint32_t pos = gt_b + min(eq_b, (uint32_t)need);
+        if (pos < (uint32_t)limit) out((int)pos, base + i * kSelThreads + tid);
+      }
+    }
+    carry = sm.carry;
+    __syncthreads();  // units / carry are rewritten by the next round
   }
-  return (int)((total >> 16) + min(total & 0xFFFFu, (uint32_t)need));
+  return min(limit, (int)((carry >> 16) + min(carry & 0xFFFFu, (uint32_t)need)));
 }
 
 // init | top-k | local | -1 padding.  With `fill_top`, the top-k part is the
@@ -222,25 +321,64 @@ __device__ __forceinline__ float dot8(const float *f, uint4 v) {
 }
 
 // Score candidate rows [lo, lo+n) of Kc for this problem into keys[0, n).
-// A half-warp scores 8 rows per step (8 x 16-byte loads in flight per lane).
-__device__ void score_rows(const uint16_t *kc_bg, const float *fs, int nf, int lo, int n,
-                           uint32_t *keys) {
-  constexpr int kRows = 8;
-  constexpr int kStep = (kSelThreads / 16) * kRows;  // rows per CTA step
+// The rows (contiguous, 256 B each) are streamed by the bulk-copy engine in
+// 128-row (32 KB) pieces through a kRing-deep shared-memory ring, so up to
+// 96 KB per CTA are in flight with no register cost; each half-warp scores 8
+// rows per piece from shared memory.  Returns false if a copy never landed
+// (bounded wait), in which case the keys are not valid.
+constexpr int kPieceRows = 128;
+constexpr int kPieceBytes = kPieceRows * kD * 2;
+constexpr int kRing = 3;
+
+__device__ __forceinline__ void issue_piece(const uint16_t *kc_bg, int lo, int n, int pc,
+                                            uint8_t *ring, uint64_t *bars) {
+  const int rows = min(kPieceRows, n - pc * kPieceRows);
+  uint64_t *bar = &bars[pc % kRing];
+  mbar_arrive_expect_tx(bar, (uint32_t)rows * kD * 2);
+  for (int r0 = 0; r0 < rows; r0 += 32)
+    bulk_g2s(ring + (pc % kRing) * kPieceBytes + r0 * kD * 2,
+             kc_bg + (long long)(lo + pc * kPieceRows + r0) * kD,
+             (uint32_t)min(32, rows - r0) * kD * 2, bar);
+}
+
+// thread 0, right after the barriers are initialised: the first pieces go
+// out before anything else is loaded
+__device__ __forceinline__ void prime_ring(const uint16_t *kc_bg, int lo, int n, uint8_t *ring,
+                                           uint64_t *bars) {
+  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
+  for (int pc = 0; pc < min(kRing, n_pc); ++pc) issue_piece(kc_bg, lo, n, pc, ring, bars);
+}
+
+__device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int lo, int n,
+                           uint32_t *keys, uint8_t *ring, uint64_t *bars) {
   const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
-  const uint16_t *base = kc_bg + hl * 8;
+  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
+  // the first pieces were issued by the caller's thread 0 right after the
+  // barriers were initialised (issue_first); the rest are refills
+  bool ok = true;
 #pragma unroll 1
-  for (int r0 = 0; r0 < n; r0 += kStep) {
-    const int row0 = r0 + hw * kRows;
-    uint4 v[kRows];
-#pragma unroll
-    for (int u = 0; u < kRows; ++u) {
-      const int e = row0 + u;
-      v[u] = e < n ? ldg_stream(base + (long long)(lo + e) * kD) : make_uint4(0, 0, 0, 0);
+  for (int pc = 0; pc < n_pc; ++pc) {
+    const bool landed = mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1));
+    if (__syncthreads_or(!landed)) {
+      ok = false;
+      // let copies still in flight land (bounded) before the ring is released
+      if (threadIdx.x == 0)
+        for (int q = pc; q < min(n_pc, pc + kRing); ++q)
+          (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
+      __syncthreads();
+      break;
     }
-    float part[kRows];
+    const int rows = min(kPieceRows, n - pc * kPieceRows);
+    const uint8_t *piece = ring + (pc % kRing) * kPieceBytes;
+    const int row0 = hw * 8;
+    uint4 v[8];
 #pragma unroll
-    for (int u = 0; u < kRows; ++u) part[u] = 0.f;
+    for (int u = 0; u < 8; ++u)
+      v[u] = row0 + u < rows ? *reinterpret_cast<const uint4 *>(piece + (row0 + u) * (kD * 2) + hl * 16)
+                             : make_uint4(0, 0, 0, 0);
+    float part[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) part[u] = 0.f;
 #pragma unroll 1
     for (int f = 0; f < nf; ++f) {
       float fv[8];
@@ -249,20 +387,25 @@ __device__ void score_rows(const uint16_t *kc_bg, const float *fs, int nf, int l
       fv[0] = a.x; fv[1] = a.y; fv[2] = a.z; fv[3] = a.w;
       fv[4] = b.x; fv[5] = b.y; fv[6] = b.z; fv[7] = b.w;
 #pragma unroll
-      for (int u = 0; u < kRows; ++u) part[u] += dot8(fv, v[u]);
+      for (int u = 0; u < 8; ++u) part[u] += dot8(fv, v[u]);
     }
-    const float s = transpose_reduce8x16(part, hl);
-    const int e = row0 + (hl >> 1);
-    if ((hl & 1) == 0 && e < n) keys[e] = orderable_key(s);
+    const float sc = transpose_reduce8x16(part, hl);
+    const int r = row0 + (hl >> 1);
+    if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
+    __syncthreads();  // piece consumed by every half-warp
+    if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
   }
+  return ok;
 }
 
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
-  extern __shared__ __align__(16) uint32_t dyn[];
-  __shared__ __align__(16) float fs[kMaxNf * kD];
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t bc[2];
-  __shared__ uint32_t scan_tmp[33];
+  // dynamic shared memory: piece ring | scoring vectors (fp32) | score keys
+  extern __shared__ __align__(128) uint8_t dyn_raw[];
+  uint8_t *ring = dyn_raw;
+  float *fs = reinterpret_cast<float *>(dyn_raw + kRing * kPieceBytes);
+  uint32_t *dyn = reinterpret_cast<uint32_t *>(dyn_raw + kRing * kPieceBytes + a.nf * kD * 4);
+  __shared__ __align__(8) uint64_t bars[kRing];
+  __shared__ RankSmem rs;
   __shared__ int s_last;
 
   // problems are laid out chunk-fastest so a problem's chunks run together
@@ -282,17 +425,26 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
     return;
   }
 
+  uint32_t *keys = dyn;
+  const int lo = bp.cand_lo + chunk * a.CH;
+  const int n = max(0, min(bp.cand_hi, lo + a.CH) - lo);
+  const uint16_t *kc_bg = a.kc + (b * a.G + g) * (long long)a.NB * kD;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
+    fence_mbar_init();
+    prime_ring(kc_bg, lo, n, ring, bars);
+  }
   // Forecast vector(s) of this problem -> fp32 in shared memory
   const uint16_t *f = a.F + (bi * a.G + g) * (long long)a.nf * kD;
   for (int t = threadIdx.x; t < a.nf * kD; t += kSelThreads)
     fs[t] = __uint_as_float(((uint32_t)f[t]) << 16);
   __syncthreads();
 
-  uint32_t *keys = dyn;
-  const int lo = bp.cand_lo + chunk * a.CH;
-  const int n = max(0, min(bp.cand_hi, lo + a.CH) - lo);
-  const uint16_t *kc_bg = a.kc + (b * a.G + g) * (long long)a.NB * kD;
-  score_rows(kc_bg, fs, a.nf, lo, n, keys);
+  if (!score_rows(kc_bg, fs, a.nf, lo, n, keys, ring, bars)) {
+    // a copy never landed: report an empty set rather than a wrong one
+    for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+    return;
+  }
   __syncthreads();
 
   uint32_t tau = 0;
@@ -300,10 +452,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   int32_t *top = out + bp.init_hi;
 
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
-    radix_threshold(keys, n, a.k, hist, bc, tau, need);
-    const int ntop = compact_kept(
-        keys, n, a.CH / kSelThreads, tau, need, scan_tmp, [&](int e) { return bp.cand_lo + e; },
-        [&](int pos, uint32_t, int id) { top[pos] = id; });
+    find_threshold(keys, n, a.k, rs, tau, need);
+    const int ntop = compact_kept(keys, n, tau, need, a.k, rs,
+                                  [&](int pos, int e) { top[pos] = bp.cand_lo + e; });
     write_set(out, bp, ntop, a.S, false);
     return;
   }
@@ -322,11 +473,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __threadfence();
   for (int e = threadIdx.x; e < ncand; e += kSelThreads) keys[e] = __ldcg(pkeys + e);
   __syncthreads();
-  radix_threshold(keys, ncand, a.k, hist, bc, tau, need);
-  const int E = (ncand + kSelThreads - 1) / kSelThreads;
-  const int ntop = compact_kept(
-      keys, ncand, E, tau, need, scan_tmp, [&](int e) { return bp.cand_lo + e; },
-      [&](int pos, uint32_t, int id) { top[pos] = id; });
+  find_threshold(keys, ncand, a.k, rs, tau, need);
+  const int ntop = compact_kept(keys, ncand, tau, need, a.k, rs,
+                                [&](int pos, int e) { top[pos] = bp.cand_lo + e; });
   write_set(out, bp, ntop, a.S, false);
   if (threadIdx.x == 0) a.counters[prob] = 0u;
 }
@@ -358,9 +507,9 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
   } else {
-    // short-lived streaming CTAs: about 512 blocks (128 KB of Kc) each, but
-    // one chunk per problem once there are plenty of problems (prefill)
-    CH = 512;
+    // streaming CTAs of 1024 blocks (256 KB of Kc) each, but one chunk per
+    // problem once there are plenty of problems (prefill)
+    CH = 1024;
     if (pl.n_problems >= 8LL * 148) CH = kMaxCand;
   }
   if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
@@ -403,21 +552,24 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.cap = pl.n_chunks * pl.CH;  // key slots per problem in the workspace
   a.counters = nullptr;
   a.cand_key = nullptr;
-  size_t smem = (size_t)pl.CH * 4;
+  size_t smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)pl.CH * 4;
   if (pl.n_chunks > 1) {
     char *w = static_cast<char *>(ws);
     a.counters = reinterpret_cast<uint32_t *>(w);
     w += ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
     a.cand_key = reinterpret_cast<uint32_t *>(w);
-    smem = (size_t)std::max(pl.CH, pl.ncand_max) * 4;
+    smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
-  if (smem > 48 * 1024) {  // raised once per device to the largest size used
+  {  // raised once per device to the largest size used; most shared memory
+     // goes to the ring, so prefer the largest carveout
     static size_t raised[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (raised[dev] < smem) {
       cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
       if (e != cudaSuccess) return e;
       raised[dev] = smem;
     }
