@@ -50,6 +50,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bound on the oracle's CPU-baseline sample")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run three passes of one decode layer (select, then attention) at "
+                         "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
+                         "K/V per attention launch) and exit: the small case that ncu captures")
     return ap.parse_args()
 
 
@@ -192,24 +196,24 @@ class DecodeLoop:
         torch.cuda.synchronize()
 
     # ---- resident: all K/V in HBM, addressed by block id ----
-    def step_resident(self, ev=None):
-        abi, w = self.abi, self.w
-        L = w.layers
-        bg = w.NB * self.blk_elems
-        for l in range(L):
-            nxt = (l + 1) % L
-            if ev is not None:
-                ev[l][0].record()
-            abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                       self.idx[nxt], self.ws_sel[l])
-            if ev is not None:
-                ev[l][1].record()
-            kv = self.kv[l]
-            abi.sparda_sparse_attn_decode(self.p, self.Q[l], kv, kv.view(-1)[w.blk * w.d:], bg,
-                                          self.blk_elems, self.idx[l], abi.SPARDA_ADDR_LOGICAL,
-                                          self.O[l], self.ws_att, self.status)
-            if ev is not None:
-                ev[l][2].record()
+    def select(self, l):
+        """Layer l's Forecast vector picks layer l+1's blocks."""
+        w, nxt = self.w, (l + 1) % self.w.layers
+        self.abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
+                                        self.idx[nxt], self.ws_sel[l])
+
+    def attention(self, l):
+        w = self.w
+        kv = self.kv[l]
+        self.abi.sparda_sparse_attn_decode(self.p, self.Q[l], kv, kv.view(-1)[w.blk * w.d:],
+                                           w.NB * self.blk_elems, self.blk_elems, self.idx[l],
+                                           self.abi.SPARDA_ADDR_LOGICAL, self.O[l], self.ws_att,
+                                           self.status)
+
+    def step_resident(self):
+        for l in range(self.w.layers):
+            self.select(l)
+            self.attention(l)
 
     # ---- host offload: K/V in pinned host memory, gathered into slots ----
     def _setup_host(self):
@@ -278,6 +282,40 @@ class DecodeLoop:
     def bytes_attn(self):
         w = self.w
         return w.B * w.G * w.S * self.blk_elems * 2 + 2 * w.B * w.Hq * w.d * 2 + w.B * w.G * w.S * 4
+
+
+PROFILE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
+KERNEL_SOURCES = {
+    "attn_tc_kernel": ["attn_decode.cu", "tc.cuh", "common.cuh"],
+}
+
+
+def kernel_source_hash(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_long_sparda_b200",
+                        "csrc")
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, algorithmic_bytes):
+    """DRAM bytes (read + write) per full launch from the committed ncu
+    summary of this kernel, or None when there is none or the kernel's
+    sources changed since it was taken."""
+    import re
+    for name in sorted(os.listdir(PROFILE_DIR)) if os.path.isdir(PROFILE_DIR) else []:
+        if not name.startswith(kernel):
+            continue
+        with open(os.path.join(PROFILE_DIR, name)) as f:
+            text = f.read()
+        m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", text)
+        m_tr = re.search(r"dram_bytes_per_full_launch:\s*([0-9]+)", text)
+        if m_hash and m_tr and m_hash.group(1) == kernel_source_hash(kernel):
+            return int(m_tr.group(1))
+    return None
 
 
 def time_steps(fn, steps, world):
@@ -387,27 +425,35 @@ def run_sparda(args):
         step()
     torch.cuda.synchronize()
     clk = clocks.stop()
-    # per-kernel durations inside a second timed pass on the same stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(L)]
-    sel_ms, att_ms = [], []
-    for _ in range(args.steps):
-        loop.step_resident(evs)
-        torch.cuda.synchronize()
+    # per-kernel durations: each kernel alone, back to back over the four
+    # layers on the same stream (as launched in the step), CUDA events around
+    # the whole run; events between kernels would break the programmatic
+    # overlap of consecutive launches
+    def kernel_loop(which):
         for l in range(L):
-            sel_ms.append(evs[l][0].elapsed_time(evs[l][1]))
-            att_ms.append(evs[l][1].elapsed_time(evs[l][2]))
+            if which == "select":
+                loop.select(l)
+            else:
+                loop.attention(l)
+    kern_us = {}
+    for which in ("select", "attention"):
+        for _ in range(3):
+            kernel_loop(which)
+        kms = time_steps(lambda: kernel_loop(which), args.steps, world)
+        kern_us[which] = kms / (args.steps * L) * 1e3
     st = int(loop.status.item())
 
     ms_step = ms / args.steps
     tokens = w.B * world
     value = tokens / (ms_step / 1e3)
     peak, peak_kind = measured_peaks()
-    att_us = statistics.mean(att_ms) * 1e3
-    sel_us = statistics.mean(sel_ms) * 1e3
+    att_us = kern_us["attention"]
+    sel_us = kern_us["select"]
     att_gbs = loop.bytes_attn() / (att_us * 1e-6) / 1e9
     sel_gbs = loop.bytes_select() / (sel_us * 1e-6) / 1e9
     layer_bytes = loop.bytes_attn() + loop.bytes_select()
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
+    traffic = profiled_traffic("attn_tc_kernel", loop.bytes_attn())
 
     e2e = None
     if want_e2e:
@@ -446,9 +492,9 @@ def run_sparda(args):
             "select_GBps": sel_gbs,
             "step_GBps": step_gbs,
             "step_hbm_frac": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "attn_decode_kernel", "achieved": att_gbs,
+            "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel", "achieved": att_gbs,
                          "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
-                         "traffic": None, "peak_kind": peak_kind,
+                         "traffic": traffic, "peak_kind": peak_kind,
                          "bytes_per_launch": loop.bytes_attn()},
             "clocks": clk,
             "e2e": e2e,
@@ -461,6 +507,27 @@ def run_sparda(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_profile_case():
+    """One decode layer at B=8, three passes: the small case for ncu."""
+    import torch
+    from block_sparse_long_sparda_b200 import abi
+    w = W.scaled(WORKLOAD, B=8, layers=2)
+    loop = DecodeLoop(w, with_host=False)
+    bg = w.NB * loop.blk_elems
+    kv = loop.kv[0]
+    for _ in range(3):
+        abi.sparda_forecast_select(loop.p, loop.F[0], 1, 1, w.T - 1, loop.kc[1], loop.idx[1],
+                                   loop.ws_sel[0])
+        abi.sparda_sparse_attn_decode(loop.p, loop.Q[0], kv, kv.view(-1)[w.blk * w.d:], bg,
+                                      loop.blk_elems, loop.idx[0], abi.SPARDA_ADDR_LOGICAL,
+                                      loop.O[0], loop.ws_att, loop.status)
+    torch.cuda.synchronize()
+    st = int(loop.status.item())
+    print("profile case: B=%d, %d select + %d attention launches, device status %d" % (w.B, 3, 3, st))
+    if st != 0:
+        sys.exit(1)
 
 
 def run_reference(args):
@@ -515,7 +582,11 @@ def run_reference(args):
 
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.profile_case:
+        from block_sparse_long_sparda_b200 import build
+        build.build()
+        run_profile_case()
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_sparda(args)

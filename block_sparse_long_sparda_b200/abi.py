@@ -27,6 +27,7 @@ SPARDA_EWORKSPACE = -6
 
 SPARDA_DEV_RANGE = 1
 SPARDA_DEV_TIMEOUT = 2
+SPARDA_DEV_LAYOUT = 4
 
 SPARDA_OP_COMPRESS = 0
 SPARDA_OP_SELECT = 1

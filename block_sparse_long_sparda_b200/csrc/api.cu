@@ -54,6 +54,7 @@ const char *sparda_status_string(int status) {
 }
 
 int sparda_status_from_device(int32_t word) {
+  if (word & SPARDA_DEV_LAYOUT) return SPARDA_ECUDA;
   if (word & SPARDA_DEV_TIMEOUT) return SPARDA_ETIMEOUT;
   if (word & SPARDA_DEV_RANGE) return SPARDA_ERANGE;
   return SPARDA_OK;

@@ -14,15 +14,19 @@
 // streams K/V at HBM speed instead of being bound by instruction issue:
 //  - stream-K: the (query, group) "pairs" and their list entries are
 //    flattened and cut into equal contiguous ranges, one per CTA, with a grid
-//    of two resident CTAs per SM -- one wave, no tail.  A range may start or
-//    end inside a pair; each piece of a pair is a "segment";
-//  - the entry list of a range is read by all threads at once and compacted
-//    with a block scan (one global-load latency per CTA);
+//    of as many CTAs as stay resident (three per SM with a two-stage ring,
+//    two with three stages) -- one wave.  A range may start or end inside a
+//    pair; each piece of a pair is a "segment";
+//  - launched as a programmatic dependent of the previous kernel: barriers
+//    and tensor maps are set up before waiting for it; the entry list of a
+//    range is then read by all threads at once and compacted with a block
+//    scan (one global-load latency per CTA);
 //  - TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) stages each
 //    block as [K lo-dims | V lo-dims | K hi-dims | V hi-dims] (8 KB each) in
-//    an NSTAGE ring, with the pair's query rows at the first block of a
-//    segment.  The M = 128 MMA for S^T reads rows 0-63 = the block's keys;
-//    its rows 64-127 alias the finite V tiles and are masked;
+//    an NSTAGE ring; the pair's query rows are loaded into the S^T issuer's
+//    registers one segment ahead.  The M = 128 MMA for S^T reads rows 0-63 =
+//    the block's keys; its rows 64-127 alias the V tiles and are never read
+//    back;
 //  - one thread issues the MMAs (N = 16: the group's heads, zero padded);
 //    softmax per head in the exp2 domain over the thread-per-key rows of
 //    S^T; P^T goes to shared memory as a bf16 K-major operand (the sum of
@@ -104,15 +108,31 @@ struct TcArgs {
   float scale_log2;
 };
 
-template <int R>
-struct TcCfg {
-  static constexpr int QB = R * kD * 2;  // raw query rows of one pair
-  static constexpr int QB_AL = (QB + 127) / 128 * 128;
-  // stages (1024-aligned) | Q^T operand | two P^T operands | raw query ring | slack
-  static size_t smem(int nstage) {
-    return (size_t)nstage * kUnitBytes + 4096 + 2 * 2048 + (size_t)nstage * QB_AL + 1024;
-  }
+// Everything else a CTA keeps in shared memory; it sits in the dynamic
+// allocation behind the operands, so the kernel has no static shared memory
+// and the allocation starts on the 1024-byte boundary the swizzled tiles need.
+template <int NSTAGE>
+struct TcCtl {
+  uint64_t full_bar[NSTAGE], empty_bar[NSTAGE];
+  uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
+  uint32_t tmem_base;
+  int s_last;
+  int s_abort;
+  int s_tmp[33];
+  int s_row[kMaxEnt];   // TMA row coordinate of the block
+  int s_rows[kMaxEnt];  // keys of the block at or before the query
+  int s_seg[kMaxEnt];   // segment (pair - pair0)
+  float red[2][kNQ];    // per-warp block maxima (softmax warps)
+  float corr_s[2][kNQ]; // rescale factor of a block (double buffer)
+  float seg_m[4][kNQ];  // running max at a segment's end (ring of 4)
+  float seg_l[4][2][kNQ];  // per-warp sums at a segment's end
 };
+
+// stages | Q^T operand (16 rows x 128 dims) | two P^T operands | control
+template <int NSTAGE>
+constexpr size_t tc_smem() {
+  return (size_t)NSTAGE * kUnitBytes + 4096 + 2 * 2048 + (sizeof(TcCtl<NSTAGE>) + 127) / 128 * 128;
+}
 
 constexpr int kWarps = 9;               // 4 correction, producer, 2 MMA issuers, 2 softmax warps
 constexpr int kWsThreads = kWarps * 32;
@@ -183,21 +203,44 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
     if (dim == 0) *s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
     named_sync(kBarCorr, 128);
     if (*s_last) {
+      // merge the pair's segments online, four heads at a time; a segment's
+      // loads for those heads are independent, so they are in flight together
       __threadfence();
       const long long base = pair * a.max_cover;
+      constexpr int HC = R < 4 ? R : 4;
 #pragma unroll 1
-      for (int h = 0; h < R; ++h) {
-        float M = -INFINITY;
-        for (int c = 0; c < n_cover; ++c) M = fmaxf(M, __ldcg(&a.ws_ml[(base + c) * R + h].x));
-        float L = 0.f, o = 0.f;
-        for (int c = 0; c < n_cover; ++c) {
-          const float2 ml = __ldcg(&a.ws_ml[(base + c) * R + h]);
-          const float fw = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-          L += fw * ml.y;
-          o += fw * __ldcg(&a.ws_o[((base + c) * R + h) * kD + dim]);
+      for (int h0 = 0; h0 < R; h0 += HC) {
+        float M[HC], L[HC], o[HC];
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          M[h] = -INFINITY;
+          L[h] = 0.f;
+          o[h] = 0.f;
         }
-        const float r = L > 0.f ? o / L : 0.f;
-        a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+#pragma unroll 1
+        for (int c = 0; c < n_cover; ++c) {
+          float2 ml[HC];
+          float ov[HC];
+#pragma unroll
+          for (int h = 0; h < HC; ++h) {
+            ml[h] = __ldcg(&a.ws_ml[(base + c) * R + h0 + h]);
+            ov[h] = __ldcg(&a.ws_o[((base + c) * R + h0 + h) * kD + dim]);
+          }
+#pragma unroll
+          for (int h = 0; h < HC; ++h) {
+            if (ml[h].x == -INFINITY) continue;  // a segment with no keys
+            const float mn = fmaxf(M[h], ml[h].x);
+            const float f_old = exp2f(M[h] - mn), f_new = exp2f(ml[h].x - mn);
+            L[h] = L[h] * f_old + ml[h].y * f_new;
+            o[h] = o[h] * f_old + ov[h] * f_new;
+            M[h] = mn;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < HC; ++h) {
+          const float r = L[h] > 0.f ? o[h] / L[h] : 0.f;
+          a.O[(pair * R + h0 + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+        }
       }
       if (dim == 0) a.counters[pair] = 0u;
     }
@@ -205,48 +248,77 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
   named_sync(kBarCorr, 128);
 }
 
+// Two stages per CTA with three CTAs per SM keep as many blocks in flight as
+// three stages with two CTAs, but give each SM three independent chains of
+// (S^T, softmax, O^T): a stage is held from its landing until its O^T MMA is
+// done, and more chains hide that hold better.  Sixteen heads per group need
+// more registers than three CTAs per SM allow.
 template <int R, int NSTAGE>
-__global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_constant__ CUtensorMap mapK,
-                                                             const __grid_constant__ CUtensorMap mapV,
-                                                             TcArgs a) {
-  using C = TcCfg<R>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+__global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                   TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
   uint8_t *stages = sm;                          // NSTAGE x 32 KB
   uint8_t *qop = sm + NSTAGE * kUnitBytes;       // Q^T operand: 16 rows x 128 dims
   uint8_t *pop = qop + 4096;                     // two P^T operands: 16 rows x 64 keys
-  uint8_t *qraw = pop + 2 * 2048;                // NSTAGE raw query slots
-  __shared__ __align__(8) uint64_t full_bar[NSTAGE], empty_bar[NSTAGE];
-  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
-  __shared__ uint32_t tmem_base;
-  __shared__ int s_row[kMaxEnt];   // TMA row coordinate of the block
-  __shared__ int s_rows[kMaxEnt];  // keys of the block at or before the query
-  __shared__ int s_seg[kMaxEnt];   // segment (pair - pair0)
-  __shared__ int s_tmp[33];
-  __shared__ int s_last;
-  __shared__ volatile int s_abort;
-  __shared__ float red[2][kNQ];            // per-warp block maxima (softmax warps)
-  __shared__ float corr_s[2][kNQ];         // rescale factor of a block (double buffer)
-  __shared__ float seg_m[4][kNQ];          // running max at a segment's end (ring of 4)
-  __shared__ float seg_l[4][2][kNQ];       // per-warp sums at a segment's end
+  TcCtl<NSTAGE> &ctl = *reinterpret_cast<TcCtl<NSTAGE> *>(pop + 2 * 2048);
+  uint64_t *full_bar = ctl.full_bar, *empty_bar = ctl.empty_bar;
+  uint64_t *s_full = ctl.s_full, *p_full = ctl.p_full, *o_full = ctl.o_full, *o_free = ctl.o_free;
+  int *s_row = ctl.s_row, *s_rows = ctl.s_rows, *s_seg = ctl.s_seg;
+  volatile int *s_abort = &ctl.s_abort;
+  float(*red)[kNQ] = ctl.red;
+  float(*corr_s)[kNQ] = ctl.corr_s;
+  float(*seg_m)[kNQ] = ctl.seg_m;
+  float(*seg_l)[2][kNQ] = ctl.seg_l;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long E = a.n_entries, NC = gridDim.x;
   const long long e0 = (long long)blockIdx.x * E / NC;
   const long long e1 = (long long)(blockIdx.x + 1) * E / NC;
+  pdl_trigger();
   if (e0 >= e1) return;
+  if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles would be misread
+    pdl_wait();
+    if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
+    return;
+  }
   const long long pair0 = e0 / a.S;
   const int n_seg = (int)((e1 - 1) / a.S - pair0 + 1);
+
+  // barriers, TMEM and the zeroed operands are set up while the block list
+  // is being loaded
+  if (tid == 0) {
+    for (int st = 0; st < NSTAGE; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 64);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_free[b], 128);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+    tc::prefetch_map(&mapK);
+    tc::prefetch_map(&mapV);
+  }
+  pdl_wait();
+  const long long e_me = e0 + tid;
+  const int j_me = (tid < kMaxEnt && e_me < e1) ? a.idx[e_me] : -1;
+  if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 64);
+  for (int i = tid; i < (4096 + 4096) / 16; i += kWsThreads)  // Q^T, P^T rows >= R stay zero
+    reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
 
   // ---- the range's valid entries, in order (at most kMaxEnt) ----
   int row_ = 0, rows_ = 0, seg_ = 0, cnt = 0;
   {
-    const long long e = e0 + tid;
+    const long long e = e_me;
     if (tid < kMaxEnt && e < e1) {
       const long long pair = e / a.S;
       const int s = (int)(e - pair * a.S);
-      const int j = a.idx[e];
+      const int j = j_me;
       if (j >= 0) {
         const int pos = a.q_start + (int)((pair / a.G) % a.nq);
         if (j >= a.NB || j > pos / kBlk) {
@@ -263,36 +335,17 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
     }
   }
   int nb;
-  const int off = block_excl_scan<kWsThreads>(cnt, s_tmp, nb);
+  const int off = block_excl_scan<kWsThreads>(cnt, ctl.s_tmp, nb);
   if (cnt) {
     s_row[off] = row_;
     s_rows[off] = rows_;
     s_seg[off] = seg_;
   }
-  if (tid == 0) {
-    for (int st = 0; st < NSTAGE; ++st) {
-      mbar_init(&full_bar[st], 1);
-      mbar_init(&empty_bar[st], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 64);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_free[b], 128);
-    }
-    s_abort = 0;
-    fence_mbar_init();
-    tc::prefetch_map(&mapK);
-    tc::prefetch_map(&mapV);
-  }
-  if (warp == 0) tc::tmem_alloc(&tmem_base, 64);
-  for (int i = tid; i < (4096 + 4096) / 16; i += kWsThreads)  // Q^T, P^T rows >= R stay zero
-    reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = tmem_base;  // S0 | S1 | O0 | O1, 16 columns each
+  const uint32_t tmem = ctl.tmem_base;  // S0 | S1 | O0 | O1, 16 columns each
   auto first_of = [&](int u) { return u == 0 || s_seg[u - 1] != s_seg[u]; };
   auto last_of = [&](int u) { return u == nb - 1 || s_seg[u + 1] != s_seg[u]; };
 
@@ -305,18 +358,15 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
       for (int u = 0; u < nb; ++u) {
         const int st = u % NSTAGE;
         if (u >= NSTAGE &&
-            !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), &s_abort))
+            !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), s_abort))
           break;
-        const bool first = first_of(u);
         uint8_t *dst = stages + st * kUnitBytes;
         const int row = s_row[u];
-        mbar_arrive_expect_tx(&full_bar[st], kUnitBytes + (first ? C::QB : 0));
+        mbar_arrive_expect_tx(&full_bar[st], kUnitBytes);
         tc::tma_load_2d(dst, &mapK, 0, row, &full_bar[st]);
         tc::tma_load_2d(dst + kTile, &mapV, 0, row, &full_bar[st]);
         tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
         tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &full_bar[st]);
-        if (first)
-          bulk_g2s(qraw + st * C::QB_AL, a.Q + (pair0 + s_seg[u]) * R * kD, C::QB, &full_bar[st]);
         produced = u + 1;
       }
     }
@@ -324,25 +374,41 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
     // ================= S^T issuer =================
     // S^T(u) as soon as its block has landed and the softmax of u-2 is done
     // with S[u & 1].
+    // The query rows of the next segment are loaded into registers one
+    // segment ahead, so their global-load latency overlaps the current one.
     constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
     const uint64_t dK = tc::sdesc(stages, 16, 1024);
     const uint64_t dQ = tc::sdesc(qop, 16, 1024);
+    constexpr int QV = (R * 16 + 31) / 32;  // 16-byte pieces of the query rows per lane
+    uint4 qn[QV];
+    auto load_q = [&](int seg) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(a.Q + (pair0 + seg) * R * kD);
+#pragma unroll
+      for (int j = 0; j < QV; ++j) {
+        const int i = lane + 32 * j;
+        qn[j] = i < R * 16 ? ldg_stream(src + i) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    if (nb > 0) load_q(s_seg[0]);
     bool ok = true;
 #pragma unroll 1
     for (int u = 0; u < nb && ok; ++u) {
       const int st = u % NSTAGE;
-      ok = wait_or_abort(&full_bar[st], (uint32_t)((u / NSTAGE) & 1), &s_abort);
-      if (ok && u >= 2) ok = wait_or_abort(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1), &s_abort);
+      ok = wait_or_abort(&full_bar[st], (uint32_t)((u / NSTAGE) & 1), s_abort);
+      if (ok && u >= 2) ok = wait_or_abort(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1), s_abort);
       const bool first = first_of(u);
       if (ok && first && u >= 1)  // the previous S^T must be done with the old query
-        ok = wait_or_abort(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1), &s_abort);
+        ok = wait_or_abort(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1), s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       if (first) {
-        const uint4 *q = reinterpret_cast<const uint4 *>(qraw + st * C::QB_AL);
-        for (int i = lane; i < R * 16; i += 32) {
-          const int h = i >> 4, c8 = i & 15;
-          *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = q[i];
+#pragma unroll
+        for (int j = 0; j < QV; ++j) {
+          const int i = lane + 32 * j;
+          if (i < R * 16) {
+            const int h = i >> 4, c8 = i & 15;
+            *reinterpret_cast<uint4 *>(qop + (c8 >> 3) * 2048 + tc::sw128_offset(h, (c8 & 7) * 8)) = qn[j];
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -357,8 +423,13 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
         tc::mma_commit(&s_full[u & 1]);
       }
       __syncwarp();
+      if (first) {  // the next segment's query rows, off the critical path
+        int u2 = u + 1;
+        while (u2 < nb && s_seg[u2] == s_seg[u]) ++u2;
+        if (u2 < nb) load_q(s_seg[u2]);
+      }
     }
-    if (!ok) s_abort = 1;
+    if (!ok) *s_abort = 1;
   } else if (warp == kWarpMma2) {
     // ================= O^T issuer =================
     // O^T(v) as soon as the softmax of v is done and the correction of v-2 has
@@ -371,8 +442,8 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
 #pragma unroll 1
     for (int v = 0; v < nb && ok; ++v) {
       const int st = v % NSTAGE;
-      ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
-      if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), &s_abort);
+      ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
+      if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       if (lane == 0) {
@@ -388,7 +459,7 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
       }
       __syncwarp();
     }
-    if (!ok) s_abort = 1;
+    if (!ok) *s_abort = 1;
   } else if (warp == 4 || warp == 5) {
     // ================= softmax (thread = key of the block) =================
     const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
@@ -407,9 +478,9 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
           l_t[h] = 0.f;
         }
       }
-      if (ok) ok = wait_or_abort(&s_full[b], (uint32_t)((u >> 1) & 1), &s_abort);
+      if (ok) ok = wait_or_abort(&s_full[b], (uint32_t)((u >> 1) & 1), s_abort);
       // block u-2 is fully corrected: its P^T and corr slots are free
-      if (ok && u >= 2) ok = wait_or_abort(&o_free[b], (uint32_t)(((u - 2) >> 1) & 1), &s_abort);
+      if (ok && u >= 2) ok = wait_or_abort(&o_free[b], (uint32_t)(((u - 2) >> 1) & 1), s_abort);
       tc::fence_after_sync();
       float x[R];
       {
@@ -443,14 +514,18 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
         *reinterpret_cast<__nv_bfloat16 *>(pb + tc::sw128_offset(h, key)) = pv;
         l_t[h] = l_t[h] * cr[h] + __bfloat162float(pv);
       }
-      if (key < R) corr_s[b][key] = cr[key];
+#pragma unroll
+      for (int h = 0; h < R; ++h)  // unrolled: no dynamic register index
+        if (key == h) corr_s[b][h] = cr[h];
       if (last_of(u)) {  // publish the segment's statistics
 #pragma unroll
         for (int h = 0; h < R; ++h) {
           const float ls = warp_sum_xor(l_t[h], 1, 32);
           if (lane == 0) seg_l[smx_k & 3][warp - 4][h] = ls;
         }
-        if (key < R) seg_m[smx_k & 3][key] = m_run[key];
+#pragma unroll
+        for (int h = 0; h < R; ++h)
+          if (key == h) seg_m[smx_k & 3][h] = m_run[h];
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
@@ -458,7 +533,7 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
       // both softmax warps finish the block before either reuses red[]
       named_sync(kBarSoftmax, 64);
     }
-    if (!ok) s_abort = 1;
+    if (!ok) *s_abort = 1;
   } else {
     // ============ correction (warps 0, 1, 6, 7; thread = output dim) ============
     const int q = warp & 3;  // TMEM lane quadrant
@@ -482,15 +557,15 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
         }
         for (int f = next_flush; f < seg; ++f)
           seg_flush<R>(a, pair0 + f, f == cur, E, NC, acc, seg_m[live_k & 3],
-                       &seg_l[live_k & 3][0][0], &s_last, dim);
+                       &seg_l[live_k & 3][0][0], &ctl.s_last, dim);
         next_flush = seg;
         cur = seg;
         ++live_k;
 #pragma unroll
         for (int h = 0; h < R; ++h) acc[h] = 0.f;
       }
-      if (ok) ok = wait_or_abort(&o_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
-      if (ok) ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), &s_abort);
+      if (ok) ok = wait_or_abort(&o_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
+      if (ok) ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
       // one vote for all four warps, so they always leave at the same barrier
       if (named_sync_or(kBarCorr, 128, !ok)) {
         ok = false;
@@ -509,12 +584,12 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
     if (ok)
       for (int f = next_flush; f < n_seg; ++f)
         seg_flush<R>(a, pair0 + f, f == cur, E, NC, acc, seg_m[live_k & 3], &seg_l[live_k & 3][0][0],
-                     &s_last, dim);
-    if (!ok) s_abort = 1;
+                     &ctl.s_last, dim);
+    if (!ok) *s_abort = 1;
   }
 
   __syncthreads();
-  if (s_abort) {
+  if (*s_abort) {
     // something never completed: give what was issued a bounded chance to
     // land before the CTA's memory is released; the status word says why
     flag_status(a.status, SPARDA_DEV_TIMEOUT);
@@ -532,7 +607,7 @@ __global__ void __launch_bounds__(kWsThreads) attn_tc_kernel(const __grid_consta
 template <int R, int NSTAGE>
 cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs &a,
                       long long grid_max, long long grid_min, cudaStream_t stream) {
-  const size_t smem = TcCfg<R>::smem(NSTAGE);
+  constexpr size_t smem = tc_smem<NSTAGE>();
   auto kern = attn_tc_kernel<R, NSTAGE>;
   // per device, once: shared-memory attributes and how many CTAs stay
   // resident (one wave: as many CTAs as the device keeps resident, never
@@ -547,16 +622,24 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     // resident CTAs per SM from the shared-memory budget (each CTA also
-    // holds its static shared memory and the per-block reservation)
-    int n_sm = 148, per_sm = 0, reserved = 0;
+    // holds its static shared memory and the per-block reservation) and
+    // from the register file (allocated per warp in 256-register units)
+    int n_sm = 148, per_sm = 0, reserved = 0, regs_sm = 65536;
     (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     (void)cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     (void)cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    (void)cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
     cudaFuncAttributes fa;
     size_t stat = 4096;
-    if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess) stat = fa.sharedSizeBytes;
+    int regs = 128;
+    if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess) {
+      stat = fa.sharedSizeBytes;
+      regs = fa.numRegs;
+    }
     (void)cudaGetLastError();
     int occ = per_sm > 0 ? (int)((size_t)per_sm / (smem + stat + (size_t)reserved)) : 1;
+    const int warp_regs = (regs * 32 + 255) / 256 * 256;
+    occ = std::min(occ, regs_sm / (warp_regs * kWarps));
     occ = std::max(1, std::min(occ, 3));
     resident[dev] = occ * n_sm;
   }
@@ -565,8 +648,8 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
   if (forced > 0) grid = forced;
   grid = std::max(grid, grid_min);
   grid = std::min(grid, grid_max);
-  kern<<<(unsigned)grid, kWsThreads, smem, stream>>>(mk, mv, a);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kWsThreads, smem, stream, mk, mv, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -641,15 +724,15 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.ws_ml = reinterpret_cast<float2 *>(w);
   w += ((parts * 8) + 255) & ~(size_t)255;
   a.counters = reinterpret_cast<uint32_t *>(w);
-  // ring depth: 3 x 32 KB with two resident CTAs per SM measured best; 4 and
-  // 6 (one CTA per SM, 5 when 16 heads share a group) stay selectable
-  // through SPARDA_DECODE_STAGES for sweeps
+  // ring depth: 2 x 32 KB with three resident CTAs per SM where the
+  // registers allow it (up to 8 heads per group), else 3 x 32 KB with two;
+  // 4 and 6 (one CTA per SM) stay selectable through SPARDA_DECODE_STAGES
   int stages = env_int("SPARDA_DECODE_STAGES");
-  if (stages == 0) stages = 3;
+  if (stages == 0) stages = R <= 8 ? 2 : 3;
 #define SPARDA_LAUNCH_R(RR)                                                             \
-  if (stages <= 3) return launch_tc<RR, 3>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages <= 2) return launch_tc<RR, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages == 3) return launch_tc<RR, 3>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
   if (stages == 4) return launch_tc<RR, 4>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (RR >= 16) return launch_tc<RR, 5>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
   return launch_tc<RR, 6>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
   switch (R) {
     case 1: SPARDA_LAUNCH_R(1)

@@ -47,6 +47,15 @@ __device__ __forceinline__ void stg_stream(void *p, uint4 v) {
                : "memory");
 }
 
+// Programmatic dependent launch.  The select and attention kernels are
+// launched so that their CTAs may become resident while the kernel before
+// them on the stream is still finishing; pdl_wait() returns once that kernel
+// has completed and its writes are visible, and every such kernel calls it
+// before its first access to global memory.  pdl_trigger() lets the next
+// kernel's CTAs be placed as soon as every CTA of this one is running.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void flag_status(int32_t *status, int bits) {
   if (status) atomicOr(status, bits);
 }

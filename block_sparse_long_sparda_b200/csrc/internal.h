@@ -9,6 +9,25 @@
 
 namespace sparda {
 
+// Launch a kernel that may start before the previous kernel on the stream
+// has finished (programmatic stream serialization); the kernel itself waits
+// for that kernel (pdl_wait) before it touches global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // The three parts of a query's block set (eq. B_l(i) of the pages):
 // initial [0, init_hi), candidates [cand_lo, cand_hi), local [local_lo, c].
 struct BlockParts {

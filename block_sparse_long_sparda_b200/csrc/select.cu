@@ -408,6 +408,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __shared__ RankSmem rs;
   __shared__ int s_last;
 
+  pdl_trigger();
+  pdl_wait();
   // problems are laid out chunk-fastest so a problem's chunks run together
   // and its merge overlaps the streaming of later problems
   const long long prob = blockIdx.x / a.n_chunks;
@@ -575,8 +577,8 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     }
   }
   const long long grid = pl.n_problems * pl.n_chunks;
-  select_kernel<<<(unsigned)grid, kSelThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(select_kernel, (unsigned)grid, kSelThreads, smem, stream, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sparda

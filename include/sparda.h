@@ -38,7 +38,9 @@
  *  - dev_status (optional, device int32): kernels OR device-side findings
  *    into it (SPARDA_DEV_RANGE: a block id outside [0, NB) or after the
  *    query's own block was skipped; SPARDA_DEV_TIMEOUT: a bounded wait gave
- *    up).  The caller zeroes it, reads it after synchronizing, and may turn
+ *    up; SPARDA_DEV_LAYOUT: a kernel found its shared memory placed off the
+ *    1024-byte boundary its swizzled tiles need and wrote nothing).  The
+ *    caller zeroes it, reads it after synchronizing, and may turn
  *    it into a status with sparda_status_from_device().
  */
 #ifndef SPARDA_H_
@@ -66,7 +68,8 @@ enum sparda_status {
 
 enum sparda_device_status_bits {
   SPARDA_DEV_RANGE = 1,
-  SPARDA_DEV_TIMEOUT = 2
+  SPARDA_DEV_TIMEOUT = 2,
+  SPARDA_DEV_LAYOUT = 4
 };
 
 /* Shapes shared by every call.  T is the number of tokens present in the

@@ -32,6 +32,7 @@ def test_status_strings_and_device_word(L):
     assert abi.sparda_status_from_device(0) == abi.SPARDA_OK
     assert abi.sparda_status_from_device(abi.SPARDA_DEV_RANGE) == abi.SPARDA_ERANGE
     assert abi.sparda_status_from_device(abi.SPARDA_DEV_TIMEOUT | abi.SPARDA_DEV_RANGE) == abi.SPARDA_ETIMEOUT
+    assert abi.sparda_status_from_device(abi.SPARDA_DEV_LAYOUT) == abi.SPARDA_ECUDA
     assert abi.sparda_version() >= 100
 
 
