@@ -50,6 +50,14 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bound on the oracle's CPU-baseline sample")
+    ap.add_argument("--prefill", action="store_true",
+                    help="also measure the prefill chunk workload (B=4, T=128K, 2048 query "
+                         "tokens): compress, per-token select and sparse attention; prints "
+                         "an extra JSON line")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also measure the selection-only sweep (Kc blocks 128..16384 x "
+                         "batch 1..16, Forecast vs the 4-head baseline selector); prints an "
+                         "extra JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
@@ -291,13 +299,19 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel):
+    """Hash of the kernel's sources with comments and blank space removed, so
+    that an edit of comments alone does not retire a profile."""
     import hashlib
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_long_sparda_b200",
                         "csrc")
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
@@ -462,12 +476,15 @@ def run_sparda(args):
         e_steps = max(3, min(args.steps, 10))
         e_ms = time_steps(loop.step_e2e, e_steps, world) / e_steps
         fetched = w.B * w.G * w.k * loop.blk_elems * 2 * L
+        link_peak = host_link_peak_gbps()
         e2e = {"value": w.B * world / (e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(loop.Q.numel() * 2 + loop.F.numel() * 2),
                "d2h_bytes_per_step": int(loop.O.numel() * 2),
                "ms_per_step": e_ms,
                "host_link_bytes_per_step": fetched,
                "host_link_GBps": fetched / (e_ms * 1e-3) / 1e9,
+               "host_link_peak_GBps": link_peak,
+               "host_link_frac": fetched / (e_ms * 1e-3) / 1e9 / link_peak,
                "note": "K/V in pinned host memory; every layer's top-k blocks gathered over the "
                        "host link on a side stream (cold sets, no reuse across steps)"}
         loop.unregister()
@@ -504,9 +521,131 @@ def run_sparda(args):
             "device_status": st,
         }
         print(json.dumps(line), flush=True)
+    if rank == 0 and world == 1 and args.prefill:
+        print(json.dumps(run_prefill(args.steps)), flush=True)
+    if rank == 0 and world == 1 and args.sweep:
+        print(json.dumps(run_sweep()), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def host_link_peak_gbps(nbytes=1 << 30, reps=5):
+    """Pinned host -> device copy bandwidth (one large cudaMemcpyAsync, best
+    of a few): the link peak the host gather is compared with."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del src, dst
+    return best
+
+
+def time_back_to_back(fn, steps, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps * 1e3      # us per call
+
+
+def run_prefill(steps):
+    """Prefill chunk: B=4 sequences of T=131072 tokens, the last 2048 tokens
+    are the queries (positions T-2048 .. T-1), per-token Forecast vectors."""
+    import torch
+    from block_sparse_long_sparda_b200 import abi
+    w = W.WORKLOADS["prefill_b4_t128k_c2k"]
+    dev = torch.device("cuda")
+    B, G, Hq, d, T, nq, NB, S = w.B, w.G, w.Hq, w.d, w.T, w.nq, w.NB, w.S
+    p = abi.make_params(B, Hq, G, T, w.k, w.n_init, w.n_local)
+    K = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+    V = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+    W.torch_normal_bf16_(K, w.seed * 16)
+    W.torch_normal_bf16_(V, w.seed * 16 + 1)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed * 16 + 2)
+    Q = torch.randn(B, nq, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+    F = torch.randn(B, nq, G, d, generator=gen, device=dev).to(torch.bfloat16)
+    kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(B, nq, G, S, dtype=torch.int32, device=dev)
+    O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_sel = abi.workspace(abi.SPARDA_OP_SELECT, p, nq, 1)
+    ws_att = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq, 1)
+    q0 = T - nq
+    compress = lambda: abi.sparda_compress_keys(p, K, T * d, d, None, kc)
+    select = lambda: abi.sparda_forecast_select(p, F, nq, 1, q0, kc, idx, ws_sel)
+    attn = lambda: abi.sparda_sparse_attn_prefill(p, Q, nq, q0, K, V, T * d, d, idx, O, ws_att,
+                                                  status)
+    n = max(3, min(steps, 10))
+    c_us = time_back_to_back(compress, n)
+    s_us = time_back_to_back(select, n)
+    a_us = time_back_to_back(attn, n)
+    st = int(status.item())
+    ncand = sum(max(0, (q0 + i) // w.blk - w.n_local + 1 - w.n_init) for i in range(nq))
+    sel_flop = 2.0 * B * G * d * ncand
+    keys = sum(min(w.k, max(0, (q0 + i) // w.blk - w.n_local + 1 - w.n_init)) * w.blk
+               + w.n_init * w.blk + (w.n_local - 1) * w.blk + ((q0 + i) % w.blk) + 1
+               for i in range(nq))
+    att_flop = 4.0 * B * Hq * d * keys
+    return {
+        "metric": "prefill chunk: compress, per-token Forecast select, sparse attention (us)",
+        "workload": w.name, "B": B, "T": T, "nq": nq, "Hq": Hq, "G": G, "k": w.k,
+        "compress_us": c_us, "compress_GBps": B * G * T * d * 2 / (c_us * 1e-6) / 1e9,
+        "select_us": s_us, "select_TFLOPs": sel_flop / (s_us * 1e-6) / 1e12,
+        "attn_us": a_us, "attn_useful_TFLOPs": att_flop / (a_us * 1e-6) / 1e12,
+        "attn_gathered_GBps": B * nq * G * S * 2 * w.blk * d * 2 / (a_us * 1e-6) / 1e9,
+        "chunk_us": s_us + a_us, "tokens_per_s": B * nq / ((s_us + a_us) * 1e-6),
+        "device_status": st, "data": "synthetic", "dtype": "bf16",
+    }
+
+
+def run_sweep():
+    """Selection-only sweep: Forecast (one vector per group) next to the
+    baseline selector (the group's 4 query heads, scores summed) on the same
+    compressed keys."""
+    import torch
+    from block_sparse_long_sparda_b200 import abi
+    dev = torch.device("cuda")
+    G, Hq, d, k = 8, 32, 128, 64
+    points = []
+    for NB in W.SWEEP_NB:
+        for B in W.SWEEP_B:
+            T = NB * 64
+            p = abi.make_params(B, Hq, G, T, k)
+            kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
+            W.torch_normal_bf16_(kc, W.SWEEP_SEED * 1000 + NB + B)
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(W.SWEEP_SEED + NB * 64 + B)
+            F = torch.randn(B, G, d, generator=gen, device=dev).to(torch.bfloat16)
+            Qh = torch.randn(B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+            idx = torch.empty(B, G, k + 3, dtype=torch.int32, device=dev)
+            ws1 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1)
+            ws4 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, Hq // G)
+            f_us = time_back_to_back(
+                lambda: abi.sparda_forecast_select(p, F, 1, 1, T - 1, kc, idx, ws1), 20)
+            b_us = time_back_to_back(
+                lambda: abi.sparda_forecast_select(p, Qh, 1, Hq // G, T - 1, kc, idx, ws4), 20)
+            nbytes = B * G * NB * d * 2
+            points.append({"NB": NB, "B": B, "forecast_us": round(f_us, 2),
+                           "baseline_us": round(b_us, 2),
+                           "forecast_GBps": round(nbytes / (f_us * 1e-6) / 1e9, 1)})
+            del kc
+    return {"metric": "selection-only sweep: Forecast vs 4-head baseline selector (us per call)",
+            "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16"}
 
 
 def run_profile_case():

@@ -1,6 +1,10 @@
 // attn_decode.cu -- GQA block-sparse attention of single query tokens over
 // their own block lists (decode; also the per-token prefill path).
 //
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
 // [p4 "The fourth projection", Eq. 5 / Algorithm 2]: O_l = attention(Q_l,
 // K_l[B_l], V_l[B_l]): each query head attends over the keys of its GQA
 // group's selected blocks only; fp32 softmax, fp32 accumulation.

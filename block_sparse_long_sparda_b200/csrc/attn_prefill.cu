@@ -1,6 +1,10 @@
 // attn_prefill.cu -- block-sparse prefill attention: every token of a query
 // chunk attends over the keys of its own block set, causal.
 //
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
 // [p4 "The fourth projection", Algorithm 1 / Eq. 5]: O_l = attention(Q_l,
 // K_l[B_l], V_l[B_l]) with every key resident on the GPU.
 //

@@ -1,5 +1,9 @@
 // compress.cu -- mean-pooled compressed keys (one per block of 64 tokens).
 //
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
 // [p1 "架构细节"]: the top-k part of a layer's block set is scored against the
 // block-mean of that layer's keys; [p4 "The problem InfLLM-V2 leaves on the
 // table"]: keys are mean-pooled into one compressed key per block.

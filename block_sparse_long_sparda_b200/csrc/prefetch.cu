@@ -1,6 +1,10 @@
 // prefetch.cu -- gather the selected K/V blocks of the next layer from pinned
 // host memory into device slots, on the caller's (side) stream.
 //
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
 // [p4 "The fourth projection", Algorithm 2]: the blocks picked for layer l+1
 // are fetched from CPU pinned memory to the GPU on a dedicated prefetch
 // stream while layer l computes; [p1 "UVA异步预取管线"]: the kernel reads

@@ -2,6 +2,10 @@
 // compressed key with the group's Forecast vector(s), keep the k best, and
 // join them with the initial and local blocks.
 //
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
 // [p4 "The fourth projection", Eq. 4]: B_{l+1} = B_init U B_local U
 //   f_top(F_l Kc_{l+1}^T, k)
 // [p4 "One Forecast head per GQA group"]: one Forecast vector per group, raw

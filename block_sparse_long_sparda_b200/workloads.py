@@ -9,8 +9,10 @@ fp32 (numpy PCG64, or torch's Philox generator for the multi-GB host KV of the
 decode loop) and rounded to bf16 to nearest, ties to even.
 
 The shapes stand in for the pages' own workloads (8B block-sparse models at
-128K context, batch 4 prefill and batch 16+ decode; p4 "Three speedups, three
-different baselines"), which use trained weights we do not have: every tensor
+128K context, batch 4 prefill and batch 16+ decode; the article "SparDA: a
+fourth projection that lets sparse attention prefetch its own KV cache",
+section "Three speedups, three different baselines"), which use trained
+weights we do not have: every tensor
 here is N(0, 1) noise with the structure the workload names (planted hot
 blocks for the recall case).
 """

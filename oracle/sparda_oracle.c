@@ -17,7 +17,7 @@
  * exact values of the bf16 inputs (a bf16 is decoded exactly into a double).
  * There is no blocking, fusion or reordering beyond what the definition says.
  *
- * Readings of points the pages leave open (all also listed in the design doc):
+ * Readings of points the pages leave open:
  *  - block j holds token positions [j*blk, (j+1)*blk); the last block of a
  *    sequence whose length is not a multiple of blk holds fewer tokens and its
  *    compressed key is the mean over the tokens it holds;
