@@ -86,23 +86,39 @@ def init_dist(world, local):
                                 device_id=torch.device("cuda", local))
 
 
+def _on_gpu():
+    import torch
+    return torch.cuda.is_available()
+
+
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest value of x over all ranks (timings: the slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def barrier(world):
     import torch
-    torch.cuda.synchronize()
+    if _on_gpu():
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if _on_gpu():
+        torch.cuda.synchronize()
+
+
+def replica_value(tokens_per_replica: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job decode throughput of `world` independent replicas: every
+    replica decodes its own batch, so the job's tokens per step are the sum
+    over replicas, and the step takes as long as the slowest replica."""
+    return tokens_per_replica * world / (ms_per_step_max / 1e3)
 
 
 class ClockSampler:
@@ -458,8 +474,7 @@ def run_sparda(args):
     st = int(loop.status.item())
 
     ms_step = ms / args.steps
-    tokens = w.B * world
-    value = tokens / (ms_step / 1e3)
+    value = replica_value(w.B, world, ms_step)
     peak, peak_kind = measured_peaks()
     att_us = kern_us["attention"]
     sel_us = kern_us["select"]
