@@ -577,53 +577,79 @@ def time_back_to_back(fn, steps, warm=3):
     return e0.elapsed_time(e1) / steps * 1e3      # us per call
 
 
+class PrefillChunk:
+    """Prefill chunk: B=4 sequences of T=131072 tokens whose last 2048 tokens
+    are the queries (positions T-2048 .. T-1), one Forecast vector per token
+    and group, K/V [B][G][T][128] in HBM."""
+
+    def __init__(self, w: W.Workload = None):
+        import torch
+        from block_sparse_long_sparda_b200 import abi
+        self.torch, self.abi = torch, abi
+        w = w or W.WORKLOADS["prefill_b4_t128k_c2k"]
+        self.w = w
+        dev = torch.device("cuda")
+        B, G, Hq, d, T, nq, NB, S = w.B, w.G, w.Hq, w.d, w.T, w.nq, w.NB, w.S
+        self.p = abi.make_params(B, Hq, G, T, w.k, w.n_init, w.n_local)
+        self.K = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+        self.V = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+        W.torch_normal_bf16_(self.K, w.seed * 16)
+        W.torch_normal_bf16_(self.V, w.seed * 16 + 1)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed * 16 + 2)
+        self.Q = torch.randn(B, nq, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+        self.F = torch.randn(B, nq, G, d, generator=gen, device=dev).to(torch.bfloat16)
+        self.kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
+        self.idx = torch.empty(B, nq, G, S, dtype=torch.int32, device=dev)
+        self.O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws_sel = abi.workspace(abi.SPARDA_OP_SELECT, self.p, nq, 1)
+        self.ws_att = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, self.p, nq, 1)
+        self.q0 = T - nq
+
+    def compress(self):
+        w = self.w
+        self.abi.sparda_compress_keys(self.p, self.K, w.T * w.d, w.d, None, self.kc)
+
+    def select(self):
+        self.abi.sparda_forecast_select(self.p, self.F, self.w.nq, 1, self.q0, self.kc, self.idx,
+                                        self.ws_sel)
+
+    def attention(self):
+        w = self.w
+        self.abi.sparda_sparse_attn_prefill(self.p, self.Q, w.nq, self.q0, self.K, self.V,
+                                            w.T * w.d, w.d, self.idx, self.O, self.ws_att,
+                                            self.status)
+
+    def flops(self):
+        """(select FLOPs, useful attention FLOPs) of one chunk."""
+        w = self.w
+        ncand = keys = 0
+        for i in range(w.nq):
+            pos = self.q0 + i
+            nc = max(0, pos // w.blk - w.n_local + 1 - w.n_init)
+            ncand += nc
+            keys += (min(w.k, nc) + w.n_init + w.n_local - 1) * w.blk + pos % w.blk + 1
+        return 2.0 * w.B * w.G * w.d * ncand, 4.0 * w.B * w.Hq * w.d * keys
+
+
 def run_prefill(steps):
-    """Prefill chunk: B=4 sequences of T=131072 tokens, the last 2048 tokens
-    are the queries (positions T-2048 .. T-1), per-token Forecast vectors."""
-    import torch
-    from block_sparse_long_sparda_b200 import abi
-    w = W.WORKLOADS["prefill_b4_t128k_c2k"]
-    dev = torch.device("cuda")
-    B, G, Hq, d, T, nq, NB, S = w.B, w.G, w.Hq, w.d, w.T, w.nq, w.NB, w.S
-    p = abi.make_params(B, Hq, G, T, w.k, w.n_init, w.n_local)
-    K = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
-    V = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
-    W.torch_normal_bf16_(K, w.seed * 16)
-    W.torch_normal_bf16_(V, w.seed * 16 + 1)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(w.seed * 16 + 2)
-    Q = torch.randn(B, nq, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
-    F = torch.randn(B, nq, G, d, generator=gen, device=dev).to(torch.bfloat16)
-    kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
-    idx = torch.empty(B, nq, G, S, dtype=torch.int32, device=dev)
-    O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws_sel = abi.workspace(abi.SPARDA_OP_SELECT, p, nq, 1)
-    ws_att = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq, 1)
-    q0 = T - nq
-    compress = lambda: abi.sparda_compress_keys(p, K, T * d, d, None, kc)
-    select = lambda: abi.sparda_forecast_select(p, F, nq, 1, q0, kc, idx, ws_sel)
-    attn = lambda: abi.sparda_sparse_attn_prefill(p, Q, nq, q0, K, V, T * d, d, idx, O, ws_att,
-                                                  status)
+    pc = PrefillChunk()
+    w = pc.w
     n = max(3, min(steps, 10))
-    c_us = time_back_to_back(compress, n)
-    s_us = time_back_to_back(select, n)
-    a_us = time_back_to_back(attn, n)
-    st = int(status.item())
-    ncand = sum(max(0, (q0 + i) // w.blk - w.n_local + 1 - w.n_init) for i in range(nq))
-    sel_flop = 2.0 * B * G * d * ncand
-    keys = sum(min(w.k, max(0, (q0 + i) // w.blk - w.n_local + 1 - w.n_init)) * w.blk
-               + w.n_init * w.blk + (w.n_local - 1) * w.blk + ((q0 + i) % w.blk) + 1
-               for i in range(nq))
-    att_flop = 4.0 * B * Hq * d * keys
+    c_us = time_back_to_back(pc.compress, n)
+    s_us = time_back_to_back(pc.select, n)
+    a_us = time_back_to_back(pc.attention, n)
+    st = int(pc.status.item())
+    sel_flop, att_flop = pc.flops()
     return {
         "metric": "prefill chunk: compress, per-token Forecast select, sparse attention (us)",
-        "workload": w.name, "B": B, "T": T, "nq": nq, "Hq": Hq, "G": G, "k": w.k,
-        "compress_us": c_us, "compress_GBps": B * G * T * d * 2 / (c_us * 1e-6) / 1e9,
+        "workload": w.name, "B": w.B, "T": w.T, "nq": w.nq, "Hq": w.Hq, "G": w.G, "k": w.k,
+        "compress_us": c_us, "compress_GBps": w.B * w.G * w.T * w.d * 2 / (c_us * 1e-6) / 1e9,
         "select_us": s_us, "select_TFLOPs": sel_flop / (s_us * 1e-6) / 1e12,
         "attn_us": a_us, "attn_useful_TFLOPs": att_flop / (a_us * 1e-6) / 1e12,
-        "attn_gathered_GBps": B * nq * G * S * 2 * w.blk * d * 2 / (a_us * 1e-6) / 1e9,
-        "chunk_us": s_us + a_us, "tokens_per_s": B * nq / ((s_us + a_us) * 1e-6),
+        "attn_gathered_GBps": w.B * w.nq * w.G * w.S * 2 * w.blk * w.d * 2 / (a_us * 1e-6) / 1e9,
+        "chunk_us": s_us + a_us, "tokens_per_s": w.B * w.nq / ((s_us + a_us) * 1e-6),
         "device_status": st, "data": "synthetic", "dtype": "bf16",
     }
 

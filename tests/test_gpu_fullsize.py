@@ -1,0 +1,121 @@
+"""Parity at the benchmark's full sizes, in the launch configuration it times.
+
+The decode loop (B=16, T=131072, 4 layers, 34 GB of K/V in HBM) and the
+prefill chunk (B=4, T=131072, 2048 query tokens) run exactly as bench.py
+runs them -- the same classes, kernels, grids and workspaces.  The oracle
+then recomputes a sample of outputs one by one on the host:
+
+- the compressed keys of the sampled (sequence, group) pairs;
+- their block sets (same bf16 Kc bytes in, the band rule for near-ties);
+- their attention outputs, over the block set the GPU used, so attention
+  parity does not depend on the selection.
+"""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_sparda_b200 import abi, build
+from tests.parity import check_attention, check_sets, host_bits, scores_f64
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    abi.lib()
+    torch.cuda.init()
+
+
+def _check_kc_bits(gpu_bits, ora_bits, what):
+    same = np.mean(gpu_bits == ora_bits)
+    diff = np.abs(gpu_bits.astype(np.int32) - ora_bits.astype(np.int32)).max()
+    assert same >= 0.999 and diff <= 1, "%s: bf16 Kc identical %.5f, max diff %d ulp" % (what, same, diff)
+
+
+def test_decode_loop_full_size_sampled():
+    import bench
+    w = bench.WORKLOAD
+    loop = bench.DecodeLoop(w, with_host=False)
+    loop.step_resident()  # select(l -> l+1) then attention(l), for the four layers
+    torch.cuda.synchronize()
+    assert int(loop.status.item()) == 0
+    L, R, d, blk, NB, T = w.layers, w.r, w.d, w.blk, w.NB, w.T
+    rng = np.random.default_rng(2024)
+    for l in range(L):
+        picks = {(0, 0), (w.B - 1, w.G - 1)}
+        while len(picks) < 3:
+            picks.add((int(rng.integers(w.B)), int(rng.integers(w.G))))
+        for b, g in sorted(picks):
+            what = "layer %d b %d g %d" % (l, b, g)
+            kv = host_bits(loop.kv[l, b, g])                    # [NB][2][64][128]
+            # compressed keys: each block's 64 K rows pooled, as the bench pools them
+            _, ora_kc = oracle.compress_keys(kv, blk, shape=(1, NB, blk, d),
+                                             strides=(2 * blk * d, d))
+            gpu_kc = host_bits(loop.kc[l, b, g])
+            _check_kc_bits(gpu_kc, ora_kc.reshape(NB, d), what)
+            # the set attention(l) used came from F_{l-1} scoring Kc_l
+            F = host_bits(loop.F[(l - 1) % L, b, g]).reshape(1, 1, 1, 1, d)
+            kc_in = gpu_kc.reshape(1, 1, NB, d)
+            ora_idx, kth, kth1 = oracle.select(F, kc_in, w.k, w.n_init, w.n_local, T - 1, blk)
+            gpu_idx = loop.idx[l, b, g].cpu().numpy().reshape(1, 1, 1, -1)
+            check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what)
+            # attention of the group's heads over the GPU's set
+            Q = host_bits(loop.Q[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+            flat = kv.reshape(-1)
+            ora_o = oracle.sparse_attention(Q, flat, flat[blk * d:], gpu_idx, T - 1, T, blk,
+                                            bg_stride=flat.size, blk_stride=2 * blk * d, G=1)
+            gpu_o = host_bits(loop.O[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+            check_attention(gpu_o, ora_o, what)
+    del loop
+    torch.cuda.empty_cache()
+
+
+def test_prefill_chunk_full_size_sampled():
+    import bench
+    pc = bench.PrefillChunk()
+    w = pc.w
+    pc.compress()
+    pc.select()
+    pc.attention()
+    torch.cuda.synchronize()
+    assert int(pc.status.item()) == 0
+    R, d, blk, NB, T, q0 = w.r, w.d, w.blk, w.NB, w.T, pc.q0
+    rng = np.random.default_rng(2025)
+    # the first and last query tokens, the two sides of a block boundary, and
+    # random ones
+    first_of_block = (64 - q0 % 64) % 64 or 64
+    tokens = {0, w.nq - 1, first_of_block - 1, first_of_block}
+    picks = set()
+    for i in tokens:
+        picks.add((int(rng.integers(w.B)), i, int(rng.integers(w.G))))
+    while len(picks) < 7:
+        picks.add((int(rng.integers(w.B)), int(rng.integers(w.nq)), int(rng.integers(w.G))))
+    kc_cache = {}
+    for b, i, g in sorted(picks):
+        what = "b %d token %d g %d" % (b, i, g)
+        K = host_bits(pc.K[b, g]).reshape(1, 1, T, d)
+        V = host_bits(pc.V[b, g]).reshape(1, 1, T, d)
+        if (b, g) not in kc_cache:
+            _, ora_kc = oracle.compress_keys(K, blk)
+            gpu_kc = host_bits(pc.kc[b, g])
+            _check_kc_bits(gpu_kc, ora_kc.reshape(NB, d), "b %d g %d" % (b, g))
+            kc_cache[(b, g)] = gpu_kc.reshape(1, 1, NB, d)
+        kc_in = kc_cache[(b, g)]
+        F = host_bits(pc.F[b, i, g]).reshape(1, 1, 1, 1, d)
+        ora_idx, kth, kth1 = oracle.select(F, kc_in, w.k, w.n_init, w.n_local, q0 + i, blk)
+        gpu_idx = pc.idx[b, i, g].cpu().numpy().reshape(1, 1, 1, -1)
+        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what)
+        Q = host_bits(pc.Q[b, i, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+        ora_o = oracle.sparse_attention(Q, K, V, gpu_idx, q0 + i, T, blk)
+        gpu_o = host_bits(pc.O[b, i, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+        check_attention(gpu_o, ora_o, what)
+    del pc
+    torch.cuda.empty_cache()
