@@ -57,9 +57,16 @@ struct SelectPlan {
   int CH;                // candidate blocks scored per thread block
   int n_chunks;          // thread blocks per problem
   int kc;                // candidates kept per chunk: min(k, CH)
+  int tensor_scores;     // 1: chunk of query tokens scored by the tcgen05 product
   size_t ws_bytes;
 };
 SelectPlan plan_select(const sparda_params &p, int nq, int nf);
+// prefill (select_prefill.cu): scores of a token chunk on the tensor cores,
+// then one warp per (token, group) row ranks them
+constexpr int kPrefillTensorMinQ = 64;  // query tokens from which the product pays
+size_t prefill_select_ws_bytes(const sparda_params &p, int nq);
+cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
+                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream);
 int select_supported(const SelectPlan &plan);
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const uint16_t *F,
                           int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,

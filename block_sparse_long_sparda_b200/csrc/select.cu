@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "rank.cuh"
 
 namespace sparda {
 
@@ -76,26 +77,6 @@ struct RankSmem {
   uint32_t list[32];
   uint32_t units[64];      // packed per-(round row, warp) counts in compaction
   uint32_t bstar, rem, cnt, n_list, tau, need, carry;
-};
-
-__device__ __forceinline__ float key_to_score(uint32_t u) {
-  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
-}
-
-// the member set after a pass: keys in [lo, hi] whose bin is `b`
-struct Members {
-  bool all;          // no pass yet: every key
-  uint32_t lo, hi;
-  bool by_score;     // bins linear in score (else linear in key)
-  float base, inv;
-  uint32_t b;
-  __device__ __forceinline__ uint32_t bin(uint32_t u) const {
-    const float x = by_score ? (key_to_score(u) - base) * inv : (float)(u - lo) * inv;
-    return min(255u, __float2uint_rz(x));
-  }
-  __device__ __forceinline__ bool has(uint32_t u) const {
-    return all || (u >= lo && u <= hi && bin(u) == b);
-  }
 };
 
 // The k-th largest of keys[0, n) (tau) and how many keys equal to it are
@@ -169,21 +150,7 @@ __device__ void find_threshold(const uint32_t *keys, int n, int k, RankSmem &sm,
       return;
     }
     // ---- bins over the members ----
-    Members nx{};
-    nx.all = false;
-    nx.lo = umin;
-    nx.hi = umax;
-    nx.by_score = false;
-    if (pass == 0) {
-      const float smin = key_to_score(umin), smax = key_to_score(umax);
-      const float inv = 256.0f / (smax - smin);
-      if (inv > 0.0f && inv < __int_as_float(0x7f800000)) {
-        nx.by_score = true;
-        nx.base = smin;
-        nx.inv = inv;
-      }
-    }
-    if (!nx.by_score) nx.inv = 256.0f / ((float)(umax - umin) + 1.0f);
+    const Members nx = make_bins(pass, umin, umax);
     for (int e = tid; e < n; e += kSelThreads) {
       const uint32_t u = keys[e];
       if (mem.has(u)) atomicAdd(&sm.hist[nx.bin(u)], 1u);
@@ -208,10 +175,10 @@ __device__ void find_threshold(const uint32_t *keys, int n, int k, RankSmem &sm,
       sm.cnt = h;
     }
     __syncthreads();
-    nx.b = sm.bstar;
+    mem = nx;
+    mem.b = sm.bstar;
     rem = sm.rem;
     m = sm.cnt;
-    mem = nx;
   }
   // not reached: the key range is a single key after at most seven passes
   tau = 0xFFFFFFFFu;
@@ -497,7 +464,6 @@ int env_int(const char *name) {
 // the workspace size is known before the call: chunking is sized for a query
 // at the end of the sequence, the most candidates any query can have.
 SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
-  (void)nf;
   SelectPlan pl{};
   pl.n_problems = (long long)p.B * nq * p.G;
   const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
@@ -505,8 +471,16 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
   pl.CH = kSelThreads;
   pl.n_chunks = 1;
   pl.kc = 0;
+  pl.tensor_scores = 0;
   pl.ws_bytes = 0;
   if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
+  if (nf == 1 && nq >= kPrefillTensorMinQ && env_int("SPARDA_SELECT_STREAM") == 0) {
+    // a chunk of query tokens: the scores are a dense product per (sequence,
+    // group), computed on the tensor cores and kept in the workspace
+    pl.tensor_scores = 1;
+    pl.ws_bytes = prefill_select_ws_bytes(p, nq);
+    return pl;
+  }
 
   const int forced = env_int("SPARDA_SELECT_CHUNK");
   int CH;
@@ -531,6 +505,7 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
 }
 
 int select_supported(const SelectPlan &pl) {
+  if (pl.tensor_scores) return 1;
   if (pl.CH > kMaxCand) return 0;
   if (pl.ncand_max > kMaxCand) return 0;
   return 1;
@@ -540,6 +515,7 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
                           int nf, int q_start, const uint16_t *kc, int32_t *idx, void *ws,
                           cudaStream_t stream) {
   if (pl.n_problems == 0) return cudaSuccess;
+  if (pl.tensor_scores) return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, stream);
   SelArgs a;
   a.F = F;
   a.kc = kc;

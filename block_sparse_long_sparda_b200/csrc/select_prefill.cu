@@ -1,0 +1,535 @@
+// select_prefill.cu -- Forecast block selection for a chunk of query tokens
+// (prefill): every token of the chunk scores every candidate block of its
+// sequence with its own Forecast vector and keeps the k best.
+//
+// Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
+// lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
+// [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
+//
+// [p4 "The fourth projection", Algorithm 1]: B_l = B_init U B_local U
+//   top_k(F_prev @ K_compressed[l].T, k), per query token, each token with
+//   its own causal candidate range;
+// [p4 "One Forecast head per GQA group"]: one Forecast vector per group, raw
+//   dot products, no softmax.
+//
+// Design (B200).  For one (sequence, group) the scores of a chunk are a
+// dense product S = F_chunk Kc^T: 2048 tokens x 2048 blocks x 128 dims, 34
+// GFLOP over the 4 x 8 pairs of the benchmark chunk.  That is a tensor-core
+// contraction, so it runs in two kernels:
+//  1. prefill_scores_kernel -- one CTA per (pair, 128-token tile, 256-block
+//     tile): TMA loads the F tile (4-D map: dims, group, token, sequence) and
+//     the Kc tile (3-D map: dims, block, pair), one thread issues eight
+//     tcgen05 MMAs (M = 128 tokens, N = 256 blocks, K = 16 each) into TMEM,
+//     and the four warps read the 128 x 256 fp32 scores back (thread = token
+//     row), turn them into orderable keys -- 0 outside the token's candidate
+//     range -- and store them to the workspace, [pair][token][block].  Tiles
+//     lying wholly after every row's candidates are skipped.
+//  2. rank_rows_kernel -- one warp per (sequence, token, group) row: the same
+//     exact search as the decode selection (a score-linear then key-linear
+//     256-bin passes, an exact rank of the last few candidates), done by one
+//     warp with a per-warp histogram in shared memory, then a ballot pass in
+//     block order that keeps every key above the k-th plus the lowest-index
+//     ties, and the set init U top-k U local written in ascending order.
+// Every wait is bounded; a timeout sets SPARDA_DEV_TIMEOUT, frees TMEM and
+// leaves the tile's keys unwritten.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "rank.cuh"
+#include "tc.cuh"
+
+namespace sparda {
+
+namespace {
+
+constexpr int kPTok = 128;      // token rows per score tile (MMA M)
+constexpr int kPBlk = 256;      // block columns per score tile (MMA N)
+constexpr int kPThreads = 128;  // four warps: TMEM lanes 0-127, thread = token row
+constexpr int kPSmem = 32768 + 65536 + 1024;  // F tile | Kc tile | barriers
+constexpr int kRWarps = 8;      // rows ranked per CTA (one warp each)
+
+struct PScoreArgs {
+  uint32_t *keys;      // [B*G][nq][ld]
+  int32_t *status;
+  int G, nq, NB, ld, q_start, n_init, n_local;
+};
+
+__global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
+    const __grid_constant__ CUtensorMap mapF, const __grid_constant__ CUtensorMap mapKc,
+    PScoreArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t *opA = smem;            // [2 dim halves][128 tokens][64 dims], 32 KB
+  uint8_t *opB = smem + 32768;    // [2 dim halves][256 blocks][64 dims], 64 KB
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 32768 + 65536);  // tma, mma
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int u = blockIdx.x, t = blockIdx.y, pair = blockIdx.z;
+  const int b = pair / a.G, g = pair % a.G;
+  const int i0 = t * kPTok;
+  const int j0 = u * kPBlk;
+  // the candidates of the tile's last row reach furthest
+  const int i_last = min(a.nq, i0 + kPTok) - 1;
+  const BlockParts bp_last = block_parts(a.q_start + i_last, kBlk, a.n_init, a.n_local);
+  pdl_trigger();
+  if (j0 >= bp_last.cand_hi || j0 + kPBlk <= a.n_init) return;  // no candidate in the tile
+  if (smem_addr(smem) & 1023u) {
+    pdl_wait();
+    if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+    tc::prefetch_map(&mapF);
+    tc::prefetch_map(&mapKc);
+  }
+  if (warp == 0) tc::tmem_alloc(tmem_slot, 256);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  bool ok = true;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars[0], 32768 + 65536);
+    tc::tma_load_4d(opA, &mapF, 0, g, i0, b, &bars[0]);
+    tc::tma_load_4d(opA + 16384, &mapF, 64, g, i0, b, &bars[0]);
+    tc::tma_load_3d(opB, &mapKc, 0, j0, pair, &bars[0]);
+    tc::tma_load_3d(opB + 32768, &mapKc, 64, j0, pair, &bars[0]);
+    ok = mbar_wait_bounded(&bars[0], 0);
+    if (ok) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(kPTok, kPBlk, false, false);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        tc::mma_bf16(tmem, tc::sdesc(opA + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                     tc::sdesc(opB + (k >> 2) * 32768 + (k & 3) * 32, 16, 1024), id, k > 0);
+      tc::mma_commit(&bars[1]);
+    }
+  }
+  const bool tma_ok = __syncthreads_and(ok);
+  if (tma_ok) ok = mbar_wait_bounded(&bars[1], 0);
+  ok = __syncthreads_and(ok);
+  if (!ok) {
+    if (tid == 0) {
+      flag_status(a.status, SPARDA_DEV_TIMEOUT);
+      // give copies still in flight a bounded chance to land before the
+      // shared memory is released
+      if (!tma_ok) (void)mbar_wait_bounded(&bars[0], 0);
+    }
+  } else {
+    tc::fence_after_sync();
+    const int i = i0 + tid;  // this thread's token row (TMEM lane tid)
+    const BlockParts bp = block_parts(a.q_start + min(i, a.nq - 1), kBlk, a.n_init, a.n_local);
+    uint32_t *row = a.keys + ((long long)pair * a.nq + i) * a.ld + j0;
+    const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+    for (int c = 0; c < kPBlk; c += 16) {
+      float v[16];
+      tc::tmem_ld16(tmem + lane_sel + c, v);  // warp-wide: every lane takes part
+      if (i < a.nq && j0 + c < a.ld) {
+        uint32_t kk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = j0 + c + e;
+          kk[e] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(v[e]) : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          reinterpret_cast<uint4 *>(row + c)[q] = make_uint4(kk[4 * q], kk[4 * q + 1], kk[4 * q + 2], kk[4 * q + 3]);
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// warp-level exact top-k of one row
+// ---------------------------------------------------------------------------
+struct WarpRankSmem {
+  uint32_t hist[256];
+  uint32_t list[32];
+};
+
+// the keys were written by the previous kernel: read-only for this one
+__device__ __forceinline__ uint32_t ld_key(const uint32_t *p) { return __ldg(p); }
+
+// The k-th largest of keys[0, n) and how many keys equal to it are kept;
+// 1 <= k < n; one warp, no block barrier.
+__device__ void warp_threshold(const uint32_t *keys, int n, int k, WarpRankSmem &sm,
+                               uint32_t &tau, int &need) {
+  const int lane = threadIdx.x & 31;
+  Members mem{};
+  mem.all = true;
+  uint32_t rem = (uint32_t)k, m = (uint32_t)n;
+#pragma unroll 1
+  for (int pass = 0; pass < 12; ++pass) {
+    if (m <= 32u) {
+      // ---- exact rank of the last few members ----
+      uint32_t cnt = 0;
+#pragma unroll 1
+      for (int base = 0; base < n; base += 32) {
+        const int e = base + lane;
+        const uint32_t u = e < n ? ld_key(keys + e) : 0u;
+        const bool in = e < n && mem.has(u);
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        const uint32_t slot = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (in && slot < 32u) sm.list[slot] = u;
+        cnt += __popc(bal);
+      }
+      __syncwarp();
+      cnt = min(cnt, 32u);
+      const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
+      uint32_t gt = 0, ge = 0;
+      for (uint32_t j = 0; j < cnt; ++j) {
+        const uint32_t y = sm.list[j];
+        gt += y > x;
+        ge += y >= x;
+      }
+      const bool hit = (uint32_t)lane < cnt && gt < rem && ge >= rem;
+      const uint32_t who = __ballot_sync(0xffffffffu, hit);
+      const int src = who ? __ffs(who) - 1 : 0;
+      tau = __shfl_sync(0xffffffffu, x, src);
+      need = (int)(rem - __shfl_sync(0xffffffffu, gt, src));
+      __syncwarp();
+      return;
+    }
+    // ---- key range of the members ----
+    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
+#pragma unroll 4
+    for (int e = lane; e < n; e += 32) {
+      const uint32_t u = ld_key(keys + e);
+      if (mem.has(u)) {
+        umin = min(umin, u);
+        umax = max(umax, u);
+      }
+    }
+    umin = __reduce_min_sync(0xffffffffu, umin);
+    umax = __reduce_max_sync(0xffffffffu, umax);
+    if (umin == umax) {
+      tau = umin;
+      need = (int)rem;
+      return;
+    }
+    // ---- histogram over the next bins ----
+    const Members nx = make_bins(pass, umin, umax);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sm.hist[lane * 8 + q] = 0u;
+    __syncwarp();
+#pragma unroll 4
+    for (int e = lane; e < n; e += 32) {
+      const uint32_t u = ld_key(keys + e);
+      if (mem.has(u)) atomicAdd(&sm.hist[nx.bin(u)], 1u);
+    }
+    __syncwarp();
+    // ---- the bin holding rank `rem` from the top ----
+    uint32_t h[8], local = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      h[q] = sm.hist[lane * 8 + q];
+      local += h[q];
+    }
+    uint32_t above = local;  // inclusive suffix over lanes, then exclusive
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
+      if (lane + o < 32) above += v;
+    }
+    above -= local;  // keys in bins of higher lanes
+    int bsel = -1;
+    uint32_t rsel = 0, csel = 0;
+#pragma unroll
+    for (int q = 7; q >= 0; --q) {
+      if (bsel < 0 && above + h[q] >= rem && above < rem) {
+        bsel = lane * 8 + q;
+        rsel = rem - above;
+        csel = h[q];
+      }
+      above += h[q];
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, bsel >= 0);
+    const int src = who ? __ffs(who) - 1 : 0;
+    mem = nx;
+    mem.b = (uint32_t)__shfl_sync(0xffffffffu, bsel, src);
+    rem = __shfl_sync(0xffffffffu, rsel, src);
+    m = __shfl_sync(0xffffffffu, csel, src);
+    __syncwarp();
+  }
+  tau = 0xFFFFFFFFu;  // not reached: the range is a single key within seven passes
+  need = 0;
+}
+
+// The same search with the row held in registers: entry e = 32*m + lane is
+// kv[m] (0 past the row's end; a valid key is never 0).  Rows of up to
+// 32 * KPL candidates; every pass runs on registers only.
+template <int KPL>
+__device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], int k, WarpRankSmem &sm,
+                                   uint32_t &tau, int &need) {
+  const int lane = threadIdx.x & 31;
+  Members mem{};
+  mem.all = true;
+  uint32_t rem = (uint32_t)k, m = 0;
+#pragma unroll
+  for (int q = 0; q < KPL; ++q) m += __popc(__ballot_sync(0xffffffffu, kv[q] != 0u));
+#pragma unroll 1
+  for (int pass = 0; pass < 12; ++pass) {
+    if (m <= 32u) {
+      uint32_t cnt = 0;
+#pragma unroll
+      for (int q = 0; q < KPL; ++q) {
+        const bool in = kv[q] != 0u && mem.has(kv[q]);
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        const uint32_t slot = cnt + __popc(bal & ((1u << lane) - 1u));
+        if (in && slot < 32u) sm.list[slot] = kv[q];
+        cnt += __popc(bal);
+      }
+      __syncwarp();
+      cnt = min(cnt, 32u);
+      const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
+      uint32_t gt = 0, ge = 0;
+      for (uint32_t j = 0; j < cnt; ++j) {
+        const uint32_t y = sm.list[j];
+        gt += y > x;
+        ge += y >= x;
+      }
+      const bool hit = (uint32_t)lane < cnt && gt < rem && ge >= rem;
+      const uint32_t who = __ballot_sync(0xffffffffu, hit);
+      const int src = who ? __ffs(who) - 1 : 0;
+      tau = __shfl_sync(0xffffffffu, x, src);
+      need = (int)(rem - __shfl_sync(0xffffffffu, gt, src));
+      __syncwarp();
+      return;
+    }
+    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
+#pragma unroll
+    for (int q = 0; q < KPL; ++q) {
+      if (kv[q] != 0u && mem.has(kv[q])) {
+        umin = min(umin, kv[q]);
+        umax = max(umax, kv[q]);
+      }
+    }
+    umin = __reduce_min_sync(0xffffffffu, umin);
+    umax = __reduce_max_sync(0xffffffffu, umax);
+    if (umin == umax) {
+      tau = umin;
+      need = (int)rem;
+      return;
+    }
+    const Members nx = make_bins(pass, umin, umax);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sm.hist[lane * 8 + q] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < KPL; ++q)
+      if (kv[q] != 0u && mem.has(kv[q])) atomicAdd(&sm.hist[nx.bin(kv[q])], 1u);
+    __syncwarp();
+    uint32_t h[8], local = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      h[q] = sm.hist[lane * 8 + q];
+      local += h[q];
+    }
+    uint32_t above = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
+      if (lane + o < 32) above += v;
+    }
+    above -= local;
+    int bsel = -1;
+    uint32_t rsel = 0, csel = 0;
+#pragma unroll
+    for (int q = 7; q >= 0; --q) {
+      if (bsel < 0 && above + h[q] >= rem && above < rem) {
+        bsel = lane * 8 + q;
+        rsel = rem - above;
+        csel = h[q];
+      }
+      above += h[q];
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, bsel >= 0);
+    const int src = who ? __ffs(who) - 1 : 0;
+    mem = nx;
+    mem.b = (uint32_t)__shfl_sync(0xffffffffu, bsel, src);
+    rem = __shfl_sync(0xffffffffu, rsel, src);
+    m = __shfl_sync(0xffffffffu, csel, src);
+    __syncwarp();
+  }
+  tau = 0xFFFFFFFFu;  // not reached
+  need = 0;
+}
+
+constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 2048)
+
+struct RankArgs {
+  const uint32_t *keys;  // [B*G][nq][ld]
+  int32_t *idx;          // [B][nq][G][S]
+  long long rows;        // B * nq * G
+  int G, nq, ld, k, n_init, n_local, q_start, S;
+};
+
+__global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
+  __shared__ WarpRankSmem wsm[kRWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kRWarps + warp;
+  pdl_trigger();
+  pdl_wait();
+  if (row >= a.rows) return;
+  const int g = (int)(row % a.G);
+  const long long bi = row / a.G;
+  const int i = (int)(bi % a.nq);
+  const long long b = bi / a.nq;
+  const BlockParts bp = block_parts(a.q_start + i, kBlk, a.n_init, a.n_local);
+  const int ncand = bp.cand_hi - bp.cand_lo;
+  int32_t *out = a.idx + row * a.S;
+  const int nloc = bp.c - bp.local_lo + 1;
+  const bool take_all = ncand <= a.k || a.k == 0;
+  const int ntop = take_all ? min(ncand, a.k) : a.k;
+  // init | top-k | local | -1 padding (the top-k part below unless every
+  // candidate, or none, is taken)
+  for (int s = lane; s < a.S; s += 32) {
+    int v;
+    if (s < bp.init_hi) {
+      v = s;
+    } else if (s < bp.init_hi + ntop) {
+      if (!take_all) continue;
+      v = bp.cand_lo + (s - bp.init_hi);
+    } else if (s < bp.init_hi + ntop + nloc) {
+      v = bp.local_lo + (s - bp.init_hi - ntop);
+    } else {
+      v = -1;
+    }
+    out[s] = v;
+  }
+  if (take_all) return;
+  const uint32_t *keys = a.keys + ((b * a.G + g) * a.nq + i) * (long long)a.ld + bp.cand_lo;
+  uint32_t tau;
+  int need;
+  int32_t *top = out + bp.init_hi;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (ncand <= kRegKeys * 32) {
+    uint32_t kv[kRegKeys];
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+      const int e = q * 32 + lane;
+      kv[q] = e < ncand ? ld_key(keys + e) : 0u;
+    }
+    warp_threshold_reg<kRegKeys>(kv, a.k, wsm[warp], tau, need);
+    // keep keys > tau and the first `need` keys == tau, in block order
+    uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+      const uint32_t u = kv[q];
+      const bool gt = u > tau, eq = u == tau && u != 0u;
+      const uint32_t bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+      const uint32_t eq_b = n_eq + __popc(beq & lt);
+      if (gt || (eq && eq_b < (uint32_t)need)) {
+        const uint32_t pos = n_gt + __popc(bgt & lt) + min(eq_b, (uint32_t)need);
+        if (pos < (uint32_t)a.k) top[pos] = bp.cand_lo + q * 32 + lane;
+      }
+      n_gt += __popc(bgt);
+      n_eq += __popc(beq);
+    }
+    return;
+  }
+  warp_threshold(keys, ncand, a.k, wsm[warp], tau, need);
+  // keep keys > tau and the first `need` keys == tau, in block order
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll 2
+  for (int base = 0; base < ncand; base += 32) {
+    const int e = base + lane;
+    const uint32_t u = e < ncand ? ld_key(keys + e) : 0u;
+    const bool gt = e < ncand && u > tau, eq = e < ncand && u == tau;
+    const uint32_t bgt = __ballot_sync(0xffffffffu, gt), beq = __ballot_sync(0xffffffffu, eq);
+    const uint32_t eq_b = n_eq + __popc(beq & lt);
+    if (gt || (eq && eq_b < (uint32_t)need)) {
+      const uint32_t pos = n_gt + __popc(bgt & lt) + min(eq_b, (uint32_t)need);
+      if (pos < (uint32_t)a.k) top[pos] = bp.cand_lo + e;
+    }
+    n_gt += __popc(bgt);
+    n_eq += __popc(beq);
+  }
+}
+
+}  // namespace
+
+// Rows of the score workspace: the block count rounded up to whole tiles.
+int prefill_ld(int NB) { return (int)ceil_div_ll(NB, kPBlk) * kPBlk; }
+
+size_t prefill_select_ws_bytes(const sparda_params &p, int nq) {
+  const int NB = (p.T + kBlk - 1) / kBlk;
+  return (((size_t)p.B * p.G * nq * prefill_ld(NB) * 4) + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
+                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream) {
+  if ((long long)p.B * nq * p.G == 0) return cudaSuccess;
+  const int NB = (p.T + kBlk - 1) / kBlk;
+  const int ld = prefill_ld(NB);
+  // F [B][nq][G][d]: dims (d, G, nq, B); Kc [B][G][NB][d]: dims (d, NB, B*G)
+  CUtensorMap mF, mK;
+  const uint64_t fd[4] = {(uint64_t)kD, (uint64_t)p.G, (uint64_t)nq, (uint64_t)p.B};
+  const uint64_t fs[3] = {(uint64_t)kD * 2, (uint64_t)p.G * kD * 2, (uint64_t)nq * p.G * kD * 2};
+  const uint32_t fb[4] = {64, 1, kPTok, 1};
+  const uint64_t kd[3] = {(uint64_t)kD, (uint64_t)NB, (uint64_t)p.B * p.G};
+  const uint64_t ks[2] = {(uint64_t)kD * 2, (uint64_t)NB * kD * 2};
+  const uint32_t kb[3] = {64, kPBlk, 1};
+  if (!tc::make_map_nd(&mF, F, 4, fd, fs, fb) || !tc::make_map_nd(&mK, kc, 3, kd, ks, kb))
+    return cudaErrorNotSupported;
+  static bool raised[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!raised[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_scores_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    raised[dev] = true;
+  }
+  PScoreArgs sa;
+  sa.keys = static_cast<uint32_t *>(ws);
+  sa.status = nullptr;
+  sa.G = p.G;
+  sa.nq = nq;
+  sa.NB = NB;
+  sa.ld = ld;
+  sa.q_start = q_start;
+  sa.n_init = p.n_init;
+  sa.n_local = p.n_local;
+  const dim3 grid((unsigned)(ld / kPBlk), (unsigned)ceil_div_ll(nq, kPTok), (unsigned)(p.B * p.G));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = kPSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scores_kernel, mF, mK, sa);
+  if (e != cudaSuccess) return e;
+  RankArgs ra;
+  ra.keys = static_cast<const uint32_t *>(ws);
+  ra.idx = idx;
+  ra.rows = (long long)p.B * nq * p.G;
+  ra.G = p.G;
+  ra.nq = nq;
+  ra.ld = ld;
+  ra.k = p.k;
+  ra.n_init = p.n_init;
+  ra.n_local = p.n_local;
+  ra.q_start = q_start;
+  ra.S = p.k + p.n_init + p.n_local;
+  e = launch_pdl(rank_rows_kernel, (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream,
+                 ra);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace sparda

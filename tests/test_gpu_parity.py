@@ -189,6 +189,37 @@ def test_select_prefill_chunk():
     _select_case(F, kc, 16, 1, 2, 0, T, "prefill from 0")
 
 
+@pytest.mark.parametrize("T,nq,q_off,k", [(40000 + 37, 200, 0, 64), (20000, 130, 7000, 100),
+                                           (8192, 64, 0, 1), (16384 + 64, 300, 3000, 512),
+                                           (200000 + 5, 64, 0, 64)])
+def test_select_prefill_tensor_scores(T, nq, q_off, k):
+    """Chunks scored on the tensor cores: several 256-block tiles, a ragged
+    last block, partial 128-token tiles, chunks ending before the sequence
+    does, budgets from 1 to 512, and rows longer than the 2048 keys a warp
+    holds in registers."""
+    rng = W.rng_for(17 + T)
+    B, G = 2, 3
+    NB = (T + 63) // 64
+    kc = W.normal_bf16(rng, (B, G, NB, 128))
+    F = W.normal_bf16(rng, (B, nq, G, 1, 128))
+    _select_case(F, kc, k, 1, 2, T - nq - q_off, T, "prefill tensor")
+
+
+def test_select_prefill_tensor_matches_streaming_path(monkeypatch):
+    """The same chunk through both selection paths gives the same sets."""
+    rng = W.rng_for(19)
+    B, G, T, nq = 1, 2, 24576, 160
+    kc = W.normal_bf16(rng, (B, G, T // 64, 128))
+    F = W.normal_bf16(rng, (B, nq, G, 1, 128))
+    a = gpu_select(F, kc, 64, 1, 2, T - nq, T)
+    monkeypatch.setenv("SPARDA_SELECT_STREAM", "1")
+    b = gpu_select(F, kc, 64, 1, 2, T - nq, T)
+    ora, kth, kth1 = oracle.select(F, kc, 64, 1, 2, T - nq)
+    sc = scores_f64(F, kc)
+    check_sets(a, ora, kth, kth1, sc, "tensor path")
+    check_sets(b, ora, kth, kth1, sc, "streaming path")
+
+
 # --------------------------------------------------------------------------
 # decode attention
 # --------------------------------------------------------------------------
