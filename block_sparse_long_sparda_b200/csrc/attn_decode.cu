@@ -109,8 +109,19 @@ struct TcArgs {
   long long n_entries;  // pairs * S
   long long bg_rows, blk_rows;  // strides in 128-element rows
   int G, S, NB, addr_mode, nq, q_start, max_cover;
+  int order_bgi;        // 1: pairs are streamed in (sequence, group, token) order
   float scale_log2;
 };
+
+// Memory index (b * nq + i) * G + g of the pair at stream position p.  With
+// several query tokens (prefill) the pairs are streamed group by group, so
+// the CTAs running at one time read the K/V of one (sequence, group) --
+// 64 MB at 128K tokens, which stays in L2 -- rather than of every group.
+__device__ __forceinline__ long long mem_pair(const TcArgs &a, long long p) {
+  if (!a.order_bgi) return p;
+  const long long i = p % a.nq, t = p / a.nq;
+  return ((t / a.G) * a.nq + i) * a.G + t % a.G;
+}
 
 // Everything else a CTA keeps in shared memory; it sits in the dynamic
 // allocation behind the operands, so the kernel has no static shared memory
@@ -195,7 +206,7 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
     const float o = live ? acc[h] : 0.f;
     if (n_cover == 1) {
       const float r = L > 0.f ? o / L : 0.f;
-      a.O[(pair * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+      a.O[(mem_pair(a, pair) * R + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
     } else {
       a.ws_o[(slot * R + h) * kD + dim] = o;
       if (dim == 0) a.ws_ml[slot * R + h] = make_float2(M, L);
@@ -243,7 +254,8 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
 #pragma unroll
         for (int h = 0; h < HC; ++h) {
           const float r = L[h] > 0.f ? o[h] / L[h] : 0.f;
-          a.O[(pair * R + h0 + h) * kD + dim] = __bfloat16_as_ushort(__float2bfloat16_rn(r));
+          a.O[(mem_pair(a, pair) * R + h0 + h) * kD + dim] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(r));
         }
       }
       if (dim == 0) a.counters[pair] = 0u;
@@ -310,7 +322,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   }
   pdl_wait();
   const long long e_me = e0 + tid;
-  const int j_me = (tid < kMaxEnt && e_me < e1) ? a.idx[e_me] : -1;
+  const long long pair_me = e_me / a.S;
+  const int s_me = (int)(e_me - pair_me * a.S);
+  const long long pm_me = mem_pair(a, pair_me);
+  const int j_me = (tid < kMaxEnt && e_me < e1) ? a.idx[pm_me * a.S + s_me] : -1;
   if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 64);
   for (int i = tid; i < (4096 + 4096) / 16; i += kWsThreads)  // Q^T, P^T rows >= R stay zero
     reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
@@ -320,15 +335,15 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   {
     const long long e = e_me;
     if (tid < kMaxEnt && e < e1) {
-      const long long pair = e / a.S;
-      const int s = (int)(e - pair * a.S);
+      const long long pair = pair_me, pm = pm_me;
+      const int s = s_me;
       const int j = j_me;
       if (j >= 0) {
-        const int pos = a.q_start + (int)((pair / a.G) % a.nq);
+        const int pos = a.q_start + (int)((pm / a.G) % a.nq);
         if (j >= a.NB || j > pos / kBlk) {
           flag_status(a.status, SPARDA_DEV_RANGE);
         } else {
-          const long long kvpair = (pair / a.G) / a.nq * a.G + pair % a.G;
+          const long long kvpair = (pm / a.G) / a.nq * a.G + pm % a.G;
           const int m = a.addr_mode == SPARDA_ADDR_SLOT ? s : j;
           row_ = (int)(kvpair * a.bg_rows + (long long)m * a.blk_rows);
           rows_ = min(kBlk, pos + 1 - j * kBlk);
@@ -386,7 +401,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     constexpr int QV = (R * 16 + 31) / 32;  // 16-byte pieces of the query rows per lane
     uint4 qn[QV];
     auto load_q = [&](int seg) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(a.Q + (pair0 + seg) * R * kD);
+      const uint4 *src = reinterpret_cast<const uint4 *>(a.Q + mem_pair(a, pair0 + seg) * R * kD);
 #pragma unroll
       for (int j = 0; j < QV; ++j) {
         const int i = lane + 32 * j;
@@ -719,6 +734,7 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.nq = nq;
   a.q_start = q_start;
   a.max_cover = pl.max_cover;
+  a.order_bgi = nq > 1 ? 1 : 0;
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
   a.scale_log2 = scale * kLog2e;
   const size_t parts = (size_t)pairs * pl.max_cover * R;

@@ -8,8 +8,9 @@
 // [p4 "The fourth projection", Algorithm 1 / Eq. 5]: O_l = attention(Q_l,
 // K_l[B_l], V_l[B_l]) with every key resident on the GPU.
 //
-// This file currently routes the chunk through the per-(token, group) gather
-// kernel (CUDA cores, one block list per query token).
+// The chunk runs through the tcgen05 gather kernel of attn_decode.cu with one
+// (token, group) pair per block list; pairs are streamed group by group so
+// that the K/V the running CTAs read stays in L2.
 #include "common.cuh"
 #include "internal.h"
 
