@@ -8,6 +8,8 @@ of 64 tokens, top-k = 64 plus 1 initial and 2 local blocks.  Per layer l:
              keys (the last layer's select the next token's layer 0) and
              keep init U top-k U local;
   attend  -- the layer's queries attend over its selected 67 blocks.
+Both need layer l-1 done and nothing from each other, so select(l) runs on a
+side stream beside attention(l), and attention(l+1) waits for both.
 
 value  : decode tokens/s with every input resident in HBM (K/V of all four
          layers, 34 GB, addressed by block id), timed with CUDA events.
@@ -214,6 +216,11 @@ class DecodeLoop:
         abi.sparda_forecast_select(self.p, self.F[L - 1], 1, 1, w.T - 1, self.kc[0], self.idx[0],
                                    self.ws_sel[0])
         self.compute = torch.cuda.current_stream()
+        # resident step: attention on a high-priority stream, selection beside it
+        self.main = torch.cuda.Stream(priority=-1)
+        self.side_sel = torch.cuda.Stream(priority=0)
+        self.ev_pre = [torch.cuda.Event() for _ in range(L)]
+        self.ev_sel = [torch.cuda.Event() for _ in range(L)]
         self.host_kv = None
         if with_host:
             self._setup_host()
@@ -235,9 +242,22 @@ class DecodeLoop:
                                            self.status)
 
     def step_resident(self):
+        """One decode token through the L layers.  select(l) -- layer l's
+        Forecast vectors picking layer l+1's blocks -- and attention(l) both
+        need layer l-1 finished and nothing from each other, so select(l)
+        runs on a side stream beside attention(l); attention(l+1) waits for
+        both (the order of Algorithm 2, which picks the next layer's blocks
+        before the current layer attends).  Launch on ``self.main``."""
+        torch = self.torch
         for l in range(self.w.layers):
-            self.select(l)
-            self.attention(l)
+            self.ev_pre[l].record(self.main)
+            self.side_sel.wait_event(self.ev_pre[l])
+            with torch.cuda.stream(self.side_sel):
+                self.select(l)
+                self.ev_sel[l].record(self.side_sel)
+            with torch.cuda.stream(self.main):
+                self.attention(l)
+            self.main.wait_event(self.ev_sel[l])
 
     # ---- host offload: K/V in pinned host memory, gathered into slots ----
     def _setup_host(self):
@@ -424,53 +444,56 @@ def run_sparda(args):
     loop = DecodeLoop(w, with_host=want_e2e, seed_offset=rank)
     L = w.layers
 
-    for _ in range(max(args.warmup, 3)):
-        loop.step_resident()
-    # the whole 4-layer step is replayed from a CUDA graph: no host work and
-    # no launch gaps inside the timed region
-    step, graph = loop.step_resident, None
-    try:
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+    # every resident-step launch, its graph capture and its timing are on the
+    # loop's high-priority main stream (selection forks onto a side stream)
+    with torch.cuda.stream(loop.main):
+        for _ in range(max(args.warmup, 3)):
             loop.step_resident()
-        graph.replay()
+        # the whole 4-layer step is replayed from a CUDA graph: no host work and
+        # no launch gaps inside the timed region
+        step, graph = loop.step_resident, None
+        try:
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=loop.main):
+                loop.step_resident()
+            graph.replay()
+            torch.cuda.synchronize()
+            step = graph.replay
+        except Exception as exc:  # keep eager launches, and say so in the line
+            print("note: graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+        for _ in range(max(args.warmup, 3)):
+            step()
+        # clocks are sampled over a ~1 s busy window that contains the timed steps
+        # (untimed padding before and after keeps the GPU in the same state)
+        est = time_steps(step, 5, world) / 5
+        pad = max(1, int(400.0 / max(est, 1e-3)))
+        clocks = ClockSampler(local)
+        for _ in range(pad):
+            step()
+        ms = time_steps(step, args.steps, world)
+        for _ in range(pad):
+            step()
         torch.cuda.synchronize()
-        step = graph.replay
-    except Exception as exc:  # keep eager launches, and say so in the line
-        print("note: graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
-        graph = None
-        torch.cuda.synchronize()
-    for _ in range(max(args.warmup, 3)):
-        step()
-    # clocks are sampled over a ~1 s busy window that contains the timed steps
-    # (untimed padding before and after keeps the GPU in the same state)
-    est = time_steps(step, 5, world) / 5
-    pad = max(1, int(400.0 / max(est, 1e-3)))
-    clocks = ClockSampler(local)
-    for _ in range(pad):
-        step()
-    ms = time_steps(step, args.steps, world)
-    for _ in range(pad):
-        step()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    # per-kernel durations: each kernel alone, back to back over the four
-    # layers on the same stream (as launched in the step), CUDA events around
-    # the whole run; events between kernels would break the programmatic
-    # overlap of consecutive launches
-    def kernel_loop(which):
-        for l in range(L):
-            if which == "select":
-                loop.select(l)
-            else:
-                loop.attention(l)
-    kern_us = {}
-    for which in ("select", "attention"):
-        for _ in range(3):
-            kernel_loop(which)
-        kms = time_steps(lambda: kernel_loop(which), args.steps, world)
-        kern_us[which] = kms / (args.steps * L) * 1e3
+        clk = clocks.stop()
+        # per-kernel durations: each kernel alone, back to back over the four
+        # layers on the same stream (as launched in the step), CUDA events around
+        # the whole run; events between kernels would break the programmatic
+        # overlap of consecutive launches
+        def kernel_loop(which):
+            for l in range(L):
+                if which == "select":
+                    loop.select(l)
+                else:
+                    loop.attention(l)
+        kern_us = {}
+        for which in ("select", "attention"):
+            for _ in range(3):
+                kernel_loop(which)
+            kms = time_steps(lambda: kernel_loop(which), args.steps, world)
+            kern_us[which] = kms / (args.steps * L) * 1e3
     st = int(loop.status.item())
 
     ms_step = ms / args.steps
@@ -518,6 +541,8 @@ def run_sparda(args):
                        "G": w.G, "d": w.d, "block": w.blk, "k": w.k, "n_init": w.n_init,
                        "n_local": w.n_local, "parallelism": "replicas" if world > 1 else "single",
                        "kv": "all layers resident in HBM (34.4 GB), read by block id",
+                       "streams": "select(l) on a side stream beside attention(l); "
+                                  "attention(l+1) waits for both",
                        "l2": "inputs larger than L2: 281 MB of selected K/V per layer, 4 layers"},
             "select_us_per_layer": sel_us,
             "attn_us_per_layer": att_us,
