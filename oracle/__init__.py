@@ -62,6 +62,10 @@ def _load():
         lib.oracle_select.restype = None
         lib.oracle_gather_blocks.argtypes = [I, I, I, I, I, I, I, I, I, I, P, P, P]
         lib.oracle_gather_blocks.restype = None
+        lib.oracle_cache_plan.argtypes = [I, I, I, I, I, P, P, P, P, P]
+        lib.oracle_cache_plan.restype = I
+        lib.oracle_gather_cached.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P]
+        lib.oracle_gather_cached.restype = None
         lib.oracle_sparse_attention.argtypes = [I, I, I, I, I, I, I, I, D, P, P, P, LL, LL, P, I, P]
         lib.oracle_sparse_attention.restype = None
         lib.oracle_dense_causal_attention.argtypes = [I, I, I, I, I, I, I, D, P, P, P, P]
@@ -163,6 +167,42 @@ def gather_blocks(host_kv: np.ndarray, idx: np.ndarray, pos: int, n_init: int, n
     _load().oracle_gather_blocks(B, G, NB, S, blk, d, pos, n_init, n_local, int(skip_resident),
                                  _ptr(host_kv), _ptr(idx), _ptr(slots))
     return slots
+
+
+def cache_plan(idx: np.ndarray, block_of: np.ndarray, hand: np.ndarray, NB: int):
+    """One step of the device slot cache (see oracle_cache_plan).
+
+    idx int32 [B][G][S]; block_of int32 [B][G][C] and hand int32 [B][G] are the
+    cache state before the step.  Returns (phys, fetch, block_of', hand')."""
+    idx = np.ascontiguousarray(idx, np.int32)
+    blk = np.ascontiguousarray(block_of, np.int32).copy()
+    hd = np.ascontiguousarray(hand, np.int32).copy()
+    B, G, S = idx.shape
+    C = blk.shape[2]
+    assert blk.shape == (B, G, C) and hd.shape == (B, G)
+    phys = np.empty((B, G, S), np.int32)
+    fetch = np.empty((B, G, S), np.int32)
+    rc = _load().oracle_cache_plan(B, G, S, C, int(NB), _ptr(idx), _ptr(blk), _ptr(hd),
+                                   _ptr(phys), _ptr(fetch))
+    if rc != 0:
+        raise ValueError("cache_plan needs C >= S (C=%d, S=%d)" % (C, S))
+    return phys, fetch, blk, hd
+
+
+def gather_cached(host_kv: np.ndarray, idx: np.ndarray, phys: np.ndarray, fetch: np.ndarray,
+                  cache: np.ndarray) -> np.ndarray:
+    """Copy the fetched blocks into their slots.  host_kv [B][G][NB][2][blk][d],
+    cache [B][G][C][2][blk][d] (returned as an updated copy)."""
+    host_kv = _u16(host_kv)
+    B, G, NB, two, blk, d = host_kv.shape
+    cache = np.ascontiguousarray(_u16(cache).copy())
+    C = cache.shape[2]
+    idx = np.ascontiguousarray(idx, np.int32)
+    S = idx.shape[-1]
+    _load().oracle_gather_cached(B, G, NB, S, C, blk, d, _ptr(host_kv), _ptr(idx),
+                                 _ptr(np.ascontiguousarray(phys, np.int32)),
+                                 _ptr(np.ascontiguousarray(fetch, np.int32)), _ptr(cache))
+    return cache
 
 
 def sparse_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray, q_start: int,

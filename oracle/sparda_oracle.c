@@ -338,6 +338,82 @@ void oracle_gather_blocks(int B, int G, int NB, int S, int blk, int d, int pos, 
 }
 
 /* ------------------------------------------------------------------------ */
+/* o3c: a device slot cache across decode steps (fetch only what is new)    */
+/*   [p4] "The fourth projection", Algorithm 2 fetches layer l+1's blocks   */
+/*   from CPU pinned memory each step; "What this doesn't fix" notes that   */
+/*   the transfer is bounded by the host link.  Blocks that stay selected   */
+/*   from one step to the next need no new transfer if they stay in the     */
+/*   device slots.  The pages give no policy, so the plainest one is taken: */
+/*   each (b,g) owns C slots; block_of[c] is the block slot c holds (-1:    */
+/*   empty) and `hand` a clock position.  For one step's list idx:          */
+/*    1. an entry whose block is held in some slot c is a hit: phys = c;    */
+/*    2. every other valid entry, in list order, is a miss: the hand moves  */
+/*       forward (cyclically) past slots holding a block of this step's     */
+/*       list, takes the next slot, and moves one further; that slot now    */
+/*       holds the entry's block, phys = that slot and fetch = 1.           */
+/*   Entries of -1 or outside [0, NB) get phys = -1, fetch = 0.  C >= S is  */
+/*   required (a free slot then always exists).                             */
+/*   idx [B][G][S]; block_of [B][G][C], hand [B][G] (updated in place);     */
+/*   phys, fetch [B][G][S] (out)                                            */
+/* ------------------------------------------------------------------------ */
+
+int oracle_cache_plan(int B, int G, int S, int C, int NB, const int32_t *idx, int32_t *block_of,
+                      int32_t *hand, int32_t *phys, int32_t *fetch) {
+  if (C < S || C < 1) return -1;
+  unsigned char *used = (unsigned char *)malloc((size_t)C);
+  if (!used) return -1;
+  for (long long bg = 0; bg < (long long)B * G; ++bg) {
+    const int32_t *row = idx + bg * S;
+    int32_t *blk = block_of + bg * C;
+    int32_t *ph = phys + bg * S;
+    int32_t *fe = fetch + bg * S;
+    memset(used, 0, (size_t)C);
+    for (int s = 0; s < S; ++s) {
+      int j = row[s];
+      ph[s] = -1;
+      fe[s] = 0;
+      if (j < 0 || j >= NB) continue;
+      for (int c = 0; c < C; ++c) {
+        if (blk[c] == j) {
+          ph[s] = c;
+          used[c] = 1;
+          break;
+        }
+      }
+    }
+    for (int s = 0; s < S; ++s) {
+      int j = row[s];
+      if (j < 0 || j >= NB || ph[s] >= 0) continue;
+      while (used[hand[bg]]) hand[bg] = (hand[bg] + 1) % C;
+      int v = hand[bg];
+      hand[bg] = (v + 1) % C;
+      blk[v] = j;
+      used[v] = 1;
+      ph[s] = v;
+      fe[s] = 1;
+    }
+  }
+  free(used);
+  return 0;
+}
+
+/* the cache side of o3: slot phys[s] of (b,g) receives block idx[s] for   */
+/* every entry with fetch[s] set; cache [B][G][C][2][blk][d]               */
+void oracle_gather_cached(int B, int G, int NB, int S, int C, int blk, int d,
+                          const uint16_t *host_kv, const int32_t *idx, const int32_t *phys,
+                          const int32_t *fetch, uint16_t *cache) {
+  long long blk_elems = 2LL * blk * d;
+  for (long long bg = 0; bg < (long long)B * G; ++bg) {
+    for (int s = 0; s < S; ++s) {
+      int j = idx[bg * S + s], c = phys[bg * S + s];
+      if (!fetch[bg * S + s] || j < 0 || j >= NB || c < 0 || c >= C) continue;
+      memcpy(cache + (bg * C + c) * blk_elems, host_kv + (bg * NB + j) * blk_elems,
+             sizeof(uint16_t) * (size_t)blk_elems);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* o4: attention of each query head over the keys of its block set          */
 /*   [p4] "The fourth projection", Eq. 5 / Algorithm 1:                     */
 /*        O_l = attention(Q_l, K_l[B_l], V_l[B_l])                          */

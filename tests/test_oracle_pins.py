@@ -402,3 +402,95 @@ def test_sparse_interleaved_layout_matches_plain_layout():
     inter = oracle.sparse_attention(Q, KV.reshape(-1), KV.reshape(-1)[blk * d:], idx, T - 1, T, blk,
                                     bg_stride=NB * 2 * blk * d, blk_stride=2 * blk * d, G=G)
     np.testing.assert_allclose(plain, inter, rtol=0, atol=0)
+
+
+# --------------------------------------------------------------------------
+# device slot cache across decode steps (the fetch-only-what-is-new policy)
+# --------------------------------------------------------------------------
+
+def test_cache_plan_hand_derived_steps():
+    """Five steps of one (b, g) with C = 4 slots, S = 3 entries, NB = 16,
+    worked by hand from the policy's definition: hits keep their slot; each
+    miss, in list order, takes the clock hand's next slot that holds none of
+    the step's blocks."""
+    NB = 16
+    blk = np.full((1, 1, 4), -1, np.int32)
+    hd = np.zeros((1, 1), np.int32)
+    steps = [
+        # idx            phys          fetch      block_of after      hand
+        ([5, 7, 9],      [0, 1, 2],    [1, 1, 1], [5, 7, 9, -1],      3),   # cold start
+        ([5, 9, 11],     [0, 2, 3],    [0, 0, 1], [5, 7, 9, 11],      0),   # two hits, hand wraps
+        ([2, 5, 12],     [1, 0, 2],    [1, 0, 1], [5, 2, 12, 11],     3),   # hand skips the hit slot 0
+        ([-1, 11, 2],    [-1, 3, 1],   [0, 0, 0], [5, 2, 12, 11],     3),   # padding, all hits
+        ([20, 3, 4],     [-1, 3, 0],   [0, 1, 1], [4, 2, 12, 3],      1),   # out of range id skipped
+    ]
+    for ids, ph_want, fe_want, blk_want, hand_want in steps:
+        idx = np.array(ids, np.int32).reshape(1, 1, 3)
+        phys, fetch, blk, hd = oracle.cache_plan(idx, blk, hd, NB)
+        assert phys.reshape(-1).tolist() == ph_want, (ids, phys)
+        assert fetch.reshape(-1).tolist() == fe_want, (ids, fetch)
+        assert blk.reshape(-1).tolist() == blk_want, (ids, blk)
+        assert int(hd[0, 0]) == hand_want
+
+
+def test_cache_plan_needs_as_many_slots_as_entries():
+    with pytest.raises(ValueError):
+        oracle.cache_plan(np.zeros((1, 1, 5), np.int32), np.full((1, 1, 4), -1, np.int32),
+                          np.zeros((1, 1), np.int32), 16)
+
+
+def test_cache_plan_invariants_over_drifting_sets():
+    """Over many steps of slowly changing sets: every valid entry ends up
+    held at its slot, exactly the blocks not held before are fetched, no slot
+    holds two blocks, and a block that stays selected never moves."""
+    rng = np.random.default_rng(5)
+    B, G, S, C, NB = 2, 3, 10, 16, 64
+    blk = np.full((B, G, C), -1, np.int32)
+    hd = np.zeros((B, G), np.int32)
+    cur = np.stack([np.stack([rng.choice(NB, S, replace=False) for _ in range(G)]) for _ in range(B)])
+    total_fetch = 0
+    for step in range(60):
+        # replace a couple of each row's blocks by new ones
+        for b in range(B):
+            for g in range(G):
+                for s in rng.choice(S, 2, replace=False):
+                    fresh = [x for x in range(NB) if x not in cur[b, g]]
+                    cur[b, g, s] = rng.choice(fresh)
+        idx = np.sort(cur, axis=2).astype(np.int32)
+        before = blk.copy()
+        phys, fetch, blk, hd = oracle.cache_plan(idx, blk, hd, NB)
+        for b in range(B):
+            for g in range(G):
+                held_before = {int(x): c for c, x in enumerate(before[b, g]) if x >= 0}
+                row_slots = phys[b, g]
+                assert len(set(row_slots.tolist())) == S
+                for s in range(S):
+                    j = int(idx[b, g, s])
+                    assert blk[b, g, row_slots[s]] == j
+                    assert fetch[b, g, s] == (0 if j in held_before else 1)
+                    if j in held_before:
+                        assert row_slots[s] == held_before[j]
+                held = blk[b, g][blk[b, g] >= 0]
+                assert len(set(held.tolist())) == len(held)
+        total_fetch += int(fetch.sum())
+        if step > 0:
+            assert fetch.sum() <= 2 * B * G  # only the replaced blocks can be new
+    assert total_fetch > 0
+
+
+def test_gather_cached_copies_only_fetched_entries():
+    rng = np.random.default_rng(6)
+    B, G, NB, S, C, blk, d = 1, 2, 12, 3, 5, 4, 8
+    host = rng.integers(0, 65535, (B, G, NB, 2, blk, d), dtype=np.uint16)
+    cache = np.zeros((B, G, C, 2, blk, d), np.uint16)
+    idx = np.array([[[1, 4, 7], [0, 2, 9]]], np.int32)
+    phys = np.array([[[3, 0, 1], [2, 4, 0]]], np.int32)
+    fetch = np.array([[[1, 0, 1], [0, 1, 1]]], np.int32)
+    out = oracle.gather_cached(host, idx, phys, fetch, cache)
+    for g in range(G):
+        for s in range(S):
+            c = phys[0, g, s]
+            if fetch[0, g, s]:
+                assert np.array_equal(out[0, g, c], host[0, g, idx[0, g, s]])
+    assert not out[0, 0, 0].any() and not out[0, 0, 2].any() and not out[0, 0, 4].any()
+    assert not out[0, 1, 1].any() and not out[0, 1, 3].any()
