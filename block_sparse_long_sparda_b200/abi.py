@@ -37,6 +37,7 @@ SPARDA_OP_ATTN_PREFILL = 4
 
 SPARDA_ADDR_LOGICAL = 0
 SPARDA_ADDR_SLOT = 1
+SPARDA_ADDR_PHYS = 2
 
 
 class SpardaError(RuntimeError):
@@ -71,6 +72,9 @@ _SIGS = {
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_decode_noalloc": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _P]),
+    "sparda_cache_plan": (_I, [_PP, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "sparda_prefetch_cached": (_I, [_PP, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "sparda_sparse_attn_decode_cached": (_I, [_PP, _I, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "sparda_workspace_size": (_SZ, [_I, _PP, _I, _I]),
     "sparda_status_string": (ctypes.c_char_p, [_I]),
     "sparda_status_from_device": (_I, [ctypes.c_int32]),
@@ -179,6 +183,28 @@ def sparda_sparse_attn_decode_noalloc(p, Q, K, V, bg_stride, blk_stride, idx, ad
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def sparda_cache_plan(p, C, idx, block_of, hand, phys, fetch, dev_status=None, stream=None):
+    _check("sparda_cache_plan",
+           lib().sparda_cache_plan(ctypes.byref(p), int(C), _ptr(idx), _ptr(block_of), _ptr(hand),
+                                   _ptr(phys), _ptr(fetch), _ptr(dev_status), _stream(stream)))
+
+
+def sparda_prefetch_cached(p, C, host_kv, idx, phys, fetch, cache, n_ctas=0, dev_status=None,
+                           stream=None):
+    _check("sparda_prefetch_cached",
+           lib().sparda_prefetch_cached(ctypes.byref(p), int(C), _ptr(host_kv), _ptr(idx),
+                                        _ptr(phys), _ptr(fetch), _ptr(cache), int(n_ctas),
+                                        _ptr(dev_status), _stream(stream)))
+
+
+def sparda_sparse_attn_decode_cached(p, C, Q, cache, idx, phys, O, ws, dev_status=None,
+                                     stream=None):
+    _check("sparda_sparse_attn_decode_cached",
+           lib().sparda_sparse_attn_decode_cached(ctypes.byref(p), int(C), _ptr(Q), _ptr(cache),
+                                                  _ptr(idx), _ptr(phys), _ptr(O), _ptr(ws),
+                                                  _nbytes(ws), _ptr(dev_status), _stream(stream)))
 
 
 def sparda_workspace_size(op, p, nq=1, nf=1) -> int:

@@ -152,6 +152,74 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ---- device slot cache ----------------------------------------------------
+static int cache_args_ok(const sparda_params *p, int C) {
+  const int S = p->k + p->n_init + p->n_local;
+  return C >= S && C >= 1 && C <= kMaxCacheSlots;
+}
+
+// device view of a page-locked, mapped host buffer (null if it is not one)
+static const uint16_t *mapped_device_view(const void *host) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, host) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (attr.type != cudaMemoryTypeHost || attr.devicePointer == nullptr) return nullptr;
+  const uint16_t *v = static_cast<const uint16_t *>(attr.devicePointer);
+  return aligned16(v) ? v : nullptr;
+}
+
+int sparda_cache_plan(const sparda_params *p, int C, const int32_t *idx, int32_t *block_of,
+                      int32_t *hand, int32_t *phys, int32_t *fetch, int32_t *dev_status,
+                      sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (!cache_args_ok(p, C)) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!idx || !block_of || !hand || !phys || !fetch) return SPARDA_EINVAL;
+  return from_cuda(launch_cache_plan(*p, C, idx, block_of, hand, phys, fetch, dev_status,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_prefetch_cached(const sparda_params *p, int C, const void *host_kv,
+                           const int32_t *idx, const int32_t *phys, const int32_t *fetch,
+                           void *cache, int n_ctas, int32_t *dev_status, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (!cache_args_ok(p, C) || n_ctas < 0) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!host_kv || !idx || !phys || !fetch || !cache) return SPARDA_EINVAL;
+  if (!aligned16(host_kv) || !aligned16(cache)) return SPARDA_EINVAL;
+  const uint16_t *dev_view = mapped_device_view(host_kv);
+  if (!dev_view) return SPARDA_EINVAL;
+  return from_cuda(launch_prefetch_cached(*p, C, dev_view, idx, phys, fetch,
+                                          static_cast<uint16_t *>(cache), n_ctas, dev_status,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_sparse_attn_decode_cached(const sparda_params *p, int C, const void *Q,
+                                     const void *cache, const int32_t *idx, const int32_t *phys,
+                                     void *O, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                     sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (!cache_args_ok(p, C)) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!Q || !cache || !idx || !phys || !O) return SPARDA_EINVAL;
+  if (!aligned16(Q) || !aligned16(cache) || !aligned16(idx) || !aligned16(phys) || !aligned16(O))
+    return SPARDA_EINVAL;
+  const DecodePlan pl = plan_decode(*p);
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  const long long blk_elems = 2LL * kBlk * kD;  // K block then V block
+  const uint16_t *K = static_cast<const uint16_t *>(cache);
+  return from_cuda(launch_attn_decode(*p, pl, static_cast<const uint16_t *>(Q), K,
+                                      K + (long long)kBlk * kD, (long long)C * blk_elems,
+                                      blk_elems, idx, SPARDA_ADDR_PHYS,
+                                      static_cast<uint16_t *>(O), ws, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream), phys, C));
+}
+
 int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, int q_start,
                                const void *K, const void *V, long long bg_stride,
                                long long tok_stride, const int32_t *idx, void *O, void *ws,

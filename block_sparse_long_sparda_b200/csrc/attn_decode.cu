@@ -102,6 +102,7 @@ struct TcArgs {
   const uint16_t *Q;
   uint16_t *O;
   const int32_t *idx;
+  const int32_t *phys;  // SPARDA_ADDR_PHYS: the slot of each entry
   float *ws_o;          // [pairs][max_cover][R][128] unnormalised segment outputs
   float2 *ws_ml;        // [pairs][max_cover][R] (max, sum) in the exp2 domain
   uint32_t *counters;   // [pairs] tickets, zero between calls
@@ -110,6 +111,7 @@ struct TcArgs {
   long long bg_rows, blk_rows;  // strides in 128-element rows
   int G, S, NB, addr_mode, nq, q_start, max_cover;
   int order_bgi;        // 1: pairs are streamed in (sequence, group, token) order
+  int n_slots;          // SPARDA_ADDR_PHYS: slots per (sequence, group)
   float scale_log2;
 };
 
@@ -325,7 +327,9 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   const long long pair_me = e_me / a.S;
   const int s_me = (int)(e_me - pair_me * a.S);
   const long long pm_me = mem_pair(a, pair_me);
-  const int j_me = (tid < kMaxEnt && e_me < e1) ? a.idx[pm_me * a.S + s_me] : -1;
+  const bool own = tid < kMaxEnt && e_me < e1;
+  const int j_me = own ? a.idx[pm_me * a.S + s_me] : -1;
+  const int phys_me = (own && a.addr_mode == SPARDA_ADDR_PHYS) ? a.phys[pm_me * a.S + s_me] : 0;
   if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 64);
   for (int i = tid; i < (4096 + 4096) / 16; i += kWsThreads)  // Q^T, P^T rows >= R stay zero
     reinterpret_cast<uint4 *>(qop)[i] = make_uint4(0, 0, 0, 0);
@@ -340,11 +344,15 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       const int j = j_me;
       if (j >= 0) {
         const int pos = a.q_start + (int)((pm / a.G) % a.nq);
-        if (j >= a.NB || j > pos / kBlk) {
+        const bool slot_bad =
+            a.addr_mode == SPARDA_ADDR_PHYS && (phys_me < 0 || phys_me >= a.n_slots);
+        if (j >= a.NB || j > pos / kBlk || slot_bad) {
           flag_status(a.status, SPARDA_DEV_RANGE);
         } else {
           const long long kvpair = (pm / a.G) / a.nq * a.G + pm % a.G;
-          const int m = a.addr_mode == SPARDA_ADDR_SLOT ? s : j;
+          const int m = a.addr_mode == SPARDA_ADDR_SLOT ? s
+                        : a.addr_mode == SPARDA_ADDR_PHYS ? phys_me
+                                                          : j;
           row_ = (int)(kvpair * a.bg_rows + (long long)m * a.blk_rows);
           rows_ = min(kBlk, pos + 1 - j * kBlk);
           seg_ = (int)(pair - pair0);
@@ -702,7 +710,7 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
                                const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                                long long bg_stride, long long blk_stride, const int32_t *idx,
                                int addr_mode, uint16_t *O, void *ws, int32_t *dev_status,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const int32_t *phys, int n_slots) {
   const long long pairs = (long long)p.B * nq * p.G;
   if (pairs == 0) return cudaSuccess;
   const int R = p.Hq / p.G;
@@ -711,7 +719,9 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   const long long bg_rows = bg_stride / kD, blk_rows = blk_stride / kD;
   // rows each tensor map may touch: up to the last row of the last block the
   // strides can address, but never past the packed end of the buffer
-  const long long m_max = addr_mode == SPARDA_ADDR_SLOT ? pl.S - 1 : NB - 1;
+  const long long m_max = addr_mode == SPARDA_ADDR_SLOT   ? pl.S - 1
+                          : addr_mode == SPARDA_ADDR_PHYS ? n_slots - 1
+                                                          : NB - 1;
   long long extent = (kv_pairs - 1) * bg_rows + m_max * blk_rows + kBlk;
   extent = std::min(extent, kv_pairs * bg_rows);
   if (extent >= (1LL << 31)) return cudaErrorInvalidValue;
@@ -723,6 +733,8 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.Q = Q;
   a.O = O;
   a.idx = idx;
+  a.phys = phys;
+  a.n_slots = n_slots;
   a.status = dev_status;
   a.n_entries = pairs * pl.S;
   a.bg_rows = bg_rows;
@@ -768,9 +780,10 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
 cudaError_t launch_attn_decode(const sparda_params &p, const DecodePlan &pl, const uint16_t *Q,
                                const uint16_t *K, const uint16_t *V, long long bg_stride,
                                long long blk_stride, const int32_t *idx, int addr_mode,
-                               uint16_t *O, void *ws, int32_t *dev_status, cudaStream_t stream) {
+                               uint16_t *O, void *ws, int32_t *dev_status, cudaStream_t stream,
+                               const int32_t *phys, int n_slots) {
   return launch_gather_attn(p, pl, 1, p.T - 1, Q, K, V, bg_stride, blk_stride, idx, addr_mode, O,
-                            ws, dev_status, stream);
+                            ws, dev_status, stream, phys, n_slots);
 }
 
 }  // namespace sparda

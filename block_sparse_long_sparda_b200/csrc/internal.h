@@ -88,16 +88,29 @@ struct DecodePlan {
 DecodePlan plan_decode(const sparda_params &p);
 DecodePlan plan_gather(const sparda_params &p, long long pairs);
 // one query per (sequence, token, group) "pair", each with its own block list
+// (addr_mode SPARDA_ADDR_PHYS: entry e reads block slot phys[e] < n_slots)
 cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int nq, int q_start,
                                const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                                long long bg_stride, long long blk_stride, const int32_t *idx,
                                int addr_mode, uint16_t *O, void *ws, int32_t *dev_status,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const int32_t *phys = nullptr,
+                               int n_slots = 0);
 cudaError_t launch_attn_decode(const sparda_params &p, const DecodePlan &plan,
                                const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                                long long bg_stride, long long blk_stride, const int32_t *idx,
                                int addr_mode, uint16_t *O, void *ws, int32_t *dev_status,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const int32_t *phys = nullptr,
+                               int n_slots = 0);
+
+// ---- device slot cache (cache.cu) -------------------------------------------
+constexpr int kMaxCacheSlots = 4096;
+cudaError_t launch_cache_plan(const sparda_params &p, int C, const int32_t *idx,
+                              int32_t *block_of, int32_t *hand, int32_t *phys, int32_t *fetch,
+                              int32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_prefetch_cached(const sparda_params &p, int C, const uint16_t *host_kv_dev,
+                                   const int32_t *idx, const int32_t *phys, const int32_t *fetch,
+                                   uint16_t *cache, int n_ctas, int32_t *dev_status,
+                                   cudaStream_t stream);
 
 // ---- prefill attention ----------------------------------------------------
 size_t prefill_ws_bytes(const sparda_params &p, int nq);

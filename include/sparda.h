@@ -99,7 +99,8 @@ enum sparda_op {
 /* how sparda_sparse_attn_decode finds the storage of list entry s */
 enum sparda_addr_mode {
   SPARDA_ADDR_LOGICAL = 0, /* block id idx[s] indexes the K/V buffer (KV resident)   */
-  SPARDA_ADDR_SLOT = 1     /* list position s indexes it (prefetched device slots)  */
+  SPARDA_ADDR_SLOT = 1,    /* list position s indexes it (prefetched device slots)  */
+  SPARDA_ADDR_PHYS = 2     /* phys[s] indexes it (slot cache; see the cached calls) */
 };
 
 /*
@@ -229,6 +230,53 @@ int sparda_sparse_attn_decode_noalloc(const sparda_params *p, const void *Q, con
                                       const void *V, long long bg_stride, long long blk_stride,
                                       const int32_t *idx, int addr_mode, void *O,
                                       int32_t *dev_status, sparda_stream_t stream);
+
+/*
+ * Device slot cache across decode steps -- fetch only what is new.
+ *   [p4 "The fourth projection", Algorithm 2] fetches every layer's selected
+ *   blocks from CPU pinned memory each step, and [p4 "What this doesn't
+ *   fix"] notes that the host link bounds that transfer.  A block still
+ *   selected at the next step need not cross the link again if it stays in
+ *   the device slots.  The pages give no policy; these calls implement the
+ *   plainest one.  Each (b,g) owns C slots (S <= C <= 4096) of one layer:
+ *     cache     bf16 [B][G][C][2][blk][d] device (K block then V block)
+ *     block_of  int32 [B][G][C] device: the block each slot holds, -1 empty
+ *               (fill with -1 before the first step)
+ *     hand      int32 [B][G] device: the clock position (0 before the first step)
+ *   The state belongs to the caller; one layer's calls must not overlap.
+ *
+ * sparda_cache_plan -- for one step's lists idx [B][G][S] (device): an entry
+ *   whose block some slot c holds is a hit (phys = c, fetch = 0); every other
+ *   entry with a block id in [0, NB), in list order, takes the next slot past
+ *   the hand that holds none of this step's blocks (phys = that slot,
+ *   fetch = 1) and the hand moves one further.  Entries of -1 get phys = -1;
+ *   ids >= NB are flagged SPARDA_DEV_RANGE.  block_of and hand are updated.
+ *   phys, fetch: int32 [B][G][S] device (out).  C < S -> SPARDA_EINVAL.
+ */
+int sparda_cache_plan(const sparda_params *p, int C, const int32_t *idx, int32_t *block_of,
+                      int32_t *hand, int32_t *phys, int32_t *fetch, int32_t *dev_status,
+                      sparda_stream_t stream);
+
+/*
+ * sparda_prefetch_cached -- copy block idx[s] of the page-locked, mapped host
+ *   buffer (layout and checks as for sparda_prefetch_blocks) into slot
+ *   phys[s] of the cache, for every entry with fetch[s] != 0 (the misses of
+ *   sparda_cache_plan); n_ctas as for sparda_prefetch_blocks.
+ */
+int sparda_prefetch_cached(const sparda_params *p, int C, const void *host_kv,
+                           const int32_t *idx, const int32_t *phys, const int32_t *fetch,
+                           void *cache, int n_ctas, int32_t *dev_status, sparda_stream_t stream);
+
+/*
+ * sparda_sparse_attn_decode_cached -- sparda_sparse_attn_decode reading list
+ *   entry s of (b,g) from cache slot phys[b,g,s] (idx gives its block id for
+ *   the causal mask).  A slot outside [0, C) is skipped and flagged
+ *   SPARDA_DEV_RANGE.  ws as for sparda_sparse_attn_decode.
+ */
+int sparda_sparse_attn_decode_cached(const sparda_params *p, int C, const void *Q,
+                                     const void *cache, const int32_t *idx, const int32_t *phys,
+                                     void *O, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                     sparda_stream_t stream);
 
 /* Bytes of device workspace an op needs for these shapes (0: none). nf is
  * the number of scoring vectors per group (select only). */

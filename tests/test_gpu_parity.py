@@ -366,6 +366,120 @@ def test_prefetch_flags_out_of_range_and_rejects_pageable_memory():
 
 
 # --------------------------------------------------------------------------
+# device slot cache across decode steps
+# --------------------------------------------------------------------------
+
+def _drifting_sets(rng, B, G, S, NB, steps, change):
+    """Per step, sorted distinct block sets that keep all but `change` blocks
+    of the previous step (plus -1 padding in one row and a stale id)."""
+    cur = np.stack([np.stack([rng.choice(NB, S, replace=False) for _ in range(G)]) for _ in range(B)])
+    out = []
+    for _ in range(steps):
+        for b in range(B):
+            for g in range(G):
+                for s in rng.choice(S, change, replace=False):
+                    fresh = np.setdiff1d(np.arange(NB), cur[b, g])
+                    cur[b, g, s] = rng.choice(fresh)
+        out.append(np.sort(cur, axis=2).astype(np.int32))
+    return out
+
+
+def test_cache_plan_matches_oracle_over_steps():
+    rng = np.random.default_rng(40)
+    B, G, k, C, NB = 2, 3, 7, 16, 64
+    S = k + 3
+    p = abi.make_params(B, G, G, NB * 64, k)
+    block_of = torch.full((B, G, C), -1, dtype=torch.int32, device="cuda")
+    hand = torch.zeros(B, G, dtype=torch.int32, device="cuda")
+    phys = torch.empty(B, G, S, dtype=torch.int32, device="cuda")
+    fetch = torch.empty_like(phys)
+    o_blk = np.full((B, G, C), -1, np.int32)
+    o_hand = np.zeros((B, G), np.int32)
+    for step, idx in enumerate(_drifting_sets(rng, B, G, S, NB, 25, 3)):
+        if step == 4:
+            idx[1, 2, -2:] = -1          # a short list
+        didx = torch.from_numpy(idx).cuda()
+        abi.sparda_cache_plan(p, C, didx, block_of, hand, phys, fetch)
+        torch.cuda.synchronize()
+        o_phys, o_fetch, o_blk, o_hand = oracle.cache_plan(idx, o_blk, o_hand, NB)
+        assert np.array_equal(phys.cpu().numpy(), o_phys), step
+        assert np.array_equal(fetch.cpu().numpy(), o_fetch), step
+        assert np.array_equal(block_of.cpu().numpy(), o_blk), step
+        assert np.array_equal(hand.cpu().numpy(), o_hand), step
+
+
+def test_cache_plan_rejects_too_few_slots_and_flags_bad_ids():
+    p = abi.make_params(1, 1, 1, 64 * 10, 4)        # S = 7
+    idx = torch.tensor([[[0, 1, 2, 3, 99, 8, 9]]], dtype=torch.int32, device="cuda")
+    blk = torch.full((1, 1, 8), -1, dtype=torch.int32, device="cuda")
+    hand = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    phys = torch.empty(1, 1, 7, dtype=torch.int32, device="cuda")
+    fetch = torch.empty_like(phys)
+    with pytest.raises(abi.SpardaError) as e:
+        abi.sparda_cache_plan(p, 6, idx, blk, hand, phys, fetch)
+    assert e.value.status == abi.SPARDA_EINVAL
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_cache_plan(p, 8, idx, blk, hand, phys, fetch, status)
+    torch.cuda.synchronize()
+    assert abi.sparda_status_from_device(int(status.item())) == abi.SPARDA_ERANGE
+    assert phys.cpu().numpy()[0, 0, 4] == -1 and fetch.cpu().numpy()[0, 0, 4] == 0
+
+
+@pytest.mark.parametrize("R", [4, 8])
+def test_cached_prefetch_and_attention_over_steps(R):
+    """Plan, fetch only the misses, attend from the cache -- three steps of
+    drifting sets: the cache holds the host bytes at every slot a list uses,
+    and attention equals the oracle over the logical block ids."""
+    rng = np.random.default_rng(41 + R)
+    B, G, NB, d, k, C = 2, 2, 96, 128, 13, 24
+    T = NB * 64 - 5
+    S = k + 3
+    host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    p = abi.make_params(B, G * R, G, T, k)
+    hkv = _pinned_bf16(host)
+    cache = torch.zeros(B, G, C, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+    block_of = torch.full((B, G, C), -1, dtype=torch.int32, device="cuda")
+    hand = torch.zeros(B, G, dtype=torch.int32, device="cuda")
+    phys = torch.empty(B, G, S, dtype=torch.int32, device="cuda")
+    fetch = torch.empty_like(phys)
+    ws = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o_cache = np.zeros((B, G, C, 2, 64, d), np.uint16)
+    o_blk, o_hand = np.full((B, G, C), -1, np.int32), np.zeros((B, G), np.int32)
+    Fb = W.normal_bf16(rng, (B, 1, G, 1, d))
+    for step in range(3):
+        if step > 0:  # the Forecast drifts a little each step, so most of the set stays
+            drift = 0.3 * rng.standard_normal(Fb.shape).astype(np.float32)
+            Fb = W.f32_to_bf16_bits(W.bf16_bits_to_f32(Fb) + drift)
+        idx, _, _ = oracle.select(Fb, kc, k, 1, 2, T - 1)
+        idx = np.ascontiguousarray(idx[:, 0])
+        didx = torch.from_numpy(idx).cuda()
+        abi.sparda_cache_plan(p, C, didx, block_of, hand, phys, fetch, status)
+        abi.sparda_prefetch_cached(p, C, hkv, didx, phys, fetch, cache, 0, status)
+        Q = W.normal_bf16(rng, (B, G * R, d))
+        O = torch.empty(B, G * R, d, dtype=torch.bfloat16, device="cuda")
+        abi.sparda_sparse_attn_decode_cached(p, C, dev_bf16(Q), cache, didx, phys, O, ws, status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        o_phys, o_fetch, o_blk, o_hand = oracle.cache_plan(idx, o_blk, o_hand, NB)
+        assert np.array_equal(phys.cpu().numpy(), o_phys)
+        assert np.array_equal(fetch.cpu().numpy(), o_fetch)
+        o_cache = oracle.gather_cached(host, idx, o_phys, o_fetch, o_cache)
+        got = host_bits(cache)
+        for b in range(B):
+            for g in range(G):
+                for s in range(S):
+                    assert np.array_equal(got[b, g, o_phys[b, g, s]], host[b, g, idx[b, g, s]])
+        assert np.array_equal(got, o_cache)
+        flat = host.reshape(-1)
+        ora = oracle.sparse_attention(Q.reshape(B, 1, G * R, d), flat, flat[64 * d:],
+                                      idx.reshape(B, 1, G, S), T - 1, T, 64,
+                                      bg_stride=NB * 2 * 64 * d, blk_stride=2 * 64 * d, G=G)
+        check_attention(host_bits(O).reshape(B, 1, G * R, d), ora, "cached step %d" % step)
+
+
+# --------------------------------------------------------------------------
 # prefill attention
 # --------------------------------------------------------------------------
 
