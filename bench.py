@@ -317,6 +317,94 @@ class DecodeLoop:
                                           self.O[l], self.ws_att, self.status)
         self.h_O.copy_(self.O, non_blocking=True)
 
+    # ---- host offload with a device slot cache: fetch only new blocks ----
+    def setup_cache(self, C: int, sigma: float, n_steps: int, seed: int = 7):
+        """C slots per (layer, b, g); the Forecast vectors of step t+1 are
+        those of step t plus sigma * N(0, 1) noise, so consecutive steps
+        select mostly the same blocks (a drift model of consecutive tokens;
+        sigma = 0 keeps the sets fixed).  The per-step Forecast vectors sit
+        in pinned host memory and are uploaded in the timed step."""
+        torch, w = self.torch, self.w
+        L, dev = w.layers, torch.device("cuda")
+        self.C = C
+        self.cache = torch.empty(L, w.B, w.G, C, 2, w.blk, w.d, dtype=torch.bfloat16, device=dev)
+        self.block_of = torch.full((L, w.B, w.G, C), -1, dtype=torch.int32, device=dev)
+        self.hand = torch.zeros(L, w.B, w.G, dtype=torch.int32, device=dev)
+        self.phys = torch.empty(L, w.B, w.G, w.S, dtype=torch.int32, device=dev)
+        self.fetch = torch.zeros(L, w.B, w.G, w.S, dtype=torch.int32, device=dev)
+        gen = torch.Generator()
+        gen.manual_seed(seed)
+        F = self.F.float().cpu()
+        steps = []
+        for _ in range(n_steps):
+            steps.append(F.to(torch.bfloat16))
+            F = F + sigma * torch.randn(F.shape, generator=gen)
+        self.h_F_steps = torch.stack(steps).pin_memory()
+        self.copy = torch.cuda.Stream()
+        self.ev_in0, self.ev_out = torch.cuda.Event(), torch.cuda.Event()
+        self.q_ev = [torch.cuda.Event() for _ in range(L)]
+        self.o_ev = [torch.cuda.Event() for _ in range(L)]
+
+    def step_e2e_cached(self, t: int):
+        """One decode step through the C ABI with the K/V cache in pinned host
+        memory and a device slot cache: upload this step's Q and Forecast
+        vectors; per layer, select the next layer's blocks, plan them against
+        the next layer's slots and fetch only the misses, all on the side
+        stream while this layer attends from its slots; read O back.  The
+        step ends once the next step's layer-0 blocks have landed, so a step
+        can be captured into a CUDA graph on its own."""
+        torch, abi, w = self.torch, self.abi, self.w
+        L, C = w.layers, self.C
+        main = torch.cuda.current_stream()
+        # inputs: the Forecast vectors first (select needs them at once); each
+        # layer's queries on a copy stream ahead of that layer's attention
+        self.F.copy_(self.h_F_steps[t % self.h_F_steps.shape[0]], non_blocking=True)
+        self.ev_in0.record(main)
+        self.copy.wait_event(self.ev_in0)
+        with torch.cuda.stream(self.copy):
+            for l in range(L):
+                self.Q[l].copy_(self.h_Q[l], non_blocking=True)
+                self.q_ev[l].record(self.copy)
+        for l in range(L):
+            nxt = (l + 1) % L
+            # select(l), the plan and the fetch of layer l+1 run on the side
+            # stream while attention(l) runs; both need layer l-1 finished
+            self.ev_pre[l].record(main)
+            self.side.wait_event(self.ev_pre[l])
+            with torch.cuda.stream(self.side):
+                abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
+                                           self.idx[nxt], self.ws_sel[l])
+                abi.sparda_cache_plan(self.p, C, self.idx[nxt], self.block_of[nxt],
+                                      self.hand[nxt], self.phys[nxt], self.fetch[nxt],
+                                      self.status)
+                abi.sparda_prefetch_cached(self.p, C, self.host_kv[nxt], self.idx[nxt],
+                                           self.phys[nxt], self.fetch[nxt], self.cache[nxt], 0,
+                                           self.status)
+                self.fetch_ev[nxt].record(self.side)
+            if l > 0:  # layer 0's blocks were joined at the end of the previous step
+                main.wait_event(self.fetch_ev[l])
+            main.wait_event(self.q_ev[l])
+            abi.sparda_sparse_attn_decode_cached(self.p, C, self.Q[l], self.cache[l],
+                                                 self.idx[l], self.phys[l], self.O[l],
+                                                 self.ws_att, self.status)
+            # this layer's output goes back while the next layers run
+            self.o_ev[l].record(main)
+            self.copy.wait_event(self.o_ev[l])
+            with torch.cuda.stream(self.copy):
+                self.h_O[l].copy_(self.O[l], non_blocking=True)
+        self.ev_out.record(self.copy)
+        main.wait_event(self.fetch_ev[0])
+        main.wait_event(self.ev_out)
+
+    def prime_cache(self):
+        """Cold start: plan and fetch layer 0's current set."""
+        w = self.w
+        self.abi.sparda_cache_plan(self.p, self.C, self.idx[0], self.block_of[0], self.hand[0],
+                                   self.phys[0], self.fetch[0], self.status)
+        self.abi.sparda_prefetch_cached(self.p, self.C, self.host_kv[0], self.idx[0], self.phys[0],
+                                        self.fetch[0], self.cache[0], 0, self.status)
+        self.torch.cuda.synchronize()
+
     # algorithmic bytes per launch
     def bytes_select(self):
         w = self.w
@@ -525,6 +613,7 @@ def run_sparda(args):
                "host_link_frac": fetched / (e_ms * 1e-3) / 1e9 / link_peak,
                "note": "K/V in pinned host memory; every layer's top-k blocks gathered over the "
                        "host link on a side stream (cold sets, no reuse across steps)"}
+        e2e["slot_cache"] = run_slot_cache_legs(loop, args, world, ms_step)
         loop.unregister()
 
     cpu = None
@@ -568,6 +657,61 @@ def run_sparda(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_slot_cache_legs(loop, args, world, resident_ms):
+    """The e2e loop with a device slot cache (2S slots per layer and group)
+    under a few drift rates of the Forecast vectors between decode steps:
+    per-step time, the share of top-k blocks that still cross the host
+    link, and the step time against the all-resident step."""
+    import torch
+    w = loop.w
+    L = w.layers
+    out = []
+    e_steps = max(3, min(args.steps, 10))
+    warm = max(args.warmup, 3)
+    for sigma in (0.0, 0.01, 0.03, 0.1):
+        n = warm + 2 * e_steps + 2
+        loop.setup_cache(2 * w.S, sigma, n)
+        loop.prime_cache()
+        # one CUDA graph per step (each uploads its own step's Forecast
+        # vectors), so host launch overhead stays out of the step
+        graphs = []
+        cap = torch.cuda.Stream()
+        with torch.cuda.stream(cap):
+            for i in range(n):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    loop.step_e2e_cached(i)
+                graphs.append(g)
+        torch.cuda.synchronize()
+        loop.block_of.fill_(-1)   # capture enqueued nothing; start the cache cold again
+        loop.hand.zero_()
+        loop.prime_cache()
+        t = [0]
+
+        def step():
+            graphs[t[0]].replay()
+            t[0] += 1
+        for _ in range(warm):
+            step()
+        ms = time_steps(step, e_steps, world) / e_steps
+        # the fetched share, measured on the steps that follow (untimed)
+        fetched = 0
+        for _ in range(e_steps):
+            step()
+            fetched += int(loop.fetch.sum().item())
+        del graphs
+        per_step = fetched / e_steps
+        topk_entries = L * w.B * w.G * w.k
+        out.append({"drift_sigma": sigma, "value": w.B * world / (ms / 1e3), "unit": "tokens/s",
+                    "ms_per_step": ms, "fetched_blocks_per_step": per_step,
+                    "fetched_frac_of_topk": per_step / topk_entries,
+                    "host_link_bytes_per_step": int(per_step * loop.blk_elems * 2),
+                    "step_vs_resident": ms / resident_ms})
+        del loop.cache, loop.block_of, loop.hand, loop.phys, loop.fetch, loop.h_F_steps
+        torch.cuda.empty_cache()
+    return out
 
 
 def host_link_peak_gbps(nbytes=1 << 30, reps=5):

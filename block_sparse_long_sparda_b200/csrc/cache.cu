@@ -20,8 +20,9 @@
 // The warp stages its slot map and list in shared memory, finds the hits in
 // parallel (lane per entry, a broadcast scan of the map), and one lane
 // places the misses in order (the policy is sequential by definition).  The
-// copy reuses the gather of prefetch.cu: 16-byte zero-copy loads from the
-// mapped host buffer, only for entries marked for fetching.
+// copy is the gather of prefetch.cu (16-byte zero-copy loads from the mapped
+// host buffer) over the entries marked for fetching, which each CTA first
+// lists a tile at a time.
 #include <algorithm>
 
 #include "common.cuh"
@@ -111,26 +112,52 @@ constexpr int kPfThreads = 256;
 constexpr int kPairBytes = 2 * kBlk * kD * 2;            // K + V block, 32 KB
 constexpr int kVecPerThread = kPairBytes / 16 / kPfThreads;  // 8
 
+// Entries are taken a tile at a time: the tile's fetch flags are read at
+// once (one load latency, not one per entry) and the marked entries listed
+// in shared memory, then each listed block is copied by the whole CTA.
+constexpr int kPfTile = 128;
+
 __global__ void __launch_bounds__(kPfThreads) prefetch_cached_kernel(
     const uint16_t *__restrict__ host_kv, const int32_t *__restrict__ idx,
     const int32_t *__restrict__ phys, const int32_t *__restrict__ fetch,
     uint16_t *__restrict__ cache, long long n_entries, int S, int C, int NB, int32_t *status) {
-  for (long long ent = blockIdx.x; ent < n_entries; ent += gridDim.x) {
-    if (!fetch[ent]) continue;
-    const int j = idx[ent], c = phys[ent];
-    if (j < 0 || j >= NB || c < 0 || c >= C) {
-      if (threadIdx.x == 0) flag_status(status, SPARDA_DEV_RANGE);
-      continue;
+  __shared__ long long s_ent[kPfTile];
+  __shared__ int s_j[kPfTile], s_c[kPfTile];
+  __shared__ int s_n;
+  const int tid = threadIdx.x;
+  for (long long base = (long long)blockIdx.x * kPfTile; base < n_entries;
+       base += (long long)gridDim.x * kPfTile) {
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    if (tid < kPfTile) {
+      const long long ent = base + tid;
+      if (ent < n_entries && fetch[ent]) {
+        const int j = idx[ent], c = phys[ent];
+        if (j < 0 || j >= NB || c < 0 || c >= C) {
+          flag_status(status, SPARDA_DEV_RANGE);
+        } else {
+          const int slot = atomicAdd(&s_n, 1);
+          s_ent[slot] = ent;
+          s_j[slot] = j;
+          s_c[slot] = c;
+        }
+      }
     }
-    const long long bg = ent / S;
-    const uint4 *src =
-        reinterpret_cast<const uint4 *>(host_kv + (bg * NB + j) * (long long)(kPairBytes / 2));
-    uint4 *dst = reinterpret_cast<uint4 *>(cache + (bg * C + c) * (long long)(kPairBytes / 2));
-    uint4 v[kVecPerThread];
+    __syncthreads();
+    const int n = s_n;
+    for (int q = 0; q < n; ++q) {
+      const long long bg = s_ent[q] / S;
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          host_kv + (bg * NB + s_j[q]) * (long long)(kPairBytes / 2));
+      uint4 *dst =
+          reinterpret_cast<uint4 *>(cache + (bg * C + s_c[q]) * (long long)(kPairBytes / 2));
+      uint4 v[kVecPerThread];
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) v[u] = ldg_plain(src + u * kPfThreads + threadIdx.x);
+      for (int u = 0; u < kVecPerThread; ++u) v[u] = ldg_plain(src + u * kPfThreads + tid);
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) stg_stream(dst + u * kPfThreads + threadIdx.x, v[u]);
+      for (int u = 0; u < kVecPerThread; ++u) stg_stream(dst + u * kPfThreads + tid, v[u]);
+    }
+    __syncthreads();  // the list is rebuilt for the next tile
   }
 }
 
@@ -170,7 +197,7 @@ cudaError_t launch_prefetch_cached(const sparda_params &p, int C, const uint16_t
     const int forced = env_int("SPARDA_PREFETCH_CTAS");
     n_ctas = forced > 0 ? forced : std::min(64, 16 + 2 * p.B);
   }
-  n_ctas = (int)std::min<long long>(n_ctas, n_entries);
+  n_ctas = (int)std::min<long long>(n_ctas, ceil_div_ll(n_entries, kPfTile));
   prefetch_cached_kernel<<<n_ctas, kPfThreads, 0, stream>>>(host_kv_dev, idx, phys, fetch, cache,
                                                             n_entries, S, C, NB, dev_status);
   return cudaGetLastError();
