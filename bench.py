@@ -63,7 +63,8 @@ def parse_args():
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
-                         "K/V per attention launch) and exit: the small case that ncu captures")
+                         "K/V per attention launch), then two passes of a 512-token prefill "
+                         "chunk of one sequence, and exit: the small cases ncu captures")
     return ap.parse_args()
 
 
@@ -875,7 +876,19 @@ def run_profile_case():
     torch.cuda.synchronize()
     st = int(loop.status.item())
     print("profile case: B=%d, %d select + %d attention launches, device status %d" % (w.B, 3, 3, st))
-    if st != 0:
+    del loop
+    torch.cuda.empty_cache()
+    # a prefill chunk of 512 tokens of one sequence (0.5 GB of K/V): two
+    # passes of its selection (score tiles, row ranking) and attention
+    pc = PrefillChunk(W.scaled(W.WORKLOADS["prefill_b4_t128k_c2k"], B=1, nq=512))
+    pc.compress()
+    for _ in range(2):
+        pc.select()
+        pc.attention()
+    torch.cuda.synchronize()
+    st2 = int(pc.status.item())
+    print("profile case: prefill B=1, 512 tokens, device status %d" % st2)
+    if st != 0 or st2 != 0:
         sys.exit(1)
 
 
