@@ -524,6 +524,7 @@ def oracle_baseline(loop: DecodeLoop, seconds: float):
 
 def run_sparda(args):
     import torch
+    from block_sparse_long_sparda_b200 import abi
     rank, world, local = dist_env()
     init_dist(world, local)
     from block_sparse_long_sparda_b200 import build
@@ -583,6 +584,22 @@ def run_sparda(args):
                 kernel_loop(which)
             kms = time_steps(lambda: kernel_loop(which), args.steps, world)
             kern_us[which] = kms / (args.steps * L) * 1e3
+        # decode append (new K/V rows + the incremental compressed key), timed
+        # by writing every layer's last-token rows back unchanged
+        pos = w.T - 1
+        c_last, r_last = pos // w.blk, pos % w.blk
+        kv_new = [loop.kv[l, :, :, c_last, :, r_last].clone() for l in range(L)]  # [B][G][2][d]
+
+        def append_all():
+            for l in range(L):
+                kv = loop.kv[l]
+                abi.sparda_append_kv(loop.p, pos, kv_new[l][:, :, 0].contiguous(),
+                                     kv_new[l][:, :, 1].contiguous(), kv,
+                                     kv.view(-1)[w.blk * w.d:], w.NB * loop.blk_elems,
+                                     loop.blk_elems, None, loop.kc[l])
+        for _ in range(3):
+            append_all()
+        kern_us["append"] = time_steps(append_all, args.steps, world) / (args.steps * L) * 1e3
     st = int(loop.status.item())
 
     ms_step = ms / args.steps
@@ -635,6 +652,7 @@ def run_sparda(args):
                                   "attention(l+1) waits for both",
                        "l2": "inputs larger than L2: 281 MB of selected K/V per layer, 4 layers"},
             "select_us_per_layer": sel_us,
+            "append_us_per_layer": kern_us["append"],
             "attn_us_per_layer": att_us,
             "select_GBps": sel_gbs,
             "step_GBps": step_gbs,

@@ -68,6 +68,7 @@ _PP = ctypes.POINTER(sparda_params)
 _SIGS = {
     "sparda_compress_keys": (_I, [_PP, _P, _LL, _LL, _P, _P, _P]),
     "sparda_forecast_select": (_I, [_PP, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "sparda_append_kv": (_I, [_PP, _I, _P, _P, _P, _P, _LL, _LL, _P, _P, _P]),
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
@@ -135,6 +136,14 @@ def sparda_compress_keys(p, K, bg_stride, tok_stride, kc_f32, kc_bf16, stream=No
     _check("sparda_compress_keys",
            lib().sparda_compress_keys(ctypes.byref(p), _ptr(K), int(bg_stride), int(tok_stride),
                                       _ptr(kc_f32), _ptr(kc_bf16), _stream(stream)))
+
+
+def sparda_append_kv(p, pos, K_new, V_new, K, V, bg_stride, blk_stride, kc_f32, kc_bf16,
+                     stream=None):
+    _check("sparda_append_kv",
+           lib().sparda_append_kv(ctypes.byref(p), int(pos), _ptr(K_new), _ptr(V_new), _ptr(K),
+                                  _ptr(V), int(bg_stride), int(blk_stride), _ptr(kc_f32),
+                                  _ptr(kc_bf16), _stream(stream)))
 
 
 def sparda_forecast_select(p, F, nq, nf, q_start, kc, idx, ws, stream=None):

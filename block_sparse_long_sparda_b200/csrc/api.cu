@@ -90,6 +90,26 @@ int sparda_compress_keys(const sparda_params *p, const void *K, long long bg_str
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const void *V_new,
+                     void *K, void *V, long long bg_stride, long long blk_stride, float *kc_f32,
+                     void *kc_bf16, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (pos < 0 || pos >= p->T) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!K_new || !V_new || !K || !V || (!kc_f32 && !kc_bf16)) return SPARDA_EINVAL;
+  if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K) || !aligned16(V) ||
+      (kc_f32 && !aligned16(kc_f32)) || (kc_bf16 && !aligned16(kc_bf16)))
+    return SPARDA_EINVAL;
+  if (!stride_ok(bg_stride) || !stride_ok(blk_stride) || blk_stride < (long long)kBlk * kD)
+    return SPARDA_EINVAL;
+  return from_cuda(launch_append(*p, pos, static_cast<const uint16_t *>(K_new),
+                                 static_cast<const uint16_t *>(V_new), static_cast<uint16_t *>(K),
+                                 static_cast<uint16_t *>(V), bg_stride, blk_stride, kc_f32,
+                                 static_cast<uint16_t *>(kc_bf16),
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
                            const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
                            sparda_stream_t stream) {

@@ -88,6 +88,60 @@ __global__ void __launch_bounds__(256, 3) compress_kernel(const uint16_t *__rest
   }
 }
 
+// One decode token appended: write its K and V rows at position `pos` and
+// recompute the compressed key of its block -- the one block whose mean
+// changes.  One warp per (b, g).  The block's earlier rows are summed from
+// memory in the same per-half, ascending-row order as compress_kernel and
+// the new row is added last in its half, so the result is bit-identical to
+// compressing the whole cache again.
+__global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict__ K_new,
+                                                     const uint16_t *__restrict__ V_new,
+                                                     uint16_t *__restrict__ K,
+                                                     uint16_t *__restrict__ V, long long bg_stride,
+                                                     long long blk_stride, int pos, int NB,
+                                                     long long n_pairs, float *__restrict__ kc32,
+                                                     uint16_t *__restrict__ kc16) {
+  const int lane = threadIdx.x & 31;
+  const long long bg = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (bg >= n_pairs) return;
+  const int half = lane >> 4, c8 = lane & 15;
+  const int c = pos / kBlk, r = pos - c * kBlk;  // block and row of the new token
+  const long long blk_off = bg * bg_stride + (long long)c * blk_stride + c8 * 8;
+  const uint4 knew = ldg_plain(K_new + bg * kD + c8 * 8);
+  if (half == 0) {
+    *reinterpret_cast<uint4 *>(K + blk_off + (long long)r * kD) = knew;
+  } else {
+    *reinterpret_cast<uint4 *>(V + blk_off + (long long)r * kD) = ldg_plain(V_new + bg * kD + c8 * 8);
+  }
+  // rows 0 .. r-1 of the block were written before this launch
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int t = half; t < r; t += 2) acc8(a, ldg_plain(K + blk_off + (long long)t * kD));
+  if ((r & 1) == half) acc8(a, knew);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+  if (half) return;
+  const float fn = (float)(r + 1);
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = a[e] / fn;
+  const long long item = bg * NB + c;
+  if (kc32) {
+    float4 *o = reinterpret_cast<float4 *>(kc32 + item * kD + c8 * 8);
+    o[0] = make_float4(m[0], m[1], m[2], m[3]);
+    o[1] = make_float4(m[4], m[5], m[6], m[7]);
+  }
+  if (kc16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e]));
+      uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e + 1]));
+      w[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(kc16 + item * kD + c8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
@@ -104,6 +158,18 @@ cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long
   else
     compress_kernel<false><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride,
                                                                     p.T, NB, items, kc32, kc16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const sparda_params &p, int pos, const uint16_t *K_new,
+                          const uint16_t *V_new, uint16_t *K, uint16_t *V, long long bg_stride,
+                          long long blk_stride, float *kc32, uint16_t *kc16, cudaStream_t stream) {
+  const long long pairs = (long long)p.B * p.G;
+  if (pairs == 0) return cudaSuccess;
+  const int NB = (p.T + kBlk - 1) / kBlk;
+  const int warps = 8;
+  append_kernel<<<(unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream>>>(
+      K_new, V_new, K, V, bg_stride, blk_stride, pos, NB, pairs, kc32, kc16);
   return cudaGetLastError();
 }
 

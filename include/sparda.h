@@ -119,6 +119,27 @@ int sparda_compress_keys(const sparda_params *p, const void *K, long long bg_str
                          sparda_stream_t stream);
 
 /*
+ * sparda_append_kv -- one decode token: write its K and V rows at position
+ * pos of every (b,g) and recompute the compressed key of the block holding
+ * pos (the only block whose mean changes), so selection can run on an up to
+ * date Kc without compressing the whole cache again.
+ *   [p4 "The fourth projection", Algorithm 2]: kv_cache.append(K_l, V_l);
+ *   k_compressed_cache.update_incremental(kv_cache).
+ * K_new, V_new  bf16 [B][G][d] device, the new token's key and value rows
+ * K, V     bf16 device caches; row t of (b,g) sits at
+ *            base + (b*G+g)*bg_stride + (t/blk)*blk_stride + (t%blk)*d
+ *          ([B][G][T][d]: bg_stride = T*d, blk_stride = blk*d; interleaved
+ *          [..][NB][2][blk][d]: V = K + blk*d, blk_stride = 2*blk*d)
+ * pos      the new token's position, 0 <= pos < T (T sizes the Kc arrays)
+ * kc_f32, kc_bf16  as for sparda_compress_keys, [B][G][NB][d]; only block
+ *          pos/blk is written.  The value is bit-identical to what
+ *          sparda_compress_keys computes over positions 0..pos.
+ */
+int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const void *V_new,
+                     void *K, void *V, long long bg_stride, long long blk_stride, float *kc_f32,
+                     void *kc_bf16, sparda_stream_t stream);
+
+/*
  * sparda_forecast_select -- block sets from Forecast scores.
  *   [p4 "The fourth projection", Eq. 4]:
  *     B_{l+1} = B_init U B_local U f_top(F_l Kc_{l+1}^T, k)

@@ -366,6 +366,93 @@ def test_prefetch_flags_out_of_range_and_rejects_pageable_memory():
 
 
 # --------------------------------------------------------------------------
+# decode append: new K/V rows and the incremental compressed key
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_append_matches_full_compression(interleaved):
+    """Append 150 tokens one at a time after a 100-token prefix: after every
+    append the cache holds the new rows and the compressed keys equal a full
+    compression of positions 0..pos, bit for bit (fp32 and bf16); at the end
+    they also match the oracle."""
+    rng = W.rng_for(50 + interleaved)
+    B, G, d, T0, T = 2, 3, 128, 100, 250
+    NB = (T + 63) // 64
+    p = abi.make_params(B, G, G, T, 1)
+    newK = W.normal_bf16(rng, (T - T0, B, G, d))
+    newV = W.normal_bf16(rng, (T - T0, B, G, d))
+    K0 = W.normal_bf16(rng, (B, G, T0, d))
+    V0 = W.normal_bf16(rng, (B, G, T0, d))
+    if interleaved:  # [B][G][NB][2][64][d]
+        cache = torch.zeros(B, G, NB, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+        for t in range(T0):
+            cache[:, :, t // 64, 0, t % 64] = dev_bf16(K0[:, :, t])
+            cache[:, :, t // 64, 1, t % 64] = dev_bf16(V0[:, :, t])
+        Kd, Vd = cache, cache.view(-1)[64 * d:]
+        bg, blk = NB * 2 * 64 * d, 2 * 64 * d
+    else:
+        Kd = torch.zeros(B, G, T, d, dtype=torch.bfloat16, device="cuda")
+        Vd = torch.zeros(B, G, T, d, dtype=torch.bfloat16, device="cuda")
+        Kd[:, :, :T0] = dev_bf16(K0)
+        Vd[:, :, :T0] = dev_bf16(V0)
+        bg, blk = T * d, 64 * d
+    kc32 = torch.zeros(B, G, NB, d, dtype=torch.float32, device="cuda")
+    kc16 = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
+    # the prefix: compress positions 0..T0-1
+    pp = abi.make_params(B, G, G, T0, 1)
+    if interleaved:
+        # each block of 64 rows compresses like a short sequence of its own
+        for j in range((T0 + 63) // 64):
+            n = min(64, T0 - 64 * j)
+            pj = abi.make_params(B, G, G, n, 1)
+            tmp32 = torch.zeros(B, G, 1, d, dtype=torch.float32, device="cuda")
+            tmp16 = torch.zeros(B, G, 1, d, dtype=torch.bfloat16, device="cuda")
+            abi.sparda_compress_keys(pj, cache[:, :, j, 0], NB * 2 * 64 * d, d, tmp32, tmp16)
+            kc32[:, :, j] = tmp32[:, :, 0]
+            kc16[:, :, j] = tmp16[:, :, 0]
+    else:
+        tmp32 = torch.zeros(B, G, (T0 + 63) // 64, d, dtype=torch.float32, device="cuda")
+        tmp16 = torch.zeros(B, G, (T0 + 63) // 64, d, dtype=torch.bfloat16, device="cuda")
+        abi.sparda_compress_keys(pp, Kd, bg, d, tmp32, tmp16)
+        kc32[:, :, :(T0 + 63) // 64] = tmp32
+        kc16[:, :, :(T0 + 63) // 64] = tmp16
+    for i, pos in enumerate(range(T0, T)):
+        abi.sparda_append_kv(p, pos, dev_bf16(newK[i]), dev_bf16(newV[i]), Kd, Vd, bg, blk, kc32,
+                             kc16)
+        if pos % 37 == 0 or pos == T - 1 or pos % 64 in (0, 63):
+            torch.cuda.synchronize()
+            # the full compression of positions 0..pos, from the same cache
+            c = pos // 64
+            n = pos - 64 * c + 1
+            if interleaved:
+                pj = abi.make_params(B, G, G, n, 1)
+                ref32 = torch.zeros(B, G, 1, d, dtype=torch.float32, device="cuda")
+                ref16 = torch.zeros(B, G, 1, d, dtype=torch.bfloat16, device="cuda")
+                abi.sparda_compress_keys(pj, cache[:, :, c, 0], NB * 2 * 64 * d, d, ref32, ref16)
+                ref32, ref16 = ref32[:, :, 0], ref16[:, :, 0]
+            else:
+                pf = abi.make_params(B, G, G, pos + 1, 1)
+                r32 = torch.zeros(B, G, c + 1, d, dtype=torch.float32, device="cuda")
+                r16 = torch.zeros(B, G, c + 1, d, dtype=torch.bfloat16, device="cuda")
+                abi.sparda_compress_keys(pf, Kd, bg, d, r32, r16)
+                ref32, ref16 = r32[:, :, c], r16[:, :, c]
+            assert torch.equal(kc32[:, :, c], ref32), pos
+            assert torch.equal(kc16[:, :, c], ref16), pos
+    torch.cuda.synchronize()
+    # rows landed where they belong, and the keys match the oracle
+    Kall = np.concatenate([K0, newK.transpose(1, 2, 0, 3)], axis=2)
+    Vall = np.concatenate([V0, newV.transpose(1, 2, 0, 3)], axis=2)
+    if interleaved:
+        got_k = host_bits(cache[:, :, :, 0]).reshape(B, G, NB * 64, d)[:, :, :T]
+        got_v = host_bits(cache[:, :, :, 1]).reshape(B, G, NB * 64, d)[:, :, :T]
+    else:
+        got_k, got_v = host_bits(Kd), host_bits(Vd)
+    assert np.array_equal(got_k, Kall) and np.array_equal(got_v, Vall)
+    o64, o16 = oracle.compress_keys(Kall)
+    check_compressed(kc32.cpu().numpy(), host_bits(kc16), o64, o16)
+
+
+# --------------------------------------------------------------------------
 # device slot cache across decode steps
 # --------------------------------------------------------------------------
 
