@@ -96,7 +96,6 @@ constexpr int kNQ = 16;                 // MMA N: the heads of a group, zero pad
 constexpr int kTile = 8192;             // 64 rows x 64 bf16, one swizzled tile
 constexpr int kUnitBytes = 4 * kTile;   // K lo | V lo | K hi | V hi
 constexpr int kMaxEnt = 128;            // list entries one CTA may own (one per thread)
-constexpr int kThreads = 128;
 
 struct TcArgs {
   const uint16_t *Q;

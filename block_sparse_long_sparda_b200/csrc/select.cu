@@ -41,7 +41,6 @@ namespace {
 
 constexpr int kSelThreads = 256;
 constexpr int kMaxCand = 24576;   // candidates one problem may have (keys fit in shared memory)
-constexpr int kMaxNf = 16;
 
 struct SelArgs {
   const uint16_t *F;
