@@ -62,6 +62,12 @@ def _load():
         lib.oracle_select.restype = None
         lib.oracle_gather_blocks.argtypes = [I, I, I, I, I, I, I, I, I, I, P, P, P]
         lib.oracle_gather_blocks.restype = None
+        lib.oracle_window_count.argtypes = [I, I, I]
+        lib.oracle_window_count.restype = I
+        lib.oracle_compress_windows.argtypes = [I, I, I, I, I, I, P, LL, LL, P, P]
+        lib.oracle_compress_windows.restype = None
+        lib.oracle_select_windows.argtypes = [I, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P]
+        lib.oracle_select_windows.restype = None
         lib.oracle_cache_plan.argtypes = [I, I, I, I, I, P, P, P, P, P]
         lib.oracle_cache_plan.restype = I
         lib.oracle_gather_cached.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P]
@@ -119,6 +125,41 @@ def compress_keys(K: np.ndarray, blk: int = 64, shape=None, strides=None):
     _load().oracle_compress_keys(B, G, T, d, blk, _ptr(K), bg_stride, tok_stride, _ptr(kc),
                                  _ptr(kcb))
     return kc, kcb
+
+
+def window_count(T: int, win: int = 32, stride: int = 16) -> int:
+    return int(_load().oracle_window_count(int(T), int(win), int(stride)))
+
+
+def compress_windows(K: np.ndarray, win: int = 32, stride: int = 16):
+    """Window-grid compressed keys: mean of positions [w*stride, w*stride+win).
+
+    K: uint16 [B][G][T][d].  Returns (kw_f64 [B][G][NW][d], kw_bf16 [B][G][NW][d])."""
+    K = _u16(K)
+    B, G, T, d = K.shape
+    NW = window_count(T, win, stride)
+    kw = np.empty((B, G, NW, d), np.float64)
+    kwb = np.empty((B, G, NW, d), np.uint16)
+    _load().oracle_compress_windows(B, G, T, d, win, stride, _ptr(K), T * d, d, _ptr(kw), _ptr(kwb))
+    return kw, kwb
+
+
+def select_windows(F: np.ndarray, kw: np.ndarray, T: int, k: int, n_init: int, n_local: int,
+                   q_start: int, blk: int = 64, win: int = 32, stride: int = 16):
+    """Block sets from window-grid keys: a block's score is the largest score
+    of the windows inside it.  F [B][nq][G][nf][d]; kw [B][G][NW][d].
+    Returns (idx [B][nq][G][S], kth, kth1) as select()."""
+    F = _u16(F)
+    kw = _u16(kw)
+    B, nq, G, nf, d = F.shape
+    assert kw.shape[:2] == (B, G) and kw.shape[2] == window_count(T, win, stride)
+    S = k + n_init + n_local
+    idx = np.empty((B, nq, G, S), np.int32)
+    kth = np.empty((B, nq, G), np.float64)
+    kth1 = np.empty((B, nq, G), np.float64)
+    _load().oracle_select_windows(B, nq, G, nf, d, blk, win, stride, T, k, n_init, n_local,
+                                  q_start, _ptr(F), _ptr(kw), _ptr(idx), _ptr(kth), _ptr(kth1))
+    return idx, kth, kth1
 
 
 def select(F: np.ndarray, kc: np.ndarray, k: int, n_init: int, n_local: int, q_start: int,

@@ -175,6 +175,50 @@ static void compress_item(void *vctx, long long item) {
   }
 }
 
+/* o1w: the window grid of the real models (f3): compressed key w is the   */
+/*   mean of the keys at positions [w*stride, w*stride + win), complete     */
+/*   windows only: NW = (T - win) / stride + 1 for T >= win, else 0.        */
+/*   [p4] "One Forecast head per GQA group": the test models pool their     */
+/*   keys with a 32-token window at stride 16.  kw [B][G][NW][d].           */
+typedef struct {
+  int T, d, win, stride, NW;
+  const uint16_t *K;
+  long long bg_stride, tok_stride;
+  double *kw;
+  uint16_t *kw_bf16;
+} window_ctx;
+
+static void window_item(void *vctx, long long item) {
+  window_ctx *c = (window_ctx *)vctx;
+  long long bg = item / c->NW;
+  int w = (int)(item % c->NW);
+  int t0 = w * c->stride;
+  for (int x = 0; x < c->d; ++x) {
+    double s = 0.0;
+    for (int t = 0; t < c->win; ++t)
+      s += bf16_to_double(c->K[bg * c->bg_stride + (long long)(t0 + t) * c->tok_stride + x]);
+    double mean = s / (double)c->win;
+    long long o = item * c->d + x;
+    if (c->kw) c->kw[o] = mean;
+    if (c->kw_bf16) c->kw_bf16[o] = oracle_double_to_bf16(mean);
+  }
+}
+
+int oracle_window_count(int T, int win, int stride) {
+  return T >= win ? (T - win) / stride + 1 : 0;
+}
+
+void oracle_compress_windows(int B, int G, int T, int d, int win, int stride, const uint16_t *K,
+                             long long bg_stride, long long tok_stride, double *kw,
+                             uint16_t *kw_bf16) {
+  window_ctx c;
+  c.T = T; c.d = d; c.win = win; c.stride = stride;
+  c.NW = oracle_window_count(T, win, stride);
+  c.K = K; c.bg_stride = bg_stride; c.tok_stride = tok_stride;
+  c.kw = kw; c.kw_bf16 = kw_bf16;
+  parallel_for((long long)B * G * c.NW, window_item, &c);
+}
+
 void oracle_compress_keys(int B, int G, int T, int d, int blk, const uint16_t *K,
                           long long bg_stride, long long tok_stride, double *kc,
                           uint16_t *kc_bf16) {
@@ -249,10 +293,23 @@ static int cmp_int(const void *a, const void *b) {
 
 typedef struct {
   int B, nq, G, nf, d, blk, NB, k, n_init, n_local, q_start, S;
+  int win, stride, NW;   /* window grid (f3); win = 0: one key per block */
   const uint16_t *F, *kc;
   int32_t *idx;
   double *kth, *kth1;
 } select_ctx;
+
+/* score of key row r for the scoring vectors f: sum over the nf vectors */
+static double row_score(const select_ctx *c, const uint16_t *f, const uint16_t *keys, long long r) {
+  double s = 0.0;
+  for (int h = 0; h < c->nf; ++h) {
+    double dot = 0.0;
+    for (int x = 0; x < c->d; ++x)
+      dot += bf16_to_double(f[h * c->d + x]) * bf16_to_double(keys[r * c->d + x]);
+    s += dot;
+  }
+  return s;
+}
 
 static void select_item(void *vctx, long long item) {
   select_ctx *c = (select_ctx *)vctx;
@@ -265,17 +322,25 @@ static void select_item(void *vctx, long long item) {
   int ncand = bp.cand_hi - bp.cand_lo;
 
   const uint16_t *f = c->F + (((long long)b * c->nq + i) * c->G + g) * c->nf * c->d;
-  const uint16_t *kc = c->kc + ((long long)b * c->G + g) * c->NB * c->d;
+  const long long rows = c->win ? c->NW : c->NB;  /* key rows per (b, g) */
+  const uint16_t *kc = c->kc + ((long long)b * c->G + g) * rows * c->d;
 
   scored *cand = (scored *)malloc(sizeof(scored) * (ncand > 0 ? ncand : 1));
   for (int n = 0; n < ncand; ++n) {
     int j = bp.cand_lo + n;
-    double s = 0.0;
-    for (int h = 0; h < c->nf; ++h) {
-      double dot = 0.0;
-      for (int x = 0; x < c->d; ++x)
-        dot += bf16_to_double(f[h * c->d + x]) * bf16_to_double(kc[(long long)j * c->d + x]);
-      s += dot;
+    double s;
+    if (c->win == 0) {
+      s = row_score(c, f, kc, j);
+    } else {
+      /* window grid (f3): the block's score is the largest score of the
+         windows lying inside it, [ceil(j*blk/stride), ...) while the window
+         ends by the block's end */
+      s = -INFINITY;
+      for (int w = (j * c->blk + c->stride - 1) / c->stride;
+           w < c->NW && w * c->stride + c->win <= (j + 1) * c->blk; ++w) {
+        double sw = row_score(c, f, kc, w);
+        if (sw > s) s = sw;
+      }
     }
     if (s == 0.0) s = 0.0; /* one zero */
     cand[n].score = s;
@@ -307,7 +372,25 @@ void oracle_select(int B, int nq, int G, int nf, int d, int blk, int NB, int k, 
   c.B = B; c.nq = nq; c.G = G; c.nf = nf; c.d = d; c.blk = blk; c.NB = NB; c.k = k;
   c.n_init = n_init; c.n_local = n_local; c.q_start = q_start;
   c.S = k + n_init + n_local;
+  c.win = 0; c.stride = 0; c.NW = 0;
   c.F = F; c.kc = kc; c.idx = idx; c.kth = kth; c.kth1 = kth1;
+  parallel_for((long long)B * nq * G, select_item, &c);
+}
+
+/* o2w: the same selection on the window grid (f3): a candidate block's score
+ * is the largest score of the windows lying inside it (max-pooling of the
+ * window scores to blocks, [p4] "Training: distilling the selector you
+ * already have" names the selector's final max-pooling step).  kw is
+ * [B][G][NW][d]; T is the sequence length that sets NB and NW. */
+void oracle_select_windows(int B, int nq, int G, int nf, int d, int blk, int win, int stride, int T,
+                           int k, int n_init, int n_local, int q_start, const uint16_t *F,
+                           const uint16_t *kw, int32_t *idx, double *kth, double *kth1) {
+  select_ctx c;
+  c.B = B; c.nq = nq; c.G = G; c.nf = nf; c.d = d; c.blk = blk; c.NB = (T + blk - 1) / blk;
+  c.k = k; c.n_init = n_init; c.n_local = n_local; c.q_start = q_start;
+  c.S = k + n_init + n_local;
+  c.win = win; c.stride = stride; c.NW = oracle_window_count(T, win, stride);
+  c.F = F; c.kc = kw; c.idx = idx; c.kth = kth; c.kth1 = kth1;
   parallel_for((long long)B * nq * G, select_item, &c);
 }
 

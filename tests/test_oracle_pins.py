@@ -494,3 +494,90 @@ def test_gather_cached_copies_only_fetched_entries():
                 assert np.array_equal(out[0, g, c], host[0, g, idx[0, g, s]])
     assert not out[0, 0, 0].any() and not out[0, 0, 2].any() and not out[0, 0, 4].any()
     assert not out[0, 1, 1].any() and not out[0, 1, 3].any()
+
+
+# --------------------------------------------------------------------------
+# the window grid of the real models (32-token windows, stride 16) with
+# max-pooled block scores
+# --------------------------------------------------------------------------
+
+def test_window_counts():
+    assert [oracle.window_count(T) for T in (0, 31, 32, 47, 48, 64, 4096)] == [0, 0, 1, 1, 2, 3, 255]
+
+
+def test_compress_windows_linear_ramp_closed_form():
+    """Keys equal to their position (exact in bf16 below 256): window w
+    averages positions 16w .. 16w+31, so its mean is 16w + 15.5."""
+    T, d = 200, 4
+    K = np.empty((1, 1, T, d), np.uint16)
+    for t in range(T):
+        K[0, 0, t, :] = oracle.double_to_bf16(float(t))
+    kw, kwb = oracle.compress_windows(K)
+    NW = (T - 32) // 16 + 1
+    assert kw.shape == (1, 1, NW, d)
+    for w in range(NW):
+        assert np.all(kw[0, 0, w] == 16 * w + 15.5)
+        assert np.all(kwb[0, 0, w] == oracle.double_to_bf16(16 * w + 15.5))
+
+
+def _window_keys(values, d=8):
+    """kw [1][1][NW][d] whose first coordinate is values[w], the rest zero."""
+    kw = np.zeros((1, 1, len(values), d), np.uint16)
+    for w, v in enumerate(values):
+        kw[0, 0, w, 0] = oracle.double_to_bf16(float(v))
+    return kw
+
+
+def test_select_windows_max_inside_block_not_crossing_windows():
+    """F = e_0, so a window's score is its first coordinate.  Block j holds
+    windows 4j, 4j+1, 4j+2 (4j+3 straddles blocks j and j+1 and belongs to
+    neither).  Block 5 has one high window, block 3 three medium ones, block 6
+    only a huge straddling window: the top-2 are {5, 3}, not 6."""
+    T = 64 * 12
+    NW = oracle.window_count(T)
+    vals = [0.0] * NW
+    vals[4 * 5 + 1] = 100.0
+    for w in (12, 13, 14):
+        vals[w] = 10.0
+    vals[4 * 6 + 3] = 1000.0          # the window starting at 64*6 + 48
+    kw = _window_keys(vals)
+    F = np.zeros((1, 1, 1, 1, 8), np.uint16)
+    F[..., 0] = oracle.double_to_bf16(1.0)
+    idx, kth, kth1 = oracle.select_windows(F, kw, T, k=2, n_init=1, n_local=2, q_start=T - 1)
+    assert idx.reshape(-1).tolist() == [0, 3, 5, 10, 11]
+    assert kth[0, 0, 0] == 10.0
+
+
+def test_select_windows_takes_the_max_not_the_mean():
+    """Block 2's windows score (9, 0, 0), block 4's (6, 6, 6): with k = 1 the
+    max picks block 2 (a mean would pick block 4)."""
+    T = 64 * 10
+    vals = [0.0] * oracle.window_count(T)
+    vals[8] = 9.0
+    vals[16] = vals[17] = vals[18] = 6.0
+    F = np.zeros((1, 1, 1, 1, 8), np.uint16)
+    F[..., 0] = oracle.double_to_bf16(1.0)
+    idx, _, _ = oracle.select_windows(F, _window_keys(vals), T, k=1, n_init=1, n_local=2,
+                                      q_start=T - 1)
+    assert idx.reshape(-1).tolist() == [0, 2, 8, 9]
+
+
+def test_select_windows_equals_block_selection_when_windows_agree():
+    """If the three windows inside every block hold the same key v_j, the
+    window selection is the block selection with Kc[j] = v_j."""
+    rng = np.random.default_rng(7)
+    B, G, nq, d, NB = 2, 3, 2, 16, 40
+    T = NB * 64
+    NW = oracle.window_count(T)
+    kc = rng.integers(0, 65535, (B, G, NB, d), dtype=np.uint16)
+    kc = np.where((kc & 0x7F80) == 0x7F80, 0, kc).astype(np.uint16)   # finite values only
+    kw = rng.integers(0, 65535, (B, G, NW, d), dtype=np.uint16)
+    kw = np.where((kw & 0x7F80) == 0x7F80, 0, kw).astype(np.uint16)
+    for j in range(NB):
+        for w in (4 * j, 4 * j + 1, 4 * j + 2):
+            if w < NW:
+                kw[:, :, w] = kc[:, :, j]
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    a = oracle.select_windows(F, kw, T, k=7, n_init=1, n_local=2, q_start=T - nq)
+    b = oracle.select(F, kc, 7, 1, 2, T - nq)
+    assert np.array_equal(a[0], b[0])
