@@ -60,6 +60,11 @@ def parse_args():
                     help="also measure the selection-only sweep (Kc blocks 128..16384 x "
                          "batch 1..16, Forecast vs the 4-head baseline selector); prints an "
                          "extra JSON line")
+    ap.add_argument("--windows", action="store_true",
+                    help="also measure the window grid of the real models (32-token windows "
+                         "at stride 16, max-pooled to blocks): window compression, decode "
+                         "selection at B=16, T=128K, and the prefill chunk's selection; prints "
+                         "an extra JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
@@ -673,6 +678,8 @@ def run_sparda(args):
         print(json.dumps(run_prefill(args.steps)), flush=True)
     if rank == 0 and world == 1 and args.sweep:
         print(json.dumps(run_sweep()), flush=True)
+    if rank == 0 and world == 1 and args.windows:
+        print(json.dumps(run_windows(args.steps)), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -840,6 +847,57 @@ def run_prefill(steps):
         "chunk_us": s_us + a_us, "tokens_per_s": w.B * w.nq / ((s_us + a_us) * 1e-6),
         "device_status": st, "data": "synthetic", "dtype": "bf16",
     }
+
+
+def run_windows(steps):
+    """The window grid: decode selection at the decode loop's shapes and the
+    prefill chunk's, plus the window compression of the chunk's keys."""
+    import torch
+    from block_sparse_long_sparda_b200 import abi
+    dev = torch.device("cuda")
+    n = max(3, min(steps, 20))
+    out = {"metric": "window-grid selection (32-token windows, stride 16, max-pooled to blocks)",
+           "data": "synthetic", "dtype": "bf16"}
+    # decode: B=16, T=128K, one Forecast vector per group
+    w = WORKLOAD
+    NW = (w.T - 32) // 16 + 1
+    p = abi.make_params(w.B, w.Hq, w.G, w.T, w.k, w.n_init, w.n_local)
+    kws = []
+    for s_ in range(2):  # two layers' window keys (536 MB), alternated
+        kw = torch.empty(w.B, w.G, NW, w.d, dtype=torch.bfloat16, device=dev)
+        W.torch_normal_bf16_(kw, 3000 + s_)
+        kws.append(kw)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(3100)
+    F = torch.randn(w.B, w.G, w.d, generator=gen, device=dev).to(torch.bfloat16)
+    idx = torch.empty(w.B, w.G, w.S, dtype=torch.int32, device=dev)
+    ws = [abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, 1, 1) for _ in range(2)]
+    t = [0]
+
+    def sel():
+        l = t[0] & 1
+        abi.sparda_forecast_select_windows(p, F, 1, 1, w.T - 1, kws[l], 32, 16, idx, ws[l])
+        t[0] += 1
+    us = time_back_to_back(sel, n)
+    nbytes = w.B * w.G * NW * w.d * 2
+    out.update({"decode_select_us": us, "decode_select_GBps": nbytes / (us * 1e-6) / 1e9,
+                "decode_window_key_bytes": nbytes})
+    del kws
+    torch.cuda.empty_cache()
+    # prefill chunk: window compression of its keys and per-token selection
+    pc = PrefillChunk()
+    pw = pc.w
+    NWp = (pw.T - 32) // 16 + 1
+    kwp = torch.empty(pw.B, pw.G, NWp, pw.d, dtype=torch.bfloat16, device=dev)
+    wsp = abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, pc.p, pw.nq, 1)
+    c_us = time_back_to_back(lambda: abi.sparda_compress_windows(
+        pc.p, pc.K, pw.T * pw.d, pw.d, 32, 16, None, kwp), n)
+    s_us = time_back_to_back(lambda: abi.sparda_forecast_select_windows(
+        pc.p, pc.F, pw.nq, 1, pc.q0, kwp, 32, 16, pc.idx, wsp), max(3, min(n, 10)))
+    out.update({"prefill_compress_windows_us": c_us,
+                "prefill_compress_windows_GBps": pw.B * pw.G * pw.T * pw.d * 2 / (c_us * 1e-6) / 1e9,
+                "prefill_select_us": s_us})
+    return out
 
 
 def run_sweep():

@@ -34,6 +34,7 @@ SPARDA_OP_SELECT = 1
 SPARDA_OP_PREFETCH = 2
 SPARDA_OP_ATTN_DECODE = 3
 SPARDA_OP_ATTN_PREFILL = 4
+SPARDA_OP_SELECT_WINDOWS = 5
 
 SPARDA_ADDR_LOGICAL = 0
 SPARDA_ADDR_SLOT = 1
@@ -69,6 +70,8 @@ _SIGS = {
     "sparda_compress_keys": (_I, [_PP, _P, _LL, _LL, _P, _P, _P]),
     "sparda_forecast_select": (_I, [_PP, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "sparda_append_kv": (_I, [_PP, _I, _P, _P, _P, _P, _LL, _LL, _P, _P, _P]),
+    "sparda_compress_windows": (_I, [_PP, _P, _LL, _LL, _I, _I, _P, _P, _P]),
+    "sparda_forecast_select_windows": (_I, [_PP, _P, _I, _I, _I, _P, _I, _I, _P, _P, _SZ, _P]),
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
@@ -144,6 +147,21 @@ def sparda_append_kv(p, pos, K_new, V_new, K, V, bg_stride, blk_stride, kc_f32, 
            lib().sparda_append_kv(ctypes.byref(p), int(pos), _ptr(K_new), _ptr(V_new), _ptr(K),
                                   _ptr(V), int(bg_stride), int(blk_stride), _ptr(kc_f32),
                                   _ptr(kc_bf16), _stream(stream)))
+
+
+def sparda_compress_windows(p, K, bg_stride, tok_stride, win, stride, kw_f32, kw_bf16,
+                            stream=None):
+    _check("sparda_compress_windows",
+           lib().sparda_compress_windows(ctypes.byref(p), _ptr(K), int(bg_stride), int(tok_stride),
+                                         int(win), int(stride), _ptr(kw_f32), _ptr(kw_bf16),
+                                         _stream(stream)))
+
+
+def sparda_forecast_select_windows(p, F, nq, nf, q_start, kw, win, stride, idx, ws, stream=None):
+    _check("sparda_forecast_select_windows",
+           lib().sparda_forecast_select_windows(ctypes.byref(p), _ptr(F), int(nq), int(nf),
+                                                int(q_start), _ptr(kw), int(win), int(stride),
+                                                _ptr(idx), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def sparda_forecast_select(p, F, nq, nf, q_start, kc, idx, ws, stream=None):

@@ -65,6 +65,8 @@ size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf) {
   switch (op) {
     case SPARDA_OP_SELECT:
       return nq < 1 ? 0 : plan_select(*p, nq, nf < 1 ? 1 : nf).ws_bytes;
+    case SPARDA_OP_SELECT_WINDOWS:
+      return nq < 1 ? 0 : plan_select(*p, nq, nf < 1 ? 1 : nf, 4).ws_bytes;
     case SPARDA_OP_ATTN_DECODE:
       return plan_decode(*p).ws_bytes;
     case SPARDA_OP_ATTN_PREFILL:
@@ -108,6 +110,44 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
                                  static_cast<uint16_t *>(V), bg_stride, blk_stride, kc_f32,
                                  static_cast<uint16_t *>(kc_bf16),
                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_compress_windows(const sparda_params *p, const void *K, long long bg_stride,
+                            long long tok_stride, int win, int stride, float *kw_f32,
+                            void *kw_bf16, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
+  if (p->B == 0) return SPARDA_OK;
+  if (!K || (!kw_f32 && !kw_bf16)) return SPARDA_EINVAL;
+  if (!aligned16(K) || (kw_f32 && !aligned16(kw_f32)) || (kw_bf16 && !aligned16(kw_bf16)))
+    return SPARDA_EINVAL;
+  if (!stride_ok(tok_stride) || !stride_ok(bg_stride) || tok_stride < kD) return SPARDA_EINVAL;
+  if (p->G > 1 && bg_stride < (long long)p->T * tok_stride) return SPARDA_EINVAL;
+  return from_cuda(launch_compress_runs(*p, static_cast<const uint16_t *>(K), bg_stride,
+                                        tok_stride, win, stride, kw_f32,
+                                        static_cast<uint16_t *>(kw_bf16),
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq, int nf,
+                                   int q_start, const void *kw, int win, int stride,
+                                   int32_t *idx, void *ws, size_t ws_bytes,
+                                   sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
+  if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
+  if (nf > 16) return SPARDA_EUNSUPPORTED;
+  if (p->B == 0) return SPARDA_OK;
+  if (!F || !kw || !idx) return SPARDA_EINVAL;
+  if (!aligned16(F) || !aligned16(kw) || !aligned16(idx)) return SPARDA_EINVAL;
+  const SelectPlan pl = plan_select(*p, nq, nf, 4);
+  if (!select_supported(pl)) return SPARDA_EUNSUPPORTED;
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), nq, nf, q_start,
+                                 static_cast<const uint16_t *>(kw), idx, ws,
+                                 reinterpret_cast<cudaStream_t>(stream), 4));
 }
 
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,

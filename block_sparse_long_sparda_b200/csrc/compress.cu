@@ -32,19 +32,23 @@ __device__ __forceinline__ void acc8(float (&a)[8], uint4 v) {
   a[7] += bf16_hi(v.w);
 }
 
+// An item is a run of `rows` positions starting at j * step: a block (rows =
+// step = 64) or a window of the window grid (rows = 32, step = 16); NB items
+// per (b, g).
 template <bool kContig>
 __global__ void __launch_bounds__(256, 3) compress_kernel(const uint16_t *__restrict__ K,
                                                        long long bg_stride, long long tok_stride,
                                                        int T, int NB, long long n_items,
                                                        float *__restrict__ kc32,
-                                                       uint16_t *__restrict__ kc16) {
+                                                       uint16_t *__restrict__ kc16, int rows,
+                                                       int step) {
   const int lane = threadIdx.x & 31;
   const long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (item >= n_items) return;
   const long long bg = item / NB;
   const int j = (int)(item - bg * NB);
-  const int t0 = j * kBlk;
-  const int n = min(kBlk, T - t0);
+  const int t0 = j * step;
+  const int n = min(rows, T - t0);
   const int half = lane >> 4;
   const int c8 = lane & 15;
   if (kContig) tok_stride = kD;  // rows packed: constant offsets, fewer live registers
@@ -147,17 +151,24 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict_
 cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
                             long long tok_stride, float *kc32, uint16_t *kc16,
                             cudaStream_t stream) {
-  const int NB = (p.T + kBlk - 1) / kBlk;
+  return launch_compress_runs(p, K, bg_stride, tok_stride, kBlk, kBlk, kc32, kc16, stream);
+}
+
+cudaError_t launch_compress_runs(const sparda_params &p, const uint16_t *K, long long bg_stride,
+                                 long long tok_stride, int rows, int step, float *kc32,
+                                 uint16_t *kc16, cudaStream_t stream) {
+  // blocks: ceil(T / 64) (the last may be partial); windows: complete ones
+  const int NB = rows == step ? (p.T + step - 1) / step : (p.T >= rows ? (p.T - rows) / step + 1 : 0);
   const long long items = (long long)p.B * p.G * NB;
   if (items == 0) return cudaSuccess;
   const int warps = 8;
   const long long grid = ceil_div_ll(items, warps);
   if (tok_stride == kD)
     compress_kernel<true><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride, p.T,
-                                                                   NB, items, kc32, kc16);
+                                                                   NB, items, kc32, kc16, rows, step);
   else
-    compress_kernel<false><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride,
-                                                                    p.T, NB, items, kc32, kc16);
+    compress_kernel<false><<<(unsigned)grid, warps * 32, 0, stream>>>(
+        K, bg_stride, tok_stride, p.T, NB, items, kc32, kc16, rows, step);
   return cudaGetLastError();
 }
 

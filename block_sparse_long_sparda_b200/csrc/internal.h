@@ -50,6 +50,12 @@ cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long
                             long long tok_stride, float *kc32, uint16_t *kc16,
                             cudaStream_t stream);
 
+// mean of every run of `rows` positions starting at multiples of `step`
+// (blocks: 64/64, the window grid: 32/16)
+cudaError_t launch_compress_runs(const sparda_params &p, const uint16_t *K, long long bg_stride,
+                                 long long tok_stride, int rows, int step, float *kc32,
+                                 uint16_t *kc16, cudaStream_t stream);
+
 // one decode token: write its K/V rows at `pos`, recompute its block's key
 cudaError_t launch_append(const sparda_params &p, int pos, const uint16_t *K_new,
                           const uint16_t *V_new, uint16_t *K, uint16_t *V, long long bg_stride,
@@ -65,17 +71,22 @@ struct SelectPlan {
   int tensor_scores;     // 1: chunk of query tokens scored by the tcgen05 product
   size_t ws_bytes;
 };
-SelectPlan plan_select(const sparda_params &p, int nq, int nf);
+// pool = 1: one compressed key per block; pool = 4: the window grid (32-token
+// windows at stride 16), a block scoring as the best window inside it
+SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool = 1);
+// windows of 32 tokens at stride 16 that fit in T tokens
+inline int window_count(int T) { return T >= 32 ? (T - 32) / 16 + 1 : 0; }
 // prefill (select_prefill.cu): scores of a token chunk on the tensor cores,
 // then one warp per (token, group) row ranks them
 constexpr int kPrefillTensorMinQ = 64;  // query tokens from which the product pays
-size_t prefill_select_ws_bytes(const sparda_params &p, int nq);
+size_t prefill_select_ws_bytes(const sparda_params &p, int nq, int pool = 1);
 cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
-                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream);
+                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream,
+                                  int pool = 1);
 int select_supported(const SelectPlan &plan);
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const uint16_t *F,
                           int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,
-                          void *ws, cudaStream_t stream);
+                          void *ws, cudaStream_t stream, int pool = 1);
 
 // ---- prefetch -------------------------------------------------------------
 cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,

@@ -319,6 +319,12 @@ __device__ __forceinline__ void prime_ring(const uint16_t *kc_bg, int lo, int n,
   for (int pc = 0; pc < min(kRing, n_pc); ++pc) issue_piece(kc_bg, lo, n, pc, ring, bars);
 }
 
+// kPool = 1: one key row per block, row r scores block lo + r.  kPool = 4:
+// the window grid (32-token windows at stride 16, four per 64-token block):
+// rows are windows, and block j's score is the largest score of the three
+// windows lying inside it (rows 4j, 4j+1, 4j+2; row 4j+3 straddles two
+// blocks and is skipped).  n counts key rows; keys are written per block.
+template <int kPool>
 __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int lo, int n,
                            uint32_t *keys, uint8_t *ring, uint64_t *bars) {
   const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
@@ -361,13 +367,25 @@ __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int l
     }
     const float sc = transpose_reduce8x16(part, hl);
     const int r = row0 + (hl >> 1);
-    if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
+    if (kPool == 1) {
+      if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
+    } else {
+      // the 8 rows of a half-warp are two blocks' 4 windows: the max of the
+      // first three windows of each group of four (lanes hl^2, hl^4 hold
+      // rows r^1, r^2)
+      float m = (r < rows && (r & 3) != 3) ? sc : -INFINITY;
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const int kb = (pc * kPieceRows + row0) / 4 + (hl >> 3);
+      if ((hl & 7) == 0 && kb * kPool < n) keys[kb] = orderable_key(m);
+    }
     __syncthreads();  // piece consumed by every half-warp
     if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
   }
   return ok;
 }
 
+template <int kPool>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   // dynamic shared memory: piece ring | scoring vectors (fp32) | score keys
   extern __shared__ __align__(128) uint8_t dyn_raw[];
@@ -400,11 +418,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   uint32_t *keys = dyn;
   const int lo = bp.cand_lo + chunk * a.CH;
   const int n = max(0, min(bp.cand_hi, lo + a.CH) - lo);
+  // key rows of this chunk: blocks, or (window grid) 4 windows per block, the
+  // last ones clipped to the windows that exist
+  const int row_lo = lo * kPool;
+  const int n_rows = kPool == 1 ? n : max(0, min(n * kPool, a.NB - row_lo));
   const uint16_t *kc_bg = a.kc + (b * a.G + g) * (long long)a.NB * kD;
   if (threadIdx.x == 0) {
     for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
     fence_mbar_init();
-    prime_ring(kc_bg, lo, n, ring, bars);
+    prime_ring(kc_bg, row_lo, n_rows, ring, bars);
   }
   // Forecast vector(s) of this problem -> fp32 in shared memory
   const uint16_t *f = a.F + (bi * a.G + g) * (long long)a.nf * kD;
@@ -412,7 +434,11 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
     fs[t] = __uint_as_float(((uint32_t)f[t]) << 16);
   __syncthreads();
 
-  if (!score_rows(kc_bg, fs, a.nf, lo, n, keys, ring, bars)) {
+  if (kPool > 1) {  // blocks whose windows all lie past the clipped rows keep a valid key
+    for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = orderable_key(-INFINITY);
+    __syncthreads();
+  }
+  if (!score_rows<kPool>(kc_bg, fs, a.nf, row_lo, n_rows, keys, ring, bars)) {
     // a copy never landed: report an empty set rather than a wrong one
     for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
     return;
@@ -462,7 +488,7 @@ int env_int(const char *name) {
 // The plan depends on the shapes only (not on where the query chunk sits), so
 // the workspace size is known before the call: chunking is sized for a query
 // at the end of the sequence, the most candidates any query can have.
-SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
+SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
   SelectPlan pl{};
   pl.n_problems = (long long)p.B * nq * p.G;
   const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
@@ -477,7 +503,7 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
     // a chunk of query tokens: the scores are a dense product per (sequence,
     // group), computed on the tensor cores and kept in the workspace
     pl.tensor_scores = 1;
-    pl.ws_bytes = prefill_select_ws_bytes(p, nq);
+    pl.ws_bytes = prefill_select_ws_bytes(p, nq, pool);
     return pl;
   }
 
@@ -486,9 +512,10 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf) {
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
   } else {
-    // streaming CTAs of 1024 blocks (256 KB of Kc) each, but one chunk per
-    // problem once there are plenty of problems (prefill)
-    CH = 1024;
+    // streaming CTAs of 256 KB of key rows each (1024 blocks, or 256 blocks
+    // of four windows), but one chunk per problem once there are plenty of
+    // problems (prefill)
+    CH = 1024 / pool;
     if (pl.n_problems >= 8LL * 148) CH = kMaxCand;
   }
   if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
@@ -512,9 +539,9 @@ int select_supported(const SelectPlan &pl) {
 
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const uint16_t *F, int nq,
                           int nf, int q_start, const uint16_t *kc, int32_t *idx, void *ws,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int pool) {
   if (pl.n_problems == 0) return cudaSuccess;
-  if (pl.tensor_scores) return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, stream);
+  if (pl.tensor_scores) return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, stream, pool);
   SelArgs a;
   a.F = F;
   a.kc = kc;
@@ -522,7 +549,7 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.nq = nq;
   a.G = p.G;
   a.nf = nf;
-  a.NB = (p.T + kBlk - 1) / kBlk;
+  a.NB = pool == 1 ? (p.T + kBlk - 1) / kBlk : window_count(p.T);  // key rows per (b, g)
   a.k = p.k;
   a.n_init = p.n_init;
   a.n_local = p.n_local;
@@ -541,22 +568,23 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     a.cand_key = reinterpret_cast<uint32_t *>(w);
     smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
-  {  // raised once per device to the largest size used; most shared memory
-     // goes to the ring, so prefer the largest carveout
-    static size_t raised[64] = {0};
+  auto kern = pool == 1 ? select_kernel<1> : select_kernel<4>;
+  {  // raised once per device and pooling to the largest size used; most
+     // shared memory goes to the ring, so prefer the largest carveout
+    static size_t raised[2][64] = {{0}};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (raised[dev] < smem) {
-      cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
+    size_t &r = raised[pool == 1 ? 0 : 1][dev];
+    if (r < smem) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
       if (e != cudaSuccess) return e;
-      raised[dev] = smem;
+      r = smem;
     }
   }
   const long long grid = pl.n_problems * pl.n_chunks;
-  const cudaError_t e = launch_pdl(select_kernel, (unsigned)grid, kSelThreads, smem, stream, a);
+  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -53,8 +53,13 @@ struct PScoreArgs {
   uint32_t *keys;      // [B*G][nq][ld]
   int32_t *status;
   int G, nq, NB, ld, q_start, n_init, n_local;
+  int n_rows;          // key rows per (b, g): blocks, or windows (kPool = 4)
 };
 
+// kPool = 1: one key row per block, tile column c is block j0 + c.  kPool = 4
+// (window grid): columns are windows, four per block, and block j scores as
+// the best of its windows 4j, 4j+1, 4j+2 (window 4j+3 straddles two blocks).
+template <int kPool>
 __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
     const __grid_constant__ CUtensorMap mapF, const __grid_constant__ CUtensorMap mapKc,
     PScoreArgs a) {
@@ -68,12 +73,13 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
   const int u = blockIdx.x, t = blockIdx.y, pair = blockIdx.z;
   const int b = pair / a.G, g = pair % a.G;
   const int i0 = t * kPTok;
-  const int j0 = u * kPBlk;
+  const int w0 = u * kPBlk;       // first key row (block or window) of the tile
+  const int j0 = w0 / kPool;      // first block of the tile
   // the candidates of the tile's last row reach furthest
   const int i_last = min(a.nq, i0 + kPTok) - 1;
   const BlockParts bp_last = block_parts(a.q_start + i_last, kBlk, a.n_init, a.n_local);
   pdl_trigger();
-  if (j0 >= bp_last.cand_hi || j0 + kPBlk <= a.n_init) return;  // no candidate in the tile
+  if (j0 >= bp_last.cand_hi || j0 + kPBlk / kPool <= a.n_init) return;  // no candidate in the tile
   if (smem_addr(smem) & 1023u) {
     pdl_wait();
     if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
@@ -98,8 +104,8 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
     mbar_arrive_expect_tx(&bars[0], 32768 + 65536);
     tc::tma_load_4d(opA, &mapF, 0, g, i0, b, &bars[0]);
     tc::tma_load_4d(opA + 16384, &mapF, 64, g, i0, b, &bars[0]);
-    tc::tma_load_3d(opB, &mapKc, 0, j0, pair, &bars[0]);
-    tc::tma_load_3d(opB + 32768, &mapKc, 64, j0, pair, &bars[0]);
+    tc::tma_load_3d(opB, &mapKc, 0, w0, pair, &bars[0]);
+    tc::tma_load_3d(opB + 32768, &mapKc, 64, w0, pair, &bars[0]);
     ok = mbar_wait_bounded(&bars[0], 0);
     if (ok) {
       tc::fence_after_sync();
@@ -131,16 +137,34 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
     for (int c = 0; c < kPBlk; c += 16) {
       float v[16];
       tc::tmem_ld16(tmem + lane_sel + c, v);  // warp-wide: every lane takes part
-      if (i < a.nq && j0 + c < a.ld) {
-        uint32_t kk[16];
+      if (kPool == 1) {
+        if (i < a.nq && j0 + c < a.ld) {
+          uint32_t kk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = j0 + c + e;
-          kk[e] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(v[e]) : 0u;
+          for (int e = 0; e < 16; ++e) {
+            const int j = j0 + c + e;
+            kk[e] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(v[e]) : 0u;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            reinterpret_cast<uint4 *>(row + c)[q] =
+                make_uint4(kk[4 * q], kk[4 * q + 1], kk[4 * q + 2], kk[4 * q + 3]);
         }
+      } else {
+        // 16 window columns = 4 blocks; windows past the last one are masked
+        if (i < a.nq) {
+          uint32_t kk[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          reinterpret_cast<uint4 *>(row + c)[q] = make_uint4(kk[4 * q], kk[4 * q + 1], kk[4 * q + 2], kk[4 * q + 3]);
+          for (int q = 0; q < 4; ++q) {
+            float m = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 3; ++e)
+              if (w0 + c + 4 * q + e < a.n_rows) m = fmaxf(m, v[4 * q + e]);
+            const int j = j0 + c / 4 + q;
+            kk[q] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(m) : 0u;
+          }
+          *reinterpret_cast<uint4 *>(row + c / 4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+        }
       }
     }
   }
@@ -460,37 +484,40 @@ __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
 
 }  // namespace
 
-// Rows of the score workspace: the block count rounded up to whole tiles.
-int prefill_ld(int NB) { return (int)ceil_div_ll(NB, kPBlk) * kPBlk; }
+// Keys per row of the score workspace: the block count rounded up to whole
+// tiles (a tile covers kPBlk / pool blocks).
+int prefill_ld(int NB, int pool) { return (int)ceil_div_ll(NB, kPBlk / pool) * (kPBlk / pool); }
 
-size_t prefill_select_ws_bytes(const sparda_params &p, int nq) {
+size_t prefill_select_ws_bytes(const sparda_params &p, int nq, int pool) {
   const int NB = (p.T + kBlk - 1) / kBlk;
-  return (((size_t)p.B * p.G * nq * prefill_ld(NB) * 4) + 255) & ~(size_t)255;
+  return (((size_t)p.B * p.G * nq * prefill_ld(NB, pool) * 4) + 255) & ~(size_t)255;
 }
 
 cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
-                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream) {
+                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream,
+                                  int pool) {
   if ((long long)p.B * nq * p.G == 0) return cudaSuccess;
   const int NB = (p.T + kBlk - 1) / kBlk;
-  const int ld = prefill_ld(NB);
+  const int ld = prefill_ld(NB, pool);
+  const int n_rows = pool == 1 ? NB : window_count(p.T);  // key rows per (b, g)
   // F [B][nq][G][d]: dims (d, G, nq, B); Kc [B][G][NB][d]: dims (d, NB, B*G)
   CUtensorMap mF, mK;
   const uint64_t fd[4] = {(uint64_t)kD, (uint64_t)p.G, (uint64_t)nq, (uint64_t)p.B};
   const uint64_t fs[3] = {(uint64_t)kD * 2, (uint64_t)p.G * kD * 2, (uint64_t)nq * p.G * kD * 2};
   const uint32_t fb[4] = {64, 1, kPTok, 1};
-  const uint64_t kd[3] = {(uint64_t)kD, (uint64_t)NB, (uint64_t)p.B * p.G};
-  const uint64_t ks[2] = {(uint64_t)kD * 2, (uint64_t)NB * kD * 2};
+  const uint64_t kd[3] = {(uint64_t)kD, (uint64_t)n_rows, (uint64_t)p.B * p.G};
+  const uint64_t ks[2] = {(uint64_t)kD * 2, (uint64_t)n_rows * kD * 2};
   const uint32_t kb[3] = {64, kPBlk, 1};
   if (!tc::make_map_nd(&mF, F, 4, fd, fs, fb) || !tc::make_map_nd(&mK, kc, 3, kd, ks, kb))
     return cudaErrorNotSupported;
-  static bool raised[64] = {false};
+  auto kern = pool == 1 ? prefill_scores_kernel<1> : prefill_scores_kernel<4>;
+  static bool raised[2][64] = {{false}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!raised[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_scores_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+  if (!raised[pool == 1 ? 0 : 1][dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
     if (e != cudaSuccess) return e;
-    raised[dev] = true;
+    raised[pool == 1 ? 0 : 1][dev] = true;
   }
   PScoreArgs sa;
   sa.keys = static_cast<uint32_t *>(ws);
@@ -499,10 +526,12 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   sa.nq = nq;
   sa.NB = NB;
   sa.ld = ld;
+  sa.n_rows = n_rows;
   sa.q_start = q_start;
   sa.n_init = p.n_init;
   sa.n_local = p.n_local;
-  const dim3 grid((unsigned)(ld / kPBlk), (unsigned)ceil_div_ll(nq, kPTok), (unsigned)(p.B * p.G));
+  const dim3 grid((unsigned)(ld / (kPBlk / pool)), (unsigned)ceil_div_ll(nq, kPTok),
+                  (unsigned)(p.B * p.G));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kPThreads);
@@ -513,7 +542,7 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_scores_kernel, mF, mK, sa);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mF, mK, sa);
   if (e != cudaSuccess) return e;
   RankArgs ra;
   ra.keys = static_cast<const uint32_t *>(ws);

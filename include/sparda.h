@@ -93,7 +93,8 @@ enum sparda_op {
   SPARDA_OP_SELECT = 1,
   SPARDA_OP_PREFETCH = 2,
   SPARDA_OP_ATTN_DECODE = 3,
-  SPARDA_OP_ATTN_PREFILL = 4
+  SPARDA_OP_ATTN_PREFILL = 4,
+  SPARDA_OP_SELECT_WINDOWS = 5
 };
 
 /* how sparda_sparse_attn_decode finds the storage of list entry s */
@@ -162,6 +163,37 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
                            const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
                            sparda_stream_t stream);
+
+/*
+ * The window grid of the models the pages measure (f3): [p4 "One Forecast
+ * head per GQA group"] -- both test models pool their keys with a 32-token
+ * window at stride 16, and [p4 "Training: distilling the selector you
+ * already have"] names the selector's final max-pooling of the scores to
+ * blocks.  The pages do not print the window-to-block map; the one taken
+ * here: block j's score is the largest score of the windows lying inside
+ * it, windows 4j, 4j+1 and 4j+2 (window 4j+3 straddles two blocks).
+ *
+ * sparda_compress_windows -- kw[b,g,w] = mean of the keys at positions
+ *   [w*stride, w*stride + win), complete windows only: NW = (T - win) /
+ *   stride + 1 for T >= win.  win = 32, stride = 16 (others:
+ *   SPARDA_EUNSUPPORTED); K as for sparda_compress_keys; kw_f32 / kw_bf16
+ *   [B][G][NW][d] (either may be null, not both).
+ */
+int sparda_compress_windows(const sparda_params *p, const void *K, long long bg_stride,
+                            long long tok_stride, int win, int stride, float *kw_f32,
+                            void *kw_bf16, sparda_stream_t stream);
+
+/*
+ * sparda_forecast_select_windows -- sparda_forecast_select on the window
+ *   grid: kw bf16 [B][G][NW][d] from sparda_compress_windows (T sets NW);
+ *   a candidate block scores as the best window inside it, then the same
+ *   top-k rule, tie rule and output.  ws: sparda_workspace_size(
+ *   SPARDA_OP_SELECT_WINDOWS, p, nq, nf) bytes, zero-filled before first use.
+ */
+int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq, int nf,
+                                   int q_start, const void *kw, int win, int stride,
+                                   int32_t *idx, void *ws, size_t ws_bytes,
+                                   sparda_stream_t stream);
 
 /*
  * sparda_prefetch_blocks -- gather the selected K/V blocks of one layer from

@@ -221,6 +221,89 @@ def test_select_prefill_tensor_matches_streaming_path(monkeypatch):
 
 
 # --------------------------------------------------------------------------
+# the window grid (32-token windows at stride 16, max-pooled to blocks)
+# --------------------------------------------------------------------------
+
+def _pooled_scores_f64(F_bits, kw_bits, NB):
+    """fp64 block scores of the window grid for the band rule: the best of
+    the windows 4j, 4j+1, 4j+2 that exist.  -> [B][nq][G][NB]"""
+    ws = scores_f64(F_bits, kw_bits)                 # [B][nq][G][NW]
+    NW = ws.shape[-1]
+    out = np.full(ws.shape[:3] + (NB,), -np.inf)
+    for j in range(NB):
+        cols = [w for w in (4 * j, 4 * j + 1, 4 * j + 2) if w < NW]
+        if cols:
+            out[..., j] = ws[..., cols].max(axis=-1)
+    return out
+
+
+@pytest.mark.parametrize("T", [31, 32, 1000, 4096 + 37])
+def test_compress_windows_parity(T):
+    rng = W.rng_for(60 + T)
+    B, G, d = 2, 3, 128
+    K = W.normal_bf16(rng, (B, G, T, d))
+    NW = oracle.window_count(T)
+    p = abi.make_params(B, G, G, T, 1)
+    kw32 = torch.zeros(B, G, max(NW, 1), d, dtype=torch.float32, device="cuda")
+    kw16 = torch.zeros(B, G, max(NW, 1), d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_windows(p, dev_bf16(K), T * d, d, 32, 16, kw32, kw16)
+    torch.cuda.synchronize()
+    o64, o16 = oracle.compress_windows(K)
+    if NW:
+        check_compressed(kw32.cpu().numpy()[:, :, :NW], host_bits(kw16)[:, :, :NW], o64, o16)
+
+
+def _select_windows_case(F, kw, T, k, n_init, n_local, q_start, what):
+    B, nq, G, nf, d = F.shape
+    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local)
+    S = k + n_init + n_local
+    idx = torch.full((B, nq, G, S), -7, dtype=torch.int32, device="cuda")
+    ws = abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, nq, nf)
+    abi.sparda_forecast_select_windows(p, dev_bf16(F), nq, nf, q_start, dev_bf16(kw), 32, 16, idx, ws)
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    assert not (got == -7).any()
+    ora, kth, kth1 = oracle.select_windows(F, kw, T, k, n_init, n_local, q_start)
+    NB = (T + 63) // 64
+    return check_sets(got, ora, kth, kth1, _pooled_scores_f64(F, kw, NB), what)
+
+
+@pytest.mark.parametrize("T,k,n_local,chunk", [(8192 + 20, 16, 2, "0"), (32768, 64, 2, "256"),
+                                                (5000 + 33, 8, 0, "0"), (20000, 40, 1, "512")])
+def test_select_windows_decode(T, k, n_local, chunk, monkeypatch):
+    rng = W.rng_for(70 + T)
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    B, G, d = 2, 3, 128
+    kw = W.normal_bf16(rng, (B, G, oracle.window_count(T), d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    _select_windows_case(F, kw, T, k, 1, n_local, T - 1, "windows decode")
+
+
+@pytest.mark.parametrize("T,nq,q_off", [(16384 + 40, 96, 0), (40000, 200, 3000)])
+def test_select_windows_prefill_tensor_path(T, nq, q_off):
+    rng = W.rng_for(80 + T)
+    B, G, d = 2, 2, 128
+    kw = W.normal_bf16(rng, (B, G, oracle.window_count(T), d))
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    _select_windows_case(F, kw, T, 32, 1, 2, T - nq - q_off, "windows prefill")
+
+
+def test_select_windows_compressed_from_keys():
+    """The chain a caller runs: compress a sequence into windows, then select."""
+    rng = W.rng_for(90)
+    B, G, T, d = 1, 2, 6000, 128
+    K = W.normal_bf16(rng, (B, G, T, d))
+    p = abi.make_params(B, G, G, T, 12)
+    NW = oracle.window_count(T)
+    kw16 = torch.zeros(B, G, NW, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_windows(p, dev_bf16(K), T * d, d, 32, 16, None, kw16)
+    torch.cuda.synchronize()
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    _select_windows_case(F, host_bits(kw16), T, 12, 1, 2, T - 1, "compressed windows")
+
+
+# --------------------------------------------------------------------------
 # decode attention
 # --------------------------------------------------------------------------
 
