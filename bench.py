@@ -590,21 +590,27 @@ def run_sparda(args):
             kms = time_steps(lambda: kernel_loop(which), args.steps, world)
             kern_us[which] = kms / (args.steps * L) * 1e3
         # decode append (new K/V rows + the incremental compressed key), timed
-        # by writing every layer's last-token rows back unchanged
+        # from a CUDA graph by writing every layer's last-token rows back
+        # unchanged
         pos = w.T - 1
         c_last, r_last = pos // w.blk, pos % w.blk
-        kv_new = [loop.kv[l, :, :, c_last, :, r_last].clone() for l in range(L)]  # [B][G][2][d]
+        k_new = [loop.kv[l, :, :, c_last, 0, r_last].contiguous() for l in range(L)]  # [B][G][d]
+        v_new = [loop.kv[l, :, :, c_last, 1, r_last].contiguous() for l in range(L)]
 
         def append_all():
             for l in range(L):
                 kv = loop.kv[l]
-                abi.sparda_append_kv(loop.p, pos, kv_new[l][:, :, 0].contiguous(),
-                                     kv_new[l][:, :, 1].contiguous(), kv,
+                abi.sparda_append_kv(loop.p, pos, k_new[l], v_new[l], kv,
                                      kv.view(-1)[w.blk * w.d:], w.NB * loop.blk_elems,
                                      loop.blk_elems, None, loop.kc[l])
         for _ in range(3):
             append_all()
-        kern_us["append"] = time_steps(append_all, args.steps, world) / (args.steps * L) * 1e3
+        torch.cuda.synchronize()
+        g_app = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_app, stream=loop.main):
+            append_all()
+        kern_us["append"] = time_steps(g_app.replay, args.steps, world) / (args.steps * L) * 1e3
+        del g_app
     st = int(loop.status.item())
 
     ms_step = ms / args.steps

@@ -117,9 +117,19 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict_
   } else {
     *reinterpret_cast<uint4 *>(V + blk_off + (long long)r * kD) = ldg_plain(V_new + bg * kD + c8 * 8);
   }
-  // rows 0 .. r-1 of the block were written before this launch
+  // rows 0 .. r-1 of the block were written before this launch; eight rows
+  // per half-warp are loaded at once and added in ascending order
   float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int t = half; t < r; t += 2) acc8(a, ldg_plain(K + blk_off + (long long)t * kD));
+#pragma unroll 1
+  for (int t0 = half; t0 < r; t0 += 16) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t0 + 2 * u < r) v[u] = ldg_plain(K + blk_off + (long long)(t0 + 2 * u) * kD);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t0 + 2 * u < r) acc8(a, v[u]);
+  }
   if ((r & 1) == half) acc8(a, knew);
 #pragma unroll
   for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
