@@ -65,6 +65,10 @@ def parse_args():
                          "at stride 16, max-pooled to blocks): window compression, decode "
                          "selection at B=16, T=128K, and the prefill chunk's selection; prints "
                          "an extra JSON line")
+    ap.add_argument("--real-model", action="store_true",
+                    help="also measure the real models' decode configuration: 96-block sets "
+                         "(1 initial, 32 local, 63 top-k) on the window grid, 16 sequences of "
+                         "mixed lengths (64K..128K), 4 layers; prints an extra JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
@@ -197,7 +201,12 @@ class DecodeLoop:
         self.torch, self.abi, self.w = torch, abi, w
         dev = torch.device("cuda")
         B, G, Hq, d, L, NB, S = w.B, w.G, w.Hq, w.d, w.layers, w.NB, w.S
-        self.p = abi.make_params(B, Hq, G, w.T, w.k, w.n_init, w.n_local)
+        # per-sequence lengths (a length mix), else every sequence holds T tokens
+        self.lens = W.decode_lengths(w)
+        self.seq_len = None
+        if w.min_len > 0:
+            self.seq_len = torch.from_numpy(self.lens).to(dev)
+        self.p = abi.make_params(B, Hq, G, w.T, w.k, w.n_init, w.n_local, seq_len=self.seq_len)
         seed = w.seed + 1000 * seed_offset
         self.blk_elems = 2 * w.blk * d                      # one K|V block pair
         # K/V cache of every layer, host layout [L][B][G][NB][2][64][128]
@@ -208,19 +217,29 @@ class DecodeLoop:
         gen.manual_seed(seed * 16 + 15)
         self.Q = torch.randn(L, B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
         self.F = torch.randn(L, B, G, d, generator=gen, device=dev).to(torch.bfloat16)
-        # compressed keys of every layer (each block pooled as its own 64-token run)
-        self.kc = torch.empty(L, B, G, NB, d, dtype=torch.bfloat16, device=dev)
-        pc = abi.make_params(1, B * G * NB, B * G * NB, w.blk, 1)
-        for l in range(L):
-            abi.sparda_compress_keys(pc, self.kv[l], self.blk_elems, d, None, self.kc[l])
+        if w.windows:
+            # window-grid keys of every layer (32-token windows at stride 16); the
+            # interleaved K|V blocks give no constant row stride across a block
+            # boundary, so the keys are drawn like the K/V they summarise
+            self.kc = None
+            self.NW = (w.T - 32) // 16 + 1
+            self.kw = torch.empty(L, B, G, self.NW, d, dtype=torch.bfloat16, device=dev)
+            for l in range(L):
+                W.torch_normal_bf16_(self.kw[l], seed * 16 + 8 + l)
+        else:
+            # compressed keys of every layer (each block pooled as its own 64-token run)
+            self.kc = torch.empty(L, B, G, NB, d, dtype=torch.bfloat16, device=dev)
+            pc = abi.make_params(1, B * G * NB, B * G * NB, w.blk, 1)
+            for l in range(L):
+                abi.sparda_compress_keys(pc, self.kv[l], self.blk_elems, d, None, self.kc[l])
         self.idx = torch.empty(L, B, G, S, dtype=torch.int32, device=dev)
         self.O = torch.empty(L, B, Hq, d, dtype=torch.bfloat16, device=dev)
-        self.ws_sel = [abi.workspace(abi.SPARDA_OP_SELECT, self.p, 1, 1) for _ in range(L)]
+        op = abi.SPARDA_OP_SELECT_WINDOWS if w.windows else abi.SPARDA_OP_SELECT
+        self.ws_sel = [abi.workspace(op, self.p, 1, 1) for _ in range(L)]
         self.ws_att = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, self.p)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         # layer 0's set comes from the previous token's last layer
-        abi.sparda_forecast_select(self.p, self.F[L - 1], 1, 1, w.T - 1, self.kc[0], self.idx[0],
-                                   self.ws_sel[0])
+        self.select(L - 1)
         self.compute = torch.cuda.current_stream()
         # resident step: attention on a high-priority stream, selection beside it
         self.main = torch.cuda.Stream(priority=-1)
@@ -236,8 +255,12 @@ class DecodeLoop:
     def select(self, l):
         """Layer l's Forecast vector picks layer l+1's blocks."""
         w, nxt = self.w, (l + 1) % self.w.layers
-        self.abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                        self.idx[nxt], self.ws_sel[l])
+        if w.windows:
+            self.abi.sparda_forecast_select_windows(self.p, self.F[l], 1, 1, w.T - 1, self.kw[nxt],
+                                                    32, 16, self.idx[nxt], self.ws_sel[l])
+        else:
+            self.abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
+                                            self.idx[nxt], self.ws_sel[l])
 
     def attention(self, l):
         w = self.w
@@ -412,14 +435,26 @@ class DecodeLoop:
         self.torch.cuda.synchronize()
 
     # algorithmic bytes per launch
-    def bytes_select(self):
+    def _ncand(self):
+        """Candidate blocks of each sequence's query (its last token)."""
         w = self.w
-        ncand = (w.T - 1) // w.blk - w.n_local + 1 - w.n_init
-        return w.B * w.G * (ncand * w.d * 2 + w.d * 2 + w.S * 4)
+        c = (self.lens.astype(np.int64) - 1) // w.blk
+        return np.maximum(0, c - w.n_local + 1 - w.n_init)
+
+    def bytes_select(self):
+        """Key rows the selection must read: one per candidate block, or on the
+        window grid the three windows inside each candidate block."""
+        w = self.w
+        rows = self._ncand() * (3 if w.windows else 1)
+        return int(w.G * (rows.sum() * w.d * 2 + w.B * (w.d * 2 + w.S * 4)))
 
     def bytes_attn(self):
+        """The K|V blocks of every set (full sets: each sequence has more
+        candidates than k), plus Q, O and the lists."""
         w = self.w
-        return w.B * w.G * w.S * self.blk_elems * 2 + 2 * w.B * w.Hq * w.d * 2 + w.B * w.G * w.S * 4
+        n_sel = np.minimum(self._ncand(), w.k) + w.n_init + w.n_local
+        return int(w.G * n_sel.sum() * self.blk_elems * 2 + 2 * w.B * w.Hq * w.d * 2
+                   + w.B * w.G * w.S * 4)
 
 
 PROFILE_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
@@ -686,6 +721,8 @@ def run_sparda(args):
         print(json.dumps(run_sweep()), flush=True)
     if rank == 0 and world == 1 and args.windows:
         print(json.dumps(run_windows(args.steps)), flush=True)
+    if rank == 0 and world == 1 and args.real_model:
+        print(json.dumps(run_real_model(args.steps)), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -903,6 +940,58 @@ def run_windows(steps):
     out.update({"prefill_compress_windows_us": c_us,
                 "prefill_compress_windows_GBps": pw.B * pw.G * pw.T * pw.d * 2 / (c_us * 1e-6) / 1e9,
                 "prefill_select_us": s_us})
+    return out
+
+
+def run_real_model(steps):
+    """The real models' decode configuration in the 4-layer loop: 96-block
+    sets (1 initial, 32 local, 63 top-k) chosen on the window grid, for 16
+    sequences of mixed lengths (64K..128K tokens), all K/V resident.  The
+    step is the resident step of the headline loop (select(l) beside
+    attention(l)), replayed from a CUDA graph."""
+    import torch
+    w = W.WORKLOADS["decode_loop_b16_t128k_budget96"]
+    loop = DecodeLoop(w, with_host=False)
+    L = w.layers
+    n = max(5, min(steps, 50))
+    with torch.cuda.stream(loop.main):
+        for _ in range(3):
+            loop.step_resident()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=loop.main):
+            loop.step_resident()
+        step_us = time_back_to_back(graph.replay, n)
+        kern = {}
+        for which in ("select", "attention"):
+            fn = (lambda: [loop.select(l) for l in range(L)]) if which == "select" else \
+                 (lambda: [loop.attention(l) for l in range(L)])
+            kern[which] = time_back_to_back(fn, n) / L
+        del graph
+    torch.cuda.synchronize()
+    st = int(loop.status.item())
+    peak, peak_kind = measured_peaks()
+    b_att, b_sel = loop.bytes_attn(), loop.bytes_select()
+    step_gbs = L * (b_att + b_sel) / (step_us * 1e-6) / 1e9
+    out = {
+        "metric": "decode tokens/s, real-model budget (96 blocks: 1 initial + 32 local + 63 "
+                  "top-k on the 32/16 window grid), mixed sequence lengths",
+        "value": w.B / (step_us * 1e-6), "unit": "tokens/s", "data": "synthetic", "dtype": "bf16",
+        "config": {"workload": w.name, "B": w.B, "T_max": w.T, "lengths": [int(x) for x in loop.lens],
+                   "layers": L, "Hq": w.Hq, "G": w.G, "k": w.k, "n_init": w.n_init,
+                   "n_local": w.n_local, "selection": "window grid, 32 tokens at stride 16",
+                   "l2": "inputs larger than L2: %.0f MB of selected K/V per layer" % (b_att / 1e6)},
+        "step_us": step_us, "step_GBps": step_gbs, "step_hbm_frac": step_gbs / peak,
+        "select_us_per_layer": kern["select"],
+        "select_GBps": b_sel / (kern["select"] * 1e-6) / 1e9,
+        "attn_us_per_layer": kern["attention"],
+        "attn_GBps": b_att / (kern["attention"] * 1e-6) / 1e9,
+        "attn_hbm_frac": b_att / (kern["attention"] * 1e-6) / 1e9 / peak,
+        "bytes_per_layer": {"attention": b_att, "select": b_sel},
+        "peak": peak, "peak_kind": peak_kind, "device_status": st,
+    }
+    del loop
+    torch.cuda.empty_cache()
     return out
 
 

@@ -51,12 +51,16 @@ class sparda_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("G", ctypes.c_int),
                 ("d", ctypes.c_int), ("blk", ctypes.c_int), ("T", ctypes.c_int),
                 ("k", ctypes.c_int), ("n_init", ctypes.c_int), ("n_local", ctypes.c_int),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("seq_len", ctypes.c_void_p)]
 
 
-def make_params(B, Hq, G, T, k, n_init=1, n_local=2, d=128, blk=64, scale=0.0) -> sparda_params:
+def make_params(B, Hq, G, T, k, n_init=1, n_local=2, d=128, blk=64, scale=0.0,
+                seq_len=None) -> sparda_params:
+    """seq_len: optional device int32 tensor [B] of per-sequence lengths (the
+    caller keeps it alive while the params are in use)."""
     return sparda_params(int(B), int(Hq), int(G), int(d), int(blk), int(T), int(k), int(n_init),
-                         int(n_local), float(scale))
+                         int(n_local), float(scale),
+                         None if seq_len is None else seq_len.data_ptr())
 
 
 _lib = None

@@ -32,6 +32,10 @@ int check_params(const sparda_params *p) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARDA_OK : SPARDA_ECUDA; }
 
+// calls that do not read per-sequence lengths refuse them rather than
+// silently using T for every sequence
+int no_seq_len(const sparda_params *p) { return p->seq_len ? SPARDA_EUNSUPPORTED : SPARDA_OK; }
+
 bool stride_ok(long long s) { return s > 0 && (s % 8) == 0; }
 
 }  // namespace
@@ -97,6 +101,7 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
                      void *kc_bf16, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
+  if ((st = no_seq_len(p)) != SPARDA_OK) return st;
   if (pos < 0 || pos >= p->T) return SPARDA_EINVAL;
   if (p->B == 0) return SPARDA_OK;
   if (!K_new || !V_new || !K || !V || (!kc_f32 && !kc_bf16)) return SPARDA_EINVAL;
@@ -138,6 +143,7 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
   if (st != SPARDA_OK) return st;
   if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
   if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
+  if (p->seq_len && nq != 1) return SPARDA_EUNSUPPORTED;  // lengths: decode queries only
   if (nf > 16) return SPARDA_EUNSUPPORTED;
   if (p->B == 0) return SPARDA_OK;
   if (!F || !kw || !idx) return SPARDA_EINVAL;
@@ -157,6 +163,7 @@ int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf
   if (st != SPARDA_OK) return st;
   if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
   if (nf > 16) return SPARDA_EUNSUPPORTED;
+  if (p->seq_len && nq != 1) return SPARDA_EUNSUPPORTED;  // lengths: decode queries only
   if (p->B == 0) return SPARDA_OK;
   if (!F || !kc || !idx) return SPARDA_EINVAL;
   if (!aligned16(F) || !aligned16(kc) || !aligned16(idx)) return SPARDA_EINVAL;
@@ -286,6 +293,7 @@ int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, in
                                size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
+  if ((st = no_seq_len(p)) != SPARDA_OK) return st;
   if (nq < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
   if (p->B == 0) return SPARDA_OK;
   if (!Q || !K || !V || !idx || !O) return SPARDA_EINVAL;

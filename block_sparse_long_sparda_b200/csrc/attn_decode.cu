@@ -102,6 +102,7 @@ struct TcArgs {
   uint16_t *O;
   const int32_t *idx;
   const int32_t *phys;  // SPARDA_ADDR_PHYS: the slot of each entry
+  const int32_t *seq_len;  // optional per-sequence lengths (decode: nq = 1)
   float *ws_o;          // [pairs][max_cover][R][128] unnormalised segment outputs
   float2 *ws_ml;        // [pairs][max_cover][R] (max, sum) in the exp2 domain
   uint32_t *counters;   // [pairs] tickets, zero between calls
@@ -111,6 +112,7 @@ struct TcArgs {
   int G, S, NB, addr_mode, nq, q_start, max_cover;
   int order_bgi;        // 1: pairs are streamed in (sequence, group, token) order
   int n_slots;          // SPARDA_ADDR_PHYS: slots per (sequence, group)
+  int T;
   float scale_log2;
 };
 
@@ -342,10 +344,14 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       const int s = s_me;
       const int j = j_me;
       if (j >= 0) {
-        const int pos = a.q_start + (int)((pm / a.G) % a.nq);
+        int pos = a.q_start + (int)((pm / a.G) % a.nq);
+        if (a.seq_len) {  // decode with per-sequence lengths: the query is the last token
+          const int len = a.seq_len[pm / a.G];
+          pos = (len >= 1 && len <= a.T) ? len - 1 : -1;  // -1: every block is flagged
+        }
         const bool slot_bad =
             a.addr_mode == SPARDA_ADDR_PHYS && (phys_me < 0 || phys_me >= a.n_slots);
-        if (j >= a.NB || j > pos / kBlk || slot_bad) {
+        if (pos < 0 || j >= a.NB || j > pos / kBlk || slot_bad) {
           flag_status(a.status, SPARDA_DEV_RANGE);
         } else {
           const long long kvpair = (pm / a.G) / a.nq * a.G + pm % a.G;
@@ -733,6 +739,8 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.O = O;
   a.idx = idx;
   a.phys = phys;
+  a.seq_len = p.seq_len;
+  a.T = p.T;
   a.n_slots = n_slots;
   a.status = dev_status;
   a.n_entries = pairs * pl.S;

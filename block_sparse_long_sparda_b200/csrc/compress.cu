@@ -41,14 +41,18 @@ __global__ void __launch_bounds__(256, 3) compress_kernel(const uint16_t *__rest
                                                        int T, int NB, long long n_items,
                                                        float *__restrict__ kc32,
                                                        uint16_t *__restrict__ kc16, int rows,
-                                                       int step) {
+                                                       int step, const int32_t *seq_len, int G) {
   const int lane = threadIdx.x & 31;
   const long long item = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (item >= n_items) return;
   const long long bg = item / NB;
   const int j = (int)(item - bg * NB);
   const int t0 = j * step;
-  const int n = min(rows, T - t0);
+  // per-sequence lengths: a block past its sequence's end, or a window not
+  // complete inside it, is left untouched
+  const int Tb = seq_len ? min(T, seq_len[bg / G]) : T;
+  const int n = min(rows, Tb - t0);
+  if (n <= 0 || (rows != step && n < rows)) return;
   const int half = lane >> 4;
   const int c8 = lane & 15;
   if (kContig) tok_stride = kD;  // rows packed: constant offsets, fewer live registers
@@ -174,11 +178,11 @@ cudaError_t launch_compress_runs(const sparda_params &p, const uint16_t *K, long
   const int warps = 8;
   const long long grid = ceil_div_ll(items, warps);
   if (tok_stride == kD)
-    compress_kernel<true><<<(unsigned)grid, warps * 32, 0, stream>>>(K, bg_stride, tok_stride, p.T,
-                                                                   NB, items, kc32, kc16, rows, step);
+    compress_kernel<true><<<(unsigned)grid, warps * 32, 0, stream>>>(
+        K, bg_stride, tok_stride, p.T, NB, items, kc32, kc16, rows, step, p.seq_len, p.G);
   else
     compress_kernel<false><<<(unsigned)grid, warps * 32, 0, stream>>>(
-        K, bg_stride, tok_stride, p.T, NB, items, kc32, kc16, rows, step);
+        K, bg_stride, tok_stride, p.T, NB, items, kc32, kc16, rows, step, p.seq_len, p.G);
   return cudaGetLastError();
 }
 

@@ -75,7 +75,7 @@ struct SelectPlan {
 // windows at stride 16), a block scoring as the best window inside it
 SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool = 1);
 // windows of 32 tokens at stride 16 that fit in T tokens
-inline int window_count(int T) { return T >= 32 ? (T - 32) / 16 + 1 : 0; }
+__host__ __device__ inline int window_count(int T) { return T >= 32 ? (T - 32) / 16 + 1 : 0; }
 // prefill (select_prefill.cu): scores of a token chunk on the tensor cores,
 // then one warp per (token, group) row ranks them
 constexpr int kPrefillTensorMinQ = 64;  // query tokens from which the product pays

@@ -38,7 +38,8 @@ constexpr int kVecPerThread = kVecPerPair / kPfThreads;  // 8
 __global__ void __launch_bounds__(kPfThreads) prefetch_kernel(
     const uint16_t *__restrict__ host_kv, const int32_t *__restrict__ idx,
     uint16_t *__restrict__ slots, long long n_entries, int S, int NB, int cand_lo, int cand_hi,
-    int skip_resident, int32_t *status) {
+    int skip_resident, int32_t *status, const int32_t *seq_len, int G, int T, int n_init,
+    int n_local) {
   for (long long ent = blockIdx.x; ent < n_entries; ent += gridDim.x) {
     const int j = idx[ent];
     if (j < 0) continue;
@@ -46,8 +47,19 @@ __global__ void __launch_bounds__(kPfThreads) prefetch_kernel(
       if (threadIdx.x == 0) flag_status(status, SPARDA_DEV_RANGE);
       continue;
     }
-    if (skip_resident && !(j >= cand_lo && j < cand_hi)) continue;
     const long long bg = ent / S;
+    int lo = cand_lo, hi = cand_hi;
+    if (seq_len) {  // the resident initial and local blocks of this sequence
+      const int len = seq_len[bg / G];
+      if (len < 1 || len > T) {
+        if (threadIdx.x == 0) flag_status(status, SPARDA_DEV_RANGE);
+        continue;
+      }
+      const BlockParts bp = block_parts(len - 1, kBlk, n_init, n_local);
+      lo = bp.cand_lo;
+      hi = bp.cand_hi;
+    }
+    if (skip_resident && !(j >= lo && j < hi)) continue;
     const uint4 *src =
         reinterpret_cast<const uint4 *>(host_kv + ((bg * NB + j) * (long long)kPairBytes / 2));
     uint4 *dst = reinterpret_cast<uint4 *>(slots + ent * (long long)(kPairBytes / 2));
@@ -78,7 +90,8 @@ cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
   n_ctas = (int)std::min<long long>(n_ctas, n_entries);
   prefetch_kernel<<<n_ctas, kPfThreads, 0, stream>>>(host_kv_dev, idx, slots, n_entries, S, NB,
                                                      bp.cand_lo, bp.cand_hi, skip_resident,
-                                                     dev_status);
+                                                     dev_status, p.seq_len, p.G, p.T, p.n_init,
+                                                     p.n_local);
   return cudaGetLastError();
 }
 

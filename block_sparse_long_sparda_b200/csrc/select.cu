@@ -43,12 +43,13 @@ constexpr int kSelThreads = 256;
 constexpr int kMaxCand = 24576;   // candidates one problem may have (keys fit in shared memory)
 
 struct SelArgs {
+  const int32_t *seq_len;  // optional per-sequence lengths (decode: nq = 1)
   const uint16_t *F;
   const uint16_t *kc;
   int32_t *idx;
   uint32_t *counters;   // one ticket per problem (multi-chunk only)
   uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
-  int nq, G, nf, NB, k, n_init, n_local, q_start, S;
+  int nq, G, nf, NB, k, n_init, n_local, q_start, S, T;
   int CH, n_chunks, cap;
 };
 
@@ -406,9 +407,28 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   const long long bi = prob / a.G;
   const int i = (int)(bi % a.nq);
   const long long b = bi / a.nq;
-  const BlockParts bp = block_parts(a.q_start + i, kBlk, a.n_init, a.n_local);
-  const int ncand = bp.cand_hi - bp.cand_lo;
+  int pos = a.q_start + i;
   int32_t *out = a.idx + prob * a.S;
+  int rows_b = a.NB;  // key rows of this sequence (the row stride stays a.NB)
+  if (a.seq_len) {  // decode with per-sequence lengths: the query is the last token
+    const int len = a.seq_len[b];
+    if (len < 1 || len > a.T) {  // an invalid length: an empty set
+      if (chunk == 0)
+        for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+      if (a.n_chunks > 1) {  // keep the ticket count of the problem right
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          const unsigned t = atomicAdd(&a.counters[prob], 1u);
+          if (t == (unsigned)(a.n_chunks - 1)) a.counters[prob] = 0u;
+        }
+      }
+      return;
+    }
+    pos = len - 1;
+    if (kPool > 1) rows_b = window_count(len);
+  }
+  const BlockParts bp = block_parts(pos, kBlk, a.n_init, a.n_local);
+  const int ncand = bp.cand_hi - bp.cand_lo;
 
   if (ncand <= a.k || a.k == 0) {  // nothing to rank: every candidate, or none, is kept
     if (chunk == 0) write_set(out, bp, min(ncand, a.k), a.S, true);
@@ -421,7 +441,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   // key rows of this chunk: blocks, or (window grid) 4 windows per block, the
   // last ones clipped to the windows that exist
   const int row_lo = lo * kPool;
-  const int n_rows = kPool == 1 ? n : max(0, min(n * kPool, a.NB - row_lo));
+  const int n_rows = kPool == 1 ? n : max(0, min(n * kPool, rows_b - row_lo));
   const uint16_t *kc_bg = a.kc + (b * a.G + g) * (long long)a.NB * kD;
   if (threadIdx.x == 0) {
     for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
@@ -543,6 +563,8 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   if (pl.n_problems == 0) return cudaSuccess;
   if (pl.tensor_scores) return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, stream, pool);
   SelArgs a;
+  a.seq_len = p.seq_len;
+  a.T = p.T;
   a.F = F;
   a.kc = kc;
   a.idx = idx;

@@ -39,6 +39,8 @@ class Workload:
     nq: int = 1            # query tokens per sequence (1 = decode)
     layers: int = 1        # decode loop depth
     planted: int = 0       # hot blocks planted per (b, g)
+    min_len: int = 0       # > 0: per-sequence lengths drawn uniformly in [min_len, T]
+    windows: int = 0       # 1: selection on the window grid (32 tokens, stride 16)
     note: str = ""
 
     @property
@@ -68,6 +70,12 @@ WORKLOADS = {
     "decode_loop_b16_t128k": Workload(
         "decode_loop_b16_t128k", B=16, T=131072, Hq=32, G=8, k=64, layers=4, seed=1003,
         note="4-layer decode loop, KV of every layer in pinned host memory"),
+    "decode_loop_b16_t128k_budget96": Workload(
+        "decode_loop_b16_t128k_budget96", B=16, T=131072, Hq=32, G=8, k=63, n_init=1, n_local=32,
+        layers=4, min_len=65536, windows=1, seed=1006,
+        note="the real models' decode configuration: 96 blocks (1 initial, 32 local = 2048 "
+             "tokens, 63 top-k) chosen on the 32/16 window grid, sequences of mixed lengths "
+             "between 64K and 128K tokens"),
     "prefill_b4_t128k_c2k": Workload(
         "prefill_b4_t128k_c2k", B=4, T=131072, Hq=32, G=8, k=64, nq=2048, seed=1004,
         note="prefill chunk of 2048 tokens at the end of a 128K sequence"),
@@ -77,6 +85,14 @@ WORKLOADS = {
 SWEEP_NB = (128, 256, 512, 1024, 2048, 4096, 8192, 16384)
 SWEEP_B = (1, 2, 4, 8, 16)
 SWEEP_SEED = 1005
+
+
+def decode_lengths(w: Workload) -> np.ndarray:
+    """Tokens held by each sequence of a decode batch, int32 [B]: all T, or
+    (min_len > 0) uniform integers in [min_len, T], seeded."""
+    if w.min_len <= 0:
+        return np.full(w.B, w.T, np.int32)
+    return rng_for(w.seed, 2).integers(w.min_len, w.T + 1, size=w.B).astype(np.int32)
 
 
 def scaled(w: Workload, **kw) -> Workload:

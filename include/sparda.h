@@ -85,6 +85,19 @@ typedef struct sparda_params {
   int n_init;   /* initial blocks (>= 0, <= 64)                                */
   int n_local;  /* local-window blocks (>= 0, <= 64)                           */
   float scale;  /* attention logit scale; <= 0 means 1/sqrt(d)                 */
+  /* Optional device int32 [B]: tokens present in each sequence, 1 <= seq_len[b]
+   * <= T (T then only sizes the arrays).  Null: every sequence holds T tokens.
+   * Honoured by sparda_compress_keys and sparda_compress_windows (blocks past
+   * the end, and windows not complete inside the sequence, are left
+   * untouched), sparda_forecast_select and sparda_forecast_select_windows
+   * (nq = 1: the query of sequence b sits at seq_len[b] - 1),
+   * sparda_prefetch_blocks and the decode attention calls; the cache plan
+   * and the cached prefetch follow the lists they are given.
+   * sparda_append_kv and sparda_sparse_attn_prefill return
+   * SPARDA_EUNSUPPORTED when it is set.  A length outside [1, T] is flagged SPARDA_DEV_RANGE
+   * where a status word is given, and that sequence's outputs are left empty
+   * (a -1 set, a zero output). */
+  const int32_t *seq_len;
 } sparda_params;
 
 /* ops for sparda_workspace_size */

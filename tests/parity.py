@@ -96,3 +96,16 @@ def check_sets(gpu_idx: np.ndarray, ora_idx: np.ndarray, kth: np.ndarray, kth1: 
             assert sc[j] >= lo, "%s %s: added block %d scoring below the band" % (what, pos, j)
         assert np.all(np.diff(g[g >= 0]) > 0), "not ascending"
     return bitexact
+
+
+def pooled_scores_f64(F_bits, kw_bits, NB):
+    """fp64 block scores of the window grid for the band rule: the best of
+    the windows 4j, 4j+1, 4j+2 that exist.  -> [B][nq][G][NB]"""
+    ws = scores_f64(F_bits, kw_bits)                 # [B][nq][G][NW]
+    NW = ws.shape[-1]
+    out = np.full(ws.shape[:3] + (NB,), -np.inf)
+    for j in range(NB):
+        cols = [w for w in (4 * j, 4 * j + 1, 4 * j + 2) if w < NW]
+        if cols:
+            out[..., j] = ws[..., cols].max(axis=-1)
+    return out

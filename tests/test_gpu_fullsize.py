@@ -19,7 +19,8 @@ import torch
 
 import oracle
 from block_sparse_long_sparda_b200 import abi, build
-from tests.parity import check_attention, check_sets, host_bits, scores_f64
+from block_sparse_long_sparda_b200 import workloads as W
+from tests.parity import check_attention, check_sets, host_bits, pooled_scores_f64, scores_f64
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -71,6 +72,46 @@ def test_decode_loop_full_size_sampled():
             Q = host_bits(loop.Q[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
             flat = kv.reshape(-1)
             ora_o = oracle.sparse_attention(Q, flat, flat[blk * d:], gpu_idx, T - 1, T, blk,
+                                            bg_stride=flat.size, blk_stride=2 * blk * d, G=1)
+            gpu_o = host_bits(loop.O[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+            check_attention(gpu_o, ora_o, what)
+    del loop
+    torch.cuda.empty_cache()
+
+
+def test_real_model_decode_loop_full_size_sampled():
+    """The real models' decode configuration as bench.py times it: 96-block
+    sets on the window grid, 16 sequences of mixed lengths.  Each sample's
+    set is checked against the oracle run on that sequence alone (its own
+    length and query position), and its attention over the GPU's set."""
+    import bench
+    w = W.WORKLOADS["decode_loop_b16_t128k_budget96"]
+    loop = bench.DecodeLoop(w, with_host=False)
+    loop.step_resident()
+    torch.cuda.synchronize()
+    assert int(loop.status.item()) == 0
+    L, R, d, blk = w.layers, w.r, w.d, w.blk
+    rng = np.random.default_rng(2026)
+    shortest = int(np.argmin(loop.lens))
+    for l in range(L):
+        picks = {(shortest, 0), (w.B - 1, w.G - 1)}
+        while len(picks) < 3:
+            picks.add((int(rng.integers(w.B)), int(rng.integers(w.G))))
+        for b, g in sorted(picks):
+            Lb = int(loop.lens[b])
+            what = "layer %d b %d g %d (length %d)" % (l, b, g, Lb)
+            nw = oracle.window_count(Lb)
+            kw = np.ascontiguousarray(host_bits(loop.kw[l, b, g])[:nw]).reshape(1, 1, nw, d)
+            F = host_bits(loop.F[(l - 1) % L, b, g]).reshape(1, 1, 1, 1, d)
+            ora_idx, kth, kth1 = oracle.select_windows(F, kw, Lb, w.k, w.n_init, w.n_local, Lb - 1)
+            gpu_idx = loop.idx[l, b, g].cpu().numpy().reshape(1, 1, 1, -1)
+            assert gpu_idx.shape[-1] == 96
+            check_sets(gpu_idx, ora_idx, kth, kth1,
+                       pooled_scores_f64(F, kw, (Lb + blk - 1) // blk), what)
+            kv = host_bits(loop.kv[l, b, g])
+            Q = host_bits(loop.Q[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+            flat = kv.reshape(-1)
+            ora_o = oracle.sparse_attention(Q, flat, flat[blk * d:], gpu_idx, Lb - 1, Lb, blk,
                                             bg_stride=flat.size, blk_stride=2 * blk * d, G=1)
             gpu_o = host_bits(loop.O[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
             check_attention(gpu_o, ora_o, what)

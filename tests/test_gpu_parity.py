@@ -12,7 +12,7 @@ import oracle
 from block_sparse_long_sparda_b200 import abi, build
 from block_sparse_long_sparda_b200 import workloads as W
 from tests.parity import (bf16_f64, check_attention, check_compressed, check_sets, dev_bf16,
-                          host_bits, scores_f64)
+                          host_bits, pooled_scores_f64, scores_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -224,19 +224,6 @@ def test_select_prefill_tensor_matches_streaming_path(monkeypatch):
 # the window grid (32-token windows at stride 16, max-pooled to blocks)
 # --------------------------------------------------------------------------
 
-def _pooled_scores_f64(F_bits, kw_bits, NB):
-    """fp64 block scores of the window grid for the band rule: the best of
-    the windows 4j, 4j+1, 4j+2 that exist.  -> [B][nq][G][NB]"""
-    ws = scores_f64(F_bits, kw_bits)                 # [B][nq][G][NW]
-    NW = ws.shape[-1]
-    out = np.full(ws.shape[:3] + (NB,), -np.inf)
-    for j in range(NB):
-        cols = [w for w in (4 * j, 4 * j + 1, 4 * j + 2) if w < NW]
-        if cols:
-            out[..., j] = ws[..., cols].max(axis=-1)
-    return out
-
-
 @pytest.mark.parametrize("T", [31, 32, 1000, 4096 + 37])
 def test_compress_windows_parity(T):
     rng = W.rng_for(60 + T)
@@ -265,7 +252,7 @@ def _select_windows_case(F, kw, T, k, n_init, n_local, q_start, what):
     assert not (got == -7).any()
     ora, kth, kth1 = oracle.select_windows(F, kw, T, k, n_init, n_local, q_start)
     NB = (T + 63) // 64
-    return check_sets(got, ora, kth, kth1, _pooled_scores_f64(F, kw, NB), what)
+    return check_sets(got, ora, kth, kth1, pooled_scores_f64(F, kw, NB), what)
 
 
 @pytest.mark.parametrize("T,k,n_local,chunk", [(8192 + 20, 16, 2, "0"), (32768, 64, 2, "256"),
@@ -301,6 +288,178 @@ def test_select_windows_compressed_from_keys():
     torch.cuda.synchronize()
     F = W.normal_bf16(rng, (B, 1, G, 1, d))
     _select_windows_case(F, host_bits(kw16), T, 12, 1, 2, T - 1, "compressed windows")
+
+
+# --------------------------------------------------------------------------
+# per-sequence lengths (decode) and a real model's budget
+# --------------------------------------------------------------------------
+
+def test_varlen_compress_leaves_blocks_past_the_end():
+    rng = W.rng_for(100)
+    B, G, T, d = 3, 2, 4096 + 5, 128
+    lens = [1000, 64, T]
+    K = W.normal_bf16(rng, (B, G, T, d))
+    NB = (T + 63) // 64
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G, G, T, 1, seq_len=sl)
+    kc32 = torch.full((B, G, NB, d), 7.0, dtype=torch.float32, device="cuda")
+    abi.sparda_compress_keys(p, dev_bf16(K), T * d, d, kc32, None)
+    torch.cuda.synchronize()
+    got = kc32.cpu().numpy()
+    for b, L in enumerate(lens):
+        o64, _ = oracle.compress_keys(np.ascontiguousarray(K[b:b + 1, :, :L]))
+        nb = (L + 63) // 64
+        assert np.abs(got[b, :, :nb] - o64[0]).max() <= 1e-3
+        assert np.all(got[b, :, nb:] == 7.0)
+
+
+@pytest.mark.parametrize("chunk", ["0", "256"])
+def test_varlen_decode_select_and_attention(chunk, monkeypatch):
+    """Four sequences of different lengths in one batch: each one's set and
+    attention output equal the oracle run on that sequence alone."""
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    rng = W.rng_for(101)
+    B, G, R, T, d, k = 4, 2, 4, 20000, 128, 16
+    lens = [T, 3000 + 17, 70, 9000]
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    NB = (T + 63) // 64
+    S = k + 3
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * R, G, T, k, seq_len=sl)
+    Kd, Vd = dev_bf16(K), dev_bf16(V)
+    kc = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_keys(p, Kd, T * d, d, None, kc)
+    idx = torch.full((B, 1, G, S), -7, dtype=torch.int32, device="cuda")
+    abi.sparda_forecast_select(p, dev_bf16(F), 1, 1, T - 1, kc, idx,
+                               abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1))
+    O = torch.empty(B, G * R, d, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_sparse_attn_decode(p, dev_bf16(Q), Kd, Vd, T * d, 64 * d, idx.view(B, G, S), 0, O,
+                                  abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kcb = host_bits(kc)
+    got_idx = idx.cpu().numpy()
+    got_o = host_bits(O)
+    for b, L in enumerate(lens):
+        Fb = F[b:b + 1]
+        kcl = np.ascontiguousarray(kcb[b:b + 1, :, :(L + 63) // 64])
+        ora, kth, kth1 = oracle.select(Fb, kcl, k, 1, 2, L - 1)
+        check_sets(got_idx[b:b + 1], ora, kth, kth1, scores_f64(Fb, kcl), "varlen b=%d" % b)
+        o = oracle.sparse_attention(Q[b:b + 1].reshape(1, 1, G * R, d),
+                                    np.ascontiguousarray(K[b:b + 1, :, :L]),
+                                    np.ascontiguousarray(V[b:b + 1, :, :L]),
+                                    got_idx[b:b + 1], L - 1, L)
+        check_attention(got_o[b:b + 1].reshape(1, 1, G * R, d), o, "varlen attention b=%d" % b)
+
+
+def test_varlen_invalid_length_gives_empty_outputs():
+    B, G, T, d, k = 2, 1, 4096, 128, 4
+    sl = torch.tensor([T, 0], dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, 4, G, T, k, seq_len=sl)
+    rng = W.rng_for(102)
+    kc = dev_bf16(W.normal_bf16(rng, (B, G, T // 64, d)))
+    F = dev_bf16(W.normal_bf16(rng, (B, 1, G, 1, d)))
+    idx = torch.full((B, 1, G, k + 3), -7, dtype=torch.int32, device="cuda")
+    abi.sparda_forecast_select(p, F, 1, 1, T - 1, kc, idx, abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1))
+    KV = dev_bf16(W.normal_bf16(rng, (B, G, T, d)))
+    good = torch.tensor([[[0, 5, 9, 62, 63, -1, -1]]] * B, dtype=torch.int32, device="cuda").view(B, G, 7)
+    O = torch.full((B, 4, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_sparse_attn_decode(p, dev_bf16(W.normal_bf16(rng, (B, 4, d))), KV, KV, T * d, 64 * d,
+                                  good, 0, O, abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p), status)
+    torch.cuda.synchronize()
+    assert np.all(idx.cpu().numpy()[1] == -1) and not np.any(idx.cpu().numpy()[0] == -7)
+    assert abi.sparda_status_from_device(int(status.item())) == abi.SPARDA_ERANGE
+    assert torch.all(O[1] == 0) and torch.isfinite(O[0].float()).all()
+
+
+def test_varlen_prefetch_keeps_each_sequences_resident_blocks():
+    rng = W.rng_for(103)
+    B, G, NB, d, k = 2, 2, 40, 128, 5
+    T = NB * 64
+    lens = [T, 1000]
+    S = k + 3
+    host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
+    idx = np.zeros((B, G, S), np.int32)
+    for b, L in enumerate(lens):
+        c = (L - 1) // 64
+        for g in range(G):
+            top = sorted(rng.choice(np.arange(1, c - 1), k, replace=False).tolist())
+            idx[b, g] = [0] + top + [c - 1, c]
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * 4, G, T, k, seq_len=sl)
+    slots = torch.zeros(B, G, S, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_prefetch_blocks(p, _pinned_bf16(host), torch.from_numpy(idx).cuda(), slots, True)
+    torch.cuda.synchronize()
+    got = host_bits(slots)
+    for b, L in enumerate(lens):
+        ora = oracle.gather_blocks(host[b:b + 1], idx[b:b + 1], L - 1, 1, 2, True)
+        assert np.array_equal(got[b:b + 1], ora), b
+
+
+@pytest.mark.parametrize("n_local,chunk", [(2, "0"), (0, "0"), (1, "512")])
+def test_varlen_window_grid(n_local, chunk, monkeypatch):
+    """Window compression and window selection with per-sequence lengths:
+    windows not complete inside a sequence are left untouched and never
+    scored (with n_local = 0 the query's own partial block is a candidate
+    and scores only through the windows its sequence completes)."""
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    rng = W.rng_for(105 + n_local)
+    B, G, T, d, k = 3, 2, 12000, 128, 12
+    lens = [T, 5000 + 45, 1030]
+    K = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    NW = oracle.window_count(T)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G, G, T, k, 1, n_local, seq_len=sl)
+    kw32 = torch.full((B, G, NW, d), 7.0, dtype=torch.float32, device="cuda")
+    kw16 = torch.zeros(B, G, NW, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_windows(p, dev_bf16(K), T * d, d, 32, 16, kw32, kw16)
+    S = k + 1 + n_local
+    idx = torch.full((B, 1, G, S), -7, dtype=torch.int32, device="cuda")
+    abi.sparda_forecast_select_windows(p, dev_bf16(F), 1, 1, T - 1, kw16, 32, 16, idx,
+                                       abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, 1, 1))
+    torch.cuda.synchronize()
+    got32, got16, got_idx = kw32.cpu().numpy(), host_bits(kw16), idx.cpu().numpy()
+    for b, L in enumerate(lens):
+        nw = oracle.window_count(L)
+        o64, o16 = oracle.compress_windows(np.ascontiguousarray(K[b:b + 1, :, :L]))
+        check_compressed(got32[b:b + 1, :, :nw], got16[b:b + 1, :, :nw], o64, o16)
+        assert np.all(got32[b, :, nw:] == 7.0)
+        kwl = np.ascontiguousarray(got16[b:b + 1, :, :nw])
+        Fb = F[b:b + 1]
+        ora, kth, kth1 = oracle.select_windows(Fb, kwl, L, k, 1, n_local, L - 1)
+        check_sets(got_idx[b:b + 1], ora, kth, kth1, pooled_scores_f64(Fb, kwl, (L + 63) // 64),
+                   "varlen windows b=%d" % b)
+
+
+@pytest.mark.parametrize("k,n_init,n_local", [(63, 1, 32), (24, 1, 16)])
+def test_real_model_budget(k, n_init, n_local):
+    """A real model's budget: 96 blocks of which 32 (2048 tokens) are the
+    local window and one the initial block, leaving 63 to top-k; and a
+    16-block local window with 24 query-aware blocks."""
+    rng = W.rng_for(104)
+    B, G, R, T, d = 2, 2, 4, 16384, 128
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    _, kcb = oracle.compress_keys(K)
+    ora, kth, kth1 = oracle.select(F, kcb, k, n_init, n_local, T - 1)
+    got = gpu_select(F, kcb, k, n_init, n_local, T - 1, T, Hq=G * R)
+    check_sets(got, ora, kth, kth1, scores_f64(F, kcb), "budget")
+    idx = got[:, 0]
+    S = k + n_init + n_local
+    assert idx.shape[-1] == S and (idx >= 0).all()
+    o = gpu_decode(Q, K, V, idx, T, k, n_init, n_local)
+    ora_o = oracle.sparse_attention(Q.reshape(B, 1, G * R, d), K, V, idx.reshape(B, 1, G, S), T - 1, T)
+    check_attention(o.reshape(B, 1, G * R, d), ora_o, "budget attention")
 
 
 # --------------------------------------------------------------------------
