@@ -190,6 +190,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
   }
 }
 
+// Device-scope ticket with acquire-release ordering.
+__device__ __forceinline__ unsigned ticket_acq_rel(uint32_t *p) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
 // End of a segment, run by the 128 correction threads (thread = output
 // dim): normalise and write the pair's output if this CTA covers the whole
 // pair, else store the segment's (max, sum, unnormalised output) and let the
@@ -216,16 +223,18 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
     }
   }
   if (n_cover > 1) {
-    __threadfence();
+    // the barrier orders every correction thread's stores before the ticket,
+    // whose release publishes them device-wide; the last CTA's acquire (and
+    // the barrier after it) orders its loads of the other segments after
     named_sync(kBarCorr, 128);
-    if (dim == 0) *s_last = (atomicAdd(&a.counters[pair], 1u) == (unsigned)(n_cover - 1));
+    if (dim == 0) *s_last = (ticket_acq_rel(&a.counters[pair]) == (unsigned)(n_cover - 1));
     named_sync(kBarCorr, 128);
     if (*s_last) {
-      // merge the pair's segments online, four heads at a time; a segment's
-      // loads for those heads are independent, so they are in flight together
-      __threadfence();
+      // merge the pair's segments online, up to four heads at a time, with
+      // the loads of several segments in flight together
       const long long base = pair * a.max_cover;
       constexpr int HC = R < 4 ? R : 4;
+      constexpr int NBAT = 8 / HC;
 #pragma unroll 1
       for (int h0 = 0; h0 < R; h0 += HC) {
         float M[HC], L[HC], o[HC];
@@ -236,22 +245,30 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
           o[h] = 0.f;
         }
 #pragma unroll 1
-        for (int c = 0; c < n_cover; ++c) {
-          float2 ml[HC];
-          float ov[HC];
+        for (int c0 = 0; c0 < n_cover; c0 += NBAT) {
+          float2 ml[NBAT][HC];
+          float ov[NBAT][HC];
 #pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            ml[h] = __ldcg(&a.ws_ml[(base + c) * R + h0 + h]);
-            ov[h] = __ldcg(&a.ws_o[((base + c) * R + h0 + h) * kD + dim]);
+          for (int q = 0; q < NBAT; ++q) {
+#pragma unroll
+            for (int h = 0; h < HC; ++h) {
+              const bool in = c0 + q < n_cover;
+              const long long sl = base + c0 + q;
+              ml[q][h] = in ? __ldcg(&a.ws_ml[sl * R + h0 + h]) : make_float2(-INFINITY, 0.f);
+              ov[q][h] = in ? __ldcg(&a.ws_o[(sl * R + h0 + h) * kD + dim]) : 0.f;
+            }
           }
 #pragma unroll
-          for (int h = 0; h < HC; ++h) {
-            if (ml[h].x == -INFINITY) continue;  // a segment with no keys
-            const float mn = fmaxf(M[h], ml[h].x);
-            const float f_old = exp2f(M[h] - mn), f_new = exp2f(ml[h].x - mn);
-            L[h] = L[h] * f_old + ml[h].y * f_new;
-            o[h] = o[h] * f_old + ov[h] * f_new;
-            M[h] = mn;
+          for (int q = 0; q < NBAT; ++q) {
+#pragma unroll
+            for (int h = 0; h < HC; ++h) {
+              if (ml[q][h].x == -INFINITY) continue;  // a segment with no keys, or none
+              const float mn = fmaxf(M[h], ml[q][h].x);
+              const float f_old = exp2f(M[h] - mn), f_new = exp2f(ml[q][h].x - mn);
+              L[h] = L[h] * f_old + ml[q][h].y * f_new;
+              o[h] = o[h] * f_old + ov[q][h] * f_new;
+              M[h] = mn;
+            }
           }
         }
 #pragma unroll
