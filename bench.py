@@ -675,6 +675,8 @@ def run_sparda(args):
                "host_link_GBps": fetched / (e_ms * 1e-3) / 1e9,
                "host_link_peak_GBps": link_peak,
                "host_link_frac": fetched / (e_ms * 1e-3) / 1e9 / link_peak,
+               # the wait the gather adds to each layer over the all-resident step
+               "exposed_wait_us_per_layer": (e_ms - ms_step) * 1e3 / L,
                "note": "K/V in pinned host memory; every layer's top-k blocks gathered over the "
                        "host link on a side stream (cold sets, no reuse across steps)"}
         e2e["slot_cache"] = run_slot_cache_legs(loop, args, world, ms_step)
@@ -777,7 +779,8 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
                     "ms_per_step": ms, "fetched_blocks_per_step": per_step,
                     "fetched_frac_of_topk": per_step / topk_entries,
                     "host_link_bytes_per_step": int(per_step * loop.blk_elems * 2),
-                    "step_vs_resident": ms / resident_ms})
+                    "step_vs_resident": ms / resident_ms,
+                    "exposed_wait_us_per_layer": (ms - resident_ms) * 1e3 / L})
         del loop.cache, loop.block_of, loop.hand, loop.phys, loop.fetch, loop.h_F_steps
         torch.cuda.empty_cache()
     return out
@@ -922,7 +925,10 @@ def run_windows(steps):
         abi.sparda_forecast_select_windows(p, F, 1, 1, w.T - 1, kws[l], 32, 16, idx, ws[l])
         t[0] += 1
     us = time_back_to_back(sel, n)
-    nbytes = w.B * w.G * NW * w.d * 2
+    # the three windows inside each candidate block (the straddling fourth
+    # window of a block is never scored, and never read)
+    ncand = (w.T - 1) // w.blk - w.n_local + 1 - w.n_init
+    nbytes = w.B * w.G * ncand * 3 * w.d * 2
     out.update({"decode_select_us": us, "decode_select_GBps": nbytes / (us * 1e-6) / 1e9,
                 "decode_window_key_bytes": nbytes})
     del kws
