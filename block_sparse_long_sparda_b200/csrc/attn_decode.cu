@@ -27,10 +27,12 @@
 //    scan (one global-load latency per CTA);
 //  - TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) stages each
 //    block as [K lo-dims | V lo-dims | K hi-dims | V hi-dims] (8 KB each) in
-//    an NSTAGE ring; the pair's query rows are loaded into the S^T issuer's
-//    registers one segment ahead.  The M = 128 MMA for S^T reads rows 0-63 =
-//    the block's keys; its rows 64-127 alias the V tiles and are never read
-//    back;
+//    an NSTAGE ring, the K and the V tiles of a slot with barriers of their
+//    own (for blocks that come from L2, K is refilled once S^T has read it
+//    and V once O^T has, so V waits less in the slot); the pair's query rows
+//    are loaded into the S^T issuer's registers one segment ahead.  The
+//    M = 128 MMA for S^T reads rows 0-63 = the block's keys; its rows 64-127
+//    alias the V tiles (which may still be loading) and are never read back;
 //  - one thread issues the MMAs (N = 16: the group's heads, zero padded);
 //    softmax per head in the exp2 domain over the thread-per-key rows of
 //    S^T; P^T goes to shared memory as a bf16 K-major operand (the sum of
@@ -113,6 +115,8 @@ struct TcArgs {
   int order_bgi;        // 1: pairs are streamed in (sequence, group, token) order
   int n_slots;          // SPARDA_ADDR_PHYS: slots per (sequence, group)
   int T;
+  int split_kv;         // 1: a slot's K and V tiles are refilled separately (see the producer;
+                        // picks the kernel instance, 2 or 3 stages)
   float scale_log2;
 };
 
@@ -129,9 +133,11 @@ __device__ __forceinline__ long long mem_pair(const TcArgs &a, long long p) {
 // Everything else a CTA keeps in shared memory; it sits in the dynamic
 // allocation behind the operands, so the kernel has no static shared memory
 // and the allocation starts on the 1024-byte boundary the swizzled tiles need.
-template <int NSTAGE>
+template <int NSTAGE, bool SPLIT>
 struct TcCtl {
-  uint64_t full_bar[NSTAGE], empty_bar[NSTAGE];
+  uint64_t full_bar[NSTAGE], empty_bar[NSTAGE];    // a slot's K tiles: landed / read by S^T
+  // with SPLIT, its V tiles: landed / read by O^T (else unused)
+  uint64_t fullv_bar[SPLIT ? NSTAGE : 1], emptyv_bar[SPLIT ? NSTAGE : 1];
   uint64_t s_full[2], p_full[2], o_full[2], o_free[2];
   uint32_t tmem_base;
   int s_last;
@@ -147,9 +153,10 @@ struct TcCtl {
 };
 
 // stages | Q^T operand (16 rows x 128 dims) | two P^T operands | control
-template <int NSTAGE>
+template <int NSTAGE, bool SPLIT>
 constexpr size_t tc_smem() {
-  return (size_t)NSTAGE * kUnitBytes + 4096 + 2 * 2048 + (sizeof(TcCtl<NSTAGE>) + 127) / 128 * 128;
+  return (size_t)NSTAGE * kUnitBytes + 4096 + 2 * 2048 +
+         (sizeof(TcCtl<NSTAGE, SPLIT>) + 127) / 128 * 128;
 }
 
 constexpr int kWarps = 9;               // 4 correction, producer, 2 MMA issuers, 2 softmax warps
@@ -289,7 +296,7 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
 // (S^T, softmax, O^T): a stage is held from its landing until its O^T MMA is
 // done, and more chains hide that hold better.  Sixteen heads per group need
 // more registers than three CTAs per SM allow.
-template <int R, int NSTAGE>
+template <int R, int NSTAGE, bool SPLIT>
 __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    TcArgs a) {
@@ -298,8 +305,9 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   uint8_t *stages = sm;                          // NSTAGE x 32 KB
   uint8_t *qop = sm + NSTAGE * kUnitBytes;       // Q^T operand: 16 rows x 128 dims
   uint8_t *pop = qop + 4096;                     // two P^T operands: 16 rows x 64 keys
-  TcCtl<NSTAGE> &ctl = *reinterpret_cast<TcCtl<NSTAGE> *>(pop + 2 * 2048);
+  TcCtl<NSTAGE, SPLIT> &ctl = *reinterpret_cast<TcCtl<NSTAGE, SPLIT> *>(pop + 2 * 2048);
   uint64_t *full_bar = ctl.full_bar, *empty_bar = ctl.empty_bar;
+  uint64_t *fullv_bar = ctl.fullv_bar, *emptyv_bar = ctl.emptyv_bar;
   uint64_t *s_full = ctl.s_full, *p_full = ctl.p_full, *o_full = ctl.o_full, *o_free = ctl.o_free;
   int *s_row = ctl.s_row, *s_rows = ctl.s_rows, *s_seg = ctl.s_seg;
   volatile int *s_abort = &ctl.s_abort;
@@ -328,6 +336,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     for (int st = 0; st < NSTAGE; ++st) {
       mbar_init(&full_bar[st], 1);
       mbar_init(&empty_bar[st], 1);
+      if (SPLIT) {
+        mbar_init(&fullv_bar[st], 1);
+        mbar_init(&emptyv_bar[st], 1);
+      }
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -398,14 +410,24 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   auto first_of = [&](int u) { return u == 0 || s_seg[u - 1] != s_seg[u]; };
   auto last_of = [&](int u) { return u == nb - 1 || s_seg[u + 1] != s_seg[u]; };
 
-  int produced = 0;  // producer: blocks whose TMA was issued
+  int produced_k = 0, produced_v = 0;  // producer: blocks whose K / V loads were issued
 
   if (warp == kWarpProducer) {
     // ================= producer =================
-    if (lane == 0) {
+    // A block's K and V tiles have barriers of their own.  With split_kv,
+    // K(u) goes out as soon as S^T(u - NSTAGE) has read its slot's K tiles
+    // and V(u) once O^T(u - NSTAGE) has read the V tiles: V is then issued
+    // later than K and lands about when the softmax of its block is done,
+    // so neither half waits long in its slot.  That pays when the blocks
+    // come from L2 (the prefill's shared blocks, ~1 us away), where the
+    // hold in the slot is a large part of a block's time; from HBM (decode,
+    // ~4 us under load) it does not, and both halves go out together.
+    if (lane == 0 && !SPLIT) {
 #pragma unroll 1
       for (int u = 0; u < nb; ++u) {
         const int st = u % NSTAGE;
+        // one barrier per slot: all four tiles land on full_bar, and O^T
+        // (the last reader) frees the slot on empty_bar
         if (u >= NSTAGE &&
             !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), s_abort))
           break;
@@ -416,13 +438,55 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
         tc::tma_load_2d(dst + kTile, &mapV, 0, row, &full_bar[st]);
         tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
         tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &full_bar[st]);
-        produced = u + 1;
+        produced_k = u + 1;
+      }
+    } else if (lane == 0) {
+      int uk = 0, uv = 0;
+      long long t0 = clock64();
+#pragma unroll 1
+      while (uv < nb) {
+        bool moved = false;
+        if (uk < nb &&
+            (uk < NSTAGE ||
+             mbar_test_wait(&empty_bar[uk % NSTAGE], (uint32_t)(((uk / NSTAGE) - 1) & 1)))) {
+          const int st = uk % NSTAGE;
+          uint8_t *dst = stages + st * kUnitBytes;
+          const int row = s_row[uk];
+          mbar_arrive_expect_tx(&full_bar[st], 2 * kTile);
+          tc::tma_load_2d(dst, &mapK, 0, row, &full_bar[st]);
+          tc::tma_load_2d(dst + 2 * kTile, &mapK, 64, row, &full_bar[st]);
+          produced_k = ++uk;
+          moved = true;
+        }
+        if (uv < uk &&
+            (uv < NSTAGE ||
+             mbar_test_wait(&emptyv_bar[uv % NSTAGE], (uint32_t)(((uv / NSTAGE) - 1) & 1)))) {
+          const int st = uv % NSTAGE;
+          uint8_t *dst = stages + st * kUnitBytes;
+          const int row = s_row[uv];
+          mbar_arrive_expect_tx(&fullv_bar[st], 2 * kTile);
+          tc::tma_load_2d(dst + kTile, &mapV, 0, row, &fullv_bar[st]);
+          tc::tma_load_2d(dst + 3 * kTile, &mapV, 64, row, &fullv_bar[st]);
+          produced_v = ++uv;
+          moved = true;
+        }
+        if (moved) {
+          t0 = clock64();
+          continue;
+        }
+        if (*s_abort) break;
+        if (clock64() - t0 > kWaitCycles) {
+          *s_abort = 1;
+          break;
+        }
+        __nanosleep(20);
       }
     }
   } else if (warp == kWarpMma) {
     // ================= S^T issuer =================
-    // S^T(u) as soon as its block has landed and the softmax of u-2 is done
-    // with S[u & 1].
+    // S^T(u) as soon as its block's K tiles have landed and the softmax of
+    // u-2 is done with S[u & 1]; with split_kv its completion frees the
+    // slot's K tiles.
     // The query rows of the next segment are loaded into registers one
     // segment ahead, so their global-load latency overlaps the current one.
     constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
@@ -470,6 +534,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
           tc::mma_bf16(tmem + (u & 1) * kNQ, base + (uint64_t)((k >> 2) * (2 * kTile >> 4) + (k & 3) * 2),
                        dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
         tc::mma_commit(&s_full[u & 1]);
+        if (SPLIT) tc::mma_commit(&empty_bar[st]);  // the slot's K tiles are read
       }
       __syncwarp();
       if (first) {  // the next segment's query rows, off the critical path
@@ -481,9 +546,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     if (!ok) *s_abort = 1;
   } else if (warp == kWarpMma2) {
     // ================= O^T issuer =================
-    // O^T(v) as soon as the softmax of v is done and the correction of v-2 has
-    // read O[v & 1]; its completion also frees the block's stage (the block's
-    // S^T finished before its softmax began).
+    // O^T(v) as soon as the softmax of v is done, its V tiles have landed and
+    // the correction of v-2 has read O[v & 1]; its completion frees the
+    // slot's V tiles (without split_kv: the whole slot, whose S^T finished
+    // before its softmax began).
     constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
     const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);
     const uint64_t dP = tc::sdesc(pop, 16, 1024);
@@ -493,6 +559,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       const int st = v % NSTAGE;
       ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
       if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), s_abort);
+      if (ok && SPLIT) ok = wait_or_abort(&fullv_bar[st], (uint32_t)((v / NSTAGE) & 1), s_abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       if (lane == 0) {
@@ -504,7 +571,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
           tc::mma_bf16(tmem + 2 * kNQ + (v & 1) * kNQ, base + (uint64_t)(k * 128), bp + (uint64_t)(k * 2),
                        id2, k > 0);
         tc::mma_commit(&o_full[v & 1]);
-        tc::mma_commit(&empty_bar[st]);
+        tc::mma_commit(SPLIT ? &emptyv_bar[st] : &empty_bar[st]);  // V tiles (or the slot) read
       }
       __syncwarp();
     }
@@ -643,8 +710,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     // land before the CTA's memory is released; the status word says why
     flag_status(a.status, SPARDA_DEV_TIMEOUT);
     if (warp == kWarpProducer && lane == 0) {
-      for (int u = max(0, produced - NSTAGE); u < produced; ++u)
+      for (int u = max(0, produced_k - NSTAGE); u < produced_k; ++u)
         (void)mbar_wait_bounded(&full_bar[u % NSTAGE], (uint32_t)((u / NSTAGE) & 1));
+      for (int u = max(0, produced_v - NSTAGE); u < produced_v; ++u)
+        (void)mbar_wait_bounded(&fullv_bar[u % NSTAGE], (uint32_t)((u / NSTAGE) & 1));
     }
   }
   tc::fence_before_sync();
@@ -653,11 +722,11 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   if (warp == 0) tc::tmem_dealloc(tmem, 64);
 }
 
-template <int R, int NSTAGE>
+template <int R, int NSTAGE, bool SPLIT>
 cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs &a,
                       long long grid_max, long long grid_min, cudaStream_t stream) {
-  constexpr size_t smem = tc_smem<NSTAGE>();
-  auto kern = attn_tc_kernel<R, NSTAGE>;
+  constexpr size_t smem = tc_smem<NSTAGE, SPLIT>();
+  auto kern = attn_tc_kernel<R, NSTAGE, SPLIT>;
   // per device, once: shared-memory attributes and how many CTAs stay
   // resident (one wave: as many CTAs as the device keeps resident, never
   // more than the plan sized the workspace for, never fewer than the lists
@@ -771,6 +840,8 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.q_start = q_start;
   a.max_cover = pl.max_cover;
   a.order_bgi = nq > 1 ? 1 : 0;
+  const int fsplit = env_int("SPARDA_SPLIT_KV");  // 1 / -1: force on / off
+  a.split_kv = fsplit != 0 ? (fsplit > 0 ? 1 : 0) : (nq > 1 ? 1 : 0);
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
   a.scale_log2 = scale * kLog2e;
   const size_t parts = (size_t)pairs * pl.max_cover * R;
@@ -785,11 +856,13 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   // 4 and 6 (one CTA per SM) stay selectable through SPARDA_DECODE_STAGES
   int stages = env_int("SPARDA_DECODE_STAGES");
   if (stages == 0) stages = R <= 8 ? 2 : 3;
-#define SPARDA_LAUNCH_R(RR)                                                             \
-  if (stages <= 2) return launch_tc<RR, 2>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (stages == 3) return launch_tc<RR, 3>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (stages == 4) return launch_tc<RR, 4>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  return launch_tc<RR, 6>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+#define SPARDA_LAUNCH_R(RR)                                                                    \
+  if (a.split_kv && stages <= 2) return launch_tc<RR, 2, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (a.split_kv && stages == 3) return launch_tc<RR, 3, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages <= 2) return launch_tc<RR, 2, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages == 3) return launch_tc<RR, 3, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  if (stages == 4) return launch_tc<RR, 4, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
+  return launch_tc<RR, 6, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
   switch (R) {
     case 1: SPARDA_LAUNCH_R(1)
     case 2: SPARDA_LAUNCH_R(2)
