@@ -832,3 +832,34 @@ def test_prefill_attention_parity(T, nq, R):
                                    torch.from_numpy(idx).cuda(), O, ws)
     torch.cuda.synchronize()
     check_attention(host_bits(O), ora, "prefill T=%d nq=%d" % (T, nq))
+
+
+@pytest.mark.parametrize("split", ["1", "-1"])
+@pytest.mark.parametrize("nq,R", [(1, 4), (1, 16), (96, 4)])
+def test_attention_both_slot_protocols(split, nq, R, monkeypatch):
+    """The attention kernel has two ring protocols: one barrier per slot
+    (the default for decode) and K and V tiles refilled separately (the
+    default for prefill).  Each is forced on the other workload too."""
+    monkeypatch.setenv("SPARDA_SPLIT_KV", split)
+    rng = W.rng_for(41, nq * 100 + R)
+    B, G, d, k, T = 2, 2, 128, 12, 6000 + 21
+    Hq = G * R
+    q_start = T - nq
+    Q = W.normal_bf16(rng, (B, nq, Hq, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, 1, 2, q_start)
+    ora = oracle.sparse_attention(Q, K, V, idx, q_start, T)
+    if nq == 1:
+        got = gpu_decode(Q.reshape(B, Hq, d), K, V, idx[:, 0], T, k)
+        check_attention(got.reshape(B, 1, Hq, d), ora, "decode split=%s R=%d" % (split, R))
+    else:
+        p = abi.make_params(B, Hq, G, T, k)
+        O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device="cuda")
+        ws = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
+        abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, q_start, dev_bf16(K), dev_bf16(V), T * d,
+                                       d, torch.from_numpy(idx).cuda(), O, ws)
+        torch.cuda.synchronize()
+        check_attention(host_bits(O), ora, "prefill split=%s" % split)
