@@ -571,7 +571,20 @@ def run_sparda(args):
     build.build()
     w = WORKLOAD
     want_e2e = not args.no_e2e
-    loop = DecodeLoop(w, with_host=want_e2e, seed_offset=rank)
+    loop = DecodeLoop(w, with_host=False, seed_offset=rank)
+    # the host-offload legs pin a 32 GiB host copy of this rank's K/V; every
+    # rank runs them or none does (their timings meet at collectives)
+    e2e_skip = None
+    if want_e2e:
+        try:
+            loop._setup_host()
+        except (RuntimeError, MemoryError) as exc:
+            e2e_skip = "pinned host copy of the K/V unavailable on rank %d: %s" % (rank, exc)
+            loop.unregister()
+        if max_over_ranks(1.0 if e2e_skip else 0.0, world) > 0:
+            want_e2e = False
+            loop.unregister()
+            e2e_skip = e2e_skip or "pinned host copy of the K/V unavailable on another rank"
     L = w.layers
 
     # every resident-step launch, its graph capture and its timing are on the
@@ -659,7 +672,7 @@ def run_sparda(args):
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
     traffic = profiled_traffic("attn_tc_kernel", loop.bytes_attn())
 
-    e2e = None
+    e2e = {"unavailable": e2e_skip} if e2e_skip else None
     if want_e2e:
         for _ in range(max(args.warmup, 3)):
             loop.step_e2e()
