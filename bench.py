@@ -73,7 +73,8 @@ def parse_args():
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
                          "K/V per attention launch), then two passes of a 512-token prefill "
-                         "chunk of one sequence, and exit: the small cases ncu captures")
+                         "chunk of one sequence, then two cold host gathers of one layer at B=2 "
+                         "(1.1 GB pinned), and exit: the small cases ncu captures")
     return ap.parse_args()
 
 
@@ -1078,7 +1079,19 @@ def run_profile_case():
     torch.cuda.synchronize()
     st2 = int(pc.status.item())
     print("profile case: prefill B=1, 512 tokens, device status %d" % st2)
-    if st != 0 or st2 != 0:
+    del pc
+    torch.cuda.empty_cache()
+    # the host gather: one layer of B=2 sequences (1.1 GB of K/V in pinned host
+    # memory), two cold gathers of every (b, g)'s 64 top-k blocks (33.5 MB)
+    wg = W.scaled(WORKLOAD, B=2, layers=1)
+    gl = DecodeLoop(wg, with_host=True)
+    for _ in range(2):
+        abi.sparda_prefetch_blocks(gl.p, gl.host_kv[0], gl.idx[0], gl.slots[0], True, 0, gl.status)
+    torch.cuda.synchronize()
+    st3 = int(gl.status.item())
+    gl.unregister()
+    print("profile case: host gather B=2, device status %d" % st3)
+    if st != 0 or st2 != 0 or st3 != 0:
         sys.exit(1)
 
 
