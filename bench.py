@@ -40,6 +40,7 @@ from block_sparse_long_sparda_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = W.WORKLOADS["decode_loop_b16_t128k"]
 METRIC = "decode tokens/s at B=16,T=128K (sparse attn+select, % HBM roofline); select us/layer"
+GRAPH_STEPS = 5  # decode steps per CUDA graph replay in the timed region
 
 
 def parse_args():
@@ -594,20 +595,36 @@ def run_sparda(args):
         for _ in range(max(args.warmup, 3)):
             loop.step_resident()
         # the whole 4-layer step is replayed from a CUDA graph: no host work and
-        # no launch gaps inside the timed region
-        step, graph = loop.step_resident, None
+        # no launch gaps inside the timed region.  A graph of GRAPH_STEPS
+        # consecutive steps (the step has no host dependency) pays one graph
+        # launch per GRAPH_STEPS steps; single-step replays make up the rest.
+        step, graph, graph_m = loop.step_resident, None, None
         try:
             torch.cuda.synchronize()
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=loop.main):
                 loop.step_resident()
             graph.replay()
+            graph_m = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_m, stream=loop.main):
+                for _ in range(GRAPH_STEPS):
+                    loop.step_resident()
+            graph_m.replay()
             torch.cuda.synchronize()
             step = graph.replay
         except Exception as exc:  # keep eager launches, and say so in the line
             print("note: graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
-            graph = None
+            graph = graph_m = None
             torch.cuda.synchronize()
+
+        def run_steps(n):
+            """n steps: multi-step graph replays, then single steps."""
+            if graph_m is not None:
+                for _ in range(n // GRAPH_STEPS):
+                    graph_m.replay()
+                n %= GRAPH_STEPS
+            for _ in range(n):
+                step()
         for _ in range(max(args.warmup, 3)):
             step()
         # clocks are sampled over a ~1 s busy window that contains the timed steps
@@ -617,7 +634,7 @@ def run_sparda(args):
         clocks = ClockSampler(local)
         for _ in range(pad):
             step()
-        ms = time_steps(step, args.steps, world)
+        ms = time_steps(lambda: run_steps(args.steps), 1, world)
         for _ in range(pad):
             step()
         torch.cuda.synchronize()
@@ -728,6 +745,7 @@ def run_sparda(args):
             "cpu_baseline": cpu,
             "gpu_launches": args.steps * L * 2,
             "cuda_graph": graph is not None,
+            "graph_steps": GRAPH_STEPS if graph_m is not None else 1,
             "device_status": st,
         }
         print(json.dumps(line), flush=True)
