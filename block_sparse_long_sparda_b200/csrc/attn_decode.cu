@@ -414,8 +414,9 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
 
   if (warp == kWarpProducer) {
     // ================= producer =================
-    // A block's K and V tiles have barriers of their own.  With split_kv,
-    // K(u) goes out as soon as S^T(u - NSTAGE) has read its slot's K tiles
+    // A block's K and V tiles have barriers of their own.  In the SPLIT
+    // variant (TcArgs::split_kv picks it), K(u) goes out as soon as
+    // S^T(u - NSTAGE) has read its slot's K tiles
     // and V(u) once O^T(u - NSTAGE) has read the V tiles: V is then issued
     // later than K and lands about when the softmax of its block is done,
     // so neither half waits long in its slot.  That pays when the blocks
@@ -485,8 +486,8 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   } else if (warp == kWarpMma) {
     // ================= S^T issuer =================
     // S^T(u) as soon as its block's K tiles have landed and the softmax of
-    // u-2 is done with S[u & 1]; with split_kv its completion frees the
-    // slot's K tiles.
+    // u-2 is done with S[u & 1]; in the SPLIT variant its completion frees
+    // the slot's K tiles.
     // The query rows of the next segment are loaded into registers one
     // segment ahead, so their global-load latency overlaps the current one.
     constexpr uint32_t id1 = tc::idesc_bf16(128, kNQ, false, false);
@@ -548,8 +549,8 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     // ================= O^T issuer =================
     // O^T(v) as soon as the softmax of v is done, its V tiles have landed and
     // the correction of v-2 has read O[v & 1]; its completion frees the
-    // slot's V tiles (without split_kv: the whole slot, whose S^T finished
-    // before its softmax began).
+    // slot's V tiles (outside the SPLIT variant: the whole slot, whose S^T
+    // finished before its softmax began).
     constexpr uint32_t id2 = tc::idesc_bf16(128, kNQ, true, false);
     const uint64_t dV = tc::sdesc(stages + kTile, 2 * kTile, 1024);
     const uint64_t dP = tc::sdesc(pop, 16, 1024);
