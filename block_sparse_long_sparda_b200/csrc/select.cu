@@ -240,6 +240,15 @@ __device__ int compact_kept(const uint32_t *keys, int n, uint32_t tau, int need,
   return min(limit, (int)((carry >> 16) + min(carry & 0xFFFFu, (uint32_t)need)));
 }
 
+// A block-list entry, stored with an L2 evict-last hint: the attention that
+// reads the list next streams hundreds of MB through L2 before it does, and
+// the list's 34 KB (B = 16) should still be there.
+__device__ __forceinline__ void st_list(int32_t *p, int v) {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(pol) : "memory");
+}
+
 // init | top-k | local | -1 padding.  With `fill_top`, the top-k part is the
 // first ntop candidates (every candidate is taken); otherwise it is written
 // by the caller.
@@ -257,7 +266,7 @@ __device__ void write_set(int32_t *out, const BlockParts &bp, int ntop, int S, b
     } else {
       v = -1;
     }
-    out[s] = v;
+    st_list(out + s, v);
   }
 }
 
@@ -472,7 +481,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
     find_threshold(keys, n, a.k, rs, tau, need);
     const int ntop = compact_kept(keys, n, tau, need, a.k, rs,
-                                  [&](int pos, int e) { top[pos] = bp.cand_lo + e; });
+                                  [&](int pos, int e) { st_list(top + pos, bp.cand_lo + e); });
     write_set(out, bp, ntop, a.S, false);
     return;
   }
@@ -493,7 +502,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __syncthreads();
   find_threshold(keys, ncand, a.k, rs, tau, need);
   const int ntop = compact_kept(keys, ncand, tau, need, a.k, rs,
-                                [&](int pos, int e) { top[pos] = bp.cand_lo + e; });
+                                [&](int pos, int e) { st_list(top + pos, bp.cand_lo + e); });
   write_set(out, bp, ntop, a.S, false);
   if (threadIdx.x == 0) a.counters[prob] = 0u;
 }
