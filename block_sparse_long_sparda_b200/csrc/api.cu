@@ -143,7 +143,6 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
   if (st != SPARDA_OK) return st;
   if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
   if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
-  if (p->seq_len && nq != 1) return SPARDA_EUNSUPPORTED;  // lengths: decode queries only
   if (nf > 16) return SPARDA_EUNSUPPORTED;
   if (p->B == 0) return SPARDA_OK;
   if (!F || !kw || !idx) return SPARDA_EINVAL;
@@ -163,7 +162,6 @@ int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf
   if (st != SPARDA_OK) return st;
   if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
   if (nf > 16) return SPARDA_EUNSUPPORTED;
-  if (p->seq_len && nq != 1) return SPARDA_EUNSUPPORTED;  // lengths: decode queries only
   if (p->B == 0) return SPARDA_OK;
   if (!F || !kc || !idx) return SPARDA_EINVAL;
   if (!aligned16(F) || !aligned16(kc) || !aligned16(idx)) return SPARDA_EINVAL;
@@ -293,7 +291,6 @@ int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, in
                                size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
-  if ((st = no_seq_len(p)) != SPARDA_OK) return st;
   if (nq < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
   if (p->B == 0) return SPARDA_OK;
   if (!Q || !K || !V || !idx || !O) return SPARDA_EINVAL;

@@ -374,9 +374,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       const int j = j_me;
       if (j >= 0) {
         int pos = a.q_start + (int)((pm / a.G) % a.nq);
-        if (a.seq_len) {  // decode with per-sequence lengths: the query is the last token
-          const int len = a.seq_len[pm / a.G];
-          pos = (len >= 1 && len <= a.T) ? len - 1 : -1;  // -1: every block is flagged
+        if (a.seq_len) {  // per-sequence lengths: the queries are the sequence's last nq tokens
+          const int len = a.seq_len[(pm / a.G) / a.nq];
+          pos = (len >= a.nq && len <= a.T) ? len - a.nq + (int)((pm / a.G) % a.nq)
+                                            : -1;  // -1: every block is flagged
         }
         const bool slot_bad =
             a.addr_mode == SPARDA_ADDR_PHYS && (phys_me < 0 || phys_me >= a.n_slots);

@@ -419,9 +419,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   int pos = a.q_start + i;
   int32_t *out = a.idx + prob * a.S;
   int rows_b = a.NB;  // key rows of this sequence (the row stride stays a.NB)
-  if (a.seq_len) {  // decode with per-sequence lengths: the query is the last token
+  if (a.seq_len) {  // per-sequence lengths: the queries are the sequence's last nq tokens
     const int len = a.seq_len[b];
-    if (len < 1 || len > a.T) {  // an invalid length: an empty set
+    if (len < a.nq || len > a.T) {  // an invalid length: an empty set
       if (chunk == 0)
         for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
       if (a.n_chunks > 1) {  // keep the ticket count of the problem right
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
       }
       return;
     }
-    pos = len - 1;
+    pos = len - a.nq + i;
     if (kPool > 1) rows_b = window_count(len);
   }
   const BlockParts bp = block_parts(pos, kBlk, a.n_init, a.n_local);

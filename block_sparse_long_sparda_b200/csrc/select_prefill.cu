@@ -54,6 +54,8 @@ struct PScoreArgs {
   int32_t *status;
   int G, nq, NB, ld, q_start, n_init, n_local;
   int n_rows;          // key rows per (b, g): blocks, or windows (kPool = 4)
+  const int32_t *seq_len;  // optional: the chunk is each sequence's last nq tokens
+  int T;
 };
 
 // kPool = 1: one key row per block, tile column c is block j0 + c.  kPool = 4
@@ -75,10 +77,21 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
   const int i0 = t * kPTok;
   const int w0 = u * kPBlk;       // first key row (block or window) of the tile
   const int j0 = w0 / kPool;      // first block of the tile
+  pdl_trigger();
+  // with per-sequence lengths the chunk is the sequence's last nq tokens (the
+  // length is read once the previous kernel is done); an invalid length
+  // leaves the rows to the ranking kernel, which writes empty sets
+  int qs = a.q_start, n_rows = a.n_rows;
+  if (a.seq_len) {
+    pdl_wait();
+    const int len = a.seq_len[b];
+    if (len < a.nq || len > a.T) return;
+    qs = len - a.nq;
+    if (kPool > 1) n_rows = window_count(len);
+  }
   // the candidates of the tile's last row reach furthest
   const int i_last = min(a.nq, i0 + kPTok) - 1;
-  const BlockParts bp_last = block_parts(a.q_start + i_last, kBlk, a.n_init, a.n_local);
-  pdl_trigger();
+  const BlockParts bp_last = block_parts(qs + i_last, kBlk, a.n_init, a.n_local);
   if (j0 >= bp_last.cand_hi || j0 + kPBlk / kPool <= a.n_init) return;  // no candidate in the tile
   if (smem_addr(smem) & 1023u) {
     pdl_wait();
@@ -130,7 +143,7 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
   } else {
     tc::fence_after_sync();
     const int i = i0 + tid;  // this thread's token row (TMEM lane tid)
-    const BlockParts bp = block_parts(a.q_start + min(i, a.nq - 1), kBlk, a.n_init, a.n_local);
+    const BlockParts bp = block_parts(qs + min(i, a.nq - 1), kBlk, a.n_init, a.n_local);
     uint32_t *row = a.keys + ((long long)pair * a.nq + i) * a.ld + j0;
     const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
 #pragma unroll 1
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
             float m = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 3; ++e)
-              if (w0 + c + 4 * q + e < a.n_rows) m = fmaxf(m, v[4 * q + e]);
+              if (w0 + c + 4 * q + e < n_rows) m = fmaxf(m, v[4 * q + e]);
             const int j = j0 + c / 4 + q;
             kk[q] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(m) : 0u;
           }
@@ -397,6 +410,8 @@ struct RankArgs {
   int32_t *idx;          // [B][nq][G][S]
   long long rows;        // B * nq * G
   int G, nq, ld, k, n_init, n_local, q_start, S;
+  const int32_t *seq_len;  // optional: the chunk is each sequence's last nq tokens
+  int T;
 };
 
 __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
@@ -410,7 +425,16 @@ __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
   const long long bi = row / a.G;
   const int i = (int)(bi % a.nq);
   const long long b = bi / a.nq;
-  const BlockParts bp = block_parts(a.q_start + i, kBlk, a.n_init, a.n_local);
+  int qs = a.q_start;
+  if (a.seq_len) {
+    const int len = a.seq_len[b];
+    if (len < a.nq || len > a.T) {  // an invalid length: an empty set
+      for (int s = lane; s < a.S; s += 32) a.idx[row * a.S + s] = -1;
+      return;
+    }
+    qs = len - a.nq;
+  }
+  const BlockParts bp = block_parts(qs + i, kBlk, a.n_init, a.n_local);
   const int ncand = bp.cand_hi - bp.cand_lo;
   int32_t *out = a.idx + row * a.S;
   const int nloc = bp.c - bp.local_lo + 1;
@@ -530,6 +554,8 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   sa.q_start = q_start;
   sa.n_init = p.n_init;
   sa.n_local = p.n_local;
+  sa.seq_len = p.seq_len;
+  sa.T = p.T;
   const dim3 grid((unsigned)(ld / (kPBlk / pool)), (unsigned)ceil_div_ll(nq, kPTok),
                   (unsigned)(p.B * p.G));
   cudaLaunchConfig_t cfg = {};
@@ -556,6 +582,8 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   ra.n_local = p.n_local;
   ra.q_start = q_start;
   ra.S = p.k + p.n_init + p.n_local;
+  ra.seq_len = p.seq_len;
+  ra.T = p.T;
   e = launch_pdl(rank_rows_kernel, (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream,
                  ra);
   return e != cudaSuccess ? e : cudaGetLastError();

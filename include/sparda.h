@@ -85,18 +85,20 @@ typedef struct sparda_params {
   int n_init;   /* initial blocks (>= 0, <= 64)                                */
   int n_local;  /* local-window blocks (>= 0, <= 64)                           */
   float scale;  /* attention logit scale; <= 0 means 1/sqrt(d)                 */
-  /* Optional device int32 [B]: tokens present in each sequence, 1 <= seq_len[b]
+  /* Optional device int32 [B]: tokens present in each sequence, seq_len[b]
    * <= T (T then only sizes the arrays).  Null: every sequence holds T tokens.
-   * Honoured by sparda_compress_keys and sparda_compress_windows (blocks past
-   * the end, and windows not complete inside the sequence, are left
-   * untouched), sparda_forecast_select and sparda_forecast_select_windows
-   * (nq = 1: the query of sequence b sits at seq_len[b] - 1),
-   * sparda_prefetch_blocks and the decode attention calls; the cache plan
-   * and the cached prefetch follow the lists they are given.
-   * sparda_append_kv and sparda_sparse_attn_prefill return
-   * SPARDA_EUNSUPPORTED when it is set.  A length outside [1, T] is flagged SPARDA_DEV_RANGE
-   * where a status word is given, and that sequence's outputs are left empty
-   * (a -1 set, a zero output). */
+   * With lengths, the nq query tokens of sequence b are its last nq tokens,
+   * positions seq_len[b] - nq .. seq_len[b] - 1 (a decode query is the last
+   * token), and the calls' q_start is not used.  Honoured by
+   * sparda_compress_keys and sparda_compress_windows (blocks past the end,
+   * and windows not complete inside the sequence, are left untouched),
+   * sparda_forecast_select and sparda_forecast_select_windows,
+   * sparda_prefetch_blocks, and the decode and prefill attention calls; the
+   * cache plan and the cached prefetch follow the lists they are given.
+   * sparda_append_kv returns SPARDA_EUNSUPPORTED when it is set.  A length
+   * outside [nq, T] (nq = 1 for decode and compression) gives that sequence
+   * empty outputs (-1 sets, zero attention output) and is flagged
+   * SPARDA_DEV_RANGE where a status word is given. */
   const int32_t *seq_len;
 } sparda_params;
 

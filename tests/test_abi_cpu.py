@@ -98,20 +98,13 @@ def test_workspace_sizes_scale_with_shapes(L):
     assert abi.sparda_workspace_size(abi.SPARDA_OP_PREFETCH, cfg3) == 0
 
 
-def test_calls_that_ignore_lengths_refuse_them():
-    """Per-sequence lengths are honoured by compression, decode selection,
-    prefetch and decode attention; append, prefill attention and selection
-    for more than one query token refuse them before touching any pointer
-    (so a dummy address is enough here)."""
+def test_append_refuses_lengths():
+    """Per-sequence lengths are honoured by every call but the decode append,
+    which takes one position for the batch; it refuses them before touching
+    any pointer (so a dummy address is enough here)."""
     p = abi.make_params(2, 8, 2, 4096, 16)
     p.seq_len = 4096  # any non-null value
     L = abi.lib()
     dummy = ctypes.c_void_p(16 * 1024)
     assert L.sparda_append_kv(ctypes.byref(p), 5, dummy, dummy, dummy, dummy, 4096 * 128, 64 * 128,
                               dummy, None, None) == abi.SPARDA_EUNSUPPORTED
-    assert L.sparda_forecast_select_windows(ctypes.byref(p), dummy, 64, 1, 0, dummy, 32, 16, dummy,
-                                            dummy, 1 << 20, None) == abi.SPARDA_EUNSUPPORTED
-    assert L.sparda_sparse_attn_prefill(ctypes.byref(p), dummy, 64, 0, dummy, dummy, 4096 * 128, 128,
-                                        dummy, dummy, dummy, 1 << 20, None, None) == abi.SPARDA_EUNSUPPORTED
-    assert L.sparda_forecast_select(ctypes.byref(p), dummy, 64, 1, 0, dummy, dummy, dummy, 1 << 20,
-                                    None) == abi.SPARDA_EUNSUPPORTED

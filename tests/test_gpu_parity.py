@@ -439,6 +439,81 @@ def test_varlen_window_grid(n_local, chunk, monkeypatch):
                    "varlen windows b=%d" % b)
 
 
+@pytest.mark.parametrize("nq,pool", [(96, 1), (5, 1), (80, 4), (3, 4)])
+def test_varlen_prefill_select(nq, pool):
+    """A prefill chunk per sequence of different lengths: each sequence's
+    chunk is its last nq tokens.  The tensor-core path (nq >= 64) and the
+    streaming path, on blocks and on the window grid; one sequence shorter
+    than the chunk gets empty sets."""
+    rng = W.rng_for(106, nq * 10 + pool)
+    B, G, T, d, k = 4, 2, 12000, 128, 10
+    lens = [T, 7000 + 13, 200, nq - 1]
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    NB = (T + 63) // 64
+    rows = NB if pool == 1 else oracle.window_count(T)
+    kc = W.normal_bf16(rng, (B, G, rows, d))
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G, G, T, k, seq_len=sl)
+    S = k + 3
+    idx = torch.full((B, nq, G, S), -7, dtype=torch.int32, device="cuda")
+    if pool == 1:
+        abi.sparda_forecast_select(p, dev_bf16(F), nq, 1, T - nq, dev_bf16(kc), idx,
+                                   abi.workspace(abi.SPARDA_OP_SELECT, p, nq, 1))
+    else:
+        abi.sparda_forecast_select_windows(p, dev_bf16(F), nq, 1, T - nq, dev_bf16(kc), 32, 16, idx,
+                                           abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, nq, 1))
+    torch.cuda.synchronize()
+    got = idx.cpu().numpy()
+    for b, L in enumerate(lens):
+        if L < nq:
+            assert np.all(got[b] == -1), "invalid length b=%d" % b
+            continue
+        Fb = F[b:b + 1]
+        if pool == 1:
+            kb = np.ascontiguousarray(kc[b:b + 1, :, :(L + 63) // 64])
+            ora, kth, kth1 = oracle.select(Fb, kb, k, 1, 2, L - nq)
+            sc = scores_f64(Fb, kb)
+        else:
+            kb = np.ascontiguousarray(kc[b:b + 1, :, :oracle.window_count(L)])
+            ora, kth, kth1 = oracle.select_windows(Fb, kb, L, k, 1, 2, L - nq)
+            sc = pooled_scores_f64(Fb, kb, (L + 63) // 64)
+        check_sets(got[b:b + 1], ora, kth, kth1, sc, "varlen prefill b=%d" % b)
+
+
+def test_varlen_prefill_attention():
+    """Prefill attention with a chunk per sequence at its own end; a sequence
+    shorter than the chunk gets a zero output and the range bit."""
+    rng = W.rng_for(107)
+    B, G, R, T, d, k, nq = 3, 2, 4, 5000, 128, 8, 70
+    lens = [T, 2000 + 31, nq - 5]
+    Q = W.normal_bf16(rng, (B, nq, G * R, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    S = k + 3
+    idx = np.full((B, nq, G, S), -1, np.int32)
+    for b, L in enumerate(lens[:2]):
+        _, kcb = oracle.compress_keys(np.ascontiguousarray(K[b:b + 1, :, :L]))
+        idx[b:b + 1], _, _ = oracle.select(F[b:b + 1], kcb, k, 1, 2, L - nq)
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * R, G, T, k, seq_len=sl)
+    O = torch.full((B, nq, G * R, d), 5.0, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # the short sequence is given a list anyway, so its blocks are flagged
+    idx[2] = idx[1]
+    abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, T - nq, dev_bf16(K), dev_bf16(V), T * d, d,
+                                   torch.from_numpy(idx).cuda(), O,
+                                   abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq), status)
+    torch.cuda.synchronize()
+    got = host_bits(O)
+    for b, L in enumerate(lens[:2]):
+        ora = oracle.sparse_attention(Q[b:b + 1], np.ascontiguousarray(K[b:b + 1, :, :L]),
+                                      np.ascontiguousarray(V[b:b + 1, :, :L]), idx[b:b + 1], L - nq, L)
+        check_attention(got[b:b + 1], ora, "varlen prefill attention b=%d" % b)
+    assert torch.all(O[2] == 0)
+    assert abi.sparda_status_from_device(int(status.item())) == abi.SPARDA_ERANGE
+
+
 @pytest.mark.parametrize("k,n_init,n_local", [(63, 1, 32), (24, 1, 16)])
 def test_real_model_budget(k, n_init, n_local):
     """A real model's budget: 96 blocks of which 32 (2048 tokens) are the
