@@ -34,7 +34,6 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARDA_OK : SPARDA_ECUD
 
 // calls that do not read per-sequence lengths refuse them rather than
 // silently using T for every sequence
-int no_seq_len(const sparda_params *p) { return p->seq_len ? SPARDA_EUNSUPPORTED : SPARDA_OK; }
 
 bool stride_ok(long long s) { return s > 0 && (s % 8) == 0; }
 
@@ -101,8 +100,7 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
                      void *kc_bf16, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
-  if ((st = no_seq_len(p)) != SPARDA_OK) return st;
-  if (pos < 0 || pos >= p->T) return SPARDA_EINVAL;
+  if (!p->seq_len && (pos < 0 || pos >= p->T)) return SPARDA_EINVAL;
   if (p->B == 0) return SPARDA_OK;
   if (!K_new || !V_new || !K || !V || (!kc_f32 && !kc_bf16)) return SPARDA_EINVAL;
   if (!aligned16(K_new) || !aligned16(V_new) || !aligned16(K) || !aligned16(V) ||

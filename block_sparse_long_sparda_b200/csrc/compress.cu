@@ -96,7 +96,8 @@ __global__ void __launch_bounds__(256, 3) compress_kernel(const uint16_t *__rest
   }
 }
 
-// One decode token appended: write its K and V rows at position `pos` and
+// One decode token appended: write its K and V rows at position `pos` (with
+// per-sequence lengths, at each sequence's last position) and
 // recompute the compressed key of its block -- the one block whose mean
 // changes.  One warp per (b, g).  The block's earlier rows are summed from
 // memory in the same per-half, ascending-row order as compress_kernel and
@@ -108,10 +109,16 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict_
                                                      uint16_t *__restrict__ V, long long bg_stride,
                                                      long long blk_stride, int pos, int NB,
                                                      long long n_pairs, float *__restrict__ kc32,
-                                                     uint16_t *__restrict__ kc16) {
+                                                     uint16_t *__restrict__ kc16,
+                                                     const int32_t *seq_len, int G, int T) {
   const int lane = threadIdx.x & 31;
   const long long bg = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (bg >= n_pairs) return;
+  if (seq_len) {  // per-sequence lengths: the new token is the sequence's last one
+    const int len = seq_len[bg / G];
+    if (len < 1 || len > T) return;  // an invalid length: nothing is appended
+    pos = len - 1;
+  }
   const int half = lane >> 4, c8 = lane & 15;
   const int c = pos / kBlk, r = pos - c * kBlk;  // block and row of the new token
   const long long blk_off = bg * bg_stride + (long long)c * blk_stride + c8 * 8;
@@ -194,7 +201,7 @@ cudaError_t launch_append(const sparda_params &p, int pos, const uint16_t *K_new
   const int NB = (p.T + kBlk - 1) / kBlk;
   const int warps = 8;
   append_kernel<<<(unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream>>>(
-      K_new, V_new, K, V, bg_stride, blk_stride, pos, NB, pairs, kc32, kc16);
+      K_new, V_new, K, V, bg_stride, blk_stride, pos, NB, pairs, kc32, kc16, p.seq_len, p.G, p.T);
   return cudaGetLastError();
 }
 

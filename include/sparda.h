@@ -94,8 +94,9 @@ typedef struct sparda_params {
    * and windows not complete inside the sequence, are left untouched),
    * sparda_forecast_select and sparda_forecast_select_windows,
    * sparda_prefetch_blocks, and the decode and prefill attention calls; the
-   * cache plan and the cached prefetch follow the lists they are given.
-   * sparda_append_kv returns SPARDA_EUNSUPPORTED when it is set.  A length
+   * cache plan and the cached prefetch follow the lists they are given;
+   * sparda_append_kv writes each sequence's new token at seq_len[b] - 1 (an
+   * invalid length appends nothing there).  A length
    * outside [nq, T] (nq = 1 for decode and compression) gives that sequence
    * empty outputs (-1 sets, zero attention output) and is flagged
    * SPARDA_DEV_RANGE where a status word is given. */
@@ -146,7 +147,9 @@ int sparda_compress_keys(const sparda_params *p, const void *K, long long bg_str
  *            base + (b*G+g)*bg_stride + (t/blk)*blk_stride + (t%blk)*d
  *          ([B][G][T][d]: bg_stride = T*d, blk_stride = blk*d; interleaved
  *          [..][NB][2][blk][d]: V = K + blk*d, blk_stride = 2*blk*d)
- * pos      the new token's position, 0 <= pos < T (T sizes the Kc arrays)
+ * pos      the new token's position, 0 <= pos < T (T sizes the Kc arrays);
+ *          not used with per-sequence lengths (p->seq_len), where sequence
+ *          b's token goes to seq_len[b] - 1
  * kc_f32, kc_bf16  as for sparda_compress_keys, [B][G][NB][d]; only block
  *          pos/blk is written.  The value is bit-identical to what
  *          sparda_compress_keys computes over positions 0..pos.

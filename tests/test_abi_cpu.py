@@ -96,15 +96,3 @@ def test_workspace_sizes_scale_with_shapes(L):
     # the workspace of an op with no scratch is zero
     assert abi.sparda_workspace_size(abi.SPARDA_OP_COMPRESS, cfg3) == 0
     assert abi.sparda_workspace_size(abi.SPARDA_OP_PREFETCH, cfg3) == 0
-
-
-def test_append_refuses_lengths():
-    """Per-sequence lengths are honoured by every call but the decode append,
-    which takes one position for the batch; it refuses them before touching
-    any pointer (so a dummy address is enough here)."""
-    p = abi.make_params(2, 8, 2, 4096, 16)
-    p.seq_len = 4096  # any non-null value
-    L = abi.lib()
-    dummy = ctypes.c_void_p(16 * 1024)
-    assert L.sparda_append_kv(ctypes.byref(p), 5, dummy, dummy, dummy, dummy, 4096 * 128, 64 * 128,
-                              dummy, None, None) == abi.SPARDA_EUNSUPPORTED

@@ -769,6 +769,50 @@ def test_append_matches_full_compression(interleaved):
     check_compressed(kc32.cpu().numpy(), host_bits(kc16), o64, o16)
 
 
+def test_append_per_sequence_positions():
+    """With per-sequence lengths each sequence appends its new token at its
+    own last position (seq_len[b] - 1); the rows land there, and the block's
+    compressed key equals a full compression of that sequence, bit for bit.
+    A sequence with an invalid length is left untouched."""
+    rng = W.rng_for(52)
+    B, G, d, T = 4, 2, 128, 300
+    lens = [250, 130, 64, 0]
+    NB = (T + 63) // 64
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    newK = W.normal_bf16(rng, (B, G, d))
+    newV = W.normal_bf16(rng, (B, G, d))
+    Kd, Vd = dev_bf16(K), dev_bf16(V)
+    kc32 = torch.full((B, G, NB, d), 9.0, dtype=torch.float32, device="cuda")
+    kc16 = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G, G, T, 1, seq_len=sl)
+    abi.sparda_append_kv(p, 0, dev_bf16(newK), dev_bf16(newV), Kd, Vd, T * d, 64 * d, kc32, kc16)
+    # the reference: the same caches with the rows written on the host,
+    # compressed in full up to each sequence's length
+    Kr, Vr = K.copy(), V.copy()
+    for b, L in enumerate(lens):
+        if L >= 1:
+            Kr[b, :, L - 1] = newK[b]
+            Vr[b, :, L - 1] = newV[b]
+    r32 = torch.zeros(B, G, NB, d, dtype=torch.float32, device="cuda")
+    r16 = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_compress_keys(p, dev_bf16(Kr), T * d, d, r32, r16)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(Kd), Kr) and np.array_equal(host_bits(Vd), Vr)
+    got32, got16, ref32, ref16 = kc32.cpu(), kc16.cpu(), r32.cpu(), r16.cpu()
+    for b, L in enumerate(lens):
+        if L < 1:
+            assert torch.all(got32[b] == 9.0)
+            continue
+        c = (L - 1) // 64
+        assert torch.equal(got32[b, :, c], ref32[b, :, c]) and torch.equal(got16[b, :, c], ref16[b, :, c])
+        o64, _ = oracle.compress_keys(np.ascontiguousarray(Kr[b:b + 1, :, :L]))
+        assert np.abs(got32[b, :, c].numpy() - o64[0, :, c]).max() <= 1e-3
+        others = [j for j in range(NB) if j != c]
+        assert torch.all(got32[b, :, others] == 9.0)  # only the token's block is written
+
+
 # --------------------------------------------------------------------------
 # device slot cache across decode steps
 # --------------------------------------------------------------------------
