@@ -74,6 +74,7 @@ _SIGS = {
     "sparda_compress_keys": (_I, [_PP, _P, _LL, _LL, _P, _P, _P]),
     "sparda_forecast_select": (_I, [_PP, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "sparda_append_kv": (_I, [_PP, _I, _P, _P, _P, _P, _LL, _LL, _P, _P, _P]),
+    "sparda_append_windows": (_I, [_PP, _I, _P, _LL, _LL, _I, _I, _P, _P, _P]),
     "sparda_compress_windows": (_I, [_PP, _P, _LL, _LL, _I, _I, _P, _P, _P]),
     "sparda_forecast_select_windows": (_I, [_PP, _P, _I, _I, _I, _P, _I, _I, _P, _P, _SZ, _P]),
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
@@ -151,6 +152,14 @@ def sparda_append_kv(p, pos, K_new, V_new, K, V, bg_stride, blk_stride, kc_f32, 
            lib().sparda_append_kv(ctypes.byref(p), int(pos), _ptr(K_new), _ptr(V_new), _ptr(K),
                                   _ptr(V), int(bg_stride), int(blk_stride), _ptr(kc_f32),
                                   _ptr(kc_bf16), _stream(stream)))
+
+
+def sparda_append_windows(p, pos, K, bg_stride, blk_stride, win, stride, kw_f32, kw_bf16,
+                          stream=None):
+    _check("sparda_append_windows",
+           lib().sparda_append_windows(ctypes.byref(p), int(pos), _ptr(K), int(bg_stride),
+                                       int(blk_stride), int(win), int(stride), _ptr(kw_f32),
+                                       _ptr(kw_bf16), _stream(stream)))
 
 
 def sparda_compress_windows(p, K, bg_stride, tok_stride, win, stride, kw_f32, kw_bf16,

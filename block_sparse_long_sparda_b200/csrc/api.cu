@@ -115,6 +115,24 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int sparda_append_windows(const sparda_params *p, int pos, const void *K, long long bg_stride,
+                          long long blk_stride, int win, int stride, float *kw_f32, void *kw_bf16,
+                          sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
+  if (!p->seq_len && (pos < 0 || pos >= p->T)) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!K || (!kw_f32 && !kw_bf16)) return SPARDA_EINVAL;
+  if (!aligned16(K) || (kw_f32 && !aligned16(kw_f32)) || (kw_bf16 && !aligned16(kw_bf16)))
+    return SPARDA_EINVAL;
+  if (!stride_ok(bg_stride) || !stride_ok(blk_stride) || blk_stride < (long long)kBlk * kD)
+    return SPARDA_EINVAL;
+  return from_cuda(launch_append_windows(*p, pos, static_cast<const uint16_t *>(K), bg_stride,
+                                         blk_stride, kw_f32, static_cast<uint16_t *>(kw_bf16),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int sparda_compress_windows(const sparda_params *p, const void *K, long long bg_stride,
                             long long tok_stride, int win, int stride, float *kw_f32,
                             void *kw_bf16, sparda_stream_t stream) {

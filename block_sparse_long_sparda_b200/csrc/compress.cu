@@ -167,7 +167,76 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict_
   }
 }
 
+// One decode token appended, window grid: if the token at `pos` (with
+// per-sequence lengths, each sequence's last position) completes a window --
+// pos = w*16 + 31 -- write that window's mean.  Rows are read through the
+// cache's block layout, so the interleaved K|V blocks work too.  The sum
+// runs in compress_kernel's order (even rows in one half-warp, odd rows in
+// the other, each ascending, then the halves added), so in the [T][d] layout
+// the key is bit-identical to compressing the windows again.
+__global__ void __launch_bounds__(256) append_window_kernel(
+    const uint16_t *__restrict__ K, long long bg_stride, long long blk_stride, int pos, int NW,
+    long long n_pairs, float *__restrict__ kw32, uint16_t *__restrict__ kw16,
+    const int32_t *seq_len, int G, int T) {
+  constexpr int kWin = 32, kStride = 16;
+  const int lane = threadIdx.x & 31;
+  const long long bg = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (bg >= n_pairs) return;
+  if (seq_len) {
+    const int len = seq_len[bg / G];
+    if (len < 1 || len > T) return;  // an invalid length: nothing is appended
+    pos = len - 1;
+  }
+  if (pos < kWin - 1 || (pos - (kWin - 1)) % kStride != 0) return;  // no window ends here
+  const int w = (pos - (kWin - 1)) / kStride;
+  if (w >= NW) return;
+  const int half = lane >> 4, c8 = lane & 15;
+  const uint16_t *base = K + bg * bg_stride + c8 * 8;
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  uint4 v[kWin / 2];
+#pragma unroll
+  for (int u = 0; u < kWin / 2; ++u) {
+    const int t = w * kStride + 2 * u + half;
+    v[u] = ldg_plain(base + (long long)(t / kBlk) * blk_stride + (long long)(t % kBlk) * kD);
+  }
+#pragma unroll
+  for (int u = 0; u < kWin / 2; ++u) acc8(a, v[u]);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+  if (half) return;
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = a[e] / (float)kWin;
+  const long long item = bg * NW + w;
+  if (kw32) {
+    float4 *o = reinterpret_cast<float4 *>(kw32 + item * kD + c8 * 8);
+    o[0] = make_float4(m[0], m[1], m[2], m[3]);
+    o[1] = make_float4(m[4], m[5], m[6], m[7]);
+  }
+  if (kw16) {
+    uint32_t q[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e]));
+      uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(m[2 * e + 1]));
+      q[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(kw16 + item * kD + c8 * 8) = make_uint4(q[0], q[1], q[2], q[3]);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_append_windows(const sparda_params &p, int pos, const uint16_t *K,
+                                  long long bg_stride, long long blk_stride, float *kw32,
+                                  uint16_t *kw16, cudaStream_t stream) {
+  const long long pairs = (long long)p.B * p.G;
+  if (pairs == 0) return cudaSuccess;
+  const int warps = 8;
+  append_window_kernel<<<(unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream>>>(
+      K, bg_stride, blk_stride, pos, window_count(p.T), pairs, kw32, kw16, p.seq_len, p.G, p.T);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
                             long long tok_stride, float *kc32, uint16_t *kc16,

@@ -56,6 +56,11 @@ cudaError_t launch_compress_runs(const sparda_params &p, const uint16_t *K, long
                                  long long tok_stride, int rows, int step, float *kc32,
                                  uint16_t *kc16, cudaStream_t stream);
 
+// one decode token on the window grid: the key of the window it completes
+cudaError_t launch_append_windows(const sparda_params &p, int pos, const uint16_t *K,
+                                  long long bg_stride, long long blk_stride, float *kw32,
+                                  uint16_t *kw16, cudaStream_t stream);
+
 // one decode token: write its K/V rows at `pos`, recompute its block's key
 cudaError_t launch_append(const sparda_params &p, int pos, const uint16_t *K_new,
                           const uint16_t *V_new, uint16_t *K, uint16_t *V, long long bg_stride,

@@ -95,8 +95,8 @@ typedef struct sparda_params {
    * sparda_forecast_select and sparda_forecast_select_windows,
    * sparda_prefetch_blocks, and the decode and prefill attention calls; the
    * cache plan and the cached prefetch follow the lists they are given;
-   * sparda_append_kv writes each sequence's new token at seq_len[b] - 1 (an
-   * invalid length appends nothing there).  A length
+   * sparda_append_kv and sparda_append_windows take each sequence's new
+   * token at seq_len[b] - 1 (an invalid length appends nothing there).  A length
    * outside [nq, T] (nq = 1 for decode and compression) gives that sequence
    * empty outputs (-1 sets, zero attention output) and is flagged
    * SPARDA_DEV_RANGE where a status word is given. */
@@ -200,6 +200,26 @@ int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf
 int sparda_compress_windows(const sparda_params *p, const void *K, long long bg_stride,
                             long long tok_stride, int win, int stride, float *kw_f32,
                             void *kw_bf16, sparda_stream_t stream);
+
+/*
+ * sparda_append_windows -- the window grid's part of a decode append: once
+ *   the new token's K row is in the cache (sparda_append_kv), write the key
+ *   of the window that token completes, if any (pos = w*stride + win - 1).
+ *   Windows that are not complete do not exist (as in
+ *   sparda_compress_windows), so no other window changes.
+ *   [p4 "The fourth projection", Algorithm 2] (update_incremental) on the
+ *   grid of [p4 "One Forecast head per GQA group"].
+ * pos, K, bg_stride, blk_stride  as for sparda_append_kv (with per-sequence
+ *          lengths, sequence b's token is at seq_len[b] - 1)
+ * win, stride  32 and 16 (others: SPARDA_EUNSUPPORTED)
+ * kw_f32, kw_bf16  [B][G][NW][d] as for sparda_compress_windows; with the
+ *          [B][G][T][d] layout the key is bit-identical to what that call
+ *          computes.
+ * Returns SPARDA_EINVAL for a bad pos (without lengths), pointer or stride.
+ */
+int sparda_append_windows(const sparda_params *p, int pos, const void *K, long long bg_stride,
+                          long long blk_stride, int win, int stride, float *kw_f32, void *kw_bf16,
+                          sparda_stream_t stream);
 
 /*
  * sparda_forecast_select_windows -- sparda_forecast_select on the window

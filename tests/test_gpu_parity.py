@@ -769,6 +769,77 @@ def test_append_matches_full_compression(interleaved):
     check_compressed(kc32.cpu().numpy(), host_bits(kc16), o64, o16)
 
 
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_append_windows_matches_full_compression(interleaved):
+    """The window grid's append: after each token, the window it completes
+    (if any) gets its key; at checkpoints the window keys equal a full window
+    compression of positions 0..pos (bit for bit in the [T][d] layout, within
+    the key tolerance against the oracle in the interleaved one)."""
+    rng = W.rng_for(53 + interleaved)
+    B, G, d, T0, T = 2, 2, 128, 40, 200
+    NB = (T + 63) // 64
+    NW = oracle.window_count(T)
+    p = abi.make_params(B, G, G, T, 1)
+    Kall = W.normal_bf16(rng, (B, G, T, d))
+    if interleaved:
+        cache = torch.zeros(B, G, NB, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+        for t in range(T0):
+            cache[:, :, t // 64, 0, t % 64] = dev_bf16(Kall[:, :, t])
+        Kd = cache
+        bg, blk = NB * 2 * 64 * d, 2 * 64 * d
+    else:
+        Kd = torch.zeros(B, G, T, d, dtype=torch.bfloat16, device="cuda")
+        Kd[:, :, :T0] = dev_bf16(Kall[:, :, :T0])
+        bg, blk = T * d, 64 * d
+    V = Kd.view(-1)[64 * d:] if interleaved else torch.zeros_like(Kd)
+    kw32 = torch.full((B, G, NW, d), 9.0, dtype=torch.float32, device="cuda")
+    kw16 = torch.zeros(B, G, NW, d, dtype=torch.bfloat16, device="cuda")
+    # the prefix's windows, from the host keys
+    o64, o16 = oracle.compress_windows(Kall[:, :, :T0])
+    nw0 = o64.shape[2]
+    kw32[:, :, :nw0] = torch.from_numpy(o64.astype(np.float32)).cuda()
+    kw16[:, :, :nw0] = dev_bf16(o16)
+    zero = torch.zeros(B, G, d, dtype=torch.bfloat16, device="cuda")
+    kc16 = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")  # the block keys (unchecked here)
+    for pos in range(T0, T):
+        abi.sparda_append_kv(p, pos, dev_bf16(Kall[:, :, pos]), zero, Kd, V, bg, blk, None, kc16)
+        abi.sparda_append_windows(p, pos, Kd, bg, blk, 32, 16, kw32, kw16)
+        if not interleaved and (pos % 16 == 15 or pos == T - 1):
+            torch.cuda.synchronize()
+            nw = oracle.window_count(pos + 1)
+            pf = abi.make_params(B, G, G, pos + 1, 1)
+            r32 = torch.zeros(B, G, max(nw, 1), d, dtype=torch.float32, device="cuda")
+            r16 = torch.zeros(B, G, max(nw, 1), d, dtype=torch.bfloat16, device="cuda")
+            abi.sparda_compress_windows(pf, Kd, bg, d, 32, 16, r32, r16)
+            torch.cuda.synchronize()
+            assert torch.equal(kw32[:, :, nw0:nw], r32[:, :, nw0:nw]), pos
+            assert torch.equal(kw16[:, :, nw0:nw], r16[:, :, nw0:nw]), pos
+            assert torch.all(kw32[:, :, nw:] == 9.0), pos  # windows not complete yet stay as they were
+    torch.cuda.synchronize()
+    o64, o16 = oracle.compress_windows(Kall)
+    check_compressed(kw32.cpu().numpy(), host_bits(kw16), o64, o16)
+
+
+def test_append_windows_per_sequence_positions():
+    rng = W.rng_for(55)
+    B, G, d, T = 3, 2, 128, 300
+    lens = [240, 127, 0]   # position 239 ends window 13; position 126 ends none
+    NW = oracle.window_count(T)
+    K = W.normal_bf16(rng, (B, G, T, d))
+    Kd = dev_bf16(K)
+    kw32 = torch.full((B, G, NW, d), 9.0, dtype=torch.float32, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G, G, T, 1, seq_len=sl)
+    abi.sparda_append_windows(p, 0, Kd, T * d, 64 * d, 32, 16, kw32, None)
+    torch.cuda.synchronize()
+    got = kw32.cpu().numpy()
+    w = (239 - 31) // 16
+    o64, _ = oracle.compress_windows(np.ascontiguousarray(K[0:1, :, :240]))
+    assert np.abs(got[0, :, w] - o64[0, :, w]).max() <= 1e-3
+    got[0, :, w] = 9.0
+    assert np.all(got == 9.0)  # nothing else was written
+
+
 def test_append_per_sequence_positions():
     """With per-sequence lengths each sequence appends its new token at its
     own last position (seq_len[b] - 1); the rows land there, and the block's
