@@ -272,15 +272,20 @@ class DecodeLoop:
                                            self.abi.SPARDA_ADDR_LOGICAL, self.O[l], self.ws_att,
                                            self.status)
 
-    def step_resident(self):
+    def step_resident(self, before_layer=None):
         """One decode token through the L layers.  select(l) -- layer l's
         Forecast vectors picking layer l+1's blocks -- and attention(l) both
         need layer l-1 finished and nothing from each other, so select(l)
         runs on a side stream beside attention(l); attention(l+1) waits for
         both (the order of Algorithm 2, which picks the next layer's blocks
-        before the current layer attends).  Launch on ``self.main``."""
+        before the current layer attends).  before_layer(l), when given, is
+        launched on the main stream ahead of layer l's two kernels (the decode
+        append of the token's K/V rows and keys).  Launch on ``self.main``."""
         torch = self.torch
         for l in range(self.w.layers):
+            if before_layer is not None:  # on the main stream, ahead of both kernels
+                with torch.cuda.stream(self.main):
+                    before_layer(l)
             self.ev_pre[l].record(self.main)
             self.side_sel.wait_event(self.ev_pre[l])
             with torch.cuda.stream(self.side_sel):
@@ -992,6 +997,21 @@ def run_real_model(steps):
     loop = DecodeLoop(w, with_host=False)
     L = w.layers
     n = max(5, min(steps, 50))
+    # the full decode order of a layer puts the append first: the new token's
+    # K/V rows and its block key (sparda_append_kv), and the window it
+    # completes (sparda_append_windows), each sequence at its own last position
+    d, blk = w.d, w.blk
+    k_new = [torch.randn(w.B, w.G, d, device="cuda").to(torch.bfloat16) for _ in range(L)]
+    v_new = [torch.randn(w.B, w.G, d, device="cuda").to(torch.bfloat16) for _ in range(L)]
+    kc_blocks = torch.empty(w.B, w.G, w.NB, d, dtype=torch.bfloat16, device="cuda")
+
+    def append(l):
+        kv = loop.kv[l]
+        loop.abi.sparda_append_kv(loop.p, w.T - 1, k_new[l], v_new[l], kv, kv.view(-1)[blk * d:],
+                                  w.NB * loop.blk_elems, loop.blk_elems, None, kc_blocks)
+        loop.abi.sparda_append_windows(loop.p, w.T - 1, kv, w.NB * loop.blk_elems, loop.blk_elems,
+                                       32, 16, None, loop.kw[l])
+
     with torch.cuda.stream(loop.main):
         for _ in range(3):
             loop.step_resident()
@@ -1000,6 +1020,11 @@ def run_real_model(steps):
         with torch.cuda.graph(graph, stream=loop.main):
             loop.step_resident()
         step_us = time_back_to_back(graph.replay, n)
+        g_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_full, stream=loop.main):
+            loop.step_resident(before_layer=append)
+        full_us = time_back_to_back(g_full.replay, n)
+        del g_full
         kern = {}
         for which in ("select", "attention"):
             fn = (lambda: [loop.select(l) for l in range(L)]) if which == "select" else \
@@ -1020,6 +1045,8 @@ def run_real_model(steps):
                    "n_local": w.n_local, "selection": "window grid, 32 tokens at stride 16",
                    "l2": "inputs larger than L2: %.0f MB of selected K/V per layer" % (b_att / 1e6)},
         "step_us": step_us, "step_GBps": step_gbs, "step_hbm_frac": step_gbs / peak,
+        "step_with_append_us": full_us,
+        "value_with_append": w.B / (full_us * 1e-6),
         "select_us_per_layer": kern["select"],
         "select_GBps": b_sel / (kern["select"] * 1e-6) / 1e9,
         "attn_us_per_layer": kern["attention"],

@@ -113,6 +113,10 @@ __global__ void __launch_bounds__(256) append_kernel(const uint16_t *__restrict_
                                                      const int32_t *seq_len, int G, int T) {
   const int lane = threadIdx.x & 31;
   const long long bg = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  // launched as a programmatic dependent: everything waits for the previous
+  // kernel (which may read the cache this writes)
+  pdl_trigger();
+  pdl_wait();
   if (bg >= n_pairs) return;
   if (seq_len) {  // per-sequence lengths: the new token is the sequence's last one
     const int len = seq_len[bg / G];
@@ -181,6 +185,8 @@ __global__ void __launch_bounds__(256) append_window_kernel(
   constexpr int kWin = 32, kStride = 16;
   const int lane = threadIdx.x & 31;
   const long long bg = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_trigger();
+  pdl_wait();  // the new row was written by the previous kernel (sparda_append_kv)
   if (bg >= n_pairs) return;
   if (seq_len) {
     const int len = seq_len[bg / G];
@@ -233,9 +239,11 @@ cudaError_t launch_append_windows(const sparda_params &p, int pos, const uint16_
   const long long pairs = (long long)p.B * p.G;
   if (pairs == 0) return cudaSuccess;
   const int warps = 8;
-  append_window_kernel<<<(unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream>>>(
-      K, bg_stride, blk_stride, pos, window_count(p.T), pairs, kw32, kw16, p.seq_len, p.G, p.T);
-  return cudaGetLastError();
+  const cudaError_t e =
+      launch_pdl(append_window_kernel, (unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream, K,
+                 bg_stride, blk_stride, pos, window_count(p.T), pairs, kw32, kw16, p.seq_len, p.G,
+                 p.T);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_compress(const sparda_params &p, const uint16_t *K, long long bg_stride,
@@ -269,9 +277,10 @@ cudaError_t launch_append(const sparda_params &p, int pos, const uint16_t *K_new
   if (pairs == 0) return cudaSuccess;
   const int NB = (p.T + kBlk - 1) / kBlk;
   const int warps = 8;
-  append_kernel<<<(unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream>>>(
-      K_new, V_new, K, V, bg_stride, blk_stride, pos, NB, pairs, kc32, kc16, p.seq_len, p.G, p.T);
-  return cudaGetLastError();
+  const cudaError_t e =
+      launch_pdl(append_kernel, (unsigned)ceil_div_ll(pairs, warps), warps * 32, 0, stream, K_new,
+                 V_new, K, V, bg_stride, blk_stride, pos, NB, pairs, kc32, kc16, p.seq_len, p.G, p.T);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sparda
