@@ -541,11 +541,19 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
   } else {
-    // streaming CTAs of 256 KB of key rows each (1024 blocks, or 256 blocks
-    // of four windows), but one chunk per problem once there are plenty of
-    // problems (prefill)
-    CH = 1024 / pool;
-    if (pl.n_problems >= 8LL * 148) CH = kMaxCand;
+    // as many chunks per problem as fill one wave of resident CTAs (two per
+    // SM), 256 to 1024 candidates each: the streams of one wave overlap
+    // best, and every later wave would restart them; one chunk per problem
+    // once there are plenty of problems (prefill)
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    (void)cudaGetLastError();
+    const long long wave = 2LL * n_sm;
+    const long long per = std::max<long long>(1, wave / std::max<long long>(1, pl.n_problems));
+    CH = (int)(ceil_div_ll(ceil_div_ll(pl.ncand_max, per), kSelThreads) * kSelThreads);
+    CH = std::min(std::max(CH, kSelThreads), 1024);  // longer streams per CTA stop paying
+    if (pl.n_problems >= 8LL * n_sm) CH = kMaxCand;
   }
   if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
   pl.CH = CH;
