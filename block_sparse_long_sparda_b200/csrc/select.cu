@@ -542,17 +542,25 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
   } else {
     // as many chunks per problem as fill one wave of resident CTAs (two per
-    // SM), 256 to 1024 candidates each: the streams of one wave overlap
+    // SM), at least 256 candidates each: the streams of one wave overlap
     // best, and every later wave would restart them; one chunk per problem
     // once there are plenty of problems (prefill)
+    static int sm_count[64] = {0};  // per device, queried once
     int dev = 0, n_sm = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+      if (sm_count[dev] == 0 &&
+          cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sm_count[dev] = 148;
+      n_sm = sm_count[dev];
+    }
     (void)cudaGetLastError();
     const long long wave = 2LL * n_sm;
     const long long per = std::max<long long>(1, wave / std::max<long long>(1, pl.n_problems));
     CH = (int)(ceil_div_ll(ceil_div_ll(pl.ncand_max, per), kSelThreads) * kSelThreads);
-    CH = std::min(std::max(CH, kSelThreads), 1024);  // longer streams per CTA stop paying
+    // longer streams per CTA stop paying; on the window grid (four rows per
+    // block) chunks stay at 256 blocks, which balanced sequences of mixed
+    // lengths better in the real models' decode step
+    CH = std::min(std::max(CH, kSelThreads), 1024 / pool);
     if (pl.n_problems >= 8LL * n_sm) CH = kMaxCand;
   }
   if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
