@@ -279,14 +279,16 @@ class DecodeLoop:
         runs on a side stream beside attention(l); attention(l+1) waits for
         both (the order of Algorithm 2, which picks the next layer's blocks
         before the current layer attends).  before_layer(l), when given, is
-        launched on the main stream ahead of layer l's two kernels (the decode
-        append of the token's K/V rows and keys).  Launch on ``self.main``."""
+        launched on the main stream ahead of attention(l): the decode append
+        of layer l's new K/V rows and keys.  select(l) does not wait for it,
+        since it reads layer l+1's keys, which that append does not touch.
+        Launch on ``self.main``."""
         torch = self.torch
         for l in range(self.w.layers):
-            if before_layer is not None:  # on the main stream, ahead of both kernels
+            self.ev_pre[l].record(self.main)
+            if before_layer is not None:  # on the main stream, ahead of attention(l)
                 with torch.cuda.stream(self.main):
                     before_layer(l)
-            self.ev_pre[l].record(self.main)
             self.side_sel.wait_event(self.ev_pre[l])
             with torch.cuda.stream(self.side_sel):
                 self.select(l)
