@@ -119,6 +119,56 @@ def test_real_model_decode_loop_full_size_sampled():
     torch.cuda.empty_cache()
 
 
+def test_decode_large_batch_multiwave_sampled():
+    """A decode batch large enough that the attention's list entries need
+    more CTAs than one wave holds (B = 128: 68,608 entries, at most 128 per
+    CTA) and the selection runs 1024 single-chunk problems: compression,
+    selection and attention on the device, sampled pairs against the oracle."""
+    B, G, R, T, d, k = 128, 8, 4, 8192, 128, 64
+    NB = T // 64
+    S = k + 3
+    dev = torch.device("cuda")
+    K = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+    V = torch.empty(B, G, T, d, dtype=torch.bfloat16, device=dev)
+    W.torch_normal_bf16_(K, 9001)
+    W.torch_normal_bf16_(V, 9002)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(9003)
+    Q = torch.randn(B, G * R, d, generator=gen, device=dev).to(torch.bfloat16)
+    F = torch.randn(B, G, d, generator=gen, device=dev).to(torch.bfloat16)
+    p = abi.make_params(B, G * R, G, T, k)
+    kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
+    abi.sparda_compress_keys(p, K, T * d, d, None, kc)
+    idx = torch.full((B, G, S), -7, dtype=torch.int32, device=dev)
+    abi.sparda_forecast_select(p, F, 1, 1, T - 1, kc, idx, abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1))
+    O = torch.empty(B, G * R, d, dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    abi.sparda_sparse_attn_decode(p, Q, K, V, T * d, 64 * d, idx, 0, O,
+                                  abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rng = np.random.default_rng(2027)
+    picks = {(0, 0), (B - 1, G - 1), (B // 2, 3)}
+    while len(picks) < 6:
+        picks.add((int(rng.integers(B)), int(rng.integers(G))))
+    for b, g in sorted(picks):
+        what = "B=128 b %d g %d" % (b, g)
+        Kb = host_bits(K[b, g]).reshape(1, 1, T, d)
+        _, ora_kc = oracle.compress_keys(Kb)
+        gpu_kc = host_bits(kc[b, g]).reshape(1, 1, NB, d)
+        _check_kc_bits(gpu_kc.reshape(NB, d), ora_kc.reshape(NB, d), what)
+        Fb = host_bits(F[b, g]).reshape(1, 1, 1, 1, d)
+        ora_idx, kth, kth1 = oracle.select(Fb, gpu_kc, k, 1, 2, T - 1)
+        gpu_idx = idx[b, g].cpu().numpy().reshape(1, 1, 1, -1)
+        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(Fb, gpu_kc), what)
+        Qb = host_bits(Q[b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
+        Vb = host_bits(V[b, g]).reshape(1, 1, T, d)
+        ora_o = oracle.sparse_attention(Qb, Kb, Vb, gpu_idx, T - 1, T)
+        check_attention(host_bits(O[b, g * R:(g + 1) * R]).reshape(1, 1, R, d), ora_o, what)
+    del K, V
+    torch.cuda.empty_cache()
+
+
 def test_prefill_chunk_full_size_sampled():
     import bench
     pc = bench.PrefillChunk()
