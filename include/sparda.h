@@ -170,7 +170,9 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
  * F     bf16 [B][nq][G][nf][d]   (nf = 1: Forecast; nf = Hq/G: baseline)
  * kc    bf16 [B][G][NB][d]       compressed keys of the layer being selected
  * idx   int32 [B][nq][G][S]      output, ascending block ids, -1 padded
- * Query token i sits at position q_start + i; 0 <= q_start, q_start + nq <= T.
+ * Query token i sits at position q_start + i; 0 <= q_start, q_start + nq <= T
+ * (with per-sequence lengths, at seq_len[b] - nq + i: q_start is checked but
+ * not used).
  * nq = 1 is the decode path; nq > 1 scores every query token (prefill).
  * Ranking: higher fp32 score first, equal scores -> lower block index.
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_SELECT, p, nq, nf)
@@ -285,7 +287,8 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
  * keys of its own block set (per token and group), causal, fp32 softmax.
  *   [p4 "The fourth projection", Algorithm 1 / Eq. 5]:
  *     O_l = attention(Q_l, K_l[B_l], V_l[B_l])   with all keys on the GPU
- * Q     bf16 [B][nq][Hq][d]; token i at position q_start + i <= T - 1
+ * Q     bf16 [B][nq][Hq][d]; token i at position q_start + i <= T - 1 (with
+ *       per-sequence lengths, at seq_len[b] - nq + i; q_start is then not used)
  * K, V  bf16, row (b,g,t) at base + (b*G+g)*bg_stride + t*tok_stride; this
  *       version needs tok_stride == d (else SPARDA_EUNSUPPORTED)
  * idx   int32 [B][nq][G][S] (as produced by sparda_forecast_select)
