@@ -998,6 +998,49 @@ def test_cached_prefetch_and_attention_over_steps(R):
         check_attention(host_bits(O).reshape(B, 1, G * R, d), ora, "cached step %d" % step)
 
 
+def test_cached_attention_with_lengths():
+    """The slot cache's attention (entries read from their slots) with
+    per-sequence lengths: each sequence against the oracle over its own
+    length, with its lists selected at its own last token."""
+    rng = np.random.default_rng(47)
+    B, G, R, NB, d, k, C = 2, 2, 4, 80, 128, 11, 20
+    T = NB * 64
+    lens = [T - 3, 2600 + 17]
+    S = k + 3
+    host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    F = W.normal_bf16(rng, (B, 1, G, 1, d))
+    idx = np.empty((B, G, S), np.int32)
+    for b, L in enumerate(lens):
+        o, _, _ = oracle.select(F[b:b + 1], np.ascontiguousarray(kc[b:b + 1, :, :(L + 63) // 64]),
+                                k, 1, 2, L - 1)
+        idx[b] = o[0, 0]
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * R, G, T, k, seq_len=sl)
+    cache = torch.zeros(B, G, C, 2, 64, d, dtype=torch.bfloat16, device="cuda")
+    block_of = torch.full((B, G, C), -1, dtype=torch.int32, device="cuda")
+    hand = torch.zeros(B, G, dtype=torch.int32, device="cuda")
+    phys = torch.empty(B, G, S, dtype=torch.int32, device="cuda")
+    fetch = torch.empty_like(phys)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    didx = torch.from_numpy(idx).cuda()
+    abi.sparda_cache_plan(p, C, didx, block_of, hand, phys, fetch, status)
+    abi.sparda_prefetch_cached(p, C, _pinned_bf16(host), didx, phys, fetch, cache, 0, status)
+    Q = W.normal_bf16(rng, (B, G * R, d))
+    O = torch.empty(B, G * R, d, dtype=torch.bfloat16, device="cuda")
+    abi.sparda_sparse_attn_decode_cached(p, C, dev_bf16(Q), cache, didx, phys, O,
+                                         abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p), status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = host_bits(O)
+    for b, L in enumerate(lens):
+        flat = np.ascontiguousarray(host[b:b + 1]).reshape(-1)
+        ora = oracle.sparse_attention(Q[b:b + 1].reshape(1, 1, G * R, d), flat, flat[64 * d:],
+                                      idx[b:b + 1].reshape(1, 1, G, S), L - 1, L, 64,
+                                      bg_stride=NB * 2 * 64 * d, blk_stride=2 * 64 * d, G=G)
+        check_attention(got[b:b + 1].reshape(1, 1, G * R, d), ora, "cached with lengths b=%d" % b)
+
+
 # --------------------------------------------------------------------------
 # prefill attention
 # --------------------------------------------------------------------------

@@ -52,6 +52,31 @@ def test_noalloc_decode_matches_workspace_entry_point_twice():
         check_attention(got, W.bf16_bits_to_f32(ref_bits).astype(np.float64), "noalloc vs workspace")
 
 
+def test_noalloc_decode_with_lengths_matches_workspace_entry_point():
+    """Per-sequence lengths take the same path through both entry points:
+    equal outputs, and blocks past a sequence's end flagged by both."""
+    build.build()
+    w, x, idx = _case()
+    sl = torch.tensor([w.T, w.T - 1000 + 7, 500, 0], dtype=torch.int32, device="cuda")
+    p = abi.make_params(w.B, w.Hq, w.G, w.T, w.k, w.n_init, w.n_local, seq_len=sl)
+    Q, K, V = dev_bf16(x["Q"]), dev_bf16(x["K"]), dev_bf16(x["V"])
+    didx = torch.from_numpy(np.ascontiguousarray(idx)).cuda()
+    bg, blk = w.T * w.d, 64 * w.d
+    ref = torch.empty(w.B, w.Hq, w.d, dtype=torch.bfloat16, device="cuda")
+    st_ref = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_sparse_attn_decode(p, Q, K, V, bg, blk, didx, abi.SPARDA_ADDR_LOGICAL, ref,
+                                  abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p), st_ref)
+    out = torch.full((w.B, w.Hq, w.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_sparse_attn_decode_noalloc(p, Q, K, V, bg, blk, didx, abi.SPARDA_ADDR_LOGICAL, out,
+                                          st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == int(st_ref.item()) and abi.sparda_status_from_device(int(st.item())) == abi.SPARDA_ERANGE
+    check_attention(host_bits(out), W.bf16_bits_to_f32(host_bits(ref)).astype(np.float64),
+                    "noalloc vs workspace, lengths")
+    assert torch.all(out[3] == 0)
+
+
 def test_noalloc_decode_refuses_shapes_beyond_its_scratch():
     build.build()
     # enough (query, group) pairs that the partial outputs outgrow the fixed array
