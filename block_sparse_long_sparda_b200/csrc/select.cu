@@ -51,6 +51,7 @@ struct SelArgs {
   uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
   int nq, G, nf, NB, k, n_init, n_local, q_start, S, T;
   int CH, n_chunks, cap;
+  int old_rank;  // 1: always the binned threshold search
 };
 
 // ---------------------------------------------------------------------------
@@ -183,6 +184,106 @@ __device__ void find_threshold(const uint32_t *keys, int n, int k, RankSmem &sm,
   // not reached: the key range is a single key after at most seven passes
   tau = 0xFFFFFFFFu;
   need = 0;
+}
+
+// The same threshold (tau, need) for k <= 64 and n <= 2048, with four block
+// barriers instead of a dozen: every warp sorts its 256 keys in registers
+// (a bitonic network, element q = 32*i + lane in register i, so partners
+// closer than 32 are a shuffle away and farther ones sit in the lane's own
+// registers), keeps its 64 largest, and three rounds of pairwise merges
+// reduce the 8 lists to the 64 largest keys of all.  tau is the k-th of
+// them and need counts how many keys equal to tau are kept; the
+// compaction then picks exactly the same entries as after find_threshold.
+// scratch: 1024 words of shared memory no one else is using.
+constexpr int kTopkMaxK = 64, kTopkMaxN = 8 * kSelThreads;
+
+__device__ __forceinline__ void cmp_swap_up(uint32_t &lo, uint32_t &hi, bool up) {
+  const uint32_t a = min(lo, hi), b = max(lo, hi);
+  lo = up ? a : b;
+  hi = up ? b : a;
+}
+
+// Sort m*32 keys held as v[i] (element 32*i + lane) ascending within runs of
+// `run` elements, the runs alternating direction as a bitonic network wants
+// (ascending where (q & run) == 0); run == m*32 gives one ascending run.
+template <int M>
+__device__ __forceinline__ void bitonic_warp(uint32_t (&v)[M], int lane, int k_from, int k_to) {
+#pragma unroll
+  for (int kk = k_from; kk <= k_to; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        const int r = j >> 5;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+          if (i & r) continue;
+          const int q = 32 * i + lane;
+          cmp_swap_up(v[i], v[i | r], (q & kk) == 0);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+          const int q = 32 * i + lane;
+          const uint32_t o = __shfl_xor_sync(0xffffffffu, v[i], j);
+          const bool up = (q & kk) == 0, lower = (lane & j) == 0;
+          v[i] = (up == lower) ? min(v[i], o) : max(v[i], o);
+        }
+      }
+    }
+  }
+}
+
+__device__ void find_threshold_topk(const uint32_t *keys, int n, int k, uint32_t *scratch,
+                                    RankSmem &sm, uint32_t &tau, int &need) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  {  // each warp: its 256 keys sorted ascending, the largest 64 to scratch
+    uint32_t v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = warp * 256 + 32 * i + lane;
+      v[i] = e < n ? keys[e] : 0u;  // 0 sorts below every finite score's key
+    }
+    bitonic_warp<8>(v, lane, 2, 256);
+    scratch[warp * 64 + lane] = v[6];
+    scratch[warp * 64 + 32 + lane] = v[7];
+  }
+  __syncthreads();
+  // merges: lists a and b (ascending) -> the 64 largest of both, ascending:
+  // c[x] = max(a[x], b[63 - x]) is bitonic and holds them, then one merge.
+  // Rounds read one half of the scratch and write the other.
+  uint32_t *src = scratch, *dst = scratch + 512;
+#pragma unroll 1
+  for (int lists = 8; lists > 1; lists >>= 1) {
+    if (warp < lists / 2) {
+      const uint32_t *a = src + (2 * warp) * 64, *b = src + (2 * warp + 1) * 64;
+      uint32_t c[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int x = 32 * i + lane;
+        c[i] = max(a[x], b[63 - x]);
+      }
+      bitonic_warp<2>(c, lane, 64, 64);
+      dst[warp * 64 + lane] = c[0];  // list `warp` of the next round
+      dst[warp * 64 + 32 + lane] = c[1];
+    }
+    __syncthreads();
+    uint32_t *t = src;
+    src = dst;
+    dst = t;
+  }
+  if (warp == 0) {
+    const uint32_t x0 = src[lane], x1 = src[32 + lane];  // ascending, x1 holds 32..63
+    const int pos = 64 - k;  // the k-th largest
+    const uint32_t t = src[pos];
+    const int gt = __popc(__ballot_sync(0xffffffffu, x0 > t)) + __popc(__ballot_sync(0xffffffffu, x1 > t));
+    if (lane == 0) {
+      sm.tau = t;
+      sm.need = (uint32_t)(k - gt);
+    }
+  }
+  __syncthreads();
+  tau = sm.tau;
+  need = (int)sm.need;
 }
 
 // Keep keys > tau plus the first `need` keys == tau (in entry order), in
@@ -479,7 +580,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   int32_t *top = out + bp.init_hi;
 
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
-    find_threshold(keys, n, a.k, rs, tau, need);
+    if (a.k <= kTopkMaxK && n <= kTopkMaxN && !a.old_rank)
+      find_threshold_topk(keys, n, a.k, reinterpret_cast<uint32_t *>(ring), rs, tau, need);
+    else
+      find_threshold(keys, n, a.k, rs, tau, need);
     const int ntop = compact_kept(keys, n, tau, need, a.k, rs,
                                   [&](int pos, int e) { st_list(top + pos, bp.cand_lo + e); });
     write_set(out, bp, ntop, a.S, false);
@@ -500,7 +604,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   __threadfence();
   for (int e = threadIdx.x; e < ncand; e += kSelThreads) keys[e] = __ldcg(pkeys + e);
   __syncthreads();
-  find_threshold(keys, ncand, a.k, rs, tau, need);
+  if (a.k <= kTopkMaxK && ncand <= kTopkMaxN && !a.old_rank)
+    find_threshold_topk(keys, ncand, a.k, reinterpret_cast<uint32_t *>(ring), rs, tau, need);
+  else
+    find_threshold(keys, ncand, a.k, rs, tau, need);
   const int ntop = compact_kept(keys, ncand, tau, need, a.k, rs,
                                 [&](int pos, int e) { st_list(top + pos, bp.cand_lo + e); });
   write_set(out, bp, ntop, a.S, false);
@@ -607,6 +714,7 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.cap = pl.n_chunks * pl.CH;  // key slots per problem in the workspace
   a.counters = nullptr;
   a.cand_key = nullptr;
+  a.old_rank = env_int("SPARDA_SELECT_BINNED") > 0 ? 1 : 0;
   size_t smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)pl.CH * 4;
   if (pl.n_chunks > 1) {
     char *w = static_cast<char *>(ws);

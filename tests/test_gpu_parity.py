@@ -143,10 +143,16 @@ def test_select_baseline_multihead():
     _select_case(Qg, x["kc"], 64, 1, 2, 2048 * 64 - 1, 2048 * 64, "baseline")
 
 
+@pytest.mark.parametrize("k", [100, 64, 17, 1])
+@pytest.mark.parametrize("binned", [False, True])
 @pytest.mark.parametrize("chunk", ["0", "256"])
-def test_select_exact_ties_lower_index_wins(chunk, monkeypatch):
+def test_select_exact_ties_lower_index_wins(chunk, binned, k, monkeypatch):
+    # k <= 64 over at most 2048 candidates takes the sorting-network threshold
+    # unless the binned search is forced; both must give the oracle's sets
     if chunk != "0":
         monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    if binned:
+        monkeypatch.setenv("SPARDA_SELECT_BINNED", "1")
     rng = np.random.default_rng(3)
     NB, B, G, d = 1500, 2, 4, 128
     kc = np.zeros((B, G, NB, d), np.float32)
@@ -154,8 +160,8 @@ def test_select_exact_ties_lower_index_wins(chunk, monkeypatch):
     F = np.zeros((B, 1, G, 1, d), np.float32)
     F[..., 0] = 1.0
     Fb, kcb = W.f32_to_bf16_bits(F), W.f32_to_bf16_bits(kc)
-    ora, _, _ = oracle.select(Fb, kcb, 100, 1, 2, NB * 64 - 1)
-    got = gpu_select(Fb, kcb, 100, 1, 2, NB * 64 - 1, NB * 64)
+    ora, _, _ = oracle.select(Fb, kcb, k, 1, 2, NB * 64 - 1)
+    got = gpu_select(Fb, kcb, k, 1, 2, NB * 64 - 1, NB * 64)
     assert np.array_equal(got, ora)
 
 
