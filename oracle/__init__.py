@@ -68,6 +68,9 @@ def _load():
         lib.oracle_compress_windows.restype = None
         lib.oracle_select_windows.argtypes = [I, I, I, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P]
         lib.oracle_select_windows.restype = None
+        lib.oracle_select_head_softmax.argtypes = [I, I, I, I, I, I, I, I, I, I, I, I, I, D,
+                                                   P, P, P, P, P, P]
+        lib.oracle_select_head_softmax.restype = None
         lib.oracle_cache_plan.argtypes = [I, I, I, I, I, P, P, P, P, P]
         lib.oracle_cache_plan.restype = I
         lib.oracle_gather_cached.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P]
@@ -187,6 +190,40 @@ def select(F: np.ndarray, kc: np.ndarray, k: int, n_init: int, n_local: int, q_s
     _load().oracle_select(B, nq, G, nf, d, blk, NB, k, n_init, n_local, q_start,
                           _ptr(F), _ptr(kc), _ptr(idx), _ptr(kth), _ptr(kth1))
     return idx, kth, kth1
+
+
+def select_head_softmax(Q: np.ndarray, kc: np.ndarray, T: int, k: int, n_init: int,
+                        n_local: int, q_start: int, tau: float, windows: bool = False,
+                        blk: int = 64, win: int = 32, stride: int = 16):
+    """The original selector's per-head softmax form ("Training: distilling
+    the selector you already have", Eq. 6): block weights
+    S = sum over the group's query heads of softmax(Q_h . Kc^T / tau) over the
+    key rows the query sees, max-pooled to blocks on the window grid; the
+    set is init U top-k(S) U local.
+
+    Q:  uint16 [B][G][nf][d] (the decode query's heads by group).
+    kc: uint16 [B][G][NB][d] block keys, or [B][G][NW][d] window keys.
+    Returns (idx [B][G][S], kth [B][G], kth1 [B][G], wblk [B][G][NB]).
+    """
+    Q = _u16(Q)
+    kc = _u16(kc)
+    B, G, nf, d = Q.shape
+    NR = kc.shape[2]
+    assert kc.shape == (B, G, NR, d)
+    NB = (T + blk - 1) // blk
+    if windows:
+        assert NR == window_count(T, win, stride)
+    else:
+        assert NR == NB
+    S = k + n_init + n_local
+    idx = np.empty((B, G, S), np.int32)
+    kth = np.empty((B, G), np.float64)
+    kth1 = np.empty((B, G), np.float64)
+    wblk = np.empty((B, G, NB), np.float64)
+    _load().oracle_select_head_softmax(B, G, nf, d, blk, win if windows else 0, stride, T, NR,
+                                       k, n_init, n_local, q_start, float(tau), _ptr(Q), _ptr(kc),
+                                       _ptr(idx), _ptr(kth), _ptr(kth1), _ptr(wblk))
+    return idx, kth, kth1, wblk
 
 
 def gather_blocks(host_kv: np.ndarray, idx: np.ndarray, pos: int, n_init: int, n_local: int,

@@ -395,6 +395,137 @@ void oracle_select_windows(int B, int nq, int G, int nf, int d, int blk, int win
 }
 
 /* ------------------------------------------------------------------------ */
+/* o2h: the original selector in its per-head softmax form (f3)             */
+/*   [p4] "Training: distilling the selector you already have", Eq. 6: the  */
+/*        original selector's shared importance score is, for each query    */
+/*        head of the group, a softmax over the compressed keys of its      */
+/*        scores divided by a temperature tau, summed over the group's      */
+/*        heads; it is taken before the selector's final max-pooling of     */
+/*        window scores to blocks.  Its top-k, minus the initial and local  */
+/*        blocks, is the selected set (the same section).                   */
+/*   [p4] "One Forecast head per GQA group": the baseline scores with every */
+/*        query head of the group, combines, then ranks.                    */
+/*                                                                          */
+/*   Readings taken here:                                                   */
+/*   - a head's softmax runs over every key row the query sees: on the      */
+/*     block grid blocks 0..c (c = the query's own block), on the window    */
+/*     grid the windows complete by the query position                      */
+/*     (w*stride + win <= pos + 1).  Initial and local rows count in the    */
+/*     normalisation but are not ranked (they are in the set anyway);      */
+/*   - on the window grid a block weighs as much as the heaviest window     */
+/*     inside it (the map of o2w), -inf when no window of it is complete;   */
+/*   - ranking: higher weight first, equal weights to the lower block id.   */
+/*                                                                          */
+/*   Q  [B][G][nf][d]  the decode query's heads, grouped (one query token)  */
+/*   kc [B][G][NR][d]  block keys (win = 0) or window keys                  */
+/*   idx [B][G][S]; kth / kth1 [B][G] as o2;                                */
+/*   wblk [B][G][NB] (optional): each block's weight (-inf past block c)    */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  int B, G, nf, d, blk, win, stride, NR, NB, k, n_init, n_local, q_start, S;
+  double tau;
+  const uint16_t *Q, *kc;
+  int32_t *idx;
+  double *kth, *kth1, *wblk;
+} hsm_ctx;
+
+static void hsm_item(void *vctx, long long item) {
+  hsm_ctx *c = (hsm_ctx *)vctx;
+  int g = (int)(item % c->G);
+  int b = (int)(item / c->G);
+  int pos = c->q_start;
+  block_parts bp = parts_for(pos, c->blk, c->n_init, c->n_local);
+  const uint16_t *q = c->Q + ((long long)b * c->G + g) * c->nf * c->d;
+  const uint16_t *kc = c->kc + ((long long)b * c->G + g) * (long long)c->NR * c->d;
+
+  /* the key rows the query sees */
+  int rows;
+  if (c->win == 0) {
+    rows = bp.c + 1;
+  } else {
+    rows = 0;
+    while (rows < c->NR && rows * c->stride + c->win <= pos + 1) ++rows;
+  }
+  if (rows > c->NR) rows = c->NR;
+
+  /* S[r] = sum_h softmax_r(q_h . kc_r / tau) */
+  double *sc = (double *)malloc(sizeof(double) * (rows > 0 ? rows : 1));
+  double *w = (double *)calloc(rows > 0 ? rows : 1, sizeof(double));
+  for (int h = 0; h < c->nf; ++h) {
+    double mx = -INFINITY;
+    for (int r = 0; r < rows; ++r) {
+      double dot = 0.0;
+      for (int x = 0; x < c->d; ++x)
+        dot += bf16_to_double(q[h * c->d + x]) * bf16_to_double(kc[(long long)r * c->d + x]);
+      sc[r] = dot / c->tau;
+      if (sc[r] > mx) mx = sc[r];
+    }
+    double z = 0.0;
+    for (int r = 0; r < rows; ++r) z += exp(sc[r] - mx);
+    for (int r = 0; r < rows; ++r) w[r] += exp(sc[r] - mx) / z;
+  }
+
+  /* block weights: the row itself, or the heaviest complete window inside */
+  double *wb = (double *)malloc(sizeof(double) * (size_t)(bp.c + 1));
+  for (int j = 0; j <= bp.c; ++j) {
+    double v;
+    if (c->win == 0) {
+      v = j < rows ? w[j] : -INFINITY;
+    } else {
+      v = -INFINITY;
+      for (int r = (j * c->blk + c->stride - 1) / c->stride;
+           r < rows && r * c->stride + c->win <= (j + 1) * c->blk; ++r)
+        if (w[r] > v) v = w[r];
+    }
+    wb[j] = v;
+  }
+  if (c->wblk) {
+    double *o = c->wblk + item * c->NB;
+    for (int j = 0; j < c->NB; ++j) o[j] = j <= bp.c ? wb[j] : -INFINITY;
+  }
+
+  int ncand = bp.cand_hi - bp.cand_lo;
+  scored *cand = (scored *)malloc(sizeof(scored) * (ncand > 0 ? ncand : 1));
+  for (int n = 0; n < ncand; ++n) {
+    cand[n].score = wb[bp.cand_lo + n];
+    cand[n].idx = bp.cand_lo + n;
+  }
+  qsort(cand, ncand, sizeof(scored), cmp_rank);
+  int ntop = ncand < c->k ? ncand : c->k;
+  if (c->kth) c->kth[item] = (c->k >= 1 && c->k <= ncand) ? cand[c->k - 1].score : -INFINITY;
+  if (c->kth1) c->kth1[item] = (c->k < ncand) ? cand[c->k].score : -INFINITY;
+
+  int *set = (int *)malloc(sizeof(int) * (size_t)(c->S + c->n_init + c->n_local + 1));
+  int m = 0;
+  for (int j = 0; j < bp.init_hi; ++j) set[m++] = j;
+  for (int n = 0; n < ntop; ++n) set[m++] = cand[n].idx;
+  for (int j = bp.local_lo; j <= bp.c; ++j) set[m++] = j;
+  qsort(set, m, sizeof(int), cmp_int);
+  int32_t *out = c->idx + item * c->S;
+  for (int s = 0; s < c->S; ++s) out[s] = s < m ? set[s] : -1;
+  free(set);
+  free(cand);
+  free(wb);
+  free(w);
+  free(sc);
+}
+
+/* win = 0: block keys, NR = NB blocks; win > 0: window keys, NR = windows of T
+ * tokens.  T sets NB; the query sits at q_start (decode: T - 1). */
+void oracle_select_head_softmax(int B, int G, int nf, int d, int blk, int win, int stride, int T,
+                                int NR, int k, int n_init, int n_local, int q_start, double tau,
+                                const uint16_t *Q, const uint16_t *kc, int32_t *idx, double *kth,
+                                double *kth1, double *wblk) {
+  hsm_ctx c;
+  c.B = B; c.G = G; c.nf = nf; c.d = d; c.blk = blk; c.win = win; c.stride = stride;
+  c.NR = NR; c.NB = (T + blk - 1) / blk; c.k = k; c.n_init = n_init; c.n_local = n_local;
+  c.q_start = q_start; c.S = k + n_init + n_local; c.tau = tau;
+  c.Q = Q; c.kc = kc; c.idx = idx; c.kth = kth; c.kth1 = kth1; c.wblk = wblk;
+  parallel_for((long long)B * G, hsm_item, &c);
+}
+
+/* ------------------------------------------------------------------------ */
 /* o3: gather of selected blocks from the host copy into device slots       */
 /*   [p4] "The fourth projection", Algorithm 2: fetch(B_next, src = CPU     */
 /*   pinned, dst = GPU).  The result is a byte copy: slot s of (b,g) holds  */

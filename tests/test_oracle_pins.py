@@ -581,3 +581,155 @@ def test_select_windows_equals_block_selection_when_windows_agree():
     a = oracle.select_windows(F, kw, T, k=7, n_init=1, n_local=2, q_start=T - nq)
     b = oracle.select(F, kc, 7, 1, 2, T - nq)
     assert np.array_equal(a[0], b[0])
+
+
+# --------------------------------------------------------------------------
+# the original selector's per-head softmax form ("Training: distilling the
+# selector you already have", Eq. 6): S = sum_h softmax(Q_h . Kc^T / tau)
+# --------------------------------------------------------------------------
+
+def _two_head_keys(a, b, d=8):
+    """Rows r = a[r] e_0 + b[r] e_1; head A queries e_0, head B e_1, so head
+    A scores a and head B scores b."""
+    R = len(a)
+    kc = np.zeros((1, 1, R, d), np.float32)
+    kc[0, 0, :, 0] = a
+    kc[0, 0, :, 1] = b
+    Q = np.zeros((1, 1, 2, d), np.float32)
+    Q[0, 0, 0, 0] = 1.0
+    Q[0, 0, 1, 1] = 1.0
+    return bits(Q), bits(kc)
+
+
+def test_head_softmax_closed_form_differs_from_summed_scores():
+    """Blocks 0..4, init {0}, local {4}, candidates {1, 2, 3}, k = 1, tau = 1.
+    Head A scores (0, 10, 9.875, 0, 0): blocks 1 and 2 split its mass.
+    Head B scores (0, 0, 0, 3, 0): block 3 keeps most of it.  Each softmax
+    runs over all five rows the query sees (the initial and local rows
+    included), so Z_A = e^10 + e^9.875 + 3 and Z_B = e^3 + 4, and
+      w1 = e^10/Z_A + 1/Z_B = 0.5727,  w2 = e^9.875/Z_A + 1/Z_B = 0.5103,
+      w3 = 1/Z_A + e^3/Z_B = 0.8339:
+    the per-head softmax keeps block 3, where summed scores (10, 9.875, 3)
+    keep block 1."""
+    Q, kc = _two_head_keys([0, 10, 9.875, 0, 0], [0, 0, 0, 3, 0])
+    T = 64 * 5
+    idx, kth, kth1, wb = oracle.select_head_softmax(Q, kc, T, k=1, n_init=1, n_local=1,
+                                                    q_start=T - 1, tau=1.0)
+    assert idx.reshape(-1).tolist() == [0, 3, 4]
+    ZA = "(exp(10) + exp(9.875) + 3)"
+    ZB = "(exp(3) + 4)"
+    want = [closed_form("1/%s + 1/%s" % (ZA, ZB)),
+            closed_form("exp(10)/%s + 1/%s" % (ZA, ZB)),
+            closed_form("exp(9.875)/%s + 1/%s" % (ZA, ZB)),
+            closed_form("1/%s + exp(3)/%s" % (ZA, ZB)),
+            closed_form("1/%s + 1/%s" % (ZA, ZB))]
+    np.testing.assert_allclose(wb[0, 0], want, rtol=1e-12)
+    assert abs(want[3] - 0.8339) < 1e-4 and abs(want[1] - 0.5727) < 1e-4
+    assert kth[0, 0] == wb[0, 0, 3] and kth1[0, 0] == wb[0, 0, 1]
+    # summed raw scores rank block 1 first
+    F = Q.reshape(1, 1, 1, 2, 8)
+    ref, _, _ = oracle.select(F, kc, 1, 1, 1, T - 1)
+    assert ref.reshape(-1).tolist() == [0, 1, 4]
+
+
+def test_head_softmax_mass_is_one_per_head():
+    """On the block grid every seen row is a block: the weights of blocks
+    0..c sum to the number of heads, and blocks past c weigh -inf."""
+    rng = np.random.default_rng(21)
+    B, G, nf, d, NB = 2, 3, 4, 32, 30
+    T = NB * 64
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    Q = W.normal_bf16(rng, (B, G, nf, d))
+    q = T - 64 * 5 - 7                       # block c = NB - 6
+    _, _, _, wb = oracle.select_head_softmax(Q, kc, T, 4, 1, 2, q, tau=math.sqrt(d))
+    c = q // 64
+    np.testing.assert_allclose(wb[..., :c + 1].sum(-1), nf, rtol=1e-12)
+    assert np.all(wb[..., c + 1:] == -np.inf)
+    assert np.all(wb[..., :c + 1] > 0) and np.all(wb[..., :c + 1] < nf)
+
+
+def test_head_softmax_shift_and_temperature_invariance():
+    """A component u shared by every key row shifts head h's scores by
+    Q_h . u, a different constant per head, which no softmax sees; scaling the
+    queries and tau by 2 together changes nothing either.  Integer entries keep
+    every product exact in fp64, so the weights agree to the last bit."""
+    rng = np.random.default_rng(22)
+    B, G, nf, d, NB = 2, 2, 4, 16, 40
+    T = NB * 64
+    kc = rng.integers(-3, 4, (B, G, NB, d)).astype(np.float32)
+    Q = rng.integers(-3, 4, (B, G, nf, d)).astype(np.float32)
+    u = rng.integers(-4, 5, (B, G, 1, d)).astype(np.float32)
+    base = oracle.select_head_softmax(bits(Q), bits(kc), T, 6, 1, 2, T - 1, tau=4.0)
+    shifted = oracle.select_head_softmax(bits(Q), bits(kc + u), T, 6, 1, 2, T - 1, tau=4.0)
+    scaled = oracle.select_head_softmax(bits(2 * Q), bits(kc), T, 6, 1, 2, T - 1, tau=8.0)
+    for other in (shifted, scaled):
+        assert np.array_equal(base[0], other[0])
+        np.testing.assert_allclose(base[3], other[3], rtol=1e-13)
+    # tau divides: with tau -> tau / 2 the weights do change
+    sharper = oracle.select_head_softmax(bits(Q), bits(kc), T, 6, 1, 2, T - 1, tau=2.0)
+    assert not np.allclose(base[3], sharper[3])
+
+
+def test_head_softmax_head_order_does_not_matter():
+    rng = np.random.default_rng(23)
+    B, G, nf, d, NB = 1, 2, 4, 32, 50
+    T = NB * 64
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    Q = W.normal_bf16(rng, (B, G, nf, d))
+    a = oracle.select_head_softmax(Q, kc, T, 8, 1, 2, T - 1, tau=math.sqrt(d))
+    b = oracle.select_head_softmax(np.ascontiguousarray(Q[:, :, ::-1]), kc, T, 8, 1, 2, T - 1,
+                                   tau=math.sqrt(d))
+    assert np.array_equal(a[0], b[0])
+    np.testing.assert_allclose(a[3], b[3], rtol=1e-12)
+
+
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_one_head_ranks_as_raw_scores(windows):
+    """With one head the weight is an increasing function of the (pooled)
+    score, so the set is the raw-score selector's."""
+    rng = np.random.default_rng(24)
+    B, G, d, NB = 2, 3, 64, 45
+    T = NB * 64 - 9
+    NR = oracle.window_count(T) if windows else NB
+    kc = W.normal_bf16(rng, (B, G, NR, d))
+    Q = W.normal_bf16(rng, (B, G, 1, d))
+    got = oracle.select_head_softmax(Q, kc, T, 9, 1, 3, T - 1, tau=8.0, windows=windows)[0]
+    F = Q.reshape(B, 1, G, 1, d)
+    if windows:
+        ref = oracle.select_windows(F, kc, T, 9, 1, 3, T - 1)[0]
+    else:
+        ref = oracle.select(F, kc, 9, 1, 3, T - 1)[0]
+    assert np.array_equal(got, ref.reshape(B, G, -1))
+
+
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_normalises_over_rows_outside_the_candidates(windows):
+    """Head A puts a score of 60 on a row that is not a candidate -- the
+    initial block (block grid) or a window straddling two blocks (window
+    grid, in the normalisation but inside no block) -- so its softmax leaves
+    every candidate below e^-50 and head B alone decides: the set is head B's
+    raw-score top-k.  Head A's scores on the candidates run opposite to head
+    B's, so a softmax over the candidates only would pick other blocks."""
+    NB, d = 24, 8
+    T = NB * 64
+    NR = oracle.window_count(T) if windows else NB
+    perm = np.random.default_rng(25).permutation(NR).astype(np.float32)
+    b = perm / 4.0                          # distinct, bf16-exact
+    a = 10.0 - b / 2.0                      # opposite order
+    if windows:
+        a[4 * 0 + 3] = 60.0                 # window 3 straddles blocks 0 and 1
+    else:
+        a[0] = 60.0                         # the initial block
+    Q, kc = _two_head_keys(a.tolist(), b.tolist(), d)
+    k = 5
+    got = oracle.select_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau=1.0, windows=windows)[0]
+    Fb = Q[:, :, 1:2].reshape(1, 1, 1, 1, d)
+    if windows:
+        ref = oracle.select_windows(Fb, kc, T, k, 1, 2, T - 1)[0]
+    else:
+        ref = oracle.select(Fb, kc, k, 1, 2, T - 1)[0]
+    assert np.array_equal(got.reshape(-1), ref.reshape(-1))
+    Fa = Q[:, :, 0:1].reshape(1, 1, 1, 1, d)
+    other = (oracle.select_windows(Fa, kc, T, k, 1, 2, T - 1) if windows
+             else oracle.select(Fa, kc, k, 1, 2, T - 1))[0]
+    assert not np.array_equal(got.reshape(-1), other.reshape(-1))
