@@ -70,12 +70,20 @@ def parse_args():
                     help="also measure the real models' decode configuration: 96-block sets "
                          "(1 initial, 32 local, 63 top-k) on the window grid, 16 sequences of "
                          "mixed lengths (64K..128K), 4 layers; prints an extra JSON line")
+    ap.add_argument("--head-softmax", action="store_true",
+                    help="also measure the original selector in its per-head softmax form "
+                         "(each of a group's 4 query heads softmax-normalised over the seen "
+                         "keys, summed) at B=16, T=128K on block keys and on window keys, "
+                         "beside Forecast and the summed-score baseline on the same keys; "
+                         "prints an extra JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
                          "K/V per attention launch), then two passes of a 512-token prefill "
                          "chunk of one sequence, then two cold host gathers of one layer at B=2 "
-                         "(1.1 GB pinned), and exit: the small cases ncu captures")
+                         "(1.1 GB pinned), then two head-softmax selections each on one "
+                         "layer of block keys and of window keys at B=16, T=128K, and exit: "
+                         "the small cases ncu captures")
     return ap.parse_args()
 
 
@@ -764,6 +772,8 @@ def run_sparda(args):
         print(json.dumps(run_windows(args.steps)), flush=True)
     if rank == 0 and world == 1 and args.real_model:
         print(json.dumps(run_real_model(args.steps)), flush=True)
+    if rank == 0 and world == 1 and args.head_softmax:
+        print(json.dumps(run_head_softmax(args.steps)), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -1097,6 +1107,98 @@ def run_sweep():
             "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16"}
 
 
+class HeadSoftmaxCase:
+    """The original selector in its per-head softmax form at the decode
+    loop's shapes (B=16, G=8 groups of 4 query heads, T=131072, k=64 with 1
+    initial and 2 local blocks), on block keys or on the window grid.  Three
+    layers' keys are alternated, so a call never finds its keys in L2
+    (201 MB of block keys, 805 MB of window keys)."""
+
+    def __init__(self, windows: bool, n_layers: int = 3, w: W.Workload = None):
+        import math
+        import torch
+        from block_sparse_long_sparda_b200 import abi
+        self.abi = abi
+        w = w or WORKLOAD
+        self.w, self.windows, self.L = w, windows, n_layers
+        dev = torch.device("cuda")
+        self.nf = w.Hq // w.G
+        self.NR = (w.T - 32) // 16 + 1 if windows else w.NB
+        self.p = abi.make_params(w.B, w.Hq, w.G, w.T, w.k, w.n_init, w.n_local)
+        self.kc = []
+        for l in range(n_layers):
+            kc = torch.empty(w.B, w.G, self.NR, w.d, dtype=torch.bfloat16, device=dev)
+            W.torch_normal_bf16_(kc, 5000 + 10 * l + int(windows))
+            self.kc.append(kc)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(5100 + int(windows))
+        self.Q = torch.randn(w.B, w.G, self.nf, w.d, generator=gen, device=dev).to(torch.bfloat16)
+        self.F = torch.randn(w.B, w.G, 1, w.d, generator=gen, device=dev).to(torch.bfloat16)
+        self.tau = math.sqrt(w.d)
+        self.idx = torch.empty(w.B, w.G, w.S, dtype=torch.int32, device=dev)
+        op_h = abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS if windows else abi.SPARDA_OP_HEAD_SOFTMAX
+        op_s = abi.SPARDA_OP_SELECT_WINDOWS if windows else abi.SPARDA_OP_SELECT
+        self.ws_h = abi.workspace(op_h, self.p, 1, self.nf)
+        self.ws_f = abi.workspace(op_s, self.p, 1, 1)
+        self.ws_s = abi.workspace(op_s, self.p, 1, self.nf)
+        self.t = 0
+
+    def _next(self):
+        l = self.t % self.L
+        self.t += 1
+        return self.kc[l]
+
+    def head_softmax(self, kc=None):
+        kc = self._next() if kc is None else kc
+        w, a = self.w, self.abi
+        if self.windows:
+            a.sparda_head_softmax_select_windows(self.p, self.Q, self.nf, w.T - 1, self.tau, kc,
+                                                 32, 16, self.idx, self.ws_h)
+        else:
+            a.sparda_head_softmax_select(self.p, self.Q, self.nf, w.T - 1, self.tau, kc,
+                                         self.idx, self.ws_h)
+
+    def scores(self, vecs, nf, ws):
+        kc = self._next()
+        w, a = self.w, self.abi
+        if self.windows:
+            a.sparda_forecast_select_windows(self.p, vecs, 1, nf, w.T - 1, kc, 32, 16, self.idx, ws)
+        else:
+            a.sparda_forecast_select(self.p, vecs, 1, nf, w.T - 1, kc, self.idx, ws)
+
+    def key_bytes(self):
+        """Keys of every row a decode query at T-1 sees (the softmax reads
+        them all)."""
+        return self.w.B * self.w.G * self.NR * self.w.d * 2
+
+
+def run_head_softmax(steps):
+    """The original selector's per-head softmax form next to Forecast and the
+    summed-score baseline, on the same keys."""
+    import torch
+    n = max(6, min(steps, 30))
+    peak, peak_kind = measured_peaks()
+    out = {"metric": "decode selection, the original selector's per-head softmax form vs "
+                     "Forecast (us per call, one layer)",
+           "data": "synthetic", "dtype": "bf16", "peak": peak, "peak_kind": peak_kind}
+    for windows in (False, True):
+        c = HeadSoftmaxCase(windows)
+        h_us = time_back_to_back(c.head_softmax, n)
+        f_us = time_back_to_back(lambda: c.scores(c.F, 1, c.ws_f), n)
+        s_us = time_back_to_back(lambda: c.scores(c.Q, c.nf, c.ws_s), n)
+        nb = c.key_bytes()
+        key = "windows" if windows else "blocks"
+        out[key] = {"B": c.w.B, "T": c.w.T, "G": c.w.G, "heads_per_group": c.nf, "k": c.w.k,
+                    "key_rows": c.NR, "key_bytes": nb,
+                    "head_softmax_us": h_us, "head_softmax_GBps": nb / (h_us * 1e-6) / 1e9,
+                    "head_softmax_hbm_frac": nb / (h_us * 1e-6) / 1e9 / peak,
+                    "forecast_us": f_us, "summed_heads_us": s_us,
+                    "l2": "3 layers' keys alternated (%.0f MB)" % (3 * nb / 1e6)}
+        del c
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_profile_case():
     """One decode layer at B=8, three passes: the small case for ncu."""
     import torch
@@ -1138,6 +1240,19 @@ def run_profile_case():
     st3 = int(gl.status.item())
     gl.unregister()
     print("profile case: host gather B=2, device status %d" % st3)
+    del gl
+    torch.cuda.empty_cache()
+    # the original selector's per-head softmax form at B=16, T=128K: two
+    # launches on one layer of block keys (67 MB), then two on window keys
+    # (268 MB)
+    for windows in (False, True):
+        hc = HeadSoftmaxCase(windows, n_layers=1)
+        for _ in range(2):
+            hc.head_softmax(hc.kc[0])
+        torch.cuda.synchronize()
+        del hc
+        torch.cuda.empty_cache()
+    print("profile case: head-softmax selection on block and window keys")
     if st != 0 or st2 != 0 or st3 != 0:
         sys.exit(1)
 

@@ -35,6 +35,8 @@ SPARDA_OP_PREFETCH = 2
 SPARDA_OP_ATTN_DECODE = 3
 SPARDA_OP_ATTN_PREFILL = 4
 SPARDA_OP_SELECT_WINDOWS = 5
+SPARDA_OP_HEAD_SOFTMAX = 6
+SPARDA_OP_HEAD_SOFTMAX_WINDOWS = 7
 
 SPARDA_ADDR_LOGICAL = 0
 SPARDA_ADDR_SLOT = 1
@@ -77,6 +79,9 @@ _SIGS = {
     "sparda_append_windows": (_I, [_PP, _I, _P, _LL, _LL, _I, _I, _P, _P, _P]),
     "sparda_compress_windows": (_I, [_PP, _P, _LL, _LL, _I, _I, _P, _P, _P]),
     "sparda_forecast_select_windows": (_I, [_PP, _P, _I, _I, _I, _P, _I, _I, _P, _P, _SZ, _P]),
+    "sparda_head_softmax_select": (_I, [_PP, _P, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "sparda_head_softmax_select_windows": (_I, [_PP, _P, _I, _I, ctypes.c_float, _P, _I, _I, _P,
+                                                _P, _SZ, _P]),
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
@@ -182,6 +187,22 @@ def sparda_forecast_select(p, F, nq, nf, q_start, kc, idx, ws, stream=None):
            lib().sparda_forecast_select(ctypes.byref(p), _ptr(F), int(nq), int(nf), int(q_start),
                                         _ptr(kc), _ptr(idx), _ptr(ws), _nbytes(ws),
                                         _stream(stream)))
+
+
+def sparda_head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, stream=None):
+    _check("sparda_head_softmax_select",
+           lib().sparda_head_softmax_select(ctypes.byref(p), _ptr(Q), int(nf), int(q_start),
+                                            float(tau), _ptr(kc), _ptr(idx), _ptr(ws), _nbytes(ws),
+                                            _stream(stream)))
+
+
+def sparda_head_softmax_select_windows(p, Q, nf, q_start, tau, kw, win, stride, idx, ws,
+                                       stream=None):
+    _check("sparda_head_softmax_select_windows",
+           lib().sparda_head_softmax_select_windows(ctypes.byref(p), _ptr(Q), int(nf),
+                                                    int(q_start), float(tau), _ptr(kw), int(win),
+                                                    int(stride), _ptr(idx), _ptr(ws), _nbytes(ws),
+                                                    _stream(stream)))
 
 
 def sparda_prefetch_blocks(p, host_kv, idx, slots, skip_resident, n_ctas=0, dev_status=None,

@@ -39,6 +39,27 @@ bool stride_ok(long long s) { return s > 0 && (s % 8) == 0; }
 
 }  // namespace
 
+// shared by the block-grid and window-grid entry points
+namespace {
+int head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start, float tau,
+                        const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
+                        sparda_stream_t stream, int pool) {
+  if (nf < 1 || q_start < 0 || q_start >= p->T) return SPARDA_EINVAL;
+  if (!(tau == tau) || tau > 3.0e38f) return SPARDA_EINVAL;  // NaN or infinite
+  if (nf > 16) return SPARDA_EUNSUPPORTED;
+  if (p->B == 0) return SPARDA_OK;
+  if (!Q || !kc || !idx) return SPARDA_EINVAL;
+  if (!aligned16(Q) || !aligned16(kc) || !aligned16(idx)) return SPARDA_EINVAL;
+  const HsmPlan pl = plan_head_softmax(*p, nf, pool);
+  if (!head_softmax_supported(pl, nf)) return SPARDA_EUNSUPPORTED;
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  const float t = tau > 0.f ? tau : sqrtf((float)p->d);
+  return from_cuda(launch_head_softmax(*p, pl, static_cast<const uint16_t *>(Q), nf, q_start, t,
+                                       static_cast<const uint16_t *>(kc), idx, ws,
+                                       reinterpret_cast<cudaStream_t>(stream), pool));
+}
+}  // namespace
+
 extern "C" {
 
 int sparda_version(void) { return 100; }
@@ -70,6 +91,10 @@ size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf) {
       return nq < 1 ? 0 : plan_select(*p, nq, nf < 1 ? 1 : nf).ws_bytes;
     case SPARDA_OP_SELECT_WINDOWS:
       return nq < 1 ? 0 : plan_select(*p, nq, nf < 1 ? 1 : nf, 4).ws_bytes;
+    case SPARDA_OP_HEAD_SOFTMAX:
+      return nq != 1 || nf < 1 ? 0 : plan_head_softmax(*p, nf, 1).ws_bytes;
+    case SPARDA_OP_HEAD_SOFTMAX_WINDOWS:
+      return nq != 1 || nf < 1 ? 0 : plan_head_softmax(*p, nf, 4).ws_bytes;
     case SPARDA_OP_ATTN_DECODE:
       return plan_decode(*p).ws_bytes;
     case SPARDA_OP_ATTN_PREFILL:
@@ -169,6 +194,24 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
   return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), nq, nf, q_start,
                                  static_cast<const uint16_t *>(kw), idx, ws,
                                  reinterpret_cast<cudaStream_t>(stream), 4));
+}
+
+int sparda_head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start,
+                               float tau, const void *kc, int32_t *idx, void *ws,
+                               size_t ws_bytes, sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  return head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, ws_bytes, stream, 1);
+}
+
+int sparda_head_softmax_select_windows(const sparda_params *p, const void *Q, int nf,
+                                       int q_start, float tau, const void *kw, int win,
+                                       int stride, int32_t *idx, void *ws, size_t ws_bytes,
+                                       sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
+  return head_softmax_select(p, Q, nf, q_start, tau, kw, idx, ws, ws_bytes, stream, 4);
 }
 
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,

@@ -93,6 +93,22 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const 
                           int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,
                           void *ws, cudaStream_t stream, int pool = 1);
 
+// the original selector's per-head softmax form (decode: one query token);
+// pool as plan_select
+struct HsmPlan {
+  long long n_problems;  // B * G
+  int ncand_max;         // candidates of a query at the end of the sequence
+  int CH;                // seen blocks per thread block
+  int n_chunks;          // thread blocks per problem
+  int rows_cap;          // head-score slots per (problem, head) in the workspace
+  size_t ws_bytes;
+};
+HsmPlan plan_head_softmax(const sparda_params &p, int nf, int pool);
+int head_softmax_supported(const HsmPlan &plan, int nf);
+cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &plan, const uint16_t *Q,
+                                int nf, int q_start, float tau, const uint16_t *kc, int32_t *idx,
+                                void *ws, cudaStream_t stream, int pool);
+
 // ---- prefetch -------------------------------------------------------------
 cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
                             const int32_t *idx, uint16_t *slots, int skip_resident, int n_ctas,

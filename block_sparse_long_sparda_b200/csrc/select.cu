@@ -614,6 +614,309 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   if (threadIdx.x == 0) a.counters[prob] = 0u;
 }
 
+// ---------------------------------------------------------------------------
+// the original selector in its per-head softmax form: for every query head h
+// of the group, a softmax over all key rows the query sees of q_h . k_r / tau,
+// summed over the heads; on the window grid a block weighs as much as its
+// heaviest window.  ["SparDA: a fourth projection..." article, "Training:
+// distilling the selector you already have", Eq. 6; "One Forecast head per
+// GQA group": the baseline scores with every query head.]
+//
+// The softmax needs each head's max and normaliser over every seen row --
+// the initial and local rows and the straddling windows too, which are never
+// ranked -- so the chunks of a problem cover all seen rows, not only the
+// candidates.  A chunk streams its rows once, writes each head's scores to
+// the workspace and keeps a running (max, sum of exp(s - max)) per head; the
+// last chunk to finish merges those into (M_h, Z_h), turns the candidates'
+// scores into weights sum_h exp(s_h - M_h) / Z_h, and ranks them exactly as
+// select_kernel ranks raw scores (same threshold search and compaction, so
+// the same tie rule).
+// ---------------------------------------------------------------------------
+constexpr int kHsmMaxHeads = 16;
+
+struct HsmArgs {
+  const int32_t *seq_len;
+  const uint16_t *Q;   // [B][G][nf][d]
+  const uint16_t *kc;  // [B][G][NR][d]
+  int32_t *idx;        // [B][G][S]
+  uint32_t *counters;  // [problem] tickets
+  uint32_t *failed;    // [problem] set when a chunk's copy never landed
+  float2 *stats;       // [problem][n_chunks][nf] (max, sum of exp(s - max))
+  float *scores;       // [problem][nf][rows_cap] q_h . k_r / tau
+  int G, nf, NR, k, n_init, n_local, q_start, S, T;
+  int CH, n_chunks, rows_cap;  // CH blocks per chunk
+  float inv_tau;
+  int old_rank;
+};
+
+// Score rows [lo, lo + n) with every head: scores to sc (head-major, row
+// stride rows_cap), and per head a running (max, sum of exp(s - max)) over
+// the rows this thread saw.  Streams like score_rows.  NFT (a power of two
+// >= nf) fixes the unrolling; heads are taken four at a time, and each row
+// is converted from bf16 once per group of four heads.
+template <int NFT>
+__device__ bool score_rows_heads(const uint16_t *kc_bg, const float *qs, int nf, float inv_tau,
+                                 int lo, int n, float *sc, int rows_cap, float (&m_run)[NFT],
+                                 float (&z_run)[NFT], uint8_t *ring, uint64_t *bars) {
+  constexpr int HG = NFT < 4 ? NFT : 4;
+  const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
+  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
+  bool ok = true;
+#pragma unroll 1
+  for (int pc = 0; pc < n_pc; ++pc) {
+    const bool landed = mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1));
+    if (__syncthreads_or(!landed)) {
+      ok = false;
+      if (threadIdx.x == 0)
+        for (int q = pc; q < min(n_pc, pc + kRing); ++q)
+          (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
+      __syncthreads();
+      break;
+    }
+    const int rows = min(kPieceRows, n - pc * kPieceRows);
+    const uint8_t *piece = ring + (pc % kRing) * kPieceBytes;
+    const int row0 = hw * 8;
+    const int r = row0 + (hl >> 1);
+    const bool mine = (hl & 1) == 0 && r < rows;
+    const long long grow = (long long)lo + pc * kPieceRows + r;
+#pragma unroll
+    for (int f0 = 0; f0 < NFT; f0 += HG) {
+      if (f0 < nf) {  // uniform over the block
+        float fv[HG][8];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+          if (f0 + h < nf) {
+            a = *reinterpret_cast<const float4 *>(qs + (f0 + h) * kD + hl * 8);
+            b = *reinterpret_cast<const float4 *>(qs + (f0 + h) * kD + hl * 8 + 4);
+          }
+          fv[h][0] = a.x; fv[h][1] = a.y; fv[h][2] = a.z; fv[h][3] = a.w;
+          fv[h][4] = b.x; fv[h][5] = b.y; fv[h][6] = b.z; fv[h][7] = b.w;
+        }
+        float part[HG][8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = row0 + u < rows
+                              ? *reinterpret_cast<const uint4 *>(piece + (row0 + u) * (kD * 2) + hl * 16)
+                              : make_uint4(0, 0, 0, 0);
+          const float c[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                              bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            float t = fv[h][0] * c[0];
+#pragma unroll
+            for (int x = 1; x < 8; ++x) t = fmaf(fv[h][x], c[x], t);
+            part[h][u] = t;
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          const int f = f0 + h;
+          if (f < nf) {
+            const float s = transpose_reduce8x16(part[h], hl) * inv_tau;
+            if (mine) {
+              sc[(long long)f * rows_cap + grow] = s;
+              if (s > m_run[f]) {
+                z_run[f] = z_run[f] * expf(m_run[f] - s) + 1.f;
+                m_run[f] = s;
+              } else {
+                z_run[f] += expf(s - m_run[f]);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();  // piece consumed by every half-warp
+    if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
+  }
+  return ok;
+}
+
+// (m, z) pairs of two row sets -> the pair of their union
+__device__ __forceinline__ void merge_stat(float &m, float &z, float mo, float zo) {
+  const float mm = fmaxf(m, mo);
+  z = mm == -INFINITY ? 0.f : z * expf(m - mm) + zo * expf(mo - mm);
+  m = mm;
+}
+
+template <int kPool, int NFT>
+__global__ void __launch_bounds__(kSelThreads, 2) hsm_select_kernel(HsmArgs a) {
+  // dynamic shared memory: piece ring | query heads (fp32) | weight keys
+  extern __shared__ __align__(128) uint8_t dyn_raw[];
+  uint8_t *ring = dyn_raw;
+  float *qs = reinterpret_cast<float *>(dyn_raw + kRing * kPieceBytes);
+  uint32_t *keys = reinterpret_cast<uint32_t *>(dyn_raw + kRing * kPieceBytes + a.nf * kD * 4);
+  __shared__ __align__(8) uint64_t bars[kRing];
+  __shared__ RankSmem rs;
+  __shared__ float2 wstat[kSelThreads / 32][kHsmMaxHeads];
+  __shared__ float s_m[kHsmMaxHeads], s_iz[kHsmMaxHeads];
+  __shared__ int s_last, s_failed;
+
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long prob = blockIdx.x / a.n_chunks;  // = b * G + g
+  const int chunk = (int)(blockIdx.x - prob * a.n_chunks);
+  const long long b = prob / a.G;
+  int pos = a.q_start;
+  int32_t *out = a.idx + prob * a.S;
+  if (a.seq_len) {  // the query is the sequence's last token
+    const int len = a.seq_len[b];
+    if (len < 1 || len > a.T) {  // an invalid length: an empty set (every chunk returns here)
+      if (chunk == 0)
+        for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+      return;
+    }
+    pos = len - 1;
+  }
+  const BlockParts bp = block_parts(pos, kBlk, a.n_init, a.n_local);
+  const int ncand = bp.cand_hi - bp.cand_lo;
+  if (ncand <= a.k || a.k == 0) {  // nothing to rank (every chunk returns here)
+    if (chunk == 0) write_set(out, bp, min(ncand, a.k), a.S, true);
+    return;
+  }
+
+  // the rows the query sees: blocks 0..c, or the windows complete by pos
+  const int dom_blocks = bp.c + 1;
+  const int dom_rows = kPool == 1 ? min(dom_blocks, a.NR) : min(window_count(pos + 1), a.NR);
+  const int blo = chunk * a.CH;
+  const int row_lo = blo * kPool;
+  const int n_rows = max(0, min(min(dom_blocks, blo + a.CH) * kPool, dom_rows) - row_lo);
+  const uint16_t *kc_bg = a.kc + prob * (long long)a.NR * kD;
+  if (tid == 0) {
+    for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
+    fence_mbar_init();
+    prime_ring(kc_bg, row_lo, n_rows, ring, bars);
+  }
+  const uint16_t *q = a.Q + prob * (long long)a.nf * kD;
+  for (int t = tid; t < a.nf * kD; t += kSelThreads) qs[t] = __uint_as_float(((uint32_t)q[t]) << 16);
+  __syncthreads();
+
+  float m_run[NFT], z_run[NFT];
+#pragma unroll
+  for (int f = 0; f < NFT; ++f) {
+    m_run[f] = -INFINITY;
+    z_run[f] = 0.f;
+  }
+  float *sc = a.scores + prob * (long long)a.nf * a.rows_cap;
+  const bool ok = score_rows_heads<NFT>(kc_bg, qs, a.nf, a.inv_tau, row_lo, n_rows, sc,
+                                        a.rows_cap, m_run, z_run, ring, bars);
+  if (!ok && tid == 0) a.failed[prob] = 1u;
+
+  // this chunk's (max, normaliser) per head
+#pragma unroll
+  for (int f = 0; f < NFT; ++f) {
+    if (f < a.nf) {
+      float m = m_run[f], z = z_run[f];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+        const float zo = __shfl_xor_sync(0xffffffffu, z, o);
+        merge_stat(m, z, mo, zo);
+      }
+      if (lane == 0) wstat[warp][f] = make_float2(m, z);
+    }
+  }
+  __syncthreads();
+  if (tid < a.nf) {
+    float m = wstat[0][tid].x, z = wstat[0][tid].y;
+    for (int w = 1; w < kSelThreads / 32; ++w) merge_stat(m, z, wstat[w][tid].x, wstat[w][tid].y);
+    a.stats[(prob * a.n_chunks + chunk) * a.nf + tid] = make_float2(m, z);
+  }
+
+  // ---- the last chunk to finish weighs and ranks the candidates ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned t = atomicAdd(&a.counters[prob], 1u);
+    s_last = (t == (unsigned)(a.n_chunks - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (tid == 0) s_failed = (int)__ldcg(a.failed + prob);
+  if (tid < a.nf) {
+    float M = -INFINITY, Z = 0.f;
+    for (int ch = 0; ch < a.n_chunks; ++ch) {
+      const float2 st = __ldcg(a.stats + (prob * a.n_chunks + ch) * a.nf + tid);
+      merge_stat(M, Z, st.x, st.y);
+    }
+    s_m[tid] = Z > 0.f ? M : 0.f;
+    s_iz[tid] = Z > 0.f ? 1.f / Z : 0.f;
+  }
+  __syncthreads();
+  if (s_failed) {  // a copy never landed: report an empty set rather than a wrong one
+    for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+    if (tid == 0) {
+      a.failed[prob] = 0u;
+      a.counters[prob] = 0u;
+    }
+    return;
+  }
+  // Weights of the candidates as keys.  A thread takes 8 candidates at a
+  // time and, head by head, issues all their loads before using any, so the
+  // L2 latency is paid once per head, not once per value; on the window grid
+  // one 16-byte load brings a block's four windows (the fourth, straddling
+  // one is not pooled).
+  constexpr int kW = kPool == 1 ? 1 : 3;
+#pragma unroll 1
+  for (int base = 0; base < ncand; base += 8 * kSelThreads) {
+    float x[8][kW];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int rr = 0; rr < kW; ++rr) x[i][rr] = 0.f;
+#pragma unroll 1
+    for (int f = 0; f < a.nf; ++f) {
+      const float *scf = sc + (long long)f * a.rows_cap;
+      float v[8][kW];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = base + i * kSelThreads + tid;
+        const int j = bp.cand_lo + min(e, ncand - 1);  // past the end: a valid row, unused
+        if (kPool == 1) {
+          v[i][0] = __ldcg(scf + j);
+        } else {
+          const float4 q4 = __ldcg(reinterpret_cast<const float4 *>(scf + 4LL * j));
+          v[i][0] = q4.x;
+          v[i][kW > 1 ? 1 : 0] = q4.y;
+          v[i][kW > 2 ? 2 : 0] = q4.z;
+        }
+      }
+      const float mf = s_m[f], izf = s_iz[f];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int rr = 0; rr < kW; ++rr) x[i][rr] += expf(v[i][rr] - mf) * izf;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int e = base + i * kSelThreads + tid;
+      if (e < ncand) {
+        const int j = bp.cand_lo + e;
+        float w = -INFINITY;
+#pragma unroll
+        for (int rr = 0; rr < kW; ++rr)
+          if (j * kPool + rr < dom_rows) w = fmaxf(w, x[i][rr]);  // windows that exist
+        keys[e] = orderable_key(w);
+      }
+    }
+  }
+  __syncthreads();
+  uint32_t tau = 0;
+  int need = 0;
+  if (a.k <= kTopkMaxK && ncand <= kTopkMaxN && !a.old_rank)
+    find_threshold_topk(keys, ncand, a.k, reinterpret_cast<uint32_t *>(ring), rs, tau, need);
+  else
+    find_threshold(keys, ncand, a.k, rs, tau, need);
+  int32_t *top = out + bp.init_hi;
+  const int ntop = compact_kept(keys, ncand, tau, need, a.k, rs,
+                                [&](int p2, int e) { st_list(top + p2, bp.cand_lo + e); });
+  write_set(out, bp, ntop, a.S, false);
+  if (tid == 0) a.counters[prob] = 0u;
+}
+
 }  // namespace
 
 int env_int(const char *name) {
@@ -730,6 +1033,118 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     size_t &r = raised[pool == 1 ? 0 : 1][dev];
+    if (r < smem) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
+      r = smem;
+    }
+  }
+  const long long grid = pl.n_problems * pl.n_chunks;
+  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Chunks cover the seen blocks 0..c of a query at the end of the sequence
+// (the most any query has), sized by the same one-wave rule as plan_select.
+HsmPlan plan_head_softmax(const sparda_params &p, int nf, int pool) {
+  HsmPlan pl{};
+  pl.n_problems = (long long)p.B * p.G;
+  const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
+  pl.ncand_max = bp.cand_hi - bp.cand_lo;
+  const int dom = bp.c + 1;
+  pl.CH = dom;
+  pl.n_chunks = 1;
+  pl.rows_cap = 0;
+  pl.ws_bytes = 0;
+  if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
+  const int forced = env_int("SPARDA_SELECT_CHUNK");
+  int CH;
+  if (forced > 0) {
+    CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
+  } else {
+    static int sm_count[64] = {0};
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+      if (sm_count[dev] == 0 &&
+          cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sm_count[dev] = 148;
+      n_sm = sm_count[dev];
+    }
+    (void)cudaGetLastError();
+    const long long wave = 2LL * n_sm;
+    const long long per = std::max<long long>(1, wave / pl.n_problems);
+    CH = (int)(ceil_div_ll(ceil_div_ll(dom, per), kSelThreads) * kSelThreads);
+    CH = std::min(std::max(CH, kSelThreads), 1024 / pool);
+  }
+  pl.CH = std::min(CH, (int)ceil_div_ll(dom, kSelThreads) * kSelThreads);
+  pl.n_chunks = (int)ceil_div_ll(dom, pl.CH);
+  pl.rows_cap = pl.n_chunks * pl.CH * pool;
+  size_t off = 2 * (((size_t)pl.n_problems * 4 + 255) & ~(size_t)255);  // tickets, failure flags
+  off += ((size_t)pl.n_problems * pl.n_chunks * nf * 8 + 255) & ~(size_t)255;  // chunk stats
+  off += (size_t)pl.n_problems * nf * pl.rows_cap * 4;                      // head scores
+  pl.ws_bytes = off;
+  return pl;
+}
+
+int head_softmax_supported(const HsmPlan &pl, int nf) {
+  if (nf < 1 || nf > kHsmMaxHeads) return 0;
+  if (pl.ncand_max > kMaxCand) return 0;
+  return 1;
+}
+
+cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const uint16_t *Q,
+                                int nf, int q_start, float tau, const uint16_t *kc, int32_t *idx,
+                                void *ws, cudaStream_t stream, int pool) {
+  if (pl.n_problems == 0) return cudaSuccess;
+  HsmArgs a;
+  a.seq_len = p.seq_len;
+  a.Q = Q;
+  a.kc = kc;
+  a.idx = idx;
+  a.G = p.G;
+  a.nf = nf;
+  a.NR = pool == 1 ? (p.T + kBlk - 1) / kBlk : window_count(p.T);
+  a.k = p.k;
+  a.n_init = p.n_init;
+  a.n_local = p.n_local;
+  a.q_start = q_start;
+  a.S = p.k + p.n_init + p.n_local;
+  a.T = p.T;
+  a.CH = pl.CH;
+  a.n_chunks = pl.n_chunks;
+  a.rows_cap = pl.rows_cap;
+  a.inv_tau = 1.f / tau;
+  a.old_rank = env_int("SPARDA_SELECT_BINNED") > 0 ? 1 : 0;
+  a.counters = nullptr;
+  a.failed = nullptr;
+  a.stats = nullptr;
+  a.scores = nullptr;
+  if (pl.ws_bytes > 0) {
+    char *w = static_cast<char *>(ws);
+    const size_t words = ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
+    a.counters = reinterpret_cast<uint32_t *>(w);
+    a.failed = reinterpret_cast<uint32_t *>(w + words);
+    a.stats = reinterpret_cast<float2 *>(w + 2 * words);
+    a.scores = reinterpret_cast<float *>(w + 2 * words +
+                                         (((size_t)pl.n_problems * pl.n_chunks * nf * 8 + 255) & ~(size_t)255));
+  }
+  const size_t smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 +
+                      (size_t)std::max(pl.ncand_max, 1) * 4;
+  // the head count rounded up to a power of two fixes the unrolling
+  const int nft_i = nf <= 1 ? 0 : nf <= 2 ? 1 : nf <= 4 ? 2 : nf <= 8 ? 3 : 4;
+  void (*const kerns[2][5])(HsmArgs) = {
+      {hsm_select_kernel<1, 1>, hsm_select_kernel<1, 2>, hsm_select_kernel<1, 4>,
+       hsm_select_kernel<1, 8>, hsm_select_kernel<1, 16>},
+      {hsm_select_kernel<4, 1>, hsm_select_kernel<4, 2>, hsm_select_kernel<4, 4>,
+       hsm_select_kernel<4, 8>, hsm_select_kernel<4, 16>}};
+  auto kern = kerns[pool == 1 ? 0 : 1][nft_i];
+  {
+    static size_t raised[2][5][64] = {{{0}}};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    size_t &r = raised[pool == 1 ? 0 : 1][nft_i][dev];
     if (r < smem) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;

@@ -110,7 +110,9 @@ enum sparda_op {
   SPARDA_OP_PREFETCH = 2,
   SPARDA_OP_ATTN_DECODE = 3,
   SPARDA_OP_ATTN_PREFILL = 4,
-  SPARDA_OP_SELECT_WINDOWS = 5
+  SPARDA_OP_SELECT_WINDOWS = 5,
+  SPARDA_OP_HEAD_SOFTMAX = 6,         /* sparda_head_softmax_select (nq = 1)         */
+  SPARDA_OP_HEAD_SOFTMAX_WINDOWS = 7  /* sparda_head_softmax_select_windows (nq = 1) */
 };
 
 /* how sparda_sparse_attn_decode finds the storage of list entry s */
@@ -177,8 +179,8 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
  * Ranking: higher fp32 score first, equal scores -> lower block index.
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_SELECT, p, nq, nf)
  *       bytes; it must be zero-filled before its first use, and each call
- *       leaves it zero-filled again.  Calls sharing one workspace must not
- *       overlap on the device.
+ *       leaves its tickets at zero again (the rest is scratch).  Calls sharing
+ *       one workspace must not overlap on the device.
  */
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
                            const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
@@ -234,6 +236,53 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
                                    int q_start, const void *kw, int win, int stride,
                                    int32_t *idx, void *ws, size_t ws_bytes,
                                    sparda_stream_t stream);
+
+/*
+ * sparda_head_softmax_select -- the original selector in its per-head softmax
+ *   form, the comparator the Forecast indexer replaces.
+ *   [p4 "Training: distilling the selector you already have"], Eq. 6: the
+ *   original selector's shared importance score is, summed over the group's
+ *   query heads, each head's softmax over the compressed keys of
+ *   Q_h Kc^T / tau; the selected set is its top-k minus the initial and
+ *   local blocks.  [p4 "One Forecast head per GQA group"]: the baseline
+ *   scores with every query head of the group (G score products and a
+ *   softmax per layer).
+ *     w_r = sum_h exp(s_hr - M_h) / Z_h,  s_hr = Q_h . Kc_r / tau,
+ *     M_h = max_r s_hr,  Z_h = sum_r exp(s_hr - M_h),
+ *   r over every key row the query sees: blocks 0..c (c = the query's own
+ *   block), or on the window grid the windows complete by the query position.
+ *   The initial and local rows and the windows straddling two blocks count
+ *   in Z_h but are never ranked.  Set = init U top-k(w) U local, ascending,
+ *   -1 padded; equal weights go to the lower block index.  Weights are fp32
+ *   (scores, exp, sums).
+ * Q     bf16 [B][G][nf][d]  the decode query's heads by group, 1 <= nf <= 16
+ * kc    bf16 [B][G][NB][d]  block keys
+ * tau   softmax temperature; <= 0 means sqrt(d)
+ * idx   int32 [B][G][S], S = k + n_init + n_local
+ * One query token per sequence: at q_start (0 <= q_start < T), or with
+ * per-sequence lengths the sequence's last token (q_start is checked only).
+ * ws    device workspace of sparda_workspace_size(SPARDA_OP_HEAD_SOFTMAX, p,
+ *       1, nf) bytes, zero-filled before its first use; each call leaves its
+ *       tickets and flags at zero again (the rest is scratch).  Calls sharing
+ *       one workspace must not overlap on the device.
+ */
+int sparda_head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start,
+                               float tau, const void *kc, int32_t *idx, void *ws,
+                               size_t ws_bytes, sparda_stream_t stream);
+
+/*
+ * sparda_head_softmax_select_windows -- the same on the window grid: kw bf16
+ *   [B][G][NW][d] window keys (win = 32, stride = 16, NW as
+ *   sparda_compress_windows gives for T), and a block weighs as much as the
+ *   heaviest of the windows inside it (windows 4j, 4j+1, 4j+2; -inf for a
+ *   block with none), the selector's final max-pooling
+ *   [p4 "Training: distilling the selector you already have"].  Workspace op
+ *   SPARDA_OP_HEAD_SOFTMAX_WINDOWS.
+ */
+int sparda_head_softmax_select_windows(const sparda_params *p, const void *Q, int nf,
+                                       int q_start, float tau, const void *kw, int win,
+                                       int stride, int32_t *idx, void *ws, size_t ws_bytes,
+                                       sparda_stream_t stream);
 
 /*
  * sparda_prefetch_blocks -- gather the selected K/V blocks of one layer from

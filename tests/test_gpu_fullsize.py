@@ -210,3 +210,24 @@ def test_prefill_chunk_full_size_sampled():
         check_attention(gpu_o, ora_o, what)
     del pc
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_full_size(windows):
+    """The original selector's per-head softmax form at the shapes bench.py
+    times (B=16, G=8 groups of 4 query heads, T=131072, k=64 + 1 initial +
+    2 local), through the same class: every (sequence, group) set against the
+    oracle on the same key bytes."""
+    import bench
+    c = bench.HeadSoftmaxCase(windows, n_layers=1)
+    c.head_softmax(c.kc[0])
+    torch.cuda.synchronize()
+    got = c.idx.cpu().numpy()
+    w = c.w
+    Q, kc = host_bits(c.Q), host_bits(c.kc[0])
+    ora, kth, kth1, wb = oracle.select_head_softmax(Q, kc, w.T, w.k, w.n_init, w.n_local, w.T - 1,
+                                                    c.tau, windows=windows)
+    B, G, S = got.shape
+    exact = check_sets(got.reshape(B, 1, G, S), ora.reshape(B, 1, G, S), kth.reshape(B, 1, G),
+                       kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), "head softmax full size")
+    assert exact >= B * G - 2, "only %d of %d sets bit-exact" % (exact, B * G)

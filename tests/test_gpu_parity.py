@@ -297,6 +297,167 @@ def test_select_windows_compressed_from_keys():
 
 
 # --------------------------------------------------------------------------
+# the original selector's per-head softmax form (block and window grids)
+# --------------------------------------------------------------------------
+
+def gpu_head_softmax(Q_bits, kc_bits, T, k, n_init, n_local, q_start, tau, windows, lens=None,
+                     ws=None):
+    """Q [B][G][nf][d] bits; kc block or window keys -> idx [B][G][S]."""
+    B, G, nf, d = Q_bits.shape
+    sl = None if lens is None else torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local, seq_len=sl)
+    S = k + n_init + n_local
+    idx = torch.full((B, G, S), -7, dtype=torch.int32, device="cuda")
+    op = abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS if windows else abi.SPARDA_OP_HEAD_SOFTMAX
+    if ws is None:
+        ws = abi.workspace(op, p, 1, nf)
+    if windows:
+        abi.sparda_head_softmax_select_windows(p, dev_bf16(Q_bits), nf, q_start, tau,
+                                               dev_bf16(kc_bits), 32, 16, idx, ws)
+    else:
+        abi.sparda_head_softmax_select(p, dev_bf16(Q_bits), nf, q_start, tau, dev_bf16(kc_bits),
+                                       idx, ws)
+    torch.cuda.synchronize()
+    out = idx.cpu().numpy()
+    assert not (out == -7).any(), "entries left unwritten"
+    return out
+
+
+def _hsm_check(got, Q, kc, T, k, n_init, n_local, q_start, tau, windows, what):
+    """got [B][G][S] against the oracle on the same inputs (band rule at near
+    ties, on the oracle's own block weights)."""
+    ora, kth, kth1, wb = oracle.select_head_softmax(Q, kc, T, k, n_init, n_local, q_start, tau,
+                                                    windows=windows)
+    B, G, S = got.shape
+    return check_sets(got.reshape(B, 1, G, S), ora.reshape(B, 1, G, S), kth.reshape(B, 1, G),
+                      kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), what)
+
+
+@pytest.mark.parametrize("T,nf,k,n_local,chunk", [
+    (8192 + 20, 4, 16, 2, "0"), (32768, 4, 64, 2, "256"), (20000, 8, 40, 1, "512"),
+    (5000 + 33, 16, 8, 0, "0"), (32768, 2, 100, 2, "0"), (65536 + 64, 4, 63, 32, "0"),
+    (12000, 1, 20, 2, "0")])
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_select(T, nf, k, n_local, chunk, windows, monkeypatch):
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    rng = W.rng_for(140 + T + nf, int(windows))
+    B, G, d = 2, 3, 128
+    NR = oracle.window_count(T) if windows else (T + 63) // 64
+    kc = W.normal_bf16(rng, (B, G, NR, d))
+    Q = W.normal_bf16(rng, (B, G, nf, d))
+    tau = float(np.sqrt(d))
+    got = gpu_head_softmax(Q, kc, T, k, 1, n_local, T - 1, tau, windows)
+    _hsm_check(got, Q, kc, T, k, 1, n_local, T - 1, tau, windows, "head softmax")
+
+
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_query_inside_the_sequence_and_default_tau(windows):
+    """A query before the end (q_start < T - 1) normalises over the rows it
+    sees only; tau <= 0 means sqrt(d)."""
+    rng = W.rng_for(150, int(windows))
+    B, G, nf, d, T = 2, 2, 4, 128, 12000
+    NR = oracle.window_count(T) if windows else (T + 63) // 64
+    kc = W.normal_bf16(rng, (B, G, NR, d))
+    Q = W.normal_bf16(rng, (B, G, nf, d))
+    q = 7000 + 21
+    got = gpu_head_softmax(Q, kc, T, 12, 1, 2, q, 0.0, windows)
+    _hsm_check(got, Q, kc, T, 12, 1, 2, q, float(np.sqrt(d)), windows, "inside")
+
+
+@pytest.mark.parametrize("binned", [False, True])
+@pytest.mark.parametrize("chunk", ["0", "256"])
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_exact_ties_lower_index_wins(windows, chunk, binned, monkeypatch):
+    """Key rows drawn from six distinct rows with integer entries along the
+    heads' axes: every product is exact, equal rows weigh exactly the same
+    on both sides, and the lower block index must win every tie."""
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    if binned:
+        monkeypatch.setenv("SPARDA_SELECT_BINNED", "1")
+    rng = np.random.default_rng(151)
+    B, G, nf, d, T = 2, 2, 4, 128, 1500 * 64
+    NR = oracle.window_count(T) if windows else T // 64
+    base = np.zeros((6, d), np.float32)
+    base[:, :nf] = rng.integers(-2, 3, (6, nf))
+    kc = W.f32_to_bf16_bits(base[rng.integers(0, 6, (B, G, NR))])
+    Qf = np.zeros((B, G, nf, d), np.float32)
+    for h in range(nf):
+        Qf[:, :, h, h] = 1.0
+    Q = W.f32_to_bf16_bits(Qf)
+    for k in (1, 17, 64, 100):
+        got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, 1.0, windows)
+        ora = oracle.select_head_softmax(Q, kc, T, k, 1, 2, T - 1, 1.0, windows=windows)[0]
+        assert np.array_equal(got, ora), "k=%d" % k
+
+
+@pytest.mark.parametrize("k,n_init,n_local", [(0, 1, 2), (61, 1, 2), (70, 1, 2), (5, 0, 0),
+                                              (5, 3, 7), (1, 0, 1)])
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_degenerate_budgets(k, n_init, n_local, windows):
+    rng = W.rng_for(152, k * 100 + n_init * 10 + n_local + 1000 * int(windows))
+    B, G, nf, T = 2, 2, 4, 64 * 64
+    NR = oracle.window_count(T) if windows else T // 64
+    kc = W.normal_bf16(rng, (B, G, NR, 128))
+    Q = W.normal_bf16(rng, (B, G, nf, 128))
+    got = gpu_head_softmax(Q, kc, T, k, n_init, n_local, T - 1, 11.3, windows)
+    _hsm_check(got, Q, kc, T, k, n_init, n_local, T - 1, 11.3, windows, "degenerate")
+
+
+@pytest.mark.parametrize("chunk", ["0", "256"])
+@pytest.mark.parametrize("windows", [False, True])
+def test_head_softmax_per_sequence_lengths(windows, chunk, monkeypatch):
+    """Sequences of different lengths in one batch, one invalid: each set is
+    the oracle's on that sequence alone; the invalid one is all -1.  A second
+    call on the same workspace gives the same sets (tickets back at zero)."""
+    if chunk != "0":
+        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    rng = W.rng_for(153, int(windows))
+    B, G, nf, d, T, k = 5, 2, 4, 128, 20000, 16
+    lens = [T, 3000 + 17, 70, 0, 9000]
+    NR = oracle.window_count(T) if windows else (T + 63) // 64
+    kc = W.normal_bf16(rng, (B, G, NR, d))
+    Q = W.normal_bf16(rng, (B, G, nf, d))
+    tau = 11.0
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    p = abi.make_params(B, G * nf, G, T, k, seq_len=sl)
+    op = abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS if windows else abi.SPARDA_OP_HEAD_SOFTMAX
+    ws = abi.workspace(op, p, 1, nf)
+    got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws)
+    again = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws)
+    assert np.array_equal(got, again)
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert np.all(got[b] == -1)
+            continue
+        nr = oracle.window_count(L) if windows else (L + 63) // 64
+        Qb = np.ascontiguousarray(Q[b:b + 1])
+        kb = np.ascontiguousarray(kc[b:b + 1, :, :nr])
+        _hsm_check(got[b:b + 1], Qb, kb, L, k, 1, 2, L - 1, tau, windows, "len %d" % L)
+
+
+def test_head_softmax_rejects_bad_arguments():
+    B, G, nf, T = 1, 2, 4, 4096
+    p = abi.make_params(B, G * nf, G, T, 8)
+    kc = torch.zeros(B, G, T // 64, 128, dtype=torch.bfloat16, device="cuda")
+    Q = torch.zeros(B, G, nf, 128, dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros(B, G, 11, dtype=torch.int32, device="cuda")
+    ws = abi.workspace(abi.SPARDA_OP_HEAD_SOFTMAX, p, 1, nf)
+    for args, status in [((nf, T, 1.0), abi.SPARDA_EINVAL),        # query past the end
+                         ((0, T - 1, 1.0), abi.SPARDA_EINVAL),     # no heads
+                         ((32, T - 1, 1.0), abi.SPARDA_EUNSUPPORTED),
+                         ((nf, T - 1, float("nan")), abi.SPARDA_EINVAL)]:
+        with pytest.raises(abi.SpardaError) as e:
+            abi.sparda_head_softmax_select(p, Q, args[0], args[1], args[2], kc, idx, ws)
+        assert e.value.status == status
+    with pytest.raises(abi.SpardaError) as e:
+        abi.sparda_head_softmax_select(p, Q, nf, T - 1, 1.0, kc, idx, None)
+    assert e.value.status == abi.SPARDA_EWORKSPACE
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX, p, 2, nf) == 0   # decode only
+
+
+# --------------------------------------------------------------------------
 # per-sequence lengths (decode) and a real model's budget
 # --------------------------------------------------------------------------
 
