@@ -34,6 +34,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "rank.cuh"
+#include "tc.cuh"
 
 namespace sparda {
 
@@ -649,90 +650,6 @@ struct HsmArgs {
   int old_rank;
 };
 
-// Score rows [lo, lo + n) with every head: scores to sc (head-major, row
-// stride rows_cap), and per head a running (max, sum of exp(s - max)) over
-// the rows this thread saw.  Streams like score_rows.  NFT (a power of two
-// >= nf) fixes the unrolling; heads are taken four at a time, and each row
-// is converted from bf16 once per group of four heads.
-template <int NFT>
-__device__ bool score_rows_heads(const uint16_t *kc_bg, const float *qs, int nf, float inv_tau,
-                                 int lo, int n, float *sc, int rows_cap, float (&m_run)[NFT],
-                                 float (&z_run)[NFT], uint8_t *ring, uint64_t *bars) {
-  constexpr int HG = NFT < 4 ? NFT : 4;
-  const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
-  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
-  bool ok = true;
-#pragma unroll 1
-  for (int pc = 0; pc < n_pc; ++pc) {
-    const bool landed = mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1));
-    if (__syncthreads_or(!landed)) {
-      ok = false;
-      if (threadIdx.x == 0)
-        for (int q = pc; q < min(n_pc, pc + kRing); ++q)
-          (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
-      __syncthreads();
-      break;
-    }
-    const int rows = min(kPieceRows, n - pc * kPieceRows);
-    const uint8_t *piece = ring + (pc % kRing) * kPieceBytes;
-    const int row0 = hw * 8;
-    const int r = row0 + (hl >> 1);
-    const bool mine = (hl & 1) == 0 && r < rows;
-    const long long grow = (long long)lo + pc * kPieceRows + r;
-#pragma unroll
-    for (int f0 = 0; f0 < NFT; f0 += HG) {
-      if (f0 < nf) {  // uniform over the block
-        float fv[HG][8];
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-          if (f0 + h < nf) {
-            a = *reinterpret_cast<const float4 *>(qs + (f0 + h) * kD + hl * 8);
-            b = *reinterpret_cast<const float4 *>(qs + (f0 + h) * kD + hl * 8 + 4);
-          }
-          fv[h][0] = a.x; fv[h][1] = a.y; fv[h][2] = a.z; fv[h][3] = a.w;
-          fv[h][4] = b.x; fv[h][5] = b.y; fv[h][6] = b.z; fv[h][7] = b.w;
-        }
-        float part[HG][8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = row0 + u < rows
-                              ? *reinterpret_cast<const uint4 *>(piece + (row0 + u) * (kD * 2) + hl * 16)
-                              : make_uint4(0, 0, 0, 0);
-          const float c[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                              bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-#pragma unroll
-          for (int h = 0; h < HG; ++h) {
-            float t = fv[h][0] * c[0];
-#pragma unroll
-            for (int x = 1; x < 8; ++x) t = fmaf(fv[h][x], c[x], t);
-            part[h][u] = t;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          const int f = f0 + h;
-          if (f < nf) {
-            const float s = transpose_reduce8x16(part[h], hl) * inv_tau;
-            if (mine) {
-              sc[(long long)f * rows_cap + grow] = s;
-              if (s > m_run[f]) {
-                z_run[f] = z_run[f] * expf(m_run[f] - s) + 1.f;
-                m_run[f] = s;
-              } else {
-                z_run[f] += expf(s - m_run[f]);
-              }
-            }
-          }
-        }
-      }
-    }
-    __syncthreads();  // piece consumed by every half-warp
-    if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
-  }
-  return ok;
-}
-
 // (m, z) pairs of two row sets -> the pair of their union
 __device__ __forceinline__ void merge_stat(float &m, float &z, float mo, float zo) {
   const float mm = fmaxf(m, mo);
@@ -740,14 +657,32 @@ __device__ __forceinline__ void merge_stat(float &m, float &z, float mo, float z
   m = mm;
 }
 
+// the group's heads as the MMA's B operand: [2 dim halves][16 heads][64 dims]
+constexpr int kHsmOpB = 2 * 16 * 128;
+constexpr int kHsmTmemCols = 32;  // two 16-column score stages
+
+// one 128-row piece of key rows by TMA (two 64-dim halves, 128-byte swizzle)
+__device__ __forceinline__ void hsm_issue_piece(const CUtensorMap *map, int row_lo, int pc,
+                                                int prob, uint8_t *ring, uint64_t *bars) {
+  uint64_t *bar = &bars[pc % kRing];
+  uint8_t *dst = ring + (pc % kRing) * kPieceBytes;
+  mbar_arrive_expect_tx(bar, (uint32_t)kPieceBytes);
+  const int y = row_lo + pc * kPieceRows;
+  tc::tma_load_3d(dst, map, 0, y, prob, bar);
+  tc::tma_load_3d(dst + kPieceBytes / 2, map, 64, y, prob, bar);
+}
+
 template <int kPool, int NFT>
-__global__ void __launch_bounds__(kSelThreads, 2) hsm_select_kernel(HsmArgs a) {
-  // dynamic shared memory: piece ring | query heads (fp32) | weight keys
-  extern __shared__ __align__(128) uint8_t dyn_raw[];
-  uint8_t *ring = dyn_raw;
-  float *qs = reinterpret_cast<float *>(dyn_raw + kRing * kPieceBytes);
-  uint32_t *keys = reinterpret_cast<uint32_t *>(dyn_raw + kRing * kPieceBytes + a.nf * kD * 4);
-  __shared__ __align__(8) uint64_t bars[kRing];
+__global__ void __launch_bounds__(kSelThreads, 2)
+    hsm_select_kernel(const __grid_constant__ CUtensorMap mapKc, HsmArgs a) {
+  // dynamic shared memory, aligned to 1024 bytes by hand (the swizzle atom):
+  // piece ring | head operand | weight keys
+  extern __shared__ __align__(128) uint8_t hsm_dyn[];
+  uint8_t *ring = hsm_dyn + ((1024u - (smem_addr(hsm_dyn) & 1023u)) & 1023u);
+  uint8_t *opB = ring + kRing * kPieceBytes;
+  uint32_t *keys = reinterpret_cast<uint32_t *>(opB + kHsmOpB);
+  __shared__ __align__(8) uint64_t bars[kRing + 2];  // piece landed x kRing, MMA done x 2 stages
+  __shared__ uint32_t tmem_slot;
   __shared__ RankSmem rs;
   __shared__ float2 wstat[kSelThreads / 32][kHsmMaxHeads];
   __shared__ float s_m[kHsmMaxHeads], s_iz[kHsmMaxHeads];
@@ -783,16 +718,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsm_select_kernel(HsmArgs a) {
   const int blo = chunk * a.CH;
   const int row_lo = blo * kPool;
   const int n_rows = max(0, min(min(dom_blocks, blo + a.CH) * kPool, dom_rows) - row_lo);
-  const uint16_t *kc_bg = a.kc + prob * (long long)a.NR * kD;
-  if (tid == 0) {
-    for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
-    fence_mbar_init();
-    prime_ring(kc_bg, row_lo, n_rows, ring, bars);
-  }
-  const uint16_t *q = a.Q + prob * (long long)a.nf * kD;
-  for (int t = tid; t < a.nf * kD; t += kSelThreads) qs[t] = __uint_as_float(((uint32_t)q[t]) << 16);
-  __syncthreads();
-
+  const int n_pc = (n_rows + kPieceRows - 1) / kPieceRows;
   float m_run[NFT], z_run[NFT];
 #pragma unroll
   for (int f = 0; f < NFT; ++f) {
@@ -800,8 +726,111 @@ __global__ void __launch_bounds__(kSelThreads, 2) hsm_select_kernel(HsmArgs a) {
     z_run[f] = 0.f;
   }
   float *sc = a.scores + prob * (long long)a.nf * a.rows_cap;
-  const bool ok = score_rows_heads<NFT>(kc_bg, qs, a.nf, a.inv_tau, row_lo, n_rows, sc,
-                                        a.rows_cap, m_run, z_run, ring, bars);
+  bool ok = true;
+
+  // ---- scores of the chunk's rows on the tensor cores: for each 128-row
+  // piece, D[row][head] = Kc_piece . Q^T (M = 128 rows, N = 16 heads, K = 128
+  // in eight steps), D double-buffered in TMEM so the product of the next
+  // piece runs while warps 0-3 read this one (thread = row = TMEM lane) ----
+  if (n_pc > 0) {
+    if ((smem_addr(ring) & 1023u) != 0u) {  // cannot happen with the sizes launched
+      ok = false;
+    } else {
+      if (tid == 0) {
+        for (int q = 0; q < kRing + 2; ++q) mbar_init(&bars[q], 1);
+        fence_mbar_init();
+        tc::prefetch_map(&mapKc);
+        for (int pc = 0; pc < min(kRing, n_pc); ++pc)
+          hsm_issue_piece(&mapKc, row_lo, pc, (int)prob, ring, bars);
+      }
+      {  // heads -> B operand (rows >= nf are zero); 256 threads, one 16-byte chunk each
+        const int half = tid >> 7, row = (tid >> 3) & 15, ch = tid & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < a.nf)
+          v = *reinterpret_cast<const uint4 *>(a.Q + (prob * a.nf + row) * (long long)kD + half * 64 + ch * 8);
+        *reinterpret_cast<uint4 *>(opB + half * (kHsmOpB / 2) + tc::sw128_offset(row, ch * 8)) = v;
+        fence_proxy_async_smem();
+      }
+      if (warp == 0) tc::tmem_alloc(&tmem_slot, kHsmTmemCols);
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      const uint32_t tmem = tmem_slot;
+      constexpr uint32_t idesc = tc::idesc_bf16(kPieceRows, 16, false, false);
+      int n_issued = 0, n_loaded = min(kRing, n_pc);  // thread 0's view
+      auto issue_mma = [&](int pc) -> bool {  // thread 0
+        if (!mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1))) return false;
+        tc::fence_after_sync();
+        const uint8_t *pa = ring + (pc % kRing) * kPieceBytes;
+        const uint32_t d = tmem + (uint32_t)((pc & 1) * 16);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16(d, tc::sdesc(pa + (kk >> 2) * (kPieceBytes / 2) + (kk & 3) * 32, 16, 1024),
+                       tc::sdesc(opB + (kk >> 2) * (kHsmOpB / 2) + (kk & 3) * 32, 16, 1024), idesc,
+                       kk > 0);
+        tc::mma_commit(&bars[kRing + (pc & 1)]);
+        n_issued = pc + 1;
+        return true;
+      };
+      int bad = 0;
+      if (tid == 0) bad = !issue_mma(0);
+      bad = __syncthreads_or(bad);
+      int pc = 0;
+#pragma unroll 1
+      for (; !bad && pc < n_pc; ++pc) {
+        int fail = 0;
+        if (tid == 0 && pc + 1 < n_pc) fail = !issue_mma(pc + 1);
+        if (warp < 4) {
+          const bool done = mbar_wait_bounded(&bars[kRing + (pc & 1)], (uint32_t)((pc >> 1) & 1));
+          if (__all_sync(0xffffffffu, done)) {
+            tc::fence_after_sync();
+            float v[16];
+            tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((pc & 1) * 16), v);
+            const int rows = min(kPieceRows, n_rows - pc * kPieceRows);
+            if (tid < rows) {
+              const long long grow = (long long)row_lo + pc * kPieceRows + tid;
+#pragma unroll
+              for (int f = 0; f < NFT; ++f) {
+                if (f < a.nf) {
+                  const float s = v[f] * a.inv_tau;
+                  sc[(long long)f * a.rows_cap + grow] = s;
+                  if (s > m_run[f]) {
+                    z_run[f] = z_run[f] * expf(m_run[f] - s) + 1.f;
+                    m_run[f] = s;
+                  } else {
+                    z_run[f] += expf(s - m_run[f]);
+                  }
+                }
+              }
+            }
+          } else {
+            fail = 1;
+          }
+        }
+        tc::fence_before_sync();
+        bad = __syncthreads_or(fail);
+        // piece pc's product is done: its ring slot takes piece pc + kRing
+        if (!bad && tid == 0 && pc + kRing < n_pc) {
+          hsm_issue_piece(&mapKc, row_lo, pc + kRing, (int)prob, ring, bars);
+          n_loaded = pc + kRing + 1;
+        }
+      }
+      if (bad) {
+        ok = false;
+        if (tid == 0) {  // let copies and products in flight finish (bounded) before release
+          for (int q = pc; q < n_loaded; ++q)
+            (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
+          if (n_issued > 0)
+            (void)mbar_wait_bounded(&bars[kRing + ((n_issued - 1) & 1)],
+                                    (uint32_t)(((n_issued - 1) >> 1) & 1));
+        }
+      }
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      if (warp == 0) tc::tmem_dealloc(tmem, kHsmTmemCols);
+    }
+  }
   if (!ok && tid == 0) a.failed[prob] = 1u;
 
   // this chunk's (max, normaliser) per head
@@ -1130,11 +1159,17 @@ cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const
     a.scores = reinterpret_cast<float *>(w + 2 * words +
                                          (((size_t)pl.n_problems * pl.n_chunks * nf * 8 + 255) & ~(size_t)255));
   }
-  const size_t smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 +
+  // Kc (or window keys) [B*G][NR][d] as a 3-D map (d, NR, B*G), 64 x 128-row boxes
+  CUtensorMap mK;
+  const uint64_t kdim[3] = {(uint64_t)kD, (uint64_t)a.NR, (uint64_t)pl.n_problems};
+  const uint64_t kstr[2] = {(uint64_t)kD * 2, (uint64_t)a.NR * kD * 2};
+  const uint32_t kbox[3] = {64, kPieceRows, 1};
+  if (a.NR < 1 || !tc::make_map_nd(&mK, kc, 3, kdim, kstr, kbox)) return cudaErrorNotSupported;
+  const size_t smem = 1024 + (size_t)kRing * kPieceBytes + kHsmOpB +
                       (size_t)std::max(pl.ncand_max, 1) * 4;
   // the head count rounded up to a power of two fixes the unrolling
   const int nft_i = nf <= 1 ? 0 : nf <= 2 ? 1 : nf <= 4 ? 2 : nf <= 8 ? 3 : 4;
-  void (*const kerns[2][5])(HsmArgs) = {
+  void (*const kerns[2][5])(CUtensorMap, HsmArgs) = {
       {hsm_select_kernel<1, 1>, hsm_select_kernel<1, 2>, hsm_select_kernel<1, 4>,
        hsm_select_kernel<1, 8>, hsm_select_kernel<1, 16>},
       {hsm_select_kernel<4, 1>, hsm_select_kernel<4, 2>, hsm_select_kernel<4, 4>,
@@ -1154,7 +1189,7 @@ cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const
     }
   }
   const long long grid = pl.n_problems * pl.n_chunks;
-  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, a);
+  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, mK, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
