@@ -854,17 +854,20 @@ def host_link_peak_gbps(nbytes=1 << 30, reps=5):
 
 
 def time_cold(fn, reps, warm=3):
-    """Median device time of one call with L2 flushed before it: a 256 MB
-    memset (twice L2) runs first on the same stream, outside the events."""
+    """Median device time of one call with L2 flushed before it: a read of
+    256 MB (twice L2) runs first on the same stream, outside the events.  A
+    read leaves L2 holding clean lines, so the timed call pays no write-back
+    of the flush (a memset would leave ~126 MB of dirty lines behind)."""
     import torch
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(reps)]
-    for e0, e1 in evs:
-        flush.zero_()
+    sink = torch.zeros(reps, dtype=torch.float32, device="cuda")
+    for i, (e0, e1) in enumerate(evs):
+        torch.sum(flush, dim=0, out=sink[i])
         e0.record()
         fn()
         e1.record()
@@ -1102,6 +1105,7 @@ def run_sweep():
     dev = torch.device("cuda")
     G, Hq, d, k = 8, 32, 128, 64
     points = []
+    clocks = ClockSampler(torch.cuda.current_device())
     for NB in W.SWEEP_NB:
         for B in W.SWEEP_B:
             T = NB * 64
@@ -1126,8 +1130,9 @@ def run_sweep():
             del kc
     return {"metric": "selection-only sweep: Forecast vs 4-head baseline selector (us per call)",
             "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16",
-            "timing": "median of 15 calls, each after a 256 MB memset that flushes L2 "
-                      "(the memset is outside the events)"}
+            "timing": "median of 15 calls, each after a 256 MB read that flushes L2 "
+                      "(the read is outside the events)",
+            "clocks": clocks.stop()}
 
 
 class HeadSoftmaxCase:
@@ -1204,6 +1209,7 @@ def run_head_softmax(steps):
     out = {"metric": "decode selection, the original selector's per-head softmax form vs "
                      "Forecast (us per call, one layer)",
            "data": "synthetic", "dtype": "bf16", "peak": peak, "peak_kind": peak_kind}
+    clocks = ClockSampler(torch.cuda.current_device())
     for windows in (False, True):
         c = HeadSoftmaxCase(windows)
         h_us = time_back_to_back(c.head_softmax, n)
@@ -1219,6 +1225,7 @@ def run_head_softmax(steps):
                     "l2": "3 layers' keys alternated (%.0f MB)" % (3 * nb / 1e6)}
         del c
         torch.cuda.empty_cache()
+    out["clocks"] = clocks.stop()
     return out
 
 
