@@ -1,6 +1,8 @@
 // select.cu -- Forecast block selection: score every candidate block's
 // compressed key with the group's Forecast vector(s), keep the k best, and
-// join them with the initial and local blocks.
+// join them with the initial and local blocks.  Also the original selector
+// in its per-head softmax form (hsm_select_kernel, further down), the
+// comparator the Forecast indexer replaces.
 //
 // Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
 // lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com);
@@ -637,8 +639,7 @@ constexpr int kHsmMaxHeads = 16;
 
 struct HsmArgs {
   const int32_t *seq_len;
-  const uint16_t *Q;   // [B][G][nf][d]
-  const uint16_t *kc;  // [B][G][NR][d]
+  const uint16_t *Q;   // [B][G][nf][d]; the keys [B][G][NR][d] come through a tensor map
   int32_t *idx;        // [B][G][S]
   uint32_t *counters;  // [problem] tickets
   uint32_t *failed;    // [problem] set when a chunk's copy never landed
@@ -1137,7 +1138,6 @@ cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const
   HsmArgs a;
   a.seq_len = p.seq_len;
   a.Q = Q;
-  a.kc = kc;
   a.idx = idx;
   a.G = p.G;
   a.nf = nf;
