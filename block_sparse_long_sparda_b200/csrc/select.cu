@@ -54,6 +54,7 @@ struct SelArgs {
   uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
   int nq, G, nf, NB, k, n_init, n_local, q_start, S, T;
   int CH, n_chunks, cap;
+  int NBf;       // window grid: blocks the key map covers (all three inner windows present)
   int old_rank;  // 1: always the binned threshold search
 };
 
@@ -433,18 +434,13 @@ __device__ __forceinline__ void prime_ring(const uint16_t *kc_bg, int lo, int n,
   for (int pc = 0; pc < min(kRing, n_pc); ++pc) issue_piece(kc_bg, lo, n, pc, ring, bars);
 }
 
-// kPool = 1: one key row per block, row r scores block lo + r.  kPool = 4:
-// the window grid (32-token windows at stride 16, four per 64-token block):
-// rows are windows, and block j's score is the largest score of the three
-// windows lying inside it (rows 4j, 4j+1, 4j+2; row 4j+3 straddles two
-// blocks and is skipped).  n counts key rows; keys are written per block.
-template <int kPool>
+// Block grid: key row r of the chunk scores block lo + r.
 __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int lo, int n,
                            uint32_t *keys, uint8_t *ring, uint64_t *bars) {
   const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
   const int n_pc = (n + kPieceRows - 1) / kPieceRows;
   // the first pieces were issued by the caller's thread 0 right after the
-  // barriers were initialised (issue_first); the rest are refills
+  // barriers were initialised; the rest are refills
   bool ok = true;
 #pragma unroll 1
   for (int pc = 0; pc < n_pc; ++pc) {
@@ -481,33 +477,131 @@ __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int l
     }
     const float sc = transpose_reduce8x16(part, hl);
     const int r = row0 + (hl >> 1);
-    if (kPool == 1) {
-      if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
-    } else {
-      // the 8 rows of a half-warp are two blocks' 4 windows: the max of the
-      // first three windows of each group of four (lanes hl^2, hl^4 hold
-      // rows r^1, r^2)
-      float m = (r < rows && (r & 3) != 3) ? sc : -INFINITY;
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      const int kb = (pc * kPieceRows + row0) / 4 + (hl >> 3);
-      if ((hl & 7) == 0 && kb * kPool < n) keys[kb] = orderable_key(m);
-    }
+    if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
     __syncthreads();  // piece consumed by every half-warp
     if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
   }
   return ok;
 }
 
+// Window grid (32-token windows at stride 16, four per 64-token block):
+// block j scores as the best of the three windows inside it, 4j, 4j+1 and
+// 4j+2; window 4j+3 straddles two blocks and is never read.  A piece is a
+// TMA box of kWBlk blocks x those 3 windows x 128 dims, from a 4-D map
+// (dims, window in block, block, (b, g)) whose block extent stops at NW / 4,
+// where every block's three windows lie inside the tensor; its row r is
+// window r % 3 of block r / 3.  The one or two blocks past the map are
+// scored with plain loads (score_tail_windows).
+constexpr int kWBlk = 40;
+constexpr int kWPieceBytes = kWBlk * 3 * kD * 2;  // 30 KB in a 32 KB ring slot
+
+__device__ __forceinline__ void issue_wpiece(const CUtensorMap *map, int blk0, int pc, int pg,
+                                             uint8_t *ring, uint64_t *bars) {
+  uint64_t *bar = &bars[pc % kRing];
+  mbar_arrive_expect_tx(bar, (uint32_t)kWPieceBytes);
+  tc::tma_load_4d(ring + (pc % kRing) * kPieceBytes, map, 0, 0, blk0 + pc * kWBlk, pg, bar);
+}
+
+// keys[e] for blocks lo + e, e < m; windows at or past wlimit do not exist for
+// this sequence and score -inf.  wsc: 128 floats of shared memory.
+__device__ bool score_windows(const CUtensorMap *map, const float *fs, int nf, int lo, int m,
+                              int wlimit, int pg, uint32_t *keys, float *wsc, uint8_t *ring,
+                              uint64_t *bars) {
+  const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
+  const int n_pc = (m + kWBlk - 1) / kWBlk;
+  bool ok = true;
+#pragma unroll 1
+  for (int pc = 0; pc < n_pc; ++pc) {
+    const bool landed = mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1));
+    if (__syncthreads_or(!landed)) {
+      ok = false;
+      if (threadIdx.x == 0)
+        for (int q = pc; q < min(n_pc, pc + kRing); ++q)
+          (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
+      __syncthreads();
+      break;
+    }
+    const int nblk = min(kWBlk, m - pc * kWBlk);
+    const int rows = 3 * nblk;
+    const uint8_t *piece = ring + (pc % kRing) * kPieceBytes;
+    const int row0 = hw * 8;
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = row0 + u < rows ? *reinterpret_cast<const uint4 *>(piece + (row0 + u) * (kD * 2) + hl * 16)
+                             : make_uint4(0, 0, 0, 0);
+    float part[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) part[u] = 0.f;
+#pragma unroll 1
+    for (int f = 0; f < nf; ++f) {
+      float fv[8];
+      const float4 a = *reinterpret_cast<const float4 *>(fs + f * kD + hl * 8);
+      const float4 b = *reinterpret_cast<const float4 *>(fs + f * kD + hl * 8 + 4);
+      fv[0] = a.x; fv[1] = a.y; fv[2] = a.z; fv[3] = a.w;
+      fv[4] = b.x; fv[5] = b.y; fv[6] = b.z; fv[7] = b.w;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) part[u] += dot8(fv, v[u]);
+    }
+    const float sc = transpose_reduce8x16(part, hl);
+    const int r = row0 + (hl >> 1);  // 0..127
+    if ((hl & 1) == 0) {
+      const int w = 4 * (lo + pc * kWBlk + r / 3) + r % 3;  // its window
+      wsc[r] = (r < rows && w < wlimit) ? sc : -INFINITY;
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < nblk) {
+      const int t = threadIdx.x;
+      keys[pc * kWBlk + t] = orderable_key(fmaxf(fmaxf(wsc[3 * t], wsc[3 * t + 1]), wsc[3 * t + 2]));
+    }
+    __syncthreads();  // piece and row scores consumed
+    if (threadIdx.x == 0 && pc + kRing < n_pc) issue_wpiece(map, lo, pc + kRing, pg, ring, bars);
+  }
+  return ok;
+}
+
+// keys[e] for blocks lo + e, m <= e < n (past the map's block extent, at most
+// two): one warp per (block, window), plain loads of the window's key row.
+__device__ void score_tail_windows(const uint16_t *kw_bg, const float *fs, int nf, int lo, int m,
+                                   int n, int wlimit, uint32_t *keys, float *wsc) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int items = (n - m) * 3;
+  for (int it = warp; it < items; it += kSelThreads / 32) {
+    const int w = 4 * (lo + m + it / 3) + it % 3;
+    float s = -INFINITY;
+    if (w < wlimit) {  // uniform over the warp
+      const uint2 kv = *reinterpret_cast<const uint2 *>(kw_bg + (long long)w * kD + lane * 4);
+      float acc = 0.f;
+      for (int f = 0; f < nf; ++f) {
+        const float4 q = *reinterpret_cast<const float4 *>(fs + f * kD + lane * 4);
+        acc += q.x * bf16_lo(kv.x) + q.y * bf16_hi(kv.x) + q.z * bf16_lo(kv.y) + q.w * bf16_hi(kv.y);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      s = acc;
+    }
+    if (lane == 0) wsc[it] = s;
+  }
+  __syncthreads();
+  for (int e = m + (int)threadIdx.x; e < n; e += kSelThreads) {
+    const int t = e - m;
+    keys[e] = orderable_key(fmaxf(fmaxf(wsc[3 * t], wsc[3 * t + 1]), wsc[3 * t + 2]));
+  }
+  __syncthreads();
+}
+
 template <int kPool>
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
-  // dynamic shared memory: piece ring | scoring vectors (fp32) | score keys
+__global__ void __launch_bounds__(kSelThreads, 2)
+    select_kernel(const __grid_constant__ CUtensorMap mapW, SelArgs a) {
+  // dynamic shared memory, the ring aligned to 128 bytes by hand (a TMA
+  // destination): piece ring | scoring vectors (fp32) | score keys
   extern __shared__ __align__(128) uint8_t dyn_raw[];
-  uint8_t *ring = dyn_raw;
-  float *fs = reinterpret_cast<float *>(dyn_raw + kRing * kPieceBytes);
-  uint32_t *dyn = reinterpret_cast<uint32_t *>(dyn_raw + kRing * kPieceBytes + a.nf * kD * 4);
+  uint8_t *ring = dyn_raw + ((128u - (smem_addr(dyn_raw) & 127u)) & 127u);
+  float *fs = reinterpret_cast<float *>(ring + kRing * kPieceBytes);
+  uint32_t *dyn = reinterpret_cast<uint32_t *>(ring + kRing * kPieceBytes + a.nf * kD * 4);
   __shared__ __align__(8) uint64_t bars[kRing];
   __shared__ RankSmem rs;
+  __shared__ float wsc[128];  // window grid: row scores of a piece
   __shared__ int s_last;
 
   pdl_trigger();
@@ -555,11 +649,20 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
   // last ones clipped to the windows that exist
   const int row_lo = lo * kPool;
   const int n_rows = kPool == 1 ? n : max(0, min(n * kPool, rows_b - row_lo));
-  const uint16_t *kc_bg = a.kc + (b * a.G + g) * (long long)a.NB * kD;
+  const int pg = (int)(b * a.G + g);  // (sequence, group): the key tensor's problem index
+  const uint16_t *kc_bg = a.kc + (long long)pg * a.NB * kD;
+  // window grid: blocks [lo, lo + m) come by TMA, the rest by plain loads
+  const int m = kPool == 1 ? 0 : max(0, min(lo + n, a.NBf) - lo);
   if (threadIdx.x == 0) {
     for (int q = 0; q < kRing; ++q) mbar_init(&bars[q], 1);
     fence_mbar_init();
-    prime_ring(kc_bg, row_lo, n_rows, ring, bars);
+    if (kPool == 1) {
+      prime_ring(kc_bg, row_lo, n_rows, ring, bars);
+    } else if (m > 0) {  // the map exists whenever a block comes by TMA
+      tc::prefetch_map(&mapW);
+      for (int pc = 0; pc < min(kRing, (m + kWBlk - 1) / kWBlk); ++pc)
+        issue_wpiece(&mapW, lo, pc, pg, ring, bars);
+    }
   }
   // Forecast vector(s) of this problem -> fp32 in shared memory
   const uint16_t *f = a.F + (bi * a.G + g) * (long long)a.nf * kD;
@@ -571,7 +674,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(SelArgs a) {
     for (int e = threadIdx.x; e < n; e += kSelThreads) keys[e] = orderable_key(-INFINITY);
     __syncthreads();
   }
-  if (!score_rows<kPool>(kc_bg, fs, a.nf, row_lo, n_rows, keys, ring, bars)) {
+  bool ok;
+  if (kPool == 1) {
+    ok = score_rows(kc_bg, fs, a.nf, row_lo, n_rows, keys, ring, bars);
+  } else {
+    ok = score_windows(&mapW, fs, a.nf, lo, m, row_lo + n_rows, pg, keys, wsc, ring, bars);
+    if (ok && m < n) score_tail_windows(kc_bg, fs, a.nf, lo, m, n, row_lo + n_rows, keys, wsc);
+  }
+  if (!ok) {
     // a copy never landed: report an empty set rather than a wrong one
     for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
     return;
@@ -1051,13 +1161,28 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.counters = nullptr;
   a.cand_key = nullptr;
   a.old_rank = env_int("SPARDA_SELECT_BINNED") > 0 ? 1 : 0;
-  size_t smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)pl.CH * 4;
+  // window grid: key rows [B*G][NW][d] as (dims, window in block, block, (b, g)),
+  // three of every four windows, blocks up to NW / 4 (all three windows inside)
+  CUtensorMap mW{};
+  a.NBf = 0;
+  if (pool != 1) {
+    a.NBf = a.NB / 4;
+    if (a.NBf > 0) {
+      const uint64_t wdim[4] = {(uint64_t)kD, 3, (uint64_t)a.NBf, (uint64_t)p.B * p.G};
+      const uint64_t wstr[3] = {(uint64_t)kD * 2, (uint64_t)4 * kD * 2, (uint64_t)a.NB * kD * 2};
+      const uint32_t wbox[4] = {(uint32_t)kD, 3, (uint32_t)kWBlk, 1};
+      if (!tc::make_map_nd(&mW, kc, 4, wdim, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorNotSupported;
+    }
+  }
+  size_t smem = 128 + (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)pl.CH * 4;
   if (pl.n_chunks > 1) {
     char *w = static_cast<char *>(ws);
     a.counters = reinterpret_cast<uint32_t *>(w);
     w += ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
     a.cand_key = reinterpret_cast<uint32_t *>(w);
-    smem = (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)std::max(pl.CH, pl.ncand_max) * 4;
+    smem = 128 + (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 +
+           (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
   auto kern = pool == 1 ? select_kernel<1> : select_kernel<4>;
   {  // raised once per device and pooling to the largest size used; most
@@ -1075,7 +1200,7 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     }
   }
   const long long grid = pl.n_problems * pl.n_chunks;
-  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, a);
+  const cudaError_t e = launch_pdl(kern, (unsigned)grid, kSelThreads, smem, stream, mW, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -61,9 +61,11 @@ inline bool make_map_2d(CUtensorMap *map, const void *base, uint64_t row_elems, 
 
 // N-D bf16 tensor map (N <= 5): dims[0] is the contiguous dimension (elements),
 // strides_bytes[i] the byte distance between consecutive indices of dims[i+1],
-// box[i] the tile extent in dims[i]; 128-byte swizzle, zero fill outside.
+// box[i] the tile extent in dims[i]; 128-byte swizzle unless told otherwise,
+// zero fill outside.
 inline bool make_map_nd(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                        const uint64_t *strides_bytes, const uint32_t *box) {
+                        const uint64_t *strides_bytes, const uint32_t *box,
+                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
@@ -75,7 +77,7 @@ inline bool make_map_nd(CUtensorMap *map, const void *base, int rank, const uint
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), d, st,
-            bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
