@@ -1107,13 +1107,11 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
     const long long wave = 2LL * n_sm;
     const long long per = std::max<long long>(1, wave / std::max<long long>(1, pl.n_problems));
     CH = (int)(ceil_div_ll(ceil_div_ll(pl.ncand_max, per), kSelThreads) * kSelThreads);
-    // longer streams per CTA stop paying past 1024 blocks.  On the window
-    // grid (four rows per block) with per-sequence lengths, chunks stay at
-    // 256 blocks: problems of different lengths then balance better (the
-    // real models' decode step, 444 against 455 us with 1024); with one
-    // length for all, one wave of 1024-block chunks streams fastest (50.0
-    // against 56.6 us at B = 16, T = 128K)
-    CH = std::min(std::max(CH, kSelThreads), (pool > 1 && p.seq_len) ? 1024 / pool : 1024);
+    // longer streams per CTA stop paying past 1024 blocks, on both grids
+    // (the window grid reads three windows per block): one wave of
+    // 1024-block chunks beat 256- and 512-block ones at B = 16, T = 128K,
+    // with one length for all and with the real models' mixed lengths
+    CH = std::min(std::max(CH, kSelThreads), 1024);
     if (pl.n_problems >= 8LL * n_sm) CH = kMaxCand;
   }
   if (CH >= pl.ncand_max) CH = std::min(kMaxCand, (int)ceil_div_ll(pl.ncand_max, kSelThreads) * kSelThreads);
