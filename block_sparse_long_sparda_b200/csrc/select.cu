@@ -16,20 +16,21 @@
 //
 // Design (B200): the decode selection is a streaming read of Kc (256 B per
 // block per group) with a tiny amount of math, so it is HBM bound.  A problem
-// (one query token of one group of one sequence) is split into chunks of CH
-// candidate blocks, one thread block each, so thousands of CTAs stream Kc at
-// once.  Inside a CTA each half-warp scores 8 blocks per step: lane l loads
-// dims [8l, 8l+8) of the 8 rows (8 x 16-byte loads in flight), multiplies by
-// the Forecast slice, and a butterfly transpose-reduce (8 shuffles for 8
-// rows) leaves the full score of each row in a pair of lanes.  Scores become
-// orderable uint32 keys.  A chunk CTA only streams and scores, writing its
-// keys to the workspace, so CTAs are short and many are in flight.  The
-// chunks of a problem meet through an atomic ticket: the last CTA to finish
-// (no waiting) loads every key of the problem from L2, a binned search finds
-// the k-th key exactly, and a ballot-and-scan pass in block order keeps
-// everything above it plus the lowest-index ties -- results come out sorted
-// by block id and ties go to the lower id -- and writes init U top-k U local.
-// No CTA ever waits for another.
+// (one query token of one group of one sequence) is split into chunks of up
+// to 1024 candidate blocks, as many as fill one wave of two CTAs per SM.  A
+// CTA streams its rows into a three-slot shared-memory ring: bulk async
+// copies of 128 contiguous rows on the block grid; on the window grid, TMA
+// boxes that bring only the three windows inside each of 40 blocks.  Each
+// half-warp scores 8 rows per piece: lane l holds dims [8l, 8l+8) of the 8
+// rows, multiplies by the Forecast slice, and a butterfly transpose-reduce
+// (8 shuffles for 8 rows) leaves the full score of each row in a pair of
+// lanes.  Scores become orderable uint32 keys.  The chunks of a problem meet
+// through an atomic ticket: the last CTA to finish (no waiting) loads every
+// key of the problem from L2 and finds the k-th key exactly -- a register
+// sorting network for k <= 64, binned passes otherwise -- and a
+// ballot-and-scan pass in block order keeps everything above it plus the
+// lowest-index ties, so results come out sorted by block id with ties to the
+// lower id, and writes init U top-k U local.  No CTA ever waits for another.
 #include <algorithm>
 #include <cstdlib>
 
