@@ -96,3 +96,34 @@ def test_workspace_sizes_scale_with_shapes(L):
     # the workspace of an op with no scratch is zero
     assert abi.sparda_workspace_size(abi.SPARDA_OP_COMPRESS, cfg3) == 0
     assert abi.sparda_workspace_size(abi.SPARDA_OP_PREFETCH, cfg3) == 0
+
+
+def test_head_softmax_validation_and_workspace(L):
+    """The per-head softmax selector's entry points refuse bad arguments on the
+    host, and its workspace is tickets + failure flags + per-chunk (max, sum)
+    pairs + one fp32 score per seen row and head.  Sizes without a GPU use the
+    default of 148 SMs, so the chunking is the one-wave rule: B*G = 128
+    problems -> 2 chunks of 1024 blocks each."""
+    byref = ctypes.byref
+    fake = ctypes.c_void_p(0x10000)
+    p = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
+    f = abi.lib().sparda_head_softmax_select
+    fw = abi.lib().sparda_head_softmax_select_windows
+    assert f(byref(p), fake, 4, 131072, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL   # past the end
+    assert f(byref(p), fake, 0, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL   # no heads
+    assert f(byref(p), fake, 17, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert f(byref(p), fake, 4, 131071, float("nan"), fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
+    assert f(byref(p), fake, 4, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
+    assert fw(byref(p), fake, 4, 131071, 1.0, fake, 64, 16, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert f(byref(abi.make_params(0, 32, 8, 131072, 64)), NULL, 4, 0, 1.0, NULL, NULL, NULL, 0,
+             NULL) == abi.SPARDA_OK                                                   # empty batch
+    words = 2 * 512                        # 128 tickets + 128 flags, each rounded to 256 B
+    stats = 128 * 2 * 4 * 8                # (max, sum) per problem, chunk and head
+    blocks = abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX, p, 1, 4)
+    windows = abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS, p, 1, 4)
+    assert blocks == words + stats + 128 * 4 * 2048 * 4
+    assert windows == words + stats + 128 * 4 * 8192 * 4
+    for op in (abi.SPARDA_OP_HEAD_SOFTMAX, abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS):
+        assert abi.sparda_workspace_size(op, p, 2, 4) == 0                          # decode only
+    small = abi.make_params(B=1, Hq=4, G=1, T=64 * 70, k=80)                    # k covers every candidate
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX, small, 1, 4) == 0
