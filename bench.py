@@ -170,28 +170,39 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
-                c = [x.strip() for x in line.split(",")]
-                if len(c) < 9:
-                    continue
-                try:
-                    sm.append(float(c[1]))
-                    smax = float(c[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, c[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
+            out = summarize_clock_samples(f)
         os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return out
 
 
-def measured_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def summarize_clock_samples(lines) -> dict:
+    """nvidia-smi CSV rows (index, clocks.sm, clocks.max.sm, power.draw, the
+    active-reasons mask, then hw_slowdown, hw_thermal_slowdown,
+    sw_thermal_slowdown, sw_power_cap as "Active" / "Not Active") -> the
+    median SM clock, the max clock and every reason seen active."""
+    sm, smax, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in lines:
+        c = [x.strip() for x in line.split(",")]
+        if len(c) < 9:
+            continue
+        try:
+            sm.append(float(c[1]))
+            smax = float(c[2])
+        except ValueError:
+            continue
+        for n, v in zip(names, c[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks(path=None):
+    """The measured HBM copy bandwidth (GB/s) the driver wrote, else the
+    earlier pool measurement, with which of the two it is."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
