@@ -127,3 +127,28 @@ def test_head_softmax_validation_and_workspace(L):
         assert abi.sparda_workspace_size(op, p, 2, 4) == 0                          # decode only
     small = abi.make_params(B=1, Hq=4, G=1, T=64 * 70, k=80)                    # k covers every candidate
     assert abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX, small, 1, 4) == 0
+
+
+def test_window_grid_validation(L):
+    """The window-grid entry points take only the 32/16 grid, check positions
+    and query ranges on the host, and want a workspace at multi-chunk sizes."""
+    byref = ctypes.byref
+    fake = ctypes.c_void_p(0x10000)
+    lib = abi.lib()
+    p = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8)
+    assert lib.sparda_compress_windows(byref(p), fake, 4096 * 128, 128, 64, 32, NULL, fake,
+                                       NULL) == abi.SPARDA_EUNSUPPORTED
+    assert lib.sparda_compress_windows(byref(p), fake, 4096 * 128, 128, 32, 16, NULL, NULL,
+                                       NULL) == abi.SPARDA_EINVAL            # no output
+    assert lib.sparda_append_windows(byref(p), 4096, fake, 4096 * 128, 64 * 128, 32, 16, NULL,
+                                     fake, NULL) == abi.SPARDA_EINVAL        # pos past the end
+    assert lib.sparda_append_windows(byref(p), 100, fake, 4096 * 128, 64 * 128, 32, 8, NULL,
+                                     fake, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert lib.sparda_forecast_select_windows(byref(p), fake, 1, 1, 4096, fake, 32, 16, fake,
+                                              NULL, 0, NULL) == abi.SPARDA_EINVAL  # query past T
+    assert lib.sparda_forecast_select_windows(byref(p), fake, 1, 1, 4095, fake, 16, 16, fake,
+                                              NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    big = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT_WINDOWS, big, 1, 1) > 0
+    assert lib.sparda_forecast_select_windows(byref(big), fake, 1, 1, 131071, fake, 32, 16, fake,
+                                              NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
