@@ -278,10 +278,11 @@ class DecodeLoop:
         w, nxt = self.w, (l + 1) % self.w.layers
         if w.windows:
             self.abi.sparda_forecast_select_windows(self.p, self.F[l], 1, 1, w.T - 1, self.kw[nxt],
-                                                    32, 16, self.idx[nxt], self.ws_sel[l])
+                                                    32, 16, self.idx[nxt], self.ws_sel[l],
+                                                    self.status)
         else:
             self.abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                            self.idx[nxt], self.ws_sel[l])
+                                            self.idx[nxt], self.ws_sel[l], self.status)
 
     def attention(self, l):
         w = self.w
@@ -361,7 +362,7 @@ class DecodeLoop:
         for l in range(L):
             nxt = (l + 1) % L
             abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                       self.idx[nxt], self.ws_sel[l])
+                                       self.idx[nxt], self.ws_sel[l], self.status)
             self.sel_ev[l].record(self.compute)
             self.side.wait_event(self.sel_ev[l])
             abi.sparda_prefetch_blocks(self.p, self.host_kv[nxt], self.idx[nxt], self.slots[nxt],
@@ -430,7 +431,7 @@ class DecodeLoop:
             self.side.wait_event(self.ev_pre[l])
             with torch.cuda.stream(self.side):
                 abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                           self.idx[nxt], self.ws_sel[l])
+                                           self.idx[nxt], self.ws_sel[l], self.status)
                 abi.sparda_cache_plan(self.p, C, self.idx[nxt], self.block_of[nxt],
                                       self.hand[nxt], self.phys[nxt], self.fetch[nxt],
                                       self.status)
@@ -938,7 +939,7 @@ class PrefillChunk:
 
     def select(self):
         self.abi.sparda_forecast_select(self.p, self.F, self.w.nq, 1, self.q0, self.kc, self.idx,
-                                        self.ws_sel)
+                                        self.ws_sel, self.status)
 
     def attention(self):
         w = self.w

@@ -49,20 +49,36 @@ class SpardaError(RuntimeError):
         self.status = status
 
 
+class sparda_tuning(ctypes.Structure):
+    _fields_ = [("select_chunk", ctypes.c_int), ("select_stream", ctypes.c_int),
+                ("select_binned", ctypes.c_int), ("attn_ctas", ctypes.c_int),
+                ("attn_stages", ctypes.c_int), ("attn_split_kv", ctypes.c_int),
+                ("prefetch_ctas", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("attn_wait_cycles", ctypes.c_longlong)]
+
+
 class sparda_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("G", ctypes.c_int),
                 ("d", ctypes.c_int), ("blk", ctypes.c_int), ("T", ctypes.c_int),
                 ("k", ctypes.c_int), ("n_init", ctypes.c_int), ("n_local", ctypes.c_int),
-                ("scale", ctypes.c_float), ("seq_len", ctypes.c_void_p)]
+                ("scale", ctypes.c_float), ("seq_len", ctypes.c_void_p),
+                ("tune", ctypes.POINTER(sparda_tuning))]
 
 
 def make_params(B, Hq, G, T, k, n_init=1, n_local=2, d=128, blk=64, scale=0.0,
-                seq_len=None) -> sparda_params:
+                seq_len=None, tune=None) -> sparda_params:
     """seq_len: optional device int32 tensor [B] of per-sequence lengths (the
-    caller keeps it alive while the params are in use)."""
-    return sparda_params(int(B), int(Hq), int(G), int(d), int(blk), int(T), int(k), int(n_init),
-                         int(n_local), float(scale),
-                         None if seq_len is None else seq_len.data_ptr())
+    caller keeps it alive while the params are in use).  tune: optional dict
+    of sparda_tuning fields (launch choices; the rest stay 0, the library's
+    own); the params keep the struct alive."""
+    p = sparda_params(int(B), int(Hq), int(G), int(d), int(blk), int(T), int(k), int(n_init),
+                      int(n_local), float(scale),
+                      None if seq_len is None else seq_len.data_ptr())
+    if tune:
+        t = sparda_tuning(**{k_: int(v) for k_, v in tune.items()})
+        p._tune_keep = t
+        p.tune = ctypes.pointer(t)
+    return p
 
 
 _lib = None
@@ -74,14 +90,16 @@ _PP = ctypes.POINTER(sparda_params)
 
 _SIGS = {
     "sparda_compress_keys": (_I, [_PP, _P, _LL, _LL, _P, _P, _P]),
-    "sparda_forecast_select": (_I, [_PP, _P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "sparda_forecast_select": (_I, [_PP, _P, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
     "sparda_append_kv": (_I, [_PP, _I, _P, _P, _P, _P, _LL, _LL, _P, _P, _P]),
     "sparda_append_windows": (_I, [_PP, _I, _P, _LL, _LL, _I, _I, _P, _P, _P]),
     "sparda_compress_windows": (_I, [_PP, _P, _LL, _LL, _I, _I, _P, _P, _P]),
-    "sparda_forecast_select_windows": (_I, [_PP, _P, _I, _I, _I, _P, _I, _I, _P, _P, _SZ, _P]),
-    "sparda_head_softmax_select": (_I, [_PP, _P, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]),
+    "sparda_forecast_select_windows": (_I, [_PP, _P, _I, _I, _I, _P, _I, _I, _P, _P, _SZ, _P,
+                                            _P]),
+    "sparda_head_softmax_select": (_I, [_PP, _P, _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P,
+                                        _P]),
     "sparda_head_softmax_select_windows": (_I, [_PP, _P, _I, _I, ctypes.c_float, _P, _I, _I, _P,
-                                                _P, _SZ, _P]),
+                                                _P, _SZ, _P, _P]),
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
@@ -175,34 +193,37 @@ def sparda_compress_windows(p, K, bg_stride, tok_stride, win, stride, kw_f32, kw
                                          _stream(stream)))
 
 
-def sparda_forecast_select_windows(p, F, nq, nf, q_start, kw, win, stride, idx, ws, stream=None):
+def sparda_forecast_select_windows(p, F, nq, nf, q_start, kw, win, stride, idx, ws,
+                                   dev_status=None, stream=None):
     _check("sparda_forecast_select_windows",
            lib().sparda_forecast_select_windows(ctypes.byref(p), _ptr(F), int(nq), int(nf),
                                                 int(q_start), _ptr(kw), int(win), int(stride),
-                                                _ptr(idx), _ptr(ws), _nbytes(ws), _stream(stream)))
+                                                _ptr(idx), _ptr(ws), _nbytes(ws), _ptr(dev_status),
+                                                _stream(stream)))
 
 
-def sparda_forecast_select(p, F, nq, nf, q_start, kc, idx, ws, stream=None):
+def sparda_forecast_select(p, F, nq, nf, q_start, kc, idx, ws, dev_status=None, stream=None):
     _check("sparda_forecast_select",
            lib().sparda_forecast_select(ctypes.byref(p), _ptr(F), int(nq), int(nf), int(q_start),
                                         _ptr(kc), _ptr(idx), _ptr(ws), _nbytes(ws),
-                                        _stream(stream)))
+                                        _ptr(dev_status), _stream(stream)))
 
 
-def sparda_head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, stream=None):
+def sparda_head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, dev_status=None,
+                               stream=None):
     _check("sparda_head_softmax_select",
            lib().sparda_head_softmax_select(ctypes.byref(p), _ptr(Q), int(nf), int(q_start),
                                             float(tau), _ptr(kc), _ptr(idx), _ptr(ws), _nbytes(ws),
-                                            _stream(stream)))
+                                            _ptr(dev_status), _stream(stream)))
 
 
 def sparda_head_softmax_select_windows(p, Q, nf, q_start, tau, kw, win, stride, idx, ws,
-                                       stream=None):
+                                       dev_status=None, stream=None):
     _check("sparda_head_softmax_select_windows",
            lib().sparda_head_softmax_select_windows(ctypes.byref(p), _ptr(Q), int(nf),
                                                     int(q_start), float(tau), _ptr(kw), int(win),
                                                     int(stride), _ptr(idx), _ptr(ws), _nbytes(ws),
-                                                    _stream(stream)))
+                                                    _ptr(dev_status), _stream(stream)))
 
 
 def sparda_prefetch_blocks(p, host_kv, idx, slots, skip_resident, n_ctas=0, dev_status=None,

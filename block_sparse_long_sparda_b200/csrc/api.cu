@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points of libsparda: argument validation on
 // the host, workspace sizing, and dispatch to the kernels.  Nothing here
 // synchronizes the device; every launch is checked with cudaGetLastError.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -15,8 +16,10 @@ namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 // shapes every entry point shares; returns a status
-int check_params(const sparda_params *p) {
+int sparda::check_params(const sparda_params *p) {
   if (!p) return SPARDA_EINVAL;
   if (p->B < 0 || p->Hq <= 0 || p->G <= 0 || p->T < 1 || p->k < 0 || p->n_init < 0 ||
       p->n_local < 0)
@@ -27,10 +30,24 @@ int check_params(const sparda_params *p) {
   if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16) return SPARDA_EUNSUPPORTED;
   if (p->k > 1024 || p->n_init > 64 || p->n_local > 64) return SPARDA_EUNSUPPORTED;
   if (p->k + p->n_init + p->n_local < 1) return SPARDA_EINVAL;
+  if (p->tune) {
+    const sparda_tuning &t = *p->tune;
+    if (t.reserved != 0 || t.select_chunk < 0 || t.attn_ctas < 0 || t.prefetch_ctas < 0 ||
+        t.attn_wait_cycles < 0)
+      return SPARDA_EINVAL;
+    if (t.attn_stages != 0 && t.attn_stages != 2 && t.attn_stages != 3 && t.attn_stages != 4 &&
+        t.attn_stages != 6)
+      return SPARDA_EINVAL;
+    if (t.attn_split_kv > 0 && t.attn_stages > 3) return SPARDA_EINVAL;  // 2 or 3 stages only
+  }
   return SPARDA_OK;
 }
 
+namespace {
+
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? SPARDA_OK : SPARDA_ECUDA; }
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
 
 // calls that do not read per-sequence lengths refuse them rather than
 // silently using T for every sequence
@@ -39,11 +56,31 @@ bool stride_ok(long long s) { return s > 0 && (s % 8) == 0; }
 
 }  // namespace
 
+namespace sparda {
+// fetched through the runtime, so the library keeps no link-time dependency
+// on libcuda
+void *current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext c = nullptr;
+  return fn(&c) == CUDA_SUCCESS ? static_cast<void *>(c) : nullptr;
+}
+}  // namespace sparda
+
 // shared by the block-grid and window-grid entry points
 namespace {
 int head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start, float tau,
                         const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
-                        sparda_stream_t stream, int pool) {
+                        int32_t *dev_status, sparda_stream_t stream, int pool) {
   if (nf < 1 || q_start < 0 || q_start >= p->T) return SPARDA_EINVAL;
   if (!(tau == tau) || tau > 3.0e38f) return SPARDA_EINVAL;  // NaN or infinite
   if (nf > 16) return SPARDA_EUNSUPPORTED;
@@ -55,7 +92,7 @@ int head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_sta
   if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
   const float t = tau > 0.f ? tau : sqrtf((float)p->d);
   return from_cuda(launch_head_softmax(*p, pl, static_cast<const uint16_t *>(Q), nf, q_start, t,
-                                       static_cast<const uint16_t *>(kc), idx, ws,
+                                       static_cast<const uint16_t *>(kc), idx, ws, dev_status,
                                        reinterpret_cast<cudaStream_t>(stream), pool));
 }
 }  // namespace
@@ -178,7 +215,7 @@ int sparda_compress_windows(const sparda_params *p, const void *K, long long bg_
 
 int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq, int nf,
                                    int q_start, const void *kw, int win, int stride,
-                                   int32_t *idx, void *ws, size_t ws_bytes,
+                                   int32_t *idx, void *ws, size_t ws_bytes, int32_t *dev_status,
                                    sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
@@ -192,31 +229,33 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
   if (!select_supported(pl)) return SPARDA_EUNSUPPORTED;
   if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
   return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), nq, nf, q_start,
-                                 static_cast<const uint16_t *>(kw), idx, ws,
+                                 static_cast<const uint16_t *>(kw), idx, ws, dev_status,
                                  reinterpret_cast<cudaStream_t>(stream), 4));
 }
 
 int sparda_head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start,
                                float tau, const void *kc, int32_t *idx, void *ws,
-                               size_t ws_bytes, sparda_stream_t stream) {
+                               size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
-  return head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, ws_bytes, stream, 1);
+  return head_softmax_select(p, Q, nf, q_start, tau, kc, idx, ws, ws_bytes, dev_status, stream,
+                             1);
 }
 
 int sparda_head_softmax_select_windows(const sparda_params *p, const void *Q, int nf,
                                        int q_start, float tau, const void *kw, int win,
                                        int stride, int32_t *idx, void *ws, size_t ws_bytes,
-                                       sparda_stream_t stream) {
+                                       int32_t *dev_status, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
   if (win != 32 || stride != 16) return SPARDA_EUNSUPPORTED;
-  return head_softmax_select(p, Q, nf, q_start, tau, kw, idx, ws, ws_bytes, stream, 4);
+  return head_softmax_select(p, Q, nf, q_start, tau, kw, idx, ws, ws_bytes, dev_status, stream,
+                             4);
 }
 
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
                            const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
-                           sparda_stream_t stream) {
+                           int32_t *dev_status, sparda_stream_t stream) {
   int st = check_params(p);
   if (st != SPARDA_OK) return st;
   if (nq < 1 || nf < 1 || q_start < 0 || (long long)q_start + nq > p->T) return SPARDA_EINVAL;
@@ -228,7 +267,7 @@ int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf
   if (!select_supported(pl)) return SPARDA_EUNSUPPORTED;
   if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
   return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), nq, nf, q_start,
-                                 static_cast<const uint16_t *>(kc), idx, ws,
+                                 static_cast<const uint16_t *>(kc), idx, ws, dev_status,
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -118,6 +118,7 @@ struct TcArgs {
   int split_kv;         // 1: a slot's K and V tiles are refilled separately (see the producer;
                         // picks the kernel instance, 2 or 3 stages)
   float scale_log2;
+  long long wait_cycles;  // bound of every wait of the pipeline, in SM clock cycles
 };
 
 // Memory index (b * nq + i) * G + g of the pair at stream position p.  With
@@ -182,15 +183,16 @@ __device__ __forceinline__ bool named_sync_or(int id, int n, bool v) {
   return r != 0;
 }
 
-// bounded wait that also gives up when another role has given up
+// bounded wait (limit in SM clock cycles) that also gives up when another
+// role has given up
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag) {
+                                              volatile int *abort_flag, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       return false;
     }
@@ -317,6 +319,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   float(*seg_l)[2][kNQ] = ctl.seg_l;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long lim = a.wait_cycles;
   const long long E = a.n_entries, NC = gridDim.x;
   const long long e0 = (long long)blockIdx.x * E / NC;
   const long long e1 = (long long)(blockIdx.x + 1) * E / NC;
@@ -412,6 +415,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   auto last_of = [&](int u) { return u == nb - 1 || s_seg[u + 1] != s_seg[u]; };
 
   int produced_k = 0, produced_v = 0;  // producer: blocks whose K / V loads were issued
+  int issued_s = 0, issued_o = 0;      // MMA issuers (lane 0): products committed
 
   if (warp == kWarpProducer) {
     // ================= producer =================
@@ -431,7 +435,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
         // one barrier per slot: all four tiles land on full_bar, and O^T
         // (the last reader) frees the slot on empty_bar
         if (u >= NSTAGE &&
-            !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), s_abort))
+            !wait_or_abort(&empty_bar[st], (uint32_t)(((u / NSTAGE) - 1) & 1), s_abort, lim))
           break;
         uint8_t *dst = stages + st * kUnitBytes;
         const int row = s_row[u];
@@ -477,7 +481,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
           continue;
         }
         if (*s_abort) break;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > lim) {
           *s_abort = 1;
           break;
         }
@@ -509,11 +513,11 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
 #pragma unroll 1
     for (int u = 0; u < nb && ok; ++u) {
       const int st = u % NSTAGE;
-      ok = wait_or_abort(&full_bar[st], (uint32_t)((u / NSTAGE) & 1), s_abort);
-      if (ok && u >= 2) ok = wait_or_abort(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1), s_abort);
+      ok = wait_or_abort(&full_bar[st], (uint32_t)((u / NSTAGE) & 1), s_abort, lim);
+      if (ok && u >= 2) ok = wait_or_abort(&p_full[u & 1], (uint32_t)(((u - 2) >> 1) & 1), s_abort, lim);
       const bool first = first_of(u);
       if (ok && first && u >= 1)  // the previous S^T must be done with the old query
-        ok = wait_or_abort(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1), s_abort);
+        ok = wait_or_abort(&s_full[(u - 1) & 1], (uint32_t)(((u - 1) >> 1) & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       if (first) {
@@ -537,6 +541,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
                        dQ + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), id1, k > 0);
         tc::mma_commit(&s_full[u & 1]);
         if (SPLIT) tc::mma_commit(&empty_bar[st]);  // the slot's K tiles are read
+        issued_s = u + 1;
       }
       __syncwarp();
       if (first) {  // the next segment's query rows, off the critical path
@@ -559,9 +564,9 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
 #pragma unroll 1
     for (int v = 0; v < nb && ok; ++v) {
       const int st = v % NSTAGE;
-      ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
-      if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), s_abort);
-      if (ok && SPLIT) ok = wait_or_abort(&fullv_bar[st], (uint32_t)((v / NSTAGE) & 1), s_abort);
+      ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort, lim);
+      if (ok && v >= 2) ok = wait_or_abort(&o_free[v & 1], (uint32_t)(((v - 2) >> 1) & 1), s_abort, lim);
+      if (ok && SPLIT) ok = wait_or_abort(&fullv_bar[st], (uint32_t)((v / NSTAGE) & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       if (lane == 0) {
@@ -574,6 +579,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
                        id2, k > 0);
         tc::mma_commit(&o_full[v & 1]);
         tc::mma_commit(SPLIT ? &emptyv_bar[st] : &empty_bar[st]);  // V tiles (or the slot) read
+        issued_o = v + 1;
       }
       __syncwarp();
     }
@@ -596,9 +602,9 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
           l_t[h] = 0.f;
         }
       }
-      if (ok) ok = wait_or_abort(&s_full[b], (uint32_t)((u >> 1) & 1), s_abort);
+      if (ok) ok = wait_or_abort(&s_full[b], (uint32_t)((u >> 1) & 1), s_abort, lim);
       // block u-2 is fully corrected: its P^T and corr slots are free
-      if (ok && u >= 2) ok = wait_or_abort(&o_free[b], (uint32_t)(((u - 2) >> 1) & 1), s_abort);
+      if (ok && u >= 2) ok = wait_or_abort(&o_free[b], (uint32_t)(((u - 2) >> 1) & 1), s_abort, lim);
       tc::fence_after_sync();
       float x[R];
       {
@@ -682,8 +688,8 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
 #pragma unroll
         for (int h = 0; h < R; ++h) acc[h] = 0.f;
       }
-      if (ok) ok = wait_or_abort(&o_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
-      if (ok) ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort);
+      if (ok) ok = wait_or_abort(&o_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort, lim);
+      if (ok) ok = wait_or_abort(&p_full[v & 1], (uint32_t)((v >> 1) & 1), s_abort, lim);
       // one vote for all four warps, so they always leave at the same barrier
       if (named_sync_or(kBarCorr, 128, !ok)) {
         ok = false;
@@ -697,12 +703,15 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       tc::fence_before_sync();
       mbar_arrive(&o_free[v & 1]);
     }
-    // all four warps agree before the last flushes (which use the barrier)
+    // all four warps agree before the last flushes (which use the barrier).
+    // After a timeout the segments not flushed yet are handed in as empty:
+    // every pair's ticket count still completes, so the last CTA to finish a
+    // pair resets its ticket and the workspace stays valid for the next call
+    // (the outputs of this one are flagged SPARDA_DEV_TIMEOUT)
     if (named_sync_or(kBarCorr, 128, !ok)) ok = false;
-    if (ok)
-      for (int f = next_flush; f < n_seg; ++f)
-        seg_flush<R>(a, pair0 + f, f == cur, E, NC, acc, seg_m[live_k & 3], &seg_l[live_k & 3][0][0],
-                     &ctl.s_last, dim);
+    for (int f = next_flush; f < n_seg; ++f)
+      seg_flush<R>(a, pair0 + f, ok && f == cur, E, NC, acc, seg_m[live_k & 3],
+                   &seg_l[live_k & 3][0][0], &ctl.s_last, dim);
     if (!ok) *s_abort = 1;
   }
 
@@ -717,6 +726,13 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
       for (int u = max(0, produced_v - NSTAGE); u < produced_v; ++u)
         (void)mbar_wait_bounded(&fullv_bar[u % NSTAGE], (uint32_t)((u / NSTAGE) & 1));
     }
+    // products still running read the ring and write TMEM: wait for the last
+    // one each issuer committed (its operands were in shared memory when it
+    // was issued, so it completes)
+    if (warp == kWarpMma && lane == 0 && issued_s > 0)
+      (void)mbar_wait_bounded(&s_full[(issued_s - 1) & 1], (uint32_t)(((issued_s - 1) >> 1) & 1));
+    if (warp == kWarpMma2 && lane == 0 && issued_o > 0)
+      (void)mbar_wait_bounded(&o_full[(issued_o - 1) & 1], (uint32_t)(((issued_o - 1) >> 1) & 1));
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -726,7 +742,7 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
 
 template <int R, int NSTAGE, bool SPLIT>
 cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs &a,
-                      long long grid_max, long long grid_min, cudaStream_t stream) {
+                      long long grid_max, long long grid_min, int forced, cudaStream_t stream) {
   constexpr size_t smem = tc_smem<NSTAGE, SPLIT>();
   auto kern = attn_tc_kernel<R, NSTAGE, SPLIT>;
   // per device, once: shared-memory attributes and how many CTAs stay
@@ -764,7 +780,6 @@ cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs
     resident[dev] = occ * n_sm;
   }
   long long grid = resident[dev];
-  const int forced = env_int("SPARDA_DECODE_CTAS");
   if (forced > 0) grid = forced;
   grid = std::max(grid, grid_min);
   grid = std::min(grid, grid_max);
@@ -781,7 +796,7 @@ DecodePlan plan_gather(const sparda_params &p, long long pairs) {
   const long long E = pairs * pl.S;
   // the workspace is sized for the largest grid a launch may use
   long long C = std::max<long long>(kGridMax, ceil_div_ll(E, kMaxEnt));
-  const int forced = env_int("SPARDA_DECODE_CTAS");
+  const int forced = tuning(p).attn_ctas;
   if (forced > 0) C = std::max<long long>(C, forced);
   if (C > E) C = E;
   if (C < 1) C = 1;
@@ -791,8 +806,11 @@ DecodePlan plan_gather(const sparda_params &p, long long pairs) {
   pl.max_cover = (int)(ceil_div_ll(pl.S, w_min) + 1);
   const size_t parts = (size_t)pairs * pl.max_cover * R;
   size_t off = ((parts * kD * 4) + 255) & ~(size_t)255;  // outputs
+  pl.ws_ml_off = off;
   off += ((parts * 8) + 255) & ~(size_t)255;              // (max, sum)
-  off += (((size_t)pairs * 4) + 255) & ~(size_t)255;      // tickets
+  pl.ws_ticket_off = off;
+  pl.ws_ticket_bytes = (size_t)pairs * 4;
+  off += (pl.ws_ticket_bytes + 255) & ~(size_t)255;       // tickets
   pl.ws_bytes = off;
   return pl;
 }
@@ -842,29 +860,28 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   a.q_start = q_start;
   a.max_cover = pl.max_cover;
   a.order_bgi = nq > 1 ? 1 : 0;
-  const int fsplit = env_int("SPARDA_SPLIT_KV");  // 1 / -1: force on / off
-  a.split_kv = fsplit != 0 ? (fsplit > 0 ? 1 : 0) : (nq > 1 ? 1 : 0);
+  const sparda_tuning &tu = tuning(p);
+  a.split_kv = tu.attn_split_kv != 0 ? (tu.attn_split_kv > 0 ? 1 : 0) : (nq > 1 ? 1 : 0);
+  a.wait_cycles = tu.attn_wait_cycles > 0 ? tu.attn_wait_cycles : kWaitCycles;
   const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
   a.scale_log2 = scale * kLog2e;
-  const size_t parts = (size_t)pairs * pl.max_cover * R;
   char *w = static_cast<char *>(ws);
   a.ws_o = reinterpret_cast<float *>(w);
-  w += ((parts * kD * 4) + 255) & ~(size_t)255;
-  a.ws_ml = reinterpret_cast<float2 *>(w);
-  w += ((parts * 8) + 255) & ~(size_t)255;
-  a.counters = reinterpret_cast<uint32_t *>(w);
+  a.ws_ml = reinterpret_cast<float2 *>(w + pl.ws_ml_off);
+  a.counters = reinterpret_cast<uint32_t *>(w + pl.ws_ticket_off);
   // ring depth: 2 x 32 KB with three resident CTAs per SM where the
   // registers allow it (up to 8 heads per group), else 3 x 32 KB with two;
-  // 4 and 6 (one CTA per SM) stay selectable through SPARDA_DECODE_STAGES
-  int stages = env_int("SPARDA_DECODE_STAGES");
+  // 4 and 6 (one CTA per SM) stay selectable through sparda_tuning
+  int stages = tu.attn_stages;
   if (stages == 0) stages = R <= 8 ? 2 : 3;
+  const int fc = tu.attn_ctas;
 #define SPARDA_LAUNCH_R(RR)                                                                    \
-  if (a.split_kv && stages <= 2) return launch_tc<RR, 2, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (a.split_kv && stages == 3) return launch_tc<RR, 3, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (stages <= 2) return launch_tc<RR, 2, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (stages == 3) return launch_tc<RR, 3, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  if (stages == 4) return launch_tc<RR, 4, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream); \
-  return launch_tc<RR, 6, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, stream);
+  if (a.split_kv && stages <= 2) return launch_tc<RR, 2, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
+  if (a.split_kv && stages == 3) return launch_tc<RR, 3, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
+  if (stages <= 2) return launch_tc<RR, 2, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
+  if (stages == 3) return launch_tc<RR, 3, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
+  if (stages == 4) return launch_tc<RR, 4, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
+  return launch_tc<RR, 6, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream);
   switch (R) {
     case 1: SPARDA_LAUNCH_R(1)
     case 2: SPARDA_LAUNCH_R(2)

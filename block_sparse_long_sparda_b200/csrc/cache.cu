@@ -194,7 +194,7 @@ cudaError_t launch_prefetch_cached(const sparda_params &p, int C, const uint16_t
   if (n_entries == 0) return cudaSuccess;
   const int NB = (p.T + kBlk - 1) / kBlk;
   if (n_ctas <= 0) {
-    const int forced = env_int("SPARDA_PREFETCH_CTAS");
+    const int forced = tuning(p).prefetch_ctas;
     n_ctas = forced > 0 ? forced : std::min(64, 16 + 2 * p.B);
   }
   n_ctas = (int)std::min<long long>(n_ctas, ceil_div_ll(n_entries, kPfTile));

@@ -86,12 +86,12 @@ __host__ __device__ inline int window_count(int T) { return T >= 32 ? (T - 32) /
 constexpr int kPrefillTensorMinQ = 64;  // query tokens from which the product pays
 size_t prefill_select_ws_bytes(const sparda_params &p, int nq, int pool = 1);
 cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
-                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream,
-                                  int pool = 1);
+                                  const uint16_t *kc, int32_t *idx, void *ws, int32_t *status,
+                                  cudaStream_t stream, int pool = 1);
 int select_supported(const SelectPlan &plan);
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const uint16_t *F,
                           int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,
-                          void *ws, cudaStream_t stream, int pool = 1);
+                          void *ws, int32_t *status, cudaStream_t stream, int pool = 1);
 
 // the original selector's per-head softmax form (decode: one query token);
 // pool as plan_select
@@ -107,7 +107,7 @@ HsmPlan plan_head_softmax(const sparda_params &p, int nf, int pool);
 int head_softmax_supported(const HsmPlan &plan, int nf);
 cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &plan, const uint16_t *Q,
                                 int nf, int q_start, float tau, const uint16_t *kc, int32_t *idx,
-                                void *ws, cudaStream_t stream, int pool);
+                                void *ws, int32_t *status, cudaStream_t stream, int pool);
 
 // ---- prefetch -------------------------------------------------------------
 cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
@@ -120,7 +120,10 @@ struct DecodePlan {
   long long n_cta;      // most thread blocks a launch may use (sizes the workspace)
   long long n_cta_min;  // fewest thread blocks the per-CTA list capacity allows
   int max_cover;    // most thread blocks any pair's entries can span
-  size_t ws_bytes;  // segment partials + tickets
+  // workspace layout, 256-byte aligned regions: segment outputs at 0, their
+  // (max, sum) at ws_ml_off, one ticket word per pair at ws_ticket_off
+  size_t ws_ml_off, ws_ticket_off, ws_ticket_bytes;
+  size_t ws_bytes;  // total
 };
 DecodePlan plan_decode(const sparda_params &p);
 DecodePlan plan_gather(const sparda_params &p, long long pairs);
@@ -156,7 +159,21 @@ cudaError_t launch_attn_prefill(const sparda_params &p, const uint16_t *Q, int n
                                 long long tok_stride, const int32_t *idx, uint16_t *O, void *ws,
                                 size_t ws_bytes, int32_t *dev_status, cudaStream_t stream);
 
-// environment overrides used for tuning sweeps (0 when unset)
-int env_int(const char *name);
+// The CUDA context current on this thread (null if none could be had).  A
+// device reset or a new primary context reloads the library's module, which
+// gives kernel attributes and device symbols new values, so host-side caches
+// of them are keyed on the context as well as the device.
+void *current_context();
+
+// the rules every entry point applies to its sparda_params (shapes, this
+// version's limits, the tuning fields); returns a status
+int check_params(const sparda_params *p);
+
+// the caller's launch choices (sparda_params::tune), or all zero: the
+// library's own
+inline const sparda_tuning &tuning(const sparda_params &p) {
+  static const sparda_tuning kNone = {};
+  return p.tune ? *p.tune : kNone;
+}
 
 }  // namespace sparda

@@ -19,9 +19,10 @@
 //    race on it and must not be issued;
 //  - the array keeps the previous call's contents, so each call clears the
 //    ticket words that must start at zero before its kernel runs;
-//  - the first call on a device resolves the array's device address
-//    (cudaGetSymbolAddress, with that device current); make that first call
-//    before any stream capture.
+//  - the first call in a CUDA context (per device, and again after a device
+//    reset or a new primary context, which reload the module and move the
+//    array) resolves the array's device address with cudaGetSymbolAddress,
+//    that device current; make that first call before any stream capture.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -36,26 +37,35 @@ static __device__ __align__(256) unsigned char g_decode_scratch[SPARDA_NOALLOC_S
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_lock;
-void *g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchAddr {
+  void *ctx;   // the context the address was resolved in
+  void *ptr;   // the array's device address there
+};
+ScratchAddr g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (resolved once
-// per device).  In host code the array's name only stands in for it.
+// Device address of the scratch array in the current context (resolved once
+// per device and context).  In host code the array's name only stands in for
+// it.
 int scratch_for_current_device(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     (void)cudaGetLastError();
     return SPARDA_ECUDA;
   }
+  void *ctx = sparda::current_context();
   std::lock_guard<std::mutex> guard(g_setup_lock);
-  if (!g_scratch_ptr[dev]) {
+  ScratchAddr &e = g_scratch[dev];
+  if (!e.ptr || !ctx || e.ctx != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
       (void)cudaGetLastError();
+      e = ScratchAddr{};
       return SPARDA_ECUDA;
     }
-    g_scratch_ptr[dev] = p;
+    // cudaGetSymbolAddress makes the primary context current if none was
+    e = ScratchAddr{ctx ? ctx : sparda::current_context(), p};
   }
-  *out = g_scratch_ptr[dev];
+  *out = e.ptr;
   return SPARDA_OK;
 }
 
@@ -68,15 +78,8 @@ extern "C" int sparda_sparse_attn_decode_noalloc(const sparda_params *p, const v
                                                  sparda_stream_t stream) {
   using namespace sparda;
   // the same argument rules as sparda_sparse_attn_decode
-  if (!p) return SPARDA_EINVAL;
-  if (p->B < 0 || p->Hq <= 0 || p->G <= 0 || p->T < 1 || p->k < 0 || p->n_init < 0 ||
-      p->n_local < 0 || p->Hq % p->G != 0)
-    return SPARDA_EINVAL;
-  if (p->d != kD || p->blk != kBlk) return SPARDA_EUNSUPPORTED;
-  const int r = p->Hq / p->G;
-  if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16) return SPARDA_EUNSUPPORTED;
-  if (p->k > 1024 || p->n_init > 64 || p->n_local > 64) return SPARDA_EUNSUPPORTED;
-  if (p->k + p->n_init + p->n_local < 1) return SPARDA_EINVAL;
+  const int pst = check_params(p);
+  if (pst != SPARDA_OK) return pst;
   if (addr_mode != SPARDA_ADDR_LOGICAL && addr_mode != SPARDA_ADDR_SLOT) return SPARDA_EINVAL;
   if (p->B == 0) return SPARDA_OK;
   if (!Q || !K || !V || !idx || !O) return SPARDA_EINVAL;
@@ -94,12 +97,10 @@ extern "C" int sparda_sparse_attn_decode_noalloc(const sparda_params *p, const v
   const int st = scratch_for_current_device(&scratch);
   if (st != SPARDA_OK) return st;
 
-  // the ticket words (last region of the scratch) must start at zero
-  const size_t pairs = (size_t)p->B * p->G;
-  const size_t parts = pairs * pl.max_cover * r;
-  const size_t tickets = (((parts * kD * 4) + 255) & ~(size_t)255) + (((parts * 8) + 255) & ~(size_t)255);
+  // the ticket words (where the plan puts them) must start at zero
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(static_cast<char *>(scratch) + tickets, 0, pairs * 4, s) != cudaSuccess) {
+  if (cudaMemsetAsync(static_cast<char *>(scratch) + pl.ws_ticket_off, 0, pl.ws_ticket_bytes, s) !=
+      cudaSuccess) {
     (void)cudaGetLastError();
     return SPARDA_ECUDA;
   }

@@ -82,7 +82,7 @@ cudaError_t launch_prefetch(const sparda_params &p, const uint16_t *host_kv_dev,
   const int NB = (p.T + kBlk - 1) / kBlk;
   const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
   if (n_ctas <= 0) {
-    const int forced = env_int("SPARDA_PREFETCH_CTAS");
+    const int forced = tuning(p).prefetch_ctas;
     // more sequences -> more concurrent host reads; bounded so the compute
     // stream keeps most SMs
     n_ctas = forced > 0 ? forced : std::min(64, 16 + 2 * p.B);

@@ -52,7 +52,9 @@ struct SelArgs {
   const uint16_t *kc;
   int32_t *idx;
   uint32_t *counters;   // one ticket per problem (multi-chunk only)
+  uint32_t *failed;     // one flag per problem: a chunk's copy never landed (multi-chunk only)
   uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
+  int32_t *status;      // optional device status word
   int nq, G, nf, NB, k, n_init, n_local, q_start, S, T;
   int CH, n_chunks, cap;
   int NBf;       // window grid: blocks the key map covers (all three inner windows present)
@@ -603,7 +605,7 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   __shared__ __align__(8) uint64_t bars[kRing];
   __shared__ RankSmem rs;
   __shared__ float wsc[128];  // window grid: row scores of a piece
-  __shared__ int s_last;
+  __shared__ int s_last, s_failed;
 
   pdl_trigger();
   pdl_wait();
@@ -621,8 +623,10 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   if (a.seq_len) {  // per-sequence lengths: the queries are the sequence's last nq tokens
     const int len = a.seq_len[b];
     if (len < a.nq || len > a.T) {  // an invalid length: an empty set
-      if (chunk == 0)
+      if (chunk == 0) {
         for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+        if (threadIdx.x == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+      }
       if (a.n_chunks > 1) {  // keep the ticket count of the problem right
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -682,11 +686,9 @@ __global__ void __launch_bounds__(kSelThreads, 2)
     ok = score_windows(&mapW, fs, a.nf, lo, m, row_lo + n_rows, pg, keys, wsc, ring, bars);
     if (ok && m < n) score_tail_windows(kc_bg, fs, a.nf, lo, m, n, row_lo + n_rows, keys, wsc);
   }
-  if (!ok) {
-    // a copy never landed: report an empty set rather than a wrong one
-    for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
-    return;
-  }
+  // a copy that never landed: the problem's set is reported empty rather
+  // than wrong (by the last chunk, when there are several)
+  if (!ok && threadIdx.x == 0) flag_status(a.status, SPARDA_DEV_TIMEOUT);
   __syncthreads();
 
   uint32_t tau = 0;
@@ -694,6 +696,10 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   int32_t *top = out + bp.init_hi;
 
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
+    if (!ok) {
+      for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+      return;
+    }
     if (a.k <= kTopkMaxK && n <= kTopkMaxN && !a.old_rank)
       find_threshold_topk(keys, n, a.k, reinterpret_cast<uint32_t *>(ring), rs, tau, need);
     else
@@ -704,9 +710,14 @@ __global__ void __launch_bounds__(kSelThreads, 2)
     return;
   }
 
-  // ---- chunk scores -> workspace; the last chunk to finish ranks them all ----
+  // ---- chunk scores -> workspace; the last chunk to finish ranks them all.
+  // A chunk whose copy never landed still takes its ticket (so the count
+  // completes and the last chunk resets it) and raises the problem's flag ----
   uint32_t *pkeys = a.cand_key + prob * (long long)a.cap;
-  for (int e = threadIdx.x; e < n; e += kSelThreads) pkeys[chunk * a.CH + e] = keys[e];
+  if (ok)
+    for (int e = threadIdx.x; e < n; e += kSelThreads) pkeys[chunk * a.CH + e] = keys[e];
+  else if (threadIdx.x == 0)
+    a.failed[prob] = 1u;
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -716,6 +727,16 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (threadIdx.x == 0) s_failed = (int)__ldcg(a.failed + prob);
+  __syncthreads();
+  if (s_failed) {
+    for (int s2 = threadIdx.x; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+    if (threadIdx.x == 0) {
+      a.failed[prob] = 0u;
+      a.counters[prob] = 0u;
+    }
+    return;
+  }
   for (int e = threadIdx.x; e < ncand; e += kSelThreads) keys[e] = __ldcg(pkeys + e);
   __syncthreads();
   if (a.k <= kTopkMaxK && ncand <= kTopkMaxN && !a.old_rank)
@@ -750,6 +771,7 @@ constexpr int kHsmMaxHeads = 16;
 
 struct HsmArgs {
   const int32_t *seq_len;
+  int32_t *status;     // optional device status word
   const uint16_t *Q;   // [B][G][nf][d]; the keys [B][G][NR][d] come through a tensor map
   int32_t *idx;        // [B][G][S]
   uint32_t *counters;  // [problem] tickets
@@ -811,8 +833,10 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   if (a.seq_len) {  // the query is the sequence's last token
     const int len = a.seq_len[b];
     if (len < 1 || len > a.T) {  // an invalid length: an empty set (every chunk returns here)
-      if (chunk == 0)
+      if (chunk == 0) {
         for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+        if (tid == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+      }
       return;
     }
     pos = len - 1;
@@ -847,6 +871,7 @@ __global__ void __launch_bounds__(kSelThreads, 2)
   if (n_pc > 0) {
     if ((smem_addr(ring) & 1023u) != 0u) {  // cannot happen with the sizes launched
       ok = false;
+      if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
     } else {
       if (tid == 0) {
         for (int q = 0; q < kRing + 2; ++q) mbar_init(&bars[q], 1);
@@ -930,6 +955,7 @@ __global__ void __launch_bounds__(kSelThreads, 2)
       if (bad) {
         ok = false;
         if (tid == 0) {  // let copies and products in flight finish (bounded) before release
+          flag_status(a.status, SPARDA_DEV_TIMEOUT);
           for (int q = pc; q < n_loaded; ++q)
             (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
           if (n_issued > 0)
@@ -1060,11 +1086,6 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 
 }  // namespace
 
-int env_int(const char *name) {
-  const char *s = getenv(name);
-  return s ? atoi(s) : 0;
-}
-
 // The plan depends on the shapes only (not on where the query chunk sits), so
 // the workspace size is known before the call: chunking is sized for a query
 // at the end of the sequence, the most candidates any query can have.
@@ -1079,7 +1100,7 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
   pl.tensor_scores = 0;
   pl.ws_bytes = 0;
   if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
-  if (nf == 1 && nq >= kPrefillTensorMinQ && env_int("SPARDA_SELECT_STREAM") == 0) {
+  if (nf == 1 && nq >= kPrefillTensorMinQ && tuning(p).select_stream == 0) {
     // a chunk of query tokens: the scores are a dense product per (sequence,
     // group), computed on the tensor cores and kept in the workspace
     pl.tensor_scores = 1;
@@ -1087,7 +1108,7 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
     return pl;
   }
 
-  const int forced = env_int("SPARDA_SELECT_CHUNK");
+  const int forced = tuning(p).select_chunk;
   int CH;
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
@@ -1120,7 +1141,7 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
   pl.n_chunks = (int)ceil_div_ll(pl.ncand_max, CH);
   if (pl.n_chunks > 1) {
     pl.kc = pl.ncand_max;  // every candidate's key is kept for the final rank
-    size_t off = ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;      // counters
+    size_t off = 2 * (((size_t)pl.n_problems * 4 + 255) & ~(size_t)255);  // tickets, flags
     off += (((size_t)pl.n_problems * pl.n_chunks * CH * 4) + 255) & ~(size_t)255;  // keys
     pl.ws_bytes = off;
   }
@@ -1136,10 +1157,13 @@ int select_supported(const SelectPlan &pl) {
 
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const uint16_t *F, int nq,
                           int nf, int q_start, const uint16_t *kc, int32_t *idx, void *ws,
-                          cudaStream_t stream, int pool) {
+                          int32_t *status, cudaStream_t stream, int pool) {
   if (pl.n_problems == 0) return cudaSuccess;
-  if (pl.tensor_scores) return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, stream, pool);
+  if (pl.tensor_scores)
+    return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, status, stream, pool);
   SelArgs a;
+  a.status = status;
+  a.failed = nullptr;
   a.seq_len = p.seq_len;
   a.T = p.T;
   a.F = F;
@@ -1159,7 +1183,7 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.cap = pl.n_chunks * pl.CH;  // key slots per problem in the workspace
   a.counters = nullptr;
   a.cand_key = nullptr;
-  a.old_rank = env_int("SPARDA_SELECT_BINNED") > 0 ? 1 : 0;
+  a.old_rank = tuning(p).select_binned != 0 ? 1 : 0;
   // window grid: key rows [B*G][NW][d] as (dims, window in block, block, (b, g)),
   // three of every four windows, blocks up to NW / 4 (all three windows inside)
   CUtensorMap mW{};
@@ -1177,9 +1201,10 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   size_t smem = 128 + (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 + (size_t)pl.CH * 4;
   if (pl.n_chunks > 1) {
     char *w = static_cast<char *>(ws);
+    const size_t words = ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
     a.counters = reinterpret_cast<uint32_t *>(w);
-    w += ((size_t)pl.n_problems * 4 + 255) & ~(size_t)255;
-    a.cand_key = reinterpret_cast<uint32_t *>(w);
+    a.failed = reinterpret_cast<uint32_t *>(w + words);
+    a.cand_key = reinterpret_cast<uint32_t *>(w + 2 * words);
     smem = 128 + (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 +
            (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
@@ -1216,7 +1241,7 @@ HsmPlan plan_head_softmax(const sparda_params &p, int nf, int pool) {
   pl.rows_cap = 0;
   pl.ws_bytes = 0;
   if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
-  const int forced = env_int("SPARDA_SELECT_CHUNK");
+  const int forced = tuning(p).select_chunk;
   int CH;
   if (forced > 0) {
     CH = std::max(kSelThreads, (forced / kSelThreads) * kSelThreads);
@@ -1257,10 +1282,11 @@ int head_softmax_supported(const HsmPlan &pl, int nf) {
 
 cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const uint16_t *Q,
                                 int nf, int q_start, float tau, const uint16_t *kc, int32_t *idx,
-                                void *ws, cudaStream_t stream, int pool) {
+                                void *ws, int32_t *status, cudaStream_t stream, int pool) {
   if (pl.n_problems == 0) return cudaSuccess;
   HsmArgs a;
   a.seq_len = p.seq_len;
+  a.status = status;
   a.Q = Q;
   a.idx = idx;
   a.G = p.G;
@@ -1276,7 +1302,7 @@ cudaError_t launch_head_softmax(const sparda_params &p, const HsmPlan &pl, const
   a.n_chunks = pl.n_chunks;
   a.rows_cap = pl.rows_cap;
   a.inv_tau = 1.f / tau;
-  a.old_rank = env_int("SPARDA_SELECT_BINNED") > 0 ? 1 : 0;
+  a.old_rank = tuning(p).select_binned != 0 ? 1 : 0;
   a.counters = nullptr;
   a.failed = nullptr;
   a.stats = nullptr;

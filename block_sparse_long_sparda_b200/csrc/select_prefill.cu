@@ -412,6 +412,7 @@ struct RankArgs {
   int G, nq, ld, k, n_init, n_local, q_start, S;
   const int32_t *seq_len;  // optional: the chunk is each sequence's last nq tokens
   int T;
+  int32_t *status;
 };
 
 __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
@@ -430,6 +431,7 @@ __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
     const int len = a.seq_len[b];
     if (len < a.nq || len > a.T) {  // an invalid length: an empty set
       for (int s = lane; s < a.S; s += 32) a.idx[row * a.S + s] = -1;
+      if (lane == 0 && i == 0 && g == 0) flag_status(a.status, SPARDA_DEV_RANGE);
       return;
     }
     qs = len - a.nq;
@@ -518,8 +520,8 @@ size_t prefill_select_ws_bytes(const sparda_params &p, int nq, int pool) {
 }
 
 cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int nq, int q_start,
-                                  const uint16_t *kc, int32_t *idx, void *ws, cudaStream_t stream,
-                                  int pool) {
+                                  const uint16_t *kc, int32_t *idx, void *ws, int32_t *status,
+                                  cudaStream_t stream, int pool) {
   if ((long long)p.B * nq * p.G == 0) return cudaSuccess;
   const int NB = (p.T + kBlk - 1) / kBlk;
   const int ld = prefill_ld(NB, pool);
@@ -545,7 +547,7 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   }
   PScoreArgs sa;
   sa.keys = static_cast<uint32_t *>(ws);
-  sa.status = nullptr;
+  sa.status = status;
   sa.G = p.G;
   sa.nq = nq;
   sa.NB = NB;
@@ -584,6 +586,7 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   ra.S = p.k + p.n_init + p.n_local;
   ra.seq_len = p.seq_len;
   ra.T = p.T;
+  ra.status = status;
   e = launch_pdl(rank_rows_kernel, (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream,
                  ra);
   return e != cudaSuccess ? e : cudaGetLastError();

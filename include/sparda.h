@@ -16,7 +16,10 @@
  *    launch failure (cudaGetLastError after the launch; the call never
  *    synchronizes).
  *  - Calls are asynchronous on the given stream (a cudaStream_t; NULL means
- *    the legacy default stream).  The library keeps no global state; calls
+ *    the legacy default stream).  Results depend only on the arguments: the
+ *    library reads no environment variables and keeps no state between calls
+ *    beyond per-device kernel attributes it caches on first use (and the
+ *    fixed scratch array of the allocation-free entry point below).  Calls
  *    on different streams with disjoint buffers may run concurrently.
  *  - All buffers are owned by the caller.  Device buffers are plain device
  *    pointers; every pointer must be 16-byte aligned and every row stride a
@@ -72,6 +75,31 @@ enum sparda_device_status_bits {
   SPARDA_DEV_LAYOUT = 4
 };
 
+/* Optional launch choices the library otherwise makes itself, for tuning
+ * sweeps and for tests that force each kernel variant.  A NULL
+ * sparda_params.tune, or a field left 0, keeps the library's own choice; no
+ * field changes what a call computes, only how.  Workspace sizes follow the
+ * same params: size a workspace with the tune pointer the calls will use. */
+typedef struct sparda_tuning {
+  int select_chunk;   /* candidate blocks per selection thread block (rounded down
+                         to a multiple of 256, at least 256)                      */
+  int select_stream;  /* nonzero: query chunks of >= 64 tokens take the streaming
+                         selection instead of the tensor-core score tiles         */
+  int select_binned;  /* nonzero: the binned threshold search even where the
+                         sorting-network threshold applies (k <= 64, <= 2048
+                         candidates)                                             */
+  int attn_ctas;      /* attention thread blocks (kept within what the lists need
+                         and the workspace was sized for)                        */
+  int attn_stages;    /* attention ring depth: 2, 3, 4 or 6 stages of 32 KB       */
+  int attn_split_kv;  /* 1: a ring slot's K and V tiles are refilled separately,
+                         -1: together; 0: separately for prefill only            */
+  int prefetch_ctas;  /* gather thread blocks when a call passes n_ctas = 0      */
+  int reserved;       /* must be 0                                               */
+  long long attn_wait_cycles;  /* bound of every wait in the attention kernel, in
+                         SM clock cycles; 0: 2e9 (about one second).  Waits that
+                         run out end the call with SPARDA_DEV_TIMEOUT            */
+} sparda_tuning;
+
 /* Shapes shared by every call.  T is the number of tokens present in the
  * sequence (the context length); the decode query sits at position T - 1. */
 typedef struct sparda_params {
@@ -101,6 +129,9 @@ typedef struct sparda_params {
    * empty outputs (-1 sets, zero attention output) and is flagged
    * SPARDA_DEV_RANGE where a status word is given. */
   const int32_t *seq_len;
+  /* Optional host pointer: launch choices (see sparda_tuning); NULL: the
+   * library's own.  Read during the call only. */
+  const sparda_tuning *tune;
 } sparda_params;
 
 /* ops for sparda_workspace_size */
@@ -179,12 +210,17 @@ int sparda_append_kv(const sparda_params *p, int pos, const void *K_new, const v
  * Ranking: higher fp32 score first, equal scores -> lower block index.
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_SELECT, p, nq, nf)
  *       bytes; it must be zero-filled before its first use, and each call
- *       leaves its tickets at zero again (the rest is scratch).  Calls sharing
- *       one workspace must not overlap on the device.
+ *       leaves its tickets and flags at zero again, a call that timed out
+ *       included (the rest is scratch).  Calls sharing one workspace must not
+ *       overlap on the device.
+ * dev_status  optional device word: SPARDA_DEV_TIMEOUT if a copy of the keys
+ *       never landed within the bounded wait; the sets of the problems it hit
+ *       are then written as -1 throughout (never a wrong set), and the others
+ *       stay valid.  SPARDA_DEV_RANGE for an invalid per-sequence length.
  */
 int sparda_forecast_select(const sparda_params *p, const void *F, int nq, int nf, int q_start,
                            const void *kc, int32_t *idx, void *ws, size_t ws_bytes,
-                           sparda_stream_t stream);
+                           int32_t *dev_status, sparda_stream_t stream);
 
 /*
  * The window grid of the models the pages measure (f3): [p4 "One Forecast
@@ -230,12 +266,13 @@ int sparda_append_windows(const sparda_params *p, int pos, const void *K, long l
  *   grid: kw bf16 [B][G][NW][d] from sparda_compress_windows (T sets NW);
  *   a candidate block scores as the best window inside it, then the same
  *   top-k rule, tie rule and output.  ws: sparda_workspace_size(
- *   SPARDA_OP_SELECT_WINDOWS, p, nq, nf) bytes, zero-filled before first use.
+ *   SPARDA_OP_SELECT_WINDOWS, p, nq, nf) bytes, zero-filled before first use;
+ *   ws and dev_status as for sparda_forecast_select.
  */
 int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq, int nf,
                                    int q_start, const void *kw, int win, int stride,
                                    int32_t *idx, void *ws, size_t ws_bytes,
-                                   sparda_stream_t stream);
+                                   int32_t *dev_status, sparda_stream_t stream);
 
 /*
  * sparda_head_softmax_select -- the original selector in its per-head softmax
@@ -263,12 +300,18 @@ int sparda_forecast_select_windows(const sparda_params *p, const void *F, int nq
  * per-sequence lengths the sequence's last token (q_start is checked only).
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_HEAD_SOFTMAX, p,
  *       1, nf) bytes, zero-filled before its first use; each call leaves its
- *       tickets and flags at zero again (the rest is scratch).  Calls sharing
- *       one workspace must not overlap on the device.
+ *       tickets and flags at zero again, a call that timed out included (the
+ *       rest is scratch).  Calls sharing one workspace must not overlap on the
+ *       device.
+ * dev_status  optional device word: SPARDA_DEV_TIMEOUT when a copy or a
+ *       product never completed within the bounded wait (that problem's set
+ *       is written as -1 throughout), SPARDA_DEV_RANGE for an invalid
+ *       per-sequence length (also an empty set), SPARDA_DEV_LAYOUT if shared
+ *       memory was misplaced.
  */
 int sparda_head_softmax_select(const sparda_params *p, const void *Q, int nf, int q_start,
                                float tau, const void *kc, int32_t *idx, void *ws,
-                               size_t ws_bytes, sparda_stream_t stream);
+                               size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream);
 
 /*
  * sparda_head_softmax_select_windows -- the same on the window grid: kw bf16
@@ -277,12 +320,13 @@ int sparda_head_softmax_select(const sparda_params *p, const void *Q, int nf, in
  *   heaviest of the windows inside it (windows 4j, 4j+1, 4j+2; -inf for a
  *   block with none), the selector's final max-pooling
  *   [p4 "Training: distilling the selector you already have"].  Workspace op
- *   SPARDA_OP_HEAD_SOFTMAX_WINDOWS.
+ *   SPARDA_OP_HEAD_SOFTMAX_WINDOWS; ws and dev_status as for
+ *   sparda_head_softmax_select.
  */
 int sparda_head_softmax_select_windows(const sparda_params *p, const void *Q, int nf,
                                        int q_start, float tau, const void *kw, int win,
                                        int stride, int32_t *idx, void *ws, size_t ws_bytes,
-                                       sparda_stream_t stream);
+                                       int32_t *dev_status, sparda_stream_t stream);
 
 /*
  * sparda_prefetch_blocks -- gather the selected K/V blocks of one layer from
@@ -324,7 +368,12 @@ int sparda_prefetch_blocks(const sparda_params *p, const void *host_kv, const in
  * O     bf16 [B][Hq][d]
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_DECODE, ...)
  *       bytes, zero-filled before its first use (each call leaves its ticket
- *       words zero again); calls sharing one workspace must not overlap.
+ *       words zero again, a call that timed out included: a thread block that
+ *       gives up still hands in its ticket for every segment it owned);
+ *       calls sharing one workspace must not overlap.
+ * dev_status  SPARDA_DEV_RANGE for skipped ids; SPARDA_DEV_TIMEOUT when a
+ *       wait ran out, in which case the outputs of the call are not valid
+ *       (the workspace is, for the next call).
  */
 int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void *K,
                               const void *V, long long bg_stride, long long blk_stride,
@@ -344,7 +393,8 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
  * O     bf16 [B][nq][Hq][d]
  * ws    device workspace of sparda_workspace_size(SPARDA_OP_ATTN_PREFILL, p, nq, 0)
  *       bytes, zero-filled before its first use; calls sharing one workspace
- *       must not overlap.
+ *       must not overlap.  ws and dev_status behave as for
+ *       sparda_sparse_attn_decode (tickets restored after a timeout).
  */
 int sparda_sparse_attn_prefill(const sparda_params *p, const void *Q, int nq, int q_start,
                                const void *K, const void *V, long long bg_stride,

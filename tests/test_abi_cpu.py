@@ -62,13 +62,13 @@ def test_validation_rejects_before_launch(L):
     assert _status("sparda_compress_keys", byref(p), odd, 4096 * 128, 128, fake, NULL, NULL) == abi.SPARDA_EINVAL
     assert _status("sparda_compress_keys", byref(p), fake, 4096 * 128, 100, fake, NULL, NULL) == abi.SPARDA_EINVAL
     # select: query positions outside the sequence, too many scoring vectors
-    assert _status("sparda_forecast_select", byref(p), fake, 1, 1, 4096, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
-    assert _status("sparda_forecast_select", byref(p), fake, 0, 1, 0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
-    assert _status("sparda_forecast_select", byref(p), fake, 1, 17, 4095, fake, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert _status("sparda_forecast_select", byref(p), fake, 1, 1, 4096, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_forecast_select", byref(p), fake, 0, 1, 0, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
+    assert _status("sparda_forecast_select", byref(p), fake, 1, 17, 4095, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EUNSUPPORTED
     # a multi-chunk select without its workspace
     big = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
     assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, big, 1, 1) > 0
-    assert _status("sparda_forecast_select", byref(big), fake, 1, 1, 131071, fake, fake, NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
+    assert _status("sparda_forecast_select", byref(big), fake, 1, 1, 131071, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EWORKSPACE
     # decode attention: bad address mode, bad block stride
     assert _status("sparda_sparse_attn_decode", byref(p), fake, fake, fake, 4096 * 128, 64 * 128, fake, 7,
                    fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
@@ -109,14 +109,15 @@ def test_head_softmax_validation_and_workspace(L):
     p = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
     f = abi.lib().sparda_head_softmax_select
     fw = abi.lib().sparda_head_softmax_select_windows
-    assert f(byref(p), fake, 4, 131072, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL   # past the end
-    assert f(byref(p), fake, 0, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL   # no heads
-    assert f(byref(p), fake, 17, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
-    assert f(byref(p), fake, 4, 131071, float("nan"), fake, fake, NULL, 0, NULL) == abi.SPARDA_EINVAL
-    assert f(byref(p), fake, 4, 131071, 1.0, fake, fake, NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
-    assert fw(byref(p), fake, 4, 131071, 1.0, fake, 64, 16, fake, NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert f(byref(p), fake, 4, 131072, 1.0, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL   # past the end
+    assert f(byref(p), fake, 0, 131071, 1.0, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL   # no heads
+    assert f(byref(p), fake, 17, 131071, 1.0, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EUNSUPPORTED
+    assert f(byref(p), fake, 4, 131071, float("nan"), fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL
+    assert f(byref(p), fake, 4, 131071, 1.0, fake, fake, NULL, 0, NULL, NULL) == abi.SPARDA_EWORKSPACE
+    assert fw(byref(p), fake, 4, 131071, 1.0, fake, 64, 16, fake, NULL, 0, NULL,
+              NULL) == abi.SPARDA_EUNSUPPORTED
     assert f(byref(abi.make_params(0, 32, 8, 131072, 64)), NULL, 4, 0, 1.0, NULL, NULL, NULL, 0,
-             NULL) == abi.SPARDA_OK                                                   # empty batch
+             NULL, NULL) == abi.SPARDA_OK                                                   # empty batch
     words = 2 * 512                        # 128 tickets + 128 flags, each rounded to 256 B
     stats = 128 * 2 * 4 * 8                # (max, sum) per problem, chunk and head
     blocks = abi.sparda_workspace_size(abi.SPARDA_OP_HEAD_SOFTMAX, p, 1, 4)
@@ -145,10 +146,42 @@ def test_window_grid_validation(L):
     assert lib.sparda_append_windows(byref(p), 100, fake, 4096 * 128, 64 * 128, 32, 8, NULL,
                                      fake, NULL) == abi.SPARDA_EUNSUPPORTED
     assert lib.sparda_forecast_select_windows(byref(p), fake, 1, 1, 4096, fake, 32, 16, fake,
-                                              NULL, 0, NULL) == abi.SPARDA_EINVAL  # query past T
+                                              NULL, 0, NULL, NULL) == abi.SPARDA_EINVAL  # query past T
     assert lib.sparda_forecast_select_windows(byref(p), fake, 1, 1, 4095, fake, 16, 16, fake,
-                                              NULL, 0, NULL) == abi.SPARDA_EUNSUPPORTED
+                                              NULL, 0, NULL, NULL) == abi.SPARDA_EUNSUPPORTED
     big = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
     assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT_WINDOWS, big, 1, 1) > 0
     assert lib.sparda_forecast_select_windows(byref(big), fake, 1, 1, 131071, fake, 32, 16, fake,
-                                              NULL, 0, NULL) == abi.SPARDA_EWORKSPACE
+                                              NULL, 0, NULL, NULL) == abi.SPARDA_EWORKSPACE
+
+
+def test_tuning_fields_are_validated_and_size_the_workspace(L):
+    """Launch choices come only from sparda_params.tune: bad values are
+    refused on the host, and the workspace sizes follow the tune pointer the
+    calls will use (never the environment)."""
+    byref = ctypes.byref
+    fake = ctypes.c_void_p(0x10000)
+    for bad in ({"reserved": 1}, {"attn_stages": 5}, {"attn_stages": 4, "attn_split_kv": 1},
+                {"select_chunk": -256}, {"attn_ctas": -1}, {"prefetch_ctas": -2},
+                {"attn_wait_cycles": -1}):
+        p = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8, tune=bad)
+        assert _status("sparda_compress_keys", byref(p), fake, 4096 * 128, 128, fake, NULL,
+                       NULL) == abi.SPARDA_EINVAL, bad
+    base = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64)
+    chunked = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64, tune={"select_chunk": 768})
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, chunked, 1, 1) != \
+        abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, base, 1, 1)
+    wide = abi.make_params(B=16, Hq=32, G=8, T=131072, k=64, tune={"attn_ctas": 2000})
+    assert abi.sparda_workspace_size(abi.SPARDA_OP_ATTN_DECODE, wide) > \
+        abi.sparda_workspace_size(abi.SPARDA_OP_ATTN_DECODE, base)
+
+
+def test_library_sources_read_no_environment():
+    """No kernel choice or workspace size may depend on environment
+    variables: the library's sources never call getenv."""
+    import glob
+    import os
+    csrc = os.path.join(os.path.dirname(abi.PKG), "block_sparse_long_sparda_b200", "csrc")
+    for f in glob.glob(os.path.join(csrc, "*")):
+        with open(f) as fh:
+            assert "getenv" not in fh.read(), f

@@ -54,6 +54,8 @@ def test_decode_loop_full_size_sampled():
         picks = {(0, 0), (w.B - 1, w.G - 1)}
         while len(picks) < 3:
             picks.add((int(rng.integers(w.B)), int(rng.integers(w.G))))
+        if l == 1:  # one layer in full: every (sequence, group)
+            picks = {(b, g) for b in range(w.B) for g in range(w.G)}
         for b, g in sorted(picks):
             what = "layer %d b %d g %d" % (l, b, g)
             kv = host_bits(loop.kv[l, b, g])                    # [NB][2][64][128]
@@ -67,7 +69,8 @@ def test_decode_loop_full_size_sampled():
             kc_in = gpu_kc.reshape(1, 1, NB, d)
             ora_idx, kth, kth1 = oracle.select(F, kc_in, w.k, w.n_init, w.n_local, T - 1, blk)
             gpu_idx = loop.idx[l, b, g].cpu().numpy().reshape(1, 1, 1, -1)
-            check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what)
+            check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what, q_pos=T - 1,
+                       n_init=w.n_init, n_local=w.n_local)
             # attention of the group's heads over the GPU's set
             Q = host_bits(loop.Q[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
             flat = kv.reshape(-1)
@@ -77,6 +80,90 @@ def test_decode_loop_full_size_sampled():
             check_attention(gpu_o, ora_o, what)
     del loop
     torch.cuda.empty_cache()
+
+
+def _check_layer_against_host(loop, l, what, rows_of, pairs=None):
+    """Layer l of a host-offload step: its sets against the oracle (F_{l-1}
+    scoring Kc_l), the device copy of every set entry byte-exact against the
+    oracle's gather from the pinned host bytes, and the attention output over
+    the host blocks of the GPU's set.  rows_of(b, g) returns the device copies
+    the attention read, in list order ([S][2][64][128] bf16 bits; slot mode:
+    slot s, slot cache: slot phys[s])."""
+    w = loop.w
+    L, R, d, blk, NB, T = w.layers, w.r, w.d, w.blk, w.NB, w.T
+    idx_all = loop.idx[l].cpu().numpy()
+    kc_all = host_bits(loop.kc[l])
+    F_all = host_bits(loop.F[(l - 1) % L])
+    Q_all = host_bits(loop.Q[l])
+    O_all = host_bits(loop.O[l])
+    pairs = pairs or [(b, g) for b in range(w.B) for g in range(w.G)]
+    for b, g in pairs:
+        tag = "%s layer %d b %d g %d" % (what, l, b, g)
+        F = F_all[b, g].reshape(1, 1, 1, 1, d)
+        kc_in = kc_all[b, g].reshape(1, 1, NB, d)
+        ora_idx, kth, kth1 = oracle.select(F, kc_in, w.k, w.n_init, w.n_local, T - 1, blk)
+        gpu_idx = idx_all[b, g].reshape(1, 1, 1, -1)
+        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), tag, q_pos=T - 1,
+                   n_init=w.n_init, n_local=w.n_local)
+        host = loop.host_kv[l, b, g].view(torch.int16).numpy().view(np.uint16)  # [NB][2][64][128]
+        ids = gpu_idx.reshape(-1)
+        want = oracle.gather_blocks(host.reshape(1, 1, NB, 2, blk, d), ids.reshape(1, 1, -1),
+                                    T - 1, w.n_init, w.n_local, False)[0, 0]
+        got = rows_of(b, g)
+        for s_ in range(len(ids)):
+            if ids[s_] >= 0:
+                assert np.array_equal(got[s_], want[s_]), "%s: entry %d (block %d)" % (tag, s_, ids[s_])
+        Q = Q_all[b, g * R:(g + 1) * R].reshape(1, 1, R, d)
+        flat = host.reshape(-1)
+        ora_o = oracle.sparse_attention(Q, flat, flat[blk * d:], gpu_idx, T - 1, T, blk,
+                                        bg_stride=flat.size, blk_stride=2 * blk * d, G=1)
+        check_attention(O_all[b, g * R:(g + 1) * R].reshape(1, 1, R, d), ora_o, tag)
+
+
+def test_offload_loop_full_size():
+    """The decode loop as bench.py's e2e legs run it, at full size: the K/V
+    of all four layers in pinned host memory (32 GiB).  One cold step -- per
+    layer the next layer's blocks are selected, gathered over the host link
+    into device slots on a side stream while this layer attends from its own
+    slots -- then three steps through the device slot cache (plan, fetch of
+    the misses only, attention reading each entry from its cache slot) with
+    drifting Forecast vectors.  After each step, every (sequence, group) of
+    the layers whose sets and slots are still those the step attended over
+    (layers 1-3; layer 0's were replaced for the next step) is checked
+    against the oracle: sets, device copies byte for byte against the host
+    bytes, and outputs."""
+    import bench
+    w = bench.WORKLOAD
+    loop = bench.DecodeLoop(w, with_host=True)
+    try:
+        loop.step_e2e()
+        torch.cuda.synchronize()
+        assert int(loop.status.item()) == 0
+        for l in range(1, w.layers):
+            _check_layer_against_host(loop, l, "slots",
+                                      lambda b, g, l=l: host_bits(loop.slots[l, b, g]))
+        loop.setup_cache(2 * w.S, 0.01, 4)
+        loop.prime_cache()
+        fetched = []
+        for t in range(3):
+            loop.step_e2e_cached(t)
+            torch.cuda.synchronize()
+            assert int(loop.status.item()) == 0
+            fetched.append(int(loop.fetch[1:].sum().item()))
+            phys = torch.from_numpy(np.maximum(loop.phys.cpu().numpy(), 0)).long().cuda()
+            pairs = [(b, g) for b in range(w.B) for g in range(w.G)] if t == 2 else \
+                [(0, 0), (w.B - 1, w.G - 1), (5, 3)]
+            for l in range(1, w.layers):
+                _check_layer_against_host(
+                    loop, l, "cache step %d" % t,
+                    lambda b, g, l=l: host_bits(loop.cache[l, b, g].index_select(0, phys[l, b, g])),
+                    pairs=pairs)
+        # drifting sets: later steps fetch only a few blocks, never the whole set
+        assert fetched[-1] < 0.1 * (w.layers - 1) * w.B * w.G * w.k, fetched
+    finally:
+        loop.unregister()
+        del loop
+        torch.cuda.empty_cache()
 
 
 def test_real_model_decode_loop_full_size_sampled():
@@ -107,7 +194,8 @@ def test_real_model_decode_loop_full_size_sampled():
             gpu_idx = loop.idx[l, b, g].cpu().numpy().reshape(1, 1, 1, -1)
             assert gpu_idx.shape[-1] == 96
             check_sets(gpu_idx, ora_idx, kth, kth1,
-                       pooled_scores_f64(F, kw, (Lb + blk - 1) // blk), what)
+                       pooled_scores_f64(F, kw, (Lb + blk - 1) // blk), what, q_pos=Lb - 1,
+                       n_init=w.n_init, n_local=w.n_local)
             kv = host_bits(loop.kv[l, b, g])
             Q = host_bits(loop.Q[l, b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
             flat = kv.reshape(-1)
@@ -160,7 +248,8 @@ def test_decode_large_batch_multiwave_sampled():
         Fb = host_bits(F[b, g]).reshape(1, 1, 1, 1, d)
         ora_idx, kth, kth1 = oracle.select(Fb, gpu_kc, k, 1, 2, T - 1)
         gpu_idx = idx[b, g].cpu().numpy().reshape(1, 1, 1, -1)
-        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(Fb, gpu_kc), what)
+        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(Fb, gpu_kc), what, q_pos=T - 1,
+                   n_init=1, n_local=2)
         Qb = host_bits(Q[b, g * R:(g + 1) * R]).reshape(1, 1, R, d)
         Vb = host_bits(V[b, g]).reshape(1, 1, T, d)
         ora_o = oracle.sparse_attention(Qb, Kb, Vb, gpu_idx, T - 1, T)
@@ -203,7 +292,8 @@ def test_prefill_chunk_full_size_sampled():
         F = host_bits(pc.F[b, i, g]).reshape(1, 1, 1, 1, d)
         ora_idx, kth, kth1 = oracle.select(F, kc_in, w.k, w.n_init, w.n_local, q0 + i, blk)
         gpu_idx = pc.idx[b, i, g].cpu().numpy().reshape(1, 1, 1, -1)
-        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what)
+        check_sets(gpu_idx, ora_idx, kth, kth1, scores_f64(F, kc_in), what, q_pos=q0 + i,
+                   n_init=w.n_init, n_local=w.n_local)
         Q = host_bits(pc.Q[b, i, g * R:(g + 1) * R]).reshape(1, 1, R, d)
         ora_o = oracle.sparse_attention(Q, K, V, gpu_idx, q0 + i, T, blk)
         gpu_o = host_bits(pc.O[b, i, g * R:(g + 1) * R]).reshape(1, 1, R, d)
@@ -229,5 +319,6 @@ def test_head_softmax_full_size(windows):
                                                     c.tau, windows=windows)
     B, G, S = got.shape
     exact = check_sets(got.reshape(B, 1, G, S), ora.reshape(B, 1, G, S), kth.reshape(B, 1, G),
-                       kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), "head softmax full size")
+                       kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), "head softmax full size",
+                       q_pos=w.T - 1, n_init=w.n_init, n_local=w.n_local)
     assert exact >= B * G - 2, "only %d of %d sets bit-exact" % (exact, B * G)

@@ -11,8 +11,8 @@ import torch
 import oracle
 from block_sparse_long_sparda_b200 import abi, build
 from block_sparse_long_sparda_b200 import workloads as W
-from tests.parity import (bf16_f64, check_attention, check_compressed, check_sets, dev_bf16,
-                          host_bits, pooled_scores_f64, scores_f64)
+from tests.parity import (Guarded, bf16_f64, check_attention, check_compressed, check_sets,
+                          dev_bf16, guarded_workspace, host_bits, pooled_scores_f64, scores_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,45 +29,51 @@ def gpu_compress(K_bits, blk=64):
     p = abi.make_params(B, G, G, T, 1)
     K = dev_bf16(K_bits)
     NB = (T + blk - 1) // blk
-    kc32 = torch.empty(B, G, NB, d, dtype=torch.float32, device="cuda")
-    kc16 = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
-    abi.sparda_compress_keys(p, K, T * d, d, kc32, kc16)
-    torch.cuda.synchronize()
-    return kc32.cpu().numpy(), host_bits(kc16)
+    kc32 = Guarded((B, G, NB, d), torch.float32)
+    kc16 = Guarded((B, G, NB, d), torch.bfloat16)
+    abi.sparda_compress_keys(p, K, T * d, d, kc32.t, kc16.t)
+    return kc32.check("fp32 Kc").cpu().numpy(), host_bits(kc16.check("bf16 Kc"))
 
 
-def gpu_select(F_bits, kc_bits, k, n_init, n_local, q_start, T, Hq=None):
-    """F [B][nq][G][nf][d] bits, kc [B][G][NB][d] bits -> idx [B][nq][G][S]."""
+def gpu_select(F_bits, kc_bits, k, n_init, n_local, q_start, T, Hq=None, tune=None):
+    """F [B][nq][G][nf][d] bits, kc [B][G][NB][d] bits -> idx [B][nq][G][S].
+    tune: optional sparda_tuning fields (forces a kernel variant)."""
     B, nq, G, nf, d = F_bits.shape
-    p = abi.make_params(B, Hq or G * max(nf, 1), G, T, k, n_init, n_local)
+    p = abi.make_params(B, Hq or G * max(nf, 1), G, T, k, n_init, n_local, tune=tune)
     S = k + n_init + n_local
-    idx = torch.full((B, nq, G, S), -7, dtype=torch.int32, device="cuda")
-    ws = abi.workspace(abi.SPARDA_OP_SELECT, p, nq, nf)
-    abi.sparda_forecast_select(p, dev_bf16(F_bits), nq, nf, q_start, dev_bf16(kc_bits), idx, ws)
-    torch.cuda.synchronize()
-    out = idx.cpu().numpy()
+    idx = Guarded((B, nq, G, S), torch.int32, fill=-7)
+    ws = guarded_workspace(abi.SPARDA_OP_SELECT, p, nq, nf)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_forecast_select(p, dev_bf16(F_bits), nq, nf, q_start, dev_bf16(kc_bits), idx.t,
+                               ws and ws.t, status)
+    out = idx.check("block sets").cpu().numpy()
+    if ws is not None:
+        ws.check("select workspace")
+    assert int(status.item()) == 0, "device status %d" % int(status.item())
     assert not (out == -7).any(), "entries left unwritten"
     return out
 
 
 def gpu_decode(Q_bits, K_bits, V_bits, idx, T, k, n_init=1, n_local=2, addr_mode=0,
-               bg_stride=None, blk_stride=None, status=None):
+               bg_stride=None, blk_stride=None, status=None, tune=None):
     B, Hq, d = Q_bits.shape
     G = idx.shape[1]
-    p = abi.make_params(B, Hq, G, T, k, n_init, n_local)
+    p = abi.make_params(B, Hq, G, T, k, n_init, n_local, tune=tune)
     K = dev_bf16(K_bits)
     V = dev_bf16(V_bits) if V_bits is not None else None
     if bg_stride is None:
         bg_stride, blk_stride = K_bits.shape[2] * d, 64 * d
-    O = torch.empty(B, Hq, d, dtype=torch.bfloat16, device="cuda")
-    ws = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p)
+    O = Guarded((B, Hq, d), torch.bfloat16)
+    ws = guarded_workspace(abi.SPARDA_OP_ATTN_DECODE, p)
     didx = torch.from_numpy(np.ascontiguousarray(idx, np.int32)).cuda()
     if V is None:  # interleaved storage: V rows follow the K rows of each block
         V = K.view(-1)[64 * d:]
     abi.sparda_sparse_attn_decode(p, dev_bf16(Q_bits), K, V, bg_stride, blk_stride, didx,
-                                  addr_mode, O, ws, status)
-    torch.cuda.synchronize()
-    return host_bits(O)
+                                  addr_mode, O.t, ws and ws.t, status)
+    out = host_bits(O.check("attention output"))
+    if ws is not None:
+        ws.check("attention workspace")
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -107,10 +113,12 @@ def test_compress_strided_rows():
 # selection
 # --------------------------------------------------------------------------
 
-def _select_case(F, kc, k, n_init, n_local, q_start, T, what):
+def _select_case(F, kc, k, n_init, n_local, q_start, T, what, tune=None):
     ora, kth, kth1 = oracle.select(F, kc, k, n_init, n_local, q_start)
-    got = gpu_select(F, kc, k, n_init, n_local, q_start, T)
-    return check_sets(got, ora, kth, kth1, scores_f64(F, kc), what)
+    got = gpu_select(F, kc, k, n_init, n_local, q_start, T, tune=tune)
+    nq = F.shape[1]
+    return check_sets(got, ora, kth, kth1, scores_f64(F, kc), what,
+                      q_pos=q_start + np.arange(nq)[None, :], n_init=n_init, n_local=n_local)
 
 
 @pytest.mark.parametrize("name", ["decode_b1_t4k", "decode_b4_t32k_planted"])
@@ -130,11 +138,11 @@ def test_select_sweep_points(NB, B):
 
 
 @pytest.mark.parametrize("chunk", ["256", "512", "8192"])
-def test_select_forced_chunking(chunk, monkeypatch):
-    monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+def test_select_forced_chunking(chunk):
     x = W.sweep_inputs(3000, 2)
     F = x["F"].reshape(2, 1, 8, 1, 128)
-    _select_case(F, x["kc"], 64, 1, 2, 3000 * 64 - 1, 3000 * 64, "chunk " + chunk)
+    _select_case(F, x["kc"], 64, 1, 2, 3000 * 64 - 1, 3000 * 64, "chunk " + chunk,
+                 tune={"select_chunk": int(chunk)})
 
 
 def test_select_baseline_multihead():
@@ -146,13 +154,10 @@ def test_select_baseline_multihead():
 @pytest.mark.parametrize("k", [100, 64, 17, 1])
 @pytest.mark.parametrize("binned", [False, True])
 @pytest.mark.parametrize("chunk", ["0", "256"])
-def test_select_exact_ties_lower_index_wins(chunk, binned, k, monkeypatch):
+def test_select_exact_ties_lower_index_wins(chunk, binned, k):
     # k <= 64 over at most 2048 candidates takes the sorting-network threshold
     # unless the binned search is forced; both must give the oracle's sets
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
-    if binned:
-        monkeypatch.setenv("SPARDA_SELECT_BINNED", "1")
+    tune = {"select_chunk": int(chunk), "select_binned": int(binned)}
     rng = np.random.default_rng(3)
     NB, B, G, d = 1500, 2, 4, 128
     kc = np.zeros((B, G, NB, d), np.float32)
@@ -161,7 +166,7 @@ def test_select_exact_ties_lower_index_wins(chunk, binned, k, monkeypatch):
     F[..., 0] = 1.0
     Fb, kcb = W.f32_to_bf16_bits(F), W.f32_to_bf16_bits(kc)
     ora, _, _ = oracle.select(Fb, kcb, k, 1, 2, NB * 64 - 1)
-    got = gpu_select(Fb, kcb, k, 1, 2, NB * 64 - 1, NB * 64)
+    got = gpu_select(Fb, kcb, k, 1, 2, NB * 64 - 1, NB * 64, tune=tune)
     assert np.array_equal(got, ora)
 
 
@@ -211,19 +216,19 @@ def test_select_prefill_tensor_scores(T, nq, q_off, k):
     _select_case(F, kc, k, 1, 2, T - nq - q_off, T, "prefill tensor")
 
 
-def test_select_prefill_tensor_matches_streaming_path(monkeypatch):
+def test_select_prefill_tensor_matches_streaming_path():
     """The same chunk through both selection paths gives the same sets."""
     rng = W.rng_for(19)
     B, G, T, nq = 1, 2, 24576, 160
     kc = W.normal_bf16(rng, (B, G, T // 64, 128))
     F = W.normal_bf16(rng, (B, nq, G, 1, 128))
     a = gpu_select(F, kc, 64, 1, 2, T - nq, T)
-    monkeypatch.setenv("SPARDA_SELECT_STREAM", "1")
-    b = gpu_select(F, kc, 64, 1, 2, T - nq, T)
+    b = gpu_select(F, kc, 64, 1, 2, T - nq, T, tune={"select_stream": 1})
     ora, kth, kth1 = oracle.select(F, kc, 64, 1, 2, T - nq)
     sc = scores_f64(F, kc)
-    check_sets(a, ora, kth, kth1, sc, "tensor path")
-    check_sets(b, ora, kth, kth1, sc, "streaming path")
+    qp = T - nq + np.arange(nq)[None, :]
+    check_sets(a, ora, kth, kth1, sc, "tensor path", q_pos=qp, n_init=1, n_local=2)
+    check_sets(b, ora, kth, kth1, sc, "streaming path", q_pos=qp, n_init=1, n_local=2)
 
 
 # --------------------------------------------------------------------------
@@ -246,31 +251,35 @@ def test_compress_windows_parity(T):
         check_compressed(kw32.cpu().numpy()[:, :, :NW], host_bits(kw16)[:, :, :NW], o64, o16)
 
 
-def _select_windows_case(F, kw, T, k, n_init, n_local, q_start, what):
+def _select_windows_case(F, kw, T, k, n_init, n_local, q_start, what, tune=None):
     B, nq, G, nf, d = F.shape
-    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local)
+    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local, tune=tune)
     S = k + n_init + n_local
-    idx = torch.full((B, nq, G, S), -7, dtype=torch.int32, device="cuda")
-    ws = abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, nq, nf)
-    abi.sparda_forecast_select_windows(p, dev_bf16(F), nq, nf, q_start, dev_bf16(kw), 32, 16, idx, ws)
-    torch.cuda.synchronize()
-    got = idx.cpu().numpy()
+    idx = Guarded((B, nq, G, S), torch.int32, fill=-7)
+    ws = guarded_workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, nq, nf)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    abi.sparda_forecast_select_windows(p, dev_bf16(F), nq, nf, q_start, dev_bf16(kw), 32, 16,
+                                       idx.t, ws and ws.t, status)
+    got = idx.check("window block sets").cpu().numpy()
+    if ws is not None:
+        ws.check("window select workspace")
+    assert int(status.item()) == 0
     assert not (got == -7).any()
     ora, kth, kth1 = oracle.select_windows(F, kw, T, k, n_init, n_local, q_start)
     NB = (T + 63) // 64
-    return check_sets(got, ora, kth, kth1, pooled_scores_f64(F, kw, NB), what)
+    return check_sets(got, ora, kth, kth1, pooled_scores_f64(F, kw, NB), what,
+                      q_pos=q_start + np.arange(nq)[None, :], n_init=n_init, n_local=n_local)
 
 
 @pytest.mark.parametrize("T,k,n_local,chunk", [(8192 + 20, 16, 2, "0"), (32768, 64, 2, "256"),
                                                 (5000 + 33, 8, 0, "0"), (20000, 40, 1, "512")])
-def test_select_windows_decode(T, k, n_local, chunk, monkeypatch):
+def test_select_windows_decode(T, k, n_local, chunk):
     rng = W.rng_for(70 + T)
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
     B, G, d = 2, 3, 128
     kw = W.normal_bf16(rng, (B, G, oracle.window_count(T), d))
     F = W.normal_bf16(rng, (B, 1, G, 1, d))
-    _select_windows_case(F, kw, T, k, 1, n_local, T - 1, "windows decode")
+    _select_windows_case(F, kw, T, k, 1, n_local, T - 1, "windows decode",
+                         tune={"select_chunk": int(chunk)})
 
 
 @pytest.mark.parametrize("T,nq,q_off", [(16384 + 40, 96, 0), (40000, 200, 3000)])
@@ -301,24 +310,33 @@ def test_select_windows_compressed_from_keys():
 # --------------------------------------------------------------------------
 
 def gpu_head_softmax(Q_bits, kc_bits, T, k, n_init, n_local, q_start, tau, windows, lens=None,
-                     ws=None):
+                     ws=None, tune=None):
     """Q [B][G][nf][d] bits; kc block or window keys -> idx [B][G][S]."""
     B, G, nf, d = Q_bits.shape
     sl = None if lens is None else torch.tensor(lens, dtype=torch.int32, device="cuda")
-    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local, seq_len=sl)
+    p = abi.make_params(B, G * nf, G, T, k, n_init, n_local, seq_len=sl, tune=tune)
     S = k + n_init + n_local
-    idx = torch.full((B, G, S), -7, dtype=torch.int32, device="cuda")
+    idx = Guarded((B, G, S), torch.int32, fill=-7)
     op = abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS if windows else abi.SPARDA_OP_HEAD_SOFTMAX
+    gws = None
     if ws is None:
-        ws = abi.workspace(op, p, 1, nf)
+        gws = guarded_workspace(op, p, 1, nf)
+        ws = gws and gws.t
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     if windows:
         abi.sparda_head_softmax_select_windows(p, dev_bf16(Q_bits), nf, q_start, tau,
-                                               dev_bf16(kc_bits), 32, 16, idx, ws)
+                                               dev_bf16(kc_bits), 32, 16, idx.t, ws, status)
     else:
         abi.sparda_head_softmax_select(p, dev_bf16(Q_bits), nf, q_start, tau, dev_bf16(kc_bits),
-                                       idx, ws)
-    torch.cuda.synchronize()
-    out = idx.cpu().numpy()
+                                       idx.t, ws, status)
+    out = idx.check("head-softmax block sets").cpu().numpy()
+    if gws is not None:
+        gws.check("head-softmax workspace")
+    st = int(status.item())
+    if lens is None or all(1 <= x <= T for x in lens):
+        assert st == 0, "device status %d" % st
+    else:
+        assert abi.sparda_status_from_device(st) == abi.SPARDA_ERANGE
     assert not (out == -7).any(), "entries left unwritten"
     return out
 
@@ -330,7 +348,8 @@ def _hsm_check(got, Q, kc, T, k, n_init, n_local, q_start, tau, windows, what):
                                                     windows=windows)
     B, G, S = got.shape
     return check_sets(got.reshape(B, 1, G, S), ora.reshape(B, 1, G, S), kth.reshape(B, 1, G),
-                      kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), what)
+                      kth1.reshape(B, 1, G), wb.reshape(B, 1, G, -1), what, q_pos=q_start,
+                      n_init=n_init, n_local=n_local)
 
 
 @pytest.mark.parametrize("T,nf,k,n_local,chunk", [
@@ -338,16 +357,15 @@ def _hsm_check(got, Q, kc, T, k, n_init, n_local, q_start, tau, windows, what):
     (5000 + 33, 16, 8, 0, "0"), (32768, 2, 100, 2, "0"), (65536 + 64, 4, 63, 32, "0"),
     (12000, 1, 20, 2, "0")])
 @pytest.mark.parametrize("windows", [False, True])
-def test_head_softmax_select(T, nf, k, n_local, chunk, windows, monkeypatch):
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+def test_head_softmax_select(T, nf, k, n_local, chunk, windows):
     rng = W.rng_for(140 + T + nf, int(windows))
     B, G, d = 2, 3, 128
     NR = oracle.window_count(T) if windows else (T + 63) // 64
     kc = W.normal_bf16(rng, (B, G, NR, d))
     Q = W.normal_bf16(rng, (B, G, nf, d))
     tau = float(np.sqrt(d))
-    got = gpu_head_softmax(Q, kc, T, k, 1, n_local, T - 1, tau, windows)
+    got = gpu_head_softmax(Q, kc, T, k, 1, n_local, T - 1, tau, windows,
+                           tune={"select_chunk": int(chunk)})
     _hsm_check(got, Q, kc, T, k, 1, n_local, T - 1, tau, windows, "head softmax")
 
 
@@ -368,14 +386,11 @@ def test_head_softmax_query_inside_the_sequence_and_default_tau(windows):
 @pytest.mark.parametrize("binned", [False, True])
 @pytest.mark.parametrize("chunk", ["0", "256"])
 @pytest.mark.parametrize("windows", [False, True])
-def test_head_softmax_exact_ties_lower_index_wins(windows, chunk, binned, monkeypatch):
+def test_head_softmax_exact_ties_lower_index_wins(windows, chunk, binned):
     """Key rows drawn from six distinct rows with integer entries along the
     heads' axes: every product is exact, equal rows weigh exactly the same
     on both sides, and the lower block index must win every tie."""
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
-    if binned:
-        monkeypatch.setenv("SPARDA_SELECT_BINNED", "1")
+    tune = {"select_chunk": int(chunk), "select_binned": int(binned)}
     rng = np.random.default_rng(151)
     B, G, nf, d, T = 2, 2, 4, 128, 1500 * 64
     NR = oracle.window_count(T) if windows else T // 64
@@ -387,7 +402,7 @@ def test_head_softmax_exact_ties_lower_index_wins(windows, chunk, binned, monkey
         Qf[:, :, h, h] = 1.0
     Q = W.f32_to_bf16_bits(Qf)
     for k in (1, 17, 64, 100):
-        got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, 1.0, windows)
+        got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, 1.0, windows, tune=tune)
         ora = oracle.select_head_softmax(Q, kc, T, k, 1, 2, T - 1, 1.0, windows=windows)[0]
         assert np.array_equal(got, ora), "k=%d" % k
 
@@ -407,12 +422,11 @@ def test_head_softmax_degenerate_budgets(k, n_init, n_local, windows):
 
 @pytest.mark.parametrize("chunk", ["0", "256"])
 @pytest.mark.parametrize("windows", [False, True])
-def test_head_softmax_per_sequence_lengths(windows, chunk, monkeypatch):
+def test_head_softmax_per_sequence_lengths(windows, chunk):
     """Sequences of different lengths in one batch, one invalid: each set is
     the oracle's on that sequence alone; the invalid one is all -1.  A second
     call on the same workspace gives the same sets (tickets back at zero)."""
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
+    tune = {"select_chunk": int(chunk)}
     rng = W.rng_for(153, int(windows))
     B, G, nf, d, T, k = 5, 2, 4, 128, 20000, 16
     lens = [T, 3000 + 17, 70, 0, 9000]
@@ -421,11 +435,11 @@ def test_head_softmax_per_sequence_lengths(windows, chunk, monkeypatch):
     Q = W.normal_bf16(rng, (B, G, nf, d))
     tau = 11.0
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    p = abi.make_params(B, G * nf, G, T, k, seq_len=sl)
+    p = abi.make_params(B, G * nf, G, T, k, seq_len=sl, tune=tune)
     op = abi.SPARDA_OP_HEAD_SOFTMAX_WINDOWS if windows else abi.SPARDA_OP_HEAD_SOFTMAX
     ws = abi.workspace(op, p, 1, nf)
-    got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws)
-    again = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws)
+    got = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws, tune=tune)
+    again = gpu_head_softmax(Q, kc, T, k, 1, 2, T - 1, tau, windows, lens=lens, ws=ws, tune=tune)
     assert np.array_equal(got, again)
     for b, L in enumerate(lens):
         if L == 0:
@@ -481,11 +495,9 @@ def test_varlen_compress_leaves_blocks_past_the_end():
 
 
 @pytest.mark.parametrize("chunk", ["0", "256"])
-def test_varlen_decode_select_and_attention(chunk, monkeypatch):
+def test_varlen_decode_select_and_attention(chunk):
     """Four sequences of different lengths in one batch: each one's set and
     attention output equal the oracle run on that sequence alone."""
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
     rng = W.rng_for(101)
     B, G, R, T, d, k = 4, 2, 4, 20000, 128, 16
     lens = [T, 3000 + 17, 70, 9000]
@@ -496,7 +508,7 @@ def test_varlen_decode_select_and_attention(chunk, monkeypatch):
     NB = (T + 63) // 64
     S = k + 3
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    p = abi.make_params(B, G * R, G, T, k, seq_len=sl)
+    p = abi.make_params(B, G * R, G, T, k, seq_len=sl, tune={"select_chunk": int(chunk)})
     Kd, Vd = dev_bf16(K), dev_bf16(V)
     kc = torch.zeros(B, G, NB, d, dtype=torch.bfloat16, device="cuda")
     abi.sparda_compress_keys(p, Kd, T * d, d, None, kc)
@@ -516,7 +528,8 @@ def test_varlen_decode_select_and_attention(chunk, monkeypatch):
         Fb = F[b:b + 1]
         kcl = np.ascontiguousarray(kcb[b:b + 1, :, :(L + 63) // 64])
         ora, kth, kth1 = oracle.select(Fb, kcl, k, 1, 2, L - 1)
-        check_sets(got_idx[b:b + 1], ora, kth, kth1, scores_f64(Fb, kcl), "varlen b=%d" % b)
+        check_sets(got_idx[b:b + 1], ora, kth, kth1, scores_f64(Fb, kcl), "varlen b=%d" % b,
+                   q_pos=L - 1, n_init=1, n_local=2)
         o = oracle.sparse_attention(Q[b:b + 1].reshape(1, 1, G * R, d),
                                     np.ascontiguousarray(K[b:b + 1, :, :L]),
                                     np.ascontiguousarray(V[b:b + 1, :, :L]),
@@ -570,13 +583,11 @@ def test_varlen_prefetch_keeps_each_sequences_resident_blocks():
 
 
 @pytest.mark.parametrize("n_local,chunk", [(2, "0"), (0, "0"), (1, "512")])
-def test_varlen_window_grid(n_local, chunk, monkeypatch):
+def test_varlen_window_grid(n_local, chunk):
     """Window compression and window selection with per-sequence lengths:
     windows not complete inside a sequence are left untouched and never
     scored (with n_local = 0 the query's own partial block is a candidate
     and scores only through the windows its sequence completes)."""
-    if chunk != "0":
-        monkeypatch.setenv("SPARDA_SELECT_CHUNK", chunk)
     rng = W.rng_for(105 + n_local)
     B, G, T, d, k = 3, 2, 12000, 128, 12
     lens = [T, 5000 + 45, 1030]
@@ -584,7 +595,7 @@ def test_varlen_window_grid(n_local, chunk, monkeypatch):
     F = W.normal_bf16(rng, (B, 1, G, 1, d))
     NW = oracle.window_count(T)
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    p = abi.make_params(B, G, G, T, k, 1, n_local, seq_len=sl)
+    p = abi.make_params(B, G, G, T, k, 1, n_local, seq_len=sl, tune={"select_chunk": int(chunk)})
     kw32 = torch.full((B, G, NW, d), 7.0, dtype=torch.float32, device="cuda")
     kw16 = torch.zeros(B, G, NW, d, dtype=torch.bfloat16, device="cuda")
     abi.sparda_compress_windows(p, dev_bf16(K), T * d, d, 32, 16, kw32, kw16)
@@ -603,7 +614,7 @@ def test_varlen_window_grid(n_local, chunk, monkeypatch):
         Fb = F[b:b + 1]
         ora, kth, kth1 = oracle.select_windows(Fb, kwl, L, k, 1, n_local, L - 1)
         check_sets(got_idx[b:b + 1], ora, kth, kth1, pooled_scores_f64(Fb, kwl, (L + 63) // 64),
-                   "varlen windows b=%d" % b)
+                   "varlen windows b=%d" % b, q_pos=L - 1, n_init=1, n_local=n_local)
 
 
 @pytest.mark.parametrize("nq,pool", [(96, 1), (5, 1), (80, 4), (3, 4)])
@@ -644,7 +655,8 @@ def test_varlen_prefill_select(nq, pool):
             kb = np.ascontiguousarray(kc[b:b + 1, :, :oracle.window_count(L)])
             ora, kth, kth1 = oracle.select_windows(Fb, kb, L, k, 1, 2, L - nq)
             sc = pooled_scores_f64(Fb, kb, (L + 63) // 64)
-        check_sets(got[b:b + 1], ora, kth, kth1, sc, "varlen prefill b=%d" % b)
+        check_sets(got[b:b + 1], ora, kth, kth1, sc, "varlen prefill b=%d" % b,
+                   q_pos=L - nq + np.arange(nq)[None, :], n_init=1, n_local=2)
 
 
 def test_varlen_prefill_attention():
@@ -695,7 +707,8 @@ def test_real_model_budget(k, n_init, n_local):
     _, kcb = oracle.compress_keys(K)
     ora, kth, kth1 = oracle.select(F, kcb, k, n_init, n_local, T - 1)
     got = gpu_select(F, kcb, k, n_init, n_local, T - 1, T, Hq=G * R)
-    check_sets(got, ora, kth, kth1, scores_f64(F, kcb), "budget")
+    check_sets(got, ora, kth, kth1, scores_f64(F, kcb), "budget", q_pos=T - 1, n_init=n_init,
+               n_local=n_local)
     idx = got[:, 0]
     S = k + n_init + n_local
     assert idx.shape[-1] == S and (idx >= 0).all()
@@ -823,11 +836,10 @@ def test_prefetch_parity(skip_resident):
     idx = idx[:, 0]
     p = abi.make_params(B, G * 4, G, T, k)
     hkv = _pinned_bf16(host)
-    slots = torch.zeros(B, G, S, 2, 64, d, dtype=torch.bfloat16, device="cuda")
-    abi.sparda_prefetch_blocks(p, hkv, torch.from_numpy(idx).cuda(), slots, skip_resident)
-    torch.cuda.synchronize()
+    slots = Guarded((B, G, S, 2, 64, d), torch.bfloat16, fill=0)
+    abi.sparda_prefetch_blocks(p, hkv, torch.from_numpy(idx).cuda(), slots.t, skip_resident)
     ora = oracle.gather_blocks(host, idx, T - 1, 1, 2, skip_resident)
-    assert np.array_equal(host_bits(slots), ora)
+    assert np.array_equal(host_bits(slots.check("slots")), ora)
 
 
 def test_prefetch_flags_out_of_range_and_rejects_pageable_memory():
@@ -1124,12 +1136,14 @@ def test_cached_prefetch_and_attention_over_steps(R):
     kc = W.normal_bf16(rng, (B, G, NB, d))
     p = abi.make_params(B, G * R, G, T, k)
     hkv = _pinned_bf16(host)
-    cache = torch.zeros(B, G, C, 2, 64, d, dtype=torch.bfloat16, device="cuda")
-    block_of = torch.full((B, G, C), -1, dtype=torch.int32, device="cuda")
-    hand = torch.zeros(B, G, dtype=torch.int32, device="cuda")
-    phys = torch.empty(B, G, S, dtype=torch.int32, device="cuda")
-    fetch = torch.empty_like(phys)
-    ws = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, p)
+    gcache = Guarded((B, G, C, 2, 64, d), torch.bfloat16, fill=0)
+    gblock_of = Guarded((B, G, C), torch.int32, fill=-1)
+    ghand = Guarded((B, G), torch.int32, fill=0)
+    gphys = Guarded((B, G, S), torch.int32, fill=0)
+    gfetch = Guarded((B, G, S), torch.int32, fill=0)
+    cache, block_of, hand, phys, fetch = gcache.t, gblock_of.t, ghand.t, gphys.t, gfetch.t
+    gws = guarded_workspace(abi.SPARDA_OP_ATTN_DECODE, p)
+    ws = gws.t
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     o_cache = np.zeros((B, G, C, 2, 64, d), np.uint16)
     o_blk, o_hand = np.full((B, G, C), -1, np.int32), np.zeros((B, G), np.int32)
@@ -1144,9 +1158,12 @@ def test_cached_prefetch_and_attention_over_steps(R):
         abi.sparda_cache_plan(p, C, didx, block_of, hand, phys, fetch, status)
         abi.sparda_prefetch_cached(p, C, hkv, didx, phys, fetch, cache, 0, status)
         Q = W.normal_bf16(rng, (B, G * R, d))
-        O = torch.empty(B, G * R, d, dtype=torch.bfloat16, device="cuda")
+        gO = Guarded((B, G * R, d), torch.bfloat16)
+        O = gO.t
         abi.sparda_sparse_attn_decode_cached(p, C, dev_bf16(Q), cache, didx, phys, O, ws, status)
-        torch.cuda.synchronize()
+        for gb, what in ((gcache, "cache"), (gblock_of, "block_of"), (ghand, "hand"),
+                         (gphys, "phys"), (gfetch, "fetch"), (gws, "workspace"), (gO, "O")):
+            gb.check(what)
         assert int(status.item()) == 0
         o_phys, o_fetch, o_blk, o_hand = oracle.cache_plan(idx, o_blk, o_hand, NB)
         assert np.array_equal(phys.cpu().numpy(), o_phys)
@@ -1226,21 +1243,23 @@ def test_prefill_attention_parity(T, nq, R):
     idx, _, _ = oracle.select(F, kcb, k, 1, 2, q_start)
     ora = oracle.sparse_attention(Q, K, V, idx, q_start, T)
     p = abi.make_params(B, Hq, G, T, k)
-    O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device="cuda")
-    ws = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
+    O = Guarded((B, nq, Hq, d), torch.bfloat16)
+    ws = guarded_workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
     abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, q_start, dev_bf16(K), dev_bf16(V), T * d, d,
-                                   torch.from_numpy(idx).cuda(), O, ws)
-    torch.cuda.synchronize()
-    check_attention(host_bits(O), ora, "prefill T=%d nq=%d" % (T, nq))
+                                   torch.from_numpy(idx).cuda(), O.t, ws.t, status)
+    ws.check("prefill workspace")
+    assert int(status.item()) == 0
+    check_attention(host_bits(O.check("prefill output")), ora, "prefill T=%d nq=%d" % (T, nq))
 
 
 @pytest.mark.parametrize("split", ["1", "-1"])
 @pytest.mark.parametrize("nq,R", [(1, 4), (1, 16), (96, 4)])
-def test_attention_both_slot_protocols(split, nq, R, monkeypatch):
+def test_attention_both_slot_protocols(split, nq, R):
     """The attention kernel has two ring protocols: one barrier per slot
     (the default for decode) and K and V tiles refilled separately (the
     default for prefill).  Each is forced on the other workload too."""
-    monkeypatch.setenv("SPARDA_SPLIT_KV", split)
+    tune = {"attn_split_kv": int(split)}
     rng = W.rng_for(41, nq * 100 + R)
     B, G, d, k, T = 2, 2, 128, 12, 6000 + 21
     Hq = G * R
@@ -1253,10 +1272,10 @@ def test_attention_both_slot_protocols(split, nq, R, monkeypatch):
     idx, _, _ = oracle.select(F, kcb, k, 1, 2, q_start)
     ora = oracle.sparse_attention(Q, K, V, idx, q_start, T)
     if nq == 1:
-        got = gpu_decode(Q.reshape(B, Hq, d), K, V, idx[:, 0], T, k)
+        got = gpu_decode(Q.reshape(B, Hq, d), K, V, idx[:, 0], T, k, tune=tune)
         check_attention(got.reshape(B, 1, Hq, d), ora, "decode split=%s R=%d" % (split, R))
     else:
-        p = abi.make_params(B, Hq, G, T, k)
+        p = abi.make_params(B, Hq, G, T, k, tune=tune)
         O = torch.empty(B, nq, Hq, d, dtype=torch.bfloat16, device="cuda")
         ws = abi.workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
         abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, q_start, dev_bf16(K), dev_bf16(V), T * d,
