@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--impl", default="sparda", choices=["sparda", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-offload e2e leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="leave the prefill-chunk and selection-sweep summaries out of the line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bound on the oracle's CPU-baseline sample")
     ap.add_argument("--prefill", action="store_true",
@@ -209,6 +211,18 @@ def measured_peaks(path=None):
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def measured_bf16_peaks(path=None):
+    """(burst, sustained) dense bf16 TFLOP/s: the driver's measurement, else
+    the earlier pool measurement, with which of the two it is."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
 
 
 # --------------------------------------------------------------------------
@@ -544,47 +558,125 @@ def time_steps(fn, steps, world):
 # CPU baseline: the oracle, as it stands, on a bounded sample
 # --------------------------------------------------------------------------
 
-def oracle_baseline(loop: DecodeLoop, seconds: float):
-    """Time the fp64 oracle's select + attention for the same 4-layer loop on a
-    sample of the sequences (the compressed keys it scores are pooled by the
-    oracle itself from the same K/V bytes, outside the timed region)."""
+class OracleDecodeSample:
+    """The decode loop's arithmetic on the fp64 oracle, for every sequence of
+    the batch: per layer, the oracle's Forecast selection of the next layer's
+    blocks for all B x G (sequence, group) problems, and its sparse attention
+    of all B x Hq heads over the layer's current sets.  Inputs are given as
+    host arrays: the compressed keys of every layer [L][B][G][NB][d], the
+    Forecast vectors [L][B][G][d], the queries [L][B][Hq][d], and the K|V
+    blocks of each layer's sets gathered in list order [L][B][G][S][2][blk][d]
+    (the attention addresses entry s at position s; every key of a decode set
+    precedes the query, so the causal mask never applies and the result is
+    the attention over the blocks themselves)."""
+
+    def __init__(self, w, kc, F, Q, kv_sets, idx0):
+        self.w, self.kc, self.F, self.Q, self.kv, self.idx0 = w, kc, F, Q, kv_sets, idx0
+        self.slot_idx = np.broadcast_to(np.arange(w.S, dtype=np.int32),
+                                        (w.B, 1, w.G, w.S)).copy()
+
+    def step(self):
+        import oracle
+        w = self.w
+        L, B, G, d, blk, S = w.layers, w.B, w.G, w.d, w.blk, w.S
+        for l in range(L):
+            nxt = (l + 1) % L
+            oracle.select(self.F[l].reshape(B, 1, G, 1, d), self.kc[nxt], w.k, w.n_init,
+                          w.n_local, w.T - 1, blk)
+            flat = self.kv[l].reshape(-1)
+            oracle.sparse_attention(self.Q[l].reshape(B, 1, w.Hq, d), flat, flat[blk * d:],
+                                    self.slot_idx, w.T - 1, w.T, blk,
+                                    bg_stride=S * 2 * blk * d, blk_stride=2 * blk * d, G=G)
+
+    def time(self, seconds: float, threads: int | None = None, max_reps: int = 1000,
+             min_reps: int = 1):
+        """(steps per second, reps, seconds) of back-to-back steps; threads
+        bounds the oracle's thread pool (None: every host core)."""
+        old = os.environ.get("SPARDA_ORACLE_THREADS")
+        if threads is not None:
+            os.environ["SPARDA_ORACLE_THREADS"] = str(threads)
+        try:
+            reps, t0 = 0, time.perf_counter()
+            while True:
+                self.step()
+                reps += 1
+                el = time.perf_counter() - t0
+                if (el >= seconds and reps >= min_reps) or reps >= max_reps:
+                    break
+        finally:
+            if threads is not None:
+                if old is None:
+                    os.environ.pop("SPARDA_ORACLE_THREADS", None)
+                else:
+                    os.environ["SPARDA_ORACLE_THREADS"] = old
+        return reps / el, reps, el
+
+
+def oracle_sets(w, kc, F):
+    """Every layer's current sets, as the loop holds them at the start of a
+    step: layer l's blocks were picked by layer l-1's Forecast vectors (layer
+    0's by the last layer's).  [L][B][G][S]"""
     import oracle
-    w = loop.w
+    L, B, G, d = w.layers, w.B, w.G, w.d
+    return np.stack([oracle.select(F[(l - 1) % L].reshape(B, 1, G, 1, d), kc[l], w.k, w.n_init,
+                                   w.n_local, w.T - 1, w.blk)[0][:, 0] for l in range(L)])
+
+
+def oracle_sample_from_loop(loop: DecodeLoop) -> OracleDecodeSample:
+    """The oracle's inputs taken from the GPU loop's own buffers: the same
+    compressed keys, Forecast vectors and queries, and the K|V blocks of the
+    sets the oracle itself picks (gathered on the device, outside any timing)."""
     import torch
-    nb = 1                                                   # sequences in the sample
-    L, G, NB, d, blk = w.layers, w.G, w.NB, w.d, w.blk
+    w = loop.w
 
     def bits(t):
         return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
-    kv = [bits(loop.kv[l, :nb]) for l in range(L)]
-    Q = bits(loop.Q[:, :nb])
-    F = bits(loop.F[:, :nb])
-    kc = []
-    for l in range(L):
-        _, kcb = oracle.compress_keys(kv[l], blk, shape=(1, nb * G * NB, blk, d),
-                                      strides=(2 * blk * d, d))
-        kc.append(kcb.reshape(nb, G, NB, d))
-    idx0, _, _ = oracle.select(F[L - 1].reshape(nb, 1, G, 1, d), kc[0], w.k, w.n_init, w.n_local, w.T - 1)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        idx = idx0
-        for l in range(L):
-            nxt = (l + 1) % L
-            nidx, _, _ = oracle.select(F[l].reshape(nb, 1, G, 1, d), kc[nxt], w.k, w.n_init,
-                                       w.n_local, w.T - 1)
-            oracle.sparse_attention(Q[l].reshape(nb, 1, w.Hq, d), kv[l].reshape(-1),
-                                    kv[l].reshape(-1)[blk * d:], idx, w.T - 1, w.T, blk,
-                                    bg_stride=NB * 2 * blk * d, blk_stride=2 * blk * d, G=G)
-            idx = nidx
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds or reps >= 1000:
-            break
-    return {"value": nb * reps / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+    kc = [bits(loop.kc[l]) for l in range(w.layers)]
+    F, Q = bits(loop.F), bits(loop.Q)
+    sets = oracle_sets(w, kc, F)
+    kv = []
+    for l in range(w.layers):
+        ids = torch.from_numpy(np.maximum(sets[l], 0).astype(np.int64)).to(loop.kv.device)
+        flat = loop.kv[l].reshape(w.B * w.G, w.NB, -1)
+        g = torch.gather(flat, 1, ids.reshape(w.B * w.G, w.S, 1).expand(-1, -1, flat.shape[2]))
+        kv.append(bits(g).reshape(w.B, w.G, w.S, 2, w.blk, w.d))
+    return OracleDecodeSample(w, kc, F, Q, kv, sets[0])
+
+
+def oracle_sample_synthetic(w, seed: int) -> OracleDecodeSample:
+    """The same sample with inputs drawn on the host (numpy, seeded): block
+    keys N(0, 1/64) like the means of 64 N(0, 1) keys, Forecast vectors and
+    queries N(0, 1), and N(0, 1) K|V for the blocks of each layer's sets."""
+    import oracle  # noqa: F401  (the oracle is built on first use)
+    L, B, G, d = w.layers, w.B, w.G, w.d
+    rng = W.rng_for(seed, 99)
+    kc = [W.f32_to_bf16_bits(rng.standard_normal((B, G, w.NB, d), dtype=np.float32) / 8)
+          for _ in range(L)]
+    F = W.normal_bf16(rng, (L, B, G, d))
+    Q = W.normal_bf16(rng, (L, B, w.Hq, d))
+    sets = oracle_sets(w, kc, F)
+    kv = [W.normal_bf16(rng, (B, G, w.S, 2, w.blk, d)) for _ in range(L)]
+    return OracleDecodeSample(w, kc, F, Q, kv, sets[0])
+
+
+def oracle_baseline(loop: DecodeLoop, seconds: float):
+    """The fp64 oracle as it stands, timed on the host cores on the whole
+    batch of the GPU loop (all 16 sequences, 4 layers, the same inputs),
+    with every host core and then with one."""
+    import oracle
+    smp = oracle_sample_from_loop(loop)
+    w = loop.w
+    rate, reps, el = smp.time(seconds, min_reps=2)
+    rate1, reps1, el1 = smp.time(0.0, threads=1, max_reps=1)
+    return {"value": w.B * rate, "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": "%d of %d sequences x %d layers (select + sparse attention), %d reps, %.1f s"
-                      % (nb, w.B, L, reps, el)}
+            "sample": "all %d sequences x %d layers per step (select of every (sequence, group) "
+                      "over %d blocks + attention of every head over its %d-block set), %d steps, "
+                      "%.1f s; inputs are the GPU loop's (K|V of the oracle's own sets)"
+                      % (w.B, w.layers, w.NB, w.S, reps, el),
+            "one_core": {"value": w.B * rate1, "unit": "tokens/s", "cores": 1,
+                         "steps": reps1, "seconds": round(el1, 2)}}
 
 
 # --------------------------------------------------------------------------
@@ -716,6 +808,7 @@ def run_sparda(args):
     layer_bytes = loop.bytes_attn() + loop.bytes_select()
     step_gbs = L * layer_bytes / (ms_step * 1e-3) / 1e9
     traffic = profiled_traffic("attn_tc_kernel", loop.bytes_attn())
+    b_attn = loop.bytes_attn()
 
     e2e = {"unavailable": e2e_skip} if e2e_skip else None
     if want_e2e:
@@ -743,6 +836,13 @@ def run_sparda(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_baseline(loop, args.cpu_seconds)
+    del loop
+    torch.cuda.empty_cache()
+    # the prefill chunk and the selection sweep, summarised in the same line
+    prefill = sweep = None
+    if world == 1 and not args.no_extra:
+        prefill = prefill_summary(run_prefill(args.steps))
+        sweep = sweep_summary()
 
     if rank == 0:
         line = {
@@ -766,10 +866,12 @@ def run_sparda(args):
             "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel", "achieved": att_gbs,
                          "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
                          "traffic": traffic, "peak_kind": peak_kind,
-                         "bytes_per_launch": loop.bytes_attn()},
+                         "bytes_per_launch": b_attn},
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "prefill": prefill,
+            "sweep": sweep,
             "gpu_launches": args.steps * L * 2,
             "cuda_graph": graph is not None,
             "graph_steps": GRAPH_STEPS if graph_m is not None else 1,
@@ -980,6 +1082,31 @@ def run_prefill(steps):
     }
 
 
+def prefill_summary(r):
+    """The prefill chunk's figures for the main JSON line."""
+    burst, sustained, kind = measured_bf16_peaks()
+    return {"workload": r["workload"], "select_us": round(r["select_us"], 1),
+            "attn_us": round(r["attn_us"], 1), "chunk_us": round(r["chunk_us"], 1),
+            "tokens_per_s": round(r["tokens_per_s"], 1),
+            "attn_useful_TFLOPs": round(r["attn_useful_TFLOPs"], 2),
+            "attn_frac_of_bf16_peak": round(r["attn_useful_TFLOPs"] / burst, 4),
+            "select_TFLOPs": round(r["select_TFLOPs"], 2),
+            "compress_us": round(r["compress_us"], 1), "compress_GBps": round(r["compress_GBps"], 1),
+            "bf16_peak_TFLOPs": burst, "peak_kind": kind, "device_status": r["device_status"]}
+
+
+def sweep_summary():
+    """The selection sweep's two cuts for the main JSON line: every block
+    count at B = 16, and every batch at NB = 2048; Forecast next to the
+    4-head baseline selector on the same keys, L2 flushed before each call."""
+    pts = [(NB, 16) for NB in W.SWEEP_NB] + [(2048, B) for B in W.SWEEP_B if B != 16]
+    r = run_sweep(pts)
+    return {"points": [[p["NB"], p["B"], p["forecast_us"], p["baseline_us"], p["forecast_GBps"]]
+                       for p in r["points"]],
+            "columns": ["NB", "B", "forecast_us", "baseline_us", "forecast_GBps"],
+            "timing": r["timing"], "clocks": r["clocks"]}
+
+
 def run_windows(steps):
     """The window grid: decode selection at the decode loop's shapes and the
     prefill chunk's, plus the window compression of the chunk's keys."""
@@ -1108,38 +1235,39 @@ def run_real_model(steps):
     return out
 
 
-def run_sweep():
+def run_sweep(pts=None):
     """Selection-only sweep: Forecast (one vector per group) next to the
     baseline selector (the group's 4 query heads, scores summed) on the same
-    compressed keys."""
+    compressed keys.  pts: (NB, B) points, default every combination."""
     import torch
     from block_sparse_long_sparda_b200 import abi
     dev = torch.device("cuda")
     G, Hq, d, k = 8, 32, 128, 64
     points = []
     clocks = ClockSampler(torch.cuda.current_device())
-    for NB in W.SWEEP_NB:
-        for B in W.SWEEP_B:
-            T = NB * 64
-            p = abi.make_params(B, Hq, G, T, k)
-            kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
-            W.torch_normal_bf16_(kc, W.SWEEP_SEED * 1000 + NB + B)
-            gen = torch.Generator(device=dev)
-            gen.manual_seed(W.SWEEP_SEED + NB * 64 + B)
-            F = torch.randn(B, G, d, generator=gen, device=dev).to(torch.bfloat16)
-            Qh = torch.randn(B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
-            idx = torch.empty(B, G, k + 3, dtype=torch.int32, device=dev)
-            ws1 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1)
-            ws4 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, Hq // G)
-            f_us = time_cold(
-                lambda: abi.sparda_forecast_select(p, F, 1, 1, T - 1, kc, idx, ws1), 15)
-            b_us = time_cold(
-                lambda: abi.sparda_forecast_select(p, Qh, 1, Hq // G, T - 1, kc, idx, ws4), 15)
-            nbytes = B * G * NB * d * 2
-            points.append({"NB": NB, "B": B, "forecast_us": round(f_us, 2),
-                           "baseline_us": round(b_us, 2),
-                           "forecast_GBps": round(nbytes / (f_us * 1e-6) / 1e9, 1)})
-            del kc
+    if pts is None:
+        pts = [(NB, B) for NB in W.SWEEP_NB for B in W.SWEEP_B]
+    for NB, B in pts:
+        T = NB * 64
+        p = abi.make_params(B, Hq, G, T, k)
+        kc = torch.empty(B, G, NB, d, dtype=torch.bfloat16, device=dev)
+        W.torch_normal_bf16_(kc, W.SWEEP_SEED * 1000 + NB + B)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(W.SWEEP_SEED + NB * 64 + B)
+        F = torch.randn(B, G, d, generator=gen, device=dev).to(torch.bfloat16)
+        Qh = torch.randn(B, Hq, d, generator=gen, device=dev).to(torch.bfloat16)
+        idx = torch.empty(B, G, k + 3, dtype=torch.int32, device=dev)
+        ws1 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1)
+        ws4 = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, Hq // G)
+        f_us = time_cold(
+            lambda: abi.sparda_forecast_select(p, F, 1, 1, T - 1, kc, idx, ws1), 15)
+        b_us = time_cold(
+            lambda: abi.sparda_forecast_select(p, Qh, 1, Hq // G, T - 1, kc, idx, ws4), 15)
+        nbytes = B * G * NB * d * 2
+        points.append({"NB": NB, "B": B, "forecast_us": round(f_us, 2),
+                       "baseline_us": round(b_us, 2),
+                       "forecast_GBps": round(nbytes / (f_us * 1e-6) / 1e9, 1)})
+        del kc
     return {"metric": "selection-only sweep: Forecast vs 4-head baseline selector (us per call)",
             "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16",
             "timing": "median of 15 calls, each after a 256 MB read that flushes L2 "
@@ -1300,51 +1428,37 @@ def run_profile_case():
 
 
 def run_reference(args):
-    """The oracle (plain fp64 CPU code) on the host cores, same metric."""
+    """The oracle (plain fp64 CPU code) on the host cores, same metric and
+    workload: every step runs the oracle's selection and attention for all 16
+    sequences and 4 layers (inputs drawn on the host, K|V only for the blocks
+    each layer's sets name)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import torch
     import oracle
     w = WORKLOAD
-    L, G, NB, d, blk = w.layers, w.G, w.NB, w.d, w.blk
-    nb = 1
-    rng = W.rng_for(w.seed, 99)
-    kv = [W.normal_bf16(rng, (nb, G, NB, 2, blk, d)) for _ in range(L)]
-    Q = W.normal_bf16(rng, (L, nb, w.Hq, d))
-    F = W.normal_bf16(rng, (L, nb, G, d))
-    kc = [oracle.compress_keys(kv[l], blk, shape=(1, nb * G * NB, blk, d), strides=(2 * blk * d, d))[1]
-          .reshape(nb, G, NB, d) for l in range(L)]
-    idx, _, _ = oracle.select(F[L - 1].reshape(nb, 1, G, 1, d), kc[0], w.k, w.n_init, w.n_local, w.T - 1)
-
-    def step():
-        nonlocal idx
-        for l in range(L):
-            nxt = (l + 1) % L
-            nidx, _, _ = oracle.select(F[l].reshape(nb, 1, G, 1, d), kc[nxt], w.k, w.n_init, w.n_local, w.T - 1)
-            oracle.sparse_attention(Q[l].reshape(nb, 1, w.Hq, d), kv[l].reshape(-1), kv[l].reshape(-1)[blk * d:],
-                                    idx, w.T - 1, w.T, blk, bg_stride=NB * 2 * blk * d,
-                                    blk_stride=2 * blk * d, G=G)
-            idx = nidx
-
+    smp = oracle_sample_synthetic(w, w.seed)
     for _ in range(args.warmup):
-        step()
+        smp.step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        step()
+        smp.step()
     el = time.perf_counter() - t0
-    v = nb * args.steps / el
+    v = w.B * args.steps / el
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "layers": L, "Hq": w.Hq, "G": G,
-                   "d": d, "block": blk, "k": w.k},
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "layers": w.layers, "Hq": w.Hq,
+                   "G": w.G, "d": w.d, "block": w.blk, "k": w.k, "n_init": w.n_init,
+                   "n_local": w.n_local},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
-                         "sample": "%d of %d sequences per step x %d layers (select + sparse "
-                                   "attention)" % (nb, w.B, L)},
+                         "sample": "all %d sequences x %d layers per step (select of every "
+                                   "(sequence, group) over %d blocks + attention of every head "
+                                   "over its %d-block set); inputs drawn on the host"
+                                   % (w.B, w.layers, w.NB, w.S)},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

@@ -78,7 +78,6 @@ def test_decode_waits_run_out_then_the_workspace_serves_the_next_call(split):
         assert int(st.item()) == 0
         check_attention(host_bits(O.check("O")).reshape(w.B, 1, w.Hq, w.d), ora,
                         "after timeouts, split=%d" % split)
-    del pl_tickets
 
 
 def test_prefill_waits_run_out_then_the_workspace_serves_the_next_call():
