@@ -841,8 +841,8 @@ def run_sparda(args):
     # the prefill chunk and the selection sweep, summarised in the same line
     prefill = sweep = None
     if world == 1 and not args.no_extra:
-        prefill = prefill_summary(run_prefill(args.steps))
-        sweep = sweep_summary()
+        prefill = prefill_summary(run_prefill(args.steps, with_oracle=rank == 0))
+        sweep = sweep_summary(with_oracle=rank == 0)
 
     if rank == 0:
         line = {
@@ -1061,7 +1061,36 @@ class PrefillChunk:
         return 2.0 * w.B * w.G * w.d * ncand, 4.0 * w.B * w.Hq * w.d * keys
 
 
-def run_prefill(steps):
+def oracle_prefill_sample(pc, n_tok: int = 32):
+    """The fp64 oracle on a bounded sample of the prefill chunk: the last
+    n_tok query tokens of sequence 0, every group, per-token selection over
+    the GPU's compressed keys and attention over the oracle's sets; the time
+    is scaled to the whole chunk (B x nq tokens)."""
+    import oracle
+    import torch
+    w = pc.w
+
+    def bits(t):
+        return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    K, V = bits(pc.K[:1]), bits(pc.V[:1])
+    kc = bits(pc.kc[:1])
+    F = bits(pc.F[:1, w.nq - n_tok:]).reshape(1, n_tok, w.G, 1, w.d)
+    Q = bits(pc.Q[:1, w.nq - n_tok:])
+    q0 = w.T - n_tok
+    t0 = time.perf_counter()
+    idx, _, _ = oracle.select(F, kc, w.k, w.n_init, w.n_local, q0, w.blk)
+    t1 = time.perf_counter()
+    oracle.sparse_attention(Q, K, V, idx, q0, w.T, w.blk)
+    t2 = time.perf_counter()
+    scale = w.B * w.nq / n_tok
+    return {"select_us": (t1 - t0) * 1e6 * scale, "attn_us": (t2 - t1) * 1e6 * scale,
+            "chunk_us": (t2 - t0) * 1e6 * scale, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "the last %d query tokens of sequence 0, all %d groups, timed once and "
+                      "scaled by %d" % (n_tok, w.G, int(scale))}
+
+
+def run_prefill(steps, with_oracle=False):
     pc = PrefillChunk()
     w = pc.w
     n = max(3, min(steps, 10))
@@ -1070,6 +1099,7 @@ def run_prefill(steps):
     a_us = time_back_to_back(pc.attention, n)
     st = int(pc.status.item())
     sel_flop, att_flop = pc.flops()
+    cpu = oracle_prefill_sample(pc) if with_oracle else None
     return {
         "metric": "prefill chunk: compress, per-token Forecast select, sparse attention (us)",
         "workload": w.name, "B": w.B, "T": w.T, "nq": w.nq, "Hq": w.Hq, "G": w.G, "k": w.k,
@@ -1078,7 +1108,7 @@ def run_prefill(steps):
         "attn_us": a_us, "attn_useful_TFLOPs": att_flop / (a_us * 1e-6) / 1e12,
         "attn_gathered_GBps": w.B * w.nq * w.G * w.S * 2 * w.blk * w.d * 2 / (a_us * 1e-6) / 1e9,
         "chunk_us": s_us + a_us, "tokens_per_s": w.B * w.nq / ((s_us + a_us) * 1e-6),
-        "device_status": st, "data": "synthetic", "dtype": "bf16",
+        "device_status": st, "data": "synthetic", "dtype": "bf16", "cpu_baseline": cpu,
     }
 
 
@@ -1092,18 +1122,22 @@ def prefill_summary(r):
             "attn_frac_of_bf16_peak": round(r["attn_useful_TFLOPs"] / burst, 4),
             "select_TFLOPs": round(r["select_TFLOPs"], 2),
             "compress_us": round(r["compress_us"], 1), "compress_GBps": round(r["compress_GBps"], 1),
-            "bf16_peak_TFLOPs": burst, "peak_kind": kind, "device_status": r["device_status"]}
+            "bf16_peak_TFLOPs": burst, "peak_kind": kind, "device_status": r["device_status"],
+            "cpu_baseline": r.get("cpu_baseline")}
 
 
-def sweep_summary():
+def sweep_summary(with_oracle=False):
     """The selection sweep's two cuts for the main JSON line: every block
     count at B = 16, and every batch at NB = 2048; Forecast next to the
-    4-head baseline selector on the same keys, L2 flushed before each call."""
+    4-head baseline selector on the same keys, L2 flushed before each call.
+    with_oracle: also the fp64 oracle's Forecast selection time at NB = 2048
+    and 16384, B = 16, on the same keys (one call each)."""
     pts = [(NB, 16) for NB in W.SWEEP_NB] + [(2048, B) for B in W.SWEEP_B if B != 16]
-    r = run_sweep(pts)
+    r = run_sweep(pts, oracle_pts=[(2048, 16), (16384, 16)] if with_oracle else ())
     return {"points": [[p["NB"], p["B"], p["forecast_us"], p["baseline_us"], p["forecast_GBps"]]
                        for p in r["points"]],
             "columns": ["NB", "B", "forecast_us", "baseline_us", "forecast_GBps"],
+            "cpu_baseline": r.get("oracle"),
             "timing": r["timing"], "clocks": r["clocks"]}
 
 
@@ -1235,7 +1269,7 @@ def run_real_model(steps):
     return out
 
 
-def run_sweep(pts=None):
+def run_sweep(pts=None, oracle_pts=()):
     """Selection-only sweep: Forecast (one vector per group) next to the
     baseline selector (the group's 4 query heads, scores summed) on the same
     compressed keys.  pts: (NB, B) points, default every combination."""
@@ -1243,7 +1277,7 @@ def run_sweep(pts=None):
     from block_sparse_long_sparda_b200 import abi
     dev = torch.device("cuda")
     G, Hq, d, k = 8, 32, 128, 64
-    points = []
+    points, o_pts = [], []
     clocks = ClockSampler(torch.cuda.current_device())
     if pts is None:
         pts = [(NB, B) for NB in W.SWEEP_NB for B in W.SWEEP_B]
@@ -1267,12 +1301,20 @@ def run_sweep(pts=None):
         points.append({"NB": NB, "B": B, "forecast_us": round(f_us, 2),
                        "baseline_us": round(b_us, 2),
                        "forecast_GBps": round(nbytes / (f_us * 1e-6) / 1e9, 1)})
+        if (NB, B) in oracle_pts:
+            import oracle
+            kcb = kc.cpu().view(torch.int16).numpy().view(np.uint16)
+            Fb = F.cpu().view(torch.int16).numpy().view(np.uint16).reshape(B, 1, G, 1, d)
+            t0 = time.perf_counter()
+            oracle.select(Fb, kcb, k, 1, 2, T - 1)
+            o_pts.append({"NB": NB, "B": B, "forecast_us": (time.perf_counter() - t0) * 1e6,
+                          "cores": oracle.num_threads(), "kind": "oracle"})
         del kc
     return {"metric": "selection-only sweep: Forecast vs 4-head baseline selector (us per call)",
             "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16",
             "timing": "median of 15 calls, each after a 256 MB read that flushes L2 "
                       "(the read is outside the events)",
-            "clocks": clocks.stop()}
+            "oracle": o_pts or None, "clocks": clocks.stop()}
 
 
 class HeadSoftmaxCase:
