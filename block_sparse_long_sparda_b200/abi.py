@@ -53,7 +53,7 @@ class sparda_tuning(ctypes.Structure):
     _fields_ = [("select_chunk", ctypes.c_int), ("select_stream", ctypes.c_int),
                 ("select_binned", ctypes.c_int), ("attn_ctas", ctypes.c_int),
                 ("attn_stages", ctypes.c_int), ("attn_split_kv", ctypes.c_int),
-                ("prefetch_ctas", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("prefetch_ctas", ctypes.c_int), ("attn_prefill_per_token", ctypes.c_int),
                 ("attn_wait_cycles", ctypes.c_longlong)]
 
 

@@ -32,8 +32,7 @@ int sparda::check_params(const sparda_params *p) {
   if (p->k + p->n_init + p->n_local < 1) return SPARDA_EINVAL;
   if (p->tune) {
     const sparda_tuning &t = *p->tune;
-    if (t.reserved != 0 || t.select_chunk < 0 || t.attn_ctas < 0 || t.prefetch_ctas < 0 ||
-        t.attn_wait_cycles < 0)
+    if (t.select_chunk < 0 || t.attn_ctas < 0 || t.prefetch_ctas < 0 || t.attn_wait_cycles < 0)
       return SPARDA_EINVAL;
     if (t.attn_stages != 0 && t.attn_stages != 2 && t.attn_stages != 3 && t.attn_stages != 4 &&
         t.attn_stages != 6)

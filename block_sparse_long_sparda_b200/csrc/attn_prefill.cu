@@ -6,17 +6,703 @@
 // [p1 <section>] = the SparDA summary page at deepresearch2agi.pages.dev.
 //
 // [p4 "The fourth projection", Algorithm 1 / Eq. 5]: O_l = attention(Q_l,
-// K_l[B_l], V_l[B_l]) with every key resident on the GPU.
+// K_l[B_l], V_l[B_l]) with every key resident on the GPU, each query token
+// with its own set B_l(i) (init U local U top-k, per token and group).
 //
-// The chunk runs through the tcgen05 gather kernel of attn_decode.cu with one
-// (token, group) pair per block list; pairs are streamed group by group so
-// that the K/V the running CTAs read stays in L2.
+// Design (B200): block-major.  With per-token sets, the tokens that chose a
+// block are scattered over the whole chunk (each block of a 128K sequence is
+// picked by ~64 of 2048 tokens), so streaming each token's own list reads
+// every block ~17 times through L2.  Here every selected block's K/V is read
+// once per (sequence, group) for all the tokens that chose it:
+//  1. invert_kernel -- one CTA per (sequence, group): the token -> blocks
+//     lists become block -> tokens lists (a counting sort in shared
+//     memory), and the blocks are cut into work items of up to 128 / R * 4
+//     tokens (four 128-row tiles);
+//  2. attn_block_kernel -- persistent, one CTA per SM.  A producer warp takes
+//     items from a global counter and brings the block's K and V by TMA
+//     (128-byte swizzle, no multicast) into a three-stage ring.  A tile is
+//     128 rows = (token, head) pairs of the item; two warpgroups of row
+//     threads take alternate tiles: each gathers its tile's query rows
+//     (cp.async, straight into the swizzled operand), and after one
+//     thread has issued S = Q K^T (tcgen05, M = 128, N = 64, K = 128, fp32
+//     in TMEM) it runs the row softmax over the block's 64 keys (exp2
+//     domain, causal inside the token's own block) and writes P (bf16); after
+//     O = P V (M = 128, N = 128, K = 64) it writes the row's partial: o / l
+//     in fp16 and (m, l) in fp32, at the (token, group, set position, head)
+//     slot.  The two warpgroups ping-pong on the tensor core, and each
+//     gathers its next tile's rows while its current product runs;
+//  3. merge_kernel -- one warp per (token, group): for each head the
+//     partials of the token's set combine as o = sum_s l_s 2^(m_s - M) o_s /
+//     sum_s l_s 2^(m_s - M), M = max_s m_s.
+// Every wait is bounded; a timeout sets SPARDA_DEV_TIMEOUT, drains what was
+// issued and frees TMEM.  Shapes the block-major path does not take (more
+// than 16384 blocks, more than 2^21 query tokens, sets of 2048 entries or
+// more), or sparda_tuning::attn_prefill_per_token, use the per-token gather
+// kernel of attn_decode.cu instead.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace sparda {
 
+namespace {
+
+constexpr int kRows = 128;            // rows (token, head) per tile: the MMA's M
+constexpr int kTilesPerItem = 4;      // tiles of one item share its K/V stage
+constexpr int kSBits = 11;            // list entry = token << kSBits | set position
+constexpr int kMaxSetEntries = (1 << kSBits) - 1;
+constexpr int kMaxTokens = 1 << (32 - kSBits);
+constexpr int kInvThreads = 1024;
+constexpr int kMaxBlocksInv = 16384;  // blocks per sequence the inversion holds in shared memory
+constexpr int kNst = 3;               // K/V ring stages (32 KB each)
+constexpr int kTileRing = 8;          // tile descriptors in flight
+constexpr int kBlkThreads = 320;      // 2 row warpgroups, producer, MMA issuer
+constexpr int kWarpProd = 8, kWarpMma = 9;
+constexpr int kTile8 = 8192;          // 64 rows x 64 bf16, one swizzled tile
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// 1. block -> tokens lists and work items
+// ---------------------------------------------------------------------------
+struct InvArgs {
+  const int32_t *idx;      // [B][nq][G][S]
+  const int32_t *seq_len;
+  int32_t *status;
+  uint32_t *list;          // [B*G][nq*S]: token << kSBits | s, grouped by block
+  int4 *items;             // {bg, block, first list entry, tokens}
+  uint32_t *counters;      // [0] items written, [1] items taken (block pass)
+  int B, G, nq, S, NB, T, q_start, tpi;
+};
+
+// exclusive prefix sums of two per-thread values over the CTA; returns the
+// totals in tot0/tot1
+__device__ void block_scan2(uint32_t v0, uint32_t v1, uint32_t &x0, uint32_t &x1, uint32_t &tot0,
+                            uint32_t &tot1, uint32_t *tmp /* [2][33] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t a = v0, b = v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ta = __shfl_up_sync(0xffffffffu, a, o), tb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += ta;
+      b += tb;
+    }
+  }
+  if (lane == 31) {
+    tmp[warp] = a;
+    tmp[33 + warp] = b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t wa = tmp[lane], wb = tmp[33 + lane];
+    uint32_t ia = wa, ib = wb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ta = __shfl_up_sync(0xffffffffu, ia, o), tb = __shfl_up_sync(0xffffffffu, ib, o);
+      if (lane >= o) {
+        ia += ta;
+        ib += tb;
+      }
+    }
+    tmp[lane] = ia - wa;
+    tmp[33 + lane] = ib - wb;
+    if (lane == 31) {
+      tmp[32] = ia;
+      tmp[65] = ib;
+    }
+  }
+  __syncthreads();
+  x0 = tmp[warp] + a - v0;
+  x1 = tmp[33 + warp] + b - v1;
+  tot0 = tmp[32];
+  tot1 = tmp[65];
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kInvThreads) invert_kernel(InvArgs a) {
+  extern __shared__ uint32_t cnt[];  // [NB]: counts, then write cursors
+  __shared__ uint32_t tmp[66];
+  __shared__ uint32_t s_base;
+  const int tid = threadIdx.x;
+  const int bg = blockIdx.x, b = bg / a.G, g = bg % a.G;
+  pdl_trigger();
+  pdl_wait();
+  int qs = a.q_start;
+  if (a.seq_len) {  // the chunk is the sequence's last nq tokens; an invalid length has no work
+    const int len = a.seq_len[b];
+    if (len < a.nq || len > a.T) return;
+    qs = len - a.nq;
+  }
+  for (int j = tid; j < a.NB; j += kInvThreads) cnt[j] = 0u;
+  __syncthreads();
+  const long long E = (long long)a.nq * a.S;
+  const int32_t *idx_bg = a.idx + (long long)b * a.nq * a.G * a.S + (long long)g * a.S;
+  bool bad = false;
+  for (long long e = tid; e < E; e += kInvThreads) {
+    const int i = (int)(e / a.S), s = (int)(e - (long long)i * a.S);
+    const int j = idx_bg[(long long)i * a.G * a.S + s];
+    if (j < 0) continue;
+    if (j >= a.NB || j > (qs + i) / kBlk) {  // not a block this token may attend to
+      bad = true;
+      continue;
+    }
+    atomicAdd(&cnt[j], 1u);
+  }
+  if (__syncthreads_or(bad) && tid == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+  // list start and item offset of every block (each thread a run of blocks)
+  const int per = (a.NB + kInvThreads - 1) / kInvThreads;
+  const int j0 = min(a.NB, tid * per), j1 = min(a.NB, j0 + per);
+  uint32_t sum_t = 0, sum_i = 0;
+  for (int j = j0; j < j1; ++j) {
+    sum_t += cnt[j];
+    sum_i += (cnt[j] + a.tpi - 1) / a.tpi;
+  }
+  uint32_t off_t, off_i, tot_t, tot_i;
+  block_scan2(sum_t, sum_i, off_t, off_i, tot_t, tot_i, tmp);
+  if (tid == 0) s_base = atomicAdd(&a.counters[0], tot_i);
+  __syncthreads();
+  const uint32_t base = s_base;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t c = cnt[j];
+    for (uint32_t k = 0; k * a.tpi < c; ++k)
+      a.items[base + off_i + k] = make_int4(bg, j, (int)(off_t + k * a.tpi),
+                                            (int)min((uint32_t)a.tpi, c - k * a.tpi));
+    off_i += (c + a.tpi - 1) / a.tpi;
+    cnt[j] = off_t;  // the block's write cursor
+    off_t += c;
+  }
+  __syncthreads();
+  uint32_t *list = a.list + (long long)bg * E;
+  for (long long e = tid; e < E; e += kInvThreads) {
+    const int i = (int)(e / a.S), s = (int)(e - (long long)i * a.S);
+    const int j = idx_bg[(long long)i * a.G * a.S + s];
+    if (j < 0 || j >= a.NB || j > (qs + i) / kBlk) continue;
+    const uint32_t p = atomicAdd(&cnt[j], 1u);
+    list[p] = ((uint32_t)i << kSBits) | (uint32_t)s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. the block pass
+// ---------------------------------------------------------------------------
+struct BlkArgs {
+  const uint16_t *Q;        // [B][nq][Hq][d]
+  const uint32_t *list;
+  const int4 *items;
+  uint32_t *counters;
+  float2 *ml;               // [B][nq][G][S][R] (m, l) in the exp2 domain
+  __half *po;               // [B][nq][G][S][R][d] o / l
+  const int32_t *seq_len;
+  int32_t *status;
+  long long bg_rows;        // K/V rows per (sequence, group)
+  int B, G, nq, S, NB, T, q_start, R, rshift;
+  float scale_log2;
+  long long wait_cycles;
+};
+
+struct TileDesc {
+  int bg, j, toff, n_rows;  // list offset of the tile's first token; valid rows
+  int stage, kv_par, last;  // K/V stage, its phase bit, last tile of the item
+  int end;                  // no more tiles
+};
+
+struct BlkCtl {
+  uint64_t kv_full[kNst], kv_empty[kNst];
+  uint64_t t_full[kTileRing], t_empty[kTileRing];
+  uint64_t a_ready[2], s_full[2], p_full[2], o_full[2];
+  TileDesc desc[kTileRing];
+  uint32_t tmem_base;
+  int s_abort;
+};
+
+// K/V ring | two query-row tiles (32 KB) | two P tiles (16 KB) | control
+constexpr size_t kBlkSmem = (size_t)kNst * 4 * kTile8 + 2 * 32768 + 2 * 16384 +
+                            (sizeof(BlkCtl) + 127) / 128 * 128;
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         long long limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kBlkThreads, 1)
+    attn_block_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                      BlkArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *kv = smem_raw;                          // kNst x [K lo | V lo | K hi | V hi]
+  uint8_t *qa = kv + kNst * 4 * kTile8;            // 2 x [2 dim halves][128 rows][64]
+  uint8_t *pa = qa + 2 * 32768;                    // 2 x [128 rows][64 keys]
+  BlkCtl &ctl = *reinterpret_cast<BlkCtl *>(pa + 2 * 16384);
+  volatile int *s_abort = &ctl.s_abort;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long lim = a.wait_cycles;
+  pdl_trigger();
+  if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles would be misread
+    pdl_wait();
+    if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kNst; ++s) {
+      mbar_init(&ctl.kv_full[s], 1);
+      mbar_init(&ctl.kv_empty[s], 1);
+    }
+    for (int q = 0; q < kTileRing; ++q) {
+      mbar_init(&ctl.t_full[q], 1);
+      mbar_init(&ctl.t_empty[q], kRows + 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&ctl.a_ready[w], kRows);
+      mbar_init(&ctl.s_full[w], 1);
+      mbar_init(&ctl.p_full[w], kRows);
+      mbar_init(&ctl.o_full[w], 1);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+    tc::prefetch_map(&mapK);
+    tc::prefetch_map(&mapV);
+  }
+  if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 512);  // S: 2 x 64 columns, O: 2 x 128
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = ctl.tmem_base;
+  pdl_wait();  // the lists and items of the inversion are complete
+
+  int produced = 0;              // producer: items whose K/V loads were issued
+  int issued_s = 0, issued_p = 0;  // MMA issuer: products committed
+
+  if (warp == kWarpProd) {
+    // ================= producer: items -> K/V stages and tile descriptors =====
+    if (lane == 0) {
+      const uint32_t n_items = __ldcg(&a.counters[0]);
+      const int tok_per_tile = kRows >> a.rshift;
+      int u = 0;
+      bool ok = true;
+      auto put = [&](const TileDesc &d) -> bool {
+        const int q = u % kTileRing;
+        if (u >= kTileRing &&
+            !wait_bar(&ctl.t_empty[q], (uint32_t)(((u / kTileRing) - 1) & 1), s_abort, lim))
+          return false;
+        ctl.desc[q] = d;
+        mbar_arrive(&ctl.t_full[q]);  // release: the descriptor is visible to its waiters
+        ++u;
+        return true;
+      };
+#pragma unroll 1
+      for (;;) {
+        const uint32_t it = atomicAdd(&a.counters[1], 1u);
+        if (it >= n_items) break;
+        const int4 rec = __ldcg(&a.items[it]);
+        const int st = produced % kNst;
+        if (produced >= kNst &&
+            !wait_bar(&ctl.kv_empty[st], (uint32_t)(((produced / kNst) - 1) & 1), s_abort, lim)) {
+          ok = false;
+          break;
+        }
+        uint8_t *dst = kv + st * 4 * kTile8;
+        const int row = (int)((long long)rec.x * a.bg_rows + (long long)rec.y * kBlk);
+        mbar_arrive_expect_tx(&ctl.kv_full[st], 4 * kTile8);
+        tc::tma_load_2d(dst, &mapK, 0, row, &ctl.kv_full[st]);
+        tc::tma_load_2d(dst + kTile8, &mapV, 0, row, &ctl.kv_full[st]);
+        tc::tma_load_2d(dst + 2 * kTile8, &mapK, 64, row, &ctl.kv_full[st]);
+        tc::tma_load_2d(dst + 3 * kTile8, &mapV, 64, row, &ctl.kv_full[st]);
+        const int kv_par = (produced / kNst) & 1;
+        ++produced;
+        const int n_tiles = (int)((((long long)rec.w << a.rshift) + kRows - 1) / kRows);
+        for (int m = 0; m < n_tiles && ok; ++m) {
+          TileDesc d;
+          d.bg = rec.x;
+          d.j = rec.y;
+          d.toff = rec.z + m * tok_per_tile;
+          d.n_rows = min(kRows, (rec.w - m * tok_per_tile) << a.rshift);
+          d.stage = st;
+          d.kv_par = kv_par;
+          d.last = m == n_tiles - 1;
+          d.end = 0;
+          ok = put(d);
+        }
+        if (!ok) break;
+      }
+      if (ok) {  // one end marker for each row warpgroup
+        TileDesc d = {};
+        d.end = 1;
+        ok = put(d) && put(d);
+      }
+      if (!ok) *s_abort = 1;
+    }
+  } else if (warp == kWarpMma) {
+    // ================= MMA issuer: S(u), then P V(u - 1) ====================
+    if (lane == 0) {
+      constexpr uint32_t id_s = tc::idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_o = tc::idesc_bf16(128, 128, false, true);
+      bool ok = true;
+      int prev_stage = 0, prev_last = 0;
+      auto issue_pv = [&](int v) -> bool {  // P V of tile v
+        const int w = v & 1;
+        if (!wait_bar(&ctl.p_full[w], (uint32_t)((v >> 1) & 1), s_abort, lim)) return false;
+        tc::fence_after_sync();
+        const uint64_t dP = tc::sdesc(pa + w * 16384, 16, 1024);
+        const uint64_t dV = tc::sdesc(kv + prev_stage * 4 * kTile8 + kTile8, 2 * kTile8, 1024);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc::mma_bf16(tmem + 128 + w * 128, dP + (uint64_t)(k * 2), dV + (uint64_t)(k * 128), id_o, k > 0);
+        tc::mma_commit(&ctl.o_full[w]);
+        if (prev_last) tc::mma_commit(&ctl.kv_empty[prev_stage]);
+        issued_p = v + 1;
+        mbar_arrive(&ctl.t_empty[v % kTileRing]);
+        return true;
+      };
+      int u = 0;
+#pragma unroll 1
+      for (;; ++u) {
+        const int q = u % kTileRing;
+        if (!wait_bar(&ctl.t_full[q], (uint32_t)((u / kTileRing) & 1), s_abort, lim)) {
+          ok = false;
+          break;
+        }
+        const TileDesc d = ctl.desc[q];
+        if (d.end) break;
+        const int w = u & 1;
+        if (!wait_bar(&ctl.kv_full[d.stage], (uint32_t)d.kv_par, s_abort, lim) ||
+            !wait_bar(&ctl.a_ready[w], (uint32_t)((u >> 1) & 1), s_abort, lim)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint64_t dA = tc::sdesc(qa + w * 32768, 16, 1024);
+        const uint64_t dK = tc::sdesc(kv + d.stage * 4 * kTile8, 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_bf16(tmem + w * 64, dA + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
+                       dK + (uint64_t)((k >> 2) * (2 * kTile8 >> 4) + (k & 3) * 2), id_s, k > 0);
+        tc::mma_commit(&ctl.s_full[w]);
+        issued_s = u + 1;
+        if (u > 0 && !issue_pv(u - 1)) {
+          ok = false;
+          break;
+        }
+        prev_stage = d.stage;
+        prev_last = d.last;
+      }
+      if (ok && u > 0 && !issue_pv(u - 1)) ok = false;
+      if (!ok) *s_abort = 1;
+    }
+  } else {
+    // ================= row warpgroups (warps 0-3: tiles 0, 2, ...; 4-7: 1, 3, ...) ==
+    const int w = warp >> 2;
+    const int r = tid & 127;                     // row of the tile = TMEM lane
+    const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
+    uint8_t *A = qa + w * 32768;
+    uint8_t *P = pa + w * 16384;
+    const int R = a.R;
+    const int h = r & (R - 1);
+    bool ok = true;
+    // the row's token: its list entry, position, query and partial slot
+    struct Row {
+      int end, valid, j, stage_last;
+      long long q_off, slot;
+      int pos;
+    };
+    auto read_desc = [&](int u, Row &row) -> bool {
+      const int q = u % kTileRing;
+      if (!wait_bar(&ctl.t_full[q], (uint32_t)((u / kTileRing) & 1), s_abort, lim)) return false;
+      const TileDesc d = ctl.desc[q];
+      row.end = d.end;
+      if (!d.end) {
+        mbar_arrive(&ctl.t_empty[q]);
+        row.valid = r < d.n_rows;
+        row.j = d.j;
+        const int b = d.bg / a.G, g = d.bg - b * a.G;
+        int i = 0, s = 0;
+        if (row.valid) {
+          const uint32_t e = __ldg(&a.list[(long long)d.bg * a.nq * a.S + d.toff + (r >> a.rshift)]);
+          i = (int)(e >> kSBits);
+          s = (int)(e & kMaxSetEntries);
+        }
+        int qs = a.q_start;
+        if (a.seq_len) qs = __ldg(&a.seq_len[b]) - a.nq;  // valid lengths only reach here
+        row.pos = qs + i;
+        const long long tok = (long long)b * a.nq + i;
+        row.q_off = (tok * a.G + g) * (long long)R * kD + (long long)h * kD;
+        row.slot = ((tok * a.G + g) * a.S + s) * (long long)R + h;
+      }
+      return true;
+    };
+    auto gather = [&](const Row &row) {  // the row's query into the swizzled A tile
+      const uint16_t *src = a.Q + row.q_off;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        cp_async16(A + (c >> 3) * 16384 + tc::sw128_offset(r, (c & 7) * 8), src + c * 8,
+                   row.valid ? 16u : 0u);
+      cp_async_commit();
+    };
+    int u = w, k = 0;
+    Row cur{}, nxt{};
+    ok = read_desc(u, cur);
+    if (ok && !cur.end) {
+      gather(cur);
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&ctl.a_ready[w]);
+    }
+#pragma unroll 1
+    while (ok && !cur.end) {
+      // ---- S(u) -> softmax -> P ----
+      ok = wait_bar(&ctl.s_full[w], (uint32_t)(k & 1), s_abort, lim);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc::fence_after_sync();
+      float x[64];
+      {
+        float t[32];
+        tc::tmem_ld32(tmem + w * 64 + lane_sel, t);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[c] = t[c];
+        tc::tmem_ld32(tmem + w * 64 + 32 + lane_sel, t);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[32 + c] = t[c];
+      }
+      const int lim_key = cur.pos - cur.j * kBlk;  // keys after the token are masked
+      float m = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = (c <= lim_key) ? x[c] * a.scale_log2 : -INFINITY;
+        m = fmaxf(m, x[c]);
+      }
+      float l = 0.f;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = (cur.valid && x[c8 * 8 + 2 * e] != -INFINITY) ? exp2f(x[c8 * 8 + 2 * e] - m) : 0.f;
+          const float p1 = (cur.valid && x[c8 * 8 + 2 * e + 1] != -INFINITY) ? exp2f(x[c8 * 8 + 2 * e + 1] - m) : 0.f;
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          l += __low2float(pb) + __high2float(pb);
+          pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+        }
+        *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c8 * 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(&ctl.p_full[w]);
+      // ---- the next tile's query rows load while P V(u) runs ----
+      ok = read_desc(u + 2, nxt);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      if (!nxt.end) gather(nxt);
+      // ---- P V(u) -> the row's partial ----
+      ok = wait_bar(&ctl.o_full[w], (uint32_t)(k & 1), s_abort, lim);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc::fence_after_sync();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __half *dst = a.po + cur.slot * kD;
+#pragma unroll
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float o[32];
+        tc::tmem_ld32(tmem + 128 + w * 128 + c0 + lane_sel, o);
+        if (cur.valid) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t hv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2 hh = __floats2half2_rn(o[q * 8 + 2 * e] * inv_l, o[q * 8 + 2 * e + 1] * inv_l);
+              hv[e] = *reinterpret_cast<const uint32_t *>(&hh);
+            }
+            *reinterpret_cast<uint4 *>(dst + c0 + q * 8) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          }
+        }
+      }
+      if (cur.valid) a.ml[cur.slot] = make_float2(m, l);
+      tc::fence_before_sync();
+      // ---- hand the next tile's rows to the MMA issuer ----
+      cur = nxt;
+      u += 2;
+      ++k;
+      if (cur.end) break;
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&ctl.a_ready[w]);
+    }
+    cp_async_wait_all();  // no copy may still target the tiles when the CTA leaves
+    if (!ok) *s_abort = 1;
+  }
+
+  __syncthreads();
+  if (*s_abort) {
+    flag_status(a.status, SPARDA_DEV_TIMEOUT);
+    // let what was issued land or finish (bounded) before the memory is released
+    if (warp == kWarpProd && lane == 0)
+      for (int v = max(0, produced - kNst); v < produced; ++v)
+        (void)mbar_wait_bounded(&ctl.kv_full[v % kNst], (uint32_t)((v / kNst) & 1));
+    if (warp == kWarpMma && lane == 0) {
+      for (int v = max(0, issued_s - 2); v < issued_s; ++v)
+        (void)mbar_wait_bounded(&ctl.s_full[v & 1], (uint32_t)((v >> 1) & 1));
+      for (int v = max(0, issued_p - 2); v < issued_p; ++v)
+        (void)mbar_wait_bounded(&ctl.o_full[v & 1], (uint32_t)((v >> 1) & 1));
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// 3. merge of each token's partials
+// ---------------------------------------------------------------------------
+struct MergeArgs {
+  const int32_t *idx;       // [B][nq][G][S]
+  const float2 *ml;
+  const __half *po;
+  uint16_t *O;              // [B][nq][Hq][d]
+  const int32_t *seq_len;
+  int32_t *status;
+  int B, G, nq, S, NB, T, q_start, R;
+};
+
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long pr = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // (b, i, g)
+  pdl_trigger();
+  pdl_wait();
+  if (pr >= (long long)a.B * a.nq * a.G) return;
+  const int g = (int)(pr % a.G);
+  const long long tok = pr / a.G;
+  const int i = (int)(tok % a.nq), b = (int)(tok / a.nq);
+  const int R = a.R;
+  uint16_t *out = a.O + (tok * a.G + g) * (long long)R * kD;
+  int qs = a.q_start;
+  if (a.seq_len) {
+    const int len = a.seq_len[b];
+    if (len < a.nq || len > a.T) {  // an invalid length: a zero output
+      for (int e = lane; e < R * kD / 8; e += 32)
+        reinterpret_cast<uint4 *>(out)[e] = make_uint4(0, 0, 0, 0);
+      if (lane == 0 && i == 0 && g == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+      return;
+    }
+    qs = len - a.nq;
+  }
+  const int pos = qs + i;
+  const int32_t *ids = a.idx + pr * a.S;
+  const float2 *ml = a.ml + pr * (long long)a.S * R;
+  const __half *po = a.po + pr * (long long)a.S * R * kD;
+  // valid entries of the set, as the inversion took them (up to 2047, in
+  // chunks of 32 per lane bit mask)
+  for (int h = 0; h < R; ++h) {
+    float M = -INFINITY;
+    for (int s = lane; s < a.S; s += 32) {
+      const int j = ids[s];
+      if (j >= 0 && j < a.NB && j <= pos / kBlk) M = fmaxf(M, ml[(long long)s * R + h].x);
+    }
+    M = warp_max_xor(M, 1, 32);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = 0.f;
+#pragma unroll 1
+    for (int s0 = 0; s0 < a.S; s0 += 32) {
+      const int s = s0 + lane;
+      float wgt = 0.f;
+      if (s < a.S) {
+        const int j = ids[s];
+        if (j >= 0 && j < a.NB && j <= pos / kBlk) {
+          const float2 v = ml[(long long)s * R + h];
+          wgt = v.y * exp2f(v.x - M);
+        }
+      }
+      L += wgt;
+      const int n = min(32, a.S - s0);
+#pragma unroll 4
+      for (int q = 0; q < n; ++q) {
+        const float wq = __shfl_sync(0xffffffffu, wgt, q);
+        if (wq != 0.f) {  // uniform over the warp
+          const uint2 raw = *reinterpret_cast<const uint2 *>(po + ((long long)(s0 + q) * R + h) * kD + lane * 4);
+          const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw.x);
+          const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw.y);
+          acc[0] += wq * __low2float(h0);
+          acc[1] += wq * __high2float(h0);
+          acc[2] += wq * __low2float(h1);
+          acc[3] += wq * __high2float(h1);
+        }
+      }
+    }
+    L = warp_sum_xor(L, 1, 32);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    const __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+    uint2 st;
+    st.x = *reinterpret_cast<const uint32_t *>(&o0);
+    st.y = *reinterpret_cast<const uint32_t *>(&o1);
+    *reinterpret_cast<uint2 *>(out + h * kD + lane * 4) = st;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host: layout of the workspace, eligibility
+// ---------------------------------------------------------------------------
+struct BlkPlan {
+  bool ok;
+  int R, S, NB, tpi;
+  long long max_items;
+  size_t off_list, off_items, off_ml, off_po, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+BlkPlan plan_block(const sparda_params &p, int nq) {
+  BlkPlan pl{};
+  pl.R = p.Hq / p.G;
+  pl.S = p.k + p.n_init + p.n_local;
+  pl.NB = (p.T + kBlk - 1) / kBlk;
+  pl.tpi = (kRows * kTilesPerItem) / pl.R;
+  pl.ok = tuning(p).attn_prefill_per_token == 0 && pl.NB <= kMaxBlocksInv && nq < kMaxTokens &&
+          pl.S <= kMaxSetEntries;
+  if (!pl.ok) return pl;
+  const long long bgs = (long long)p.B * p.G;
+  const long long entries = bgs * nq * pl.S;  // list entries and partial slots per head
+  pl.max_items = bgs * (ceil_div_ll((long long)nq * pl.S, pl.tpi) + pl.NB);
+  size_t off = 256;                                           // two counters
+  pl.off_list = off;
+  off += align256((size_t)entries * 4);
+  pl.off_items = off;
+  off += align256((size_t)pl.max_items * 16);
+  pl.off_ml = off;
+  off += align256((size_t)entries * pl.R * 8);
+  pl.off_po = off;
+  off += align256((size_t)entries * pl.R * kD * 2);
+  pl.total = off;
+  return pl;
+}
+
+}  // namespace
+
 size_t prefill_ws_bytes(const sparda_params &p, int nq) {
+  const BlkPlan pl = plan_block(p, nq);
+  if (pl.ok) return pl.total;
   return plan_gather(p, (long long)p.B * nq * p.G).ws_bytes;
 }
 
@@ -25,9 +711,112 @@ cudaError_t launch_attn_prefill(const sparda_params &p, const uint16_t *Q, int n
                                 long long tok_stride, const int32_t *idx, uint16_t *O, void *ws,
                                 size_t ws_bytes, int32_t *dev_status, cudaStream_t stream) {
   (void)ws_bytes;
-  const DecodePlan pl = plan_gather(p, (long long)p.B * nq * p.G);
-  return launch_gather_attn(p, pl, nq, q_start, Q, K, V, bg_stride, (long long)kBlk * tok_stride,
-                            idx, SPARDA_ADDR_LOGICAL, O, ws, dev_status, stream);
+  const BlkPlan pl = plan_block(p, nq);
+  if (!pl.ok) {  // the per-token gather kernel
+    const DecodePlan gp = plan_gather(p, (long long)p.B * nq * p.G);
+    return launch_gather_attn(p, gp, nq, q_start, Q, K, V, bg_stride, (long long)kBlk * tok_stride,
+                              idx, SPARDA_ADDR_LOGICAL, O, ws, dev_status, stream);
+  }
+  if ((long long)p.B * nq * p.G == 0) return cudaSuccess;
+  char *w = static_cast<char *>(ws);
+  uint32_t *counters = reinterpret_cast<uint32_t *>(w);
+  cudaError_t e = cudaMemsetAsync(counters, 0, 8, stream);
+  if (e != cudaSuccess) return e;
+  // ---- 1. inversion ----
+  InvArgs ia;
+  ia.idx = idx;
+  ia.seq_len = p.seq_len;
+  ia.status = dev_status;
+  ia.list = reinterpret_cast<uint32_t *>(w + pl.off_list);
+  ia.items = reinterpret_cast<int4 *>(w + pl.off_items);
+  ia.counters = counters;
+  ia.B = p.B;
+  ia.G = p.G;
+  ia.nq = nq;
+  ia.S = pl.S;
+  ia.NB = pl.NB;
+  ia.T = p.T;
+  ia.q_start = q_start;
+  ia.tpi = pl.tpi;
+  const size_t inv_smem = (size_t)pl.NB * 4;
+  struct Cached {
+    void *ctx;
+    int n_sm;
+  };
+  static Cached cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  void *ctx = current_context();
+  if (cache[dev].n_sm == 0 || cache[dev].ctx != ctx) {
+    int n_sm = 148;
+    (void)cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaFuncSetAttribute(invert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kMaxBlocksInv * 4);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kBlkSmem);
+    if (e != cudaSuccess) return e;
+    cache[dev].n_sm = n_sm;
+    cache[dev].ctx = ctx;
+  }
+  e = launch_pdl(invert_kernel, (unsigned)(p.B * p.G), kInvThreads, inv_smem, stream, ia);
+  if (e != cudaSuccess) return e;
+  // ---- 2. the block pass ----
+  const long long kv_pairs = (long long)p.B * p.G;
+  const long long bg_rows = bg_stride / kD;
+  long long extent = (kv_pairs - 1) * bg_rows + (long long)pl.NB * kBlk;
+  extent = std::min(extent, kv_pairs * bg_rows);
+  if (extent >= (1LL << 31)) return cudaErrorInvalidValue;
+  CUtensorMap mk, mv;
+  if (!tc::make_map_2d(&mk, K, kD, (uint64_t)extent, kD, 64, 64) ||
+      !tc::make_map_2d(&mv, V, kD, (uint64_t)extent, kD, 64, 64))
+    return cudaErrorNotSupported;
+  BlkArgs ba;
+  ba.Q = Q;
+  ba.list = ia.list;
+  ba.items = ia.items;
+  ba.counters = counters;
+  ba.ml = reinterpret_cast<float2 *>(w + pl.off_ml);
+  ba.po = reinterpret_cast<__half *>(w + pl.off_po);
+  ba.seq_len = p.seq_len;
+  ba.status = dev_status;
+  ba.bg_rows = bg_rows;
+  ba.B = p.B;
+  ba.G = p.G;
+  ba.nq = nq;
+  ba.S = pl.S;
+  ba.NB = pl.NB;
+  ba.T = p.T;
+  ba.q_start = q_start;
+  ba.R = pl.R;
+  ba.rshift = __builtin_ctz((unsigned)pl.R);
+  const float scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
+  ba.scale_log2 = scale * kLog2e;
+  const sparda_tuning &tu = tuning(p);
+  ba.wait_cycles = tu.attn_wait_cycles > 0 ? tu.attn_wait_cycles : kWaitCycles;
+  e = launch_pdl(attn_block_kernel, (unsigned)cache[dev].n_sm, kBlkThreads, kBlkSmem, stream, mk,
+                 mv, ba);
+  if (e != cudaSuccess) return e;
+  // ---- 3. merge ----
+  MergeArgs ma;
+  ma.idx = idx;
+  ma.ml = ba.ml;
+  ma.po = ba.po;
+  ma.O = O;
+  ma.seq_len = p.seq_len;
+  ma.status = dev_status;
+  ma.B = p.B;
+  ma.G = p.G;
+  ma.nq = nq;
+  ma.S = pl.S;
+  ma.NB = pl.NB;
+  ma.T = p.T;
+  ma.q_start = q_start;
+  ma.R = pl.R;
+  const long long rows = (long long)p.B * nq * p.G;
+  e = launch_pdl(merge_kernel, (unsigned)ceil_div_ll(rows, kMergeWarps), kMergeWarps * 32, 0,
+                 stream, ma);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sparda

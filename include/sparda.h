@@ -94,7 +94,9 @@ typedef struct sparda_tuning {
   int attn_split_kv;  /* 1: a ring slot's K and V tiles are refilled separately,
                          -1: together; 0: separately for prefill only            */
   int prefetch_ctas;  /* gather thread blocks when a call passes n_ctas = 0      */
-  int reserved;       /* must be 0                                               */
+  int attn_prefill_per_token;  /* nonzero: prefill attention streams each token's
+                         own block list (the decode kernel, one (token, group)
+                         pair per list) instead of the block-major kernels     */
   long long attn_wait_cycles;  /* bound of every wait in the attention kernel, in
                          SM clock cycles; 0: 2e9 (about one second).  Waits that
                          run out end the call with SPARDA_DEV_TIMEOUT            */

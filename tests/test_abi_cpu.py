@@ -161,7 +161,7 @@ def test_tuning_fields_are_validated_and_size_the_workspace(L):
     calls will use (never the environment)."""
     byref = ctypes.byref
     fake = ctypes.c_void_p(0x10000)
-    for bad in ({"reserved": 1}, {"attn_stages": 5}, {"attn_stages": 4, "attn_split_kv": 1},
+    for bad in ({"attn_stages": 5}, {"attn_stages": 4, "attn_split_kv": 1},
                 {"select_chunk": -256}, {"attn_ctas": -1}, {"prefetch_ctas": -2},
                 {"attn_wait_cycles": -1}):
         p = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8, tune=bad)

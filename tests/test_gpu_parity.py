@@ -1256,10 +1256,11 @@ def test_prefill_attention_parity(T, nq, R):
 @pytest.mark.parametrize("split", ["1", "-1"])
 @pytest.mark.parametrize("nq,R", [(1, 4), (1, 16), (96, 4)])
 def test_attention_both_slot_protocols(split, nq, R):
-    """The attention kernel has two ring protocols: one barrier per slot
-    (the default for decode) and K and V tiles refilled separately (the
-    default for prefill).  Each is forced on the other workload too."""
-    tune = {"attn_split_kv": int(split)}
+    """The per-token attention kernel has two ring protocols: one barrier per
+    slot (the default for decode) and K and V tiles refilled separately (its
+    default for prefill chunks).  Each is forced on the other workload too
+    (prefill through the per-token kernel rather than the block-major one)."""
+    tune = {"attn_split_kv": int(split), "attn_prefill_per_token": int(nq > 1)}
     rng = W.rng_for(41, nq * 100 + R)
     B, G, d, k, T = 2, 2, 128, 12, 6000 + 21
     Hq = G * R
@@ -1282,3 +1283,66 @@ def test_attention_both_slot_protocols(split, nq, R):
                                        d, torch.from_numpy(idx).cuda(), O, ws)
         torch.cuda.synchronize()
         check_attention(host_bits(O), ora, "prefill split=%s" % split)
+
+
+def _prefill_case(B, G, R, T, nq, k, seed, n_init=1, n_local=2):
+    rng = W.rng_for(seed, T + nq + R)
+    d = 128
+    Q = W.normal_bf16(rng, (B, nq, G * R, d))
+    K = W.normal_bf16(rng, (B, G, T, d))
+    V = W.normal_bf16(rng, (B, G, T, d))
+    F = W.normal_bf16(rng, (B, nq, G, 1, d))
+    _, kcb = oracle.compress_keys(K)
+    idx, _, _ = oracle.select(F, kcb, k, n_init, n_local, T - nq)
+    return Q, K, V, idx
+
+
+def _gpu_prefill(Q, K, V, idx, T, k, tune=None, n_init=1, n_local=2, status=None):
+    B, nq, Hq, d = Q.shape
+    G = K.shape[1]
+    p = abi.make_params(B, Hq, G, T, k, n_init, n_local, tune=tune)
+    O = Guarded((B, nq, Hq, d), torch.bfloat16, fill=float("nan"))
+    ws = guarded_workspace(abi.SPARDA_OP_ATTN_PREFILL, p, nq)
+    abi.sparda_sparse_attn_prefill(p, dev_bf16(Q), nq, T - nq, dev_bf16(K), dev_bf16(V), T * d, d,
+                                   torch.from_numpy(np.ascontiguousarray(idx)).cuda(), O.t, ws.t,
+                                   status)
+    ws.check("prefill workspace")
+    return host_bits(O.check("prefill output"))
+
+
+@pytest.mark.parametrize("R,T,nq,k", [(1, 5000 + 13, 300, 12), (16, 3000, 90, 7), (4, 9000, 520, 40),
+                                      (2, 640, 640, 3)])
+def test_prefill_block_major_matches_oracle_and_per_token_kernel(R, T, nq, k):
+    """The block-major prefill kernels (block -> tokens inversion, one read
+    of each selected block for all the tokens that chose it, partials merged
+    per token) against the oracle and against the per-token kernel, for 1
+    and 16 heads per group, chunks whose initial block is chosen by several
+    items' worth of tokens, and a chunk that starts at position 0."""
+    Q, K, V, idx = _prefill_case(2, 2, R, T, nq, k, 44)
+    ora = oracle.sparse_attention(Q, K, V, idx, T - nq, T)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = _gpu_prefill(Q, K, V, idx, T, k, status=st)
+    assert int(st.item()) == 0
+    check_attention(got, ora, "block-major R=%d" % R)
+    ref = _gpu_prefill(Q, K, V, idx, T, k, tune={"attn_prefill_per_token": 1})
+    check_attention(ref, ora, "per-token R=%d" % R)
+    a, b = bf16_f64(got), bf16_f64(ref)
+    assert np.abs(a - b).max() <= 1e-2
+
+
+def test_prefill_block_major_skips_and_flags_bad_ids():
+    """Ids past a token's own block (or past the sequence) are skipped and
+    flagged; the rest of the set is attended as if they were absent."""
+    B, G, R, T, nq, k = 1, 2, 4, 4096, 100, 6
+    Q, K, V, idx = _prefill_case(B, G, R, T, nq, k, 45)
+    bad = idx.copy()
+    bad[0, 10, 1, 2] = 9999           # past the sequence
+    bad[0, 20, 0, 3] = (T - nq + 20) // 64 + 1   # after the token's own block
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = _gpu_prefill(Q, K, V, bad, T, k, status=st)
+    assert abi.sparda_status_from_device(int(st.item())) == abi.SPARDA_ERANGE
+    clean = bad.copy()
+    clean[0, 10, 1, 2] = -1
+    clean[0, 20, 0, 3] = -1
+    ora = oracle.sparse_attention(Q, K, V, clean, T - nq, T)
+    check_attention(got, ora, "bad ids skipped")
