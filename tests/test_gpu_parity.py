@@ -1326,8 +1326,8 @@ def test_prefill_block_major_matches_oracle_and_per_token_kernel(R, T, nq, k):
     check_attention(got, ora, "block-major R=%d" % R)
     ref = _gpu_prefill(Q, K, V, idx, T, k, tune={"attn_prefill_per_token": 1})
     check_attention(ref, ora, "per-token R=%d" % R)
-    a, b = bf16_f64(got), bf16_f64(ref)
-    assert np.abs(a - b).max() <= 1e-2
+    # each is within the tolerance of the oracle, so within twice it of the other
+    assert np.abs(bf16_f64(got) - bf16_f64(ref)).max() <= 2e-2
 
 
 def test_prefill_block_major_skips_and_flags_bad_ids():
