@@ -78,6 +78,8 @@ def parse_args():
                          "keys, summed) at B=16, T=128K on block keys and on window keys, "
                          "beside Forecast and the summed-score baseline on the same keys; "
                          "prints an extra JSON line")
+    ap.add_argument("--only", choices=["prefill", "sweep", "windows", "real-model", "head-softmax"],
+                    help="run this one leg alone (no decode loop) and print its JSON line")
     ap.add_argument("--profile-case", action="store_true",
                     help="run three passes of one decode layer (select, then attention) at "
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
@@ -1505,6 +1507,21 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_only(args):
+    """One leg alone, on one GPU, its JSON line only (for profiling a leg)."""
+    import torch
+    from block_sparse_long_sparda_b200 import build
+    build.build()
+    torch.cuda.set_device(0)
+    fn = {"prefill": lambda: run_prefill(args.steps), "sweep": run_sweep,
+          "windows": lambda: run_windows(args.steps), "real-model": lambda: run_real_model(args.steps),
+          "head-softmax": lambda: run_head_softmax(args.steps)}[args.only]
+    out = fn()
+    print(json.dumps(out), flush=True)
+    if out.get("device_status", 0) != 0:
+        sys.exit(1)
+
+
 def main():
     args = parse_args()
     if args.profile_case:
@@ -1513,6 +1530,8 @@ def main():
         run_profile_case()
     elif args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_only(args)
     else:
         run_sparda(args)
 
