@@ -139,18 +139,32 @@ __global__ void __launch_bounds__(kInvThreads) invert_kernel(InvArgs a) {
   }
   for (int j = tid; j < a.NB; j += kInvThreads) cnt[j] = 0u;
   __syncthreads();
-  const long long E = (long long)a.nq * a.S;
+  const uint32_t E = (uint32_t)a.nq * (uint32_t)a.S;  // < 2^32 (nq < 2^21, S < 2^11)
   const int32_t *idx_bg = a.idx + (long long)b * a.nq * a.G * a.S + (long long)g * a.S;
-  bool bad = false;
-  for (long long e = tid; e < E; e += kInvThreads) {
-    const int i = (int)(e / a.S), s = (int)(e - (long long)i * a.S);
-    const int j = idx_bg[(long long)i * a.G * a.S + s];
-    if (j < 0) continue;
-    if (j >= a.NB || j > (qs + i) / kBlk) {  // not a block this token may attend to
-      bad = true;
-      continue;
+  const long long tok_stride = (long long)a.G * a.S;
+  // entry e of (b, g): token e / S, set position e % S; four loads in flight per thread
+  auto load4 = [&](uint32_t e0, int (&j)[4], int (&i)[4], int (&sp)[4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t e = e0 + (uint32_t)q * kInvThreads;
+      i[q] = (int)(e / (uint32_t)a.S);
+      sp[q] = (int)(e - (uint32_t)i[q] * (uint32_t)a.S);
+      j[q] = e < E ? __ldg(idx_bg + i[q] * tok_stride + sp[q]) : -1;
     }
-    atomicAdd(&cnt[j], 1u);
+  };
+  bool bad = false;
+  for (uint32_t e0 = tid; e0 < E; e0 += 4u * kInvThreads) {
+    int j[4], i[4], sp[4];
+    load4(e0, j, i, sp);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (j[q] < 0) continue;
+      if (j[q] >= a.NB || j[q] > (qs + i[q]) / kBlk) {  // not a block this token may attend to
+        bad = true;
+        continue;
+      }
+      atomicAdd(&cnt[j[q]], 1u);
+    }
   }
   if (__syncthreads_or(bad) && tid == 0) flag_status(a.status, SPARDA_DEV_RANGE);
   // list start and item offset of every block (each thread a run of blocks)
@@ -177,12 +191,15 @@ __global__ void __launch_bounds__(kInvThreads) invert_kernel(InvArgs a) {
   }
   __syncthreads();
   uint32_t *list = a.list + (long long)bg * E;
-  for (long long e = tid; e < E; e += kInvThreads) {
-    const int i = (int)(e / a.S), s = (int)(e - (long long)i * a.S);
-    const int j = idx_bg[(long long)i * a.G * a.S + s];
-    if (j < 0 || j >= a.NB || j > (qs + i) / kBlk) continue;
-    const uint32_t p = atomicAdd(&cnt[j], 1u);
-    list[p] = ((uint32_t)i << kSBits) | (uint32_t)s;
+  for (uint32_t e0 = tid; e0 < E; e0 += 4u * kInvThreads) {
+    int j[4], i[4], sp[4];
+    load4(e0, j, i, sp);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (j[q] < 0 || j[q] >= a.NB || j[q] > (qs + i[q]) / kBlk) continue;
+      const uint32_t p = atomicAdd(&cnt[j[q]], 1u);
+      list[p] = ((uint32_t)i[q] << kSBits) | (uint32_t)sp[q];
+    }
   }
 }
 
@@ -205,9 +222,10 @@ struct BlkArgs {
 };
 
 struct TileDesc {
-  int bg, j, toff, n_rows;  // list offset of the tile's first token; valid rows
+  int bg, j, n_rows;        // (sequence, group), block, valid rows of the tile
   int stage, kv_par, last;  // K/V stage, its phase bit, last tile of the item
   int end;                  // no more tiles
+  uint32_t ent[kRows];      // list entries of the tile's tokens (token << kSBits | s)
 };
 
 struct BlkCtl {
@@ -289,37 +307,41 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
   const uint32_t tmem = ctl.tmem_base;
   pdl_wait();  // the lists and items of the inversion are complete
 
-  int produced = 0;              // producer: items whose K/V loads were issued
+  int produced = 0;                // producer: items whose K/V loads were issued
   int issued_s = 0, issued_p = 0;  // MMA issuer: products committed
 
   if (warp == kWarpProd) {
-    // ================= producer: items -> K/V stages and tile descriptors =====
-    if (lane == 0) {
-      const uint32_t n_items = __ldcg(&a.counters[0]);
-      const int tok_per_tile = kRows >> a.rshift;
-      int u = 0;
-      bool ok = true;
-      auto put = [&](const TileDesc &d) -> bool {
-        const int q = u % kTileRing;
-        if (u >= kTileRing &&
-            !wait_bar(&ctl.t_empty[q], (uint32_t)(((u / kTileRing) - 1) & 1), s_abort, lim))
-          return false;
-        ctl.desc[q] = d;
-        mbar_arrive(&ctl.t_full[q]);  // release: the descriptor is visible to its waiters
-        ++u;
-        return true;
-      };
+    // ====== producer (whole warp): items -> K/V stages and tile descriptors ======
+    // Lane 0 takes items and issues the TMA; the warp copies each tile's list
+    // entries into its descriptor, so the row threads find them in shared memory.
+    const uint32_t n_items = __ldcg(&a.counters[0]);
+    const int tok_per_tile = kRows >> a.rshift;
+    const long long E = (long long)a.nq * a.S;
+    int u = 0;
+    bool ok = true;
+    // wait until ring slot u is free (whole warp, uniform result)
+    auto slot_free = [&]() -> bool {
+      bool f = true;
+      if (lane == 0 && u >= kTileRing)
+        f = wait_bar(&ctl.t_empty[u % kTileRing], (uint32_t)(((u / kTileRing) - 1) & 1), s_abort, lim);
+      return __shfl_sync(0xffffffffu, (int)f, 0) != 0;
+    };
 #pragma unroll 1
-      for (;;) {
-        const uint32_t it = atomicAdd(&a.counters[1], 1u);
-        if (it >= n_items) break;
-        const int4 rec = __ldcg(&a.items[it]);
-        const int st = produced % kNst;
-        if (produced >= kNst &&
-            !wait_bar(&ctl.kv_empty[st], (uint32_t)(((produced / kNst) - 1) & 1), s_abort, lim)) {
-          ok = false;
-          break;
-        }
+    for (;;) {
+      uint32_t it = 0;
+      if (lane == 0) it = atomicAdd(&a.counters[1], 1u);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it >= n_items) break;
+      const int4 rec = __ldcg(&a.items[it]);
+      const int st = produced % kNst;
+      bool free_ok = true;
+      if (lane == 0 && produced >= kNst)
+        free_ok = wait_bar(&ctl.kv_empty[st], (uint32_t)(((produced / kNst) - 1) & 1), s_abort, lim);
+      if (!__shfl_sync(0xffffffffu, (int)free_ok, 0)) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
         uint8_t *dst = kv + st * 4 * kTile8;
         const int row = (int)((long long)rec.x * a.bg_rows + (long long)rec.y * kBlk);
         mbar_arrive_expect_tx(&ctl.kv_full[st], 4 * kTile8);
@@ -327,89 +349,120 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
         tc::tma_load_2d(dst + kTile8, &mapV, 0, row, &ctl.kv_full[st]);
         tc::tma_load_2d(dst + 2 * kTile8, &mapK, 64, row, &ctl.kv_full[st]);
         tc::tma_load_2d(dst + 3 * kTile8, &mapV, 64, row, &ctl.kv_full[st]);
-        const int kv_par = (produced / kNst) & 1;
-        ++produced;
-        const int n_tiles = (int)((((long long)rec.w << a.rshift) + kRows - 1) / kRows);
-        for (int m = 0; m < n_tiles && ok; ++m) {
-          TileDesc d;
+      }
+      const int kv_par = (produced / kNst) & 1;
+      ++produced;
+      const int n_tiles = (int)((((long long)rec.w << a.rshift) + kRows - 1) / kRows);
+      const uint32_t *src = a.list + (long long)rec.x * E + rec.z;
+      for (int m = 0; m < n_tiles; ++m) {
+        if (!slot_free()) {
+          ok = false;
+          break;
+        }
+        TileDesc &d = ctl.desc[u % kTileRing];
+        const int n_tok = min(tok_per_tile, rec.w - m * tok_per_tile);
+        for (int e = lane; e < n_tok; e += 32) d.ent[e] = __ldg(src + m * tok_per_tile + e);
+        if (lane == 0) {
           d.bg = rec.x;
           d.j = rec.y;
-          d.toff = rec.z + m * tok_per_tile;
-          d.n_rows = min(kRows, (rec.w - m * tok_per_tile) << a.rshift);
+          d.n_rows = n_tok << a.rshift;
           d.stage = st;
           d.kv_par = kv_par;
           d.last = m == n_tiles - 1;
           d.end = 0;
-          ok = put(d);
         }
-        if (!ok) break;
+        __syncwarp();  // the lanes' entries are written before lane 0 publishes the slot
+        if (lane == 0) mbar_arrive(&ctl.t_full[u % kTileRing]);
+        ++u;
       }
-      if (ok) {  // one end marker for each row warpgroup
-        TileDesc d = {};
-        d.end = 1;
-        ok = put(d) && put(d);
-      }
-      if (!ok) *s_abort = 1;
+      if (!ok) break;
     }
+    // one end marker for each row warpgroup
+    for (int e = 0; e < 2 && ok; ++e) {
+      if (!slot_free()) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        ctl.desc[u % kTileRing].end = 1;
+        mbar_arrive(&ctl.t_full[u % kTileRing]);
+      }
+      ++u;
+    }
+    if (!ok && lane == 0) *s_abort = 1;
   } else if (warp == kWarpMma) {
-    // ================= MMA issuer: S(u), then P V(u - 1) ====================
+    // ====== MMA issuer: S(u) and P V(v), each in tile order, whichever is ready ======
+    // S(u) needs the tile's descriptor, its K/V stage and its query rows; the
+    // row warpgroup hands those in only after it has read S and O of its
+    // previous tile, so S and O of a warpgroup are never overwritten early.
     if (lane == 0) {
       constexpr uint32_t id_s = tc::idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_o = tc::idesc_bf16(128, 128, false, true);
+      int n_s = 0, n_p = 0, total = -1;  // S issued, PV issued, tiles (once the end is seen)
+      long long t0 = clock64();
       bool ok = true;
-      int prev_stage = 0, prev_last = 0;
-      auto issue_pv = [&](int v) -> bool {  // P V of tile v
-        const int w = v & 1;
-        if (!wait_bar(&ctl.p_full[w], (uint32_t)((v >> 1) & 1), s_abort, lim)) return false;
-        tc::fence_after_sync();
-        const uint64_t dP = tc::sdesc(pa + w * 16384, 16, 1024);
-        const uint64_t dV = tc::sdesc(kv + prev_stage * 4 * kTile8 + kTile8, 2 * kTile8, 1024);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc::mma_bf16(tmem + 128 + w * 128, dP + (uint64_t)(k * 2), dV + (uint64_t)(k * 128), id_o, k > 0);
-        tc::mma_commit(&ctl.o_full[w]);
-        if (prev_last) tc::mma_commit(&ctl.kv_empty[prev_stage]);
-        issued_p = v + 1;
-        mbar_arrive(&ctl.t_empty[v % kTileRing]);
-        return true;
-      };
-      int u = 0;
 #pragma unroll 1
-      for (;; ++u) {
-        const int q = u % kTileRing;
-        if (!wait_bar(&ctl.t_full[q], (uint32_t)((u / kTileRing) & 1), s_abort, lim)) {
-          ok = false;
-          break;
-        }
-        const TileDesc d = ctl.desc[q];
-        if (d.end) break;
-        const int w = u & 1;
-        if (!wait_bar(&ctl.kv_full[d.stage], (uint32_t)d.kv_par, s_abort, lim) ||
-            !wait_bar(&ctl.a_ready[w], (uint32_t)((u >> 1) & 1), s_abort, lim)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        const uint64_t dA = tc::sdesc(qa + w * 32768, 16, 1024);
-        const uint64_t dK = tc::sdesc(kv + d.stage * 4 * kTile8, 16, 1024);
+      while (total < 0 || n_p < total) {
+        bool moved = false;
+        if (total < 0 && n_s - n_p < 2) {
+          const int q = n_s % kTileRing, w = n_s & 1;
+          if (mbar_test_wait(&ctl.t_full[q], (uint32_t)((n_s / kTileRing) & 1))) {
+            if (ctl.desc[q].end) {
+              total = n_s;
+              moved = true;
+            } else if (mbar_test_wait(&ctl.kv_full[ctl.desc[q].stage], (uint32_t)ctl.desc[q].kv_par) &&
+                       mbar_test_wait(&ctl.a_ready[w], (uint32_t)((n_s >> 1) & 1))) {
+              const int st = ctl.desc[q].stage;
+              tc::fence_after_sync();
+              const uint64_t dA = tc::sdesc(qa + w * 32768, 16, 1024);
+              const uint64_t dK = tc::sdesc(kv + st * 4 * kTile8, 16, 1024);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          tc::mma_bf16(tmem + w * 64, dA + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
-                       dK + (uint64_t)((k >> 2) * (2 * kTile8 >> 4) + (k & 3) * 2), id_s, k > 0);
-        tc::mma_commit(&ctl.s_full[w]);
-        issued_s = u + 1;
-        if (u > 0 && !issue_pv(u - 1)) {
+              for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tmem + w * 64, dA + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
+                             dK + (uint64_t)((k >> 2) * (2 * kTile8 >> 4) + (k & 3) * 2), id_s, k > 0);
+              tc::mma_commit(&ctl.s_full[w]);
+              issued_s = ++n_s;
+              moved = true;
+            }
+          }
+        }
+        if (n_p < n_s) {
+          const int q = n_p % kTileRing, w = n_p & 1;
+          if (mbar_test_wait(&ctl.p_full[w], (uint32_t)((n_p >> 1) & 1))) {
+            tc::fence_after_sync();
+            // the tile's descriptor stays in its slot until this product is issued
+            const int st = ctl.desc[q].stage;
+            const uint64_t dP = tc::sdesc(pa + w * 16384, 16, 1024);
+            const uint64_t dV = tc::sdesc(kv + st * 4 * kTile8 + kTile8, 2 * kTile8, 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc::mma_bf16(tmem + 128 + w * 128, dP + (uint64_t)(k * 2), dV + (uint64_t)(k * 128),
+                           id_o, k > 0);
+            tc::mma_commit(&ctl.o_full[w]);
+            if (ctl.desc[q].last) tc::mma_commit(&ctl.kv_empty[st]);
+            mbar_arrive(&ctl.t_empty[q]);
+            issued_p = ++n_p;
+            moved = true;
+          }
+        }
+        if (moved) {
+          t0 = clock64();
+          continue;
+        }
+        if (*s_abort) {
           ok = false;
           break;
         }
-        prev_stage = d.stage;
-        prev_last = d.last;
+        if (clock64() - t0 > lim) {
+          ok = false;
+          break;
+        }
+        __nanosleep(32);
       }
-      if (ok && u > 0 && !issue_pv(u - 1)) ok = false;
       if (!ok) *s_abort = 1;
     }
   } else {
-    // ================= row warpgroups (warps 0-3: tiles 0, 2, ...; 4-7: 1, 3, ...) ==
+    // ====== row warpgroups (warps 0-3: tiles 0, 2, ...; 4-7: 1, 3, ...) ======
     const int w = warp >> 2;
     const int r = tid & 127;                     // row of the tile = TMEM lane
     const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
@@ -418,35 +471,29 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     const int R = a.R;
     const int h = r & (R - 1);
     bool ok = true;
-    // the row's token: its list entry, position, query and partial slot
+    // the row's token: its block, position, query and partial slot
     struct Row {
-      int end, valid, j, stage_last;
+      int end, valid, j, pos;
       long long q_off, slot;
-      int pos;
     };
     auto read_desc = [&](int u, Row &row) -> bool {
       const int q = u % kTileRing;
       if (!wait_bar(&ctl.t_full[q], (uint32_t)((u / kTileRing) & 1), s_abort, lim)) return false;
-      const TileDesc d = ctl.desc[q];
+      const TileDesc &d = ctl.desc[q];
       row.end = d.end;
-      if (!d.end) {
-        mbar_arrive(&ctl.t_empty[q]);
-        row.valid = r < d.n_rows;
-        row.j = d.j;
-        const int b = d.bg / a.G, g = d.bg - b * a.G;
-        int i = 0, s = 0;
-        if (row.valid) {
-          const uint32_t e = __ldg(&a.list[(long long)d.bg * a.nq * a.S + d.toff + (r >> a.rshift)]);
-          i = (int)(e >> kSBits);
-          s = (int)(e & kMaxSetEntries);
-        }
-        int qs = a.q_start;
-        if (a.seq_len) qs = __ldg(&a.seq_len[b]) - a.nq;  // valid lengths only reach here
-        row.pos = qs + i;
-        const long long tok = (long long)b * a.nq + i;
-        row.q_off = (tok * a.G + g) * (long long)R * kD + (long long)h * kD;
-        row.slot = ((tok * a.G + g) * a.S + s) * (long long)R + h;
-      }
+      if (d.end) return true;
+      row.valid = r < d.n_rows;
+      row.j = d.j;
+      const int bg = d.bg, b = bg / a.G, g = bg - b * a.G;
+      const uint32_t e = row.valid ? d.ent[r >> a.rshift] : 0u;
+      mbar_arrive(&ctl.t_empty[q]);
+      const int i = (int)(e >> kSBits), s = (int)(e & kMaxSetEntries);
+      int qs = a.q_start;
+      if (a.seq_len) qs = __ldg(&a.seq_len[b]) - a.nq;  // valid lengths only reach here
+      row.pos = qs + i;
+      const long long tok = (long long)b * a.nq + i;
+      row.q_off = (tok * a.G + g) * (long long)R * kD + (long long)h * kD;
+      row.slot = ((tok * a.G + g) * a.S + s) * (long long)R + h;
       return true;
     };
     auto gather = [&](const Row &row) {  // the row's query into the swizzled A tile
@@ -468,50 +515,51 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     }
 #pragma unroll 1
     while (ok && !cur.end) {
-      // ---- S(u) -> softmax -> P ----
+      // ---- S(u) is done: A is free, so the next tile's query rows start loading ----
       ok = wait_bar(&ctl.s_full[w], (uint32_t)(k & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
+      ok = __all_sync(0xffffffffu, read_desc(u + 2, nxt));
+      if (!ok) break;
+      if (!nxt.end) gather(nxt);
+      // ---- softmax of the row over the block's keys -> P ----
       tc::fence_after_sync();
-      float x[64];
-      {
-        float t[32];
-        tc::tmem_ld32(tmem + w * 64 + lane_sel, t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = t[c];
-        tc::tmem_ld32(tmem + w * 64 + 32 + lane_sel, t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 + c] = t[c];
-      }
       const int lim_key = cur.pos - cur.j * kBlk;  // keys after the token are masked
       float m = -INFINITY;
+      {
+        float t[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = (c <= lim_key) ? x[c] * a.scale_log2 : -INFINITY;
-        m = fmaxf(m, x[c]);
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          tc::tmem_ld32(tmem + w * 64 + c0 + lane_sel, t);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c <= lim_key) m = fmaxf(m, t[c] * a.scale_log2);
+        }
       }
       float l = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t pk[4];
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        float t[32];
+        tc::tmem_ld32(tmem + w * 64 + c0 + lane_sel, t);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = (cur.valid && x[c8 * 8 + 2 * e] != -INFINITY) ? exp2f(x[c8 * 8 + 2 * e] - m) : 0.f;
-          const float p1 = (cur.valid && x[c8 * 8 + 2 * e + 1] != -INFINITY) ? exp2f(x[c8 * 8 + 2 * e + 1] - m) : 0.f;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          l += __low2float(pb) + __high2float(pb);
-          pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kk = c0 + c8 * 8 + 2 * e;
+            const float p0 = (cur.valid && kk <= lim_key) ? exp2f(t[c8 * 8 + 2 * e] * a.scale_log2 - m) : 0.f;
+            const float p1 = (cur.valid && kk + 1 <= lim_key) ? exp2f(t[c8 * 8 + 2 * e + 1] * a.scale_log2 - m) : 0.f;
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            l += __low2float(pb) + __high2float(pb);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+          }
+          *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c0 + c8 * 8)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c8 * 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(&ctl.p_full[w]);
-      // ---- the next tile's query rows load while P V(u) runs ----
-      ok = read_desc(u + 2, nxt);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      if (!nxt.end) gather(nxt);
       // ---- P V(u) -> the row's partial ----
       ok = wait_bar(&ctl.o_full[w], (uint32_t)(k & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
@@ -586,79 +634,98 @@ struct MergeArgs {
 
 constexpr int kMergeWarps = 8;
 
+// One warp per (token, group, head); lane = 4 output dims.  The loads of
+// eight set entries are in flight together; a slot no valid entry wrote is
+// loaded too (it lies inside the workspace) but selected away, never used.
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
   const int lane = threadIdx.x & 31;
-  const long long pr = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // (b, i, g)
+  const long long wi = (long long)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);  // (b, i, g, h)
   pdl_trigger();
   pdl_wait();
-  if (pr >= (long long)a.B * a.nq * a.G) return;
+  const int R = a.R;
+  if (wi >= (long long)a.B * a.nq * a.G * R) return;
+  const int h = (int)(wi % R);
+  const long long pr = wi / R;  // (b, i, g)
   const int g = (int)(pr % a.G);
   const long long tok = pr / a.G;
   const int i = (int)(tok % a.nq), b = (int)(tok / a.nq);
-  const int R = a.R;
-  uint16_t *out = a.O + (tok * a.G + g) * (long long)R * kD;
+  uint16_t *out = a.O + (pr * R + h) * (long long)kD;
   int qs = a.q_start;
   if (a.seq_len) {
     const int len = a.seq_len[b];
     if (len < a.nq || len > a.T) {  // an invalid length: a zero output
-      for (int e = lane; e < R * kD / 8; e += 32)
-        reinterpret_cast<uint4 *>(out)[e] = make_uint4(0, 0, 0, 0);
-      if (lane == 0 && i == 0 && g == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+      reinterpret_cast<uint2 *>(out)[lane] = make_uint2(0, 0);
+      if (lane == 0 && i == 0 && g == 0 && h == 0) flag_status(a.status, SPARDA_DEV_RANGE);
       return;
     }
     qs = len - a.nq;
   }
-  const int pos = qs + i;
+  const int c = (qs + i) / kBlk;
   const int32_t *ids = a.idx + pr * a.S;
-  const float2 *ml = a.ml + pr * (long long)a.S * R;
-  const __half *po = a.po + pr * (long long)a.S * R * kD;
-  // valid entries of the set, as the inversion took them (up to 2047, in
-  // chunks of 32 per lane bit mask)
-  for (int h = 0; h < R; ++h) {
-    float M = -INFINITY;
-    for (int s = lane; s < a.S; s += 32) {
-      const int j = ids[s];
-      if (j >= 0 && j < a.NB && j <= pos / kBlk) M = fmaxf(M, ml[(long long)s * R + h].x);
-    }
-    M = warp_max_xor(M, 1, 32);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float L = 0.f;
-#pragma unroll 1
-    for (int s0 = 0; s0 < a.S; s0 += 32) {
-      const int s = s0 + lane;
-      float wgt = 0.f;
-      if (s < a.S) {
-        const int j = ids[s];
-        if (j >= 0 && j < a.NB && j <= pos / kBlk) {
-          const float2 v = ml[(long long)s * R + h];
-          wgt = v.y * exp2f(v.x - M);
-        }
-      }
-      L += wgt;
-      const int n = min(32, a.S - s0);
-#pragma unroll 4
-      for (int q = 0; q < n; ++q) {
-        const float wq = __shfl_sync(0xffffffffu, wgt, q);
-        if (wq != 0.f) {  // uniform over the warp
-          const uint2 raw = *reinterpret_cast<const uint2 *>(po + ((long long)(s0 + q) * R + h) * kD + lane * 4);
-          const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw.x);
-          const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw.y);
-          acc[0] += wq * __low2float(h0);
-          acc[1] += wq * __high2float(h0);
-          acc[2] += wq * __low2float(h1);
-          acc[3] += wq * __high2float(h1);
-        }
-      }
-    }
-    L = warp_sum_xor(L, 1, 32);
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    const __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-    uint2 st;
-    st.x = *reinterpret_cast<const uint32_t *>(&o0);
-    st.y = *reinterpret_cast<const uint32_t *>(&o1);
-    *reinterpret_cast<uint2 *>(out + h * kD + lane * 4) = st;
+  const float2 *ml = a.ml + pr * (long long)a.S * R + h;
+  const __half *po = a.po + (pr * a.S * R + h) * (long long)kD + lane * 4;
+  const long long po_stride = (long long)R * kD;
+  float M = -INFINITY;
+  for (int s = lane; s < a.S; s += 32) {
+    const int j = __ldg(ids + s);
+    if (j >= 0 && j < a.NB && j <= c) M = fmaxf(M, ml[(long long)s * R].x);
   }
+  M = warp_max_xor(M, 1, 32);
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f, L = 0.f;
+#pragma unroll 1
+  for (int s0 = 0; s0 < a.S; s0 += 32) {
+    const int s = s0 + lane;
+    float wgt = 0.f;
+    if (s < a.S) {
+      const int j = __ldg(ids + s);
+      if (j >= 0 && j < a.NB && j <= c) {
+        const float2 v = ml[(long long)s * R];
+        wgt = v.y * exp2f(v.x - M);
+      }
+    }
+    L += wgt;
+    const int n = min(32, a.S - s0);
+    const __half *p0 = po + (long long)s0 * po_stride;
+    int q = 0;
+#pragma unroll 1
+    for (; q + 8 <= n; q += 8) {
+      uint2 raw[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) raw[t] = __ldcs(reinterpret_cast<const uint2 *>(p0 + (long long)(q + t) * po_stride));
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float wq = __shfl_sync(0xffffffffu, wgt, q + t);
+        const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw[t].x);
+        const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw[t].y);
+        if (wq != 0.f) {
+          acc0 = fmaf(wq, __low2float(h0), acc0);
+          acc1 = fmaf(wq, __high2float(h0), acc1);
+          acc2 = fmaf(wq, __low2float(h1), acc2);
+          acc3 = fmaf(wq, __high2float(h1), acc3);
+        }
+      }
+    }
+    for (; q < n; ++q) {
+      const uint2 raw = __ldcs(reinterpret_cast<const uint2 *>(p0 + (long long)q * po_stride));
+      const float wq = __shfl_sync(0xffffffffu, wgt, q);
+      const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw.x);
+      const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw.y);
+      if (wq != 0.f) {
+        acc0 = fmaf(wq, __low2float(h0), acc0);
+        acc1 = fmaf(wq, __high2float(h0), acc1);
+        acc2 = fmaf(wq, __low2float(h1), acc2);
+        acc3 = fmaf(wq, __high2float(h1), acc3);
+      }
+    }
+  }
+  L = warp_sum_xor(L, 1, 32);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc0 * inv, acc1 * inv);
+  const __nv_bfloat162 o1 = __floats2bfloat162_rn(acc2 * inv, acc3 * inv);
+  uint2 st;
+  st.x = *reinterpret_cast<const uint32_t *>(&o0);
+  st.y = *reinterpret_cast<const uint32_t *>(&o1);
+  reinterpret_cast<uint2 *>(out)[lane] = st;
 }
 
 // ---------------------------------------------------------------------------
@@ -813,7 +880,7 @@ cudaError_t launch_attn_prefill(const sparda_params &p, const uint16_t *Q, int n
   ma.T = p.T;
   ma.q_start = q_start;
   ma.R = pl.R;
-  const long long rows = (long long)p.B * nq * p.G;
+  const long long rows = (long long)p.B * nq * p.G * pl.R;  // (token, group, head)
   e = launch_pdl(merge_kernel, (unsigned)ceil_div_ll(rows, kMergeWarps), kMergeWarps * 32, 0,
                  stream, ma);
   return e != cudaSuccess ? e : cudaGetLastError();
