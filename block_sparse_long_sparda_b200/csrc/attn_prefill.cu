@@ -228,11 +228,18 @@ struct TileDesc {
   uint32_t ent[kRows];      // list entries of the tile's tokens (token << kSBits | s)
 };
 
+// where a row's query comes from and where its partial goes (null: no row)
+struct RowAddr {
+  const uint16_t *src;
+  __half *dst;
+};
+
 struct BlkCtl {
   uint64_t kv_full[kNst], kv_empty[kNst];
   uint64_t t_full[kTileRing], t_empty[kTileRing];
   uint64_t a_ready[2], s_full[2], p_full[2], o_full[2];
   TileDesc desc[kTileRing];
+  RowAddr rows[2][2][kRows];  // [warpgroup][tile parity][row]
   uint32_t tmem_base;
   int s_abort;
 };
@@ -312,74 +319,86 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
 
   if (warp == kWarpProd) {
     // ====== producer (whole warp): items -> K/V stages and tile descriptors ======
-    // Lane 0 takes items and issues the TMA; the warp copies each tile's list
-    // entries into its descriptor, so the row threads find them in shared memory.
+    // Lane 0 takes items (two per atomic, the next pair requested while the
+    // current one is set up) and issues the TMA; the warp copies each item's
+    // list entries straight into its tiles' descriptors, so the row threads
+    // find them in shared memory.
     const uint32_t n_items = __ldcg(&a.counters[0]);
-    const int tok_per_tile = kRows >> a.rshift;
+    const int tshift = 7 - a.rshift;  // tokens per tile = 128 / R = 1 << tshift
     const long long E = (long long)a.nq * a.S;
     int u = 0;
     bool ok = true;
-    // wait until ring slot u is free (whole warp, uniform result)
-    auto slot_free = [&]() -> bool {
-      bool f = true;
-      if (lane == 0 && u >= kTileRing)
-        f = wait_bar(&ctl.t_empty[u % kTileRing], (uint32_t)(((u / kTileRing) - 1) & 1), s_abort, lim);
-      return __shfl_sync(0xffffffffu, (int)f, 0) != 0;
-    };
+    uint32_t it0 = 0;
+    if (lane == 0) it0 = atomicAdd(&a.counters[1], 2u);
+    it0 = __shfl_sync(0xffffffffu, it0, 0);
 #pragma unroll 1
-    for (;;) {
-      uint32_t it = 0;
-      if (lane == 0) it = atomicAdd(&a.counters[1], 1u);
-      it = __shfl_sync(0xffffffffu, it, 0);
-      if (it >= n_items) break;
-      const int4 rec = __ldcg(&a.items[it]);
-      const int st = produced % kNst;
-      bool free_ok = true;
-      if (lane == 0 && produced >= kNst)
-        free_ok = wait_bar(&ctl.kv_empty[st], (uint32_t)(((produced / kNst) - 1) & 1), s_abort, lim);
-      if (!__shfl_sync(0xffffffffu, (int)free_ok, 0)) {
-        ok = false;
-        break;
-      }
-      if (lane == 0) {
-        uint8_t *dst = kv + st * 4 * kTile8;
-        const int row = (int)((long long)rec.x * a.bg_rows + (long long)rec.y * kBlk);
-        mbar_arrive_expect_tx(&ctl.kv_full[st], 4 * kTile8);
-        tc::tma_load_2d(dst, &mapK, 0, row, &ctl.kv_full[st]);
-        tc::tma_load_2d(dst + kTile8, &mapV, 0, row, &ctl.kv_full[st]);
-        tc::tma_load_2d(dst + 2 * kTile8, &mapK, 64, row, &ctl.kv_full[st]);
-        tc::tma_load_2d(dst + 3 * kTile8, &mapV, 64, row, &ctl.kv_full[st]);
-      }
-      const int kv_par = (produced / kNst) & 1;
-      ++produced;
-      const int n_tiles = (int)((((long long)rec.w << a.rshift) + kRows - 1) / kRows);
-      const uint32_t *src = a.list + (long long)rec.x * E + rec.z;
-      for (int m = 0; m < n_tiles; ++m) {
-        if (!slot_free()) {
+    while (ok && it0 < n_items) {
+      uint32_t it_next = 0;
+      if (lane == 0) it_next = atomicAdd(&a.counters[1], 2u);  // used one round later
+#pragma unroll 1
+      for (uint32_t it = it0; it < min(it0 + 2u, n_items) && ok; ++it) {
+        const int4 rec = __ldcg(&a.items[it]);
+        const int st = produced % kNst;
+        bool f = true;
+        if (lane == 0 && produced >= kNst)
+          f = wait_bar(&ctl.kv_empty[st], (uint32_t)(((produced / kNst) - 1) & 1), s_abort, lim);
+        if (!__shfl_sync(0xffffffffu, (int)f, 0)) {
           ok = false;
           break;
         }
-        TileDesc &d = ctl.desc[u % kTileRing];
-        const int n_tok = min(tok_per_tile, rec.w - m * tok_per_tile);
-        for (int e = lane; e < n_tok; e += 32) d.ent[e] = __ldg(src + m * tok_per_tile + e);
         if (lane == 0) {
-          d.bg = rec.x;
-          d.j = rec.y;
-          d.n_rows = n_tok << a.rshift;
-          d.stage = st;
-          d.kv_par = kv_par;
-          d.last = m == n_tiles - 1;
-          d.end = 0;
+          uint8_t *dst = kv + st * 4 * kTile8;
+          const int row = (int)((long long)rec.x * a.bg_rows + (long long)rec.y * kBlk);
+          mbar_arrive_expect_tx(&ctl.kv_full[st], 4 * kTile8);
+          tc::tma_load_2d(dst, &mapK, 0, row, &ctl.kv_full[st]);
+          tc::tma_load_2d(dst + kTile8, &mapV, 0, row, &ctl.kv_full[st]);
+          tc::tma_load_2d(dst + 2 * kTile8, &mapK, 64, row, &ctl.kv_full[st]);
+          tc::tma_load_2d(dst + 3 * kTile8, &mapV, 64, row, &ctl.kv_full[st]);
         }
-        __syncwarp();  // the lanes' entries are written before lane 0 publishes the slot
-        if (lane == 0) mbar_arrive(&ctl.t_full[u % kTileRing]);
-        ++u;
+        const int kv_par = (produced / kNst) & 1;
+        ++produced;
+        const int n_tiles = (rec.w + (1 << tshift) - 1) >> tshift;
+        // the item's tiles need free descriptor slots
+        for (int m = 0; m < n_tiles; ++m) {
+          const int v = u + m;
+          bool fr = true;
+          if (lane == 0 && v >= kTileRing)
+            fr = wait_bar(&ctl.t_empty[v % kTileRing], (uint32_t)(((v / kTileRing) - 1) & 1), s_abort, lim);
+          if (!__shfl_sync(0xffffffffu, (int)fr, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        const uint32_t *src = a.list + (long long)rec.x * E + rec.z;
+#pragma unroll 4
+        for (int e = lane; e < rec.w; e += 32)
+          ctl.desc[(u + (e >> tshift)) % kTileRing].ent[e & ((1 << tshift) - 1)] = __ldg(src + e);
+        if (lane == 0) {
+          for (int m = 0; m < n_tiles; ++m) {
+            TileDesc &d = ctl.desc[(u + m) % kTileRing];
+            d.bg = rec.x;
+            d.j = rec.y;
+            d.n_rows = min(1 << tshift, rec.w - (m << tshift)) << a.rshift;
+            d.stage = st;
+            d.kv_par = kv_par;
+            d.last = m == n_tiles - 1;
+            d.end = 0;
+          }
+        }
+        __syncwarp();  // the lanes' entries are written before lane 0 publishes the tiles
+        if (lane == 0)
+          for (int m = 0; m < n_tiles; ++m) mbar_arrive(&ctl.t_full[(u + m) % kTileRing]);
+        u += n_tiles;
       }
-      if (!ok) break;
+      it0 = __shfl_sync(0xffffffffu, it_next, 0);
     }
     // one end marker for each row warpgroup
     for (int e = 0; e < 2 && ok; ++e) {
-      if (!slot_free()) {
+      bool fr = true;
+      if (lane == 0 && u >= kTileRing)
+        fr = wait_bar(&ctl.t_empty[u % kTileRing], (uint32_t)(((u / kTileRing) - 1) & 1), s_abort, lim);
+      if (!__shfl_sync(0xffffffffu, (int)fr, 0)) {
         ok = false;
         break;
       }
@@ -463,20 +482,24 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     }
   } else {
     // ====== row warpgroups (warps 0-3: tiles 0, 2, ...; 4-7: 1, 3, ...) ======
-    const int w = warp >> 2;
+    // Thread r owns row r (TMEM lane r) for the softmax; the loads of query
+    // rows and the stores of partials are done by whole warps over their 32
+    // rows, eight lanes per 128-byte half row, so every access is whole lines.
+    const int w = warp >> 2, wq = warp & 3;
     const int r = tid & 127;                     // row of the tile = TMEM lane
-    const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t lane_sel = (uint32_t)(wq * 32) << 16;
     uint8_t *A = qa + w * 32768;
     uint8_t *P = pa + w * 16384;
     const int R = a.R;
     const int h = r & (R - 1);
     bool ok = true;
-    // the row's token: its block, position, query and partial slot
     struct Row {
       int end, valid, j, pos;
-      long long q_off, slot;
+      long long slot;
     };
-    auto read_desc = [&](int u, Row &row) -> bool {
+    // the tile's descriptor -> this row's token; its addresses go to the
+    // warpgroup's row table (parity par) for the warp-wide loads and stores
+    auto read_desc = [&](int u, int par, Row &row) -> bool {
       const int q = u % kTileRing;
       if (!wait_bar(&ctl.t_full[q], (uint32_t)((u / kTileRing) & 1), s_abort, lim)) return false;
       const TileDesc &d = ctl.desc[q];
@@ -492,23 +515,32 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       if (a.seq_len) qs = __ldg(&a.seq_len[b]) - a.nq;  // valid lengths only reach here
       row.pos = qs + i;
       const long long tok = (long long)b * a.nq + i;
-      row.q_off = (tok * a.G + g) * (long long)R * kD + (long long)h * kD;
       row.slot = ((tok * a.G + g) * a.S + s) * (long long)R + h;
+      RowAddr ra;
+      ra.src = row.valid ? a.Q + (tok * a.G + g) * (long long)R * kD + (long long)h * kD : nullptr;
+      ra.dst = row.valid ? a.po + row.slot * kD : nullptr;
+      ctl.rows[w][par][r] = ra;
       return true;
     };
-    auto gather = [&](const Row &row) {  // the row's query into the swizzled A tile
-      const uint16_t *src = a.Q + row.q_off;
+    // the warp's 32 query rows of the tile (parity par) into the swizzled A tile
+    auto gather = [&](int par) {
+      __syncwarp();  // the warp's row table entries are written
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        cp_async16(A + (c >> 3) * 16384 + tc::sw128_offset(r, (c & 7) * 8), src + c * 8,
-                   row.valid ? 16u : 0u);
+      for (int t = 0; t < 8; ++t) {
+        const int rr = wq * 32 + t * 4 + (lane >> 3), c = lane & 7;
+        const uint16_t *src = ctl.rows[w][par][rr].src;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+          cp_async16(A + hf * 16384 + tc::sw128_offset(rr, c * 8), src ? src + hf * 64 + c * 8 : a.Q,
+                     src ? 16u : 0u);
+      }
       cp_async_commit();
     };
     int u = w, k = 0;
     Row cur{}, nxt{};
-    ok = read_desc(u, cur);
+    ok = __all_sync(0xffffffffu, read_desc(u, 0, cur));
     if (ok && !cur.end) {
-      gather(cur);
+      gather(0);
       cp_async_wait_all();
       fence_proxy_async_smem();
       mbar_arrive(&ctl.a_ready[w]);
@@ -519,9 +551,9 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       ok = wait_bar(&ctl.s_full[w], (uint32_t)(k & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, read_desc(u + 2, nxt));
+      ok = __all_sync(0xffffffffu, read_desc(u + 2, (k + 1) & 1, nxt));
       if (!ok) break;
-      if (!nxt.end) gather(nxt);
+      if (!nxt.end) gather((k + 1) & 1);
       // ---- softmax of the row over the block's keys -> P ----
       tc::fence_after_sync();
       const int lim_key = cur.pos - cur.j * kBlk;  // keys after the token are masked
@@ -560,29 +592,48 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(&ctl.p_full[w]);
-      // ---- P V(u) -> the row's partial ----
+      // ---- P V(u) -> the partials, staged through P (free once P V is done) ----
       ok = wait_bar(&ctl.o_full[w], (uint32_t)(k & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc::fence_after_sync();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __half *dst = a.po + cur.slot * kD;
+      uint8_t *stg = P + wq * 4096;  // the warp's 32 rows x 128 bytes
+      const int par = k & 1;
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        float o[32];
-        tc::tmem_ld32(tmem + 128 + w * 128 + c0 + lane_sel, o);
-        if (cur.valid) {
+      for (int hf = 0; hf < 2; ++hf) {
+        float o[64];
+        {
+          float t[32];
+          tc::tmem_ld32(tmem + 128 + w * 128 + hf * 64 + lane_sel, t);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t hv[4];
+          for (int c = 0; c < 32; ++c) o[c] = t[c];
+          tc::tmem_ld32(tmem + 128 + w * 128 + hf * 64 + 32 + lane_sel, t);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __half2 hh = __floats2half2_rn(o[q * 8 + 2 * e] * inv_l, o[q * 8 + 2 * e + 1] * inv_l);
-              hv[e] = *reinterpret_cast<const uint32_t *>(&hh);
-            }
-            *reinterpret_cast<uint4 *>(dst + c0 + q * 8) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          }
+          for (int c = 0; c < 32; ++c) o[32 + c] = t[c];
         }
+        // this lane's half row -> staging (chunks rotated by row: no bank conflicts)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t hv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 hh = __floats2half2_rn(o[c * 8 + 2 * e] * inv_l, o[c * 8 + 2 * e + 1] * inv_l);
+            hv[e] = *reinterpret_cast<const uint32_t *>(&hh);
+          }
+          *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+        __syncwarp();
+        // whole 128-byte lines out: eight lanes per row, four rows per store
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int rl = t * 4 + (lane >> 3), c = lane & 7;
+          const uint4 v = *reinterpret_cast<const uint4 *>(stg + rl * 128 + ((c ^ (rl & 7)) << 4));
+          __half *dst = ctl.rows[w][par][wq * 32 + rl].dst;
+          if (dst) *reinterpret_cast<uint4 *>(dst + hf * 64 + c * 8) = v;
+        }
+        __syncwarp();  // staging is reused by the next half
       }
       if (cur.valid) a.ml[cur.slot] = make_float2(m, l);
       tc::fence_before_sync();
