@@ -307,7 +307,10 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     tc::prefetch_map(&mapK);
     tc::prefetch_map(&mapV);
   }
-  if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 512);  // S: 2 x 64 columns, O: 2 x 128
+  // TMEM: per warpgroup two 128-column regions, alternating by tile; a
+  // tile's S takes the first 64 columns of its region and its O (written
+  // after the softmax has read S) all 128
+  if (warp == 0) tc::tmem_alloc(&ctl.tmem_base, 512);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -335,9 +338,13 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     while (ok && it0 < n_items) {
       uint32_t it_next = 0;
       if (lane == 0) it_next = atomicAdd(&a.counters[1], 2u);  // used one round later
+      int4 recs[2];  // both records load together
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        recs[q] = it0 + q < n_items ? __ldcg(&a.items[it0 + q]) : make_int4(0, 0, 0, 0);
 #pragma unroll 1
       for (uint32_t it = it0; it < min(it0 + 2u, n_items) && ok; ++it) {
-        const int4 rec = __ldcg(&a.items[it]);
+        const int4 rec = recs[it - it0];
         const int st = produced % kNst;
         bool f = true;
         if (lane == 0 && produced >= kNst)
@@ -423,8 +430,9 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
 #pragma unroll 1
       while (total < 0 || n_p < total) {
         bool moved = false;
-        if (total < 0 && n_s - n_p < 2) {
+        if (total < 0 && n_s - n_p < 4) {
           const int q = n_s % kTileRing, w = n_s & 1;
+          const uint32_t reg = (uint32_t)(w * 256 + ((n_s >> 1) & 1) * 128);  // the tile's TMEM region
           if (mbar_test_wait(&ctl.t_full[q], (uint32_t)((n_s / kTileRing) & 1))) {
             if (ctl.desc[q].end) {
               total = n_s;
@@ -437,7 +445,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
               const uint64_t dK = tc::sdesc(kv + st * 4 * kTile8, 16, 1024);
 #pragma unroll
               for (int k = 0; k < 8; ++k)
-                tc::mma_bf16(tmem + w * 64, dA + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
+                tc::mma_bf16(tmem + reg, dA + (uint64_t)((k >> 2) * (16384 >> 4) + (k & 3) * 2),
                              dK + (uint64_t)((k >> 2) * (2 * kTile8 >> 4) + (k & 3) * 2), id_s, k > 0);
               tc::mma_commit(&ctl.s_full[w]);
               issued_s = ++n_s;
@@ -447,6 +455,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
         }
         if (n_p < n_s) {
           const int q = n_p % kTileRing, w = n_p & 1;
+          const uint32_t reg = (uint32_t)(w * 256 + ((n_p >> 1) & 1) * 128);
           if (mbar_test_wait(&ctl.p_full[w], (uint32_t)((n_p >> 1) & 1))) {
             tc::fence_after_sync();
             // the tile's descriptor stays in its slot until this product is issued
@@ -455,8 +464,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
             const uint64_t dV = tc::sdesc(kv + st * 4 * kTile8 + kTile8, 2 * kTile8, 1024);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              tc::mma_bf16(tmem + 128 + w * 128, dP + (uint64_t)(k * 2), dV + (uint64_t)(k * 128),
-                           id_o, k > 0);
+              tc::mma_bf16(tmem + reg, dP + (uint64_t)(k * 2), dV + (uint64_t)(k * 128), id_o, k > 0);
             tc::mma_commit(&ctl.o_full[w]);
             if (ctl.desc[q].last) tc::mma_commit(&ctl.kv_empty[st]);
             mbar_arrive(&ctl.t_empty[q]);
@@ -556,42 +564,52 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       if (!nxt.end) gather((k + 1) & 1);
       // ---- softmax of the row over the block's keys -> P ----
       tc::fence_after_sync();
+      const uint32_t reg = tmem + (uint32_t)(w * 256 + (k & 1) * 128) + lane_sel;  // S(u), then O(u)
       const int lim_key = cur.pos - cur.j * kBlk;  // keys after the token are masked
       float m = -INFINITY;
       {
-        float t[32];
+        float t[32], mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 32) {
-          tc::tmem_ld32(tmem + w * 64 + c0 + lane_sel, t);
+          tc::tmem_ld32(reg + c0, t);
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (c0 + c <= lim_key) m = fmaxf(m, t[c] * a.scale_log2);
+            if (c0 + c <= lim_key) mq[c & 3] = fmaxf(mq[c & 3], t[c]);
         }
+        m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * a.scale_log2;
       }
-      float l = 0.f;
+      float lq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c0 = 0; c0 < 64; c0 += 32) {
         float t[32];
-        tc::tmem_ld32(tmem + w * 64 + c0 + lane_sel, t);
+        tc::tmem_ld32(reg + c0, t);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int kk = c0 + c8 * 8 + 2 * e;
-            const float p0 = (cur.valid && kk <= lim_key) ? exp2f(t[c8 * 8 + 2 * e] * a.scale_log2 - m) : 0.f;
-            const float p1 = (cur.valid && kk + 1 <= lim_key) ? exp2f(t[c8 * 8 + 2 * e + 1] * a.scale_log2 - m) : 0.f;
+            const float p0 = (cur.valid && kk <= lim_key) ? exp2f(fmaf(t[c8 * 8 + 2 * e], a.scale_log2, -m)) : 0.f;
+            const float p1 = (cur.valid && kk + 1 <= lim_key) ? exp2f(fmaf(t[c8 * 8 + 2 * e + 1], a.scale_log2, -m)) : 0.f;
             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            l += __low2float(pb) + __high2float(pb);
+            lq[e] += __low2float(pb) + __high2float(pb);
             pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
           *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c0 + c8 * 8)) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
+      const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
       fence_proxy_async_smem();
       tc::fence_before_sync();
       mbar_arrive(&ctl.p_full[w]);
+      // ---- the next tile's query rows go to the MMA issuer now, so its S
+      // runs (in the other TMEM region) while P V(u) and the epilogue do ----
+      if (!nxt.end) {
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&ctl.a_ready[w]);
+      }
       // ---- P V(u) -> the partials, staged through P (free once P V is done) ----
       ok = wait_bar(&ctl.o_full[w], (uint32_t)(k & 1), s_abort, lim);
       ok = __all_sync(0xffffffffu, ok);
@@ -605,10 +623,10 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
         float o[64];
         {
           float t[32];
-          tc::tmem_ld32(tmem + 128 + w * 128 + hf * 64 + lane_sel, t);
+          tc::tmem_ld32(reg + hf * 64, t);
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = t[c];
-          tc::tmem_ld32(tmem + 128 + w * 128 + hf * 64 + 32 + lane_sel, t);
+          tc::tmem_ld32(reg + hf * 64 + 32, t);
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[32 + c] = t[c];
         }
@@ -637,14 +655,9 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       }
       if (cur.valid) a.ml[cur.slot] = make_float2(m, l);
       tc::fence_before_sync();
-      // ---- hand the next tile's rows to the MMA issuer ----
       cur = nxt;
       u += 2;
       ++k;
-      if (cur.end) break;
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&ctl.a_ready[w]);
     }
     cp_async_wait_all();  // no copy may still target the tiles when the CTA leaves
     if (!ok) *s_abort = 1;
