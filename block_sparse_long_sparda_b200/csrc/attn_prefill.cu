@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
         recs[q] = it0 + q < n_items ? __ldcg(&a.items[it0 + q]) : make_int4(0, 0, 0, 0);
 #pragma unroll 1
       for (uint32_t it = it0; it < min(it0 + 2u, n_items) && ok; ++it) {
-        const int4 rec = recs[it - it0];
+        const int4 rec = it == it0 ? recs[0] : recs[1];
         const int st = produced % kNst;
         bool f = true;
         if (lane == 0 && produced >= kNst)
@@ -566,38 +566,37 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       tc::fence_after_sync();
       const uint32_t reg = tmem + (uint32_t)(w * 256 + (k & 1) * 128) + lane_sel;  // S(u), then O(u)
       const int lim_key = cur.pos - cur.j * kBlk;  // keys after the token are masked
-      float m = -INFINITY;
+      float sv[64];
+      tc::tmem_ld64(reg, sv);
+      float m;
       {
-        float t[32], mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (lim_key >= kBlk - 1) {  // a block before the token's own: every key counts
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          tc::tmem_ld32(reg + c0, t);
+          for (int c = 0; c < 64; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+        } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c0 + c <= lim_key) mq[c & 3] = fmaxf(mq[c & 3], t[c]);
+          for (int c = 0; c < 64; ++c)
+            if (c <= lim_key) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
         }
         m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * a.scale_log2;
       }
+      // a row with no token (past the tile's rows) gets P = 0: exp2(x - inf)
+      const float msub = cur.valid ? m : INFINITY;
       float lq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c0 = 0; c0 < 64; c0 += 32) {
-        float t[32];
-        tc::tmem_ld32(reg + c0, t);
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t pk[4];
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kk = c0 + c8 * 8 + 2 * e;
-            const float p0 = (cur.valid && kk <= lim_key) ? exp2f(fmaf(t[c8 * 8 + 2 * e], a.scale_log2, -m)) : 0.f;
-            const float p1 = (cur.valid && kk + 1 <= lim_key) ? exp2f(fmaf(t[c8 * 8 + 2 * e + 1], a.scale_log2, -m)) : 0.f;
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            lq[e] += __low2float(pb) + __high2float(pb);
-            pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
-          }
-          *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c0 + c8 * 8)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int kk = c8 * 8 + 2 * e;
+          const float x0 = kk <= lim_key ? fmaf(sv[kk], a.scale_log2, -msub) : -INFINITY;
+          const float x1 = kk + 1 <= lim_key ? fmaf(sv[kk + 1], a.scale_log2, -msub) : -INFINITY;
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(tc::ex2_approx(x0), tc::ex2_approx(x1));
+          lq[e] += __low2float(pb) + __high2float(pb);
+          pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
         }
+        *reinterpret_cast<uint4 *>(P + tc::sw128_offset(r, c8 * 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
       fence_proxy_async_smem();
@@ -621,15 +620,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         float o[64];
-        {
-          float t[32];
-          tc::tmem_ld32(reg + hf * 64, t);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = t[c];
-          tc::tmem_ld32(reg + hf * 64 + 32, t);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[32 + c] = t[c];
-        }
+        tc::tmem_ld64(reg + hf * 64, o);
         // this lane's half row -> staging (chunks rotated by row: no bank conflicts)
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
