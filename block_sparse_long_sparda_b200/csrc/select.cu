@@ -37,455 +37,12 @@
 #include "common.cuh"
 #include "internal.h"
 #include "rank.cuh"
+#include "select_dev.cuh"
 #include "tc.cuh"
 
 namespace sparda {
 
 namespace {
-
-constexpr int kSelThreads = 256;
-constexpr int kMaxCand = 24576;   // candidates one problem may have (keys fit in shared memory)
-
-struct SelArgs {
-  const int32_t *seq_len;  // optional per-sequence lengths (decode: nq = 1)
-  const uint16_t *F;
-  const uint16_t *kc;
-  int32_t *idx;
-  uint32_t *counters;   // one ticket per problem (multi-chunk only)
-  uint32_t *failed;     // one flag per problem: a chunk's copy never landed (multi-chunk only)
-  uint32_t *cand_key;   // [problem][cap] score keys (multi-chunk only)
-  int32_t *status;      // optional device status word
-  int nq, G, nf, NB, k, n_init, n_local, q_start, S, T;
-  int CH, n_chunks, cap;
-  int NBf;       // window grid: blocks the key map covers (all three inner windows present)
-  int old_rank;  // 1: always the binned threshold search
-};
-
-// ---------------------------------------------------------------------------
-// block-wide helpers (blockDim.x == kSelThreads)
-// ---------------------------------------------------------------------------
-
-// ---------------------------------------------------------------------------
-// exact k-th largest key
-// ---------------------------------------------------------------------------
-// Every pass below splits the current members -- the keys inside one
-// contiguous key interval, all keys at first -- into 256 bins by a bin
-// function that is monotone in the key, so the keys of one bin again form an
-// interval and equal keys share a bin.  The bin that holds the wanted rank
-// becomes the next members.  The first pass bins linearly in score value
-// (for the usual bell-shaped scores the wanted bin then holds a handful of
-// keys); later passes bin linearly in key space, which cuts the key range
-// about 256-fold per pass, so at most six more passes reach a single key.
-// Once 32 or fewer members remain, one warp ranks them exactly.  A pass costs
-// four block barriers and a fixed number of conflict-free shared-memory
-// reads per thread; no step depends on another thread's atomic result.
-struct RankSmem {
-  uint32_t hist[256];
-  uint32_t wmin[kSelThreads / 32], wmax[kSelThreads / 32], wsum[kSelThreads / 32];
-  uint32_t list[32];
-  uint32_t units[64];      // packed per-(round row, warp) counts in compaction
-  uint32_t bstar, rem, cnt, n_list, tau, need, carry;
-};
-
-// The k-th largest of keys[0, n) (tau) and how many keys equal to it are
-// kept (need); 1 <= k < n.
-__device__ void find_threshold(const uint32_t *keys, int n, int k, RankSmem &sm, uint32_t &tau,
-                               int &need) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int nw = kSelThreads / 32;
-  Members mem{};
-  mem.all = true;
-  uint32_t rem = (uint32_t)k, m = (uint32_t)n;
-#pragma unroll 1
-  for (int pass = 0; pass < 12; ++pass) {
-    if (m <= 32u) {
-      // ---- exact rank of the last few members by one warp ----
-      if (tid == 0) sm.n_list = 0;
-      __syncthreads();
-      for (int e = tid; e < n; e += kSelThreads) {
-        const uint32_t u = keys[e];
-        if (mem.has(u)) {
-          const uint32_t slot = atomicAdd(&sm.n_list, 1u);
-          if (slot < 32u) sm.list[slot] = u;
-        }
-      }
-      __syncthreads();
-      if (warp == 0) {
-        const uint32_t cnt = min(sm.n_list, 32u);
-        const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
-        uint32_t gt = 0, ge = 0;
-        for (uint32_t j = 0; j < cnt; ++j) {
-          const uint32_t y = sm.list[j];
-          gt += y > x;
-          ge += y >= x;
-        }
-        if ((uint32_t)lane < cnt && gt < rem && ge >= rem) {
-          sm.tau = x;  // every lane holding this key writes the same values
-          sm.need = rem - gt;
-        }
-      }
-      __syncthreads();
-      tau = sm.tau;
-      need = (int)sm.need;
-      return;
-    }
-    // ---- key range of the members ----
-    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
-    for (int e = tid; e < n; e += kSelThreads) {
-      const uint32_t u = keys[e];
-      if (mem.has(u)) {
-        umin = min(umin, u);
-        umax = max(umax, u);
-      }
-    }
-    umin = __reduce_min_sync(0xffffffffu, umin);
-    umax = __reduce_max_sync(0xffffffffu, umax);
-    if (lane == 0) {
-      sm.wmin[warp] = umin;
-      sm.wmax[warp] = umax;
-    }
-    sm.hist[tid] = 0u;  // kSelThreads == 256 bins
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < nw; ++w) {
-      umin = min(umin, sm.wmin[w]);
-      umax = max(umax, sm.wmax[w]);
-    }
-    if (umin == umax) {  // the members are all one key
-      tau = umin;
-      need = (int)rem;
-      __syncthreads();  // wmin / wmax are rewritten by nobody after this
-      return;
-    }
-    // ---- bins over the members ----
-    const Members nx = make_bins(pass, umin, umax);
-    for (int e = tid; e < n; e += kSelThreads) {
-      const uint32_t u = keys[e];
-      if (mem.has(u)) atomicAdd(&sm.hist[nx.bin(u)], 1u);
-    }
-    __syncthreads();
-    // ---- the bin holding rank `rem` from the top: suffix sums over bins ----
-    const uint32_t h = sm.hist[tid];
-    uint32_t suf = h;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_down_sync(0xffffffffu, suf, o);
-      if (lane + o < 32) suf += t;
-    }
-    if (lane == 0) sm.wsum[warp] = suf;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < nw; ++w)
-      if (w > warp) suf += sm.wsum[w];
-    if (suf >= rem && suf - h < rem) {
-      sm.bstar = (uint32_t)tid;
-      sm.rem = rem - (suf - h);
-      sm.cnt = h;
-    }
-    __syncthreads();
-    mem = nx;
-    mem.b = sm.bstar;
-    rem = sm.rem;
-    m = sm.cnt;
-  }
-  // not reached: the key range is a single key after at most seven passes
-  tau = 0xFFFFFFFFu;
-  need = 0;
-}
-
-// The same threshold (tau, need) for k <= 64 and n <= 2048, with four block
-// barriers instead of a dozen: every warp sorts its 256 keys in registers
-// (a bitonic network, element q = 32*i + lane in register i, so partners
-// closer than 32 are a shuffle away and farther ones sit in the lane's own
-// registers), keeps its 64 largest, and three rounds of pairwise merges
-// reduce the 8 lists to the 64 largest keys of all.  tau is the k-th of
-// them and need counts how many keys equal to tau are kept; the
-// compaction then picks exactly the same entries as after find_threshold.
-// scratch: 1024 words of shared memory no one else is using.
-constexpr int kTopkMaxK = 64, kTopkMaxN = 8 * kSelThreads;
-
-__device__ __forceinline__ void cmp_swap_up(uint32_t &lo, uint32_t &hi, bool up) {
-  const uint32_t a = min(lo, hi), b = max(lo, hi);
-  lo = up ? a : b;
-  hi = up ? b : a;
-}
-
-// Sort m*32 keys held as v[i] (element 32*i + lane) ascending within runs of
-// `run` elements, the runs alternating direction as a bitonic network wants
-// (ascending where (q & run) == 0); run == m*32 gives one ascending run.
-template <int M>
-__device__ __forceinline__ void bitonic_warp(uint32_t (&v)[M], int lane, int k_from, int k_to) {
-#pragma unroll
-  for (int kk = k_from; kk <= k_to; kk <<= 1) {
-#pragma unroll
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      if (j >= 32) {
-        const int r = j >> 5;
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-          if (i & r) continue;
-          const int q = 32 * i + lane;
-          cmp_swap_up(v[i], v[i | r], (q & kk) == 0);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-          const int q = 32 * i + lane;
-          const uint32_t o = __shfl_xor_sync(0xffffffffu, v[i], j);
-          const bool up = (q & kk) == 0, lower = (lane & j) == 0;
-          v[i] = (up == lower) ? min(v[i], o) : max(v[i], o);
-        }
-      }
-    }
-  }
-}
-
-__device__ void find_threshold_topk(const uint32_t *keys, int n, int k, uint32_t *scratch,
-                                    RankSmem &sm, uint32_t &tau, int &need) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  {  // each warp: its 256 keys sorted ascending, the largest 64 to scratch
-    uint32_t v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = warp * 256 + 32 * i + lane;
-      v[i] = e < n ? keys[e] : 0u;  // 0 sorts below every finite score's key
-    }
-    bitonic_warp<8>(v, lane, 2, 256);
-    scratch[warp * 64 + lane] = v[6];
-    scratch[warp * 64 + 32 + lane] = v[7];
-  }
-  __syncthreads();
-  // merges: lists a and b (ascending) -> the 64 largest of both, ascending:
-  // c[x] = max(a[x], b[63 - x]) is bitonic and holds them, then one merge.
-  // Rounds read one half of the scratch and write the other.
-  uint32_t *src = scratch, *dst = scratch + 512;
-#pragma unroll 1
-  for (int lists = 8; lists > 1; lists >>= 1) {
-    if (warp < lists / 2) {
-      const uint32_t *a = src + (2 * warp) * 64, *b = src + (2 * warp + 1) * 64;
-      uint32_t c[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int x = 32 * i + lane;
-        c[i] = max(a[x], b[63 - x]);
-      }
-      bitonic_warp<2>(c, lane, 64, 64);
-      dst[warp * 64 + lane] = c[0];  // list `warp` of the next round
-      dst[warp * 64 + 32 + lane] = c[1];
-    }
-    __syncthreads();
-    uint32_t *t = src;
-    src = dst;
-    dst = t;
-  }
-  if (warp == 0) {
-    const uint32_t x0 = src[lane], x1 = src[32 + lane];  // ascending, x1 holds 32..63
-    const int pos = 64 - k;  // the k-th largest
-    const uint32_t t = src[pos];
-    const int gt = __popc(__ballot_sync(0xffffffffu, x0 > t)) + __popc(__ballot_sync(0xffffffffu, x1 > t));
-    if (lane == 0) {
-      sm.tau = t;
-      sm.need = (uint32_t)(k - gt);
-    }
-  }
-  __syncthreads();
-  tau = sm.tau;
-  need = (int)sm.need;
-}
-
-// Keep keys > tau plus the first `need` keys == tau (in entry order), in
-// entry order: out(pos, e) for each kept entry e, pos < limit.  Entries are
-// visited 32 consecutive ones per warp step; the position of each kept entry
-// comes from ballots inside the warp plus one block scan of per-warp counts
-// per round of 8 x 256 entries.  Returns the number kept.
-template <class Out>
-__device__ int compact_kept(const uint32_t *keys, int n, uint32_t tau, int need, int limit,
-                            RankSmem &sm, Out out) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  uint32_t carry = 0;  // packed (gt << 16 | eq) counts of earlier rounds
-#pragma unroll 1
-  for (int base = 0; base < n; base += 8 * kSelThreads) {
-    uint32_t bgt[8], beq[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = base + i * kSelThreads + tid;
-      const uint32_t u = e < n ? keys[e] : 0u;
-      bgt[i] = __ballot_sync(0xffffffffu, e < n && u > tau);
-      beq[i] = __ballot_sync(0xffffffffu, e < n && u == tau);
-      if (lane == 0) sm.units[i * 8 + warp] = ((uint32_t)__popc(bgt[i]) << 16) | (uint32_t)__popc(beq[i]);
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive scan of the 64 unit counts, two per lane
-      const uint32_t a0 = sm.units[2 * lane], a1 = sm.units[2 * lane + 1];
-      const uint32_t s = a0 + a1;
-      uint32_t x = s;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += t;
-      }
-      const uint32_t ex = carry + x - s;
-      sm.units[2 * lane] = ex;
-      sm.units[2 * lane + 1] = ex + a0;
-      if (lane == 31) sm.carry = carry + x;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t pre = sm.units[i * 8 + warp];
-      const uint32_t gt_b = (pre >> 16) + (uint32_t)__popc(bgt[i] & lt);
-      const uint32_t eq_b = (pre & 0xFFFFu) + (uint32_t)__popc(beq[i] & lt);
-      const bool gt = (bgt[i] >> lane) & 1u, eq = (beq[i] >> lane) & 1u;
-      if (gt || (eq && eq_b < (uint32_t)need)) {
-        const uint32_t pos = gt_b + min(eq_b, (uint32_t)need);
-        if (pos < (uint32_t)limit) out((int)pos, base + i * kSelThreads + tid);
-      }
-    }
-    carry = sm.carry;
-    __syncthreads();  // units / carry are rewritten by the next round
-  }
-  return min(limit, (int)((carry >> 16) + min(carry & 0xFFFFu, (uint32_t)need)));
-}
-
-// A block-list entry, stored with an L2 evict-last hint: the attention that
-// reads the list next streams hundreds of MB through L2 before it does, and
-// the list's 34 KB (B = 16) should still be there.
-__device__ __forceinline__ void st_list(int32_t *p, int v) {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(pol) : "memory");
-}
-
-// init | top-k | local | -1 padding.  With `fill_top`, the top-k part is the
-// first ntop candidates (every candidate is taken); otherwise it is written
-// by the caller.
-__device__ void write_set(int32_t *out, const BlockParts &bp, int ntop, int S, bool fill_top) {
-  const int nloc = bp.c - bp.local_lo + 1;
-  for (int s = threadIdx.x; s < S; s += kSelThreads) {
-    int v;
-    if (s < bp.init_hi) {
-      v = s;
-    } else if (s < bp.init_hi + ntop) {
-      if (!fill_top) continue;
-      v = bp.cand_lo + (s - bp.init_hi);
-    } else if (s < bp.init_hi + ntop + nloc) {
-      v = bp.local_lo + (s - bp.init_hi - ntop);
-    } else {
-      v = -1;
-    }
-    st_list(out + s, v);
-  }
-}
-
-// Butterfly transpose-reduce of 8 row partials over the 16 lanes of a
-// half-warp: 3 exchange stages on lane bits 3, 2, 1 and a final pairwise sum
-// leave the complete score of row (hl >> 1) in lanes hl and hl ^ 1.
-__device__ __forceinline__ float transpose_reduce8x16(float (&p)[8], int hl) {
-#pragma unroll
-  for (int half = 4; half >= 1; half >>= 1) {
-    const int lanebit = half * 2;
-    const bool up = (hl & lanebit) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = up ? p[i] : p[i + half];
-      const float keep = up ? p[i + half] : p[i];
-      p[i] = keep + __shfl_xor_sync(0xffffffffu, send, lanebit);
-    }
-  }
-  return p[0] + __shfl_xor_sync(0xffffffffu, p[0], 1);
-}
-
-__device__ __forceinline__ float dot8(const float *f, uint4 v) {
-  float s = f[0] * bf16_lo(v.x);
-  s = fmaf(f[1], bf16_hi(v.x), s);
-  s = fmaf(f[2], bf16_lo(v.y), s);
-  s = fmaf(f[3], bf16_hi(v.y), s);
-  s = fmaf(f[4], bf16_lo(v.z), s);
-  s = fmaf(f[5], bf16_hi(v.z), s);
-  s = fmaf(f[6], bf16_lo(v.w), s);
-  s = fmaf(f[7], bf16_hi(v.w), s);
-  return s;
-}
-
-// Score candidate rows [lo, lo+n) of Kc for this problem into keys[0, n).
-// The rows (contiguous, 256 B each) are streamed by the bulk-copy engine in
-// 128-row (32 KB) pieces through a kRing-deep shared-memory ring, so up to
-// 96 KB per CTA are in flight with no register cost; each half-warp scores 8
-// rows per piece from shared memory.  Returns false if a copy never landed
-// (bounded wait), in which case the keys are not valid.
-constexpr int kPieceRows = 128;
-constexpr int kPieceBytes = kPieceRows * kD * 2;
-constexpr int kRing = 3;
-
-__device__ __forceinline__ void issue_piece(const uint16_t *kc_bg, int lo, int n, int pc,
-                                            uint8_t *ring, uint64_t *bars) {
-  const int rows = min(kPieceRows, n - pc * kPieceRows);
-  uint64_t *bar = &bars[pc % kRing];
-  mbar_arrive_expect_tx(bar, (uint32_t)rows * kD * 2);
-  for (int r0 = 0; r0 < rows; r0 += 32)
-    bulk_g2s(ring + (pc % kRing) * kPieceBytes + r0 * kD * 2,
-             kc_bg + (long long)(lo + pc * kPieceRows + r0) * kD,
-             (uint32_t)min(32, rows - r0) * kD * 2, bar);
-}
-
-// thread 0, right after the barriers are initialised: the first pieces go
-// out before anything else is loaded
-__device__ __forceinline__ void prime_ring(const uint16_t *kc_bg, int lo, int n, uint8_t *ring,
-                                           uint64_t *bars) {
-  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
-  for (int pc = 0; pc < min(kRing, n_pc); ++pc) issue_piece(kc_bg, lo, n, pc, ring, bars);
-}
-
-// Block grid: key row r of the chunk scores block lo + r.
-__device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int lo, int n,
-                           uint32_t *keys, uint8_t *ring, uint64_t *bars) {
-  const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15;
-  const int n_pc = (n + kPieceRows - 1) / kPieceRows;
-  // the first pieces were issued by the caller's thread 0 right after the
-  // barriers were initialised; the rest are refills
-  bool ok = true;
-#pragma unroll 1
-  for (int pc = 0; pc < n_pc; ++pc) {
-    const bool landed = mbar_wait_bounded(&bars[pc % kRing], (uint32_t)((pc / kRing) & 1));
-    if (__syncthreads_or(!landed)) {
-      ok = false;
-      // let copies still in flight land (bounded) before the ring is released
-      if (threadIdx.x == 0)
-        for (int q = pc; q < min(n_pc, pc + kRing); ++q)
-          (void)mbar_wait_bounded(&bars[q % kRing], (uint32_t)((q / kRing) & 1));
-      __syncthreads();
-      break;
-    }
-    const int rows = min(kPieceRows, n - pc * kPieceRows);
-    const uint8_t *piece = ring + (pc % kRing) * kPieceBytes;
-    const int row0 = hw * 8;
-    uint4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      v[u] = row0 + u < rows ? *reinterpret_cast<const uint4 *>(piece + (row0 + u) * (kD * 2) + hl * 16)
-                             : make_uint4(0, 0, 0, 0);
-    float part[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) part[u] = 0.f;
-#pragma unroll 1
-    for (int f = 0; f < nf; ++f) {
-      float fv[8];
-      const float4 a = *reinterpret_cast<const float4 *>(fs + f * kD + hl * 8);
-      const float4 b = *reinterpret_cast<const float4 *>(fs + f * kD + hl * 8 + 4);
-      fv[0] = a.x; fv[1] = a.y; fv[2] = a.z; fv[3] = a.w;
-      fv[4] = b.x; fv[5] = b.y; fv[6] = b.z; fv[7] = b.w;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) part[u] += dot8(fv, v[u]);
-    }
-    const float sc = transpose_reduce8x16(part, hl);
-    const int r = row0 + (hl >> 1);
-    if ((hl & 1) == 0 && r < rows) keys[pc * kPieceRows + r] = orderable_key(sc);
-    __syncthreads();  // piece consumed by every half-warp
-    if (threadIdx.x == 0 && pc + kRing < n_pc) issue_piece(kc_bg, lo, n, pc + kRing, ring, bars);
-  }
-  return ok;
-}
 
 // Window grid (32-token windows at stride 16, four per 64-token block):
 // block j scores as the best of the three windows inside it, 4j, 4j+1 and
@@ -609,6 +166,20 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 
   pdl_trigger();
   pdl_wait();
+  if constexpr (kPool == 1) {  // the block grid: the item body shared with the attention tail
+    __shared__ int s_flags[2];
+    SelSmem sm;
+    sm.ring = ring;
+    sm.fs = fs;
+    sm.keys = dyn;
+    sm.rank_keys = dyn;
+    sm.scratch = reinterpret_cast<uint32_t *>(ring);
+    sm.bars = bars;
+    sm.rs = &rs;
+    sm.flags = s_flags;
+    select_block_item<kRing>(a, blockIdx.x, sm);
+    return;
+  }
   // problems are laid out chunk-fastest so a problem's chunks run together
   // and its merge overlaps the streaming of later problems
   const long long prob = blockIdx.x / a.n_chunks;
@@ -1143,6 +714,28 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
     pl.kc = pl.ncand_max;  // every candidate's key is kept for the final rank
     size_t off = 2 * (((size_t)pl.n_problems * 4 + 255) & ~(size_t)255);  // tickets, flags
     off += (((size_t)pl.n_problems * pl.n_chunks * CH * 4) + 255) & ~(size_t)255;  // keys
+    pl.ws_bytes = off;
+  }
+  return pl;
+}
+
+SelectPlan plan_select_tail(const sparda_params &p) {
+  SelectPlan pl{};
+  pl.n_problems = (long long)p.B * p.G;
+  const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
+  pl.ncand_max = bp.cand_hi - bp.cand_lo;
+  const int forced = tuning(p).select_chunk;
+  pl.CH = forced > 0 ? std::max(kSelThreads, (forced / kSelThreads) * kSelThreads) : kSelThreads;
+  pl.n_chunks = 1;
+  pl.kc = 0;
+  pl.tensor_scores = 0;
+  pl.ws_bytes = 0;
+  if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
+  pl.n_chunks = (int)ceil_div_ll(pl.ncand_max, pl.CH);
+  if (pl.n_chunks > 1) {
+    pl.kc = pl.ncand_max;
+    size_t off = 2 * (((size_t)pl.n_problems * 4 + 255) & ~(size_t)255);  // tickets, flags
+    off += (((size_t)pl.n_problems * pl.n_chunks * pl.CH * 4) + 255) & ~(size_t)255;  // keys
     pl.ws_bytes = off;
   }
   return pl;
