@@ -274,10 +274,6 @@ class DecodeLoop:
         op = abi.SPARDA_OP_SELECT_WINDOWS if w.windows else abi.SPARDA_OP_SELECT
         self.ws_sel = [abi.workspace(op, self.p, 1, 1) for _ in range(L)]
         self.ws_att = abi.workspace(abi.SPARDA_OP_ATTN_DECODE, self.p)
-        # one decode layer per call (attention + the next layer's selection);
-        # the block grid only
-        self.ws_layer = None if w.windows else \
-            [abi.workspace(abi.SPARDA_OP_DECODE_LAYER, self.p) for _ in range(L)]
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         # layer 0's set comes from the previous token's last layer
         self.select(L - 1)
@@ -336,23 +332,6 @@ class DecodeLoop:
             with torch.cuda.stream(self.main):
                 self.attention(l)
             self.main.wait_event(self.ev_sel[l])
-
-    def layer(self, l):
-        """Layer l in one call: attention(l) over its sets, and layer l's
-        Forecast vectors picking layer l+1's blocks, in one kernel."""
-        w, nxt = self.w, (l + 1) % self.w.layers
-        kv = self.kv[l]
-        self.abi.sparda_decode_layer(self.p, self.Q[l], kv, kv.view(-1)[w.blk * w.d:],
-                                     w.NB * self.blk_elems, self.blk_elems, self.idx[l],
-                                     self.abi.SPARDA_ADDR_LOGICAL, self.O[l], self.F[l],
-                                     self.kc[nxt], self.idx[nxt], self.ws_layer[l], self.status)
-
-    def step_fused(self):
-        """One decode token through the L layers, one launch per layer on the
-        current stream: each attention kernel's thread blocks run the next
-        layer's selection once their share of the attention is done."""
-        for l in range(self.w.layers):
-            self.layer(l)
 
     # ---- host offload: K/V in pinned host memory, gathered into slots ----
     def _setup_host(self):
@@ -740,38 +719,19 @@ def run_sparda(args):
         # no launch gaps inside the timed region.  A graph of GRAPH_STEPS
         # consecutive steps (the step has no host dependency) pays one graph
         # launch per GRAPH_STEPS steps; single-step replays make up the rest.
-        # two forms of the same step: one launch per layer (attention, with
-        # the next layer's selection in its tail), and select(l) on a side
-        # stream beside attention(l); the faster one, measured here, is timed
-        def capture(fn):
-            torch.cuda.synchronize()
-            g1 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g1, stream=loop.main):
-                fn()
-            g1.replay()
-            gm = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gm, stream=loop.main):
-                for _ in range(GRAPH_STEPS):
-                    fn()
-            gm.replay()
-            torch.cuda.synchronize()
-            return g1, gm
-        variants = {}
-        forms = {"two_streams": loop.step_resident}
-        if loop.ws_layer is not None:
-            forms["one_launch_per_layer"] = loop.step_fused
-            for _ in range(max(args.warmup, 3)):
-                loop.step_fused()
-        step_path = "two_streams"
         step, graph, graph_m = loop.step_resident, None, None
         try:
-            graphs = {name: capture(fn) for name, fn in forms.items()}
-            for _ in range(2):  # alternate the forms, keep each one's best
-                for name, (g1, gm) in graphs.items():
-                    t = time_steps(lambda: [gm.replay() for _ in range(4)], 1, world) / (4 * GRAPH_STEPS)
-                    variants[name] = min(variants.get(name, 1e30), t * 1e3)
-            step_path = min(variants, key=variants.get)
-            graph, graph_m = graphs[step_path]
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=loop.main):
+                loop.step_resident()
+            graph.replay()
+            graph_m = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_m, stream=loop.main):
+                for _ in range(GRAPH_STEPS):
+                    loop.step_resident()
+            graph_m.replay()
+            torch.cuda.synchronize()
             step = graph.replay
         except Exception as exc:  # keep eager launches, and say so in the line
             print("note: graph capture failed (%s); timing eager launches" % exc, file=sys.stderr)
@@ -896,10 +856,7 @@ def run_sparda(args):
                        "G": w.G, "d": w.d, "block": w.blk, "k": w.k, "n_init": w.n_init,
                        "n_local": w.n_local, "parallelism": "replicas" if world > 1 else "single",
                        "kv": "all layers resident in HBM (34.4 GB), read by block id",
-                       "streams": "one launch per layer: attention(l), its thread blocks then "
-                                  "run the selection of layer l+1's blocks"
-                                  if step_path == "one_launch_per_layer" else
-                                  "select(l) on a side stream beside attention(l); "
+                       "streams": "select(l) on a side stream beside attention(l); "
                                   "attention(l+1) waits for both",
                        "l2": "inputs larger than L2: 281 MB of selected K/V per layer, 4 layers"},
             "select_us_per_layer": sel_us,
@@ -917,9 +874,7 @@ def run_sparda(args):
             "cpu_baseline": cpu,
             "prefill": prefill,
             "sweep": sweep,
-            "gpu_launches": args.steps * L * (1 if step_path == "one_launch_per_layer" else 2),
-            "step_path": step_path,
-            "step_variants_us": {k_: round(v, 2) for k_, v in variants.items()},
+            "gpu_launches": args.steps * L * 2,
             "cuda_graph": graph is not None,
             "graph_steps": GRAPH_STEPS if graph_m is not None else 1,
             "device_status": st,

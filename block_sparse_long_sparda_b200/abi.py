@@ -37,7 +37,6 @@ SPARDA_OP_ATTN_PREFILL = 4
 SPARDA_OP_SELECT_WINDOWS = 5
 SPARDA_OP_HEAD_SOFTMAX = 6
 SPARDA_OP_HEAD_SOFTMAX_WINDOWS = 7
-SPARDA_OP_DECODE_LAYER = 8
 
 SPARDA_ADDR_LOGICAL = 0
 SPARDA_ADDR_SLOT = 1
@@ -104,7 +103,6 @@ _SIGS = {
     "sparda_prefetch_blocks": (_I, [_PP, _P, _P, _P, _I, _I, _P, _P]),
     "sparda_sparse_attn_decode": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_prefill": (_I, [_PP, _P, _I, _I, _P, _P, _LL, _LL, _P, _P, _P, _SZ, _P, _P]),
-    "sparda_decode_layer": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "sparda_sparse_attn_decode_noalloc": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _P]),
     "sparda_cache_plan": (_I, [_PP, _I, _P, _P, _P, _P, _P, _P, _P]),
     "sparda_prefetch_cached": (_I, [_PP, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
@@ -243,15 +241,6 @@ def sparda_sparse_attn_decode(p, Q, K, V, bg_stride, blk_stride, idx, addr_mode,
                                            int(bg_stride), int(blk_stride), _ptr(idx),
                                            int(addr_mode), _ptr(O), _ptr(ws), _nbytes(ws),
                                            _ptr(dev_status), _stream(stream)))
-
-
-def sparda_decode_layer(p, Q, K, V, bg_stride, blk_stride, idx, addr_mode, O, F_next, kc_next,
-                        idx_next, ws, dev_status=None, stream=None):
-    _check("sparda_decode_layer",
-           lib().sparda_decode_layer(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), int(bg_stride),
-                                     int(blk_stride), _ptr(idx), int(addr_mode), _ptr(O),
-                                     _ptr(F_next), _ptr(kc_next), _ptr(idx_next), _ptr(ws),
-                                     _nbytes(ws), _ptr(dev_status), _stream(stream)))
 
 
 def sparda_sparse_attn_prefill(p, Q, nq, q_start, K, V, bg_stride, tok_stride, idx, O, ws,

@@ -135,8 +135,6 @@ size_t sparda_workspace_size(int op, const sparda_params *p, int nq, int nf) {
       return plan_decode(*p).ws_bytes;
     case SPARDA_OP_ATTN_PREFILL:
       return nq < 1 ? 0 : prefill_ws_bytes(*p, nq);
-    case SPARDA_OP_DECODE_LAYER:
-      return plan_decode_layer(*p).ws_bytes;
     default:
       return 0;
   }
@@ -314,33 +312,6 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
                                       static_cast<const uint16_t *>(V), bg_stride, blk_stride,
                                       idx, addr_mode, static_cast<uint16_t *>(O), ws, dev_status,
                                       reinterpret_cast<cudaStream_t>(stream)));
-}
-
-int sparda_decode_layer(const sparda_params *p, const void *Q, const void *K, const void *V,
-                        long long bg_stride, long long blk_stride, const int32_t *idx,
-                        int addr_mode, void *O, const void *F_next, const void *kc_next,
-                        int32_t *idx_next, void *ws, size_t ws_bytes, int32_t *dev_status,
-                        sparda_stream_t stream) {
-  int st = check_params(p);
-  if (st != SPARDA_OK) return st;
-  if (addr_mode != SPARDA_ADDR_LOGICAL && addr_mode != SPARDA_ADDR_SLOT) return SPARDA_EINVAL;
-  if (p->B == 0) return SPARDA_OK;
-  if (!Q || !K || !V || !idx || !O || !F_next || !kc_next || !idx_next) return SPARDA_EINVAL;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O) ||
-      !aligned16(F_next) || !aligned16(kc_next) || !aligned16(idx_next))
-    return SPARDA_EINVAL;
-  if (idx_next == idx) return SPARDA_EINVAL;
-  if (!stride_ok(bg_stride) || !stride_ok(blk_stride) || blk_stride < (long long)kBlk * kD)
-    return SPARDA_EINVAL;
-  const DecodeLayerPlan dl = plan_decode_layer(*p);
-  if (!dl.fused && !select_supported(plan_select(*p, 1, 1))) return SPARDA_EUNSUPPORTED;
-  if (!ws || ws_bytes < dl.ws_bytes || !aligned16(ws)) return SPARDA_EWORKSPACE;
-  return from_cuda(launch_decode_layer(
-      *p, dl, static_cast<const uint16_t *>(Q), static_cast<const uint16_t *>(K),
-      static_cast<const uint16_t *>(V), bg_stride, blk_stride, idx, addr_mode,
-      static_cast<uint16_t *>(O), static_cast<const uint16_t *>(F_next),
-      static_cast<const uint16_t *>(kc_next), idx_next, ws, dev_status,
-      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // ---- device slot cache ----------------------------------------------------

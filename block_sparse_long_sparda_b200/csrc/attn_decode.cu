@@ -49,7 +49,6 @@
 
 #include "common.cuh"
 #include "internal.h"
-#include "select_dev.cuh"
 #include "tc.cuh"
 
 namespace sparda {
@@ -120,61 +119,7 @@ struct TcArgs {
                         // picks the kernel instance, 2 or 3 stages)
   float scale_log2;
   long long wait_cycles;  // bound of every wait of the pipeline, in SM clock cycles
-  // the next layer's Forecast selection, run by each CTA once its attention
-  // range is done (decode layer calls): items = problems x chunks, taken from
-  // sel_ctr[0]; sel_ctr[1] counts the CTAs that are done, and the last resets both
-  SelArgs sel;
-  uint32_t *sel_ctr;
-  long long sel_items;
 };
-
-// Shared memory of the selection tail: [0, 64 KB) a two-piece ring, then the
-// Forecast vector, the chunk's keys, the ranking scratch, barriers and flags
-// -- all below the attention's control block (at NSTAGE x 32 KB + 8 KB), so
-// no late mbarrier arrival of the attention pipeline can land in them.
-constexpr int kTailRing = 2;
-constexpr int kTailMaxCH = 512;      // candidates per selection chunk
-constexpr int kTailMaxCand = 2048;   // candidates per problem (their keys are ranked in the ring)
-struct TailSmem {
-  float fs[kD];
-  uint32_t keys[kTailMaxCH];
-  RankSmem rs;
-  uint64_t bars[kTailRing];
-  int flags[2];
-  long long item;
-};
-static_assert(kTailRing * kPieceBytes + sizeof(TailSmem) <= 2 * kUnitBytes + 8192,
-              "the selection tail must stay below the attention's control block");
-
-// Threads 0-255 take selection items until none is left; warp 8 takes no part.
-__device__ void select_tail(const TcArgs &a, uint8_t *smem) {
-  if (threadIdx.x >= kSelThreads) return;
-  TailSmem &ts = *reinterpret_cast<TailSmem *>(smem + kTailRing * kPieceBytes);
-  SelSmem sm;
-  sm.ring = smem;
-  sm.fs = ts.fs;
-  sm.keys = ts.keys;
-  sm.rank_keys = reinterpret_cast<uint32_t *>(smem);             // 8 KB, once the ring is idle
-  sm.scratch = reinterpret_cast<uint32_t *>(smem + kPieceBytes);  // 4 KB, in the second piece
-  sm.bars = ts.bars;
-  sm.rs = &ts.rs;
-  sm.flags = ts.flags;
-  for (;;) {
-    sel_sync();  // the previous item is done with the ring, barriers and item slot
-    if (threadIdx.x == 0) ts.item = (long long)atomicAdd(&a.sel_ctr[0], 1u);
-    sel_sync();
-    const long long item = ts.item;
-    if (item >= a.sel_items) break;
-    select_block_item<kTailRing>(a.sel, item, sm);
-  }
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&a.sel_ctr[1], 1u) == gridDim.x - 1) {  // the last CTA: counters back to zero
-      a.sel_ctr[0] = 0u;
-      a.sel_ctr[1] = 0u;
-    }
-  }
-}
 
 // Memory index (b * nq + i) * G + g of the pair at stream position p.  With
 // several query tokens (prefill) the pairs are streamed group by group, so
@@ -353,7 +298,7 @@ __device__ __forceinline__ void seg_flush(const TcArgs &a, long long pair, bool 
 // (S^T, softmax, O^T): a stage is held from its landing until its O^T MMA is
 // done, and more chains hide that hold better.  Sixteen heads per group need
 // more registers than three CTAs per SM allow.
-template <int R, int NSTAGE, bool SPLIT, bool FUSE>
+template <int R, int NSTAGE, bool SPLIT>
 __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    const __grid_constant__ TcArgs a) {
@@ -379,17 +324,10 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   const long long e0 = (long long)blockIdx.x * E / NC;
   const long long e1 = (long long)(blockIdx.x + 1) * E / NC;
   pdl_trigger();
-  if (e0 >= e1) {  // no attention work: only the selection tail
-    if constexpr (FUSE) {
-      pdl_wait();
-      select_tail(a, smem_raw);
-    }
-    return;
-  }
+  if (e0 >= e1) return;
   if (smem_addr(smem_raw) & 1023u) {  // the swizzled tiles would be misread
     pdl_wait();
     if (tid == 0) flag_status(a.status, SPARDA_DEV_LAYOUT);
-    if constexpr (FUSE) select_tail(a, smem_raw);
     return;
   }
   const long long pair0 = e0 / a.S;
@@ -800,14 +738,13 @@ __global__ void __launch_bounds__(kWsThreads, (R <= 8 && NSTAGE <= 2) ? 3 : 2)
   __syncthreads();
   tc::fence_after_sync();
   if (warp == 0) tc::tmem_dealloc(tmem, 64);
-  if constexpr (FUSE) select_tail(a, smem_raw);
 }
 
-template <int R, int NSTAGE, bool SPLIT, bool FUSE = false>
+template <int R, int NSTAGE, bool SPLIT>
 cudaError_t launch_tc(const CUtensorMap &mk, const CUtensorMap &mv, const TcArgs &a,
                       long long grid_max, long long grid_min, int forced, cudaStream_t stream) {
   constexpr size_t smem = tc_smem<NSTAGE, SPLIT>();
-  auto kern = attn_tc_kernel<R, NSTAGE, SPLIT, FUSE>;
+  auto kern = attn_tc_kernel<R, NSTAGE, SPLIT>;
   // per device, once: shared-memory attributes and how many CTAs stay
   // resident (one wave: as many CTAs as the device keeps resident, never
   // more than the plan sized the workspace for, never fewer than the lists
@@ -973,95 +910,6 @@ cudaError_t launch_gather_attn(const sparda_params &p, const DecodePlan &pl, int
   if (stages == 3) return launch_tc<RR, 3, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
   if (stages == 4) return launch_tc<RR, 4, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
   return launch_tc<RR, 6, false>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream);
-  switch (R) {
-    case 1: SPARDA_LAUNCH_R(1)
-    case 2: SPARDA_LAUNCH_R(2)
-    case 4: SPARDA_LAUNCH_R(4)
-    case 8: SPARDA_LAUNCH_R(8)
-    case 16: SPARDA_LAUNCH_R(16)
-    default: return cudaErrorInvalidValue;
-  }
-#undef SPARDA_LAUNCH_R
-}
-
-DecodeLayerPlan plan_decode_layer(const sparda_params &p) {
-  DecodeLayerPlan dl{};
-  dl.att = plan_decode(p);
-  dl.sel = plan_select_tail(p);
-  const int R = p.G > 0 ? p.Hq / p.G : 1;
-  const int stages = ring_stages(p);
-  // the tail runs in the non-split two- or three-stage instances; its chunk
-  // keys and, for a multi-chunk problem, every candidate's key must fit the
-  // shared memory it may use
-  dl.fused = tuning(p).attn_split_kv <= 0 && (stages == 2 || stages == 3) &&
-             (R == 1 || R == 2 || R == 4 || R == 8 || R == 16) && dl.sel.CH <= kTailMaxCH &&
-             dl.sel.ncand_max <= kTailMaxCand;
-  size_t off = (dl.att.ws_bytes + 255) & ~(size_t)255;
-  dl.sel_off = off;
-  off += (dl.sel.ws_bytes + 255) & ~(size_t)255;
-  dl.ctr_off = off;
-  off += 256;  // the tail's item and done counters
-  dl.ws_bytes = off;
-  return dl;
-}
-
-cudaError_t launch_decode_layer(const sparda_params &p, const DecodeLayerPlan &dl,
-                                const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                                long long bg_stride, long long blk_stride, const int32_t *idx,
-                                int addr_mode, uint16_t *O, const uint16_t *F_next,
-                                const uint16_t *kc_next, int32_t *idx_next, void *ws,
-                                int32_t *dev_status, cudaStream_t stream) {
-  char *w = static_cast<char *>(ws);
-  if (!dl.fused) {  // two launches on the stream: this layer's attention, then the selection
-    const cudaError_t e = launch_attn_decode(p, dl.att, Q, K, V, bg_stride, blk_stride, idx,
-                                             addr_mode, O, w, dev_status, stream);
-    if (e != cudaSuccess) return e;
-    return launch_select(p, plan_select(p, 1, 1), F_next, 1, 1, p.T - 1, kc_next, idx_next,
-                         w + dl.sel_off, dev_status, stream);
-  }
-  if ((long long)p.B * p.G == 0) return cudaSuccess;
-  const int R = p.Hq / p.G;
-  TcArgs a;
-  CUtensorMap mk, mv;
-  const cudaError_t eb = build_tc(p, dl.att, 1, p.T - 1, Q, K, V, bg_stride, blk_stride, idx,
-                                  addr_mode, O, w, dev_status, nullptr, 0, a, mk, mv);
-  if (eb != cudaSuccess) return eb;
-  // the next layer's selection (Forecast, one vector per group, block grid)
-  SelArgs &sa = a.sel;
-  const SelectPlan &sp = dl.sel;
-  sa.seq_len = p.seq_len;
-  sa.T = p.T;
-  sa.F = F_next;
-  sa.kc = kc_next;
-  sa.idx = idx_next;
-  sa.nq = 1;
-  sa.G = p.G;
-  sa.nf = 1;
-  sa.NB = (p.T + kBlk - 1) / kBlk;
-  sa.k = p.k;
-  sa.n_init = p.n_init;
-  sa.n_local = p.n_local;
-  sa.q_start = p.T - 1;
-  sa.S = p.k + p.n_init + p.n_local;
-  sa.CH = sp.CH;
-  sa.n_chunks = sp.n_chunks;
-  sa.cap = sp.n_chunks * sp.CH;
-  sa.NBf = 0;
-  sa.old_rank = tuning(p).select_binned != 0 ? 1 : 0;
-  sa.status = dev_status;
-  char *ws_sel = w + dl.sel_off;
-  const size_t words = ((size_t)sp.n_problems * 4 + 255) & ~(size_t)255;
-  sa.counters = reinterpret_cast<uint32_t *>(ws_sel);
-  sa.failed = reinterpret_cast<uint32_t *>(ws_sel + words);
-  sa.cand_key = reinterpret_cast<uint32_t *>(ws_sel + 2 * words);
-  a.sel_ctr = reinterpret_cast<uint32_t *>(w + dl.ctr_off);
-  a.sel_items = sp.n_problems * sp.n_chunks;
-  const int stages = ring_stages(p);
-  const int fc = tuning(p).attn_ctas;
-  const DecodePlan &pl = dl.att;
-#define SPARDA_LAUNCH_R(RR)                                                                           \
-  if (stages <= 2) return launch_tc<RR, 2, false, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream); \
-  return launch_tc<RR, 3, false, true>(mk, mv, a, pl.n_cta, pl.n_cta_min, fc, stream);
   switch (R) {
     case 1: SPARDA_LAUNCH_R(1)
     case 2: SPARDA_LAUNCH_R(2)

@@ -142,27 +142,6 @@ cudaError_t launch_attn_decode(const sparda_params &p, const DecodePlan &plan,
                                cudaStream_t stream, const int32_t *phys = nullptr,
                                int n_slots = 0);
 
-// ---- one decode layer: attention, and the next layer's selection in the
-// attention kernel's tail (attn_decode.cu) ----------------------------------
-// the selection plan of the tail: chunks of sparda_tuning::select_chunk (else
-// 256) candidates, all items taken dynamically by the attention CTAs
-SelectPlan plan_select_tail(const sparda_params &p);
-struct DecodeLayerPlan {
-  DecodePlan att;
-  SelectPlan sel;
-  bool fused;       // one launch; else attention then selection
-  size_t sel_off;   // the selection's part of the workspace
-  size_t ctr_off;   // the tail's two counters
-  size_t ws_bytes;
-};
-DecodeLayerPlan plan_decode_layer(const sparda_params &p);
-cudaError_t launch_decode_layer(const sparda_params &p, const DecodeLayerPlan &dl,
-                                const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                                long long bg_stride, long long blk_stride, const int32_t *idx,
-                                int addr_mode, uint16_t *O, const uint16_t *F_next,
-                                const uint16_t *kc_next, int32_t *idx_next, void *ws,
-                                int32_t *dev_status, cudaStream_t stream);
-
 // ---- device slot cache (cache.cu) -------------------------------------------
 constexpr int kMaxCacheSlots = 4096;
 cudaError_t launch_cache_plan(const sparda_params &p, int C, const int32_t *idx,

@@ -719,28 +719,6 @@ SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool) {
   return pl;
 }
 
-SelectPlan plan_select_tail(const sparda_params &p) {
-  SelectPlan pl{};
-  pl.n_problems = (long long)p.B * p.G;
-  const BlockParts bp = block_parts(p.T - 1, kBlk, p.n_init, p.n_local);
-  pl.ncand_max = bp.cand_hi - bp.cand_lo;
-  const int forced = tuning(p).select_chunk;
-  pl.CH = forced > 0 ? std::max(kSelThreads, (forced / kSelThreads) * kSelThreads) : kSelThreads;
-  pl.n_chunks = 1;
-  pl.kc = 0;
-  pl.tensor_scores = 0;
-  pl.ws_bytes = 0;
-  if (pl.ncand_max <= p.k || p.k == 0 || pl.n_problems == 0) return pl;
-  pl.n_chunks = (int)ceil_div_ll(pl.ncand_max, pl.CH);
-  if (pl.n_chunks > 1) {
-    pl.kc = pl.ncand_max;
-    size_t off = 2 * (((size_t)pl.n_problems * 4 + 255) & ~(size_t)255);  // tickets, flags
-    off += (((size_t)pl.n_problems * pl.n_chunks * pl.CH * 4) + 255) & ~(size_t)255;  // keys
-    pl.ws_bytes = off;
-  }
-  return pl;
-}
-
 int select_supported(const SelectPlan &pl) {
   if (pl.tensor_scores) return 1;
   if (pl.CH > kMaxCand) return 0;

@@ -145,8 +145,7 @@ enum sparda_op {
   SPARDA_OP_ATTN_PREFILL = 4,
   SPARDA_OP_SELECT_WINDOWS = 5,
   SPARDA_OP_HEAD_SOFTMAX = 6,         /* sparda_head_softmax_select (nq = 1)         */
-  SPARDA_OP_HEAD_SOFTMAX_WINDOWS = 7, /* sparda_head_softmax_select_windows (nq = 1) */
-  SPARDA_OP_DECODE_LAYER = 8          /* sparda_decode_layer                          */
+  SPARDA_OP_HEAD_SOFTMAX_WINDOWS = 7  /* sparda_head_softmax_select_windows (nq = 1) */
 };
 
 /* how sparda_sparse_attn_decode finds the storage of list entry s */
@@ -382,41 +381,6 @@ int sparda_sparse_attn_decode(const sparda_params *p, const void *Q, const void 
                               const void *V, long long bg_stride, long long blk_stride,
                               const int32_t *idx, int addr_mode, void *O, void *ws,
                               size_t ws_bytes, int32_t *dev_status, sparda_stream_t stream);
-
-/*
- * sparda_decode_layer -- one decode layer of the pipelined loop in one call:
- * this layer's sparse attention over the sets it was given (exactly
- * sparda_sparse_attn_decode), and the Forecast selection of the next layer's
- * block sets (exactly sparda_forecast_select with nq = nf = 1, the query at
- * T - 1 or each sequence's last token).
- *   [p4 "The fourth projection", Algorithm 2]: at layer l, F_l picks
- *   B_{l+1} while layer l attends over B_l; [p4 "One Forecast head per GQA
- *   group"]: the selection is taken off the critical path of attention.
- * The two need nothing from each other, so they share one kernel: each
- * attention thread block, once its share of the attention is done, takes
- * chunks of the selection from a counter in the workspace; the selection
- * fills the time the attention's blocks spend finishing unevenly, and needs
- * no launch of its own.  Shapes whose selection does not fit the attention
- * kernel's shared memory (more than 2048 candidate blocks, chunks of more
- * than 512), or tuning that selects another attention instance, run as the
- * two calls one after the other on the stream, with the same results.
- * Q, K, V, bg_stride, blk_stride, idx, addr_mode, O: as for
- *        sparda_sparse_attn_decode (SPARDA_ADDR_LOGICAL or SPARDA_ADDR_SLOT)
- * F_next  bf16 [B][G][d]: the Forecast vector of each (sequence, group)
- * kc_next bf16 [B][G][NB][d]: the compressed keys of the next layer
- * idx_next int32 [B][G][S] (out): the next layer's sets, as sparda_forecast_select
- *        writes them; must not alias idx
- * ws     sparda_workspace_size(SPARDA_OP_DECODE_LAYER, p, 1, 1) bytes,
- *        zero-filled before its first use; each call leaves its tickets and
- *        counters at zero again.  Calls sharing a workspace must not overlap.
- * dev_status  as for the two calls (SPARDA_DEV_RANGE, SPARDA_DEV_TIMEOUT).
- * Chunk size of the selection: sparda_tuning::select_chunk (else 256).
- */
-int sparda_decode_layer(const sparda_params *p, const void *Q, const void *K, const void *V,
-                        long long bg_stride, long long blk_stride, const int32_t *idx,
-                        int addr_mode, void *O, const void *F_next, const void *kc_next,
-                        int32_t *idx_next, void *ws, size_t ws_bytes, int32_t *dev_status,
-                        sparda_stream_t stream);
 
 /*
  * sparda_sparse_attn_prefill -- every token of a query chunk attends over the

@@ -41,18 +41,11 @@ def _check_kc_bits(gpu_bits, ora_bits, what):
     assert same >= 0.999 and diff <= 1, "%s: bf16 Kc identical %.5f, max diff %d ulp" % (what, same, diff)
 
 
-@pytest.mark.parametrize("form", ["two_streams", "one_launch_per_layer"])
-def test_decode_loop_full_size_sampled(form):
-    """The bench's step in both forms: select(l) beside attention(l) on two
-    streams, and one sparda_decode_layer launch per layer (the selection in
-    the attention kernel's tail)."""
+def test_decode_loop_full_size_sampled():
     import bench
     w = bench.WORKLOAD
     loop = bench.DecodeLoop(w, with_host=False)
-    if form == "two_streams":
-        loop.step_resident()  # select(l -> l+1) beside attention(l), for the four layers
-    else:
-        loop.step_fused()
+    loop.step_resident()  # select(l -> l+1) beside attention(l), for the four layers
     torch.cuda.synchronize()
     assert int(loop.status.item()) == 0
     L, R, d, blk, NB, T = w.layers, w.r, w.d, w.blk, w.NB, w.T

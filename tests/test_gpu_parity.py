@@ -1346,88 +1346,3 @@ def test_prefill_block_major_skips_and_flags_bad_ids():
     clean[0, 20, 0, 3] = -1
     ora = oracle.sparse_attention(Q, K, V, clean, T - nq, T)
     check_attention(got, ora, "bad ids skipped")
-
-
-# --------------------------------------------------------------------------
-# one decode layer in one call: attention + the next layer's selection
-# --------------------------------------------------------------------------
-
-def _decode_layer_case(B, G, R, T, k, seed, lens=None, tune=None, n_init=1, n_local=2, calls=2):
-    """Run sparda_decode_layer `calls` times on one workspace and check each
-    call's attention output and next-layer sets against the oracle."""
-    rng = W.rng_for(seed, T + R)
-    d = 128
-    K = W.normal_bf16(rng, (B, G, T, d))
-    V = W.normal_bf16(rng, (B, G, T, d))
-    Q = W.normal_bf16(rng, (B, G * R, d))
-    F = W.normal_bf16(rng, (B, 1, G, 1, d))        # this layer's sets come from F
-    F2 = W.normal_bf16(rng, (B, 1, G, 1, d))       # F2 picks the next layer's sets
-    NB = (T + 63) // 64
-    kc_next = W.normal_bf16(rng, (B, G, NB, d))
-    _, kcb = oracle.compress_keys(K)
-    sl = None if lens is None else torch.tensor(lens, dtype=torch.int32, device="cuda")
-    p = abi.make_params(B, G * R, G, T, k, n_init, n_local, seq_len=sl, tune=tune)
-    S = k + n_init + n_local
-    ws = guarded_workspace(abi.SPARDA_OP_DECODE_LAYER, p)
-    Kd, Vd, Qd = dev_bf16(K), dev_bf16(V), dev_bf16(Q)
-    L = [T] * B if lens is None else lens
-    idx_this = np.full((B, G, S), -1, np.int32)
-    for b, Lb in enumerate(L):
-        if 1 <= Lb <= T:
-            o, _, _ = oracle.select(F[b:b + 1], np.ascontiguousarray(kcb[b:b + 1, :, :(Lb + 63) // 64]),
-                                    k, n_init, n_local, Lb - 1)
-            idx_this[b] = o[0, 0]
-    didx = torch.from_numpy(idx_this).cuda()
-    for call in range(calls):
-        O = Guarded((B, G * R, d), torch.bfloat16, fill=float("nan"))
-        nxt = Guarded((B, G, S), torch.int32, fill=-7)
-        st = torch.zeros(1, dtype=torch.int32, device="cuda")
-        abi.sparda_decode_layer(p, Qd, Kd, Vd, T * d, 64 * d, didx, abi.SPARDA_ADDR_LOGICAL, O.t,
-                                dev_bf16(F2.reshape(B, G, d)), dev_bf16(kc_next), nxt.t,
-                                ws.t, st)
-        got_o = host_bits(O.check("layer output"))
-        got_i = nxt.check("next sets").cpu().numpy()
-        ws.check("layer workspace")
-        word = int(st.item())
-        for b, Lb in enumerate(L):
-            what = "call %d b %d" % (call, b)
-            if not 1 <= Lb <= T:
-                assert np.all(got_i[b] == -1) and np.all(got_o[b] == 0), what
-                continue
-            assert not (got_i[b] == -7).any(), what
-            kcl = np.ascontiguousarray(kc_next[b:b + 1, :, :(Lb + 63) // 64])
-            ora, kth, kth1 = oracle.select(F2[b:b + 1], kcl, k, n_init, n_local, Lb - 1)
-            check_sets(got_i[b:b + 1].reshape(1, 1, G, S), ora, kth, kth1, scores_f64(F2[b:b + 1], kcl),
-                       what, q_pos=Lb - 1, n_init=n_init, n_local=n_local)
-            ora_o = oracle.sparse_attention(Q[b:b + 1].reshape(1, 1, G * R, d),
-                                            np.ascontiguousarray(K[b:b + 1, :, :Lb]),
-                                            np.ascontiguousarray(V[b:b + 1, :, :Lb]),
-                                            idx_this[b:b + 1].reshape(1, 1, G, S), Lb - 1, Lb)
-            check_attention(got_o[b:b + 1].reshape(1, 1, G * R, d), ora_o, what)
-        if lens is None:
-            assert word == 0, word
-        else:
-            assert abi.sparda_status_from_device(word) == abi.SPARDA_ERANGE
-
-
-@pytest.mark.parametrize("B,G,R,T,k", [(1, 2, 8, 4096, 4), (4, 8, 4, 32768, 32), (2, 2, 16, 20000 + 37, 40),
-                                        (3, 2, 1, 9000, 100), (2, 8, 4, 131072, 64)])
-def test_decode_layer_matches_oracle(B, G, R, T, k):
-    """Attention and the next layer's selection in one launch: single- and
-    multi-chunk problems, 1 to 16 heads per group (the two- and three-stage
-    kernel instances), the bench's own shape (2045 candidates in 8 chunks),
-    two calls on one workspace (tickets and counters back at zero)."""
-    _decode_layer_case(B, G, R, T, k, 46)
-
-
-def test_decode_layer_with_lengths_and_an_invalid_one():
-    _decode_layer_case(4, 2, 4, 20000, 16, 47, lens=[20000, 3000 + 17, 70, 0])
-
-
-@pytest.mark.parametrize("tune", [{"select_chunk": 512}, {"select_chunk": 1024}, {"attn_split_kv": 1},
-                                  {"select_binned": 1}])
-def test_decode_layer_chunkings_and_the_two_launch_path(tune):
-    """Chunks of 512 candidates; and tunings that keep the selection out of
-    the attention kernel (chunks above 512, the split ring), which run the
-    same two computations as two launches."""
-    _decode_layer_case(2, 4, 4, 40000, 24, 48, tune=tune)
