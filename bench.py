@@ -396,8 +396,9 @@ class DecodeLoop:
         """C slots per (layer, b, g); the Forecast vectors of step t+1 are
         those of step t plus sigma * N(0, 1) noise, so consecutive steps
         select mostly the same blocks (a drift model of consecutive tokens;
-        sigma = 0 keeps the sets fixed).  The per-step Forecast vectors sit
-        in pinned host memory and are uploaded in the timed step."""
+        sigma = 0 keeps the sets fixed).  Each step's inputs -- the queries
+        and Forecast vectors of every layer -- sit packed in pinned host
+        memory, one buffer per step, and cross the link as one copy."""
         torch, w = self.torch, self.w
         L, dev = w.layers, torch.device("cuda")
         self.C = C
@@ -409,66 +410,105 @@ class DecodeLoop:
         gen = torch.Generator()
         gen.manual_seed(seed)
         F = self.F.float().cpu()
+        q = self.Q.cpu().reshape(-1)
+        self.n_q = q.numel()
         steps = []
         for _ in range(n_steps):
-            steps.append(F.to(torch.bfloat16))
+            steps.append(torch.cat([q, F.to(torch.bfloat16).reshape(-1)]))
             F = F + sigma * torch.randn(F.shape, generator=gen)
-        self.h_F_steps = torch.stack(steps).pin_memory()
+        self.h_in = torch.stack(steps).pin_memory()          # [step][Q | F]
+        self.d_in = torch.empty(2, self.h_in.shape[1], dtype=torch.bfloat16, device=dev)
+        self.d_out = torch.empty((2,) + tuple(self.O.shape), dtype=torch.bfloat16, device=dev)
+        self.h_out = torch.empty(self.O.shape, dtype=torch.bfloat16).pin_memory()
         self.copy = torch.cuda.Stream()
-        self.ev_in0, self.ev_out = torch.cuda.Event(), torch.cuda.Event()
-        self.q_ev = [torch.cuda.Event() for _ in range(L)]
-        self.o_ev = [torch.cuda.Event() for _ in range(L)]
+        # the selection, plan and fetch of the next layer go first: its thread
+        # blocks take SMs ahead of the attention's, so the fetch of the misses
+        # overlaps the attention instead of following it
+        self.sel_hi = torch.cuda.Stream(priority=-1)
+        self.ev_begin, self.ev_o = torch.cuda.Event(), torch.cuda.Event()
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_dl = [torch.cuda.Event() for _ in range(2)]
+        self._recorded = set()
+
+    def step_inputs(self, t: int):
+        """(Q, F, O) of step t: views of the step's device buffers."""
+        w, b = self.w, t % 2
+        Q = self.d_in[b, :self.n_q].view(self.Q.shape)
+        F = self.d_in[b, self.n_q:].view(self.F.shape)
+        return Q, F, self.d_out[b]
+
+    def begin_cached(self, t: int):
+        """Before a run of cached steps from step t: upload step t's inputs
+        (each step uploads the next step's)."""
+        self.d_in[t % 2].copy_(self.h_in[t % self.h_in.shape[0]])
+        self.torch.cuda.synchronize()
+        self._recorded = set()
+
+    def end_cached(self, t_next: int):
+        """After a run of cached steps: join the copies still in flight (the
+        next step's inputs, the last step's outputs)."""
+        main = self.torch.cuda.current_stream()
+        for ev in (("in", t_next % 2), ("dl", (t_next - 1) % 2)):
+            if ev in self._recorded:
+                main.wait_event((self.ev_in if ev[0] == "in" else self.ev_dl)[ev[1]])
+        self._recorded = set()
 
     def step_e2e_cached(self, t: int):
         """One decode step through the C ABI with the K/V cache in pinned host
-        memory and a device slot cache: upload this step's Q and Forecast
-        vectors; per layer, select the next layer's blocks, plan them against
-        the next layer's slots and fetch only the misses, all on the side
-        stream while this layer attends from its slots; read O back.  The
-        step ends once the next step's layer-0 blocks have landed, so a step
-        can be captured into a CUDA graph on its own."""
+        memory and a device slot cache.  Per layer, one launch selects the
+        next layer's blocks, plans them against that layer's slots and
+        copies only the misses from the host, on a high-priority stream,
+        while this layer attends from its slots.  Step t's inputs were
+        uploaded during step t-1 (begin_cached for the first); this step
+        uploads step t+1's into the other buffer and sends its outputs back
+        while the next step runs.  Runs of steps are captured into one CUDA
+        graph."""
         torch, abi, w = self.torch, self.abi, self.w
         L, C = w.layers, self.C
         main = torch.cuda.current_stream()
-        # inputs: the Forecast vectors first (select needs them at once); each
-        # layer's queries on a copy stream ahead of that layer's attention
-        self.F.copy_(self.h_F_steps[t % self.h_F_steps.shape[0]], non_blocking=True)
-        self.ev_in0.record(main)
-        self.copy.wait_event(self.ev_in0)
+        cur, oth = t % 2, (t + 1) % 2
+        if ("in", cur) in self._recorded:
+            main.wait_event(self.ev_in[cur])
+        if ("dl", cur) in self._recorded:  # step t-2's outputs have left this buffer
+            main.wait_event(self.ev_dl[cur])
+        # step t+1's inputs go into the other buffer, which step t-1 no longer reads
+        self.ev_begin.record(main)
+        self.copy.wait_event(self.ev_begin)
         with torch.cuda.stream(self.copy):
-            for l in range(L):
-                self.Q[l].copy_(self.h_Q[l], non_blocking=True)
-                self.q_ev[l].record(self.copy)
+            self.d_in[oth].copy_(self.h_in[(t + 1) % self.h_in.shape[0]], non_blocking=True)
+            self.ev_in[oth].record(self.copy)
+        self._recorded.add(("in", oth))
+        Q, F, O = self.step_inputs(t)
         for l in range(L):
             nxt = (l + 1) % L
-            # select(l), the plan and the fetch of layer l+1 run on the side
-            # stream while attention(l) runs; both need layer l-1 finished
             self.ev_pre[l].record(main)
-            self.side.wait_event(self.ev_pre[l])
-            with torch.cuda.stream(self.side):
-                abi.sparda_forecast_select(self.p, self.F[l], 1, 1, w.T - 1, self.kc[nxt],
-                                           self.idx[nxt], self.ws_sel[l], self.status)
-                abi.sparda_cache_plan(self.p, C, self.idx[nxt], self.block_of[nxt],
-                                      self.hand[nxt], self.phys[nxt], self.fetch[nxt],
-                                      self.status)
-                abi.sparda_prefetch_cached(self.p, C, self.host_kv[nxt], self.idx[nxt],
-                                           self.phys[nxt], self.fetch[nxt], self.cache[nxt], 0,
-                                           self.status)
-                self.fetch_ev[nxt].record(self.side)
+            self.sel_hi.wait_event(self.ev_pre[l])
+            with torch.cuda.stream(self.sel_hi):
+                abi.sparda_forecast_select_cached(self.p, F[l], 1, w.T - 1, self.kc[nxt],
+                                                  self.idx[nxt], self.ws_sel[l], C,
+                                                  self.block_of[nxt], self.hand[nxt],
+                                                  self.phys[nxt], self.fetch[nxt],
+                                                  self.host_kv[nxt], self.cache[nxt],
+                                                  self.status)
+                self.fetch_ev[nxt].record(self.sel_hi)
             if l > 0:  # layer 0's blocks were joined at the end of the previous step
                 main.wait_event(self.fetch_ev[l])
-            main.wait_event(self.q_ev[l])
-            abi.sparda_sparse_attn_decode_cached(self.p, C, self.Q[l], self.cache[l],
-                                                 self.idx[l], self.phys[l], self.O[l],
-                                                 self.ws_att, self.status)
-            # this layer's output goes back while the next layers run
-            self.o_ev[l].record(main)
-            self.copy.wait_event(self.o_ev[l])
-            with torch.cuda.stream(self.copy):
-                self.h_O[l].copy_(self.O[l], non_blocking=True)
-        self.ev_out.record(self.copy)
+            abi.sparda_sparse_attn_decode_cached(self.p, C, Q[l], self.cache[l], self.idx[l],
+                                                 self.phys[l], O[l], self.ws_att, self.status)
+        # the outputs go back while the next step runs
+        self.ev_o.record(main)
+        self.copy.wait_event(self.ev_o)
+        with torch.cuda.stream(self.copy):
+            self.h_out.copy_(O, non_blocking=True)
+            self.ev_dl[cur].record(self.copy)
+        self._recorded.add(("dl", cur))
         main.wait_event(self.fetch_ev[0])
-        main.wait_event(self.ev_out)
+
+    def cached_steps(self, t0: int, n: int):
+        """Steps t0 .. t0+n-1 back to back (one graph when captured)."""
+        for t in range(t0, t0 + n):
+            self.step_e2e_cached(t)
+        self.end_cached(t0 + n)
 
     def prime_cache(self):
         """Cold start: plan and fetch layer 0's current set."""
@@ -899,7 +939,9 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
     """The e2e loop with a device slot cache (2S slots per layer and group)
     under a few drift rates of the Forecast vectors between decode steps:
     per-step time, the share of top-k blocks that still cross the host
-    link, and the step time against the all-resident step."""
+    link, and the step time against the all-resident step.  Timed as one
+    CUDA graph of the timed steps (each uploads the next step's inputs and
+    sends its outputs back), after a warm-up graph of the steps before."""
     import torch
     w = loop.w
     L = w.layers
@@ -907,36 +949,37 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
     e_steps = max(3, min(args.steps, 10))
     warm = max(args.warmup, 3)
     for sigma in (0.0, 0.01, 0.03, 0.1):
-        n = warm + 2 * e_steps + 2
+        n = warm + 2 * e_steps + 1
         loop.setup_cache(2 * w.S, sigma, n)
-        loop.prime_cache()
-        # one CUDA graph per step (each uploads its own step's Forecast
-        # vectors), so host launch overhead stays out of the step
-        graphs = []
+        loop.prime_cache()  # one eager step first: every launch's one-time setup is done
+        loop.begin_cached(0)
+        loop.cached_steps(0, 1)
+        torch.cuda.synchronize()
         cap = torch.cuda.Stream()
+        graphs = []
         with torch.cuda.stream(cap):
-            for i in range(n):
+            for t0, cnt in ((0, warm), (warm, e_steps)):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=cap):
-                    loop.step_e2e_cached(i)
+                    loop.cached_steps(t0, cnt)
                 graphs.append(g)
         torch.cuda.synchronize()
         loop.block_of.fill_(-1)   # capture enqueued nothing; start the cache cold again
         loop.hand.zero_()
         loop.prime_cache()
-        t = [0]
-
-        def step():
-            graphs[t[0]].replay()
-            t[0] += 1
-        for _ in range(warm):
-            step()
-        ms = time_steps(step, e_steps, world) / e_steps
-        # the fetched share, measured on the steps that follow (untimed)
+        loop.begin_cached(0)
+        graphs[0].replay()
+        ms = time_steps(graphs[1].replay, 1, world) / e_steps
+        # the fetched share, on the steps that follow (run eagerly, untimed)
         fetched = 0
-        for _ in range(e_steps):
-            step()
+        t0 = warm + e_steps
+        loop.begin_cached(t0)
+        for t in range(t0, t0 + e_steps):
+            loop.step_e2e_cached(t)
+            torch.cuda.synchronize()
             fetched += int(loop.fetch.sum().item())
+        loop.end_cached(t0 + e_steps)
+        torch.cuda.synchronize()
         del graphs
         per_step = fetched / e_steps
         topk_entries = L * w.B * w.G * w.k
@@ -944,9 +987,12 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
                     "ms_per_step": ms, "fetched_blocks_per_step": per_step,
                     "fetched_frac_of_topk": per_step / topk_entries,
                     "host_link_bytes_per_step": int(per_step * loop.blk_elems * 2),
+                    "h2d_bytes_per_step": int(loop.h_in.shape[1] * 2),
+                    "d2h_bytes_per_step": int(loop.h_out.numel() * 2),
                     "step_vs_resident": ms / resident_ms,
                     "exposed_wait_us_per_layer": (ms - resident_ms) * 1e3 / L})
-        del loop.cache, loop.block_of, loop.hand, loop.phys, loop.fetch, loop.h_F_steps
+        del loop.cache, loop.block_of, loop.hand, loop.phys, loop.fetch, loop.h_in, loop.d_in
+        del loop.d_out, loop.h_out
         torch.cuda.empty_cache()
     return out
 

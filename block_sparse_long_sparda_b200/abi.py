@@ -106,6 +106,8 @@ _SIGS = {
     "sparda_sparse_attn_decode_noalloc": (_I, [_PP, _P, _P, _P, _LL, _LL, _P, _I, _P, _P, _P]),
     "sparda_cache_plan": (_I, [_PP, _I, _P, _P, _P, _P, _P, _P, _P]),
     "sparda_prefetch_cached": (_I, [_PP, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "sparda_forecast_select_cached": (_I, [_PP, _P, _I, _I, _P, _P, _P, _SZ, _I, _P, _P, _P,
+                                           _P, _P, _P, _P, _P]),
     "sparda_sparse_attn_decode_cached": (_I, [_PP, _I, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "sparda_workspace_size": (_SZ, [_I, _PP, _I, _I]),
     "sparda_status_string": (ctypes.c_char_p, [_I]),
@@ -279,6 +281,16 @@ def sparda_prefetch_cached(p, C, host_kv, idx, phys, fetch, cache, n_ctas=0, dev
            lib().sparda_prefetch_cached(ctypes.byref(p), int(C), _ptr(host_kv), _ptr(idx),
                                         _ptr(phys), _ptr(fetch), _ptr(cache), int(n_ctas),
                                         _ptr(dev_status), _stream(stream)))
+
+
+def sparda_forecast_select_cached(p, F, nf, q_start, kc, idx, ws, C, block_of, hand, phys,
+                                  fetch, host_kv, cache, dev_status=None, stream=None):
+    _check("sparda_forecast_select_cached",
+           lib().sparda_forecast_select_cached(ctypes.byref(p), _ptr(F), int(nf), int(q_start),
+                                               _ptr(kc), _ptr(idx), _ptr(ws), _nbytes(ws), int(C),
+                                               _ptr(block_of), _ptr(hand), _ptr(phys), _ptr(fetch),
+                                               _ptr(host_kv), _ptr(cache), _ptr(dev_status),
+                                               _stream(stream)))
 
 
 def sparda_sparse_attn_decode_cached(p, C, Q, cache, idx, phys, O, ws, dev_status=None,

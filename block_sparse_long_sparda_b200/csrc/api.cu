@@ -360,6 +360,40 @@ int sparda_prefetch_cached(const sparda_params *p, int C, const void *host_kv,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int sparda_forecast_select_cached(const sparda_params *p, const void *F, int nf, int q_start,
+                                  const void *kc, int32_t *idx, void *ws, size_t ws_bytes, int C,
+                                  int32_t *block_of, int32_t *hand, int32_t *phys, int32_t *fetch,
+                                  const void *host_kv, void *cache, int32_t *dev_status,
+                                  sparda_stream_t stream) {
+  int st = check_params(p);
+  if (st != SPARDA_OK) return st;
+  if (nf < 1 || q_start < 0 || q_start >= p->T) return SPARDA_EINVAL;
+  if (nf > 16) return SPARDA_EUNSUPPORTED;
+  if (!cache_args_ok(p, C)) return SPARDA_EINVAL;
+  if (p->B == 0) return SPARDA_OK;
+  if (!F || !kc || !idx || !block_of || !hand || !phys || !fetch || !host_kv || !cache)
+    return SPARDA_EINVAL;
+  if (!aligned16(F) || !aligned16(kc) || !aligned16(idx) || !aligned16(host_kv) ||
+      !aligned16(cache))
+    return SPARDA_EINVAL;
+  const uint16_t *dev_view = mapped_device_view(host_kv);
+  if (!dev_view) return SPARDA_EINVAL;
+  const SelectPlan pl = plan_select(*p, 1, nf);
+  if (!select_supported(pl) || pl.tensor_scores) return SPARDA_EUNSUPPORTED;
+  if (pl.ws_bytes > 0 && (!ws || ws_bytes < pl.ws_bytes || !aligned16(ws))) return SPARDA_EWORKSPACE;
+  SelCache cc;
+  cc.C = C;
+  cc.block_of = block_of;
+  cc.hand = hand;
+  cc.phys = phys;
+  cc.fetch = fetch;
+  cc.cache = static_cast<uint16_t *>(cache);
+  cc.host_kv = dev_view;
+  return from_cuda(launch_select(*p, pl, static_cast<const uint16_t *>(F), 1, nf, q_start,
+                                 static_cast<const uint16_t *>(kc), idx, ws, dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream), 1, &cc));
+}
+
 int sparda_sparse_attn_decode_cached(const sparda_params *p, int C, const void *Q,
                                      const void *cache, const int32_t *idx, const int32_t *phys,
                                      void *O, void *ws, size_t ws_bytes, int32_t *dev_status,

@@ -76,6 +76,18 @@ struct SelectPlan {
   int tensor_scores;     // 1: chunk of query tokens scored by the tcgen05 product
   size_t ws_bytes;
 };
+// The slot cache of the cached decode selection (C == 0: none): per (b, g)
+// C slots of one layer, their blocks and clock hand, the step's slot map and
+// fetch flags, and the device view of the mapped host K|V blocks.
+struct SelCache {
+  int C;
+  int32_t *block_of;        // [B][G][C]
+  int32_t *hand;            // [B][G]
+  int32_t *phys;            // [B][G][S]
+  int32_t *fetch;           // [B][G][S]
+  uint16_t *cache;          // [B][G][C][2][blk][d]
+  const uint16_t *host_kv;  // [B][G][NB][2][blk][d]
+};
 // pool = 1: one compressed key per block; pool = 4: the window grid (32-token
 // windows at stride 16), a block scoring as the best window inside it
 SelectPlan plan_select(const sparda_params &p, int nq, int nf, int pool = 1);
@@ -91,7 +103,8 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
 int select_supported(const SelectPlan &plan);
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &plan, const uint16_t *F,
                           int nq, int nf, int q_start, const uint16_t *kc, int32_t *idx,
-                          void *ws, int32_t *status, cudaStream_t stream, int pool = 1);
+                          void *ws, int32_t *status, cudaStream_t stream, int pool = 1,
+                          const SelCache *cache = nullptr);
 
 // the original selector's per-head softmax form (decode: one query token);
 // pool as plan_select

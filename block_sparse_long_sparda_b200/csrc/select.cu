@@ -150,7 +150,7 @@ __device__ void score_tail_windows(const uint16_t *kw_bg, const float *fs, int n
   __syncthreads();
 }
 
-template <int kPool>
+template <int kPool, bool kCached = false>
 __global__ void __launch_bounds__(kSelThreads, 2)
     select_kernel(const __grid_constant__ CUtensorMap mapW, SelArgs a) {
   // dynamic shared memory, the ring aligned to 128 bytes by hand (a TMA
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 
   pdl_trigger();
   pdl_wait();
-  if constexpr (kPool == 1) {  // the block grid: the item body shared with the attention tail
+  if constexpr (kPool == 1) {  // the block grid (select_dev.cuh), optionally with the slot cache
     __shared__ int s_flags[2];
     SelSmem sm;
     sm.ring = ring;
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kSelThreads, 2)
     sm.bars = bars;
     sm.rs = &rs;
     sm.flags = s_flags;
-    select_block_item<kRing>(a, blockIdx.x, sm);
+    select_block_item<kRing, kCached>(a, blockIdx.x, sm);
     return;
   }
   // problems are laid out chunk-fastest so a problem's chunks run together
@@ -728,7 +728,7 @@ int select_supported(const SelectPlan &pl) {
 
 cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const uint16_t *F, int nq,
                           int nf, int q_start, const uint16_t *kc, int32_t *idx, void *ws,
-                          int32_t *status, cudaStream_t stream, int pool) {
+                          int32_t *status, cudaStream_t stream, int pool, const SelCache *cache) {
   if (pl.n_problems == 0) return cudaSuccess;
   if (pl.tensor_scores)
     return launch_select_prefill(p, F, nq, q_start, kc, idx, ws, status, stream, pool);
@@ -755,6 +755,13 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
   a.counters = nullptr;
   a.cand_key = nullptr;
   a.old_rank = tuning(p).select_binned != 0 ? 1 : 0;
+  a.cc = SelCache{};
+  if (cache) {  // decode on the block grid only, with the step's words inside the ring
+    if (pool != 1 || nq != 1 || cache->C < a.S ||
+        cache_step_words(cache->C, a.S) * 4 > (long long)kRing * kPieceBytes)
+      return cudaErrorNotSupported;
+    a.cc = *cache;
+  }
   // window grid: key rows [B*G][NW][d] as (dims, window in block, block, (b, g)),
   // three of every four windows, blocks up to NW / 4 (all three windows inside)
   CUtensorMap mW{};
@@ -779,13 +786,13 @@ cudaError_t launch_select(const sparda_params &p, const SelectPlan &pl, const ui
     smem = 128 + (size_t)kRing * kPieceBytes + (size_t)nf * kD * 4 +
            (size_t)std::max(pl.CH, pl.ncand_max) * 4;
   }
-  auto kern = pool == 1 ? select_kernel<1> : select_kernel<4>;
-  {  // raised once per device and pooling to the largest size used; most
+  auto kern = cache ? select_kernel<1, true> : pool == 1 ? select_kernel<1> : select_kernel<4>;
+  {  // raised once per device and kernel to the largest size used; most
      // shared memory goes to the ring, so prefer the largest carveout
-    static size_t raised[2][64] = {{0}};
+    static size_t raised[3][64] = {{0}};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    size_t &r = raised[pool == 1 ? 0 : 1][dev];
+    size_t &r = raised[cache ? 2 : pool == 1 ? 0 : 1][dev];
     if (r < smem) {
       cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;

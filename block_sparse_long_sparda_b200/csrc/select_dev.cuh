@@ -1,16 +1,14 @@
-// select_dev.cuh -- device pieces of the Forecast block selection, shared by
-// the selection kernel (select.cu) and the tail of the decode attention
-// kernel (attn_decode.cu), which runs the next layer's selection in the same
-// launch.
+// select_dev.cuh -- device pieces of the Forecast block selection on the
+// block grid: the work of one (problem, chunk) item, and the slot-cache step
+// the cached decode selection runs once a (b, g)'s set is written.
 //
 // Pages cited: [p4 <section>] = the article "SparDA: a fourth projection that
 // lets sparse attention prefetch its own KV cache" (ai.thesatyajit.com).
 // [p4 "The fourth projection", Eq. 4]: B_{l+1} = B_init U B_local U
 //   f_top(F_l Kc_{l+1}^T, k); [p4 "One Forecast head per GQA group"].
 //
-// Everything here runs on kSelThreads = 256 threads (threads 0-255 of the
-// CTA) and synchronises them with named barrier 3, never with the whole
-// CTA: the attention kernel's CTA has a ninth warp that takes no part.
+// Everything here runs on kSelThreads = 256 threads and synchronises them
+// with named barrier 3.
 #pragma once
 
 #include <algorithm>
@@ -53,6 +51,7 @@ struct SelArgs {
   int CH, n_chunks, cap;
   int NBf;       // window grid: blocks the key map covers (all three inner windows present)
   int old_rank;  // 1: always the binned threshold search
+  SelCache cc;   // the cached decode selection's slot cache (cc.C == 0: none)
 };
 
 // ---------------------------------------------------------------------------
@@ -485,6 +484,169 @@ __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int l
 }
 
 
+// ---------------------------------------------------------------------------
+// slot cache step of the cached decode selection
+// ---------------------------------------------------------------------------
+// [p4 "The fourth projection", Algorithm 2]: layer l+1's blocks come from
+// CPU pinned memory while layer l computes.  The policy (the pages give
+// none) is that of the plan kernel: a selected block some slot holds is a
+// hit and keeps the slot; every other valid entry, in list order, takes the
+// next slot past the clock hand that holds none of this step's blocks, and
+// the hand moves one further.  Here the block that wrote a (b, g)'s set plans
+// it and copies its misses, so the results equal those of the plan and
+// gather calls made after the selection.
+
+// words of the ring the step works in: slot map, list, slot of each entry,
+// lowest slot holding each entry's block, slots in use (bits), misses, and
+// the miss count
+__host__ __device__ constexpr long long cache_step_words(int C, int S) {
+  return (long long)C + 4LL * S + (C + 31) / 32 + 1;
+}
+
+constexpr int kPlanMissMark = -2;
+constexpr int kHitNone = 0x7fffffff;
+
+// An empty set (every entry -1): nothing is held or fetched, and the hand is
+// only brought into range, as the plan leaves it.
+__device__ void cache_step_empty(const SelArgs &a, long long pair) {
+  const SelCache &cc = a.cc;
+  for (int s = threadIdx.x; s < a.S; s += kSelThreads) {
+    cc.phys[pair * a.S + s] = -1;
+    cc.fetch[pair * a.S + s] = 0;
+  }
+  if (threadIdx.x == 0) {
+    const int h = cc.hand[pair];
+    if (h < 0 || h >= cc.C) cc.hand[pair] = 0;
+  }
+}
+
+// The set out[S] this block has just written (ascending block ids, then -1
+// padding), past a barrier: plan it against the pair's C slots, write the
+// plan's outputs and copy every miss from the mapped host blocks.  smem: the
+// ring, idle once the set is written, of cache_step_words(C, S) words.  The
+// list is sorted, so each slot finds the entry of its block by binary search
+// (entries of -1 compare above every block id); a block held by several
+// slots hits the lowest of them, as in the plan kernel.
+__device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out, uint8_t *smem) {
+  const SelCache &cc = a.cc;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int C = cc.C, S = a.S, words = (C + 31) / 32;
+  int32_t *blk = reinterpret_cast<int32_t *>(smem);          // [C] block of each slot
+  int32_t *ids = blk + C;                                     // [S] the list
+  int32_t *ph = ids + S;                                      // [S] slot, -1, or the miss mark
+  int32_t *hit = ph + S;                                      // [S] lowest slot holding it
+  uint32_t *used = reinterpret_cast<uint32_t *>(hit + S);     // [words] slots this step uses
+  int32_t *miss = reinterpret_cast<int32_t *>(used + words);  // [S] entries to copy
+  int32_t *n_miss = miss + S;
+  int32_t *bo = cc.block_of + pair * C;
+  for (int c = tid; c < C; c += kSelThreads) blk[c] = bo[c];
+  for (int s = tid; s < S; s += kSelThreads) {
+    ids[s] = __ldcg(out + s);
+    hit[s] = kHitNone;
+  }
+  for (int w = tid; w < words; w += kSelThreads) used[w] = 0u;
+  sel_sync();
+  // hits: every slot looks its block up in the list
+  for (int c = tid; c < C; c += kSelThreads) {
+    const int j = blk[c];
+    if (j < 0) continue;
+    int lo = 0, hi = S;  // the first entry not below j
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      const int v = ids[mid];
+      if (v >= 0 && v < j) lo = mid + 1;
+      else hi = mid;
+    }
+    if (lo < S && ids[lo] == j) atomicMin(&hit[lo], c);
+  }
+  sel_sync();
+  for (int s = tid; s < S; s += kSelThreads) {
+    const int j = ids[s];
+    int p = -1;
+    if (j >= a.NB) {
+      flag_status(a.status, SPARDA_DEV_RANGE);
+    } else if (j >= 0) {
+      p = hit[s];
+      if (p != kHitNone) atomicOr(&used[p >> 5], 1u << (p & 31));
+      else p = kPlanMissMark;
+    }
+    ph[s] = p;
+  }
+  sel_sync();
+  // misses, in list order, placed by one lane (the policy is sequential);
+  // the warp finds them 32 entries at a time
+  if (tid < 32) {
+    int h = cc.hand[pair];
+    if (h < 0 || h >= C) h = 0;
+    int nm = 0;
+    for (int base = 0; base < S; base += 32) {
+      const int s = base + lane;
+      unsigned m = __ballot_sync(0xffffffffu, s < S && ph[s] == kPlanMissMark);
+      while (m) {
+        const int s2 = base + __ffs(m) - 1;
+        m &= m - 1;
+        if (lane == 0) {
+          int guard = 0;  // a free slot exists while C >= S; bounded all the same
+          while (((used[h >> 5] >> (h & 31)) & 1u) && guard < C) {
+            h = (h + 1 == C) ? 0 : h + 1;
+            ++guard;
+          }
+          if (guard >= C) {
+            ph[s2] = -1;
+            flag_status(a.status, SPARDA_DEV_RANGE);
+          } else {
+            blk[h] = ids[s2];
+            used[h >> 5] |= 1u << (h & 31);
+            ph[s2] = C + h;
+            miss[nm++] = s2;
+            h = (h + 1 == C) ? 0 : h + 1;
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) {
+      cc.hand[pair] = h;
+      *n_miss = nm;
+    }
+  }
+  sel_sync();
+  for (int c = tid; c < C; c += kSelThreads) bo[c] = blk[c];
+  for (int s = tid; s < S; s += kSelThreads) {
+    const int p = ph[s];
+    cc.phys[pair * S + s] = p >= C ? p - C : p;
+    cc.fetch[pair * S + s] = p >= C ? 1 : 0;
+  }
+  // the copies: 16-byte zero-copy loads of the mapped host blocks, two
+  // blocks' loads in flight per thread ahead of their stores
+  constexpr int kVec = 2 * kBlk * kD * 2 / 16;  // 16-byte vectors of a K|V block pair
+  constexpr int kPer = kVec / kSelThreads;      // 8 per thread
+  const long long blk_elems = 2LL * kBlk * kD;
+  const int nm = *n_miss;
+  for (int q = 0; q < nm; q += 2) {
+    const int nb = min(2, nm - q);
+    uint4 v[2][kPer];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (t < nb) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            cc.host_kv + (pair * a.NB + ids[miss[q + t]]) * blk_elems);
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) v[t][u] = ldg_plain(src + u * kSelThreads + tid);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (t < nb) {
+        uint4 *dst = reinterpret_cast<uint4 *>(cc.cache +
+                                               (pair * C + (ph[miss[q + t]] - C)) * blk_elems);
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) stg_stream(dst + u * kSelThreads + tid, v[t][u]);
+      }
+    }
+  }
+}
+
 // Shared memory one selection item works in.
 struct SelSmem {
   uint8_t *ring;        // RING pieces of 32 KB, 16-byte aligned
@@ -503,7 +665,7 @@ struct SelSmem {
 // is ranked at once, otherwise the keys go to the workspace and the chunk
 // that takes the problem's last ticket ranks every key of it.  Runs on
 // threads 0-255; every branch is uniform over them.
-template <int RING>
+template <int RING, bool CACHED>
 __device__ void select_block_item(const SelArgs &a, long long item, const SelSmem &sm) {
   const int tid = threadIdx.x;
   const long long prob = item / a.n_chunks;
@@ -520,6 +682,7 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
       if (chunk == 0) {
         for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
         if (tid == 0) flag_status(a.status, SPARDA_DEV_RANGE);
+        if (CACHED) cache_step_empty(a, prob);
       }
       if (a.n_chunks > 1) {  // keep the ticket count of the problem right
         sel_sync();
@@ -535,7 +698,13 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
   const BlockParts bp = block_parts(pos, kBlk, a.n_init, a.n_local);
   const int ncand = bp.cand_hi - bp.cand_lo;
   if (ncand <= a.k || a.k == 0) {  // nothing to rank: every candidate, or none, is kept
-    if (chunk == 0) write_set(out, bp, min(ncand, a.k), a.S, true);
+    if (chunk == 0) {
+      write_set(out, bp, min(ncand, a.k), a.S, true);
+      if (CACHED) {  // no copy was issued: the ring is free
+        sel_sync();
+        cache_step(a, prob, out, sm.ring);
+      }
+    }
     return;
   }
   const int lo = bp.cand_lo + chunk * a.CH;
@@ -560,8 +729,9 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
   int need = 0;
   int32_t *top = out + bp.init_hi;
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
-    if (!ok) {
+    if (!ok) {  // a copy may still land in the ring: the empty step uses none of it
       for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
+      if (CACHED) cache_step_empty(a, prob);
       return;
     }
     if (a.k <= kTopkMaxK && n <= kTopkMaxN && !a.old_rank)
@@ -571,6 +741,10 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
     const int ntop = compact_kept(sm.keys, n, tau, need, a.k, *sm.rs,
                                   [&](int p2, int e) { st_list(top + p2, bp.cand_lo + e); });
     write_set(out, bp, ntop, a.S, false);
+    if (CACHED) {
+      sel_sync();
+      cache_step(a, prob, out, sm.ring);
+    }
     return;
   }
   // ---- chunk scores -> workspace; the last chunk to finish ranks them all.
@@ -598,6 +772,7 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
       a.failed[prob] = 0u;
       a.counters[prob] = 0u;
     }
+    if (CACHED) cache_step_empty(a, prob);
     return;
   }
   uint32_t *keys = sm.rank_keys;
@@ -611,6 +786,10 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
                                 [&](int p2, int e) { st_list(top + p2, bp.cand_lo + e); });
   write_set(out, bp, ntop, a.S, false);
   if (tid == 0) a.counters[prob] = 0u;
+  if (CACHED) {  // this block's own copies all landed (else the problem failed)
+    sel_sync();
+    cache_step(a, prob, out, sm.ring);
+  }
 }
 
 

@@ -463,6 +463,30 @@ int sparda_prefetch_cached(const sparda_params *p, int C, const void *host_kv,
                            void *cache, int n_ctas, int32_t *dev_status, sparda_stream_t stream);
 
 /*
+ * sparda_forecast_select_cached -- the decode selection (one query token)
+ *   fused with the slot cache: the results of sparda_forecast_select (nq = 1)
+ *   followed by sparda_cache_plan on the lists it wrote and
+ *   sparda_prefetch_cached of the misses, from one launch.  The thread block
+ *   that writes a (b,g)'s set plans that set against the pair's slots and
+ *   copies its misses, so the next layer's attention waits on a single
+ *   kernel, and the fetch of a pair starts as soon as its set is known.
+ *   [p4 "The fourth projection", Algorithm 2]: select the next layer's
+ *   blocks, then fetch them while the current layer computes.
+ * F, nf, q_start, kc, idx, ws, ws_bytes  as for sparda_forecast_select with
+ *       nq = 1 (the workspace of SPARDA_OP_SELECT with nq = 1)
+ * C, block_of, hand, phys, fetch, cache  as for sparda_cache_plan and
+ *       sparda_prefetch_cached (one layer's slots, updated in place)
+ * host_kv  the page-locked, mapped host blocks, as for sparda_prefetch_cached
+ * Block grid only; the cached state must not be shared with a call that
+ * may overlap this one.  dev_status collects the flags of the three calls.
+ */
+int sparda_forecast_select_cached(const sparda_params *p, const void *F, int nf, int q_start,
+                                  const void *kc, int32_t *idx, void *ws, size_t ws_bytes, int C,
+                                  int32_t *block_of, int32_t *hand, int32_t *phys, int32_t *fetch,
+                                  const void *host_kv, void *cache, int32_t *dev_status,
+                                  sparda_stream_t stream);
+
+/*
  * sparda_sparse_attn_decode_cached -- sparda_sparse_attn_decode reading list
  *   entry s of (b,g) from cache slot phys[b,g,s] (idx gives its block id for
  *   the causal mask).  A slot outside [0, C) is skipped and flagged

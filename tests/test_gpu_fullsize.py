@@ -82,20 +82,22 @@ def test_decode_loop_full_size_sampled():
     torch.cuda.empty_cache()
 
 
-def _check_layer_against_host(loop, l, what, rows_of, pairs=None):
+def _check_layer_against_host(loop, l, what, rows_of, pairs=None, QFO=None):
     """Layer l of a host-offload step: its sets against the oracle (F_{l-1}
     scoring Kc_l), the device copy of every set entry byte-exact against the
     oracle's gather from the pinned host bytes, and the attention output over
     the host blocks of the GPU's set.  rows_of(b, g) returns the device copies
     the attention read, in list order ([S][2][64][128] bf16 bits; slot mode:
-    slot s, slot cache: slot phys[s])."""
+    slot s, slot cache: slot phys[s]).  QFO: the step's (Q, F, O) device
+    tensors when they are not the loop's own."""
     w = loop.w
     L, R, d, blk, NB, T = w.layers, w.r, w.d, w.blk, w.NB, w.T
     idx_all = loop.idx[l].cpu().numpy()
     kc_all = host_bits(loop.kc[l])
-    F_all = host_bits(loop.F[(l - 1) % L])
-    Q_all = host_bits(loop.Q[l])
-    O_all = host_bits(loop.O[l])
+    Qd, Fd, Od = QFO if QFO is not None else (loop.Q, loop.F, loop.O)
+    F_all = host_bits(Fd[(l - 1) % L])
+    Q_all = host_bits(Qd[l])
+    O_all = host_bits(Od[l])
     pairs = pairs or [(b, g) for b in range(w.B) for g in range(w.G)]
     for b, g in pairs:
         tag = "%s layer %d b %d g %d" % (what, l, b, g)
@@ -125,9 +127,11 @@ def test_offload_loop_full_size():
     of all four layers in pinned host memory (32 GiB).  One cold step -- per
     layer the next layer's blocks are selected, gathered over the host link
     into device slots on a side stream while this layer attends from its own
-    slots -- then three steps through the device slot cache (plan, fetch of
-    the misses only, attention reading each entry from its cache slot) with
-    drifting Forecast vectors.  After each step, every (sequence, group) of
+    slots -- then three steps through the device slot cache (one launch
+    selecting, planning and fetching the misses only, on a high-priority
+    stream; attention reading each entry from its cache slot; inputs
+    uploaded and outputs sent back on a copy stream) with drifting Forecast
+    vectors.  After each step, every (sequence, group) of
     the layers whose sets and slots are still those the step attended over
     (layers 1-3; layer 0's were replaced for the next step) is checked
     against the oracle: sets, device copies byte for byte against the host
@@ -144,6 +148,7 @@ def test_offload_loop_full_size():
                                       lambda b, g, l=l: host_bits(loop.slots[l, b, g]))
         loop.setup_cache(2 * w.S, 0.01, 4)
         loop.prime_cache()
+        loop.begin_cached(0)
         fetched = []
         for t in range(3):
             loop.step_e2e_cached(t)
@@ -157,7 +162,10 @@ def test_offload_loop_full_size():
                 _check_layer_against_host(
                     loop, l, "cache step %d" % t,
                     lambda b, g, l=l: host_bits(loop.cache[l, b, g].index_select(0, phys[l, b, g])),
-                    pairs=pairs)
+                    pairs=pairs, QFO=loop.step_inputs(t))
+            # the outputs that went back to the host are the step's
+            assert torch.equal(loop.h_out.view(torch.int16),
+                               loop.step_inputs(t)[2].cpu().view(torch.int16))
         # drifting sets: later steps fetch only a few blocks, never the whole set
         assert fetched[-1] < 0.1 * (w.layers - 1) * w.B * w.G * w.k, fetched
     finally:

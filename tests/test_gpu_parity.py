@@ -1225,6 +1225,126 @@ def test_cached_attention_with_lengths():
         check_attention(got[b:b + 1].reshape(1, 1, G * R, d), ora, "cached with lengths b=%d" % b)
 
 
+def _t(g):
+    return None if g is None else g.t
+
+
+@pytest.mark.parametrize("case", ["multi_chunk", "one_chunk", "lengths"])
+def test_select_cached_matches_oracle_over_steps(case):
+    """The cached selection -- selection, slot plan and fetch of the misses
+    from one launch -- over five steps of drifting Forecast vectors: the sets
+    equal the oracle's selection, and the slot map, fetch flags, cache state
+    and slot bytes equal the oracle's plan and gather of those sets; the
+    three separate calls on the same inputs leave the same bytes.  Cases: a
+    problem in several chunks (the ranking block plans), one chunk per
+    problem, and per-sequence lengths with a sequence whose candidates all
+    fit the budget and one whose length is invalid (empty set, flagged)."""
+    seed = {"multi_chunk": 50, "one_chunk": 51, "lengths": 52}[case]
+    rng = np.random.default_rng(seed)
+    B, G, d, k = (3 if case == "lengths" else 2), 3, 128, 12
+    NB = 300 if case == "one_chunk" else 700
+    T = NB * 64 - 9
+    S = k + 3
+    C = S + 5  # few spare slots: misses recycle slots within a few steps
+    host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
+    kc = W.normal_bf16(rng, (B, G, NB, d))
+    lens = [T] * B
+    sl = None
+    if case == "lengths":
+        lens = [T - 3, 64 * 14 + 5, 0]  # long; every candidate kept; invalid
+        sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    tune = {"select_chunk": 256 if case == "multi_chunk" else 1024}
+    p = abi.make_params(B, G * 4, G, T, k, seq_len=sl, tune=tune)
+    hkv = _pinned_bf16(host)
+    dkc = dev_bf16(kc)
+    st = {}
+    for side in ("fused", "split"):
+        st[side] = dict(
+            idx=Guarded((B, G, S), torch.int32, fill=0),
+            cache=Guarded((B, G, C, 2, 64, d), torch.bfloat16, fill=0),
+            block_of=Guarded((B, G, C), torch.int32, fill=-1),
+            hand=Guarded((B, G), torch.int32, fill=0),
+            phys=Guarded((B, G, S), torch.int32, fill=0),
+            fetch=Guarded((B, G, S), torch.int32, fill=0),
+            ws=guarded_workspace(abi.SPARDA_OP_SELECT, p, 1, 1),
+            status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    o_cache = np.zeros((B, G, C, 2, 64, d), np.uint16)
+    o_blk, o_hand = np.full((B, G, C), -1, np.int32), np.zeros((B, G), np.int32)
+    Fb = W.normal_bf16(rng, (B, 1, G, 1, d))
+    fetched = 0
+    for step in range(5):
+        if step > 0:
+            drift = 0.3 * rng.standard_normal(Fb.shape).astype(np.float32)
+            Fb = W.f32_to_bf16_bits(W.bf16_bits_to_f32(Fb) + drift)
+        dF = dev_bf16(Fb)
+        f, s_ = st["fused"], st["split"]
+        abi.sparda_forecast_select_cached(p, dF, 1, T - 1, dkc, f["idx"].t, _t(f["ws"]), C,
+                                          f["block_of"].t, f["hand"].t, f["phys"].t,
+                                          f["fetch"].t, hkv, f["cache"].t, f["status"])
+        abi.sparda_forecast_select(p, dF, 1, 1, T - 1, dkc, s_["idx"].t, _t(s_["ws"]),
+                                   s_["status"])
+        abi.sparda_cache_plan(p, C, s_["idx"].t, s_["block_of"].t, s_["hand"].t, s_["phys"].t,
+                              s_["fetch"].t, s_["status"])
+        abi.sparda_prefetch_cached(p, C, hkv, s_["idx"].t, s_["phys"].t, s_["fetch"].t,
+                                   s_["cache"].t, 0, s_["status"])
+        torch.cuda.synchronize()
+        for side in st.values():
+            for name in ("idx", "cache", "block_of", "hand", "phys", "fetch", "ws"):
+                if side[name] is not None:
+                    side[name].check("%s step %d" % (name, step))
+        want_status = abi.SPARDA_ERANGE if case == "lengths" else abi.SPARDA_OK
+        for side in st.values():
+            assert abi.sparda_status_from_device(int(side["status"].item())) == want_status
+        # the oracle: every sequence's set at its own last token, then the plan
+        o_idx = np.full((B, G, S), -1, np.int32)
+        for b, L in enumerate(lens):
+            if L < 1:
+                continue
+            o, _, _ = oracle.select(Fb[b:b + 1], np.ascontiguousarray(kc[b:b + 1, :, :(L + 63) // 64]),
+                                    k, 1, 2, L - 1)
+            o_idx[b] = o[0, 0]
+        got_idx = f["idx"].t.cpu().numpy()
+        assert np.array_equal(got_idx, o_idx), "sets, step %d" % step
+        o_phys, o_fetch, o_blk, o_hand = oracle.cache_plan(o_idx, o_blk, o_hand, NB)
+        o_cache = oracle.gather_cached(host, o_idx, o_phys, o_fetch, o_cache)
+        assert np.array_equal(f["phys"].t.cpu().numpy(), o_phys), step
+        assert np.array_equal(f["fetch"].t.cpu().numpy(), o_fetch), step
+        assert np.array_equal(f["block_of"].t.cpu().numpy(), o_blk), step
+        assert np.array_equal(f["hand"].t.cpu().numpy(), o_hand), step
+        assert np.array_equal(host_bits(f["cache"].t), o_cache), step
+        for name in ("idx", "block_of", "hand", "phys", "fetch"):
+            assert torch.equal(f[name].t, s_[name].t), (name, step)
+        assert torch.equal(f["cache"].t.view(torch.int16), s_["cache"].t.view(torch.int16)), step
+        fetched += int(o_fetch.sum())
+    # the steps exercise both hits and misses
+    assert 0 < fetched < 5 * B * G * S
+
+
+def test_select_cached_rejects_bad_arguments():
+    """Argument checks of the cached selection: fewer slots than list
+    entries, and device memory given as the mapped host buffer."""
+    B, G, NB, k = 1, 2, 40, 6
+    T = NB * 64
+    S = k + 3
+    p = abi.make_params(B, G * 4, G, T, k)
+    dev = torch.device("cuda")
+    F = torch.zeros(B, G, 128, dtype=torch.bfloat16, device=dev)
+    kc = torch.zeros(B, G, NB, 128, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(B, G, S, dtype=torch.int32, device=dev)
+    ws = abi.workspace(abi.SPARDA_OP_SELECT, p, 1, 1)
+    blk = torch.full((B, G, S), -1, dtype=torch.int32, device=dev)
+    hand = torch.zeros(B, G, dtype=torch.int32, device=dev)
+    phys = torch.empty(B, G, S, dtype=torch.int32, device=dev)
+    fetch = torch.empty_like(phys)
+    cache = torch.empty(B, G, S, 2, 64, 128, dtype=torch.bfloat16, device=dev)
+    host = torch.zeros(B, G, NB, 2, 64, 128, dtype=torch.bfloat16).pin_memory()
+    for C, hk in ((S - 1, host), (S, cache)):  # too few slots; device memory as the host buffer
+        with pytest.raises(abi.SpardaError) as e:
+            abi.sparda_forecast_select_cached(p, F, 1, T - 1, kc, idx, ws, C, blk, hand, phys,
+                                              fetch, hk, cache)
+        assert e.value.status == abi.SPARDA_EINVAL
+
+
 # --------------------------------------------------------------------------
 # prefill attention
 # --------------------------------------------------------------------------
