@@ -284,6 +284,7 @@ class DecodeLoop:
         self.ev_pre = [torch.cuda.Event() for _ in range(L)]
         self.ev_sel = [torch.cuda.Event() for _ in range(L)]
         self.host_kv = None
+        self.cached_sel_first = False  # the cached step's selection stream (setup_cache)
         if with_host:
             self._setup_host()
         torch.cuda.synchronize()
@@ -421,10 +422,10 @@ class DecodeLoop:
         self.d_out = torch.empty((2,) + tuple(self.O.shape), dtype=torch.bfloat16, device=dev)
         self.h_out = torch.empty(self.O.shape, dtype=torch.bfloat16).pin_memory()
         self.copy = torch.cuda.Stream()
-        # the selection, plan and fetch of the next layer go first: its thread
-        # blocks take SMs ahead of the attention's, so the fetch of the misses
-        # overlaps the attention instead of following it
-        self.sel_hi = torch.cuda.Stream(priority=-1)
+        # the stream of the fused selection, plan and fetch: beside the
+        # attention at a lower priority (as in the resident step), or ahead
+        # of it at a higher one, so the fetch of the misses starts early
+        self.sel_cached = torch.cuda.Stream(priority=-1 if self.cached_sel_first else 0)
         self.ev_begin, self.ev_o = torch.cuda.Event(), torch.cuda.Event()
         self.ev_in = [torch.cuda.Event() for _ in range(2)]
         self.ev_dl = [torch.cuda.Event() for _ in range(2)]
@@ -457,20 +458,18 @@ class DecodeLoop:
         """One decode step through the C ABI with the K/V cache in pinned host
         memory and a device slot cache.  Per layer, one launch selects the
         next layer's blocks, plans them against that layer's slots and
-        copies only the misses from the host, on a high-priority stream,
-        while this layer attends from its slots.  Step t's inputs were
+        copies only the misses from the host, on a side stream, while this
+        layer attends from its slots.  Step t's inputs were
         uploaded during step t-1 (begin_cached for the first); this step
         uploads step t+1's into the other buffer and sends its outputs back
-        while the next step runs.  Runs of steps are captured into one CUDA
-        graph."""
+        while the next step runs.  The main stream never waits on the copy
+        stream directly: the copies join the selection stream ahead of the
+        last layer's selection, which the next step's first attention waits
+        for.  Runs of steps are captured into one CUDA graph."""
         torch, abi, w = self.torch, self.abi, self.w
         L, C = w.layers, self.C
         main = torch.cuda.current_stream()
         cur, oth = t % 2, (t + 1) % 2
-        if ("in", cur) in self._recorded:
-            main.wait_event(self.ev_in[cur])
-        if ("dl", cur) in self._recorded:  # step t-2's outputs have left this buffer
-            main.wait_event(self.ev_dl[cur])
         # step t+1's inputs go into the other buffer, which step t-1 no longer reads
         self.ev_begin.record(main)
         self.copy.wait_event(self.ev_begin)
@@ -482,15 +481,24 @@ class DecodeLoop:
         for l in range(L):
             nxt = (l + 1) % L
             self.ev_pre[l].record(main)
-            self.sel_hi.wait_event(self.ev_pre[l])
-            with torch.cuda.stream(self.sel_hi):
+            self.sel_cached.wait_event(self.ev_pre[l])
+            if l == L - 1:
+                # the copies step t+1 depends on -- its inputs, issued at this
+                # step's start, and step t-1's outputs leaving the buffer step
+                # t+1 writes -- join here, long after they ended; attention(0)
+                # of step t+1 waits for this selection anyway
+                for ev in (("in", oth), ("dl", oth)):
+                    if ev in self._recorded:
+                        self.sel_cached.wait_event(
+                            (self.ev_in if ev[0] == "in" else self.ev_dl)[ev[1]])
+            with torch.cuda.stream(self.sel_cached):
                 abi.sparda_forecast_select_cached(self.p, F[l], 1, w.T - 1, self.kc[nxt],
                                                   self.idx[nxt], self.ws_sel[l], C,
                                                   self.block_of[nxt], self.hand[nxt],
                                                   self.phys[nxt], self.fetch[nxt],
                                                   self.host_kv[nxt], self.cache[nxt],
                                                   self.status)
-                self.fetch_ev[nxt].record(self.sel_hi)
+                self.fetch_ev[nxt].record(self.sel_cached)
             if l > 0:  # layer 0's blocks were joined at the end of the previous step
                 main.wait_event(self.fetch_ev[l])
             abi.sparda_sparse_attn_decode_cached(self.p, C, Q[l], self.cache[l], self.idx[l],
@@ -935,7 +943,7 @@ def run_sparda(args):
         dist.destroy_process_group()
 
 
-def run_slot_cache_legs(loop, args, world, resident_ms):
+def run_slot_cache_legs(loop, args, world, resident_ms, sigmas=(0.0, 0.01, 0.03, 0.1)):
     """The e2e loop with a device slot cache (2S slots per layer and group)
     under a few drift rates of the Forecast vectors between decode steps:
     per-step time, the share of top-k blocks that still cross the host
@@ -948,14 +956,17 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
     out = []
     e_steps = max(3, min(args.steps, 10))
     warm = max(args.warmup, 3)
-    for sigma in (0.0, 0.01, 0.03, 0.1):
+    for sigma in sigmas:
         n = warm + 2 * e_steps + 1
         loop.setup_cache(2 * w.S, sigma, n)
-        loop.prime_cache()  # one eager step first: every launch's one-time setup is done
-        loop.begin_cached(0)
-        loop.cached_steps(0, 1)
+        # launched and captured like the resident step: attention on the
+        # high-priority main stream, unless the selection goes first
+        cap = torch.cuda.Stream() if loop.cached_sel_first else loop.main
+        with torch.cuda.stream(cap):  # one eager step first: every launch's setup is done
+            loop.prime_cache()
+            loop.begin_cached(0)
+            loop.cached_steps(0, 1)
         torch.cuda.synchronize()
-        cap = torch.cuda.Stream()
         graphs = []
         with torch.cuda.stream(cap):
             for t0, cnt in ((0, warm), (warm, e_steps)):
@@ -966,19 +977,20 @@ def run_slot_cache_legs(loop, args, world, resident_ms):
         torch.cuda.synchronize()
         loop.block_of.fill_(-1)   # capture enqueued nothing; start the cache cold again
         loop.hand.zero_()
-        loop.prime_cache()
-        loop.begin_cached(0)
-        graphs[0].replay()
-        ms = time_steps(graphs[1].replay, 1, world) / e_steps
-        # the fetched share, on the steps that follow (run eagerly, untimed)
-        fetched = 0
-        t0 = warm + e_steps
-        loop.begin_cached(t0)
-        for t in range(t0, t0 + e_steps):
-            loop.step_e2e_cached(t)
-            torch.cuda.synchronize()
-            fetched += int(loop.fetch.sum().item())
-        loop.end_cached(t0 + e_steps)
+        with torch.cuda.stream(cap):
+            loop.prime_cache()
+            loop.begin_cached(0)
+            graphs[0].replay()
+            ms = time_steps(graphs[1].replay, 1, world) / e_steps
+            # the fetched share, on the steps that follow (run eagerly, untimed)
+            fetched = 0
+            t0 = warm + e_steps
+            loop.begin_cached(t0)
+            for t in range(t0, t0 + e_steps):
+                loop.step_e2e_cached(t)
+                torch.cuda.synchronize()
+                fetched += int(loop.fetch.sum().item())
+            loop.end_cached(t0 + e_steps)
         torch.cuda.synchronize()
         del graphs
         per_step = fetched / e_steps

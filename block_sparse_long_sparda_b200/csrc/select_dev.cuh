@@ -352,8 +352,10 @@ __device__ __forceinline__ void st_list(int32_t *p, int v) {
 
 // init | top-k | local | -1 padding.  With `fill_top`, the top-k part is the
 // first ntop candidates (every candidate is taken); otherwise it is written
-// by the caller.
-__device__ void write_set(int32_t *out, const BlockParts &bp, int ntop, int S, bool fill_top) {
+// by the caller.  mirror (optional, shared memory): the entries written here
+// are also stored there, at the same positions.
+__device__ void write_set(int32_t *out, const BlockParts &bp, int ntop, int S, bool fill_top,
+                          int32_t *mirror = nullptr) {
   const int nloc = bp.c - bp.local_lo + 1;
   for (int s = threadIdx.x; s < S; s += kSelThreads) {
     int v;
@@ -368,6 +370,7 @@ __device__ void write_set(int32_t *out, const BlockParts &bp, int ntop, int S, b
       v = -1;
     }
     st_list(out + s, v);
+    if (mirror) mirror[s] = v;
   }
 }
 
@@ -496,15 +499,50 @@ __device__ bool score_rows(const uint16_t *kc_bg, const float *fs, int nf, int l
 // it and copies its misses, so the results equal those of the plan and
 // gather calls made after the selection.
 
-// words of the ring the step works in: slot map, list, slot of each entry,
-// lowest slot holding each entry's block, slots in use (bits), misses, and
-// the miss count
+// The ring, idle once a set is written, holds the step's state (words):
+// [0, 1024) the ranking's scratch | the list [S] (stored as it is written) |
+// slot map [C] and hand [1] (loaded while the set is ranked) | slot of each
+// entry [S] | lowest slot holding each entry's block [S] | slots in use
+// (bits) | entries to copy [S] | their count [1]
 __host__ __device__ constexpr long long cache_step_words(int C, int S) {
-  return (long long)C + 4LL * S + (C + 31) / 32 + 1;
+  return 1024LL + 4LL * S + C + (C + 31) / 32 + 2;
+}
+
+struct CacheSmem {
+  int32_t *ids, *blk, *hand, *ph, *hit;
+  uint32_t *used;
+  int32_t *miss, *n_miss;
+};
+
+__device__ __forceinline__ CacheSmem cache_smem(uint8_t *ring, int C, int S) {
+  CacheSmem cs;
+  cs.ids = reinterpret_cast<int32_t *>(ring) + 1024;
+  cs.blk = cs.ids + S;
+  cs.hand = cs.blk + C;
+  cs.ph = cs.hand + 1;
+  cs.hit = cs.ph + S;
+  cs.used = reinterpret_cast<uint32_t *>(cs.hit + S);
+  cs.miss = reinterpret_cast<int32_t *>(cs.used + (C + 31) / 32);
+  cs.n_miss = cs.miss + S;
+  return cs;
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 
 constexpr int kPlanMissMark = -2;
 constexpr int kHitNone = 0x7fffffff;
+
+// Start loading the pair's slot map and hand into the ring (asynchronous
+// copies, waited for by cache_step), once the block knows it writes the set.
+__device__ void cache_load_state(const SelArgs &a, long long pair, uint8_t *ring) {
+  const CacheSmem cs = cache_smem(ring, a.cc.C, a.S);
+  const int32_t *bo = a.cc.block_of + pair * a.cc.C;
+  for (int c = threadIdx.x; c < a.cc.C; c += kSelThreads) cp_async4(cs.blk + c, bo + c);
+  if (threadIdx.x == 0) cp_async4(cs.hand, a.cc.hand + pair);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
 
 // An empty set (every entry -1): nothing is held or fetched, and the hand is
 // only brought into range, as the plan leaves it.
@@ -520,85 +558,75 @@ __device__ void cache_step_empty(const SelArgs &a, long long pair) {
   }
 }
 
-// The set out[S] this block has just written (ascending block ids, then -1
-// padding), past a barrier: plan it against the pair's C slots, write the
-// plan's outputs and copy every miss from the mapped host blocks.  smem: the
-// ring, idle once the set is written, of cache_step_words(C, S) words.  The
-// list is sorted, so each slot finds the entry of its block by binary search
-// (entries of -1 compare above every block id); a block held by several
-// slots hits the lowest of them, as in the plan kernel.
-__device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out, uint8_t *smem) {
+// The set this block has just written (ascending block ids, then -1
+// padding; its entries also in cs.ids), after cache_load_state: plan it
+// against the pair's C slots, write the plan's outputs and copy every miss
+// from the mapped host blocks.  The list is sorted, so each slot finds the
+// entry of its block by binary search (entries of -1 compare above every
+// block id); a block held by several slots hits the lowest of them, as in
+// the plan kernel.
+__device__ void cache_step(const SelArgs &a, long long pair, uint8_t *ring) {
   const SelCache &cc = a.cc;
   const int tid = threadIdx.x, lane = tid & 31;
   const int C = cc.C, S = a.S, words = (C + 31) / 32;
-  int32_t *blk = reinterpret_cast<int32_t *>(smem);          // [C] block of each slot
-  int32_t *ids = blk + C;                                     // [S] the list
-  int32_t *ph = ids + S;                                      // [S] slot, -1, or the miss mark
-  int32_t *hit = ph + S;                                      // [S] lowest slot holding it
-  uint32_t *used = reinterpret_cast<uint32_t *>(hit + S);     // [words] slots this step uses
-  int32_t *miss = reinterpret_cast<int32_t *>(used + words);  // [S] entries to copy
-  int32_t *n_miss = miss + S;
-  int32_t *bo = cc.block_of + pair * C;
-  for (int c = tid; c < C; c += kSelThreads) blk[c] = bo[c];
-  for (int s = tid; s < S; s += kSelThreads) {
-    ids[s] = __ldcg(out + s);
-    hit[s] = kHitNone;
-  }
-  for (int w = tid; w < words; w += kSelThreads) used[w] = 0u;
+  const CacheSmem cs = cache_smem(ring, C, S);
+  for (int s = tid; s < S; s += kSelThreads) cs.hit[s] = kHitNone;
+  for (int w = tid; w < words; w += kSelThreads) cs.used[w] = 0u;
+  asm volatile("cp.async.wait_all;" ::: "memory");
   sel_sync();
   // hits: every slot looks its block up in the list
   for (int c = tid; c < C; c += kSelThreads) {
-    const int j = blk[c];
+    const int j = cs.blk[c];
     if (j < 0) continue;
     int lo = 0, hi = S;  // the first entry not below j
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      const int v = ids[mid];
+      const int v = cs.ids[mid];
       if (v >= 0 && v < j) lo = mid + 1;
       else hi = mid;
     }
-    if (lo < S && ids[lo] == j) atomicMin(&hit[lo], c);
+    if (lo < S && cs.ids[lo] == j) atomicMin(&cs.hit[lo], c);
   }
   sel_sync();
-  for (int s = tid; s < S; s += kSelThreads) {
-    const int j = ids[s];
-    int p = -1;
-    if (j >= a.NB) {
-      flag_status(a.status, SPARDA_DEV_RANGE);
-    } else if (j >= 0) {
-      p = hit[s];
-      if (p != kHitNone) atomicOr(&used[p >> 5], 1u << (p & 31));
-      else p = kPlanMissMark;
-    }
-    ph[s] = p;
-  }
-  sel_sync();
-  // misses, in list order, placed by one lane (the policy is sequential);
-  // the warp finds them 32 entries at a time
+  // one warp: the hits' slots marked in use, then the misses, in list order,
+  // placed by one lane (the policy is sequential), found 32 entries at a time
   if (tid < 32) {
-    int h = cc.hand[pair];
+    for (int s = lane; s < S; s += 32) {
+      const int j = cs.ids[s];
+      int p = -1;
+      if (j >= a.NB) {
+        flag_status(a.status, SPARDA_DEV_RANGE);
+      } else if (j >= 0) {
+        p = cs.hit[s];
+        if (p != kHitNone) atomicOr(&cs.used[p >> 5], 1u << (p & 31));
+        else p = kPlanMissMark;
+      }
+      cs.ph[s] = p;
+    }
+    __syncwarp();
+    int h = *cs.hand;
     if (h < 0 || h >= C) h = 0;
     int nm = 0;
     for (int base = 0; base < S; base += 32) {
       const int s = base + lane;
-      unsigned m = __ballot_sync(0xffffffffu, s < S && ph[s] == kPlanMissMark);
+      unsigned m = __ballot_sync(0xffffffffu, s < S && cs.ph[s] == kPlanMissMark);
       while (m) {
         const int s2 = base + __ffs(m) - 1;
         m &= m - 1;
         if (lane == 0) {
           int guard = 0;  // a free slot exists while C >= S; bounded all the same
-          while (((used[h >> 5] >> (h & 31)) & 1u) && guard < C) {
+          while (((cs.used[h >> 5] >> (h & 31)) & 1u) && guard < C) {
             h = (h + 1 == C) ? 0 : h + 1;
             ++guard;
           }
           if (guard >= C) {
-            ph[s2] = -1;
+            cs.ph[s2] = -1;
             flag_status(a.status, SPARDA_DEV_RANGE);
           } else {
-            blk[h] = ids[s2];
-            used[h >> 5] |= 1u << (h & 31);
-            ph[s2] = C + h;
-            miss[nm++] = s2;
+            cs.blk[h] = cs.ids[s2];
+            cs.used[h >> 5] |= 1u << (h & 31);
+            cs.ph[s2] = C + h;
+            cs.miss[nm++] = s2;
             h = (h + 1 == C) ? 0 : h + 1;
           }
         }
@@ -607,13 +635,14 @@ __device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out,
     }
     if (lane == 0) {
       cc.hand[pair] = h;
-      *n_miss = nm;
+      *cs.n_miss = nm;
     }
   }
   sel_sync();
-  for (int c = tid; c < C; c += kSelThreads) bo[c] = blk[c];
+  int32_t *bo = cc.block_of + pair * C;
+  for (int c = tid; c < C; c += kSelThreads) bo[c] = cs.blk[c];
   for (int s = tid; s < S; s += kSelThreads) {
-    const int p = ph[s];
+    const int p = cs.ph[s];
     cc.phys[pair * S + s] = p >= C ? p - C : p;
     cc.fetch[pair * S + s] = p >= C ? 1 : 0;
   }
@@ -622,7 +651,7 @@ __device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out,
   constexpr int kVec = 2 * kBlk * kD * 2 / 16;  // 16-byte vectors of a K|V block pair
   constexpr int kPer = kVec / kSelThreads;      // 8 per thread
   const long long blk_elems = 2LL * kBlk * kD;
-  const int nm = *n_miss;
+  const int nm = *cs.n_miss;
   for (int q = 0; q < nm; q += 2) {
     const int nb = min(2, nm - q);
     uint4 v[2][kPer];
@@ -630,7 +659,7 @@ __device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out,
     for (int t = 0; t < 2; ++t) {
       if (t < nb) {
         const uint4 *src = reinterpret_cast<const uint4 *>(
-            cc.host_kv + (pair * a.NB + ids[miss[q + t]]) * blk_elems);
+            cc.host_kv + (pair * a.NB + cs.ids[cs.miss[q + t]]) * blk_elems);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) v[t][u] = ldg_plain(src + u * kSelThreads + tid);
       }
@@ -638,8 +667,8 @@ __device__ void cache_step(const SelArgs &a, long long pair, const int32_t *out,
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if (t < nb) {
-        uint4 *dst = reinterpret_cast<uint4 *>(cc.cache +
-                                               (pair * C + (ph[miss[q + t]] - C)) * blk_elems);
+        uint4 *dst = reinterpret_cast<uint4 *>(
+            cc.cache + (pair * C + (cs.ph[cs.miss[q + t]] - C)) * blk_elems);
 #pragma unroll
         for (int u = 0; u < kPer; ++u) stg_stream(dst + u * kSelThreads + tid, v[t][u]);
       }
@@ -699,11 +728,10 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
   const int ncand = bp.cand_hi - bp.cand_lo;
   if (ncand <= a.k || a.k == 0) {  // nothing to rank: every candidate, or none, is kept
     if (chunk == 0) {
-      write_set(out, bp, min(ncand, a.k), a.S, true);
-      if (CACHED) {  // no copy was issued: the ring is free
-        sel_sync();
-        cache_step(a, prob, out, sm.ring);
-      }
+      if (CACHED) cache_load_state(a, prob, sm.ring);  // no copy was issued: the ring is free
+      write_set(out, bp, min(ncand, a.k), a.S, true,
+                CACHED ? cache_smem(sm.ring, a.cc.C, a.S).ids : nullptr);
+      if (CACHED) cache_step(a, prob, sm.ring);
     }
     return;
   }
@@ -728,23 +756,25 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
   uint32_t tau = 0;
   int need = 0;
   int32_t *top = out + bp.init_hi;
+  // the list's shared-memory copy (the slot cache only)
+  int32_t *mirror = CACHED ? cache_smem(sm.ring, a.cc.C, a.S).ids : nullptr;
   if (a.n_chunks == 1) {  // n == ncand > k: rank in shared memory
     if (!ok) {  // a copy may still land in the ring: the empty step uses none of it
       for (int s2 = tid; s2 < a.S; s2 += kSelThreads) out[s2] = -1;
       if (CACHED) cache_step_empty(a, prob);
       return;
     }
+    if (CACHED) cache_load_state(a, prob, sm.ring);  // every copy of this block landed
     if (a.k <= kTopkMaxK && n <= kTopkMaxN && !a.old_rank)
       find_threshold_topk(sm.keys, n, a.k, sm.scratch, *sm.rs, tau, need);
     else
       find_threshold(sm.keys, n, a.k, *sm.rs, tau, need);
-    const int ntop = compact_kept(sm.keys, n, tau, need, a.k, *sm.rs,
-                                  [&](int p2, int e) { st_list(top + p2, bp.cand_lo + e); });
-    write_set(out, bp, ntop, a.S, false);
-    if (CACHED) {
-      sel_sync();
-      cache_step(a, prob, out, sm.ring);
-    }
+    const int ntop = compact_kept(sm.keys, n, tau, need, a.k, *sm.rs, [&](int p2, int e) {
+      st_list(top + p2, bp.cand_lo + e);
+      if (CACHED) mirror[bp.init_hi + p2] = bp.cand_lo + e;
+    });
+    write_set(out, bp, ntop, a.S, false, mirror);
+    if (CACHED) cache_step(a, prob, sm.ring);
     return;
   }
   // ---- chunk scores -> workspace; the last chunk to finish ranks them all.
@@ -776,20 +806,21 @@ __device__ void select_block_item(const SelArgs &a, long long item, const SelSme
     return;
   }
   uint32_t *keys = sm.rank_keys;
+  // this block's own copies all landed (else the problem failed): the ring is free
+  if (CACHED) cache_load_state(a, prob, sm.ring);
   for (int e = tid; e < ncand; e += kSelThreads) keys[e] = __ldcg(pkeys + e);
   sel_sync();
   if (a.k <= kTopkMaxK && ncand <= kTopkMaxN && !a.old_rank)
     find_threshold_topk(keys, ncand, a.k, sm.scratch, *sm.rs, tau, need);
   else
     find_threshold(keys, ncand, a.k, *sm.rs, tau, need);
-  const int ntop = compact_kept(keys, ncand, tau, need, a.k, *sm.rs,
-                                [&](int p2, int e) { st_list(top + p2, bp.cand_lo + e); });
-  write_set(out, bp, ntop, a.S, false);
+  const int ntop = compact_kept(keys, ncand, tau, need, a.k, *sm.rs, [&](int p2, int e) {
+    st_list(top + p2, bp.cand_lo + e);
+    if (CACHED) mirror[bp.init_hi + p2] = bp.cand_lo + e;
+  });
+  write_set(out, bp, ntop, a.S, false, mirror);
   if (tid == 0) a.counters[prob] = 0u;
-  if (CACHED) {  // this block's own copies all landed (else the problem failed)
-    sel_sync();
-    cache_step(a, prob, out, sm.ring);
-  }
+  if (CACHED) cache_step(a, prob, sm.ring);
 }
 
 
