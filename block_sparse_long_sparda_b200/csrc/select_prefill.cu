@@ -303,31 +303,61 @@ __device__ void warp_threshold(const uint32_t *keys, int n, int k, WarpRankSmem 
   need = 0;
 }
 
-// The same search with the row held in registers: entry e = 32*m + lane is
-// kv[m] (0 past the row's end; a valid key is never 0).  Rows of up to
-// 32 * KPL candidates; every pass runs on registers only.
-template <int KPL>
-__device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], int k, WarpRankSmem &sm,
-                                   uint32_t &tau, int &need) {
+// The smallest key u in [lo, hi] whose bin is at least b (hi when none is
+// below it): bins are monotone in the key, so the warp splits [lo, hi] 32
+// ways per round, each lane testing one cut (at most seven rounds).
+__device__ __forceinline__ uint32_t first_key_with_bin(const Members &mem, uint32_t lo,
+                                                       uint32_t hi, uint32_t b) {
   const int lane = threadIdx.x & 31;
-  Members mem{};
-  mem.all = true;
-  uint32_t rem = (uint32_t)k, m = 0;
-#pragma unroll
-  for (int q = 0; q < KPL; ++q) m += __popc(__ballot_sync(0xffffffffu, kv[q] != 0u));
+#pragma unroll 1
+  for (int round = 0; round < 10 && lo < hi; ++round) {
+    const uint64_t span = (uint64_t)(hi - lo);
+    const uint32_t cut = lo + (uint32_t)((span * (uint64_t)(lane + 1)) >> 5);  // lane 31: hi
+    const uint32_t ok = __ballot_sync(0xffffffffu, mem.bin(cut) >= b);
+    const int first = ok ? __ffs(ok) - 1 : 31;
+    const uint32_t below = __shfl_sync(0xffffffffu, cut, first > 0 ? first - 1 : 0);
+    const uint32_t at = __shfl_sync(0xffffffffu, cut, first);
+    if (!ok) return hi;  // not reached: bin(hi) >= b for the bins searched here
+    lo = first > 0 ? below + 1 : lo;
+    hi = at;
+  }
+  return hi;
+}
+
+// The same search with the row held in registers: entry e = 32*q + lane is
+// kv[q] (0 past the row's end; a valid key is never 0), m of them valid,
+// umin / umax the smallest and largest valid key.  Each pass histograms the
+// members in shared memory; once the bin holding the wanted rank has at most
+// 32 members, its key interval is found by a 32-way search of the monotone
+// bin function and the members are ranked exactly.  n_tau: the row's keys
+// equal to tau.
+template <int KPL>
+__device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], uint32_t m, uint32_t umin,
+                                   uint32_t umax, int k, WarpRankSmem &sm, uint32_t &tau,
+                                   int &need, int &n_tau) {
+  const int lane = threadIdx.x & 31;
+  uint32_t rem = (uint32_t)k;
+  uint32_t lo = umin, hi = umax;  // the members: valid keys in [lo, hi]
 #pragma unroll 1
   for (int pass = 0; pass < 12; ++pass) {
-    if (m <= 32u) {
+    if (m <= 32u || lo == hi) {
+      // ---- exact rank of the last few members ----
       uint32_t cnt = 0;
 #pragma unroll
       for (int q = 0; q < KPL; ++q) {
-        const bool in = kv[q] != 0u && mem.has(kv[q]);
+        const bool in = kv[q] >= lo && kv[q] <= hi && kv[q] != 0u;
         const uint32_t bal = __ballot_sync(0xffffffffu, in);
         const uint32_t slot = cnt + __popc(bal & ((1u << lane) - 1u));
         if (in && slot < 32u) sm.list[slot] = kv[q];
         cnt += __popc(bal);
       }
       __syncwarp();
+      if (lo == hi) {  // every member equal
+        tau = lo;
+        need = (int)rem;
+        n_tau = (int)cnt;
+        return;
+      }
       cnt = min(cnt, 32u);
       const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
       uint32_t gt = 0, ge = 0;
@@ -341,32 +371,20 @@ __device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], int k, WarpRankSme
       const int src = who ? __ffs(who) - 1 : 0;
       tau = __shfl_sync(0xffffffffu, x, src);
       need = (int)(rem - __shfl_sync(0xffffffffu, gt, src));
+      n_tau = (int)(__shfl_sync(0xffffffffu, ge - gt, src));
       __syncwarp();
       return;
     }
-    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
-#pragma unroll
-    for (int q = 0; q < KPL; ++q) {
-      if (kv[q] != 0u && mem.has(kv[q])) {
-        umin = min(umin, kv[q]);
-        umax = max(umax, kv[q]);
-      }
-    }
-    umin = __reduce_min_sync(0xffffffffu, umin);
-    umax = __reduce_max_sync(0xffffffffu, umax);
-    if (umin == umax) {
-      tau = umin;
-      need = (int)rem;
-      return;
-    }
-    const Members nx = make_bins(pass, umin, umax);
+    // ---- histogram of the members over the next bins ----
+    const Members nx = make_bins(pass, lo, hi);
 #pragma unroll
     for (int q = 0; q < 8; ++q) sm.hist[lane * 8 + q] = 0u;
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < KPL; ++q)
-      if (kv[q] != 0u && mem.has(kv[q])) atomicAdd(&sm.hist[nx.bin(kv[q])], 1u);
+      if (kv[q] >= lo && kv[q] <= hi && kv[q] != 0u) atomicAdd(&sm.hist[nx.bin(kv[q])], 1u);
     __syncwarp();
+    // ---- the bin holding rank `rem` from the top ----
     uint32_t h[8], local = 0;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -393,14 +411,20 @@ __device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], int k, WarpRankSme
     }
     const uint32_t who = __ballot_sync(0xffffffffu, bsel >= 0);
     const int src = who ? __ffs(who) - 1 : 0;
-    mem = nx;
-    mem.b = (uint32_t)__shfl_sync(0xffffffffu, bsel, src);
+    const uint32_t b = (uint32_t)__shfl_sync(0xffffffffu, bsel, src);
     rem = __shfl_sync(0xffffffffu, rsel, src);
     m = __shfl_sync(0xffffffffu, csel, src);
+    // the bin's key interval within [lo, hi]
+    const uint32_t a = first_key_with_bin(nx, lo, hi, b);
+    const uint32_t c = b >= 255u ? hi : first_key_with_bin(nx, lo, hi, b + 1);
+    const bool c_in = b < 255u && nx.bin(c) > b;  // c is past the bin: its last key is c - 1
+    lo = a;
+    hi = c_in ? c - 1 : c;
     __syncwarp();
   }
-  tau = 0xFFFFFFFFu;  // not reached
+  tau = 0xFFFFFFFFu;  // not reached: the range is a single key within a few passes
   need = 0;
+  n_tau = 0;
 }
 
 constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 2048)
@@ -415,7 +439,7 @@ struct RankArgs {
   int32_t *status;
 };
 
-__global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
+__global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) {
   __shared__ WarpRankSmem wsm[kRWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kRWarps + warp;
@@ -466,12 +490,32 @@ __global__ void __launch_bounds__(kRWarps * 32) rank_rows_kernel(RankArgs a) {
   const uint32_t lt = (1u << lane) - 1u;
   if (ncand <= kRegKeys * 32) {
     uint32_t kv[kRegKeys];
+    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
 #pragma unroll
     for (int q = 0; q < kRegKeys; ++q) {
       const int e = q * 32 + lane;
       kv[q] = e < ncand ? ld_key(keys + e) : 0u;
+      if (e < ncand) {
+        umin = min(umin, kv[q]);
+        umax = max(umax, kv[q]);
+      }
     }
-    warp_threshold_reg<kRegKeys>(kv, a.k, wsm[warp], tau, need);
+    umin = __reduce_min_sync(0xffffffffu, umin);
+    umax = __reduce_max_sync(0xffffffffu, umax);
+    int n_tau;
+    warp_threshold_reg<kRegKeys>(kv, (uint32_t)ncand, umin, umax, a.k, wsm[warp], tau, need,
+                                 n_tau);
+    if (need == n_tau) {  // every key equal to tau is kept: keep the keys >= tau
+      uint32_t n = 0;
+#pragma unroll
+      for (int q = 0; q < kRegKeys; ++q) {
+        const bool keep = kv[q] >= tau;  // tau > 0, so never an empty entry
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) top[n + __popc(bal & lt)] = bp.cand_lo + q * 32 + lane;
+        n += __popc(bal);
+      }
+      return;
+    }
     // keep keys > tau and the first `need` keys == tau, in block order
     uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll

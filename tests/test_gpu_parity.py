@@ -216,6 +216,27 @@ def test_select_prefill_tensor_scores(T, nq, q_off, k):
     _select_case(F, kc, k, 1, 2, T - nq - q_off, T, "prefill tensor")
 
 
+@pytest.mark.parametrize("k", [1, 17, 64, 300])
+def test_select_prefill_exact_ties_lower_index_wins(k):
+    """The row ranking of the tensor-core prefill path (>= 64 query tokens)
+    on integer scores: runs of exactly equal keys at the threshold, rows
+    whose threshold bin is one key, and rows keeping only some of the keys
+    equal to the k-th; the lower block index must win every tie, as in the
+    oracle.  Some tokens score with the opposite sign, so both ends of the
+    key range are ranked."""
+    rng = np.random.default_rng(5 + k)
+    NB, B, G, nq = 1500, 1, 2, 96
+    T = NB * 64
+    kc = np.zeros((B, G, NB, 128), np.float32)
+    kc[..., 0] = rng.integers(-3, 4, size=(B, G, NB))
+    F = np.zeros((B, nq, G, 1, 128), np.float32)
+    F[..., 0] = np.where(rng.random((B, nq, G, 1)) < 0.5, 1.0, -1.0)
+    Fb, kcb = W.f32_to_bf16_bits(F), W.f32_to_bf16_bits(kc)
+    ora, _, _ = oracle.select(Fb, kcb, k, 1, 2, T - nq)
+    got = gpu_select(Fb, kcb, k, 1, 2, T - nq, T)
+    assert np.array_equal(got, ora)
+
+
 def test_select_prefill_tensor_matches_streaming_path():
     """The same chunk through both selection paths gives the same sets."""
     rng = W.rng_for(19)
