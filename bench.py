@@ -486,11 +486,13 @@ class DecodeLoop:
                 # the copies step t+1 depends on -- its inputs, issued at this
                 # step's start, and step t-1's outputs leaving the buffer step
                 # t+1 writes -- join here, long after they ended; attention(0)
-                # of step t+1 waits for this selection anyway
-                for ev in (("in", oth), ("dl", oth)):
-                    if ev in self._recorded:
-                        self.sel_cached.wait_event(
-                            (self.ev_in if ev[0] == "in" else self.ev_dl)[ev[1]])
+                # of step t+1 waits for this selection anyway.  The copy
+                # stream runs in order and issued step t-1's outputs before
+                # step t+1's inputs, so the inputs' event covers both
+                if ("in", oth) in self._recorded:
+                    self.sel_cached.wait_event(self.ev_in[oth])
+                elif ("dl", oth) in self._recorded:
+                    self.sel_cached.wait_event(self.ev_dl[oth])
             with torch.cuda.stream(self.sel_cached):
                 abi.sparda_forecast_select_cached(self.p, F[l], 1, w.T - 1, self.kc[nxt],
                                                   self.idx[nxt], self.ws_sel[l], C,

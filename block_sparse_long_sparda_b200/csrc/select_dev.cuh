@@ -624,6 +624,7 @@ __device__ void cache_step(const SelArgs &a, long long pair, uint8_t *ring) {
             flag_status(a.status, SPARDA_DEV_RANGE);
           } else {
             cs.blk[h] = cs.ids[s2];
+            cc.block_of[pair * C + h] = cs.ids[s2];  // only the slots that change are written
             cs.used[h >> 5] |= 1u << (h & 31);
             cs.ph[s2] = C + h;
             cs.miss[nm++] = s2;
@@ -639,8 +640,6 @@ __device__ void cache_step(const SelArgs &a, long long pair, uint8_t *ring) {
     }
   }
   sel_sync();
-  int32_t *bo = cc.block_of + pair * C;
-  for (int c = tid; c < C; c += kSelThreads) bo[c] = cs.blk[c];
   for (int s = tid; s < S; s += kSelThreads) {
     const int p = cs.ph[s];
     cc.phys[pair * S + s] = p >= C ? p - C : p;
