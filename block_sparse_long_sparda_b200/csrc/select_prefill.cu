@@ -337,15 +337,19 @@ __device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], uint32_t m, uint32
                                    int &need, int &n_tau) {
   const int lane = threadIdx.x & 31;
   uint32_t rem = (uint32_t)k;
-  uint32_t lo = umin, hi = umax;  // the members: valid keys in [lo, hi]
+  // the members: valid keys in [lo, hi].  lo >= umin >= 1, so with one
+  // unsigned comparison of kv - lo against hi - lo an empty entry (0) wraps
+  // past the interval
+  uint32_t lo = umin, hi = umax;
 #pragma unroll 1
   for (int pass = 0; pass < 12; ++pass) {
+    const uint32_t width = hi - lo;
     if (m <= 32u || lo == hi) {
       // ---- exact rank of the last few members ----
       uint32_t cnt = 0;
 #pragma unroll
       for (int q = 0; q < KPL; ++q) {
-        const bool in = kv[q] >= lo && kv[q] <= hi && kv[q] != 0u;
+        const bool in = kv[q] - lo <= width;
         const uint32_t bal = __ballot_sync(0xffffffffu, in);
         const uint32_t slot = cnt + __popc(bal & ((1u << lane) - 1u));
         if (in && slot < 32u) sm.list[slot] = kv[q];
@@ -382,7 +386,7 @@ __device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], uint32_t m, uint32
     __syncwarp();
 #pragma unroll
     for (int q = 0; q < KPL; ++q)
-      if (kv[q] >= lo && kv[q] <= hi && kv[q] != 0u) atomicAdd(&sm.hist[nx.bin(kv[q])], 1u);
+      if (kv[q] - lo <= width) atomicAdd(&sm.hist[nx.bin(kv[q])], 1u);
     __syncwarp();
     // ---- the bin holding rank `rem` from the top ----
     uint32_t h[8], local = 0;
@@ -503,6 +507,9 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
     umin = __reduce_min_sync(0xffffffffu, umin);
     umax = __reduce_max_sync(0xffffffffu, umax);
     int n_tau;
+    // an entry of 0 is empty (a score's key never is), so the search starts at 1
+    umin = max(umin, 1u);
+    umax = max(umax, umin);
     warp_threshold_reg<kRegKeys>(kv, (uint32_t)ncand, umin, umax, a.k, wsm[warp], tau, need,
                                  n_tau);
     if (need == n_tau) {  // every key equal to tau is kept: keep the keys >= tau
@@ -511,7 +518,8 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
       for (int q = 0; q < kRegKeys; ++q) {
         const bool keep = kv[q] >= tau;  // tau > 0, so never an empty entry
         const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-        if (keep) top[n + __popc(bal & lt)] = bp.cand_lo + q * 32 + lane;
+        const uint32_t pos = n + __popc(bal & lt);
+        if (keep && pos < (uint32_t)a.k) top[pos] = bp.cand_lo + q * 32 + lane;
         n += __popc(bal);
       }
       return;
