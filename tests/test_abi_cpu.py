@@ -87,6 +87,30 @@ def test_validation_rejects_before_launch(L):
     assert _status("sparda_compress_keys", byref(none), fake, 4096 * 128, 128, fake, NULL, NULL) == abi.SPARDA_EINVAL
 
 
+def test_cached_selection_validates_before_touching_the_device(L):
+    """sparda_forecast_select_cached rejects bad shapes and arguments on the
+    host: a query outside the sequence, too many scoring vectors, fewer slots
+    than list entries, missing buffers; an empty batch is a no-op."""
+    byref = ctypes.byref
+    fake = ctypes.c_void_p(0x10000)
+    p = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8)      # S = 11
+
+    def call(prm, nf=1, q_start=4095, C=16, host=fake, idx=fake):
+        return _status("sparda_forecast_select_cached", byref(prm), fake, nf, q_start, fake, idx,
+                       NULL, 0, C, fake, fake, fake, fake, host, fake, NULL, NULL)
+    assert call(p, q_start=4096) == abi.SPARDA_EINVAL
+    assert call(p, nf=0) == abi.SPARDA_EINVAL
+    assert call(p, nf=17) == abi.SPARDA_EUNSUPPORTED
+    assert call(p, C=10) == abi.SPARDA_EINVAL                 # C < S
+    assert call(p, C=5000) == abi.SPARDA_EINVAL               # more slots than supported
+    assert call(p, idx=NULL) == abi.SPARDA_EINVAL
+    assert call(p, host=NULL) == abi.SPARDA_EINVAL
+    bad_tune = abi.make_params(B=2, Hq=32, G=8, T=4096, k=8, tune={"attn_stages": 5})
+    assert call(bad_tune) == abi.SPARDA_EINVAL
+    empty = abi.make_params(B=0, Hq=32, G=8, T=4096, k=8)
+    assert call(empty) == abi.SPARDA_OK
+
+
 def test_workspace_sizes_scale_with_shapes(L):
     small = abi.make_params(B=1, Hq=16, G=2, T=4096, k=4)
     assert abi.sparda_workspace_size(abi.SPARDA_OP_SELECT, small, 1, 1) >= 0
