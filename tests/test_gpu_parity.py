@@ -1250,7 +1250,7 @@ def _t(g):
     return None if g is None else g.t
 
 
-@pytest.mark.parametrize("case", ["multi_chunk", "one_chunk", "lengths"])
+@pytest.mark.parametrize("case", ["multi_chunk", "one_chunk", "lengths", "big_budget"])
 def test_select_cached_matches_oracle_over_steps(case):
     """The cached selection -- selection, slot plan and fetch of the misses
     from one launch -- over five steps of drifting Forecast vectors: the sets
@@ -1259,14 +1259,18 @@ def test_select_cached_matches_oracle_over_steps(case):
     three separate calls on the same inputs leave the same bytes.  Cases: a
     problem in several chunks (the ranking block plans), one chunk per
     problem, and per-sequence lengths with a sequence whose candidates all
-    fit the budget and one whose length is invalid (empty set, flagged)."""
-    seed = {"multi_chunk": 50, "one_chunk": 51, "lengths": 52}[case]
+    fit the budget and one whose length is invalid (empty set, flagged), and a
+    budget of 300 blocks (lists and slot maps longer than the 256 threads of
+    a block, the binned threshold search) with 340 slots."""
+    seed = {"multi_chunk": 50, "one_chunk": 51, "lengths": 52, "big_budget": 53}[case]
     rng = np.random.default_rng(seed)
     B, G, d, k = (3 if case == "lengths" else 2), 3, 128, 12
     NB = 300 if case == "one_chunk" else 700
+    if case == "big_budget":
+        G, k, NB = 2, 300, 1500
     T = NB * 64 - 9
     S = k + 3
-    C = S + 5  # few spare slots: misses recycle slots within a few steps
+    C = S + (37 if case == "big_budget" else 5)  # few spare slots: misses recycle slots
     host = W.normal_bf16(rng, (B, G, NB, 2, 64, d))
     kc = W.normal_bf16(rng, (B, G, NB, d))
     lens = [T] * B
@@ -1274,7 +1278,7 @@ def test_select_cached_matches_oracle_over_steps(case):
     if case == "lengths":
         lens = [T - 3, 64 * 14 + 5, 0]  # long; every candidate kept; invalid
         sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    tune = {"select_chunk": 256 if case == "multi_chunk" else 1024}
+    tune = {"select_chunk": {"multi_chunk": 256, "big_budget": 512}.get(case, 1024)}
     p = abi.make_params(B, G * 4, G, T, k, seq_len=sl, tune=tune)
     hkv = _pinned_bf16(host)
     dkc = dev_bf16(kc)
