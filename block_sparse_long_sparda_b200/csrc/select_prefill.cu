@@ -151,17 +151,32 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
       float v[16];
       tc::tmem_ld16(tmem + lane_sel + c, v);  // warp-wide: every lane takes part
       if (kPool == 1) {
-        if (i < a.nq && j0 + c < a.ld) {
+        if (j0 + c < a.ld) {
+          // the warp's 32 rows x 16 keys go through shared memory (the A
+          // operand's space, free once the products are done), so each store
+          // writes whole 64-byte row pieces: 16-byte chunks rotated by row
           uint32_t kk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int j = j0 + c + e;
             kk[e] = (j >= bp.cand_lo && j < bp.cand_hi) ? orderable_key(v[e]) : 0u;
           }
+          uint8_t *stg = opA + warp * 2048;  // [32 rows][64 bytes]
+          const int rl = tid & 31;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            reinterpret_cast<uint4 *>(row + c)[q] =
+            *reinterpret_cast<uint4 *>(stg + rl * 64 + ((q ^ (rl & 3)) << 4)) =
                 make_uint4(kk[4 * q], kk[4 * q + 1], kk[4 * q + 2], kk[4 * q + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const int r2 = t2 * 8 + (rl >> 2), q2 = rl & 3;  // row of the warp, chunk
+            const int i2 = i0 + warp * 32 + r2;
+            const uint4 val = *reinterpret_cast<const uint4 *>(stg + r2 * 64 + ((q2 ^ (r2 & 3)) << 4));
+            if (i2 < a.nq)
+              reinterpret_cast<uint4 *>(a.keys + ((long long)pair * a.nq + i2) * a.ld + j0 + c)[q2] = val;
+          }
+          __syncwarp();  // the staging rows are rewritten by the next step
         }
       } else {
         // 16 window columns = 4 blocks; windows past the last one are masked
