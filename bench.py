@@ -1030,27 +1030,35 @@ def host_link_peak_gbps(nbytes=1 << 30, reps=5):
 
 
 def time_cold(fn, reps, warm=3):
-    """Median device time of one call with L2 flushed before it: a read of
-    256 MB (twice L2) runs first on the same stream, outside the events.  A
-    read leaves L2 holding clean lines, so the timed call pays no write-back
-    of the flush (a memset would leave ~126 MB of dirty lines behind)."""
+    """Device time of one call with L2 flushed before it: a read of 256 MB
+    (twice L2) runs before every call on the same stream.  A read leaves L2
+    holding clean lines, so the timed call pays no write-back of the flush
+    (a memset would leave ~126 MB of dirty lines behind).  CUDA events here
+    tick in ~2 us steps, too coarse for a 10-30 us call, so `reps` (flush,
+    call) pairs are timed as one span and `reps` flushes alone as another;
+    the call's time is their difference over reps, the median of 3 trials."""
     import torch
     flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.zeros(reps, dtype=torch.float32, device="cuda")
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(reps)]
-    sink = torch.zeros(reps, dtype=torch.float32, device="cuda")
-    for i, (e0, e1) in enumerate(evs):
-        torch.sum(flush, dim=0, out=sink[i])
+
+    def span(with_call):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        fn()
+        for i in range(reps):
+            torch.sum(flush, dim=0, out=sink[i])
+            if with_call:
+                fn()
         e1.record()
-    torch.cuda.synchronize()
-    t = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1e3
+    span(True)
+    span(False)
+    trials = sorted((span(True) - span(False)) / reps for _ in range(3))
     del flush
-    return t[len(t) // 2]                          # us per call
+    return trials[1]                               # us per call
 
 
 def time_back_to_back(fn, steps, warm=3):
@@ -1374,8 +1382,8 @@ def run_sweep(pts=None, oracle_pts=()):
         del kc
     return {"metric": "selection-only sweep: Forecast vs 4-head baseline selector (us per call)",
             "G": G, "k": k, "points": points, "data": "synthetic", "dtype": "bf16",
-            "timing": "median of 15 calls, each after a 256 MB read that flushes L2 "
-                      "(the read is outside the events)",
+            "timing": "15 calls, each after a 256 MB read that flushes L2, timed as one span "
+                      "less a span of the 15 reads alone; median of 3 trials",
             "oracle": o_pts or None, "clocks": clocks.stop()}
 
 
