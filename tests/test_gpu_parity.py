@@ -1259,12 +1259,13 @@ def test_select_cached_matches_oracle_over_steps(case):
     three separate calls on the same inputs leave the same bytes.  Cases: a
     problem in several chunks (the ranking block plans), one chunk per
     problem, and per-sequence lengths with a sequence whose candidates all
-    fit the budget and one whose length is invalid (empty set, flagged), and a
+    fit the budget, one whose length is invalid (empty set, flagged) and one
+    whose set is shorter than the list (-1 padding), and a
     budget of 300 blocks (lists and slot maps longer than the 256 threads of
     a block, the binned threshold search) with 340 slots."""
     seed = {"multi_chunk": 50, "one_chunk": 51, "lengths": 52, "big_budget": 53}[case]
     rng = np.random.default_rng(seed)
-    B, G, d, k = (3 if case == "lengths" else 2), 3, 128, 12
+    B, G, d, k = (4 if case == "lengths" else 2), 3, 128, 12
     NB = 300 if case == "one_chunk" else 700
     if case == "big_budget":
         G, k, NB = 2, 300, 1500
@@ -1276,7 +1277,7 @@ def test_select_cached_matches_oracle_over_steps(case):
     lens = [T] * B
     sl = None
     if case == "lengths":
-        lens = [T - 3, 64 * 14 + 5, 0]  # long; every candidate kept; invalid
+        lens = [T - 3, 64 * 14 + 5, 0, 64 * 5 + 7]  # long; every candidate kept; invalid; padded
         sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
     tune = {"select_chunk": {"multi_chunk": 256, "big_budget": 512}.get(case, 1024)}
     p = abi.make_params(B, G * 4, G, T, k, seq_len=sl, tune=tune)
