@@ -85,7 +85,7 @@ def parse_args():
                          "B=8 with the bench's other shapes (4.3 GB of K/V, 140 MB of selected "
                          "K/V per attention launch), then two passes of a 512-token prefill "
                          "chunk of one sequence, then two cold host gathers of one layer at B=2 "
-                         "(1.1 GB pinned), then two head-softmax selections each on one "
+                         "(1.1 GB pinned) and two cached selections (cold, then warm), then two head-softmax selections each on one "
                          "layer of block keys and of window keys at B=16, T=128K, and exit: "
                          "the small cases ncu captures")
     return ap.parse_args()
@@ -1518,10 +1518,18 @@ def run_profile_case():
     gl = DecodeLoop(wg, with_host=True)
     for _ in range(2):
         abi.sparda_prefetch_blocks(gl.p, gl.host_kv[0], gl.idx[0], gl.slots[0], True, 0, gl.status)
+    # the cached selection into the layer's slot cache (2S slots): cold, then
+    # warm (every block a hit)
+    gl.setup_cache(2 * wg.S, 0.0, 2)
+    for _ in range(2):
+        abi.sparda_forecast_select_cached(gl.p, gl.F[0], 1, wg.T - 1, gl.kc[0], gl.idx[0],
+                                          gl.ws_sel[0], gl.C, gl.block_of[0], gl.hand[0],
+                                          gl.phys[0], gl.fetch[0], gl.host_kv[0], gl.cache[0],
+                                          gl.status)
     torch.cuda.synchronize()
     st3 = int(gl.status.item())
     gl.unregister()
-    print("profile case: host gather B=2, device status %d" % st3)
+    print("profile case: host gather and cached selection B=2, device status %d" % st3)
     del gl
     torch.cuda.empty_cache()
     # the original selector's per-head softmax form at B=16, T=128K: two
