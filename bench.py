@@ -1075,6 +1075,28 @@ def time_back_to_back(fn, steps, warm=3):
     return e0.elapsed_time(e1) / steps * 1e3      # us per call
 
 
+def time_graph(fn, steps, warm=3):
+    """us per call of `steps` calls captured into one CUDA graph and replayed:
+    for calls of a few tens of us, the host's per-call launch cost (tensor
+    maps, argument marshalling) would otherwise set the pace."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(steps):
+                fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    us = time_back_to_back(g.replay, 3, warm=0) / steps
+    del g
+    return us
+
+
 class PrefillChunk:
     """Prefill chunk: B=4 sequences of T=131072 tokens whose last 2048 tokens
     are the queries (positions T-2048 .. T-1), one Forecast vector per token
@@ -1240,7 +1262,7 @@ def run_windows(steps):
         l = t[0] & 1
         abi.sparda_forecast_select_windows(p, F, 1, 1, w.T - 1, kws[l], 32, 16, idx, ws[l])
         t[0] += 1
-    us = time_back_to_back(sel, n)
+    us = time_graph(sel, n)
     # the three windows inside each candidate block (the straddling fourth
     # window of a block is never scored, and never read)
     ncand = (w.T - 1) // w.blk - w.n_local + 1 - w.n_init
@@ -1308,7 +1330,7 @@ def run_real_model(steps):
         for which in ("select", "attention"):
             fn = (lambda: [loop.select(l) for l in range(L)]) if which == "select" else \
                  (lambda: [loop.attention(l) for l in range(L)])
-            kern[which] = time_back_to_back(fn, n) / L
+            kern[which] = time_graph(fn, n) / L
         del graph
     torch.cuda.synchronize()
     st = int(loop.status.item())
@@ -1464,9 +1486,9 @@ def run_head_softmax(steps):
     clocks = ClockSampler(torch.cuda.current_device())
     for windows in (False, True):
         c = HeadSoftmaxCase(windows)
-        h_us = time_back_to_back(c.head_softmax, n)
-        f_us = time_back_to_back(lambda: c.scores(c.F, 1, c.ws_f), n)
-        s_us = time_back_to_back(lambda: c.scores(c.Q, c.nf, c.ws_s), n)
+        h_us = time_graph(c.head_softmax, n)
+        f_us = time_graph(lambda: c.scores(c.F, 1, c.ws_f), n)
+        s_us = time_graph(lambda: c.scores(c.Q, c.nf, c.ws_s), n)
         nb = c.key_bytes()
         key = "windows" if windows else "blocks"
         out[key] = {"B": c.w.B, "T": c.w.T, "G": c.w.G, "heads_per_group": c.nf, "k": c.w.k,
