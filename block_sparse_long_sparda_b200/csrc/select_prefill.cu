@@ -24,12 +24,18 @@
 //     row), turn them into orderable keys -- 0 outside the token's candidate
 //     range -- and store them to the workspace, [pair][token][block].  Tiles
 //     lying wholly after every row's candidates are skipped.
-//  2. rank_rows_kernel -- one warp per (sequence, token, group) row: the same
-//     exact search as the decode selection (a score-linear then key-linear
-//     256-bin passes, an exact rank of the last few candidates), done by one
-//     warp with a per-warp histogram in shared memory, then a ballot pass in
-//     block order that keeps every key above the k-th plus the lowest-index
-//     ties, and the set init U top-k U local written in ascending order.
+//  2. rank_rows_kernel -- one warp per (sequence, token, group) row.  For
+//     k <= 64 and rows of 1024 to 2048 keys it first takes a threshold t0
+//     that at least 64 keys pass (the least over the lanes of each lane's
+//     second-largest key), lists the keys >= t0 (about 8 % of a row) and
+//     ranks only those: one histogram, an exact rank of the threshold bin,
+//     and a bitmap that puts the kept blocks in order.  Other rows, and rows
+//     whose lists or ties that does not settle, take the same exact search as
+//     the decode selection (a score-linear then key-linear 256-bin passes, an
+//     exact rank of the last few candidates) with a per-warp histogram in
+//     shared memory, then a ballot pass in block order that keeps every key
+//     above the k-th plus the lowest-index ties.  The set is init U top-k U
+//     local, written in ascending order.
 // Every wait is bounded; a timeout sets SPARDA_DEV_TIMEOUT, frees TMEM and
 // leaves the tile's keys unwritten.
 #include <algorithm>
@@ -205,9 +211,14 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
 // ---------------------------------------------------------------------------
 // warp-level exact top-k of one row
 // ---------------------------------------------------------------------------
+constexpr int kListCap = 16;  // keys per lane the sampled threshold may list
+
 struct WarpRankSmem {
   uint32_t hist[256];
   uint32_t list[32];
+  uint2 cand[kListCap + 1][32];  // per lane: (key, register q) of its keys >= t0; row
+                                 // kListCap takes the writes past the cap
+  uint32_t sel[64];              // kept entries: word q, bit lane = entry 32 q + lane
 };
 
 // the keys were written by the previous kernel: read-only for this one
@@ -448,6 +459,137 @@ __device__ void warp_threshold_reg(const uint32_t (&kv)[KPL], uint32_t m, uint32
 
 constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 2048)
 
+// The row's top k from a sampled threshold, for k <= 64 and rows of 1024 to
+// 2048 keys, each lane taking the entries e = 32 q + lane as in the register
+// search above (0 past the row).  t0 is the smallest over the lanes
+// of each lane's second-largest key, so every lane holds two keys >= t0 and
+// at least 64 >= k keys pass it: the k-th largest key is >= t0, and so is
+// every key the set keeps.  On scores of roughly one shape across the row a
+// lane holds about five such keys of its 64.  Each lane lists its keys >= t0
+// in shared memory (list_keys_from), one histogram of the listed keys finds
+// the bin of the k-th largest, its members are ranked exactly, and the kept
+// entries are placed in block order through a bitmap (word q, bit lane) and
+// its prefix counts (warp_topk_listed).  warp_topk_listed returns false,
+// having written nothing, when a lane lists more than kListCap keys, the bin
+// holds more than 32 keys, or only some of the keys equal to the k-th are
+// kept (the lower block indices would have to win); the caller then runs
+// the full search.
+
+// c = the lane's keys >= t0 (t0 >= 1, so never an empty entry), read again
+// from memory (L1 holds the row just read); only the first kListCap are
+// stored
+__device__ __forceinline__ int list_keys_from(const uint32_t *keys, int ncand, uint32_t t0,
+                                              WarpRankSmem &sm) {
+  const int lane = threadIdx.x & 31;
+  int c = 0;
+#pragma unroll 8
+  for (int q = 0; q < kRegKeys; ++q) {
+    const int e = q * 32 + lane;
+    const uint32_t u = e < ncand ? ld_key(keys + e) : 0u;
+    if (u >= t0) {
+      sm.cand[min(c, kListCap)][lane] = make_uint2(u, (uint32_t)q);
+      ++c;
+    }
+  }
+  return c;
+}
+
+__device__ bool warp_topk_listed(int c, uint32_t t0, uint32_t umax, int k, WarpRankSmem &sm,
+                                 int32_t *top, int cand_lo) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (__any_sync(0xffffffffu, c > kListCap)) return false;
+  const int cmax = __reduce_max_sync(0xffffffffu, (uint32_t)c);
+  // ---- one histogram of the listed keys, bins linear in score over [t0, umax] ----
+  const Members nx = make_bins(0, t0, umax);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) sm.hist[lane * 8 + q] = 0u;
+  __syncwarp();
+  for (int i = 0; i < c; ++i) atomicAdd(&sm.hist[nx.bin(sm.cand[i][lane].x)], 1u);
+  __syncwarp();
+  uint32_t h[8], local = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    h[q] = sm.hist[lane * 8 + q];
+    local += h[q];
+  }
+  uint32_t above = local;  // keys in the bins of this lane and the lanes above it
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
+    if (lane + o < 32) above += v;
+  }
+  above -= local;
+  const uint32_t rank = (uint32_t)k;
+  int bsel = -1;
+  uint32_t rsel = 0, csel = 0;
+#pragma unroll
+  for (int q = 7; q >= 0; --q) {
+    if (bsel < 0 && above + h[q] >= rank && above < rank) {
+      bsel = lane * 8 + q;
+      rsel = rank - above;
+      csel = h[q];
+    }
+    above += h[q];
+  }
+  const uint32_t who_b = __ballot_sync(0xffffffffu, bsel >= 0);
+  const int src_b = who_b ? __ffs(who_b) - 1 : 0;
+  const uint32_t b = (uint32_t)__shfl_sync(0xffffffffu, bsel, src_b);
+  const uint32_t rem = __shfl_sync(0xffffffffu, rsel, src_b);
+  const uint32_t m = __shfl_sync(0xffffffffu, csel, src_b);
+  if (!who_b || m > 32u) return false;
+  // ---- the bin's keys, ranked exactly ----
+  uint32_t cnt = 0;
+  for (int i = 0; i < cmax; ++i) {
+    const uint32_t u = i < c ? sm.cand[i][lane].x : 0u;
+    const bool in = i < c && nx.bin(u) == b;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (in) sm.list[cnt + __popc(bal & lt)] = u;
+    cnt += __popc(bal);
+  }
+  __syncwarp();
+  const uint32_t x = (uint32_t)lane < cnt ? sm.list[lane] : 0u;
+  uint32_t gt = 0, ge = 0;
+  for (uint32_t j = 0; j < cnt; ++j) {
+    const uint32_t y = sm.list[j];
+    gt += y > x;
+    ge += y >= x;
+  }
+  const bool hit = (uint32_t)lane < cnt && gt < rem && ge >= rem;
+  const uint32_t who = __ballot_sync(0xffffffffu, hit);
+  const int src = who ? __ffs(who) - 1 : 0;
+  const uint32_t tau = __shfl_sync(0xffffffffu, x, src);
+  const uint32_t need = rem - __shfl_sync(0xffffffffu, gt, src);
+  const uint32_t n_tau = __shfl_sync(0xffffffffu, ge - gt, src);
+  if (!who || need != n_tau) return false;
+  // ---- exactly k listed keys are >= tau: place them in block order ----
+  sm.sel[lane] = 0u;
+  sm.sel[lane + 32] = 0u;
+  __syncwarp();
+  for (int i = 0; i < c; ++i) {
+    const uint2 e = sm.cand[i][lane];
+    if (e.x >= tau) atomicOr(&sm.sel[e.y], 1u << lane);
+  }
+  __syncwarp();
+  const uint32_t w0 = sm.sel[2 * lane], w1 = sm.sel[2 * lane + 1];
+  const uint32_t n0 = __popc(w0), n01 = n0 + __popc(w1);
+  uint32_t incl = n01;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  sm.hist[2 * lane] = incl - n01;  // kept entries before word 2 lane
+  sm.hist[2 * lane + 1] = incl - n01 + n0;
+  __syncwarp();
+  for (int i = 0; i < c; ++i) {
+    const uint2 e = sm.cand[i][lane];
+    if (e.x >= tau) top[sm.hist[e.y] + __popc(sm.sel[e.y] & lt)] = cand_lo + 32 * (int)e.y + lane;
+  }
+  __syncwarp();
+  return true;
+}
+
 struct RankArgs {
   const uint32_t *keys;  // [B*G][nq][ld]
   int32_t *idx;          // [B][nq][G][S]
@@ -458,17 +600,35 @@ struct RankArgs {
   int32_t *status;
 };
 
-__global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) {
-  __shared__ WarpRankSmem wsm[kRWarps];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = (long long)blockIdx.x * kRWarps + warp;
-  pdl_trigger();
-  pdl_wait();
-  if (row >= a.rows) return;
-  const int g = (int)(row % a.G);
-  const long long bi = row / a.G;
-  const int i = (int)(bi % a.nq);
-  const long long b = bi / a.nq;
+struct RowPos {
+  long long b;
+  int g, i;
+};
+
+// row = (b * nq + i) * G + g
+__device__ __forceinline__ RowPos row_pos(const RankArgs &a, long long row) {
+  RowPos r;
+  if (a.rows <= 0x7fffffffLL) {  // 32-bit division where the rows allow it
+    const uint32_t r32 = (uint32_t)row, bi = r32 / (uint32_t)a.G;
+    r.g = (int)(r32 - bi * (uint32_t)a.G);
+    r.i = (int)(bi % (uint32_t)a.nq);
+    r.b = (long long)(bi / (uint32_t)a.nq);
+  } else {
+    r.g = (int)(row % a.G);
+    const long long bi = row / a.G;
+    r.i = (int)(bi % a.nq);
+    r.b = bi / a.nq;
+  }
+  return r;
+}
+
+// One row, by one warp.
+template <bool kListed>
+__device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPos rp,
+                                         WarpRankSmem &sm) {
+  const int lane = threadIdx.x & 31;
+  const long long b = rp.b;
+  const int g = rp.g, i = rp.i;
   int qs = a.q_start;
   if (a.seq_len) {
     const int len = a.seq_len[b];
@@ -507,6 +667,28 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
   int need;
   int32_t *top = out + bp.init_hi;
   const uint32_t lt = (1u << lane) - 1u;
+  if (kListed && ncand >= 1024 && ncand <= kRegKeys * 32) {
+    // the lane's largest and second-largest keys, all 64 loads in flight at
+    // once; the row is not kept in registers: the listing reads it again
+    // from L1, and the register search below loads it for the rows the
+    // listed threshold does not settle
+    uint32_t u1 = 0u, u2 = 0u;
+#pragma unroll
+    for (int q = 0; q < kRegKeys; ++q) {
+      const int e = q * 32 + lane;
+      const uint32_t u = e < ncand ? ld_key(keys + e) : 0u;
+      u2 = max(u2, min(u1, u));
+      u1 = max(u1, u);
+    }
+    const uint32_t t0 = __reduce_min_sync(0xffffffffu, u2);
+    const uint32_t top_key = __reduce_max_sync(0xffffffffu, u1);
+    // t0 = 0: a lane with fewer than two keys; t0 = the top key: all listed keys equal
+    if (t0 != 0u && t0 < top_key &&
+        warp_topk_listed(list_keys_from(keys, ncand, t0, sm), t0, top_key, a.k, sm, top,
+                         bp.cand_lo))
+      return;
+    __syncwarp();
+  }
   if (ncand <= kRegKeys * 32) {
     uint32_t kv[kRegKeys];
     uint32_t umin = 0xFFFFFFFFu, umax = 0u;
@@ -525,7 +707,7 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
     // an entry of 0 is empty (a score's key never is), so the search starts at 1
     umin = max(umin, 1u);
     umax = max(umax, umin);
-    warp_threshold_reg<kRegKeys>(kv, (uint32_t)ncand, umin, umax, a.k, wsm[warp], tau, need,
+    warp_threshold_reg<kRegKeys>(kv, (uint32_t)ncand, umin, umax, a.k, sm, tau, need,
                                  n_tau);
     if (need == n_tau) {  // every key equal to tau is kept: keep the keys >= tau
       uint32_t n = 0;
@@ -556,7 +738,7 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
     }
     return;
   }
-  warp_threshold(keys, ncand, a.k, wsm[warp], tau, need);
+  warp_threshold(keys, ncand, a.k, sm, tau, need);
   // keep keys > tau and the first `need` keys == tau, in block order
   uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll 2
@@ -573,6 +755,21 @@ __global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) 
     n_gt += __popc(bgt);
     n_eq += __popc(beq);
   }
+}
+
+// kListed: every row of the chunk has 1024 to 2048 candidates and k <= 64
+// (the host checks), and rows try the listed threshold first; rows it does
+// not settle, and every row of the other variant, take the binned search on
+// the row held in registers (rows of up to 2048 candidates) or in memory.
+// One warp per row.
+template <bool kListed>
+__global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) {
+  __shared__ WarpRankSmem wsm[kRWarps];
+  const int warp = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kRWarps + warp;
+  pdl_trigger();
+  pdl_wait();
+  if (row < a.rows) rank_row<kListed>(a, row, row_pos(a, row), wsm[warp]);
 }
 
 }  // namespace
@@ -654,8 +851,15 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   ra.seq_len = p.seq_len;
   ra.T = p.T;
   ra.status = status;
-  e = launch_pdl(rank_rows_kernel, (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream,
-                 ra);
+  // the listed threshold when every row qualifies: no lengths (the chunk sits
+  // at q_start), k <= 64, and 1024 to 2048 candidates from the chunk's first
+  // token to its last
+  const int nc_first = block_parts(q_start, kBlk, p.n_init, p.n_local).cand_hi - p.n_init;
+  const int nc_last = block_parts(q_start + nq - 1, kBlk, p.n_init, p.n_local).cand_hi - p.n_init;
+  const bool listed = tuning(p).select_binned == 0 && p.seq_len == nullptr && p.k >= 1 &&
+                      p.k <= 64 && nc_first >= 1024 && nc_last <= kRegKeys * 32;
+  e = launch_pdl(listed ? rank_rows_kernel<true> : rank_rows_kernel<false>,
+                 (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream, ra);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -87,7 +87,9 @@ typedef struct sparda_tuning {
                          selection instead of the tensor-core score tiles         */
   int select_binned;  /* nonzero: the binned threshold search even where the
                          sorting-network threshold applies (k <= 64, <= 2048
-                         candidates)                                             */
+                         candidates), and, for query chunks ranked row by row,
+                         even where the listed sample threshold applies
+                         (k <= 64, 1024 to 2048 candidates)                      */
   int attn_ctas;      /* attention thread blocks (kept within what the lists need
                          and the workspace was sized for)                        */
   int attn_stages;    /* attention ring depth: 2, 3, 4 or 6 stages of 32 KB       */

@@ -306,6 +306,16 @@ def test_prefill_chunk_full_size_sampled():
         ora_o = oracle.sparse_attention(Q, K, V, gpu_idx, q0 + i, T, blk)
         gpu_o = host_bits(pc.O[b, i, g * R:(g + 1) * R]).reshape(1, 1, R, d)
         check_attention(gpu_o, ora_o, what)
+    # every row of the chunk: the listed-threshold ranking against the full
+    # binned search on the same score keys (both exact, so bit for bit)
+    p_full = abi.make_params(w.B, w.Hq, w.G, T, w.k, w.n_init, w.n_local,
+                             tune={"select_binned": 1})
+    idx_full = torch.full_like(pc.idx, -7)
+    abi.sparda_forecast_select(p_full, pc.F, w.nq, 1, q0, pc.kc, idx_full, pc.ws_sel, pc.status)
+    torch.cuda.synchronize()
+    assert int(pc.status.item()) == 0
+    assert torch.equal(idx_full, pc.idx), "%d of %d rows differ" % (
+        int((idx_full != pc.idx).any(dim=-1).sum()), w.B * w.nq * w.G)
     del pc
     torch.cuda.empty_cache()
 

@@ -237,6 +237,63 @@ def test_select_prefill_exact_ties_lower_index_wins(k):
     assert np.array_equal(got, ora)
 
 
+def _exact_score_case(rng, B, G, NB, nq, pattern):
+    """Forecast vectors and compressed keys whose scores are exact in bf16
+    products and fp32 sums: score = a + b / 256 with integer a, b in
+    [-128, 128] (F = (+-1, +-1/256, 0, ...)), so the device keys and the
+    oracle's fp64 scores order the blocks identically and the sets must match
+    bit for bit."""
+    kc = np.zeros((B, G, NB, 128), np.float32)
+    a = rng.integers(-128, 129, size=(B, G, NB))
+    b = rng.integers(-128, 129, size=(B, G, NB))
+    if pattern == "lane":  # one lane's entries (block 1 + 32 m + 5) all score high
+        a[..., 6::32] = rng.integers(100, 129, size=a[..., 6::32].shape)
+    elif pattern == "outlier":  # one far outlier: every other listed key shares a bin
+        a[...] = rng.integers(0, 2, size=a.shape)
+        a[..., NB // 2] = 128
+    elif pattern == "ties":  # few distinct values: ties straddle the k-th
+        a[...] = rng.integers(0, 4, size=a.shape)
+        b[...] = 0
+    kc[..., 0], kc[..., 1] = a, b
+    F = np.zeros((B, nq, G, 1, 128), np.float32)
+    sgn = np.where(rng.random((B, nq, G, 1)) < 0.8, 1.0, -1.0)
+    F[..., 0] = sgn
+    F[..., 1] = sgn / 256.0
+    return W.f32_to_bf16_bits(F), W.f32_to_bf16_bits(kc)
+
+
+@pytest.mark.parametrize("k", [1, 8, 33, 64])
+@pytest.mark.parametrize("pattern", ["random", "lane", "outlier", "ties"])
+def test_select_prefill_listed_threshold_exact(k, pattern):
+    """The row ranking's listed threshold (k <= 64, rows of 1024-2048 keys)
+    and every way it hands a row to the full search -- a lane listing more
+    keys than it holds, a threshold bin of more than 32 keys, keys equal to
+    the k-th only partly kept -- on exactly representable scores: the sets
+    equal the oracle's bit for bit, and those of the full search on every
+    row (select_binned)."""
+    rng = np.random.default_rng(23 + 7 * k + len(pattern))
+    B, G, NB, nq = 1, 2, 2048, 96
+    T = NB * 64
+    Fb, kcb = _exact_score_case(rng, B, G, NB, nq, pattern)
+    ora, _, _ = oracle.select(Fb, kcb, k, 1, 2, T - nq)
+    got = gpu_select(Fb, kcb, k, 1, 2, T - nq, T)
+    assert np.array_equal(got, ora), pattern
+    full = gpu_select(Fb, kcb, k, 1, 2, T - nq, T, tune={"select_binned": 1})
+    assert np.array_equal(full, ora), pattern
+
+
+def test_select_prefill_listed_threshold_short_rows():
+    """Rows of 1024 keys, the shortest the listed threshold takes, next to
+    rows just below it, which the full search ranks."""
+    rng = np.random.default_rng(31)
+    B, G, NB, nq = 1, 2, 1027, 96
+    T = NB * 64
+    Fb, kcb = _exact_score_case(rng, B, G, NB, nq, "random")
+    for k in (16, 64):
+        ora, _, _ = oracle.select(Fb, kcb, k, 1, 2, T - nq)
+        assert np.array_equal(gpu_select(Fb, kcb, k, 1, 2, T - nq, T), ora)
+
+
 def test_select_prefill_tensor_matches_streaming_path():
     """The same chunk through both selection paths gives the same sets."""
     rng = W.rng_for(19)
