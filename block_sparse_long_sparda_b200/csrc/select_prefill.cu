@@ -481,6 +481,7 @@ constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 204
 __device__ __forceinline__ int list_keys_from(const uint32_t *keys, int ncand, uint32_t t0,
                                               WarpRankSmem &sm) {
   const int lane = threadIdx.x & 31;
+  __builtin_assume(ncand >= 1024);  // the listed threshold takes rows of 1024 keys or more
   int c = 0;
 #pragma unroll 8
   for (int q = 0; q < kRegKeys; ++q) {
@@ -668,6 +669,7 @@ __device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPo
   int32_t *top = out + bp.init_hi;
   const uint32_t lt = (1u << lane) - 1u;
   if (kListed && ncand >= 1024 && ncand <= kRegKeys * 32) {
+    __builtin_assume(ncand >= 1024);  // entries 0..1023 exist: no bound test for them
     // the lane's largest and second-largest keys, all 64 loads in flight at
     // once; the row is not kept in registers: the listing reads it again
     // from L1, and the register search below loads it for the rows the
