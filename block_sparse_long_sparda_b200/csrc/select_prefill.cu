@@ -27,7 +27,7 @@
 //  2. rank_rows_kernel -- one warp per (sequence, token, group) row.  For
 //     k <= 64 and rows of 1024 to 2048 keys it first takes a threshold t0
 //     that at least 64 keys pass (the least over the lanes of each lane's
-//     second-largest key), lists the keys >= t0 (about 8 % of a row) and
+//     second-largest key), lists the keys >= t0 (about 9 % of a row) and
 //     ranks only those: one histogram, an exact rank of the threshold bin,
 //     and a bitmap that puts the kept blocks in order.  Other rows, and rows
 //     whose lists or ties that does not settle, take the same exact search as
@@ -465,7 +465,8 @@ constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 204
 // of each lane's second-largest key, so every lane holds two keys >= t0 and
 // at least 64 >= k keys pass it: the k-th largest key is >= t0, and so is
 // every key the set keeps.  On scores of roughly one shape across the row a
-// lane holds about five such keys of its 64.  Each lane lists its keys >= t0
+// lane holds about six such keys of its 64 (more than kListCap in about 2 %
+// of Gaussian rows).  Each lane lists its keys >= t0
 // in shared memory (list_keys_from), one histogram of the listed keys finds
 // the bin of the k-th largest, its members are ranked exactly, and the kept
 // entries are placed in block order through a bitmap (word q, bit lane) and
