@@ -360,13 +360,26 @@ def test_select_windows_decode(T, k, n_local, chunk):
                          tune={"select_chunk": int(chunk)})
 
 
-@pytest.mark.parametrize("T,nq,q_off", [(16384 + 40, 96, 0), (40000, 200, 3000)])
+@pytest.mark.parametrize("T,nq,q_off", [(16384 + 40, 96, 0), (40000, 200, 3000),
+                                         (2048 * 64 + 40, 96, 0)])
 def test_select_windows_prefill_tensor_path(T, nq, q_off):
+    """The last case has 2045-2046 candidates per token: its rows take the
+    listed threshold, and must equal the full search's bit for bit."""
     rng = W.rng_for(80 + T)
     B, G, d = 2, 2, 128
     kw = W.normal_bf16(rng, (B, G, oracle.window_count(T), d))
     F = W.normal_bf16(rng, (B, nq, G, 1, d))
     _select_windows_case(F, kw, T, 32, 1, 2, T - nq - q_off, "windows prefill")
+    if T > 2048 * 64:
+        sets = []
+        for tune in (None, {"select_binned": 1}):
+            p = abi.make_params(B, G, G, T, 32, 1, 2, tune=tune)
+            idx = torch.full((B, nq, G, 35), -7, dtype=torch.int32, device="cuda")
+            abi.sparda_forecast_select_windows(
+                p, dev_bf16(F), nq, 1, T - nq - q_off, dev_bf16(kw), 32, 16, idx,
+                abi.workspace(abi.SPARDA_OP_SELECT_WINDOWS, p, nq, 1))
+            sets.append(idx.cpu())
+        assert torch.equal(sets[0], sets[1])
 
 
 def test_select_windows_compressed_from_keys():
