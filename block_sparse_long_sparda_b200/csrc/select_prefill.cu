@@ -461,20 +461,19 @@ constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 204
 
 // The row's top k from a sampled threshold, for k <= 64 and rows of 1024 to
 // 2048 keys, each lane taking the entries e = 32 q + lane as in the register
-// search above (0 past the row).  t0 is the smallest over the lanes
-// of each lane's second-largest key, so every lane holds two keys >= t0 and
-// at least 64 >= k keys pass it: the k-th largest key is >= t0, and so is
-// every key the set keeps.  On scores of roughly one shape across the row a
-// lane holds about six such keys of its 64 (more than kListCap in about 2 %
-// of Gaussian rows).  Each lane lists its keys >= t0
-// in shared memory (list_keys_from), one histogram of the listed keys finds
-// the bin of the k-th largest, its members are ranked exactly, and the kept
-// entries are placed in block order through a bitmap (word q, bit lane) and
-// its prefix counts (warp_topk_listed).  warp_topk_listed returns false,
-// having written nothing, when a lane lists more than kListCap keys, the bin
-// holds more than 32 keys, or only some of the keys equal to the k-th are
-// kept (the lower block indices would have to win); the caller then runs
-// the full search.
+// search above (0 past the row).  t0 is the smallest over the lanes of each
+// lane's second-largest key, so every lane holds two keys >= t0 and at least
+// 64 >= k keys pass it: the k-th largest key is >= t0, and so is every key
+// the set keeps.  On scores of roughly one shape across the row a lane holds
+// about six such keys of its 64 (more than kListCap in about 2 % of Gaussian
+// rows).  Each lane lists its keys >= t0 in shared memory (list_keys_from),
+// one histogram of the listed keys finds the bin of the k-th largest, its
+// members are ranked exactly, and the kept entries are placed in block order
+// through a bitmap (word q, bit lane) and its prefix counts
+// (warp_topk_listed).  warp_topk_listed returns false, having written
+// nothing, when a lane lists more than kListCap keys, the bin holds more than
+// 32 keys, or only some of the keys equal to the k-th are kept (the lower
+// block indices would have to win); the caller then runs the full search.
 
 // c = the lane's keys >= t0 (t0 >= 1, so never an empty entry), read again
 // from memory (L1 holds the row just read); only the first kListCap are
