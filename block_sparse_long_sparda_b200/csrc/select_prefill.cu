@@ -53,7 +53,7 @@ constexpr int kPTok = 128;      // token rows per score tile (MMA M)
 constexpr int kPBlk = 256;      // block columns per score tile (MMA N)
 constexpr int kPThreads = 128;  // four warps: TMEM lanes 0-127, thread = token row
 constexpr int kPSmem = 32768 + 65536 + 1024;  // F tile | Kc tile | barriers
-constexpr int kRWarps = 8;      // rows ranked per CTA (one warp each)
+constexpr int kRWarps = 4;      // rows ranked per CTA (one warp each)
 
 struct PScoreArgs {
   uint32_t *keys;      // [B*G][nq][ld]
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kPThreads) prefill_scores_kernel(
 // ---------------------------------------------------------------------------
 // warp-level exact top-k of one row
 // ---------------------------------------------------------------------------
-constexpr int kListCap = 16;  // keys per lane the sampled threshold may list
+constexpr int kListCap = 24;  // keys per lane the sampled threshold may list
 
 struct WarpRankSmem {
   uint32_t hist[256];
@@ -765,7 +765,7 @@ __device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPo
 // the row held in registers (rows of up to 2048 candidates) or in memory.
 // One warp per row.
 template <bool kListed>
-__global__ void __launch_bounds__(kRWarps * 32, 2) rank_rows_kernel(RankArgs a) {
+__global__ void __launch_bounds__(kRWarps * 32, 4) rank_rows_kernel(RankArgs a) {
   __shared__ WarpRankSmem wsm[kRWarps];
   const int warp = threadIdx.x >> 5;
   const long long row = (long long)blockIdx.x * kRWarps + warp;
