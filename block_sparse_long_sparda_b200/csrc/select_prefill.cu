@@ -39,6 +39,7 @@
 // Every wait is bounded; a timeout sets SPARDA_DEV_TIMEOUT, frees TMEM and
 // leaves the tile's keys unwritten.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -53,7 +54,8 @@ constexpr int kPTok = 128;      // token rows per score tile (MMA M)
 constexpr int kPBlk = 256;      // block columns per score tile (MMA N)
 constexpr int kPThreads = 128;  // four warps: TMEM lanes 0-127, thread = token row
 constexpr int kPSmem = 32768 + 65536 + 1024;  // F tile | Kc tile | barriers
-constexpr int kRWarps = 4;      // rows ranked per CTA (one warp each)
+constexpr int kRWarps = 8;        // rows ranked per CTA (one warp each), binned search alone
+constexpr int kRWarpsListed = 4;  // the same with the listed threshold (larger per-warp lists)
 
 struct PScoreArgs {
   uint32_t *keys;      // [B*G][nq][ld]
@@ -216,6 +218,10 @@ constexpr int kListCap = 24;  // keys per lane the sampled threshold may list
 struct WarpRankSmem {
   uint32_t hist[256];
   uint32_t list[32];
+};
+
+// the listed threshold's lists on top
+struct WarpListSmem : WarpRankSmem {
   uint2 cand[kListCap + 1][32];  // per lane: (key, register q) of its keys >= t0; row
                                  // kListCap takes the writes past the cap
   uint32_t sel[64];              // kept entries: word q, bit lane = entry 32 q + lane
@@ -479,7 +485,7 @@ constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 204
 // from memory (L1 holds the row just read); only the first kListCap are
 // stored
 __device__ __forceinline__ int list_keys_from(const uint32_t *keys, int ncand, uint32_t t0,
-                                              WarpRankSmem &sm) {
+                                              WarpListSmem &sm) {
   const int lane = threadIdx.x & 31;
   __builtin_assume(ncand >= 1024);  // the listed threshold takes rows of 1024 keys or more
   int c = 0;
@@ -495,7 +501,7 @@ __device__ __forceinline__ int list_keys_from(const uint32_t *keys, int ncand, u
   return c;
 }
 
-__device__ bool warp_topk_listed(int c, uint32_t t0, uint32_t umax, int k, WarpRankSmem &sm,
+__device__ bool warp_topk_listed(int c, uint32_t t0, uint32_t umax, int k, WarpListSmem &sm,
                                  int32_t *top, int cand_lo) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
@@ -623,10 +629,9 @@ __device__ __forceinline__ RowPos row_pos(const RankArgs &a, long long row) {
   return r;
 }
 
-// One row, by one warp.
-template <bool kListed>
-__device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPos rp,
-                                         WarpRankSmem &sm) {
+// One row, by one warp (Smem: WarpListSmem for kListed, else WarpRankSmem).
+template <bool kListed, class Smem>
+__device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPos rp, Smem &sm) {
   const int lane = threadIdx.x & 31;
   const long long b = rp.b;
   const int g = rp.g, i = rp.i;
@@ -668,28 +673,30 @@ __device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPo
   int need;
   int32_t *top = out + bp.init_hi;
   const uint32_t lt = (1u << lane) - 1u;
-  if (kListed && ncand >= 1024 && ncand <= kRegKeys * 32) {
-    __builtin_assume(ncand >= 1024);  // entries 0..1023 exist: no bound test for them
-    // the lane's largest and second-largest keys, all 64 loads in flight at
-    // once; the row is not kept in registers: the listing reads it again
-    // from L1, and the register search below loads it for the rows the
-    // listed threshold does not settle
-    uint32_t u1 = 0u, u2 = 0u;
+  if constexpr (kListed) {
+    if (ncand >= 1024 && ncand <= kRegKeys * 32) {
+      __builtin_assume(ncand >= 1024);  // entries 0..1023 exist: no bound test for them
+      // the lane's largest and second-largest keys, all 64 loads in flight at
+      // once; the row is not kept in registers: the listing reads it again
+      // from L1, and the register search below loads it for the rows the
+      // listed threshold does not settle
+      uint32_t u1 = 0u, u2 = 0u;
 #pragma unroll
-    for (int q = 0; q < kRegKeys; ++q) {
-      const int e = q * 32 + lane;
-      const uint32_t u = e < ncand ? ld_key(keys + e) : 0u;
-      u2 = max(u2, min(u1, u));
-      u1 = max(u1, u);
+      for (int q = 0; q < kRegKeys; ++q) {
+        const int e = q * 32 + lane;
+        const uint32_t u = e < ncand ? ld_key(keys + e) : 0u;
+        u2 = max(u2, min(u1, u));
+        u1 = max(u1, u);
+      }
+      const uint32_t t0 = __reduce_min_sync(0xffffffffu, u2);
+      const uint32_t top_key = __reduce_max_sync(0xffffffffu, u1);
+      // t0 = 0: a lane with fewer than two keys; t0 = the top key: all listed keys equal
+      if (t0 != 0u && t0 < top_key &&
+          warp_topk_listed(list_keys_from(keys, ncand, t0, sm), t0, top_key, a.k, sm, top,
+                           bp.cand_lo))
+        return;
+      __syncwarp();
     }
-    const uint32_t t0 = __reduce_min_sync(0xffffffffu, u2);
-    const uint32_t top_key = __reduce_max_sync(0xffffffffu, u1);
-    // t0 = 0: a lane with fewer than two keys; t0 = the top key: all listed keys equal
-    if (t0 != 0u && t0 < top_key &&
-        warp_topk_listed(list_keys_from(keys, ncand, t0, sm), t0, top_key, a.k, sm, top,
-                         bp.cand_lo))
-      return;
-    __syncwarp();
   }
   if (ncand <= kRegKeys * 32) {
     uint32_t kv[kRegKeys];
@@ -765,10 +772,12 @@ __device__ __forceinline__ void rank_row(const RankArgs &a, long long row, RowPo
 // the row held in registers (rows of up to 2048 candidates) or in memory.
 // One warp per row.
 template <bool kListed>
-__global__ void __launch_bounds__(kRWarps * 32, 4) rank_rows_kernel(RankArgs a) {
-  __shared__ WarpRankSmem wsm[kRWarps];
+__global__ void __launch_bounds__((kListed ? kRWarpsListed : kRWarps) * 32, kListed ? 4 : 2)
+    rank_rows_kernel(RankArgs a) {
+  constexpr int kW = kListed ? kRWarpsListed : kRWarps;
+  __shared__ std::conditional_t<kListed, WarpListSmem, WarpRankSmem> wsm[kW];
   const int warp = threadIdx.x >> 5;
-  const long long row = (long long)blockIdx.x * kRWarps + warp;
+  const long long row = (long long)blockIdx.x * kW + warp;
   pdl_trigger();
   pdl_wait();
   if (row < a.rows) rank_row<kListed>(a, row, row_pos(a, row), wsm[warp]);
@@ -860,8 +869,9 @@ cudaError_t launch_select_prefill(const sparda_params &p, const uint16_t *F, int
   const int nc_last = block_parts(q_start + nq - 1, kBlk, p.n_init, p.n_local).cand_hi - p.n_init;
   const bool listed = tuning(p).select_binned == 0 && p.seq_len == nullptr && p.k >= 1 &&
                       p.k <= 64 && nc_first >= 1024 && nc_last <= kRegKeys * 32;
+  const int warps = listed ? kRWarpsListed : kRWarps;
   e = launch_pdl(listed ? rank_rows_kernel<true> : rank_rows_kernel<false>,
-                 (unsigned)ceil_div_ll(ra.rows, kRWarps), kRWarps * 32, 0, stream, ra);
+                 (unsigned)ceil_div_ll(ra.rows, warps), warps * 32, 0, stream, ra);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
