@@ -471,8 +471,8 @@ constexpr int kRegKeys = 64;  // keys per lane held in registers (rows up to 204
 // lane's second-largest key, so every lane holds two keys >= t0 and at least
 // 64 >= k keys pass it: the k-th largest key is >= t0, and so is every key
 // the set keeps.  On scores of roughly one shape across the row a lane holds
-// about six such keys of its 64 (more than kListCap in about 2 % of Gaussian
-// rows).  Each lane lists its keys >= t0 in shared memory (list_keys_from),
+// about six such keys of its 64 (more than kListCap = 24 in none of 3000
+// modelled Gaussian rows; 16 would overflow in about 2 %).  Each lane lists its keys >= t0 in shared memory (list_keys_from),
 // one histogram of the listed keys finds the bin of the k-th largest, its
 // members are ranked exactly, and the kept entries are placed in block order
 // through a bitmap (word q, bit lane) and its prefix counts
